@@ -1,0 +1,288 @@
+"""CPU oracle for the KDA + modality-aware short-convolution forward pass.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package.  It shares no code
+with the CUDA path (``linear_attention_video_b200``) and never imports it.
+
+Two independent formulations live here, both in fp64:
+
+* ``kda_oracle.c`` -- the definition: the depthwise short convolution written
+  out tap by tap, and the token-by-token KDA recurrence
+  (paper.rainbus.top, section 方法步骤详情, step (5);
+  genai-atlas, section "How it works").
+* this module's numpy code -- the chunked (UT/WY) form for any chunk length,
+  the dense lower-triangular form, and the update exactly as printed on the
+  page (explicit (I - beta k k^T) Diag(alpha) products), used only to
+  cross-check the recurrence on small inputs.
+
+Readings of points the pages leave open (each also listed in the design doc):
+  * read-out o_t = S_t^T q_t, no scale on q;
+  * kernels: causal 4 taps over text, 3x3x3 over the visual grid, applied as a
+    cross-correlation (tap j of the text kernel multiplies x[t-(K-1)+j]);
+  * the 3D conv is centred and zero-padded in T, H and W by default; with
+    ``vis_causal_t`` its temporal taps cover frames t-kt+1..t instead;
+  * no bias, activation or normalisation after the conv;
+  * separate depthwise weights for q, k and v;
+  * one causal scan over text then visual tokens, no reset in between;
+  * batch items are independent and share the text length.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "kda_oracle.c")
+_LIB = os.path.join(_HERE, "libkdaoracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle (plain -O2, IEEE fp64 arithmetic, no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        subprocess.check_call(["gcc", "-O2", "-fPIC", "-shared", "-pthread", "-o", _LIB, _SRC, "-lm"])
+    return _LIB
+
+
+class ConvShape(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in (
+        "B", "N", "text_len", "grid_t", "grid_h", "grid_w", "text_k",
+        "vis_kt", "vis_kh", "vis_kw", "vis_causal_t")]
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB)
+            i64, vp, i32 = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int
+            lib.kdao_shortconv.argtypes = [ctypes.POINTER(ConvShape), i64, i64, i64, vp, vp, vp, vp, i32]
+            lib.kdao_shortconv.restype = i32
+            lib.kdao_scan.argtypes = [i64, i64, i64, i64, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i32]
+            lib.kdao_scan.restype = i32
+            _lib = lib
+    return _lib
+
+
+def default_threads() -> int:
+    return max(1, os.cpu_count() or 1)
+
+
+def widen(a: np.ndarray, dtype: str) -> np.ndarray:
+    """Exact float32 view of stored inputs: bf16 bit patterns or float32."""
+    if dtype == "bf16":
+        return (a.astype(np.uint32) << 16).view(np.float32)
+    return np.asarray(a, dtype=np.float32)
+
+
+def conv_shape(B, N, text_len, grid, text_k=4, vis_k=(3, 3, 3), vis_causal_t=False) -> ConvShape:
+    T, Hg, Wg = grid
+    if N != text_len + T * Hg * Wg:
+        raise ValueError("N must equal text_len + T*Hg*Wg")
+    return ConvShape(B, N, text_len, T, Hg, Wg, text_k, vis_k[0], vis_k[1], vis_k[2], int(bool(vis_causal_t)))
+
+
+def shortconv(shape: ConvShape, x: np.ndarray, w_text: np.ndarray, w_vis: np.ndarray,
+              c0: int = 0, c1: int | None = None, nthreads: int | None = None) -> np.ndarray:
+    """Per-modality depthwise short convolution of x [B, N, C] (float32) in fp64.
+
+    Returns y[:, :, c0:c1] as float64 [B, N, c1-c0].  w_text [C, text_k] and
+    w_vis [C, kt*kh*kw] are float32.
+    """
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    B, N, C = x.shape
+    c1 = C if c1 is None else c1
+    wt = np.ascontiguousarray(w_text, dtype=np.float32)
+    wv = np.ascontiguousarray(w_vis, dtype=np.float32)
+    assert wt.shape == (C, shape.text_k) and wv.shape == (C, shape.vis_kt * shape.vis_kh * shape.vis_kw)
+    y = np.empty((B, N, c1 - c0), dtype=np.float64)
+    rc = _load().kdao_shortconv(ctypes.byref(shape), C, c0, c1, x.ctypes.data, wt.ctypes.data,
+                                wv.ctypes.data, y.ctypes.data, nthreads or default_threads())
+    if rc:
+        raise ValueError(f"kdao_shortconv failed ({rc})")
+    return y
+
+
+def scan(q, k, v, log_alpha, beta, S0=None, j0=0, j1=None, nthreads=None):
+    """Token-by-token KDA recurrence for ONE head, fp64.
+
+    q, k, log_alpha : [B, N, dk];  v : [B, N, dv];  beta : [B, N];  S0 : [B, dk, dv] or None.
+    Returns (o [B, N, dv], S_N [B, dk, dv]); only columns [j0, j1) are computed
+    (the others are zero).
+    """
+    q, k, v, la, bt = (np.ascontiguousarray(a, dtype=np.float64) for a in (q, k, v, log_alpha, beta))
+    B, N, dk = q.shape
+    dv = v.shape[-1]
+    j1 = dv if j1 is None else j1
+    o = np.zeros((B, N, dv), dtype=np.float64)
+    SN = np.zeros((B, dk, dv), dtype=np.float64)
+    s0p = None
+    if S0 is not None:
+        S0 = np.ascontiguousarray(S0, dtype=np.float64)
+        assert S0.shape == (B, dk, dv)
+        s0p = S0.ctypes.data
+    rc = _load().kdao_scan(B, N, dk, dv, q.ctypes.data, k.ctypes.data, v.ctypes.data, la.ctypes.data,
+                           bt.ctypes.data, s0p, o.ctypes.data, SN.ctypes.data, j0, j1,
+                           nthreads or default_threads())
+    if rc:
+        raise ValueError(f"kdao_scan failed ({rc})")
+    return o, SN
+
+
+def _heads_inputs(inp: dict, h: int, shape: ConvShape, d: int, nthreads=None, v_cols=None):
+    """Convolved q', k', v' and the gates of head h, all float64."""
+    B, N, H, _ = inp["shape"]
+    dt = inp["dtype"]
+    C = H * d
+    out = []
+    for idx, name in enumerate(("q", "k", "v")):
+        x = widen(inp[name], dt).reshape(B, N, C)
+        c0, c1 = h * d, (h + 1) * d
+        if name == "v" and v_cols is not None:
+            c0, c1 = h * d + v_cols[0], h * d + v_cols[1]
+        out.append(shortconv(shape, x, inp["w_text"][idx], inp["w_vis"][idx], c0, c1, nthreads))
+    la = inp["log_alpha"].reshape(B, N, H, d)[:, :, h, :].astype(np.float64)
+    bt = widen(inp["beta"], dt).reshape(B, N, H)[:, :, h].astype(np.float64)
+    return out[0], out[1], out[2], la, bt
+
+
+def forward(inp: dict, text_len: int, grid, S0=None, heads=None, text_k=4, vis_k=(3, 3, 3),
+            vis_causal_t=False, nthreads=None):
+    """Conv on q, k, v, then the KDA recurrence, for every (or the listed) head.
+
+    ``inp`` is a dict as produced by ``kda_synth.generate``.  Returns
+    (o [B, N, H, d] float64, S_N [B, H, d, d] float64).
+    """
+    B, N, H, d = inp["shape"]
+    shape = conv_shape(B, N, text_len, grid, text_k, vis_k, vis_causal_t)
+    o = np.zeros((B, N, H, d), dtype=np.float64)
+    SN = np.zeros((B, H, d, d), dtype=np.float64)
+    for h in (range(H) if heads is None else heads):
+        qh, kh, vh, la, bt = _heads_inputs(inp, h, shape, d, nthreads)
+        s0 = None if S0 is None else np.asarray(S0)[:, h]
+        oh, sh = scan(qh, kh, vh, la, bt, s0, nthreads=nthreads)
+        o[:, :, h, :] = oh
+        SN[:, h] = sh
+    return o, SN
+
+
+def forward_columns(inp: dict, text_len: int, grid, items, S0=None, text_k=4, vis_k=(3, 3, 3),
+                    vis_causal_t=False, nthreads=None):
+    """o[b, :, h, j] for each (h, j) in ``items`` and every batch item b.
+
+    Column j of the state depends only on column j of v, so each sampled
+    column is exact at any sequence length.  Returns float64 [len(items), B, N].
+    """
+    B, N, H, d = inp["shape"]
+    shape = conv_shape(B, N, text_len, grid, text_k, vis_k, vis_causal_t)
+    res = np.zeros((len(items), B, N), dtype=np.float64)
+    by_head = {}
+    for i, (h, j) in enumerate(items):
+        by_head.setdefault(h, []).append((i, j))
+    for h, lst in by_head.items():
+        qh, kh, _, la, bt = _heads_inputs(inp, h, shape, d, nthreads, v_cols=(0, 1))
+        for i, j in lst:
+            x = widen(inp["v"], inp["dtype"]).reshape(B, N, H * d)
+            vj = shortconv(shape, x, inp["w_text"][2], inp["w_vis"][2], h * d + j, h * d + j + 1, nthreads)
+            vfull = np.zeros((B, N, d), dtype=np.float64)
+            vfull[:, :, j] = vj[:, :, 0]
+            s0 = None if S0 is None else np.asarray(S0)[:, h]
+            oh, _ = scan(qh, kh, vfull, la, bt, s0, j0=j, j1=j + 1, nthreads=nthreads)
+            res[i] = oh[:, :, j]
+    return res
+
+
+# ---------------------------------------------------------------------------
+# Second formulations (numpy, fp64), for cross-checking the recurrence.
+# ---------------------------------------------------------------------------
+
+def printed_form_scan(q, k, v, log_alpha, beta, S0=None):
+    """The update exactly as printed (paper.rainbus.top, 方法步骤详情 step (5)):
+    S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T, then
+    o_t = S_t^T q_t.  One head, one batch item: q, k, log_alpha [N, dk]; v [N, dv]."""
+    N, dk = q.shape
+    dv = v.shape[1]
+    S = np.zeros((dk, dv)) if S0 is None else np.array(S0, dtype=np.float64)
+    o = np.zeros((N, dv))
+    I = np.eye(dk)
+    for t in range(N):
+        kt = k[t][:, None]
+        S = (I - beta[t] * kt @ kt.T) @ np.diag(np.exp(log_alpha[t])) @ S + beta[t] * kt @ v[t][None, :]
+        o[t] = S.T @ q[t]
+    return o, S
+
+
+def _chunk_terms(qc, kc, lac, bc):
+    """Per-chunk quantities of the chunked form for one head.
+
+    With g_r = sum_{i<=r} log a_i (within the chunk, vector over dk):
+      A[r,i] = beta_r sum_c k_rc k_ic exp(g_rc - g_ic)   (i < r)
+      P[r,i] = sum_c q_rc k_ic exp(g_rc - g_ic)          (i <= r)
+      T = (I + A)^{-1} Diag(beta)
+    """
+    n = qc.shape[0]
+    g = np.cumsum(lac, axis=0)
+    diff = g[:, None, :] - g[None, :, :]
+    lower = np.tril(np.ones((n, n), dtype=bool))
+    diff = np.where(lower[:, :, None], diff, -np.inf)
+    E = np.exp(diff)
+    A = np.tril(bc[:, None] * np.einsum("rc,ic,ric->ri", kc, kc, E), -1)
+    P = np.tril(np.einsum("rc,ic,ric->ri", qc, kc, E))
+    T = np.linalg.solve(np.eye(n) + A, np.diag(bc))
+    return g, A, P, T
+
+
+def chunked_scan(q, k, v, log_alpha, beta, S0=None, chunk=64):
+    """The chunked (UT/WY) form for one head and one batch item, fp64.
+
+    Per chunk, from the entering state S:
+      W = T (K * exp(g)),  U~ = T V,  U = U~ - W S
+      O = (Q * exp(g)) S + P U
+      S <- Diag(exp(g_last)) S + (K * exp(g_last - g))^T U
+    The last chunk may be shorter than ``chunk``.
+    """
+    N, dk = q.shape
+    dv = v.shape[1]
+    S = np.zeros((dk, dv)) if S0 is None else np.array(S0, dtype=np.float64)
+    o = np.zeros((N, dv))
+    for c0 in range(0, N, chunk):
+        sl = slice(c0, min(N, c0 + chunk))
+        qc, kc, vc, lac, bc = q[sl], k[sl], v[sl], log_alpha[sl], beta[sl]
+        g, A, P, T = _chunk_terms(qc, kc, lac, bc)
+        W = T @ (kc * np.exp(g))
+        U = T @ vc - W @ S
+        o[sl] = (qc * np.exp(g)) @ S + P @ U
+        S = np.exp(g[-1])[:, None] * S + (kc * np.exp(g[-1][None, :] - g)).T @ U
+    return o, S
+
+
+def dense_scan(q, k, v, log_alpha, beta):
+    """Dense lower-triangular form from a zero state, one head, one batch item.
+
+    Written independently of the chunked form: the decays enter as ratios of
+    the running products Gamma_t = prod_{i<=t} alpha_i, and
+        (I + A) U = Diag(beta) V,   O = P U
+    with A[r,i] = beta_r sum_c k_rc k_ic Gamma_rc / Gamma_ic (i < r) and
+    P[r,i] = sum_c q_rc k_ic Gamma_rc / Gamma_ic (i <= r), solved by forward
+    substitution.  Only for short sequences with moderate decay (the running
+    products must not underflow).
+    """
+    import scipy.linalg
+    N = q.shape[0]
+    gam = np.cumprod(np.exp(log_alpha), axis=0)
+    A = np.zeros((N, N))
+    P = np.zeros((N, N))
+    for r in range(N):
+        for i in range(r + 1):
+            ratio = gam[r] / gam[i]
+            P[r, i] = np.sum(q[r] * k[i] * ratio)
+            if i < r:
+                A[r, i] = beta[r] * np.sum(k[r] * k[i] * ratio)
+    U = scipy.linalg.solve_triangular(np.eye(N) + A, beta[:, None] * v, lower=True, unit_diagonal=True)
+    return P @ U
