@@ -1,0 +1,353 @@
+"""Throughput of the KDA + modality-aware short-conv forward pass on B200.
+
+One step = one `kda_fwd` call through the C ABI (short conv on q, k, v, then the
+chunked KDA scan) over one batch of the synthetic workload, inputs resident in
+HBM.  Default workload: the 30-second 480x832 video (512 text tokens + a
+121x30x52 latent grid = 189,272 tokens, H=16, d=128, bf16), whose inputs
+(4.66 GB) are far larger than the 126 MB L2, so no flush is needed between steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+Prints one JSON line (rank 0).  Under torchrun every rank runs its own copy of
+the workload (weak scaling, no collective on the data path); the value is the
+tokens of all ranks divided by the slowest rank's device time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import kda_synth  # noqa: E402
+
+METRIC = "KDA+shortconv fwd tokens/sec on 1 B200 (30 s video); % of roofline"
+DEFAULT_WORKLOAD = "video_30s_480x832"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        d["source"] = "measured"
+        return d
+    return dict(FALLBACK_PEAKS)
+
+
+def workload_by_name(name):
+    for i, w in enumerate(kda_synth.WORKLOADS):
+        if w.name == name:
+            return i, w
+    raise SystemExit(f"unknown workload {name}; choose from {[w.name for w in kda_synth.WORKLOADS]}")
+
+
+def algorithmic_bytes(w):
+    """Bytes the fused path must move once: q, k, v, beta and o in the storage
+    dtype, log alpha in fp32 (weights and states are negligible)."""
+    e = 2 if w.dtype == "bf16" else 4
+    per_tok = 3 * w.H * w.d * e + w.H * w.d * 4 + w.H * e + w.H * w.d * e
+    return per_tok * w.tokens
+
+
+def conv_bytes(w):
+    e = 2 if w.dtype == "bf16" else 4
+    return 2 * 3 * w.H * w.d * e * w.tokens
+
+
+def tensor_flops(w):
+    """Algorithmic tensor-core flops of the chunked scan: H*(6 d^2 + 5 C d) per token."""
+    return w.H * (6 * w.d * w.d + 5 * w.chunk * w.d) * w.tokens
+
+
+# ---------------------------------------------------------------------------
+# clock sampling during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(self.gpu_index)], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        try:
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        finally:
+            os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        hi = max(sm) if sm else 0
+        loaded = [s for s in sm if s >= 0.5 * hi] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle baseline (a bounded sample of the same workload)
+# ---------------------------------------------------------------------------
+def oracle_sample_workload(w, frames):
+    """The workload cut to its first `frames` frames (same shapes otherwise)."""
+    import dataclasses
+    T, Hg, Wg = w.grid
+    return dataclasses.replace(w, grid=(min(frames, T), Hg, Wg), B=1)
+
+
+def run_oracle_sample(w, idx, frames, heads):
+    import oracle
+    ws = oracle_sample_workload(w, frames)
+    inp = kda_synth.generate(ws, kda_synth.seed_for(idx))
+    oracle.build()
+    t0 = time.perf_counter()
+    oracle.forward(inp, ws.text_len, ws.grid, heads=list(range(heads)))
+    dt = time.perf_counter() - t0
+    # throughput in full-width tokens: the sample covers `heads` of H heads
+    tokens_equiv = ws.N * heads / w.H
+    sample = (f"oracle (fp64 conv + token recurrence) on 1 batch item, heads 0..{heads - 1} of {w.H}, "
+              f"first {ws.grid[0]} of {w.grid[0]} frames ({ws.N} tokens)")
+    return tokens_equiv / dt, dt, sample
+
+
+def sample_frames(w):
+    """All frames of the workload (the sample is bounded by the head count)."""
+    return w.grid[0]
+
+
+def reference_arm(args, w, idx, rank):
+    cores = os.cpu_count()
+    if rank != 0:
+        return
+    frames = sample_frames(w) if w.grid[0] > 1 else 1
+    heads = 1
+    vals = []
+    for i in range(args.warmup + args.steps):
+        v, dt, sample = run_oracle_sample(w, idx, frames, heads)
+        if i >= args.warmup:
+            vals.append(v)
+    value = statistics.mean(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * w.tokens / value,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "N": w.N, "H": w.H, "d": w.d, "text_len": w.text_len,
+                   "grid": list(w.grid), "chunk": w.chunk},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def time_calls(fn, steps, stream):
+    import torch
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for _ in range(steps):
+        fn()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    return ev0.elapsed_time(ev1) / steps
+
+
+def ours_arm(args, w, idx, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import linear_attention_video_b200 as kda
+    from tests._util import to_device
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.current_stream(dev)
+    peaks = load_peaks()
+
+    inp = kda_synth.generate(w, kda_synth.seed_for(idx))
+    B, N, H, d = inp["shape"]
+    t = to_device(inp, dev)
+    dt = t["q"].dtype
+    p = kda.problem(B, H, d, w.text_len, w.grid, chunk=w.chunk)
+    o = torch.empty(B, N, H, d, dtype=dt, device=dev)
+    ws = kda.alloc_workspace(p, dt, dev)
+
+    def step():
+        kda.kda_fwd(p, t["q"], t["k"], t["v"], t["log_alpha"], t["beta"], t["w_text"], t["w_vis"], o, ws,
+                    stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = kda.kda_read_status(ws, stream)
+    if st != kda.KDA_OK:
+        raise SystemExit(f"device status after warm-up: {kda.kda_status_str(st)}")
+    launches_per_step = kda.kda_last_launch_count()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        ms = time_calls(step, args.steps, stream)
+    clocks = clk.summary()
+    ms_t = torch.tensor([ms], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms = float(ms_t.item())
+    tokens_all = w.tokens * world
+    value = tokens_all / (ms * 1e-3)
+
+    # per-kernel timings (same kernels, launched through the single-op entry points)
+    conv_out = [torch.empty_like(t["q"]) for _ in range(3)]
+
+    def conv_step():
+        kda.kda_shortconv_fwd(p, t["q"], t["k"], t["v"], t["w_text"], t["w_vis"], *conv_out, stream=stream)
+
+    def scan_step():
+        kda.kda_chunk_fwd(p, conv_out[0], conv_out[1], conv_out[2], t["log_alpha"], t["beta"], o, ws,
+                          stream=stream)
+    conv_step()
+    ms_conv = time_calls(conv_step, args.steps, stream)
+    ms_scan = time_calls(scan_step, args.steps, stream)
+    del conv_out
+
+    scan_bytes = algorithmic_bytes(w)
+    scan_gbs = scan_bytes / (ms_scan * 1e-3) / 1e9
+    conv_gbs = conv_bytes(w) / (ms_conv * 1e-3) / 1e9
+    hbm = float(peaks["hbm_gbs"])
+    dominant = "kda_chunk" if ms_scan >= ms_conv else "shortconv"
+    achieved = scan_gbs if dominant == "kda_chunk" else conv_gbs
+    traffic = None
+    prof = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(prof):
+        try:
+            traffic = json.load(open(prof)).get(dominant, {}).get(w.name)
+        except (ValueError, OSError):
+            traffic = None
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                "traffic": traffic, "kernel": dominant, "peak_source": peaks["source"] + " hbm_gbs"}
+    step_roof_ms = max(algorithmic_bytes(w) / (hbm * 1e9), tensor_flops(w) / (float(peaks["bf16_tflops"]) * 1e12)) * 1e3
+
+    # end to end through the public API: pinned host inputs -> device, kda_fwd, o -> host
+    e2e = None
+    if not args.no_e2e:
+        host = {k2: v.cpu().pin_memory() for k2, v in t.items()}
+        dev_in = {k2: torch.empty_like(v) for k2, v in t.items()}
+        o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        h2d = sum(v.numel() * v.element_size() for v in host.values())
+        d2h = o_host.numel() * o_host.element_size()
+
+        def e2e_step():
+            for k2 in host:
+                dev_in[k2].copy_(host[k2], non_blocking=True)
+            kda.kda_fwd(p, dev_in["q"], dev_in["k"], dev_in["v"], dev_in["log_alpha"], dev_in["beta"],
+                        dev_in["w_text"], dev_in["w_vis"], o, ws, stream=stream)
+            o_host.copy_(o, non_blocking=True)
+        e2e_step()
+        e2e_steps = max(3, min(args.steps, 10))
+        ms_e2e = time_calls(e2e_step, e2e_steps, stream)
+        e2e_t = torch.tensor([ms_e2e], device=dev, dtype=torch.float64)
+        if world > 1:
+            dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
+        e2e = {"value": tokens_all / (float(e2e_t.item()) * 1e-3), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+        del host, dev_in
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        frames = sample_frames(w)
+        v, secs, sample = run_oracle_sample(w, idx, frames, args.cpu_heads)
+        cpu = {"value": v, "unit": "tokens/s", "cores": os.cpu_count(), "kind": "oracle", "sample": sample,
+               "seconds": secs}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "N": w.N, "H": w.H, "d": w.d, "text_len": w.text_len,
+                       "grid": list(w.grid), "chunk": w.chunk, "parallelism": f"replicas{world}",
+                       "l2": "inputs larger than L2 (no flush)"},
+            "roofline": roofline,
+            "roofline_step": {"time_ms": step_roof_ms, "frac": step_roof_ms / ms,
+                              "bytes": algorithmic_bytes(w), "tensor_flops": tensor_flops(w)},
+            "kernels_ms": {"shortconv": ms_conv, "kda_chunk": ms_scan},
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-heads", type=int, default=4, help="heads in the CPU-baseline sample")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    idx, w = workload_by_name(args.workload)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        reference_arm(args, w, idx, rank)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        ours_arm(args, w, idx, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,137 @@
+/*
+ * kda.h -- C ABI of the B200 (sm_100a) forward pass of the modality-aware
+ * short convolution followed by the Kimi Delta Attention (KDA) scan.
+ *
+ * What is computed (sources are the pages about "Chimera: Designing and
+ * Chinchilla-Scaling Hybrid Visual Diffusion Transformers"):
+ *
+ *  - Token stream: per batch item, text_len text tokens followed by the visual
+ *    tokens of a (grid_t, grid_h, grid_w) latent grid in time-major raster
+ *    order, N = text_len + grid_t*grid_h*grid_w
+ *    (paper.rainbus.top, section 核心方法 and 方法步骤详情 step (2)).
+ *  - Short convolution, per modality, depthwise, separately on q, k and v
+ *    (genai-atlas, section "How it works"; paper.rainbus.top, section 核心方法):
+ *      text token t:  x'[t,c] = sum_{j<text_k} w_text[c][j] * x[t-(text_k-1)+j, c]
+ *                     (positions before the first token read 0);
+ *      visual token (t,h,w):
+ *                     x' = sum_{a,b,e} w_vis[c][(a*kh+b)*kw+e] * x(t+a-pt, h+b-ph, w+e-pw)
+ *                     with ph=(kh-1)/2, pw=(kw-1)/2, pt=(kt-1)/2, or pt=kt-1 when
+ *                     KDA_FLAG_VIS_CAUSAL_T is set; positions outside the grid
+ *                     read 0; text and visual tokens never read each other.
+ *  - KDA scan (paper.rainbus.top, section 方法步骤详情 step (5), and section
+ *    前置知识 "Kimi Delta Attention"), per (batch item, head), in stream order:
+ *      S_t = (I - beta_t k'_t k'_t^T) Diag(alpha_t) S_{t-1} + beta_t k'_t v'_t^T,
+ *      o_t = S_t^T q'_t            (alpha_t = exp(log_alpha_t), no scale on q)
+ *    with S_{-1} = initial_state (or 0).  The scan is evaluated in chunks of
+ *    `chunk` tokens (the chunked KDA form named in section 复现评估); the result
+ *    does not depend on the chunk length beyond rounding.
+ *
+ * Layouts (row-major, contiguous):
+ *    q, k, log_alpha : [B, N, H, dk]      v, o : [B, N, H, dv]      beta : [B, N, H]
+ *    w_text : [3][H*dk][text_k]           w_vis : [3][H*dk][vis_kt*vis_kh*vis_kw]
+ *             (slot 0 for q, 1 for k, 2 for v; fp32)
+ *    initial_state, final_state : [B, H, dk, dv] fp32
+ * q, k, v, beta and o have the element type `dtype`; log_alpha is always fp32
+ * and must be finite and <= 0.
+ *
+ * Conventions for every entry point:
+ *  - All data pointers are DEVICE pointers owned by the caller; the library
+ *    never allocates, frees or synchronises (kda_read_status excepted, which
+ *    synchronises the given stream).  `stream` is a cudaStream_t (NULL = the
+ *    legacy default stream); work is enqueued asynchronously on it.
+ *  - Argument errors are detected on the host and returned WITHOUT launching
+ *    anything: a NULL required pointer, a non-positive size, an unsupported
+ *    size (dk, dv, chunk, kernel extents), a data pointer that is not 16-byte
+ *    aligned, or a workspace smaller than kda_workspace_bytes().
+ *  - Outputs must not alias inputs.
+ *  - Device-side conditions (bounded waits that gave up, the gate range check
+ *    of the bf16 tensor-core path) are recorded in a status word at the start
+ *    of the workspace; read it with kda_read_status() once the stream has
+ *    reached the call.  Kernels never trap.
+ */
+#ifndef KDA_H
+#define KDA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  KDA_OK = 0,
+  KDA_ERR_INVALID_ARG = 1,    /* NULL pointer, non-positive or inconsistent size */
+  KDA_ERR_UNSUPPORTED = 2,    /* valid but not implemented (e.g. dk != dv, dk not 64/128) */
+  KDA_ERR_MISALIGNED = 3,     /* a data pointer is not 16-byte aligned */
+  KDA_ERR_WORKSPACE = 4,      /* workspace NULL or smaller than kda_workspace_bytes() */
+  KDA_ERR_CUDA = 5,           /* a CUDA runtime call failed (launch, copy) */
+  KDA_ERR_TIMEOUT = 6,        /* device: a bounded wait gave up */
+  KDA_ERR_DEVICE_ASSERT = 7,  /* device: an internal consistency check failed */
+  KDA_ERR_RANGE = 8           /* device: a chunk's gate decay exceeds what the bf16 tensor path handles */
+} kda_status;
+
+typedef enum { KDA_DT_BF16 = 0, KDA_DT_F32 = 1 } kda_dtype;
+
+/* Temporal taps of the 3D conv cover frames t-kt+1..t instead of being centred. */
+#define KDA_FLAG_VIS_CAUSAL_T 1u
+
+typedef struct {
+  int32_t B, H, dk, dv;             /* batch items, heads, key and value head dims */
+  int64_t text_len;                 /* text tokens per item (>= 0), same for all items */
+  int32_t grid_t, grid_h, grid_w;   /* visual grid (each >= 0; all 0 or all > 0) */
+  int32_t text_k;                   /* causal text kernel length, 1..8 */
+  int32_t vis_kt, vis_kh, vis_kw;   /* 3D kernel extents; only 3,3,3 is implemented */
+  int32_t chunk;                    /* scan chunk length: 16, 32 or 64 (fp32); 64 (bf16) */
+  uint32_t flags;                   /* KDA_FLAG_* */
+} kda_problem;
+
+/* Tokens per batch item, N = text_len + grid_t*grid_h*grid_w, or -1 if the
+ * problem is inconsistent. */
+int64_t kda_tokens(const kda_problem* p);
+
+/* Bytes of device workspace any entry point below needs for problem p and
+ * element type dtype (0 if p is invalid).  The workspace must be 256-byte
+ * aligned; its first 256 bytes hold the status word. */
+size_t kda_workspace_bytes(const kda_problem* p, kda_dtype dtype);
+
+/* Short convolution only: q_out = conv_q(q), k_out = conv_k(k), v_out = conv_v(v),
+ * all [B, N, H, d] of `dtype` (fp32 accumulation, one rounding to dtype).
+ * Returns a kda_status. */
+int kda_shortconv_fwd(const kda_problem* p, kda_dtype dtype,
+                      const void* q, const void* k, const void* v,
+                      const float* w_text, const float* w_vis,
+                      void* q_out, void* k_out, void* v_out, void* stream);
+
+/* KDA scan only, on already-convolved q', k', v'.  initial_state may be NULL
+ * (zero state); final_state may be NULL (not written).  Returns a kda_status. */
+int kda_chunk_fwd(const kda_problem* p, kda_dtype dtype,
+                  const void* q, const void* k, const void* v,
+                  const float* log_alpha, const void* beta,
+                  const float* initial_state, void* o, float* final_state,
+                  void* workspace, size_t workspace_bytes, void* stream);
+
+/* Short convolution followed by the KDA scan.  Returns a kda_status. */
+int kda_fwd(const kda_problem* p, kda_dtype dtype,
+            const void* q, const void* k, const void* v,
+            const float* log_alpha, const void* beta,
+            const float* w_text, const float* w_vis,
+            const float* initial_state, void* o, float* final_state,
+            void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronises `stream`, then returns and clears the device status word kept
+ * in `workspace` (KDA_OK if no device-side condition was recorded). */
+int kda_read_status(void* workspace, void* stream);
+
+/* Static description of a kda_status value. */
+const char* kda_status_str(int status);
+
+/* Number of kernel launches the most recent successful call on this host
+ * thread enqueued (for launch accounting in benchmarks). */
+int kda_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H */

@@ -1,0 +1,47 @@
+// Shared definitions of the CUDA path (kernels and the C-ABI layer).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kda.h"
+
+namespace kda {
+
+// Problem description after host-side validation, with derived sizes.
+struct Dims {
+  int B, H, dk, dv;
+  int64_t N, L;          // tokens per item, text prefix length
+  int T, Hg, Wg;         // visual grid
+  int text_k;
+  int pt, ph, pw;        // 3D conv padding (tap offsets are a - pt etc.)
+  int chunk;
+};
+
+// Device status word: the first uint32 of the workspace.
+__device__ __forceinline__ void set_status(uint32_t* status, uint32_t code) {
+  if (status) atomicCAS(status, 0u, code);
+}
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// Launchers (defined in the .cu files).
+cudaError_t launch_shortconv(const Dims& d, kda_dtype dt, const void* q, const void* k, const void* v,
+                             const float* w_text, const float* w_vis, void* qo, void* ko, void* vo,
+                             cudaStream_t s, int* launches);
+
+cudaError_t launch_chunk_simt(const Dims& d, kda_dtype dt, const void* q, const void* k, const void* v,
+                              const float* log_alpha, const void* beta, const float* S0, void* o,
+                              float* SN, uint32_t* status, cudaStream_t s, int* launches);
+
+size_t chunk_simt_smem_bytes(int dk, int chunk);
+
+}  // namespace kda

@@ -135,20 +135,24 @@ def scan(q, k, v, log_alpha, beta, S0=None, j0=0, j1=None, nthreads=None):
     return o, SN
 
 
-def _heads_inputs(inp: dict, h: int, shape: ConvShape, d: int, nthreads=None, v_cols=None):
+def _widened(inp: dict):
+    """q, k, v widened once to float32 [B, N, H*d]."""
+    B, N, H, d = inp["shape"]
+    return [widen(inp[n], inp["dtype"]).reshape(B, N, H * d) for n in ("q", "k", "v")]
+
+
+def _heads_inputs(inp: dict, h: int, shape: ConvShape, d: int, nthreads=None, v_cols=None, xs=None):
     """Convolved q', k', v' and the gates of head h, all float64."""
     B, N, H, _ = inp["shape"]
-    dt = inp["dtype"]
-    C = H * d
+    xs = _widened(inp) if xs is None else xs
     out = []
-    for idx, name in enumerate(("q", "k", "v")):
-        x = widen(inp[name], dt).reshape(B, N, C)
+    for idx in range(3):
         c0, c1 = h * d, (h + 1) * d
-        if name == "v" and v_cols is not None:
+        if idx == 2 and v_cols is not None:
             c0, c1 = h * d + v_cols[0], h * d + v_cols[1]
-        out.append(shortconv(shape, x, inp["w_text"][idx], inp["w_vis"][idx], c0, c1, nthreads))
+        out.append(shortconv(shape, xs[idx], inp["w_text"][idx], inp["w_vis"][idx], c0, c1, nthreads))
     la = inp["log_alpha"].reshape(B, N, H, d)[:, :, h, :].astype(np.float64)
-    bt = widen(inp["beta"], dt).reshape(B, N, H)[:, :, h].astype(np.float64)
+    bt = widen(inp["beta"], inp["dtype"]).reshape(B, N, H)[:, :, h].astype(np.float64)
     return out[0], out[1], out[2], la, bt
 
 
@@ -157,14 +161,15 @@ def forward(inp: dict, text_len: int, grid, S0=None, heads=None, text_k=4, vis_k
     """Conv on q, k, v, then the KDA recurrence, for every (or the listed) head.
 
     ``inp`` is a dict as produced by ``kda_synth.generate``.  Returns
-    (o [B, N, H, d] float64, S_N [B, H, d, d] float64).
+    (o [B, N, H, d] float64, S_N [B, H, d, d] float64); heads not listed stay 0.
     """
     B, N, H, d = inp["shape"]
     shape = conv_shape(B, N, text_len, grid, text_k, vis_k, vis_causal_t)
+    xs = _widened(inp)
     o = np.zeros((B, N, H, d), dtype=np.float64)
     SN = np.zeros((B, H, d, d), dtype=np.float64)
     for h in (range(H) if heads is None else heads):
-        qh, kh, vh, la, bt = _heads_inputs(inp, h, shape, d, nthreads)
+        qh, kh, vh, la, bt = _heads_inputs(inp, h, shape, d, nthreads, xs=xs)
         s0 = None if S0 is None else np.asarray(S0)[:, h]
         oh, sh = scan(qh, kh, vh, la, bt, s0, nthreads=nthreads)
         o[:, :, h, :] = oh
@@ -181,15 +186,15 @@ def forward_columns(inp: dict, text_len: int, grid, items, S0=None, text_k=4, vi
     """
     B, N, H, d = inp["shape"]
     shape = conv_shape(B, N, text_len, grid, text_k, vis_k, vis_causal_t)
+    xs = _widened(inp)
     res = np.zeros((len(items), B, N), dtype=np.float64)
     by_head = {}
     for i, (h, j) in enumerate(items):
         by_head.setdefault(h, []).append((i, j))
     for h, lst in by_head.items():
-        qh, kh, _, la, bt = _heads_inputs(inp, h, shape, d, nthreads, v_cols=(0, 1))
+        qh, kh, _, la, bt = _heads_inputs(inp, h, shape, d, nthreads, v_cols=(0, 1), xs=xs)
         for i, j in lst:
-            x = widen(inp["v"], inp["dtype"]).reshape(B, N, H * d)
-            vj = shortconv(shape, x, inp["w_text"][2], inp["w_vis"][2], h * d + j, h * d + j + 1, nthreads)
+            vj = shortconv(shape, xs[2], inp["w_text"][2], inp["w_vis"][2], h * d + j, h * d + j + 1, nthreads)
             vfull = np.zeros((B, N, d), dtype=np.float64)
             vfull[:, :, j] = vj[:, :, 0]
             s0 = None if S0 is None else np.asarray(S0)[:, h]

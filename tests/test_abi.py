@@ -1,0 +1,92 @@
+"""The C-ABI library loads, exports every symbol its header declares, and
+rejects bad arguments on the host before touching the GPU (CPU only)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kda.h")
+LIB = os.path.join(ROOT, "linear_attention_video_b200", "libkda.so")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:[A-Za-z_][\w\s\*]*?)\b(kda_\w+)\s*\(", src, flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def kda():
+    if not os.path.exists(LIB):
+        import importlib.util
+        spec = importlib.util.spec_from_file_location("kda_build", os.path.join(ROOT, "linear_attention_video_b200", "build.py"))
+        mod = importlib.util.module_from_spec(spec)
+        spec.loader.exec_module(mod)
+        mod.build()
+    import linear_attention_video_b200 as kda
+    return kda
+
+
+def test_header_declares_the_boundary():
+    fns = declared_functions()
+    for name in ("kda_shortconv_fwd", "kda_chunk_fwd", "kda_fwd", "kda_workspace_bytes", "kda_read_status"):
+        assert name in fns
+
+
+def test_library_exports_every_declared_symbol(kda):
+    lib = ctypes.CDLL(LIB)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert set(kda.EXPORTS) == set(declared_functions())
+
+
+def _p(kda, **kw):
+    args = dict(B=1, H=2, d=64, text_len=32, grid=(1, 14, 16))
+    args.update(kw)
+    return kda.problem(**args)
+
+
+def test_sizes_and_workspace(kda):
+    p = _p(kda)
+    assert kda.kda_tokens(p) == 32 + 224
+    ws = kda.kda_workspace_bytes(p, kda.KDA_DT_F32)
+    assert ws >= 256 + 3 * 256 * 2 * 64 * 4
+    assert kda.kda_workspace_bytes(p, kda.KDA_DT_BF16) < ws
+    assert kda.kda_workspace_bytes(_p(kda, d=96), kda.KDA_DT_F32) == 0
+    assert kda.kda_tokens(kda.problem(1, 1, 64, 5, (0, 3, 0))) == -1
+    assert kda.kda_status_str(kda.KDA_ERR_MISALIGNED).startswith("data pointer")
+
+
+def _call_fwd(kda, p, dt=0, q=256, k=256, v=256, la=256, beta=256, wt=256, wv=256, s0=None, o=256, sn=None,
+              ws=512, ws_bytes=1 << 40):
+    lib = kda._lib
+    return lib.kda_fwd(ctypes.byref(p), dt, q, k, v, la, beta, wt, wv, s0, o, sn, ws, ws_bytes, None)
+
+
+def test_host_side_rejections_launch_nothing(kda):
+    """Fake (never dereferenced) addresses: validation fails before any CUDA call."""
+    p = _p(kda)
+    assert _call_fwd(kda, p, q=None) == kda.KDA_ERR_INVALID_ARG
+    assert _call_fwd(kda, p, o=0x1008) == kda.KDA_ERR_MISALIGNED
+    assert _call_fwd(kda, p, s0=0x1004) == kda.KDA_ERR_MISALIGNED
+    assert _call_fwd(kda, p, ws=0x1010) == kda.KDA_ERR_WORKSPACE
+    assert _call_fwd(kda, p, ws_bytes=100) == kda.KDA_ERR_WORKSPACE
+    assert _call_fwd(kda, p, dt=7) == kda.KDA_ERR_INVALID_ARG
+    assert _call_fwd(kda, _p(kda, B=0)) == kda.KDA_ERR_INVALID_ARG
+    assert _call_fwd(kda, _p(kda, d=96)) == kda.KDA_ERR_UNSUPPORTED
+    assert _call_fwd(kda, _p(kda, dv=128)) == kda.KDA_ERR_UNSUPPORTED
+    assert _call_fwd(kda, _p(kda, chunk=48)) == kda.KDA_ERR_UNSUPPORTED
+    assert _call_fwd(kda, _p(kda, vis_k=(3, 5, 3))) == kda.KDA_ERR_UNSUPPORTED
+    assert _call_fwd(kda, _p(kda, text_k=9)) == kda.KDA_ERR_UNSUPPORTED
+    assert _call_fwd(kda, _p(kda, grid=(1, 0, 16))) == kda.KDA_ERR_INVALID_ARG
+    bad = _p(kda)
+    bad.flags = 1 << 5
+    assert _call_fwd(kda, bad) == kda.KDA_ERR_INVALID_ARG
+    lib = kda._lib
+    assert lib.kda_shortconv_fwd(ctypes.byref(p), 0, 256, 256, 256, 256, 256, 256, 256, 0x1002, None) == \
+        kda.KDA_ERR_MISALIGNED
+    assert lib.kda_chunk_fwd(ctypes.byref(p), 0, 256, 256, 256, 256, None, None, 256, None, 512, 1 << 40, None) == \
+        kda.KDA_ERR_INVALID_ARG
+    assert kda.kda_last_launch_count() == 0

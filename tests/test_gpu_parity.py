@@ -1,0 +1,206 @@
+"""CUDA path vs the CPU oracle, through the C ABI (needs a B200).
+
+Small workloads are compared element by element; the full-size video and
+4096^2 workloads on sampled value columns, which the oracle computes exactly
+at any length (a column of the state only depends on the same column of v).
+"""
+import numpy as np
+import pytest
+import torch
+
+import kda_synth
+import oracle
+from tests._util import assert_parity, rel_l2, to_device
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def kda():
+    import linear_attention_video_b200 as kda
+    assert torch.cuda.is_available()
+    return kda
+
+
+_cache = {}
+
+
+def workload_inputs(i, tokens=None):
+    key = (i, tokens)
+    if key not in _cache:
+        w = kda_synth.WORKLOADS[i]
+        _cache[key] = kda_synth.generate(w, kda_synth.seed_for(i), tokens=tokens)
+    return _cache[key]
+
+
+def run_fwd(kda, w, inp, chunk=64, S0=None, want_state=False, vis_causal_t=False, grid=None, text_len=None):
+    B, N, H, d = inp["shape"]
+    p = kda.problem(B, H, d, w.text_len if text_len is None else text_len, w.grid if grid is None else grid,
+                    chunk=chunk, vis_causal_t=vis_causal_t)
+    t = to_device(inp)
+    dt = t["q"].dtype
+    o = torch.empty(B, N, H, d, dtype=dt, device="cuda")
+    ws = kda.alloc_workspace(p, dt)
+    s0 = None if S0 is None else torch.from_numpy(np.ascontiguousarray(S0, np.float32)).cuda()
+    sn = torch.empty(B, H, d, d, dtype=torch.float32, device="cuda") if want_state else None
+    kda.kda_fwd(p, t["q"], t["k"], t["v"], t["log_alpha"], t["beta"], t["w_text"], t["w_vis"], o, ws,
+                initial_state=s0, final_state=sn)
+    assert kda.kda_read_status(ws) == kda.KDA_OK
+    torch.cuda.synchronize()
+    return o.float().cpu().numpy(), (sn.cpu().numpy() if want_state else None)
+
+
+@pytest.mark.parametrize("chunk", [16, 32, 64])
+def test_tiny_fp32_exact_path(kda, chunk):
+    w = kda_synth.WORKLOADS[0]
+    inp = workload_inputs(0)
+    S0 = kda_synth.initial_state(7, 1, w.H, w.d, w.d)
+    ref, ref_s = oracle.forward(inp, w.text_len, w.grid, S0=S0)
+    o, s = run_fwd(kda, w, inp, chunk=chunk, S0=S0, want_state=True)
+    assert_parity(o, ref, "f32", "o")
+    assert rel_l2(s, ref_s) <= 1e-5
+
+
+@pytest.mark.parametrize("i", [1, 2])
+def test_bf16_full_parity(kda, i):
+    w = kda_synth.WORKLOADS[i]
+    inp = workload_inputs(i)
+    heads = [0, 7, 15]
+    ref, _ = oracle.forward(inp, w.text_len, w.grid, heads=heads)
+    o, _ = run_fwd(kda, w, inp)
+    for h in heads:
+        assert_parity(o[:, :, h], ref[:, :, h], "bf16", f"head {h}")
+
+
+@pytest.mark.parametrize("i", [3, 4])
+def test_bf16_full_size_sampled_columns(kda, i):
+    w = kda_synth.WORKLOADS[i]
+    inp = workload_inputs(i)
+    items = [(0, 0), (5, 77), (15, 127)]
+    ref = oracle.forward_columns(inp, w.text_len, w.grid, items)
+    o, _ = run_fwd(kda, w, inp)
+    for n, (h, j) in enumerate(items):
+        got = o[:, :, h, j]
+        assert_parity(got, ref[n], "bf16", f"head {h} col {j}")
+
+
+def test_shortconv_entry_point(kda):
+    w = kda_synth.WORKLOADS[2]
+    inp = workload_inputs(2)
+    B, N, H, d = inp["shape"]
+    p = kda.problem(B, H, d, w.text_len, w.grid)
+    t = to_device(inp)
+    outs = [torch.empty_like(t["q"]) for _ in range(3)]
+    kda.kda_shortconv_fwd(p, t["q"], t["k"], t["v"], t["w_text"], t["w_vis"], *outs)
+    torch.cuda.synchronize()
+    shape = oracle.conv_shape(B, N, w.text_len, w.grid)
+    for idx, name in enumerate("qkv"):
+        x = oracle.widen(inp[name], "bf16").reshape(B, N, H * d)
+        ref = oracle.shortconv(shape, x, inp["w_text"][idx], inp["w_vis"][idx], 0, 256)
+        got = outs[idx].reshape(B, N, H * d)[:, :, :256].float().cpu().numpy()
+        # one bf16 rounding of an fp32 sum: within half a bf16 ulp plus fp32 accumulation error
+        assert np.all(np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-6), name
+
+
+def test_chunk_entry_point_matches_fwd(kda):
+    w = kda_synth.WORKLOADS[1]
+    inp = workload_inputs(1)
+    B, N, H, d = inp["shape"]
+    p = kda.problem(B, H, d, w.text_len, w.grid)
+    t = to_device(inp)
+    conv = [torch.empty_like(t["q"]) for _ in range(3)]
+    kda.kda_shortconv_fwd(p, t["q"], t["k"], t["v"], t["w_text"], t["w_vis"], *conv)
+    o1 = torch.empty_like(t["q"])
+    ws = kda.alloc_workspace(p, t["q"].dtype)
+    kda.kda_chunk_fwd(p, conv[0], conv[1], conv[2], t["log_alpha"], t["beta"], o1, ws)
+    o2 = torch.empty_like(t["q"])
+    kda.kda_fwd(p, t["q"], t["k"], t["v"], t["log_alpha"], t["beta"], t["w_text"], t["w_vis"], o2, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2)
+
+
+def test_chunk_length_invariance_and_continuation(kda):
+    w = kda_synth.WORKLOADS[0]
+    inp = workload_inputs(0)
+    B, N, H, d = inp["shape"]
+    o16, s16 = run_fwd(kda, w, inp, chunk=16, want_state=True)
+    o64, s64 = run_fwd(kda, w, inp, chunk=64, want_state=True)
+    assert rel_l2(o16, o64) < 1e-5 and rel_l2(s16, s64) < 1e-5
+    # split the text prefix: scan tokens [0, m) then [m, N) from the carried state,
+    # using the already-convolved sequence through kda_chunk_fwd
+    p = kda.problem(B, H, d, w.text_len, w.grid)
+    t = to_device(inp)
+    conv = [torch.empty_like(t["q"]) for _ in range(3)]
+    kda.kda_shortconv_fwd(p, t["q"], t["k"], t["v"], t["w_text"], t["w_vis"], *conv)
+    m = 100
+    parts = []
+    state = None
+    for lo, hi in ((0, m), (m, N)):
+        pp = kda.problem(B, H, d, hi - lo, (0, 0, 0))
+        sl = [c[:, lo:hi].contiguous() for c in conv]
+        la, bt = t["log_alpha"][:, lo:hi].contiguous(), t["beta"][:, lo:hi].contiguous()
+        o = torch.empty_like(sl[0])
+        sn = torch.empty(B, H, d, d, device="cuda")
+        ws = kda.alloc_workspace(pp, o.dtype)
+        kda.kda_chunk_fwd(pp, sl[0], sl[1], sl[2], la, bt, o, ws, initial_state=state, final_state=sn)
+        parts.append(o)
+        state = sn
+    torch.cuda.synchronize()
+    o_split = torch.cat(parts, dim=1).cpu().numpy()
+    assert rel_l2(o_split, o64) < 1e-5
+    assert rel_l2(state.cpu().numpy(), s64) < 1e-5
+
+
+@pytest.mark.parametrize("case", ["text_only", "visual_only", "ragged", "batch3", "causal_t", "tiny_grid"])
+def test_edge_shapes_fp32(kda, case):
+    """Shapes with ragged last chunks, one modality only, several batch items."""
+    import dataclasses
+    base = kda_synth.WORKLOADS[0]
+    shapes = {
+        "text_only": dict(text_len=77, grid=(0, 0, 0)),
+        "visual_only": dict(text_len=0, grid=(3, 5, 7)),
+        "ragged": dict(text_len=5, grid=(2, 3, 11)),
+        "batch3": dict(text_len=9, grid=(2, 4, 4), B=3),
+        "causal_t": dict(text_len=4, grid=(4, 3, 5)),
+        "tiny_grid": dict(text_len=1, grid=(1, 1, 1)),
+    }[case]
+    w = dataclasses.replace(base, **shapes)
+    inp = kda_synth.generate(w, 99)
+    causal = case == "causal_t"
+    ref, ref_s = oracle.forward(inp, w.text_len, w.grid, vis_causal_t=causal)
+    o, s = run_fwd(kda, w, inp, chunk=32, want_state=True, vis_causal_t=causal)
+    assert_parity(o, ref, "f32", case)
+    assert rel_l2(s, ref_s) <= 1e-5
+
+
+def test_empty_sequence_copies_state(kda):
+    p = kda.problem(2, 2, 64, 0, (0, 0, 0))
+    z = torch.empty(2, 0, 2, 64, device="cuda")
+    la = torch.empty(2, 0, 2, 64, device="cuda")
+    bt = torch.empty(2, 0, 2, device="cuda")
+    wt = torch.zeros(3, 128, 4, device="cuda")
+    wv = torch.zeros(3, 128, 27, device="cuda")
+    s0 = torch.randn(2, 2, 64, 64, device="cuda")
+    sn = torch.zeros_like(s0)
+    ws = torch.empty(4096, dtype=torch.uint8, device="cuda")
+    # zero-sized tensors may have a null data pointer: pass a valid dummy address
+    dummy = torch.empty(16, device="cuda")
+    args = [x if x.numel() else dummy for x in (z, z, z, la, bt)]
+    kda.kda_fwd(p, *args, wt, wv, dummy, ws, initial_state=s0, final_state=sn)
+    torch.cuda.synchronize()
+    assert torch.equal(sn, s0)
+
+
+def test_strong_decay_takes_exact_branch(kda):
+    """A chunk whose decay exceeds the factorised range (log alpha = -50 on a
+    few tokens) still matches the oracle on the fp32 path."""
+    import dataclasses
+    w = dataclasses.replace(kda_synth.WORKLOADS[0], text_len=40, grid=(1, 8, 8))
+    inp = kda_synth.generate(w, 123)
+    la = inp["log_alpha"].reshape(1, -1, w.H, w.d)
+    la[0, 10, :, :5] = -50.0
+    la[0, 70, 1, :] = -90.0
+    inp["log_alpha"] = la.reshape(-1).copy()
+    ref, _ = oracle.forward(inp, w.text_len, w.grid)
+    o, _ = run_fwd(kda, w, inp, chunk=64)
+    assert_parity(o, ref, "f32", "strong decay")
