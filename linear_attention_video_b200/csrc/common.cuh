@@ -34,14 +34,22 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 }
 
 // Launchers (defined in the .cu files).
+// out_f16: write fp16 outputs (the internal format the tensor-core scan reads) instead of dtype.
 cudaError_t launch_shortconv(const Dims& d, kda_dtype dt, const void* q, const void* k, const void* v,
                              const float* w_text, const float* w_vis, void* qo, void* ko, void* vo,
-                             cudaStream_t s, int* launches);
+                             cudaStream_t s, int* launches, bool out_f16 = false);
 
 cudaError_t launch_chunk_simt(const Dims& d, kda_dtype dt, const void* q, const void* k, const void* v,
                               const float* log_alpha, const void* beta, const float* S0, void* o,
                               float* SN, uint32_t* status, cudaStream_t s, int* launches);
 
 size_t chunk_simt_smem_bytes(int dk, int chunk);
+
+// tcgen05 path (bf16 problems with d_k = d_v = 128)
+bool chunk_tc_supported(const Dims& d);
+size_t chunk_tc_workspace_bytes(const Dims& d);
+cudaError_t launch_chunk_tc(const Dims& d, bool in_f16, const void* q, const void* k, const void* v,
+                            const float* log_alpha, const void* beta, const float* S0, void* o, float* SN,
+                            void* ws, uint32_t* status, cudaStream_t s, int* launches);
 
 }  // namespace kda

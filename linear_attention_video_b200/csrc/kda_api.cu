@@ -50,9 +50,16 @@ size_t act_bytes(const kda::Dims& d, kda_dtype dt) {
   return (size_t)d.B * d.N * d.H * d.dk * elem_size(dt);
 }
 
+bool use_tc(const kda::Dims& d, kda_dtype dt) { return dt == KDA_DT_BF16 && kda::chunk_tc_supported(d); }
+
+// status word | q', k', v' (conv outputs) | tensor-core scan records
 size_t workspace_bytes(const kda::Dims& d, kda_dtype dt) {
-  return kStatusBytes + 3 * align256(act_bytes(d, dt));
+  size_t n = kStatusBytes + 3 * align256(act_bytes(d, dt));
+  if (use_tc(d, dt)) n += align256(kda::chunk_tc_workspace_bytes(d));
+  return n;
 }
+
+size_t tc_records_offset(const kda::Dims& d, kda_dtype dt) { return kStatusBytes + 3 * align256(act_bytes(d, dt)); }
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA; }
 
@@ -73,9 +80,11 @@ int check_workspace(const kda::Dims& d, kda_dtype dt, void* ws, size_t ws_bytes)
 }
 
 // The scan itself; the workspace status word has been cleared by the caller.
+// in_f16: q', k', v' are the internal fp16 conv outputs (tensor-core path only).
 int run_scan(const kda::Dims& d, kda_dtype dt, const void* q, const void* k, const void* v,
              const float* la, const void* beta, const float* S0, void* o, float* SN,
-             uint32_t* status, cudaStream_t s, int* launches) {
+             void* workspace, cudaStream_t s, int* launches, bool in_f16) {
+  uint32_t* status = static_cast<uint32_t*>(workspace);
   if (d.N == 0) {
     if (SN) {
       const size_t bytes = (size_t)d.B * d.H * d.dk * d.dv * sizeof(float);
@@ -84,6 +93,10 @@ int run_scan(const kda::Dims& d, kda_dtype dt, const void* q, const void* k, con
       return cuda_status(e);
     }
     return KDA_OK;
+  }
+  if (use_tc(d, dt)) {
+    void* rec = static_cast<char*>(workspace) + tc_records_offset(d, dt);
+    return cuda_status(kda::launch_chunk_tc(d, in_f16, q, k, v, la, beta, S0, o, SN, rec, status, s, launches));
   }
   return cuda_status(kda::launch_chunk_simt(d, dt, q, k, v, la, beta, S0, o, SN, status, s, launches));
 }
@@ -134,7 +147,8 @@ int kda_chunk_fwd(const kda_problem* p, kda_dtype dtype, const void* q, const vo
   uint32_t* status = static_cast<uint32_t*>(workspace);
   if ((st = cuda_status(cudaMemsetAsync(status, 0, sizeof(uint32_t), s)))) return st;
   int launches = 0;
-  st = run_scan(d, dtype, q, k, v, log_alpha, beta, initial_state, o, final_state, status, s, &launches);
+  st = run_scan(d, dtype, q, k, v, log_alpha, beta, initial_state, o, final_state, workspace, s, &launches,
+                false);
   if (!st) g_last_launches = launches;
   return st;
 }
@@ -159,11 +173,12 @@ int kda_fwd(const kda_problem* p, kda_dtype dtype, const void* q, const void* k,
   void* vc = ws + kStatusBytes + 2 * act;
   if ((st = cuda_status(cudaMemsetAsync(status, 0, sizeof(uint32_t), s)))) return st;
   int launches = 0;
+  const bool tc = use_tc(d, dtype);
   if (d.N > 0) {
-    st = cuda_status(kda::launch_shortconv(d, dtype, q, k, v, w_text, w_vis, qc, kc, vc, s, &launches));
+    st = cuda_status(kda::launch_shortconv(d, dtype, q, k, v, w_text, w_vis, qc, kc, vc, s, &launches, tc));
     if (st) return st;
   }
-  st = run_scan(d, dtype, qc, kc, vc, log_alpha, beta, initial_state, o, final_state, status, s, &launches);
+  st = run_scan(d, dtype, qc, kc, vc, log_alpha, beta, initial_state, o, final_state, workspace, s, &launches, tc);
   if (!st) g_last_launches = launches;
   return st;
 }

@@ -12,6 +12,8 @@
 // lane.  The block's weights are staged transposed in shared memory
 // ([tap][channel]) so each lane reads its 8 weights of a tap as two 16-byte
 // shared loads.
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 
 namespace kda {
@@ -69,7 +71,19 @@ template <> struct Vec8<float> {
   }
 };
 
-template <typename T>
+template <> struct Vec8<__half> {
+  static __device__ __forceinline__ void store(__half* p, const float (&v)[8]) {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      __half2 h = __floats2half2_rn(v[2 * i], v[2 * i + 1]);
+      w[i] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+};
+
+template <typename T, typename TOut>
 __global__ void __launch_bounds__(256) shortconv_kernel(ConvArgs a) {
   __shared__ __align__(16) float wv[kVisTaps][kChanPerBlock];
   __shared__ __align__(16) float wt[kMaxTextK][kChanPerBlock];
@@ -87,7 +101,7 @@ __global__ void __launch_bounds__(256) shortconv_kernel(ConvArgs a) {
   __syncthreads();
 
   const T* __restrict__ x = static_cast<const T*>(a.x[tensor]);
-  T* __restrict__ y = static_cast<T*>(a.y[tensor]);
+  TOut* __restrict__ y = static_cast<TOut*>(a.y[tensor]);
   const int lane = threadIdx.x & 31;
   const int cl = lane * 8;  // channel offset within the block
   const int c0 = cb + cl;
@@ -142,7 +156,7 @@ __global__ void __launch_bounds__(256) shortconv_kernel(ConvArgs a) {
         }
       }
     }
-    Vec8<T>::store(y + b * a.N * C + n * C + c0, acc);
+    Vec8<TOut>::store(y + b * a.N * C + n * C + c0, acc);
   }
 }
 
@@ -150,7 +164,7 @@ __global__ void __launch_bounds__(256) shortconv_kernel(ConvArgs a) {
 
 cudaError_t launch_shortconv(const Dims& d, kda_dtype dt, const void* q, const void* k, const void* v,
                              const float* w_text, const float* w_vis, void* qo, void* ko, void* vo,
-                             cudaStream_t s, int* launches) {
+                             cudaStream_t s, int* launches, bool out_f16) {
   ConvArgs a;
   a.x[0] = q; a.x[1] = k; a.x[2] = v;
   a.y[0] = qo; a.y[1] = ko; a.y[2] = vo;
@@ -163,8 +177,9 @@ cudaError_t launch_shortconv(const Dims& d, kda_dtype dt, const void* q, const v
   if (a.total == 0) return cudaSuccess;
   dim3 grid((unsigned)((a.total + kTokPerBlock - 1) / kTokPerBlock),
             (unsigned)((a.C + kChanPerBlock - 1) / kChanPerBlock), 3);
-  if (dt == KDA_DT_BF16) shortconv_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(a);
-  else shortconv_kernel<float><<<grid, 256, 0, s>>>(a);
+  if (dt == KDA_DT_BF16 && out_f16) shortconv_kernel<__nv_bfloat16, __half><<<grid, 256, 0, s>>>(a);
+  else if (dt == KDA_DT_BF16) shortconv_kernel<__nv_bfloat16, __nv_bfloat16><<<grid, 256, 0, s>>>(a);
+  else shortconv_kernel<float, float><<<grid, 256, 0, s>>>(a);
   if (launches) ++*launches;
   return cudaGetLastError();
 }

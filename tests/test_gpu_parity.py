@@ -102,7 +102,9 @@ def test_shortconv_entry_point(kda):
         assert np.all(np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-6), name
 
 
-def test_chunk_entry_point_matches_fwd(kda):
+def test_chunk_entry_point_on_caller_convolved_inputs(kda):
+    """kda_chunk_fwd on q', k', v' the caller already convolved (bf16): compared
+    with the oracle's recurrence fed exactly those bf16 values."""
     w = kda_synth.WORKLOADS[1]
     inp = workload_inputs(1)
     B, N, H, d = inp["shape"]
@@ -113,10 +115,72 @@ def test_chunk_entry_point_matches_fwd(kda):
     o1 = torch.empty_like(t["q"])
     ws = kda.alloc_workspace(p, t["q"].dtype)
     kda.kda_chunk_fwd(p, conv[0], conv[1], conv[2], t["log_alpha"], t["beta"], o1, ws)
-    o2 = torch.empty_like(t["q"])
-    kda.kda_fwd(p, t["q"], t["k"], t["v"], t["log_alpha"], t["beta"], t["w_text"], t["w_vis"], o2, ws)
-    torch.cuda.synchronize()
-    assert torch.equal(o1, o2)
+    assert kda.kda_read_status(ws) == kda.KDA_OK
+    got = o1.float().cpu().numpy()
+    cv = [c.float().cpu().numpy().astype(np.float64) for c in conv]
+    la = inp["log_alpha"].reshape(B, N, H, d).astype(np.float64)
+    bt = oracle.widen(inp["beta"], "bf16").reshape(B, N, H).astype(np.float64)
+    for h in (0, 9):
+        ref, _ = oracle.scan(cv[0][:, :, h], cv[1][:, :, h], cv[2][:, :, h], la[:, :, h], bt[:, :, h])
+        assert_parity(got[:, :, h], ref, "bf16", f"head {h}")
+
+
+def test_bf16_tensor_core_state_io(kda):
+    """Initial and final state through the tensor-core path (d = 128)."""
+    import dataclasses
+    w = dataclasses.replace(kda_synth.WORKLOADS[1], text_len=100, grid=(2, 9, 13))
+    inp = kda_synth.generate(w, 31)
+    B, N, H, d = inp["shape"]
+    S0 = kda_synth.initial_state(8, B, H, d, d, std=0.05)
+    ref, ref_s = oracle.forward(inp, w.text_len, w.grid, S0=S0, heads=[0, 3])
+    o, s = run_fwd(kda, w, inp, S0=S0, want_state=True)
+    for h in (0, 3):
+        assert_parity(o[:, :, h], ref[:, :, h], "bf16", f"head {h}")
+        assert rel_l2(s[:, h], ref_s[:, h]) < 5e-3
+
+
+def test_bf16_tensor_core_continuation(kda):
+    """Two kda_chunk_fwd calls chained through the state equal one call (bf16, d = 128)."""
+    w = kda_synth.WORKLOADS[1]
+    inp = workload_inputs(1)
+    B, N, H, d = inp["shape"]
+    t = to_device(inp)
+    q, k, v = (t[n] for n in "qkv")
+
+    def call(lo, hi, s0):
+        pp = kda.problem(B, H, d, hi - lo, (0, 0, 0))
+        o = torch.empty(B, hi - lo, H, d, dtype=q.dtype, device="cuda")
+        sn = torch.empty(B, H, d, d, device="cuda")
+        ws = kda.alloc_workspace(pp, q.dtype)
+        kda.kda_chunk_fwd(pp, *(x[:, lo:hi].contiguous() for x in (q, k, v, t["log_alpha"], t["beta"])), o, ws,
+                          initial_state=s0, final_state=sn)
+        assert kda.kda_read_status(ws) == kda.KDA_OK
+        return o, sn
+    o_full, s_full = call(0, N, None)
+    m = 1000   # not a multiple of the 128-token block
+    o_a, s_a = call(0, m, None)
+    o_b, s_b = call(m, N, s_a)
+    o_split = torch.cat([o_a, o_b], dim=1).float().cpu().numpy()
+    assert rel_l2(o_split, o_full.float().cpu().numpy()) < 2e-3
+    assert rel_l2(s_b.cpu().numpy(), s_full.cpu().numpy()) < 2e-3
+
+
+def test_bf16_range_guard_reports_status(kda):
+    """Gates too strong for the tensor-core path's fp16 factors are reported
+    (KDA_ERR_RANGE) instead of silently returning wrong values."""
+    import dataclasses
+    w = dataclasses.replace(kda_synth.WORKLOADS[1], text_len=64, grid=(1, 8, 8))
+    inp = kda_synth.generate(w, 5)
+    la = inp["log_alpha"].reshape(1, -1, w.H, w.d)
+    la[0, 3:40, 2, 7] = -1.0        # 37 nats of decay inside one 64-token sub-chunk
+    inp["log_alpha"] = la.reshape(-1).copy()
+    B, N, H, d = inp["shape"]
+    p = kda.problem(B, H, d, w.text_len, w.grid)
+    t = to_device(inp)
+    o = torch.empty_like(t["q"])
+    ws = kda.alloc_workspace(p, t["q"].dtype)
+    kda.kda_fwd(p, t["q"], t["k"], t["v"], t["log_alpha"], t["beta"], t["w_text"], t["w_vis"], o, ws)
+    assert kda.kda_read_status(ws) == kda.KDA_ERR_RANGE
 
 
 def test_chunk_length_invariance_and_continuation(kda):
