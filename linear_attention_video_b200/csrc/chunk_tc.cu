@@ -46,7 +46,7 @@ constexpr float kRange = 9.f;     // max |g - g_m| allowed for the fp16 factors
 constexpr size_t kMBytes = 32768;   // M: fp16, 2 K-major panels [128][64]
 constexpr size_t kBBytes = 65536;   // B: fp32, [half][c/4][a][4]
 constexpr size_t kRBytes = 32768;   // R: fp16, 2 K-major panels [128][64]
-constexpr size_t kOBytes = 65536;   // O'': fp32 [128][128]
+constexpr size_t kOBytes = 65536;   // O'': fp32, float4 units [c/4][r]
 constexpr size_t kSBytes = 32768;   // S entering the block: fp16, 2 MN-major panels [128][64]
 constexpr size_t kBlockBytes = kMBytes + kBBytes + kRBytes + kOBytes + kSBytes;
 
@@ -206,6 +206,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a) {
   float* gm_s = ekt + 128;                                      // 128
   float* tot_s = gm_s + 128;                                    // 128
   uint64_t* bar = reinterpret_cast<uint64_t*>(tot_s + 128);
+  uint64_t* ldbar = bar + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 2);
   int* range_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
@@ -225,12 +226,12 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a) {
 
   if (*(volatile uint32_t*)a.status == KDA_ERR_TIMEOUT) return;   // an earlier CTA gave up: skip the work
   if (warp == 0) { tmem_alloc(tmem_slot, 512); tmem_relinquish(); }
-  if (tid == 0) { mbar_init(bar, 1); fence_mbar_init(); *range_flag = 0; }
+  if (tid == 0) { mbar_init(bar, 1); mbar_init(ldbar, 1); fence_mbar_init(); *range_flag = 0; }
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
   const uint32_t tm = *tmem_slot;
-  uint32_t phase = 0;
+  uint32_t phase = 0, ldphase = 0;
   bool alive = true;
 
   const uint32_t id_ap = idesc_f16(128, 64, false, false);
@@ -242,30 +243,48 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a) {
     const int64_t t0 = (int64_t)blk * BLK + s * SUB;
     const int nv = (int)max((int64_t)0, min((int64_t)SUB, a.N - t0));
     // ---------------- load + gate factors ----------------
+    // raw k, q, v rows (256 B each) -> staging by bulk copies; staging lives in
+    // the solve scratch and T/P tiles, which are dead at this point
+    uint8_t* stg_k = sm + OFF_AS;
+    uint8_t* stg_q = sm + OFF_AS + 16384;
+    uint8_t* stg_v = sm + OFF_TT;
+    if (tid == 0 && nv > 0) {
+      mbar_arrive_expect_tx(ldbar, (uint32_t)nv * 768u);
+      for (int r = 0; r < nv; ++r) {
+        const int64_t go = (t0 + r) * tok_stride;
+        bulk_g2s(stg_k + r * 256, kb + go, 256, ldbar);
+        bulk_g2s(stg_q + r * 256, qb + go, 256, ldbar);
+        bulk_g2s(stg_v + r * 256, vb + go, 256, ldbar);
+      }
+    }
     {
       const int c = tid & 127, half = tid >> 7;
-      float g = 0.f;
       float gl[32];
-#pragma unroll 8
+#pragma unroll
       for (int t = 0; t < 32; ++t) {
         const int tok = 32 * half + t;
-        const float x = tok < nv ? lab[(t0 + tok) * tok_stride + c] : 0.f;
-        g += x;
-        gl[t] = g;
+        gl[t] = tok < nv ? lab[(t0 + tok) * tok_stride + c] : 0.f;
       }
+#pragma unroll
+      for (int t = 1; t < 32; ++t) gl[t] += gl[t - 1];
       // half 0: factors relative to its own last value (g_m); half 1: g is already relative to g_m
       const float ref = half == 0 ? gl[31] : 0.f;
       if (half == 0) gm_s[c] = gl[31]; else tot_s[c] = gl[31];
       const float worst = half == 0 ? gl[0] - gl[31] : -gl[31];
       if (worst > kRange) *range_flag = 1;
+      if (tid < SUB) beta_s[tid] = tid < nv ? __bfloat162float(bb[(t0 + tid) * a.H]) : 0.f;
+      bool got = true;
+      if (nv > 0) got = mbar_wait(ldbar, ldphase);
+      ldphase ^= (nv > 0) ? 1u : 0u;
+      if (!got) set_status(a.status, KDA_ERR_TIMEOUT);
 #pragma unroll 4
       for (int t = 0; t < 32; ++t) {
         const int tok = 32 * half + t;
         float kv = 0.f, qv = 0.f, vv = 0.f;
-        if (tok < nv) {
-          kv = ld_act(kb + (t0 + tok) * tok_stride + c);
-          qv = ld_act(qb + (t0 + tok) * tok_stride + c);
-          vv = ld_act(vb + (t0 + tok) * tok_stride + c);
+        if (tok < nv && got) {
+          kv = ld_act(reinterpret_cast<const TIn*>(stg_k + tok * 256) + c);
+          qv = ld_act(reinterpret_cast<const TIn*>(stg_q + tok * 256) + c);
+          vv = ld_act(reinterpret_cast<const TIn*>(stg_v + tok * 256) + c);
         }
         const float x = gl[t] - ref;
         const float ep = __expf(x), en = __expf(-x);
@@ -275,7 +294,6 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a) {
         st_h(KN + pnl * 8192, swz_off(tok, cc), kv * en);
         st_h(VV + pnl * 8192, swz_off(tok, cc), vv);
       }
-      if (tid < SUB) beta_s[tid] = tid < nv ? ld_act(bb + (t0 + tid) * a.H) : 0.f;
     }
     fence_proxy_async();
     __syncthreads();
@@ -431,9 +449,10 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a) {
 #pragma unroll
           for (int j = 0; j < 16; ++j) qg[j] = (qg[j] - pw[j]) * egm[col0 + j];
           st_row16_h(gR + (col0 >> 6) * 16384, r, col0 & 63, qg);
-          float4* o4 = reinterpret_cast<float4*>(gO + r * 128 + col0);
+          float4* o4 = reinterpret_cast<float4*>(gO);
 #pragma unroll
-          for (int j = 0; j < 4; ++j) o4[j] = make_float4(pu[4 * j], pu[4 * j + 1], pu[4 * j + 2], pu[4 * j + 3]);
+          for (int j = 0; j < 4; ++j)
+            o4[((col0 >> 2) + j) * 128 + r] = make_float4(pu[4 * j], pu[4 * j + 1], pu[4 * j + 2], pu[4 * j + 3]);
         }
       }
       fence_proxy_async();
@@ -519,9 +538,11 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a) {
           tmem_wait_ld();
           if (lane < 16) {
             st_row16_h(gR + (col0 >> 6) * 16384, 64 + r, col0 & 63, rr);
-            float4* o4 = reinterpret_cast<float4*>(gO + (64 + r) * 128 + col0);
+            float4* o4 = reinterpret_cast<float4*>(gO);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) o4[j] = make_float4(oo[4 * j], oo[4 * j + 1], oo[4 * j + 2], oo[4 * j + 3]);
+            for (int j = 0; j < 4; ++j)
+              o4[((col0 >> 2) + j) * 128 + 64 + r] =
+                  make_float4(oo[4 * j], oo[4 * j + 1], oo[4 * j + 2], oo[4 * j + 3]);
           }
         }
       }
@@ -591,12 +612,9 @@ __global__ void __launch_bounds__(128, 1) kda_tc_chain(ChainArgs a) {
     S[c] = a.S0 ? a.S0[(((int64_t)b * a.H + h) * D + row) * D + 64 * half + c] : 0.f;
 
   const uint32_t idesc = idesc_f16(128, 64, false, true);
-  uint32_t mphase = 0;
-  bool ok = true;
-  int j = 0;
-  for (; j < a.n_blocks; ++j) {
-    // S (fp16) -> shared B operand and -> workspace (state entering block j)
-    uint8_t* gS = a.ws + (rec0 + j) * kBlockBytes + kMBytes + kBBytes + kRBytes + kOBytes + half * 16384;
+  auto state_out = [&](int jj) {
+    // S (fp16) -> shared B operand and -> workspace (state entering block jj)
+    uint8_t* gS = a.ws + (rec0 + jj) * kBlockBytes + kMBytes + kBBytes + kRBytes + kOBytes + half * 16384;
 #pragma unroll
     for (int c0 = 0; c0 < 64; c0 += 16) {
       float v[16];
@@ -606,18 +624,28 @@ __global__ void __launch_bounds__(128, 1) kda_tc_chain(ChainArgs a) {
       st_row16_h(gS, row, c0, v);
     }
     fence_proxy_async();
+  };
+  state_out(0);
+  __syncthreads();
+  uint32_t mphase = 0;
+  bool ok = true;
+  int j = 0;
+  for (; j < a.n_blocks; ++j) {
     const int st = j % CH_STAGES;
-    const bool got = mbar_wait(&bars[st], (uint32_t)(j / CH_STAGES) & 1u);
-    ok = __syncthreads_and(got) && ok;
-    if (!ok) break;
     uint8_t* stage = sm + CH_OFF_RING + st * CH_STAGE_BYTES;
+    bool issued_ok = true;
     if (tid == 0) {
-      fence_after_sync();
-      for (int k16 = 0; k16 < 8; ++k16)
-        mma_ss(tmem_at(tm, 0, 0), desc_kmajor(smem_u32(stage), k16, 16384), desc_mnmajor(smem_u32(Ssm), k16, 16384),
-               idesc, k16 > 0);
-      mma_commit(&bars[3]);
+      issued_ok = mbar_wait(&bars[st], (uint32_t)(j / CH_STAGES) & 1u);
+      if (issued_ok) {
+        fence_after_sync();
+        for (int k16 = 0; k16 < 8; ++k16)
+          mma_ss(tmem_at(tm, 0, 0), desc_kmajor(smem_u32(stage), k16, 16384), desc_mnmajor(smem_u32(Ssm), k16, 16384),
+                 idesc, k16 > 0);
+        mma_commit(&bars[3]);
+      }
     }
+    ok = __syncthreads_and(issued_ok) && ok;
+    if (!ok) break;
     const bool done = mbar_wait(&bars[3], mphase);
     mphase ^= 1u;
     ok = __syncthreads_and(done) && ok;
@@ -625,21 +653,24 @@ __global__ void __launch_bounds__(128, 1) kda_tc_chain(ChainArgs a) {
     fence_after_sync();
     const float4* Bs = reinterpret_cast<const float4*>(stage + 32768);
 #pragma unroll
-    for (int c0 = 0; c0 < 64; c0 += 16) {
-      float v[16];
-      tmem_ld16(tmem_at(tm, 32 * warp, c0), v);
+    for (int c0 = 0; c0 < 64; c0 += 32) {
+      float v[32];
+      tmem_ld32(tmem_at(tm, 32 * warp, c0), v);
+      float4 bv[8];
+#pragma unroll
+      for (int q4 = 0; q4 < 8; ++q4) bv[q4] = Bs[((c0 >> 2) + q4) * 128 + row];
       tmem_wait_ld();
 #pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        const float4 bv = Bs[((c0 >> 2) + q4) * 128 + row];
-        S[c0 + 4 * q4 + 0] = v[4 * q4 + 0] + bv.x;
-        S[c0 + 4 * q4 + 1] = v[4 * q4 + 1] + bv.y;
-        S[c0 + 4 * q4 + 2] = v[4 * q4 + 2] + bv.z;
-        S[c0 + 4 * q4 + 3] = v[4 * q4 + 3] + bv.w;
+      for (int q4 = 0; q4 < 8; ++q4) {
+        S[c0 + 4 * q4 + 0] = v[4 * q4 + 0] + bv[q4].x;
+        S[c0 + 4 * q4 + 1] = v[4 * q4 + 1] + bv[q4].y;
+        S[c0 + 4 * q4 + 2] = v[4 * q4 + 2] + bv[q4].z;
+        S[c0 + 4 * q4 + 3] = v[4 * q4 + 3] + bv[q4].w;
       }
     }
+    if (j + 1 < a.n_blocks) state_out(j + 1);
     fence_before_sync();
-    __syncthreads();   // stage consumed, TMEM read
+    __syncthreads();   // stage j consumed, TMEM read, next S in shared memory
     if (tid == 0 && j + CH_STAGES < a.n_blocks) issue(j + CH_STAGES);
   }
   if (!ok) {
@@ -706,17 +737,29 @@ __global__ void __launch_bounds__(128) kda_tc_out(uint8_t* ws, TOut* o, int64_t 
     fence_after_sync();
     const int r = tid;  // token row within the block = TMEM lane
     const int64_t tok = (int64_t)blk * BLK + r;
-    const float* Oo = reinterpret_cast<const float*>(rec + kMBytes + kBBytes + kRBytes) + r * 128;
+    const float4* Oo = reinterpret_cast<const float4*>(rec + kMBytes + kBBytes + kRBytes);
     TOut* orow = o + ((int64_t)b * N + tok) * H * D + (int64_t)h * D;
-    for (int c0 = 0; c0 < 128; c0 += 16) {
-      float v[16];
-      tmem_ld16(tmem_at(tm, 32 * warp, c0), v);
+    for (int c0 = 0; c0 < 128; c0 += 32) {
+      float v[32];
+      tmem_ld32(tmem_at(tm, 32 * warp, c0), v);
+      float4 oo[8];
+#pragma unroll
+      for (int q4 = 0; q4 < 8; ++q4) oo[q4] = __ldg(Oo + ((c0 >> 2) + q4) * 128 + r);
       tmem_wait_ld();
       if (tok < N) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) v[j] += Oo[c0 + j];
+        for (int q4 = 0; q4 < 8; ++q4) {
+          v[4 * q4] += oo[q4].x; v[4 * q4 + 1] += oo[q4].y; v[4 * q4 + 2] += oo[q4].z; v[4 * q4 + 3] += oo[q4].w;
+        }
+        uint32_t w[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) orow[c0 + j] = from_f32<TOut>(v[j]);
+        for (int j = 0; j < 16; ++j) {
+          __nv_bfloat162 hh = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
+          w[j] = *reinterpret_cast<uint32_t*>(&hh);
+        }
+        uint4* dst = reinterpret_cast<uint4*>(orow + c0);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) dst[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
       }
     }
   }
