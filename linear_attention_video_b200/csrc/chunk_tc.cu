@@ -53,11 +53,14 @@ constexpr size_t kBlockBytes = kMBytes + kBBytes + kRBytes + kOBytes + kSBytes;
 // ---------------------------------------------------------------------------
 // small helpers
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ float ld_act(const __half* p) { return __half2float(*p); }
-__device__ __forceinline__ float ld_act(const __nv_bfloat16* p) { return __bfloat162float(*p); }
 
-__device__ __forceinline__ void st_h(uint8_t* tile, uint32_t off, float v) {
-  *reinterpret_cast<__half*>(tile + off) = __float2half_rn(v);
+__device__ __forceinline__ float2 ld_act2(const __half* p) { return __half22float2(*reinterpret_cast<const __half2*>(p)); }
+__device__ __forceinline__ float2 ld_act2(const __nv_bfloat16* p) {
+  return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
+}
+
+__device__ __forceinline__ void st_h2(uint8_t* p, float a, float b) {
+  *reinterpret_cast<__half2*>(p) = __floats2half2_rn(a, b);
 }
 
 // 16 consecutive fp32 values -> 16 fp16 at (row, col0..col0+15) of a swizzled panel.
@@ -148,41 +151,57 @@ __device__ void unit_lower_inverse64(const float* As, float* Xs, float* Ys) {
     for (int r = 0; r < 16; ++r) Xs[(o + r) * LDX + o + l] = x[r];
   }
   __syncthreads();
-  // 32x32 merges: for p in {0,1}: X[32p+16.., 32p..] = -X22 (A21 X11)
+  // 32x32 merges: for p in {0,1}: X[32p+16.., 32p..] = -X22 (A21 X11); one 2x1 tile per thread
   {
-    const int p = tid >> 7, e0 = tid & 127;
+    const int p = tid >> 7, e = tid & 127;
     const int o = 32 * p;
     float* Y = Ys + p * 16 * 17;
-    for (int e = e0; e < 256; e += 128) {
-      const int r = e >> 4, c = e & 15;
-      float acc = 0.f;
-      for (int m = c; m < 16; ++m) acc += As[(o + 16 + r) * LDX + o + m] * Xs[(o + m) * LDX + o + c];
-      Y[r * 17 + c] = acc;
+    const int r0 = 2 * (e >> 4), c = e & 15;
+    {
+      float a0 = 0.f, a1 = 0.f;
+      for (int m = c; m < 16; ++m) {
+        const float x = Xs[(o + m) * LDX + o + c];
+        a0 += As[(o + 16 + r0) * LDX + o + m] * x;
+        a1 += As[(o + 17 + r0) * LDX + o + m] * x;
+      }
+      Y[r0 * 17 + c] = a0;
+      Y[(r0 + 1) * 17 + c] = a1;
     }
     __syncthreads();
-    for (int e = e0; e < 256; e += 128) {
-      const int r = e >> 4, c = e & 15;
-      float acc = 0.f;
-      for (int m = 0; m <= r; ++m) acc += Xs[(o + 16 + r) * LDX + o + 16 + m] * Y[m * 17 + c];
-      Xs[(o + 16 + r) * LDX + o + c] = -acc;
+    {
+      float a0 = 0.f, a1 = 0.f;
+      for (int m = 0; m <= r0 + 1; ++m) {
+        const float y = Y[m * 17 + c];
+        a0 += (m <= r0 ? Xs[(o + 16 + r0) * LDX + o + 16 + m] : 0.f) * y;
+        a1 += Xs[(o + 17 + r0) * LDX + o + 16 + m] * y;
+      }
+      Xs[(o + 16 + r0) * LDX + o + c] = -a0;
+      Xs[(o + 17 + r0) * LDX + o + c] = -a1;
     }
     __syncthreads();
   }
-  // 64 merge: X[32.., 0..31] = -X22 (A21 X11)
-  for (int e = tid; e < 1024; e += 256) {
-    const int r = e >> 5, c = e & 31;
-    float acc = 0.f;
-    for (int m = c; m < 32; ++m) acc += As[(32 + r) * LDX + m] * Xs[m * LDX + c];
-    Ys[r * 33 + c] = acc;
+  // 64 merge: X[32.., 0..31] = -X22 (A21 X11); one 2x2 tile per thread
+  {
+    const int r0 = 2 * (tid >> 4), c0 = 2 * (tid & 15);
+    float a00 = 0.f, a01 = 0.f, a10 = 0.f, a11 = 0.f;
+    for (int m = c0; m < 32; ++m) {
+      const float x0 = Xs[m * LDX + c0], x1 = Xs[m * LDX + c0 + 1];
+      const float u0 = As[(32 + r0) * LDX + m], u1 = As[(33 + r0) * LDX + m];
+      a00 += u0 * x0; a01 += u0 * x1; a10 += u1 * x0; a11 += u1 * x1;
+    }
+    Ys[r0 * 33 + c0] = a00; Ys[r0 * 33 + c0 + 1] = a01;
+    Ys[(r0 + 1) * 33 + c0] = a10; Ys[(r0 + 1) * 33 + c0 + 1] = a11;
+    __syncthreads();
+    a00 = a01 = a10 = a11 = 0.f;
+    for (int m = 0; m <= r0 + 1; ++m) {
+      const float y0 = Ys[m * 33 + c0], y1 = Ys[m * 33 + c0 + 1];
+      const float u0 = m <= r0 ? Xs[(32 + r0) * LDX + 32 + m] : 0.f, u1 = Xs[(33 + r0) * LDX + 32 + m];
+      a00 += u0 * y0; a01 += u0 * y1; a10 += u1 * y0; a11 += u1 * y1;
+    }
+    Xs[(32 + r0) * LDX + c0] = -a00; Xs[(32 + r0) * LDX + c0 + 1] = -a01;
+    Xs[(33 + r0) * LDX + c0] = -a10; Xs[(33 + r0) * LDX + c0 + 1] = -a11;
+    __syncthreads();
   }
-  __syncthreads();
-  for (int e = tid; e < 1024; e += 256) {
-    const int r = e >> 5, c = e & 31;
-    float acc = 0.f;
-    for (int m = 0; m <= r; ++m) acc += Xs[(32 + r) * LDX + 32 + m] * Ys[m * 33 + c];
-    Xs[(32 + r) * LDX + c] = -acc;
-  }
-  __syncthreads();
 }
 
 template <typename TIn>
@@ -206,7 +225,6 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a) {
   float* gm_s = ekt + 128;                                      // 128
   float* tot_s = gm_s + 128;                                    // 128
   uint64_t* bar = reinterpret_cast<uint64_t*>(tot_s + 128);
-  uint64_t* ldbar = bar + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 2);
   int* range_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
@@ -226,12 +244,12 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a) {
 
   if (*(volatile uint32_t*)a.status == KDA_ERR_TIMEOUT) return;   // an earlier CTA gave up: skip the work
   if (warp == 0) { tmem_alloc(tmem_slot, 512); tmem_relinquish(); }
-  if (tid == 0) { mbar_init(bar, 1); mbar_init(ldbar, 1); fence_mbar_init(); *range_flag = 0; }
+  if (tid == 0) { mbar_init(bar, 1); fence_mbar_init(); *range_flag = 0; }
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
   const uint32_t tm = *tmem_slot;
-  uint32_t phase = 0, ldphase = 0;
+  uint32_t phase = 0;
   bool alive = true;
 
   const uint32_t id_ap = idesc_f16(128, 64, false, false);
@@ -243,56 +261,74 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a) {
     const int64_t t0 = (int64_t)blk * BLK + s * SUB;
     const int nv = (int)max((int64_t)0, min((int64_t)SUB, a.N - t0));
     // ---------------- load + gate factors ----------------
-    // raw k, q, v rows (256 B each) -> staging by bulk copies; staging lives in
-    // the solve scratch and T/P tiles, which are dead at this point
+    // raw k, q, v rows (256 B each) -> staging with 16-byte asynchronous copies
+    // spread over all threads; staging lives in the solve scratch and T/P
+    // tiles, which are dead at this point
     uint8_t* stg_k = sm + OFF_AS;
     uint8_t* stg_q = sm + OFF_AS + 16384;
     uint8_t* stg_v = sm + OFF_TT;
-    if (tid == 0 && nv > 0) {
-      mbar_arrive_expect_tx(ldbar, (uint32_t)nv * 768u);
-      for (int r = 0; r < nv; ++r) {
-        const int64_t go = (t0 + r) * tok_stride;
-        bulk_g2s(stg_k + r * 256, kb + go, 256, ldbar);
-        bulk_g2s(stg_q + r * 256, qb + go, 256, ldbar);
-        bulk_g2s(stg_v + r * 256, vb + go, 256, ldbar);
-      }
+    for (int e = tid; e < nv * 16; e += 256) {
+      const int r = e >> 4, ch = (e & 15) * 8;     // row, first of 8 channels
+      const int64_t go = (t0 + r) * tok_stride + ch;
+      cp_async16(stg_k + r * 256 + ch * 2, kb + go);
+      cp_async16(stg_q + r * 256 + ch * 2, qb + go);
+      cp_async16(stg_v + r * 256 + ch * 2, vb + go);
     }
+    cp_async_commit();
     {
-      const int c = tid & 127, half = tid >> 7;
-      float gl[32];
+      // thread: channels 2cp, 2cp+1 and tokens 16*qt .. 16*qt+15 of the sub-chunk
+      const int cp = (tid & 31) + 32 * ((tid >> 5) & 1);
+      const int qt = tid >> 6;
+      const int c = 2 * cp;
+      float2 gl[16];
 #pragma unroll
-      for (int t = 0; t < 32; ++t) {
-        const int tok = 32 * half + t;
-        gl[t] = tok < nv ? lab[(t0 + tok) * tok_stride + c] : 0.f;
+      for (int t = 0; t < 16; ++t) {
+        const int tok = 16 * qt + t;
+        gl[t] = tok < nv ? *reinterpret_cast<const float2*>(lab + (t0 + tok) * tok_stride + c) : make_float2(0.f, 0.f);
       }
 #pragma unroll
-      for (int t = 1; t < 32; ++t) gl[t] += gl[t - 1];
-      // half 0: factors relative to its own last value (g_m); half 1: g is already relative to g_m
-      const float ref = half == 0 ? gl[31] : 0.f;
-      if (half == 0) gm_s[c] = gl[31]; else tot_s[c] = gl[31];
-      const float worst = half == 0 ? gl[0] - gl[31] : -gl[31];
-      if (worst > kRange) *range_flag = 1;
+      for (int t = 1; t < 16; ++t) { gl[t].x += gl[t - 1].x; gl[t].y += gl[t - 1].y; }
+      float2* qtot = reinterpret_cast<float2*>(Ys);      // [4][64] quarter totals (Ys is free here)
+      qtot[qt * 64 + cp] = gl[15];
       if (tid < SUB) beta_s[tid] = tid < nv ? __bfloat162float(bb[(t0 + tid) * a.H]) : 0.f;
-      bool got = true;
-      if (nv > 0) got = mbar_wait(ldbar, ldphase);
-      ldphase ^= (nv > 0) ? 1u : 0u;
-      if (!got) set_status(a.status, KDA_ERR_TIMEOUT);
+      __syncthreads();
+      float2 pre = make_float2(0.f, 0.f), gmv = make_float2(0.f, 0.f), tot = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 v = qtot[j * 64 + cp];
+        if (j < qt) { pre.x += v.x; pre.y += v.y; }
+        if (j < 2) { gmv.x += v.x; gmv.y += v.y; } else { tot.x += v.x; tot.y += v.y; }
+      }
+      if (qt == 0) {
+        gm_s[c] = gmv.x; gm_s[c + 1] = gmv.y;       // g_m: decay through token 31
+        tot_s[c] = tot.x; tot_s[c + 1] = tot.y;     // decay over tokens 32..63
+      }
+      // exponent x = g - g_m; the extremes sit at token 0 and token 63
+      if (qt == 0 && (pre.x + gl[0].x - gmv.x > kRange || pre.y + gl[0].y - gmv.y > kRange)) *range_flag = 1;
+      if (qt == 3 && (-tot.x > kRange || -tot.y > kRange)) *range_flag = 1;
+      cp_async_wait_all();
+      __syncthreads();
+      const bool got = true;
+      const int pnl = c >> 6, cc = c & 63;
+      uint8_t* kq = KQ + pnl * 16384;
+      uint8_t* kn = KN + pnl * 8192;
+      uint8_t* vv = VV + pnl * 8192;
 #pragma unroll 4
-      for (int t = 0; t < 32; ++t) {
-        const int tok = 32 * half + t;
-        float kv = 0.f, qv = 0.f, vv = 0.f;
+      for (int t = 0; t < 16; ++t) {
+        const int tok = 16 * qt + t;
+        float2 kv = make_float2(0.f, 0.f), qv = kv, vv2 = kv;
         if (tok < nv && got) {
-          kv = ld_act(reinterpret_cast<const TIn*>(stg_k + tok * 256) + c);
-          qv = ld_act(reinterpret_cast<const TIn*>(stg_q + tok * 256) + c);
-          vv = ld_act(reinterpret_cast<const TIn*>(stg_v + tok * 256) + c);
+          kv = ld_act2(reinterpret_cast<const TIn*>(stg_k + tok * 256) + c);
+          qv = ld_act2(reinterpret_cast<const TIn*>(stg_q + tok * 256) + c);
+          vv2 = ld_act2(reinterpret_cast<const TIn*>(stg_v + tok * 256) + c);
         }
-        const float x = gl[t] - ref;
-        const float ep = __expf(x), en = __expf(-x);
-        const int pnl = c >> 6, cc = c & 63;
-        st_h(KQ + pnl * 16384, swz_off(tok, cc), kv * ep);
-        st_h(KQ + pnl * 16384, swz_off(64 + tok, cc), qv * ep);
-        st_h(KN + pnl * 8192, swz_off(tok, cc), kv * en);
-        st_h(VV + pnl * 8192, swz_off(tok, cc), vv);
+        const float x0 = pre.x + gl[t].x - gmv.x, x1 = pre.y + gl[t].y - gmv.y;
+        const float ep0 = __expf(x0), ep1 = __expf(x1), en0 = __expf(-x0), en1 = __expf(-x1);
+        const uint32_t off = swz_off(tok, cc);
+        st_h2(kq + off, kv.x * ep0, kv.y * ep1);
+        st_h2(kq + swz_off(64 + tok, cc), qv.x * ep0, qv.y * ep1);
+        st_h2(kn + off, kv.x * en0, kv.y * en1);
+        st_h2(vv + off, vv2.x, vv2.y);
       }
     }
     fence_proxy_async();
