@@ -119,6 +119,33 @@ int kda_fwd(const kda_problem* p, kda_dtype dtype,
             const float* initial_state, void* o, float* final_state,
             void* workspace, size_t workspace_bytes, void* stream);
 
+/* kda_chunk_fwd without a workspace, for callers that cannot allocate device
+ * memory (code running inside an allocator or memory-pool callback, runtimes
+ * that forbid allocation after start-up, plugins handed only their input and
+ * output buffers).  The pages describe no counterpart; this is an interface
+ * convenience.
+ *
+ * Same operation, arguments and errors as kda_chunk_fwd, with these differences:
+ *  - Scratch comes from a static device array of 64 MiB that the library holds
+ *    on every GPU that loads it, until the process exits.  A problem whose
+ *    scratch exceeds it (256 B + 224 KiB per (batch item, head, 128-token block)
+ *    on the bf16 d=128 tensor-core path) returns KDA_ERR_WORKSPACE without
+ *    launching anything.
+ *  - The first call on a device looks up that array's device address (once per
+ *    device); make it before any stream capture.
+ *  - Calls share the array: calls whose GPU work overlaps (other streams, other
+ *    host threads on the same device) race.  Run them on one stream.
+ *  - Device-side conditions (see kda_read_status) are written to *device_status
+ *    (a 4-byte-aligned device word, cleared at the start of the call) when it is
+ *    not NULL, otherwise to a word inside the static array that callers cannot
+ *    read.
+ *  - No cudaMalloc, cudaFree or other allocating call is made. */
+int kda_chunk_fwd_noalloc(const kda_problem* p, kda_dtype dtype,
+                          const void* q, const void* k, const void* v,
+                          const float* log_alpha, const void* beta,
+                          const float* initial_state, void* o, float* final_state,
+                          uint32_t* device_status, void* stream);
+
 /* Synchronises `stream`, then returns and clears the device status word kept
  * in `workspace` (KDA_OK if no device-side condition was recorded). */
 int kda_read_status(void* workspace, void* stream);

@@ -30,7 +30,7 @@ KDA_DT_BF16, KDA_DT_F32 = 0, 1
 KDA_FLAG_VIS_CAUSAL_T = 1
 
 EXPORTS = ("kda_tokens", "kda_workspace_bytes", "kda_shortconv_fwd", "kda_chunk_fwd", "kda_fwd",
-           "kda_read_status", "kda_status_str", "kda_last_launch_count")
+           "kda_chunk_fwd_noalloc", "kda_read_status", "kda_status_str", "kda_last_launch_count")
 
 
 class kda_problem(ctypes.Structure):
@@ -53,6 +53,8 @@ _lib.kda_chunk_fwd.argtypes = [_pp, _i] + [_vp] * 9 + [_sz, _vp]
 _lib.kda_chunk_fwd.restype = _i
 _lib.kda_fwd.argtypes = [_pp, _i] + [_vp] * 11 + [_sz, _vp]
 _lib.kda_fwd.restype = _i
+_lib.kda_chunk_fwd_noalloc.argtypes = [_pp, _i] + [_vp] * 10
+_lib.kda_chunk_fwd_noalloc.restype = _i
 _lib.kda_read_status.argtypes = [_vp, _vp]
 _lib.kda_read_status.restype = _i
 _lib.kda_status_str.argtypes = [_i]
@@ -150,6 +152,16 @@ def kda_fwd(p, q, k, v, log_alpha, beta, w_text, w_vis, o, workspace, initial_st
                         _ptr(w_text), _ptr(w_vis), _ptr(initial_state), _ptr(o), _ptr(final_state),
                         _ptr(workspace), nbytes, _stream(stream)),
            "kda_fwd")
+
+
+def kda_chunk_fwd_noalloc(p, q, k, v, log_alpha, beta, o, initial_state=None, final_state=None,
+                          device_status=None, stream=None):
+    """kda_chunk_fwd without a workspace: scratch is the library's static device
+    array (see include/kda.h for its limit and sharing rules)."""
+    _check(_lib.kda_chunk_fwd_noalloc(ctypes.byref(p), _dt(q.dtype), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
+                                      _ptr(beta), _ptr(initial_state), _ptr(o), _ptr(final_state),
+                                      _ptr(device_status), _stream(stream)),
+           "kda_chunk_fwd_noalloc")
 
 
 def kda_read_status(workspace, stream=None) -> int:

@@ -52,4 +52,9 @@ cudaError_t launch_chunk_tc(const Dims& d, bool in_f16, const void* q, const voi
                             const float* log_alpha, const void* beta, const float* S0, void* o, float* SN,
                             void* ws, uint32_t* status, cudaStream_t s, int* launches);
 
+// Host-side validation (kda_api.cu), returning a kda_status.
+int validate_problem(const kda_problem* p, kda_dtype dt, Dims* d);
+int validate_scan_pointers(const void* q, const void* k, const void* v, const void* la, const void* beta, const void* o,
+                           const void* s0, const void* sn);
+
 }  // namespace kda

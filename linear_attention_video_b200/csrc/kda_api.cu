@@ -103,6 +103,15 @@ int run_scan(const kda::Dims& d, kda_dtype dt, const void* q, const void* k, con
 
 }  // namespace
 
+namespace kda {
+// Validation shared with the allocation-free entry point (noalloc.cu).
+int validate_problem(const kda_problem* p, kda_dtype dt, Dims* d) { return make_dims(p, dt, d); }
+int validate_scan_pointers(const void* q, const void* k, const void* v, const void* la, const void* beta, const void* o,
+                           const void* s0, const void* sn) {
+  return check_ptrs({q, k, v, la, beta, o}, {s0, sn});
+}
+}  // namespace kda
+
 extern "C" {
 
 int64_t kda_tokens(const kda_problem* p) {
