@@ -128,7 +128,7 @@ int kda_fwd(const kda_problem* p, kda_dtype dtype,
  * Same operation, arguments and errors as kda_chunk_fwd, with these differences:
  *  - Scratch comes from a static device array of 64 MiB that the library holds
  *    on every GPU that loads it, until the process exits.  A problem whose
- *    scratch exceeds it (256 B + 224 KiB per (batch item, head, 128-token block)
+ *    scratch exceeds it (256 B + 128 KiB per (batch item, head, 128-token block)
  *    on the bf16 d=128 tensor-core path) returns KDA_ERR_WORKSPACE without
  *    launching anything.
  *  - The first call on a device looks up that array's device address (once per

@@ -19,13 +19,13 @@
 //   M = M_2 M_1,  B = M_2 B_1 + B_2,  R = [Q^_1 ; Q^_2 M_1],  O'' = [O'_1 ; Q^_2 B_1 + O'_2]
 // and the block maps S to O = R S + O'' and S <- M S + B.
 //
-// Three kernels:
-//   kda_tc_prep   one CTA per (batch item, head, block): everything above,
-//                 written to the workspace (M, B, R, O'' per block).
+// Two kernels:
+//   kda_tc_prep   persistent, one CTA per SM, looping over (block, batch item,
+//                 head) units: everything above, written to the workspace as one
+//                 record per unit (M, B, R, O'' in fp16 operand images).
 //   kda_tc_chain  one CTA per (batch item, head, half of the value columns):
 //                 the serial pass S <- M S + B, state kept in registers (fp32),
-//                 saving the state entering each block.
-//   kda_tc_out    one CTA per (batch item, head, block): O = R S + O''.
+//                 and beside it the block outputs O = R S + O''.
 // Padding tokens of the last block carry k = q = v = 0, beta = 0, log alpha = 0.
 #include "common.cuh"
 #include "tc.cuh"
@@ -42,51 +42,63 @@ constexpr int SUB = 64;           // tokens per sub-chunk
 constexpr int D = 128;            // d_k = d_v
 constexpr float kRange = 9.f;     // max |g - g_m| allowed for the fp16 factors
 
-// Workspace bytes per (batch item, head, block).
-constexpr size_t kMBytes = 32768;   // M: fp16, 2 K-major panels [128][64]
-constexpr size_t kBBytes = 65536;   // B: fp32, [half][c/4][a][4]
-constexpr size_t kRBytes = 32768;   // R: fp16, 2 K-major panels [128][64]
-constexpr size_t kOBytes = 65536;   // O'': fp32, float4 units [c/4][r]
-constexpr size_t kSBytes = 32768;   // S entering the block: fp16, 2 MN-major panels [128][64]
-constexpr size_t kBlockBytes = kMBytes + kBBytes + kRBytes + kOBytes + kSBytes;
+// Record per (batch item, head, block), all fp16:
+//   M   K-major operand image: 2 panels [128 rows][64 cols]            32 KB
+//   B   [half][c/8][row a][8]  (16-byte units)                         32 KB
+//   R   K-major operand image: 2 panels [128 rows][64 cols]            32 KB
+//   O'' [c/8][row r][8]        (16-byte units)                         32 KB
+constexpr size_t kMOff = 0, kBOff = 32768, kROff = 65536, kOOff = 98304;
+constexpr size_t kBlockBytes = 131072;
 
 // ---------------------------------------------------------------------------
 // small helpers
 // ---------------------------------------------------------------------------
+template <typename T> constexpr bool kIsHalf = false;
+template <> constexpr bool kIsHalf<__half> = true;
 
-__device__ __forceinline__ float2 ld_act2(const __half* p) { return __half22float2(*reinterpret_cast<const __half2*>(p)); }
-__device__ __forceinline__ float2 ld_act2(const __nv_bfloat16* p) {
+__device__ __forceinline__ float2 ld_act2(const uint8_t* p, __half*) {
+  return __half22float2(*reinterpret_cast<const __half2*>(p));
+}
+__device__ __forceinline__ float2 ld_act2(const uint8_t* p, __nv_bfloat16*) {
   return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
 }
-
 __device__ __forceinline__ void st_h2(uint8_t* p, float a, float b) {
   *reinterpret_cast<__half2*>(p) = __floats2half2_rn(a, b);
 }
-
-// 16 consecutive fp32 values -> 16 fp16 at (row, col0..col0+15) of a swizzled panel.
-__device__ __forceinline__ void st_row16_h(uint8_t* panel, int row, int col0, const float (&v)[16]) {
-  uint32_t w[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    __half2 h = __floats2half2_rn(v[2 * i], v[2 * i + 1]);
-    w[i] = *reinterpret_cast<uint32_t*>(&h);
-  }
-  *reinterpret_cast<uint4*>(panel + swz_off(row, col0)) = make_uint4(w[0], w[1], w[2], w[3]);
-  *reinterpret_cast<uint4*>(panel + swz_off(row, col0 + 8)) = make_uint4(w[4], w[5], w[6], w[7]);
+__device__ __forceinline__ uint32_t pack_h2(float a, float b) {
+  __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
 }
-
-// 16 fp16 at (row, col0..) of a swizzled panel -> fp32
-__device__ __forceinline__ void ld_row16_h(const uint8_t* panel, int row, int col0, float (&v)[16]) {
-  const uint4 a = *reinterpret_cast<const uint4*>(panel + swz_off(row, col0));
-  const uint4 b = *reinterpret_cast<const uint4*>(panel + swz_off(row, col0 + 8));
-  const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+__device__ __forceinline__ uint4 pack8(const float* v) {
+  return make_uint4(pack_h2(v[0], v[1]), pack_h2(v[2], v[3]), pack_h2(v[4], v[5]), pack_h2(v[6], v[7]));
+}
+__device__ __forceinline__ void unpack8(uint4 u, float* v) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const __half2 h = *reinterpret_cast<const __half2*>(&w[i]);
-    const float2 f = __half22float2(h);
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[i]));
     v[2 * i] = f.x;
     v[2 * i + 1] = f.y;
   }
+}
+
+// 32 consecutive fp32 values -> fp16 at (row, col0..col0+31) of a swizzled
+// panel (col0 a multiple of 32).  The four 16-byte chunks are written in an
+// order rotated by `rot`, so rows that share a bank group (row, row+8, ...)
+// write different chunks at the same time.
+__device__ __forceinline__ void st_row32_h(uint8_t* panel, int row, int col0, const float (&v)[32], int rot) {
+  const uint4 p0 = pack8(v), p1 = pack8(v + 8), p2 = pack8(v + 16), p3 = pack8(v + 24);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int c = (i + rot) & 3;
+    const uint4 d = c == 0 ? p0 : c == 1 ? p1 : c == 2 ? p2 : p3;
+    *reinterpret_cast<uint4*>(panel + swz_off(row, col0 + 8 * c)) = d;
+  }
+}
+// 16 consecutive fp16 values at (row, col0..) of a swizzled panel -> fp32
+__device__ __forceinline__ void ld_row16_h(const uint8_t* panel, int row, int col0, float* v) {
+  unpack8(*reinterpret_cast<const uint4*>(panel + swz_off(row, col0)), v);
+  unpack8(*reinterpret_cast<const uint4*>(panel + swz_off(row, col0 + 8)), v + 8);
 }
 
 __device__ __forceinline__ uint32_t tmem_at(uint32_t base, int lane0, int col) {
@@ -106,17 +118,17 @@ __device__ __forceinline__ bool wait_mma(uint64_t* bar, uint32_t& phase, uint32_
 // kda_tc_prep
 // ---------------------------------------------------------------------------
 // shared memory map (bytes from a 1024-aligned base)
-constexpr uint32_t OFF_KQ = 0;          // [128 rows][128] fp16: rows 0-63 KG (later W'), 64-127 QG; 2 panels of 16 KB
-constexpr uint32_t OFF_KN = 32768;      // [64][128] fp16: KN, then K~; 2 panels of 8 KB
-constexpr uint32_t OFF_VV = 49152;      // [64][128] fp16: V, then U~ (then Q^_2); 2 panels of 8 KB
+constexpr uint32_t OFF_KQ = 0;          // [128 rows][128] fp16: rows 0-63 KG (later W'), 64-127 QG; later M_2
+constexpr uint32_t OFF_KN = 32768;      // [64][128] fp16: KN, then K~
+constexpr uint32_t OFF_VV = 49152;      // [64][128] fp16: V, then U~, then Q^_2
 constexpr uint32_t OFF_TT = 65536;      // [64][64] fp16: T
 constexpr uint32_t OFF_PP = 73728;      // [64][64] fp16: P
-constexpr uint32_t OFF_M1 = 81920;      // [128][128] fp16: M_1; 2 panels of 16 KB
-constexpr uint32_t OFF_B1 = 114688;     // [128][128] fp16: B_1; 2 panels of 16 KB
+constexpr uint32_t OFF_M1 = 81920;      // [128][128] fp16: M_1 (MN-major operand image)
+constexpr uint32_t OFF_B1 = 114688;     // [128][128] fp16: B_1 (MN-major operand image)
 constexpr uint32_t OFF_AS = 147456;     // fp32 [64][65]: A (strictly lower, beta applied)
 constexpr uint32_t OFF_XS = 164096;     // fp32 [64][65]: (I + A)^{-1}
-constexpr uint32_t OFF_YS = 180736;     // fp32 [32][33]: merge scratch
-constexpr uint32_t OFF_MISC = 184960;   // beta[64], egm[128], egl[128], ekt[128], gm[128], tot[128], bars, tmem
+constexpr uint32_t OFF_YS = 180736;     // fp32 [32][33]: merge scratch / quarter totals
+constexpr uint32_t OFF_MISC = 184960;   // beta[64], egm, egl, ekt, gm, tot [128 each], barrier, tmem slot, flag
 constexpr uint32_t PREP_SMEM = OFF_MISC + 4096 + 1024;   // + alignment slack
 
 constexpr int LDX = 65;
@@ -129,7 +141,7 @@ struct PrepArgs {
   const void* q; const void* k; const void* v;
   const float* la; const void* beta;
   uint8_t* ws;            // block records
-  int64_t N; int H; int n_blocks;
+  int64_t N; int H; int BH; int n_blocks; int n_units;
   uint32_t* status;
 };
 
@@ -229,18 +241,8 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a) {
   int* range_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int blk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int sub = warp & 3, chalf = warp >> 2;
   const int64_t tok_stride = (int64_t)a.H * D;
-  const TIn* qb = static_cast<const TIn*>(a.q) + (int64_t)b * a.N * tok_stride + (int64_t)h * D;
-  const TIn* kb = static_cast<const TIn*>(a.k) + (int64_t)b * a.N * tok_stride + (int64_t)h * D;
-  const TIn* vb = static_cast<const TIn*>(a.v) + (int64_t)b * a.N * tok_stride + (int64_t)h * D;
-  const float* lab = a.la + (int64_t)b * a.N * tok_stride + (int64_t)h * D;
-  const __nv_bfloat16* bb = static_cast<const __nv_bfloat16*>(a.beta) + (int64_t)b * a.N * a.H + h;
-  uint8_t* rec = a.ws + (((int64_t)b * a.H + h) * a.n_blocks + blk) * kBlockBytes;
-  uint8_t* gM = rec;
-  float* gB = reinterpret_cast<float*>(rec + kMBytes);
-  uint8_t* gR = rec + kMBytes + kBBytes;
-  float* gO = reinterpret_cast<float*>(rec + kMBytes + kBBytes + kRBytes);
 
   if (*(volatile uint32_t*)a.status == KDA_ERR_TIMEOUT) return;   // an earlier CTA gave up: skip the work
   if (warp == 0) { tmem_alloc(tmem_slot, 512); tmem_relinquish(); }
@@ -252,30 +254,76 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a) {
   uint32_t phase = 0;
   bool alive = true;
 
+  // operand descriptors of the fixed tiles (stepped along K by kstep / mstep)
+  const uint64_t dKQk = kdesc0(smem_u32(KQ)), dKQm = mdesc0(smem_u32(KQ), 16384);
+  const uint64_t dKNk = kdesc0(smem_u32(KN)), dKNm = mdesc0(smem_u32(KN), 8192);
+  const uint64_t dVVk = kdesc0(smem_u32(VV)), dVVm = mdesc0(smem_u32(VV), 8192);
+  const uint64_t dTTk = kdesc0(smem_u32(TT)), dPPk = kdesc0(smem_u32(PP));
+  const uint64_t dM1m = mdesc0(smem_u32(M1), 16384), dB1m = mdesc0(smem_u32(B1), 16384);
   const uint32_t id_ap = idesc_f16(128, 64, false, false);
   const uint32_t id_64x128_kmn = idesc_f16(64, 128, false, true);
   const uint32_t id_128x128_mnmn = idesc_f16(128, 128, true, true);
   const uint32_t id_128x128_kmn = idesc_f16(128, 128, false, true);
 
-  for (int s = 0; s < 2; ++s) {
-    const int64_t t0 = (int64_t)blk * BLK + s * SUB;
-    const int nv = (int)max((int64_t)0, min((int64_t)SUB, a.N - t0));
-    // ---------------- load + gate factors ----------------
-    // raw k, q, v rows (256 B each) -> staging with 16-byte asynchronous copies
-    // spread over all threads; staging lives in the solve scratch and T/P
-    // tiles, which are dead at this point
-    uint8_t* stg_k = sm + OFF_AS;
-    uint8_t* stg_q = sm + OFF_AS + 16384;
-    uint8_t* stg_v = sm + OFF_TT;
-    for (int e = tid; e < nv * 16; e += 256) {
-      const int r = e >> 4, ch = (e & 15) * 8;     // row, first of 8 channels
-      const int64_t go = (t0 + r) * tok_stride + ch;
-      cp_async16(stg_k + r * 256 + ch * 2, kb + go);
-      cp_async16(stg_q + r * 256 + ch * 2, qb + go);
-      cp_async16(stg_v + r * 256 + ch * 2, vb + go);
-    }
-    cp_async_commit();
-    {
+  for (int unit = blockIdx.x; unit < a.n_units && alive; unit += gridDim.x) {
+    const int blk = unit / a.BH, bh = unit - blk * a.BH;
+    const int b = bh / a.H, h = bh - b * a.H;
+    const TIn* qb = static_cast<const TIn*>(a.q) + (int64_t)b * a.N * tok_stride + (int64_t)h * D;
+    const TIn* kb = static_cast<const TIn*>(a.k) + (int64_t)b * a.N * tok_stride + (int64_t)h * D;
+    const TIn* vb = static_cast<const TIn*>(a.v) + (int64_t)b * a.N * tok_stride + (int64_t)h * D;
+    const float* lab = a.la + (int64_t)b * a.N * tok_stride + (int64_t)h * D;
+    const __nv_bfloat16* bb = static_cast<const __nv_bfloat16*>(a.beta) + (int64_t)b * a.N * a.H + h;
+    uint8_t* rec = a.ws + (((int64_t)b * a.H + h) * a.n_blocks + blk) * kBlockBytes;
+    uint8_t* gM = rec + kMOff;
+    uint8_t* gB = rec + kBOff;
+    uint8_t* gR = rec + kROff;
+    uint8_t* gO = rec + kOOff;
+
+    for (int s = 0; s < 2; ++s) {
+      const int64_t t0 = (int64_t)blk * BLK + s * SUB;
+      const int nv = (int)max((int64_t)0, min((int64_t)SUB, a.N - t0));
+      {
+        // bring the rows of this CTA's next sub-chunk into L2 while this one is processed
+        int64_t nt0 = t0 + SUB, noff = 0;
+        bool have = s == 0;
+        if (s == 1 && unit + (int)gridDim.x < a.n_units) {
+          const int nunit = unit + (int)gridDim.x;
+          const int nblk = nunit / a.BH, nbh = nunit - nblk * a.BH;
+          const int nb_ = nbh / a.H, nh = nbh - nb_ * a.H;
+          nt0 = (int64_t)nblk * BLK;
+          noff = ((int64_t)nb_ - b) * a.N * tok_stride + (int64_t)(nh - h) * D;
+          have = true;
+        }
+        const int r = tid & 63, which = tid >> 6;
+        if (have && nt0 + r < a.N) {
+          const int64_t go = (nt0 + r) * tok_stride + noff;
+          if (which == 0) prefetch_l2(kb + go, D * sizeof(TIn));
+          else if (which == 1) prefetch_l2(qb + go, D * sizeof(TIn));
+          else if (which == 2) prefetch_l2(vb + go, D * sizeof(TIn));
+          else prefetch_l2(lab + go, D * sizeof(float));
+        }
+      }
+      // ---------------- inputs ----------------
+      // raw k, q, v rows copied straight into their swizzled tile slots
+      // (k -> KQ rows 0-63, q -> KQ rows 64-127, v -> VV); padding rows zeroed
+      for (int e = tid; e < SUB * 16; e += 256) {
+        const int r = e >> 4, ch = (e & 15) * 8, pnl = ch >> 6, cc = ch & 63;
+        uint8_t* dk = KQ + pnl * 16384 + swz_off(r, cc);
+        uint8_t* dq = KQ + pnl * 16384 + swz_off(64 + r, cc);
+        uint8_t* dv = VV + pnl * 8192 + swz_off(r, cc);
+        if (r < nv) {
+          const int64_t go = (t0 + r) * tok_stride + ch;
+          cp_async16(dk, kb + go);
+          cp_async16(dq, qb + go);
+          cp_async16(dv, vb + go);
+        } else {
+          const uint4 z = make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4*>(dk) = z;
+          *reinterpret_cast<uint4*>(dq) = z;
+          *reinterpret_cast<uint4*>(dv) = z;
+        }
+      }
+      cp_async_commit();
       // thread: channels 2cp, 2cp+1 and tokens 16*qt .. 16*qt+15 of the sub-chunk
       const int cp = (tid & 31) + 32 * ((tid >> 5) & 1);
       const int qt = tid >> 6;
@@ -288,9 +336,10 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a) {
       }
 #pragma unroll
       for (int t = 1; t < 16; ++t) { gl[t].x += gl[t - 1].x; gl[t].y += gl[t - 1].y; }
-      float2* qtot = reinterpret_cast<float2*>(Ys);      // [4][64] quarter totals (Ys is free here)
+      float2* qtot = reinterpret_cast<float2*>(Ys);      // [4][64] quarter totals
       qtot[qt * 64 + cp] = gl[15];
       if (tid < SUB) beta_s[tid] = tid < nv ? __bfloat162float(bb[(t0 + tid) * a.H]) : 0.f;
+      cp_async_wait_all();
       __syncthreads();
       float2 pre = make_float2(0.f, 0.f), gmv = make_float2(0.f, 0.f), tot = make_float2(0.f, 0.f);
 #pragma unroll
@@ -303,284 +352,258 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a) {
         gm_s[c] = gmv.x; gm_s[c + 1] = gmv.y;       // g_m: decay through token 31
         tot_s[c] = tot.x; tot_s[c + 1] = tot.y;     // decay over tokens 32..63
       }
-      // exponent x = g - g_m; the extremes sit at token 0 and token 63
+      // exponent x = g - g_m; its extremes sit at token 0 and token 63
       if (qt == 0 && (pre.x + gl[0].x - gmv.x > kRange || pre.y + gl[0].y - gmv.y > kRange)) *range_flag = 1;
       if (qt == 3 && (-tot.x > kRange || -tot.y > kRange)) *range_flag = 1;
-      cp_async_wait_all();
-      __syncthreads();
-      const bool got = true;
-      const int pnl = c >> 6, cc = c & 63;
-      uint8_t* kq = KQ + pnl * 16384;
-      uint8_t* kn = KN + pnl * 8192;
-      uint8_t* vv = VV + pnl * 8192;
-#pragma unroll 4
-      for (int t = 0; t < 16; ++t) {
-        const int tok = 16 * qt + t;
-        float2 kv = make_float2(0.f, 0.f), qv = kv, vv2 = kv;
-        if (tok < nv && got) {
-          kv = ld_act2(reinterpret_cast<const TIn*>(stg_k + tok * 256) + c);
-          qv = ld_act2(reinterpret_cast<const TIn*>(stg_q + tok * 256) + c);
-          vv2 = ld_act2(reinterpret_cast<const TIn*>(stg_v + tok * 256) + c);
-        }
-        const float x0 = pre.x + gl[t].x - gmv.x, x1 = pre.y + gl[t].y - gmv.y;
-        const float ep0 = __expf(x0), ep1 = __expf(x1), en0 = __expf(-x0), en1 = __expf(-x1);
-        const uint32_t off = swz_off(tok, cc);
-        st_h2(kq + off, kv.x * ep0, kv.y * ep1);
-        st_h2(kq + swz_off(64 + tok, cc), qv.x * ep0, qv.y * ep1);
-        st_h2(kn + off, kv.x * en0, kv.y * en1);
-        st_h2(vv + off, vv2.x, vv2.y);
-      }
-    }
-    fence_proxy_async();
-    __syncthreads();
-    if (tid < 128) {
-      const float gm = gm_s[tid], tot = tot_s[tid];
-      egm[tid] = __expf(gm);
-      egl[tid] = __expf(gm + tot);
-      ekt[tid] = __expf(tot);
-    }
-    // ---------------- A, P = [KG; QG] KN^T ----------------
-    if (tid == 0 && alive) {
-      fence_after_sync();
-      for (int k16 = 0; k16 < 8; ++k16)
-        mma_ss(tmem_at(tm, 0, C_AP), desc_kmajor(smem_u32(KQ), k16, 16384), desc_kmajor(smem_u32(KN), k16, 8192),
-               id_ap, k16 > 0);
-      mma_commit(bar);
-    }
-    alive = __syncthreads_and(wait_mma(bar, phase, a.status, alive));
-    fence_after_sync();
-    {
-      // A rows (TMEM lanes 0-63) -> As (beta, strict lower); P rows (lanes 64-127) -> PP (lower)
-      const int sub = warp & 3, chalf = warp >> 2;
-      const int row = 32 * sub + lane;
-      for (int cb = 0; cb < 2; ++cb) {
-        const int col0 = 32 * chalf + 16 * cb;
-        float v[16];
-        tmem_ld16(tmem_at(tm, 32 * sub, C_AP + col0), v);
-        tmem_wait_ld();
-        if (sub < 2) {
-          const float bt = beta_s[row];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) As[row * LDX + col0 + j] = (col0 + j < row) ? bt * v[j] : 0.f;
-        } else {
-          const int r = row - 64;
-#pragma unroll
-          for (int j = 0; j < 16; ++j) v[j] = (col0 + j <= r) ? v[j] : 0.f;
-          st_row16_h(PP, r, col0, v);
-        }
-      }
-    }
-    for (int i = tid; i < SUB * LDX; i += 256) Xs[i] = 0.f;
-    fence_before_sync();
-    __syncthreads();
-    unit_lower_inverse64(As, Xs, Ys);
-    // T = X Diag(beta) -> TT (fp16, [r][i])
-    for (int e = tid; e < SUB * 8; e += 256) {
-      const int r = e >> 3, c0 = (e & 7) * 8;
-      float v[16];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) v[j] = Xs[r * LDX + c0 + j] * beta_s[c0 + j];
-      uint32_t w[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        __half2 hh = __floats2half2_rn(v[2 * j], v[2 * j + 1]);
-        w[j] = *reinterpret_cast<uint32_t*>(&hh);
-      }
-      *reinterpret_cast<uint4*>(TT + swz_off(r, c0)) = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-    fence_proxy_async();
-    __syncthreads();
-    // ---------------- W' = T KG, U~ = T V ----------------
-    if (tid == 0 && alive) {
-      fence_after_sync();
-      for (int k16 = 0; k16 < 4; ++k16) {
-        const uint64_t ad = desc_kmajor(smem_u32(TT), k16, 8192);
-        mma_ss(tmem_at(tm, 0, C_W), ad, desc_mnmajor(smem_u32(KQ), k16, 16384), id_64x128_kmn, k16 > 0);
-        mma_ss(tmem_at(tm, 0, C_U), ad, desc_mnmajor(smem_u32(VV), k16, 8192), id_64x128_kmn, k16 > 0);
-      }
-      mma_commit(bar);
-    }
-    // KN -> K~ = KN e^{g_l - g_m} in place (KN is no longer read by the tensor core)
-    for (int e = tid; e < SUB * 16; e += 256) {
-      const int r = e >> 4, ch = (e & 15) * 8;           // row, first of 8 channels
-      uint8_t* pnl = KN + (ch >> 6) * 8192;
-      uint4* p = reinterpret_cast<uint4*>(pnl + swz_off(r, ch & 63));
-      uint4 u = *p;
-      uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        float2 f = __half22float2(*reinterpret_cast<__half2*>(&w[j]));
-        f.x *= ekt[ch + 2 * j];
-        f.y *= ekt[ch + 2 * j + 1];
-        __half2 hh = __floats2half2_rn(f.x, f.y);
-        w[j] = *reinterpret_cast<uint32_t*>(&hh);
-      }
-      *p = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-    fence_proxy_async();
-    alive = __syncthreads_and(wait_mma(bar, phase, a.status, alive));
-    fence_after_sync();
-    // W' -> KQ rows 0-63 (fp16), U~ -> VV (fp16); M=64 accumulator layout
-    {
-      const int sub = warp & 3, chalf = warp >> 2;
-      const int row = 16 * sub + lane;     // valid for lane < 16
-      for (int cb = 0; cb < 4; ++cb) {
-        const int col0 = 64 * chalf + 16 * cb;
-        float w[16], u[16];
-        tmem_ld16(tmem_at(tm, 32 * sub, C_W + col0), w);
-        tmem_ld16(tmem_at(tm, 32 * sub, C_U + col0), u);
-        tmem_wait_ld();
-        if (lane < 16) {
-          st_row16_h(KQ + (col0 >> 6) * 16384, row, col0 & 63, w);
-          st_row16_h(VV + (col0 >> 6) * 8192, row, col0 & 63, u);
-        }
-      }
-    }
-    fence_proxy_async();
-    fence_before_sync();
-    __syncthreads();
-    // ---------------- K~^T W', K~^T U~, P W', P U~ ----------------
-    if (tid == 0 && alive) {
-      fence_after_sync();
-      for (int k16 = 0; k16 < 4; ++k16) {
-        const uint64_t kt = desc_mnmajor(smem_u32(KN), k16, 8192);
-        const uint64_t wd = desc_mnmajor(smem_u32(KQ), k16, 16384);
-        const uint64_t ud = desc_mnmajor(smem_u32(VV), k16, 8192);
-        const uint64_t pd = desc_kmajor(smem_u32(PP), k16, 8192);
-        mma_ss(tmem_at(tm, 0, C_MK), kt, wd, id_128x128_mnmn, k16 > 0);
-        mma_ss(tmem_at(tm, 0, C_BK), kt, ud, id_128x128_mnmn, k16 > 0);
-        mma_ss(tmem_at(tm, 0, C_PW), pd, wd, id_64x128_kmn, k16 > 0);
-        mma_ss(tmem_at(tm, 0, C_PU), pd, ud, id_64x128_kmn, k16 > 0);
-      }
-      mma_commit(bar);
-    }
-    alive = __syncthreads_and(wait_mma(bar, phase, a.status, alive));
-    fence_after_sync();
-    const int sub = warp & 3, chalf = warp >> 2;
-    if (s == 0) {
-      // M_1 = Diag(e^{g_l}) - MK Diag(e^{g_m}) -> M1 tile;  B_1 -> B1 tile
-      const int row = 32 * sub + lane;
-      for (int cb = 0; cb < 4; ++cb) {
-        const int col0 = 64 * chalf + 16 * cb;
-        float m[16], bv[16];
-        tmem_ld16(tmem_at(tm, 32 * sub, C_MK + col0), m);
-        tmem_ld16(tmem_at(tm, 32 * sub, C_BK + col0), bv);
-        tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < 16; ++j) m[j] = (row == col0 + j ? egl[row] : 0.f) - m[j] * egm[col0 + j];
-        st_row16_h(M1 + (col0 >> 6) * 16384, row, col0 & 63, m);
-        st_row16_h(B1 + (col0 >> 6) * 16384, row, col0 & 63, bv);
-      }
-      // R_1 = (QG - P W') Diag(e^{g_m}) -> global R rows 0-63;  O'_1 -> global O'' rows 0-63
-      const int r = 16 * sub + lane;
-      for (int cb = 0; cb < 4; ++cb) {
-        const int col0 = 64 * chalf + 16 * cb;
-        float pw[16], pu[16];
-        tmem_ld16(tmem_at(tm, 32 * sub, C_PW + col0), pw);
-        tmem_ld16(tmem_at(tm, 32 * sub, C_PU + col0), pu);
-        tmem_wait_ld();
-        if (lane < 16) {
-          float qg[16];
-          ld_row16_h(KQ + (col0 >> 6) * 16384, 64 + r, col0 & 63, qg);
-#pragma unroll
-          for (int j = 0; j < 16; ++j) qg[j] = (qg[j] - pw[j]) * egm[col0 + j];
-          st_row16_h(gR + (col0 >> 6) * 16384, r, col0 & 63, qg);
-          float4* o4 = reinterpret_cast<float4*>(gO);
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            o4[((col0 >> 2) + j) * 128 + r] = make_float4(pu[4 * j], pu[4 * j + 1], pu[4 * j + 2], pu[4 * j + 3]);
-        }
-      }
-      fence_proxy_async();
-      fence_before_sync();
-      __syncthreads();
-    } else {
-      // Q^_2 = (QG - P W') Diag(e^{g_m}) -> VV region (U~ no longer needed)
       {
-        const int r = 16 * sub + lane;
-        for (int cb = 0; cb < 4; ++cb) {
-          const int col0 = 64 * chalf + 16 * cb;
-          float pw[16];
-          tmem_ld16(tmem_at(tm, 32 * sub, C_PW + col0), pw);
-          tmem_wait_ld();
-          if (lane < 16) {
-            float qg[16];
-            ld_row16_h(KQ + (col0 >> 6) * 16384, 64 + r, col0 & 63, qg);
+        const int pnl = c >> 6, cc = c & 63;
+        uint8_t* kq = KQ + pnl * 16384;
+        uint8_t* kn = KN + pnl * 8192;
+        uint8_t* vv = VV + pnl * 8192;
 #pragma unroll
-            for (int j = 0; j < 16; ++j) qg[j] = (qg[j] - pw[j]) * egm[col0 + j];
-            st_row16_h(VV + (col0 >> 6) * 8192, r, col0 & 63, qg);
+        for (int t = 0; t < 16; ++t) {
+          const int tok = 16 * qt + t;
+          const uint32_t off = swz_off(tok, cc), offq = swz_off(64 + tok, cc);
+          const float2 kv = ld_act2(kq + off, (TIn*)nullptr);
+          const float2 qv = ld_act2(kq + offq, (TIn*)nullptr);
+          const float x0 = pre.x + gl[t].x - gmv.x, x1 = pre.y + gl[t].y - gmv.y;
+          const float ep0 = __expf(x0), ep1 = __expf(x1), en0 = __expf(-x0), en1 = __expf(-x1);
+          st_h2(kq + off, kv.x * ep0, kv.y * ep1);
+          st_h2(kq + offq, qv.x * ep0, qv.y * ep1);
+          st_h2(kn + off, kv.x * en0, kv.y * en1);
+          if constexpr (!kIsHalf<TIn>) {
+            const float2 vv2 = ld_act2(vv + off, (TIn*)nullptr);
+            st_h2(vv + off, vv2.x, vv2.y);
           }
         }
       }
-      __syncthreads();
-      // M_2 -> KQ region (A operand, K-major, 2 panels of 16 KB)
-      {
-        const int row = 32 * sub + lane;
-        for (int cb = 0; cb < 4; ++cb) {
-          const int col0 = 64 * chalf + 16 * cb;
-          float m[16];
-          tmem_ld16(tmem_at(tm, 32 * sub, C_MK + col0), m);
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 16; ++j) m[j] = (row == col0 + j ? egl[row] : 0.f) - m[j] * egm[col0 + j];
-          st_row16_h(KQ + (col0 >> 6) * 16384, row, col0 & 63, m);
-        }
-      }
       fence_proxy_async();
-      fence_before_sync();
       __syncthreads();
-      // ---------------- combine ----------------
+      if (tid < 128) {
+        const float gmx = gm_s[tid], totx = tot_s[tid];
+        egm[tid] = __expf(gmx);
+        egl[tid] = __expf(gmx + totx);
+        ekt[tid] = __expf(totx);
+      }
+      // ---------------- A, P = [KG; QG] KN^T ----------------
       if (tid == 0 && alive) {
         fence_after_sync();
-        const uint32_t id_q = idesc_f16(64, 128, false, true);
-        for (int k16 = 0; k16 < 8; ++k16) {
-          const uint64_t m2 = desc_kmajor(smem_u32(KQ), k16, 16384);
-          const uint64_t q2 = desc_kmajor(smem_u32(VV), k16, 8192);
-          const uint64_t m1 = desc_mnmajor(smem_u32(M1), k16, 16384);
-          const uint64_t b1 = desc_mnmajor(smem_u32(B1), k16, 16384);
-          mma_ss(tmem_at(tm, 0, C_MK), m2, m1, id_128x128_kmn, k16 > 0);   // M = M_2 M_1
-          mma_ss(tmem_at(tm, 0, C_BK), m2, b1, id_128x128_kmn, 1);         // B = B_2 + M_2 B_1
-          mma_ss(tmem_at(tm, 0, C_PW), q2, m1, id_q, k16 > 0);             // R_2 = Q^_2 M_1
-          mma_ss(tmem_at(tm, 0, C_PU), q2, b1, id_q, 1);                   // O''_2 = O'_2 + Q^_2 B_1
-        }
+#pragma unroll
+        for (int k16 = 0; k16 < 8; ++k16)
+          mma_ss(tmem_at(tm, 0, C_AP), dKQk + kstep(k16, 16384), dKNk + kstep(k16, 8192), id_ap, k16 > 0);
         mma_commit(bar);
       }
       alive = __syncthreads_and(wait_mma(bar, phase, a.status, alive));
       fence_after_sync();
       {
+        // A rows (TMEM lanes 0-63) -> As (beta, strict lower); P rows (lanes 64-127) -> PP (lower)
         const int row = 32 * sub + lane;
-        for (int cb = 0; cb < 4; ++cb) {
-          const int col0 = 64 * chalf + 16 * cb;
-          float m[16], bv[16];
-          tmem_ld16(tmem_at(tm, 32 * sub, C_MK + col0), m);
-          tmem_ld16(tmem_at(tm, 32 * sub, C_BK + col0), bv);
-          tmem_wait_ld();
-          st_row16_h(gM + (col0 >> 6) * 16384, row, col0 & 63, m);
-          // B in [half][c/4][a][4] layout (half = col / 64)
-          const int hv = col0 >> 6;
+        const int col0 = 32 * chalf;
+        float v[32];
+        tmem_ld32(tmem_at(tm, 32 * sub, C_AP + col0), v);
+        tmem_wait_ld();
+        if (sub < 2) {
+          const float bt = beta_s[row];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int cq = ((col0 & 63) >> 2) + j;
-            reinterpret_cast<float4*>(gB)[((hv * 16 + cq) * 128) + row] =
-                make_float4(bv[4 * j], bv[4 * j + 1], bv[4 * j + 2], bv[4 * j + 3]);
-          }
+          for (int j = 0; j < 32; ++j) As[row * LDX + col0 + j] = (col0 + j < row) ? bt * v[j] : 0.f;
+        } else {
+          const int r = row - 64;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = (col0 + j <= r) ? v[j] : 0.f;
+          st_row32_h(PP, r, col0, v, (r >> 3) & 3);
         }
+      }
+      for (int i = tid; i < SUB * LDX; i += 256) Xs[i] = 0.f;
+      fence_before_sync();
+      __syncthreads();
+      unit_lower_inverse64(As, Xs, Ys);
+      // T = X Diag(beta) -> TT (fp16, [r][i])
+      for (int e = tid; e < SUB * 8; e += 256) {
+        const int r = e >> 3, c0 = (e & 7) * 8;
+        float v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = Xs[r * LDX + c0 + j] * beta_s[c0 + j];
+        *reinterpret_cast<uint4*>(TT + swz_off(r, c0)) = pack8(v);
+      }
+      fence_proxy_async();
+      __syncthreads();
+      // ---------------- W' = T KG, U~ = T V ----------------
+      if (tid == 0 && alive) {
+        fence_after_sync();
+#pragma unroll
+        for (int k16 = 0; k16 < 4; ++k16) {
+          const uint64_t ad = dTTk + kstep(k16, 8192);
+          mma_ss(tmem_at(tm, 0, C_W), ad, dKQm + mstep(k16), id_64x128_kmn, k16 > 0);
+          mma_ss(tmem_at(tm, 0, C_U), ad, dVVm + mstep(k16), id_64x128_kmn, k16 > 0);
+        }
+        mma_commit(bar);
+      }
+      // KN -> K~ = KN e^{g_l - g_m} in place (KN is no longer read by the tensor core)
+      for (int e = tid; e < SUB * 16; e += 256) {
+        const int r = e >> 4, ch = (e & 15) * 8;
+        uint4* p = reinterpret_cast<uint4*>(KN + (ch >> 6) * 8192 + swz_off(r, ch & 63));
+        float f[8];
+        unpack8(*p, f);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) f[j] *= ekt[ch + j];
+        *p = pack8(f);
+      }
+      fence_proxy_async();
+      alive = __syncthreads_and(wait_mma(bar, phase, a.status, alive));
+      fence_after_sync();
+      // W' -> KQ rows 0-63, U~ -> VV (fp16); M=64 accumulator layout: rows 16*sub + lane (lane < 16)
+      {
         const int r = 16 * sub + lane;
-        for (int cb = 0; cb < 4; ++cb) {
-          const int col0 = 64 * chalf + 16 * cb;
-          float rr[16], oo[16];
-          tmem_ld16(tmem_at(tm, 32 * sub, C_PW + col0), rr);
-          tmem_ld16(tmem_at(tm, 32 * sub, C_PU + col0), oo);
+        const int rot = 2 * ((lane >> 3) & 1);
+        for (int cb = 0; cb < 2; ++cb) {
+          const int col0 = 64 * chalf + 32 * cb;
+          float w[32], u[32];
+          tmem_ld32(tmem_at(tm, 32 * sub, C_W + col0), w);
+          tmem_ld32(tmem_at(tm, 32 * sub, C_U + col0), u);
           tmem_wait_ld();
           if (lane < 16) {
-            st_row16_h(gR + (col0 >> 6) * 16384, 64 + r, col0 & 63, rr);
-            float4* o4 = reinterpret_cast<float4*>(gO);
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              o4[((col0 >> 2) + j) * 128 + 64 + r] =
-                  make_float4(oo[4 * j], oo[4 * j + 1], oo[4 * j + 2], oo[4 * j + 3]);
+            st_row32_h(KQ + chalf * 16384, r, col0 & 63, w, rot);
+            st_row32_h(VV + chalf * 8192, r, col0 & 63, u, rot);
           }
         }
+      }
+      fence_proxy_async();
+      fence_before_sync();
+      __syncthreads();
+      // ---------------- K~^T W', K~^T U~, P W', P U~ ----------------
+      if (tid == 0 && alive) {
+        fence_after_sync();
+#pragma unroll
+        for (int k16 = 0; k16 < 4; ++k16) {
+          const uint64_t kt = dKNm + mstep(k16);
+          const uint64_t wd = dKQm + mstep(k16);
+          const uint64_t ud = dVVm + mstep(k16);
+          const uint64_t pd = dPPk + kstep(k16, 8192);
+          mma_ss(tmem_at(tm, 0, C_MK), kt, wd, id_128x128_mnmn, k16 > 0);
+          mma_ss(tmem_at(tm, 0, C_BK), kt, ud, id_128x128_mnmn, k16 > 0);
+          mma_ss(tmem_at(tm, 0, C_PW), pd, wd, id_64x128_kmn, k16 > 0);
+          mma_ss(tmem_at(tm, 0, C_PU), pd, ud, id_64x128_kmn, k16 > 0);
+        }
+        mma_commit(bar);
+      }
+      alive = __syncthreads_and(wait_mma(bar, phase, a.status, alive));
+      fence_after_sync();
+      const int row = 32 * sub + lane;        // M=128 layout row
+      const int rot128 = (row >> 3) & 3;
+      const int r64 = 16 * sub + lane;        // M=64 layout row (lane < 16)
+      const int rot64 = 2 * ((lane >> 3) & 1);
+      if (s == 0) {
+        // M_1 = Diag(e^{g_l}) - MK Diag(e^{g_m}) -> M1 tile;  B_1 -> B1 tile
+        for (int cb = 0; cb < 2; ++cb) {
+          const int col0 = 64 * chalf + 32 * cb;
+          float m[32], bv[32];
+          tmem_ld32(tmem_at(tm, 32 * sub, C_MK + col0), m);
+          tmem_ld32(tmem_at(tm, 32 * sub, C_BK + col0), bv);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) m[j] = (row == col0 + j ? egl[row] : 0.f) - m[j] * egm[col0 + j];
+          st_row32_h(M1 + chalf * 16384, row, col0 & 63, m, rot128);
+          st_row32_h(B1 + chalf * 16384, row, col0 & 63, bv, rot128);
+        }
+        // R_1 = (QG - P W') Diag(e^{g_m}) -> record R rows 0-63;  O'_1 -> record O'' rows 0-63
+        for (int cb = 0; cb < 2; ++cb) {
+          const int col0 = 64 * chalf + 32 * cb;
+          float pw[32], pu[32];
+          tmem_ld32(tmem_at(tm, 32 * sub, C_PW + col0), pw);
+          tmem_ld32(tmem_at(tm, 32 * sub, C_PU + col0), pu);
+          tmem_wait_ld();
+          if (lane < 16) {
+            float qg[32];
+            ld_row16_h(KQ + chalf * 16384, 64 + r64, col0 & 63, qg);
+            ld_row16_h(KQ + chalf * 16384, 64 + r64, (col0 & 63) + 16, qg + 16);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) qg[j] = (qg[j] - pw[j]) * egm[col0 + j];
+            st_row32_h(gR + chalf * 16384, r64, col0 & 63, qg, rot64);
+            uint4* o16 = reinterpret_cast<uint4*>(gO);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) o16[((col0 >> 3) + i) * 128 + r64] = pack8(pu + 8 * i);
+          }
+        }
+        fence_proxy_async();
+        fence_before_sync();
+        __syncthreads();
+      } else {
+        // Q^_2 = (QG - P W') Diag(e^{g_m}) -> VV region (U~ no longer needed)
+        for (int cb = 0; cb < 2; ++cb) {
+          const int col0 = 64 * chalf + 32 * cb;
+          float pw[32];
+          tmem_ld32(tmem_at(tm, 32 * sub, C_PW + col0), pw);
+          tmem_wait_ld();
+          if (lane < 16) {
+            float qg[32];
+            ld_row16_h(KQ + chalf * 16384, 64 + r64, col0 & 63, qg);
+            ld_row16_h(KQ + chalf * 16384, 64 + r64, (col0 & 63) + 16, qg + 16);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) qg[j] = (qg[j] - pw[j]) * egm[col0 + j];
+            st_row32_h(VV + chalf * 8192, r64, col0 & 63, qg, rot64);
+          }
+        }
+        __syncthreads();
+        // M_2 -> KQ region (A operand, K-major, 2 panels of 16 KB)
+        for (int cb = 0; cb < 2; ++cb) {
+          const int col0 = 64 * chalf + 32 * cb;
+          float m[32];
+          tmem_ld32(tmem_at(tm, 32 * sub, C_MK + col0), m);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) m[j] = (row == col0 + j ? egl[row] : 0.f) - m[j] * egm[col0 + j];
+          st_row32_h(KQ + chalf * 16384, row, col0 & 63, m, rot128);
+        }
+        fence_proxy_async();
+        fence_before_sync();
+        __syncthreads();
+        // ---------------- combine ----------------
+        if (tid == 0 && alive) {
+          fence_after_sync();
+          const uint32_t id_q = idesc_f16(64, 128, false, true);
+#pragma unroll
+          for (int k16 = 0; k16 < 8; ++k16) {
+            const uint64_t m2 = dKQk + kstep(k16, 16384);
+            const uint64_t q2 = dVVk + kstep(k16, 8192);
+            const uint64_t m1 = dM1m + mstep(k16);
+            const uint64_t b1 = dB1m + mstep(k16);
+            mma_ss(tmem_at(tm, 0, C_MK), m2, m1, id_128x128_kmn, k16 > 0);   // M = M_2 M_1
+            mma_ss(tmem_at(tm, 0, C_BK), m2, b1, id_128x128_kmn, 1);         // B = B_2 + M_2 B_1
+            mma_ss(tmem_at(tm, 0, C_PW), q2, m1, id_q, k16 > 0);             // R_2 = Q^_2 M_1
+            mma_ss(tmem_at(tm, 0, C_PU), q2, b1, id_q, 1);                   // O''_2 = O'_2 + Q^_2 B_1
+          }
+          mma_commit(bar);
+        }
+        alive = __syncthreads_and(wait_mma(bar, phase, a.status, alive));
+        fence_after_sync();
+        for (int cb = 0; cb < 2; ++cb) {
+          const int col0 = 64 * chalf + 32 * cb;
+          float m[32], bv[32];
+          tmem_ld32(tmem_at(tm, 32 * sub, C_MK + col0), m);
+          tmem_ld32(tmem_at(tm, 32 * sub, C_BK + col0), bv);
+          tmem_wait_ld();
+          st_row32_h(gM + chalf * 16384, row, col0 & 63, m, rot128);
+          // B: [half][c/8][row][8], half = chalf
+          uint4* b16 = reinterpret_cast<uint4*>(gB);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) b16[(chalf * 8 + ((col0 & 63) >> 3) + i) * 128 + row] = pack8(bv + 8 * i);
+        }
+        for (int cb = 0; cb < 2; ++cb) {
+          const int col0 = 64 * chalf + 32 * cb;
+          float rr[32], oo[32];
+          tmem_ld32(tmem_at(tm, 32 * sub, C_PW + col0), rr);
+          tmem_ld32(tmem_at(tm, 32 * sub, C_PU + col0), oo);
+          tmem_wait_ld();
+          if (lane < 16) {
+            st_row32_h(gR + chalf * 16384, 64 + r64, col0 & 63, rr, rot64);
+            uint4* o16 = reinterpret_cast<uint4*>(gO);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) o16[((col0 >> 3) + i) * 128 + 64 + r64] = pack8(oo + 8 * i);
+          }
+        }
+        fence_before_sync();
+        __syncthreads();   // TMEM and shared tiles free for the next unit
+        fence_after_sync();
       }
     }
   }
@@ -592,241 +615,261 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// kda_tc_chain: S <- M S + B over all blocks, per (b, h, half of value columns)
+// kda_tc_chain: per (batch item, head, half of the value columns) the serial
+// pass S <- M S + B over the blocks, fused with the block outputs O = R S + O''.
+//   warps 0-3, the state group: thread t owns row t of S (fp32, in registers);
+//     thread 0 loads M, B and issues M S.
+//   warps 4-7, the output group: thread 128 + t owns token row t of the block;
+//     thread 128 loads R, O'' and issues R S, off the serial path.
+// Both products read the fp16 image of S_j; two images alternate so the next
+// state is written while R S_j may still be reading the current one.
 // ---------------------------------------------------------------------------
-constexpr int CH_STAGES = 3;
-constexpr uint32_t CH_OFF_S = 0;                         // S fp16 [128][64] MN-major panel (16 KB)
-constexpr uint32_t CH_OFF_RING = 16384;                  // stages of {M 32 KB, B-half 32 KB}
-constexpr uint32_t CH_STAGE_BYTES = 65536;
-constexpr uint32_t CH_OFF_BAR = CH_OFF_RING + CH_STAGES * CH_STAGE_BYTES;
+constexpr uint32_t CH_SLOT = 49152;                  // 32 KB operand image + 16 KB fp16 half-width tile
+constexpr uint32_t CH_OFF_A = 0;                     // ring A: M_j, B_j   (2 slots)
+constexpr uint32_t CH_OFF_B = 2 * CH_SLOT;           // ring B: R_j, O''_j (2 slots)
+constexpr uint32_t CH_OFF_S = 4 * CH_SLOT;           // S_j fp16 MN-major images (2 x 16 KB)
+constexpr uint32_t CH_OFF_BAR = CH_OFF_S + 32768;
 constexpr uint32_t CHAIN_SMEM = CH_OFF_BAR + 256 + 1024;
 
 struct ChainArgs {
-  uint8_t* ws;
+  const uint8_t* ws;
   const float* S0;
   float* SN;
-  int H; int n_blocks;
+  __nv_bfloat16* o;
+  int64_t N; int H; int n_blocks;
   uint32_t* status;
 };
 
-__global__ void __launch_bounds__(128, 1) kda_tc_chain(ChainArgs a) {
-  extern __shared__ uint8_t dyn[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn) + 1023) & ~uintptr_t(1023));
-  uint8_t* Ssm = sm + CH_OFF_S;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + CH_OFF_BAR);   // [0..2] loads, [3] mma
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int half = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int64_t rec0 = ((int64_t)b * a.H + h) * a.n_blocks;
-
-  if (warp == 0) { tmem_alloc(tmem_slot, 64); tmem_relinquish(); }
-  if (tid == 0) {
-    for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
-    fence_mbar_init();
+// Bounded wait that also gives up as soon as another thread of the CTA gave up.
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > 500000000ull) { *abort_flag = 1; return false; }
   }
-  fence_before_sync();
-  __syncthreads();
-  fence_after_sync();
-  const uint32_t tm = *tmem_slot;
-
-  auto issue = [&](int j) {
-    const int st = j % CH_STAGES;
-    uint8_t* dst = sm + CH_OFF_RING + st * CH_STAGE_BYTES;
-    const uint8_t* rec = a.ws + (rec0 + j) * kBlockBytes;
-    mbar_arrive_expect_tx(&bars[st], 65536);
-    bulk_g2s(dst, rec, 32768, &bars[st]);
-    bulk_g2s(dst + 32768, rec + kMBytes + half * 32768, 32768, &bars[st]);
-  };
-  if (tid == 0)
-    for (int j = 0; j < CH_STAGES && j < a.n_blocks; ++j) issue(j);
-
-  // state row a = tid (TMEM lane), columns [64 half, 64 half + 64)
-  const int row = tid;
-  float S[64];
-#pragma unroll
-  for (int c = 0; c < 64; ++c)
-    S[c] = a.S0 ? a.S0[(((int64_t)b * a.H + h) * D + row) * D + 64 * half + c] : 0.f;
-
-  const uint32_t idesc = idesc_f16(128, 64, false, true);
-  auto state_out = [&](int jj) {
-    // S (fp16) -> shared B operand and -> workspace (state entering block jj)
-    uint8_t* gS = a.ws + (rec0 + jj) * kBlockBytes + kMBytes + kBBytes + kRBytes + kOBytes + half * 16384;
-#pragma unroll
-    for (int c0 = 0; c0 < 64; c0 += 16) {
-      float v[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) v[i] = S[c0 + i];
-      st_row16_h(Ssm, row, c0, v);
-      st_row16_h(gS, row, c0, v);
-    }
-    fence_proxy_async();
-  };
-  state_out(0);
-  __syncthreads();
-  uint32_t mphase = 0;
-  bool ok = true;
-  int j = 0;
-  for (; j < a.n_blocks; ++j) {
-    const int st = j % CH_STAGES;
-    uint8_t* stage = sm + CH_OFF_RING + st * CH_STAGE_BYTES;
-    bool issued_ok = true;
-    if (tid == 0) {
-      issued_ok = mbar_wait(&bars[st], (uint32_t)(j / CH_STAGES) & 1u);
-      if (issued_ok) {
-        fence_after_sync();
-        for (int k16 = 0; k16 < 8; ++k16)
-          mma_ss(tmem_at(tm, 0, 0), desc_kmajor(smem_u32(stage), k16, 16384), desc_mnmajor(smem_u32(Ssm), k16, 16384),
-                 idesc, k16 > 0);
-        mma_commit(&bars[3]);
-      }
-    }
-    ok = __syncthreads_and(issued_ok) && ok;
-    if (!ok) break;
-    const bool done = mbar_wait(&bars[3], mphase);
-    mphase ^= 1u;
-    ok = __syncthreads_and(done) && ok;
-    if (!ok) break;
-    fence_after_sync();
-    const float4* Bs = reinterpret_cast<const float4*>(stage + 32768);
-#pragma unroll
-    for (int c0 = 0; c0 < 64; c0 += 32) {
-      float v[32];
-      tmem_ld32(tmem_at(tm, 32 * warp, c0), v);
-      float4 bv[8];
-#pragma unroll
-      for (int q4 = 0; q4 < 8; ++q4) bv[q4] = Bs[((c0 >> 2) + q4) * 128 + row];
-      tmem_wait_ld();
-#pragma unroll
-      for (int q4 = 0; q4 < 8; ++q4) {
-        S[c0 + 4 * q4 + 0] = v[4 * q4 + 0] + bv[q4].x;
-        S[c0 + 4 * q4 + 1] = v[4 * q4 + 1] + bv[q4].y;
-        S[c0 + 4 * q4 + 2] = v[4 * q4 + 2] + bv[q4].z;
-        S[c0 + 4 * q4 + 3] = v[4 * q4 + 3] + bv[q4].w;
-      }
-    }
-    if (j + 1 < a.n_blocks) state_out(j + 1);
-    fence_before_sync();
-    __syncthreads();   // stage j consumed, TMEM read, next S in shared memory
-    if (tid == 0 && j + CH_STAGES < a.n_blocks) issue(j + CH_STAGES);
-  }
-  if (!ok) {
-    if (tid == 0) {
-      set_status(a.status, KDA_ERR_TIMEOUT);
-      // let copies already issued land before the CTA exits
-      const int issued = min(a.n_blocks, j + CH_STAGES);
-      for (int jj = j; jj < issued; ++jj) mbar_wait(&bars[jj % CH_STAGES], (uint32_t)(jj / CH_STAGES) & 1u, 100000000ull);
-    }
-  } else if (a.SN) {
-#pragma unroll
-    for (int c = 0; c < 64; ++c) a.SN[(((int64_t)b * a.H + h) * D + row) * D + 64 * half + c] = S[c];
-  }
-  fence_before_sync();
-  __syncthreads();
-  fence_after_sync();
-  if (warp == 0) tmem_dealloc(tm, 64);
+  return true;
 }
 
-// ---------------------------------------------------------------------------
-// kda_tc_out: O = R S + O''
-// ---------------------------------------------------------------------------
-constexpr uint32_t OUT_SMEM = 65536 + 256 + 1024;
-
-template <typename TOut>
-__global__ void __launch_bounds__(128) kda_tc_out(uint8_t* ws, TOut* o, int64_t N, int H, int n_blocks,
-                                                  uint32_t* status) {
+__global__ void __launch_bounds__(256, 1) kda_tc_chain(ChainArgs a) {
   extern __shared__ uint8_t dyn[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + 65536);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + CH_OFF_BAR);
+  uint64_t* fullA = bars;        // [2] ring A slot landed
+  uint64_t* fullB = bars + 2;    // [2] ring B slot landed
+  uint64_t* msDone = bars + 4;   // M S_j complete
+  uint64_t* oDone = bars + 5;    // [2] R S_j complete (TMEM buffer j&1)
+  uint64_t* sReady = bars + 7;   // [2] S_j image written (128 arrivals)
+  uint64_t* sFree = bars + 9;    // [2] R S_j no longer reads S image j&1
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int tid = threadIdx.x, warp = tid >> 5;
-  const int blk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const uint8_t* rec = ws + (((int64_t)b * H + h) * n_blocks + blk) * kBlockBytes;
-  if (*(volatile uint32_t*)status == KDA_ERR_TIMEOUT) return;   // an earlier CTA gave up: skip the work
-  if (warp == 0) { tmem_alloc(tmem_slot, 128); tmem_relinquish(); }
+  const int half = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int nb = a.n_blocks;
+  const int64_t rec0 = ((int64_t)b * a.H + h) * nb;
+  if (*(volatile uint32_t*)a.status == KDA_ERR_TIMEOUT) return;   // an earlier kernel gave up
+
+  if (warp == 0) { tmem_alloc(tmem_slot, 256); tmem_relinquish(); }
   if (tid == 0) {
-    mbar_init(&bars[0], 1);
-    mbar_init(&bars[1], 1);
+    for (int i = 0; i < 11; ++i) mbar_init(&bars[i], (i == 7 || i == 8) ? 128 : 1);
+    *abort_flag = 0;
     fence_mbar_init();
   }
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
   const uint32_t tm = *tmem_slot;
-  if (tid == 0) {
-    mbar_arrive_expect_tx(&bars[0], 65536);
-    bulk_g2s(sm, rec + kMBytes + kBBytes, 32768, &bars[0]);                               // R
-    bulk_g2s(sm + 32768, rec + kMBytes + kBBytes + kRBytes + kOBytes, 32768, &bars[0]);   // S
-  }
-  bool ok = __syncthreads_and(mbar_wait(&bars[0], 0));
-  if (ok && tid == 0) {
-    fence_after_sync();
-    const uint32_t idesc = idesc_f16(128, 128, false, true);
-    for (int k16 = 0; k16 < 8; ++k16)
-      mma_ss(tm, desc_kmajor(smem_u32(sm), k16, 16384), desc_mnmajor(smem_u32(sm + 32768), k16, 16384), idesc,
-             k16 > 0);
-    mma_commit(&bars[1]);
-  }
-  if (ok) ok = __syncthreads_and(mbar_wait(&bars[1], 0));
-  if (!ok) {
-    if (tid == 0) set_status(status, KDA_ERR_TIMEOUT);
-  } else {
-    fence_after_sync();
-    const int r = tid;  // token row within the block = TMEM lane
-    const int64_t tok = (int64_t)blk * BLK + r;
-    const float4* Oo = reinterpret_cast<const float4*>(rec + kMBytes + kBBytes + kRBytes);
-    TOut* orow = o + ((int64_t)b * N + tok) * H * D + (int64_t)h * D;
-    for (int c0 = 0; c0 < 128; c0 += 32) {
-      float v[32];
-      tmem_ld32(tmem_at(tm, 32 * warp, c0), v);
-      float4 oo[8];
+  const uint32_t idesc = idesc_f16(128, 64, false, true);
+  const uint64_t dS = mdesc0(smem_u32(sm + CH_OFF_S), 16384);
+  const int lane_base = 32 * (warp & 3);
+  bool ok = true;
+
+  if (warp < 4) {
+    // ---------------- state group ----------------
+    const int row = tid;
+    auto load_A = [&](int j) {
+      uint8_t* dst = sm + CH_OFF_A + (j & 1) * CH_SLOT;
+      const uint8_t* rec = a.ws + (rec0 + j) * kBlockBytes;
+      mbar_arrive_expect_tx(&fullA[j & 1], CH_SLOT);
+      bulk_g2s(dst, rec + kMOff, 32768, &fullA[j & 1]);
+      bulk_g2s(dst + 32768, rec + kBOff + half * 16384, 16384, &fullA[j & 1]);
+    };
+    int issuedA = 0, seenA = 0, mma_pending = 0;
+    if (tid == 0)
+      for (; issuedA < 2 && issuedA < nb; ++issuedA) load_A(issuedA);
+    float S[64];
 #pragma unroll
-      for (int q4 = 0; q4 < 8; ++q4) oo[q4] = __ldg(Oo + ((c0 >> 2) + q4) * 128 + r);
-      tmem_wait_ld();
-      if (tok < N) {
+    for (int c = 0; c < 64; ++c)
+      S[c] = a.S0 ? a.S0[(((int64_t)b * a.H + h) * D + row) * D + 64 * half + c] : 0.f;
+    auto store_S = [&](int slot) {
+      uint8_t* img = sm + CH_OFF_S + slot * 16384;
 #pragma unroll
-        for (int q4 = 0; q4 < 8; ++q4) {
-          v[4 * q4] += oo[q4].x; v[4 * q4 + 1] += oo[q4].y; v[4 * q4 + 2] += oo[q4].z; v[4 * q4 + 3] += oo[q4].w;
+      for (int i = 0; i < 8; ++i) *reinterpret_cast<uint4*>(img + swz_off(row, 8 * i)) = pack8(S + 8 * i);
+      fence_proxy_async();
+      mbar_arrive(&sReady[slot]);
+    };
+    store_S(0);
+    ok = named_sync_and(1, 128, ok);
+    const uint64_t dA = kdesc0(smem_u32(sm + CH_OFF_A));
+    int j = 0;
+    for (; j < nb && ok; ++j) {
+      if (tid == 0) {
+        const bool landed = wait_or_abort(&fullA[j & 1], (uint32_t)(j >> 1) & 1u, abort_flag);
+        if (landed) {
+          ++seenA;
+          fence_after_sync();
+          const uint64_t da = dA + (uint32_t)(j & 1) * (CH_SLOT >> 4);
+          const uint64_t db = dS + (uint32_t)(j & 1) * (16384u >> 4);
+#pragma unroll
+          for (int k16 = 0; k16 < 8; ++k16) mma_ss(tm, da + kstep(k16, 16384), db + mstep(k16), idesc, k16 > 0);
+          mma_commit(msDone);
+          mma_pending = 1;
         }
-        uint32_t w[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          __nv_bfloat162 hh = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
-          w[j] = *reinterpret_cast<uint32_t*>(&hh);
-        }
-        uint4* dst = reinterpret_cast<uint4*>(orow + c0);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) dst[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
       }
+      bool mine = wait_or_abort(msDone, (uint32_t)j & 1u, abort_flag);
+      if (tid == 0 && mine) mma_pending = 0;
+      mine = mine && wait_or_abort(&fullA[j & 1], (uint32_t)(j >> 1) & 1u, abort_flag);   // B_j visible here too
+      if (mine) {
+        fence_after_sync();
+        const uint4* Bs = reinterpret_cast<const uint4*>(sm + CH_OFF_A + (j & 1) * CH_SLOT + 32768);
+#pragma unroll
+        for (int c0 = 0; c0 < 64; c0 += 32) {
+          float v[32];
+          tmem_ld32(tmem_at(tm, lane_base, c0), v);
+          uint4 bu[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) bu[i] = Bs[((c0 >> 3) + i) * 128 + row];
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            float bf[8];
+            unpack8(bu[i], bf);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) S[c0 + 8 * i + e] = v[8 * i + e] + bf[e];
+          }
+        }
+        if (j + 1 < nb) {
+          // image (j+1)&1 last held S_{j-1}; R S_{j-1} must be done with it
+          if (j >= 1) mine = wait_or_abort(&sFree[(j - 1) & 1], (uint32_t)((j - 1) >> 1) & 1u, abort_flag);
+          if (mine) store_S((j + 1) & 1);
+        }
+      }
+      fence_before_sync();
+      ok = named_sync_and(1, 128, mine);   // ring A slot j consumed, S_{j+1} image written
+      if (ok && tid == 0 && issuedA < nb) { load_A(issuedA); ++issuedA; }
+    }
+    if (ok && a.SN) {
+#pragma unroll
+      for (int c = 0; c < 64; ++c) a.SN[(((int64_t)b * a.H + h) * D + row) * D + 64 * half + c] = S[c];
+    }
+    if (tid == 0) {
+      if (mma_pending) mbar_wait(msDone, (uint32_t)(j - 1) & 1u, 100000000ull);
+      for (int jj = seenA; jj < issuedA; ++jj) mbar_wait(&fullA[jj & 1], (uint32_t)(jj >> 1) & 1u, 100000000ull);
+    }
+  } else {
+    // ---------------- output group ----------------
+    const int r = tid - 128;   // token row of the block = TMEM lane
+    const bool leader = r == 0;
+    auto load_B = [&](int j) {
+      uint8_t* dst = sm + CH_OFF_B + (j & 1) * CH_SLOT;
+      const uint8_t* rec = a.ws + (rec0 + j) * kBlockBytes;
+      mbar_arrive_expect_tx(&fullB[j & 1], CH_SLOT);
+      bulk_g2s(dst, rec + kROff, 32768, &fullB[j & 1]);
+      bulk_g2s(dst + 32768, rec + kOOff + half * 16384, 16384, &fullB[j & 1]);
+    };
+    int issuedB = 0, seenB = 0, o_pending = -1;
+    if (leader)
+      for (; issuedB < 2 && issuedB < nb; ++issuedB) load_B(issuedB);
+    const uint64_t dR = kdesc0(smem_u32(sm + CH_OFF_B));
+    const int64_t tok_stride = (int64_t)a.H * D;
+    __nv_bfloat16* obase = a.o + (int64_t)b * a.N * tok_stride + (int64_t)h * D + 64 * half;
+    for (int j = 0; j < nb && ok; ++j) {
+      if (leader) {
+        bool go = wait_or_abort(&sReady[j & 1], (uint32_t)(j >> 1) & 1u, abort_flag);
+        go = go && wait_or_abort(&fullB[j & 1], (uint32_t)(j >> 1) & 1u, abort_flag);
+        if (go) {
+          ++seenB;
+          fence_after_sync();
+          const uint64_t da = dR + (uint32_t)(j & 1) * (CH_SLOT >> 4);
+          const uint64_t db = dS + (uint32_t)(j & 1) * (16384u >> 4);
+          const uint32_t d = tm + 64 + 64 * (uint32_t)(j & 1);
+#pragma unroll
+          for (int k16 = 0; k16 < 8; ++k16) mma_ss(d, da + kstep(k16, 16384), db + mstep(k16), idesc, k16 > 0);
+          mma_commit(&oDone[j & 1]);
+          mma_commit(&sFree[j & 1]);
+          o_pending = j;
+        }
+      }
+      bool mine = wait_or_abort(&oDone[j & 1], (uint32_t)(j >> 1) & 1u, abort_flag);
+      if (leader && mine) o_pending = -1;
+      mine = mine && wait_or_abort(&fullB[j & 1], (uint32_t)(j >> 1) & 1u, abort_flag);   // O''_j visible here too
+      if (mine) {
+        fence_after_sync();
+        const uint4* Oo = reinterpret_cast<const uint4*>(sm + CH_OFF_B + (j & 1) * CH_SLOT + 32768);
+        const int64_t tok = (int64_t)j * BLK + r;
+        __nv_bfloat16* orow = obase + tok * tok_stride;
+#pragma unroll
+        for (int c0 = 0; c0 < 64; c0 += 32) {
+          float v[32];
+          tmem_ld32(tmem_at(tm, lane_base, 64 + 64 * (j & 1) + c0), v);
+          uint4 ou[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) ou[i] = Oo[((c0 >> 3) + i) * 128 + r];
+          tmem_wait_ld();
+          if (tok < a.N) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              float of[8];
+              unpack8(ou[i], of);
+              uint32_t w[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                __nv_bfloat162 hh = __floats2bfloat162_rn(v[8 * i + 2 * e] + of[2 * e], v[8 * i + 2 * e + 1] + of[2 * e + 1]);
+                w[e] = *reinterpret_cast<uint32_t*>(&hh);
+              }
+              reinterpret_cast<uint4*>(orow + c0)[i] = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+          }
+        }
+      }
+      fence_before_sync();
+      ok = named_sync_and(2, 128, mine);   // TMEM buffer j&1 read, ring B slot j consumed
+      if (ok && leader && issuedB < nb) { load_B(issuedB); ++issuedB; }
+    }
+    if (leader) {
+      if (o_pending >= 0) mbar_wait(&oDone[o_pending & 1], (uint32_t)(o_pending >> 1) & 1u, 100000000ull);
+      for (int jj = seenB; jj < issuedB; ++jj) mbar_wait(&fullB[jj & 1], (uint32_t)(jj >> 1) & 1u, 100000000ull);
     }
   }
+  if (tid == 0 && *abort_flag) set_status(a.status, KDA_ERR_TIMEOUT);
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
-  if (warp == 0) tmem_dealloc(tm, 128);
+  if (warp == 0) tmem_dealloc(tm, 256);
 }
 
-template <typename TIn, typename TOut>
+template <typename TIn>
 cudaError_t launch_all(const Dims& d, const void* q, const void* k, const void* v, const float* la,
                        const void* beta, const float* S0, void* o, float* SN, uint8_t* ws, uint32_t* status,
                        cudaStream_t s, int* launches) {
   const int n_blocks = (int)((d.N + BLK - 1) / BLK);
   cudaError_t e;
+  int dev = 0, n_sm = 148;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
   e = cudaFuncSetAttribute(kda_tc_prep<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize, PREP_SMEM);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(kda_tc_chain, cudaFuncAttributeMaxDynamicSharedMemorySize, CHAIN_SMEM);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(kda_tc_out<TOut>, cudaFuncAttributeMaxDynamicSharedMemorySize, OUT_SMEM);
-  if (e != cudaSuccess) return e;
-  PrepArgs pa{q, k, v, la, beta, ws, d.N, d.H, n_blocks, status};
-  kda_tc_prep<TIn><<<dim3(n_blocks, d.H, d.B), 256, PREP_SMEM, s>>>(pa);
+  const int BH = d.B * d.H;
+  const int n_units = BH * n_blocks;
+  PrepArgs pa{q, k, v, la, beta, ws, d.N, d.H, BH, n_blocks, n_units, status};
+  kda_tc_prep<TIn><<<dim3((unsigned)min(n_units, n_sm)), 256, PREP_SMEM, s>>>(pa);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  ChainArgs ca{ws, S0, SN, d.H, n_blocks, status};
-  kda_tc_chain<<<dim3(2, d.H, d.B), 128, CHAIN_SMEM, s>>>(ca);
+  ChainArgs ca{ws, S0, SN, static_cast<__nv_bfloat16*>(o), d.N, d.H, n_blocks, status};
+  kda_tc_chain<<<dim3(2, d.H, d.B), 256, CHAIN_SMEM, s>>>(ca);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  kda_tc_out<TOut><<<dim3(n_blocks, d.H, d.B), 128, OUT_SMEM, s>>>(ws, static_cast<TOut*>(o), d.N, d.H, n_blocks,
-                                                                   status);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  if (launches) *launches += 3;
+  if (launches) *launches += 2;
   return cudaSuccess;
 }
 
@@ -844,10 +887,10 @@ cudaError_t launch_chunk_tc(const Dims& d, bool in_f16, const void* q, const voi
                             void* ws, uint32_t* status, cudaStream_t s, int* launches) {
   // beta and o are bf16 (the problem dtype); q', k', v' are fp16 (internal conv output) or bf16 (caller)
   if (in_f16)
-    return launch_all<__half, __nv_bfloat16>(d, q, k, v, log_alpha, beta, S0, o, SN, static_cast<uint8_t*>(ws),
-                                             status, s, launches);
-  return launch_all<__nv_bfloat16, __nv_bfloat16>(d, q, k, v, log_alpha, beta, S0, o, SN,
-                                                  static_cast<uint8_t*>(ws), status, s, launches);
+    return launch_all<__half>(d, q, k, v, log_alpha, beta, S0, o, SN, static_cast<uint8_t*>(ws), status, s,
+                              launches);
+  return launch_all<__nv_bfloat16>(d, q, k, v, log_alpha, beta, S0, o, SN, static_cast<uint8_t*>(ws), status, s,
+                                   launches);
 }
 
 }  // namespace kda

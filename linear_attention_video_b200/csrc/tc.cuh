@@ -54,6 +54,15 @@ __device__ __forceinline__ uint64_t desc_mnmajor(uint32_t base, int k16, uint32_
   return sdesc(base + (uint32_t)k16 * 2048u, panel_bytes, 1024u);
 }
 
+// The same descriptors built once per tile and stepped along K by adding to the
+// start-address field (address >> 4; the sum stays inside shared memory).
+__device__ __forceinline__ uint64_t kdesc0(uint32_t base) { return sdesc(base, 16u, 1024u); }
+__device__ __forceinline__ uint64_t mdesc0(uint32_t base, uint32_t panel_bytes) { return sdesc(base, panel_bytes, 1024u); }
+__host__ __device__ constexpr uint32_t kstep(int k16, uint32_t panel_bytes) {
+  return ((uint32_t)(k16 >> 2) * panel_bytes + (uint32_t)(k16 & 3) * 32u) >> 4;
+}
+__host__ __device__ constexpr uint32_t mstep(int k16) { return (uint32_t)k16 * 128u; }
+
 // Instruction descriptor: kind::f16, fp16 x fp16 -> fp32 (A and B of one MMA share a type).
 __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool a_mn, bool b_mn, bool neg_a = false) {
   return (1u << 4)                       // D format f32
@@ -199,6 +208,40 @@ __device__ __forceinline__ void bulk_g2s(void* dst_smem, const void* src_gmem, u
   asm volatile(
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
       :: "r"(smem_u32(dst_smem)), "l"(src_gmem), "r"(bytes), "r"(smem_u32(bar)) : "memory");
+}
+
+// Bulk copy shared -> global, completion tracked per thread with bulk groups.
+__device__ __forceinline__ void bulk_s2g(void* dst_gmem, const void* src_smem, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+               :: "l"(dst_gmem), "r"(smem_u32(src_smem)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Source shared memory of every committed bulk store may be overwritten.
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// Every committed bulk store is complete (visible in global memory).
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// Hint: bring a global range (16-byte aligned, multiple of 16 bytes) into L2.
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" :: "l"(p), "r"(bytes) : "memory");
+}
+
+// Plain arrive (count 1) on an mbarrier.
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(smem_u32(bar)) : "memory");
+}
+
+// Barrier over `count` threads (a multiple of 32) on hardware barrier `id`
+// (1..15; 0 is __syncthreads); returns the AND of `pred` over those threads.
+__device__ __forceinline__ bool named_sync_and(uint32_t id, uint32_t count, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}\n"
+      : "=r"(r) : "r"((uint32_t)pred), "r"(id), "r"(count) : "memory");
+  return r != 0;
 }
 
 // 16-byte asynchronous global -> shared copy (LSU path), grouped by commit/wait.

@@ -31,7 +31,7 @@ def _inputs(B, N, H, d, seed):
 def test_noalloc_matches_chunk_fwd_on_two_calls():
     import linear_attention_video_b200 as kda
     lib = kda._lib
-    B, N, H, d = 1, 1000, 16, 128            # 8 blocks x 16 heads: ~29 MB of scratch
+    B, N, H, d = 1, 1000, 16, 128            # 8 blocks x 16 heads: 16 MiB of scratch
     p = kda.problem(B, H, d, N, (0, 0, 0))
     ref_o = torch.empty(B, N, H, d, dtype=torch.bfloat16, device="cuda")
     ref_s = torch.empty(B, H, d, d, device="cuda")
@@ -58,7 +58,7 @@ def test_noalloc_matches_chunk_fwd_on_two_calls():
 def test_noalloc_rejects_problems_beyond_its_scratch():
     import linear_attention_video_b200 as kda
     lib = kda._lib
-    p = kda.problem(1, 16, 128, 40000, (0, 0, 0))   # 313 blocks x 16 heads: ~1.1 GB of scratch
+    p = kda.problem(1, 16, 128, 40000, (0, 0, 0))   # 313 blocks x 16 heads: ~626 MiB of scratch
     rc = lib.kda_chunk_fwd_noalloc(ctypes.byref(p), kda.KDA_DT_BF16, 256, 256, 256, 256, 256, None, 256, None,
                                    None, None)
     assert rc == kda.KDA_ERR_WORKSPACE
