@@ -254,7 +254,7 @@ def ours_arm(args, w, idx, rank, world, local_rank):
     scan_gbs = scan_bytes / (ms_scan * 1e-3) / 1e9
     conv_gbs = conv_bytes(w) / (ms_conv * 1e-3) / 1e9
     hbm = float(peaks["hbm_gbs"])
-    # the scan entry point (prep + chain + out kernels) is the dominant launch; its algorithmic bytes are
+    # the scan entry point (prep + chain kernels) is the dominant launch; its algorithmic bytes are
     # those of the fused step: q', k', v', log alpha, beta read once and o written once
     dominant = "kda_chunk" if ms_scan >= ms_conv else "shortconv"
     achieved = scan_gbs if dominant == "kda_chunk" else conv_gbs
@@ -266,7 +266,7 @@ def ours_arm(args, w, idx, rank, world, local_rank):
         except (ValueError, OSError):
             traffic = None
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                "traffic": traffic, "kernel": dominant + (" (kda_chunk_fwd: prep + chain + out kernels)"
+                "traffic": traffic, "kernel": dominant + (" (kda_chunk_fwd: prep + chain kernels)"
                                                           if dominant == "kda_chunk" else ""),
                 "peak_source": peaks["source"] + " hbm_gbs"}
     step_roof_ms = max(algorithmic_bytes(w) / (hbm * 1e9), tensor_flops(w) / (float(peaks["bf16_tflops"]) * 1e12)) * 1e3

@@ -46,7 +46,7 @@ constexpr float kRange = 9.f;     // max |g - g_m| allowed for the fp16 factors
 //   M   K-major operand image: 2 panels [128 rows][64 cols]            32 KB
 //   B   [half][c/8][row a][8]  (16-byte units)                         32 KB
 //   R   K-major operand image: 2 panels [128 rows][64 cols]            32 KB
-//   O'' [c/8][row r][8]        (16-byte units)                         32 KB
+//   O'' [row half][c/8][row r % 64][8]  (16-byte units)                32 KB
 constexpr size_t kMOff = 0, kBOff = 32768, kROff = 65536, kOOff = 98304;
 constexpr size_t kBlockBytes = 131072;
 
@@ -145,58 +145,67 @@ struct PrepArgs {
   uint32_t* status;
 };
 
-// Blocked inverse of the unit lower-triangular (I + A), A in As (strictly lower).
+// Blocked inverse X = (I + A)^{-1} of the unit lower-triangular 64x64 matrix,
+// A strictly lower in As.  16x16 diagonal blocks by forward substitution, then
+// two doubling merges (X_21 = -X_22 A_21 X_11) at 32 and 64.  Every loop has a
+// fixed trip count; the zero blocks above the diagonal of X_11 and X_22 are
+// written here, the rest of the upper triangle is never read.
 __device__ void unit_lower_inverse64(const float* As, float* Xs, float* Ys) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // diagonal 16x16 blocks: warp b, lane l = column 16b + l
   if (warp < 4 && lane < 16) {
-    const int b = warp, l = lane, o = 16 * b;
+    // diagonal block `warp`, column `lane`: right-looking substitution
+    const int o = 16 * warp, l = lane;
     float x[16];
 #pragma unroll
-    for (int r = 0; r < 16; ++r) {
-      float acc = 0.f;
+    for (int r = 0; r < 16; ++r) x[r] = r == l ? 1.f : 0.f;
 #pragma unroll
-      for (int m = 0; m < r; ++m) acc += As[(o + r) * LDX + o + m] * x[m];
-      x[r] = r < l ? 0.f : (r == l ? 1.f : -acc);
+    for (int m = 0; m < 15; ++m) {
+#pragma unroll
+      for (int r = m + 1; r < 16; ++r) x[r] -= As[(o + r) * LDX + o + m] * x[m];
     }
 #pragma unroll
     for (int r = 0; r < 16; ++r) Xs[(o + r) * LDX + o + l] = x[r];
+  } else if (warp >= 4) {
+    // zero blocks (0,1) and (2,3)
+    const int e = tid - 128, r = e >> 3, c = 2 * (e & 7);   // 16 rows x 8 column pairs
+    Xs[r * LDX + 16 + c] = 0.f;
+    Xs[r * LDX + 17 + c] = 0.f;
+    Xs[(32 + r) * LDX + 48 + c] = 0.f;
+    Xs[(32 + r) * LDX + 49 + c] = 0.f;
   }
   __syncthreads();
-  // 32x32 merges: for p in {0,1}: X[32p+16.., 32p..] = -X22 (A21 X11); one 2x1 tile per thread
   {
+    // 32-merges p = 0, 1: X[32p+16.., 32p..] = -D_{2p+1} (A_{2p+1,2p} D_{2p}); 2x1 outputs per thread
     const int p = tid >> 7, e = tid & 127;
-    const int o = 32 * p;
+    const int o = 32 * p, i0 = 2 * (e >> 4), j = e & 15;
     float* Y = Ys + p * 16 * 17;
-    const int r0 = 2 * (e >> 4), c = e & 15;
-    {
-      float a0 = 0.f, a1 = 0.f;
-      for (int m = c; m < 16; ++m) {
-        const float x = Xs[(o + m) * LDX + o + c];
-        a0 += As[(o + 16 + r0) * LDX + o + m] * x;
-        a1 += As[(o + 17 + r0) * LDX + o + m] * x;
-      }
-      Y[r0 * 17 + c] = a0;
-      Y[(r0 + 1) * 17 + c] = a1;
+    float y0 = 0.f, y1 = 0.f;
+#pragma unroll
+    for (int m = 0; m < 16; ++m) {
+      const float d = Xs[(o + m) * LDX + o + j];
+      y0 += As[(o + 16 + i0) * LDX + o + m] * d;
+      y1 += As[(o + 17 + i0) * LDX + o + m] * d;
     }
+    Y[i0 * 17 + j] = y0;
+    Y[(i0 + 1) * 17 + j] = y1;
     __syncthreads();
-    {
-      float a0 = 0.f, a1 = 0.f;
-      for (int m = 0; m <= r0 + 1; ++m) {
-        const float y = Y[m * 17 + c];
-        a0 += (m <= r0 ? Xs[(o + 16 + r0) * LDX + o + 16 + m] : 0.f) * y;
-        a1 += Xs[(o + 17 + r0) * LDX + o + 16 + m] * y;
-      }
-      Xs[(o + 16 + r0) * LDX + o + c] = -a0;
-      Xs[(o + 17 + r0) * LDX + o + c] = -a1;
+    float z0 = 0.f, z1 = 0.f;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const float y = Y[k * 17 + j];
+      z0 += Xs[(o + 16 + i0) * LDX + o + 16 + k] * y;
+      z1 += Xs[(o + 17 + i0) * LDX + o + 16 + k] * y;
     }
-    __syncthreads();
+    Xs[(o + 16 + i0) * LDX + o + j] = -z0;
+    Xs[(o + 17 + i0) * LDX + o + j] = -z1;
   }
-  // 64 merge: X[32.., 0..31] = -X22 (A21 X11); one 2x2 tile per thread
+  __syncthreads();
   {
+    // 64-merge: X[32.., 0..31] = -X_22 (A_21 X_11); 2x2 outputs per thread
     const int r0 = 2 * (tid >> 4), c0 = 2 * (tid & 15);
     float a00 = 0.f, a01 = 0.f, a10 = 0.f, a11 = 0.f;
-    for (int m = c0; m < 32; ++m) {
+#pragma unroll
+    for (int m = 0; m < 32; ++m) {
       const float x0 = Xs[m * LDX + c0], x1 = Xs[m * LDX + c0 + 1];
       const float u0 = As[(32 + r0) * LDX + m], u1 = As[(33 + r0) * LDX + m];
       a00 += u0 * x0; a01 += u0 * x1; a10 += u1 * x0; a11 += u1 * x1;
@@ -205,9 +214,10 @@ __device__ void unit_lower_inverse64(const float* As, float* Xs, float* Ys) {
     Ys[(r0 + 1) * 33 + c0] = a10; Ys[(r0 + 1) * 33 + c0 + 1] = a11;
     __syncthreads();
     a00 = a01 = a10 = a11 = 0.f;
-    for (int m = 0; m <= r0 + 1; ++m) {
+#pragma unroll
+    for (int m = 0; m < 32; ++m) {
       const float y0 = Ys[m * 33 + c0], y1 = Ys[m * 33 + c0 + 1];
-      const float u0 = m <= r0 ? Xs[(32 + r0) * LDX + 32 + m] : 0.f, u1 = Xs[(33 + r0) * LDX + 32 + m];
+      const float u0 = Xs[(32 + r0) * LDX + 32 + m], u1 = Xs[(33 + r0) * LDX + 32 + m];
       a00 += u0 * y0; a01 += u0 * y1; a10 += u1 * y0; a11 += u1 * y1;
     }
     Xs[(32 + r0) * LDX + c0] = -a00; Xs[(32 + r0) * LDX + c0 + 1] = -a01;
@@ -393,6 +403,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a) {
           mma_ss(tmem_at(tm, 0, C_AP), dKQk + kstep(k16, 16384), dKNk + kstep(k16, 8192), id_ap, k16 > 0);
         mma_commit(bar);
       }
+      if (tid == 0) bulk_wait_read();   // staged records read: their tiles may be rewritten
       alive = __syncthreads_and(wait_mma(bar, phase, a.status, alive));
       fence_after_sync();
       {
@@ -413,16 +424,15 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a) {
           st_row32_h(PP, r, col0, v, (r >> 3) & 3);
         }
       }
-      for (int i = tid; i < SUB * LDX; i += 256) Xs[i] = 0.f;
       fence_before_sync();
       __syncthreads();
       unit_lower_inverse64(As, Xs, Ys);
-      // T = X Diag(beta) -> TT (fp16, [r][i])
+      // T = X Diag(beta) -> TT (fp16, [r][i]); X is lower triangular
       for (int e = tid; e < SUB * 8; e += 256) {
         const int r = e >> 3, c0 = (e & 7) * 8;
         float v[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) v[j] = Xs[r * LDX + c0 + j] * beta_s[c0 + j];
+        for (int j = 0; j < 8; ++j) v[j] = c0 + j <= r ? Xs[r * LDX + c0 + j] * beta_s[c0 + j] : 0.f;
         *reinterpret_cast<uint4*>(TT + swz_off(r, c0)) = pack8(v);
       }
       fence_proxy_async();
@@ -449,6 +459,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a) {
         *p = pack8(f);
       }
       fence_proxy_async();
+      if (tid == 0) bulk_wait_read();   // staged records read: their tiles may be rewritten
       alive = __syncthreads_and(wait_mma(bar, phase, a.status, alive));
       fence_after_sync();
       // W' -> KQ rows 0-63, U~ -> VV (fp16); M=64 accumulator layout: rows 16*sub + lane (lane < 16)
@@ -486,6 +497,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a) {
         }
         mma_commit(bar);
       }
+      if (tid == 0) bulk_wait_read();   // staged records read: their tiles may be rewritten
       alive = __syncthreads_and(wait_mma(bar, phase, a.status, alive));
       fence_after_sync();
       const int row = 32 * sub + lane;        // M=128 layout row
@@ -505,7 +517,9 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a) {
           st_row32_h(M1 + chalf * 16384, row, col0 & 63, m, rot128);
           st_row32_h(B1 + chalf * 16384, row, col0 & 63, bv, rot128);
         }
-        // R_1 = (QG - P W') Diag(e^{g_m}) -> record R rows 0-63;  O'_1 -> record O'' rows 0-63
+        // R_1 = (QG - P W') Diag(e^{g_m}) and O'_1, staged for the record (R rows 0-63, O'' rows 0-63)
+        uint8_t* stR = reinterpret_cast<uint8_t*>(Xs);   // [panel][64 rows][128 B], swizzled
+        uint4* stO = reinterpret_cast<uint4*>(As);       // [c/8][64 rows][8]
         for (int cb = 0; cb < 2; ++cb) {
           const int col0 = 64 * chalf + 32 * cb;
           float pw[32], pu[32];
@@ -518,15 +532,20 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a) {
             ld_row16_h(KQ + chalf * 16384, 64 + r64, (col0 & 63) + 16, qg + 16);
 #pragma unroll
             for (int j = 0; j < 32; ++j) qg[j] = (qg[j] - pw[j]) * egm[col0 + j];
-            st_row32_h(gR + chalf * 16384, r64, col0 & 63, qg, rot64);
-            uint4* o16 = reinterpret_cast<uint4*>(gO);
+            st_row32_h(stR + chalf * 8192, r64, col0 & 63, qg, rot64);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) o16[((col0 >> 3) + i) * 128 + r64] = pack8(pu + 8 * i);
+            for (int i = 0; i < 4; ++i) stO[((col0 >> 3) + i) * 64 + r64] = pack8(pu + 8 * i);
           }
         }
         fence_proxy_async();
         fence_before_sync();
         __syncthreads();
+        if (tid == 0) {
+          bulk_s2g(gR, stR, 8192);
+          bulk_s2g(gR + 16384, stR + 8192, 8192);
+          bulk_s2g(gO, stO, 16384);
+          bulk_commit();
+        }
       } else {
         // Q^_2 = (QG - P W') Diag(e^{g_m}) -> VV region (U~ no longer needed)
         for (int cb = 0; cb < 2; ++cb) {
@@ -574,19 +593,24 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a) {
           }
           mma_commit(bar);
         }
+        if (tid == 0) bulk_wait_read();   // staged records read: their tiles may be rewritten
         alive = __syncthreads_and(wait_mma(bar, phase, a.status, alive));
         fence_after_sync();
+        // records staged in tiles the combine products no longer read:
+        //   M -> M1 region, B -> B1 region, R_2 -> TT/PP region, O''_2 -> Xs region
+        uint8_t* stR = TT;                               // [panel][64 rows][128 B], swizzled
+        uint4* stO = reinterpret_cast<uint4*>(Xs);       // [c/8][64 rows][8]
         for (int cb = 0; cb < 2; ++cb) {
           const int col0 = 64 * chalf + 32 * cb;
           float m[32], bv[32];
           tmem_ld32(tmem_at(tm, 32 * sub, C_MK + col0), m);
           tmem_ld32(tmem_at(tm, 32 * sub, C_BK + col0), bv);
           tmem_wait_ld();
-          st_row32_h(gM + chalf * 16384, row, col0 & 63, m, rot128);
-          // B: [half][c/8][row][8], half = chalf
-          uint4* b16 = reinterpret_cast<uint4*>(gB);
+          st_row32_h(M1 + chalf * 16384, row, col0 & 63, m, rot128);
+          // B: [c/8][row][8]
+          uint4* b16 = reinterpret_cast<uint4*>(B1);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) b16[(chalf * 8 + ((col0 & 63) >> 3) + i) * 128 + row] = pack8(bv + 8 * i);
+          for (int i = 0; i < 4; ++i) b16[((col0 >> 3) + i) * 128 + row] = pack8(bv + 8 * i);
         }
         for (int cb = 0; cb < 2; ++cb) {
           const int col0 = 64 * chalf + 32 * cb;
@@ -595,11 +619,21 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a) {
           tmem_ld32(tmem_at(tm, 32 * sub, C_PU + col0), oo);
           tmem_wait_ld();
           if (lane < 16) {
-            st_row32_h(gR + chalf * 16384, 64 + r64, col0 & 63, rr, rot64);
-            uint4* o16 = reinterpret_cast<uint4*>(gO);
+            st_row32_h(stR + chalf * 8192, r64, col0 & 63, rr, rot64);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) o16[((col0 >> 3) + i) * 128 + 64 + r64] = pack8(oo + 8 * i);
+            for (int i = 0; i < 4; ++i) stO[((col0 >> 3) + i) * 64 + r64] = pack8(oo + 8 * i);
           }
+        }
+        fence_proxy_async();
+        fence_before_sync();
+        __syncthreads();
+        if (tid == 0) {
+          bulk_s2g(gM, M1, 32768);
+          bulk_s2g(gB, B1, 32768);
+          bulk_s2g(gR + 8192, stR, 8192);
+          bulk_s2g(gR + 16384 + 8192, stR + 8192, 8192);
+          bulk_s2g(gO + 16384, stO, 16384);
+          bulk_commit();
         }
         fence_before_sync();
         __syncthreads();   // TMEM and shared tiles free for the next unit
@@ -607,6 +641,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a) {
       }
     }
   }
+  if (tid == 0) bulk_wait_all();
   if (tid == 0 && *range_flag) set_status(a.status, KDA_ERR_RANGE);
   fence_before_sync();
   __syncthreads();
@@ -775,7 +810,8 @@ __global__ void __launch_bounds__(256, 1) kda_tc_chain(ChainArgs a) {
       const uint8_t* rec = a.ws + (rec0 + j) * kBlockBytes;
       mbar_arrive_expect_tx(&fullB[j & 1], CH_SLOT);
       bulk_g2s(dst, rec + kROff, 32768, &fullB[j & 1]);
-      bulk_g2s(dst + 32768, rec + kOOff + half * 16384, 16384, &fullB[j & 1]);
+      bulk_g2s(dst + 32768, rec + kOOff + half * 8192, 8192, &fullB[j & 1]);
+      bulk_g2s(dst + 40960, rec + kOOff + 16384 + half * 8192, 8192, &fullB[j & 1]);
     };
     int issuedB = 0, seenB = 0, o_pending = -1;
     if (leader)
@@ -814,7 +850,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_chain(ChainArgs a) {
           tmem_ld32(tmem_at(tm, lane_base, 64 + 64 * (j & 1) + c0), v);
           uint4 ou[4];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) ou[i] = Oo[((c0 >> 3) + i) * 128 + r];
+          for (int i = 0; i < 4; ++i) ou[i] = Oo[((r >> 6) * 8 + (c0 >> 3) + i) * 64 + (r & 63)];
           tmem_wait_ld();
           if (tok < a.N) {
 #pragma unroll

@@ -35,6 +35,8 @@ int make_dims(const kda_problem* p, kda_dtype dt, kda::Dims* d) {
   // keep every element index well inside int64 and grid dims inside CUDA limits
   if (N > (int64_t(1) << 31) || (int64_t)p->B * N * p->H * p->dk > (int64_t(1) << 40))
     return KDA_ERR_UNSUPPORTED;
+  // the 3D conv indexes one frame (grid_h * grid_w tokens x all channels) with 32-bit offsets
+  if ((int64_t)p->grid_h * p->grid_w * p->H * p->dk >= (int64_t(1) << 31)) return KDA_ERR_UNSUPPORTED;
   d->B = p->B; d->H = p->H; d->dk = p->dk; d->dv = p->dv;
   d->N = N; d->L = p->text_len;
   d->T = p->grid_t; d->Hg = p->grid_h; d->Wg = p->grid_w;

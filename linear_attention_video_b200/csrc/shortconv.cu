@@ -6,17 +6,19 @@
 // one rounding to the output type.
 //
 // Visual part (the bulk of the work, bound by the fp32 FMA pipe): a CTA owns
-// 32 channels of one tensor and a tile of up to 4 rows x 64 columns of the
-// grid, and slides through time.  Input planes (the tile plus a one-pixel halo)
-// of three consecutive frames sit in shared memory as fp32, so each input
-// element is read from global memory and converted once; the next plane's
-// global loads are in flight while the current frame is computed.  A thread
-// owns 2 channels (their 54 weights live in registers) and a run of up to 16
-// pixels along a row, so every value it reads from shared memory feeds 3
-// horizontal taps.
+// 32 channels of one tensor (one per lane) and a tile of 4 rows x (4 runs) of
+// the grid, and slides through time.  Input planes (the tile plus a one-pixel
+// halo, zero outside the grid) are copied as they are by cp.async into a ring
+// of four shared-memory slots, three planes ahead of the one being computed.
+// Each plane is read from shared memory once: a thread keeps the partial sums
+// of the three output frames that plane feeds (t = f + pt - a for temporal tap
+// a) in registers, so every value it reads feeds up to 27 taps.  The frame
+// whose last tap arrived is written out and its registers start the frame
+// three ahead.
 //
 // Text part: a small kernel, one thread per (token, 8 channels).
 #include <cuda_fp16.h>
+
 
 #include "common.cuh"
 
@@ -24,14 +26,11 @@ namespace kda {
 namespace {
 
 constexpr int kVisTaps = 27;
-constexpr int CG = 32;            // channels per CTA
-constexpr int TH = 4;             // tile rows
-constexpr int TWMAX = 64;         // tile columns
-constexpr int PH = TH + 2, PW = TWMAX + 2;
-constexpr int PLANE_FLOATS = PH * PW * CG;
-constexpr int RUNMAX = TWMAX / 4;
-constexpr int kThreads = 256;
-constexpr int kPrefetch = (PH * PW * (CG / 8) + kThreads - 1) / kThreads;   // 16-byte chunks per thread
+constexpr int CG = 32;            // channels per CTA, one per lane
+constexpr int TH = 4;             // tile rows, one per warp row
+constexpr int NRUN = 4;           // runs per tile row
+constexpr int kThreads = 32 * TH * NRUN;
+constexpr int PH = TH + 2;        // plane rows incl. halo
 
 struct ConvArgs {
   const void* x[3];
@@ -91,6 +90,12 @@ template <> __device__ __forceinline__ void store2<float>(float* p, float a, flo
   *reinterpret_cast<float2*>(p) = make_float2(a, b);
 }
 
+// store one channel
+template <typename T> __device__ __forceinline__ void store1(T* p, float a);
+template <> __device__ __forceinline__ void store1<__nv_bfloat16>(__nv_bfloat16* p, float a) { *p = __float2bfloat16_rn(a); }
+template <> __device__ __forceinline__ void store1<__half>(__half* p, float a) { *p = __float2half_rn(a); }
+template <> __device__ __forceinline__ void store1<float>(float* p, float a) { *p = a; }
+
 // raw 16-byte chunk holding 8 channels (bf16: one uint4; fp32: two float4 -> handled separately)
 template <typename T> struct Chunk { uint4 a; };
 template <> struct Chunk<float> { float4 a, b; };
@@ -120,119 +125,155 @@ template <> __device__ __forceinline__ void chunk_store<float>(float* dst, const
 
 // ---- visual kernel -----------------------------------------------------------
 // RUN: pixels per thread along a row (compile-time, so the FMA loop carries no
-// predicates); a tile is 4 runs wide.  Columns past the grid edge read the zero
-// padding of the plane and their outputs are not stored.
-template <typename TIn, typename TOut, int RUN>
+// predicates); a tile is NRUN runs wide.  Columns past the grid edge read the
+// zero padding of the plane and their outputs are not stored.  PT: temporal
+// offset of the first tap (1 centred, 2 causal).
+constexpr int NSLOT = 4;   // plane slots in shared memory (3 planes in flight)
+
+__device__ __forceinline__ float widen1(__nv_bfloat16 h) { return __bfloat162float(h); }
+__device__ __forceinline__ float widen1(float v) { return v; }
+
+// 16-byte cp.async that reads `src_bytes` (16 or 0: zero fill) from global memory
+__device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" :: "r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+
+template <typename TIn, int RUN>
+struct VisPlane {
+  static constexpr int PWr = NRUN * RUN + 2;                       // plane columns incl. halo
+  static constexpr int PIX_CHUNKS = CG * (int)sizeof(TIn) / 16;    // 16-byte chunks per pixel
+  static constexpr int NCHUNK = PH * PWr * PIX_CHUNKS;
+  static constexpr int NPF = (NCHUNK + kThreads - 1) / kThreads;   // chunks per thread
+  static constexpr int BYTES = PH * PWr * CG * (int)sizeof(TIn);
+};
+
+// One plane f: FMAs into the three frames it feeds, then the completed frame out.
+template <typename TIn, typename TOut, int RUN, int PT>
+__device__ __forceinline__ void vis_plane_step(const TIn* pl, bool compute, const float (&wv)[kVisTaps],
+                                               float (&an)[RUN], float (&ac)[RUN], float (&ap)[RUN],
+                                               TOut* yo, bool emit, int nrun, int64_t C) {
+  constexpr int PWr = VisPlane<TIn, RUN>::PWr;
+  if (compute) {
+#pragma unroll
+    for (int tb = 0; tb < 3; ++tb) {
+      const TIn* src = pl + tb * PWr * CG;
+      float in[RUN + 2];
+#pragma unroll
+      for (int i = 0; i < RUN + 2; ++i) in[i] = widen1(src[i * CG]);
+#pragma unroll
+      for (int te = 0; te < 3; ++te) {
+        const float c0 = wv[tb * 3 + te], c1 = wv[9 + tb * 3 + te], c2 = wv[18 + tb * 3 + te];
+#pragma unroll
+        for (int i = 0; i < RUN; ++i) {
+          an[i] = fmaf(c0, in[i + te], an[i]);
+          ac[i] = fmaf(c1, in[i + te], ac[i]);
+          ap[i] = fmaf(c2, in[i + te], ap[i]);
+        }
+      }
+    }
+  }
+  if (emit) {
+#pragma unroll
+    for (int i = 0; i < RUN; ++i)
+      if (i < nrun) store1<TOut>(yo + (int64_t)i * C, ap[i]);
+  }
+#pragma unroll
+  for (int i = 0; i < RUN; ++i) ap[i] = 0.f;   // ap becomes the frame three ahead
+}
+
+template <typename TIn, typename TOut, int RUN, int PT>
 __global__ void __launch_bounds__(kThreads, 1) vis_conv_kernel(ConvArgs a) {
-  extern __shared__ __align__(16) float planes[];   // [3][PH][PW][CG]
-  const int tid = threadIdx.x;
+  using VP = VisPlane<TIn, RUN>;
+  constexpr int PWr = VP::PWr;
+  extern __shared__ __align__(128) uint8_t slots[];   // [NSLOT][PH][PWr][CG] of TIn
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int tile = blockIdx.x;
   const int wt = tile % a.n_wtiles, hb = tile / a.n_wtiles;
   const int cg0 = blockIdx.y * CG;
   const int tensor = blockIdx.z % 3, b = blockIdx.z / 3;
   const int C = a.C;
-  const int tw0 = wt * (4 * RUN), th0 = hb * TH;
-  const int TW = min(4 * RUN, a.Wg - tw0), THh = min(TH, a.Hg - th0);
+  const int tw0 = wt * (NRUN * RUN), th0 = hb * TH;
+  const int TW = min(NRUN * RUN, a.Wg - tw0), THh = min(TH, a.Hg - th0);
   const int64_t HW = (int64_t)a.Hg * a.Wg;
-  const TIn* x = static_cast<const TIn*>(a.x[tensor]) + ((int64_t)b * a.N + a.L) * C + cg0;
-  TOut* y = static_cast<TOut*>(a.y[tensor]) + ((int64_t)b * a.N + a.L) * C + cg0;
+  // pointers chosen by selects, so the argument block is not copied to local memory
+  const void* xs = tensor == 0 ? a.x[0] : (tensor == 1 ? a.x[1] : a.x[2]);
+  void* ys = tensor == 0 ? a.y[0] : (tensor == 1 ? a.y[1] : a.y[2]);
+  const TIn* x = static_cast<const TIn*>(xs) + ((int64_t)b * a.N + a.L) * C + cg0;
+  TOut* y = static_cast<TOut*>(ys) + ((int64_t)b * a.N + a.L) * C + cg0;
 
-  // thread roles
-  const int cp = tid & 15;              // channel pair
-  const int wk = tid >> 4;              // worker 0..15: row wk&3, run wk>>2
-  const int row = wk & 3, run = wk >> 2;
+  const int row = warp % TH, run = warp / TH;
   const int w0 = run * RUN;
   const int nrun = max(0, min(RUN, TW - w0));
   const bool active = row < THh && nrun > 0;
 
-  // weights of channels cg0+2cp, +1
-  float wv0[kVisTaps], wv1[kVisTaps];
+  float wv[kVisTaps];
   {
-    const float* wbase = a.w_vis + ((int64_t)tensor * C + cg0 + 2 * cp) * kVisTaps;
+    const float* wbase = a.w_vis + ((int64_t)tensor * C + cg0 + lane) * kVisTaps;
 #pragma unroll
-    for (int i = 0; i < kVisTaps; ++i) {
-      wv0[i] = wbase[i];
-      wv1[i] = wbase[kVisTaps + i];
-    }
+    for (int i = 0; i < kVisTaps; ++i) wv[i] = wbase[i];
   }
 
-  // plane loader: chunk index e -> (prow, pcol, channel block of 8)
-  const int PWr = 4 * RUN + 2;                       // plane columns read by the runs (incl. halo)
-  const int n_chunks = PH * PWr * (CG / 8);
-  auto plane_fetch = [&](int f, Chunk<TIn> (&buf)[kPrefetch]) {
+  // this thread's chunks of a plane: element offset inside a frame (-1: outside the grid)
+  int goff[VP::NPF];
 #pragma unroll
-    for (int i = 0; i < kPrefetch; ++i) {
-      const int e = tid + i * kThreads;
-      chunk_zero<TIn>(buf[i]);
-      if (e < n_chunks && f >= 0 && f < a.T) {
-        const int cb = e & 3, pix = e >> 2;
-        const int pr = pix / PWr, pc = pix - pr * PWr;
-        const int hh = th0 + pr - 1, ww = tw0 + pc - 1;
-        if (hh >= 0 && hh < a.Hg && ww >= 0 && ww < a.Wg)
-          chunk_load<TIn>(x + ((int64_t)f * HW + (int64_t)hh * a.Wg + ww) * C + cb * 8, buf[i]);
+  for (int i = 0; i < VP::NPF; ++i) {
+    const int e = tid + i * kThreads;
+    goff[i] = -2;   // beyond the plane: nothing to copy
+    if (e < VP::NCHUNK) {
+      const int cb = e % VP::PIX_CHUNKS, pix = e / VP::PIX_CHUNKS;
+      const int pr = pix / PWr, pc = pix - pr * PWr;
+      const int hh = th0 + pr - 1, ww = tw0 + pc - 1;
+      goff[i] = (hh >= 0 && hh < a.Hg && ww >= 0 && ww < a.Wg)
+                    ? (hh * a.Wg + ww) * C + cb * (16 / (int)sizeof(TIn)) : -1;
+    }
+  }
+  const uint32_t slot0 = (uint32_t)__cvta_generic_to_shared(slots);
+  auto issue = [&](int f) {   // plane f -> slot f % NSLOT, one commit group per call
+    if (f < a.T) {
+      const TIn* xf = x + (int64_t)f * HW * C;
+      const uint32_t dst = slot0 + (uint32_t)(f % NSLOT) * VP::BYTES;
+#pragma unroll
+      for (int i = 0; i < VP::NPF; ++i) {
+        if (goff[i] >= -1)
+          cp_async16_zfill(dst + (uint32_t)(tid + i * kThreads) * 16u, goff[i] >= 0 ? xf + goff[i] : x,
+                           goff[i] >= 0 ? 16u : 0u);
       }
     }
-  };
-  auto plane_store = [&](int f, const Chunk<TIn> (&buf)[kPrefetch]) {
-    float* pl = planes + (((f % 3) + 3) % 3) * PLANE_FLOATS;
-#pragma unroll
-    for (int i = 0; i < kPrefetch; ++i) {
-      const int e = tid + i * kThreads;
-      if (e < n_chunks) {
-        const int cb = e & 3, pix = e >> 2;
-        const int pr = pix / PWr, pc = pix - pr * PWr;
-        chunk_store<TIn>(pl + (pr * PW + pc) * CG + cb * 8, buf[i]);
-      }
-    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
   };
 
-  // Frame t reads planes t-pt .. t+2-pt.  Three plane slots in shared memory
-  // (slot = frame mod 3) plus one plane in flight in registers.
-  Chunk<TIn> buf[kPrefetch];
-  for (int f = -a.pt; f <= 2 - a.pt; ++f) {
-    plane_fetch(f, buf);
-    plane_store(f, buf);
-  }
-  __syncthreads();
+  float s0[RUN], s1[RUN], s2[RUN];
+#pragma unroll
+  for (int i = 0; i < RUN; ++i) { s0[i] = 0.f; s1[i] = 0.f; s2[i] = 0.f; }
+  for (int f = 0; f < NSLOT - 1; ++f) issue(f);
 
-  for (int t = 0; t < a.T; ++t) {
-    const int f_next = t + 3 - a.pt;   // first plane frame t+1 needs that is not resident
-    plane_fetch(f_next, buf);          // global loads overlap the compute of frame t
-    if (active) {
-      float acc0[RUN], acc1[RUN];
-#pragma unroll
-      for (int i = 0; i < RUN; ++i) { acc0[i] = 0.f; acc1[i] = 0.f; }
-#pragma unroll
-      for (int ta = 0; ta < 3; ++ta) {
-        const int f = t + ta - a.pt;
-        if (f < 0 || f >= a.T) continue;
-        const float* pl = planes + (f % 3) * PLANE_FLOATS;
-#pragma unroll
-        for (int tb = 0; tb < 3; ++tb) {
-          const float2* src = reinterpret_cast<const float2*>(pl + ((row + tb) * PW + w0) * CG + 2 * cp);
-          float2 in[RUN + 2];
-#pragma unroll
-          for (int i = 0; i < RUN + 2; ++i) in[i] = src[i * (CG / 2)];
-#pragma unroll
-          for (int te = 0; te < 3; ++te) {
-            const float c0 = wv0[(ta * 3 + tb) * 3 + te], c1 = wv1[(ta * 3 + tb) * 3 + te];
-#pragma unroll
-            for (int i = 0; i < RUN; ++i) {
-              acc0[i] = fmaf(c0, in[i + te].x, acc0[i]);
-              acc1[i] = fmaf(c1, in[i + te].y, acc1[i]);
-            }
-          }
-        }
-      }
-      TOut* yo = y + ((int64_t)t * HW + (int64_t)(th0 + row) * a.Wg + tw0 + w0) * C + 2 * cp;
-#pragma unroll
-      for (int i = 0; i < RUN; ++i)
-        if (i < nrun) store2<TOut>(yo + (int64_t)i * C, acc0[i], acc1[i]);
+  // after plane f, frame f+PT-2 is complete; with PT = 1 one step past the last
+  // plane (no data) flushes frame T-1
+  const int f_end = a.T + (PT == 1 ? 1 : 0);
+  const TIn* pl_base = reinterpret_cast<const TIn*>(slots) + (row * PWr + w0) * CG + lane;
+  TOut* y_base = y + ((int64_t)(th0 + row) * a.Wg + tw0 + w0) * C + lane;
+  auto step = [&](int f, float (&an)[RUN], float (&ac)[RUN], float (&ap)[RUN]) {
+    asm volatile("cp.async.wait_group %0;" :: "n"(NSLOT - 2) : "memory");
+    __syncthreads();   // plane f in place everywhere; slot (f-1) % NSLOT no longer read
+    issue(f + NSLOT - 1);
+    const int t = f + PT - 2;
+    vis_plane_step<TIn, TOut, RUN, PT>(pl_base + (f % NSLOT) * (VP::BYTES / (int)sizeof(TIn)),
+                                       active && f < a.T, wv, an, ac, ap, y_base + (int64_t)t * HW * C,
+                                       active && t >= 0 && t < a.T, nrun, C);
+  };
+  // roles rotate with f % 3: (frame f+PT, f+PT-1, f+PT-2) live in sets ((f+PT)%3, ...)
+  for (int f = 0; f < f_end; f += 3) {
+    if (PT == 1) {
+      step(f, s1, s0, s2);
+      if (f + 1 < f_end) step(f + 1, s2, s1, s0);
+      if (f + 2 < f_end) step(f + 2, s0, s2, s1);
+    } else {
+      step(f, s2, s1, s0);
+      if (f + 1 < f_end) step(f + 1, s0, s2, s1);
+      if (f + 2 < f_end) step(f + 2, s1, s0, s2);
     }
-    __syncthreads();                   // every thread is done with the slot of frame t-pt
-    plane_store(f_next, buf);
-    __syncthreads();
   }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 
 // ---- text kernel -------------------------------------------------------------
@@ -262,17 +303,22 @@ __global__ void __launch_bounds__(256) text_conv_kernel(ConvArgs a) {
   for (int e = 0; e < 8; e += 2) store2<TOut>(y + n * C + c0 + e, acc[e], acc[e + 1]);
 }
 
+template <typename TIn, typename TOut, int RUN, int PT>
+cudaError_t launch_vis_pt(const ConvArgs& a, cudaStream_t s) {
+  const size_t smem = (size_t)NSLOT * VisPlane<TIn, RUN>::BYTES;
+  cudaError_t e = cudaFuncSetAttribute(vis_conv_kernel<TIn, TOut, RUN, PT>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)(a.n_wtiles * a.n_hbands), (unsigned)(a.C / CG), (unsigned)(3 * a.B));
+  vis_conv_kernel<TIn, TOut, RUN, PT><<<grid, kThreads, smem, s>>>(a);
+  return cudaGetLastError();
+}
+
 template <typename TIn, typename TOut, int RUN>
 cudaError_t launch_vis(const ConvArgs& a0, cudaStream_t s) {
   ConvArgs a = a0;
-  a.n_wtiles = (a.Wg + 4 * RUN - 1) / (4 * RUN);
-  const size_t smem = 3 * PLANE_FLOATS * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(vis_conv_kernel<TIn, TOut, RUN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
-  if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)(a.n_wtiles * a.n_hbands), (unsigned)(a.C / CG), (unsigned)(3 * a.B));
-  vis_conv_kernel<TIn, TOut, RUN><<<grid, kThreads, smem, s>>>(a);
-  return cudaGetLastError();
+  a.n_wtiles = (a.Wg + NRUN * RUN - 1) / (NRUN * RUN);
+  return a.pt == 2 ? launch_vis_pt<TIn, TOut, RUN, 2>(a, s) : launch_vis_pt<TIn, TOut, RUN, 1>(a, s);
 }
 
 template <typename TIn, typename TOut>
@@ -303,7 +349,7 @@ cudaError_t launch_shortconv(const Dims& d, kda_dtype dt, const void* q, const v
   a.C = d.H * d.dk;
   a.text_k = d.text_k;
   a.T = d.T; a.Hg = d.Hg; a.Wg = d.Wg; a.pt = d.pt;
-  a.n_wtiles = d.T > 0 ? (d.Wg + TWMAX - 1) / TWMAX : 0;
+  a.n_wtiles = 0;   // set per run length by launch_vis
   a.n_hbands = d.T > 0 ? (d.Hg + TH - 1) / TH : 0;
   if ((int64_t)d.B * d.N == 0) return cudaSuccess;
   cudaError_t e;

@@ -81,6 +81,8 @@ def test_host_side_rejections_launch_nothing(kda):
     assert _call_fwd(kda, _p(kda, vis_k=(3, 5, 3))) == kda.KDA_ERR_UNSUPPORTED
     assert _call_fwd(kda, _p(kda, text_k=9)) == kda.KDA_ERR_UNSUPPORTED
     assert _call_fwd(kda, _p(kda, grid=(1, 0, 16))) == kda.KDA_ERR_INVALID_ARG
+    # one frame of 4096 x 4096 tokens x 128 channels exceeds the conv's 32-bit frame offsets
+    assert _call_fwd(kda, _p(kda, d=128, H=1, grid=(1, 4096, 4096))) == kda.KDA_ERR_UNSUPPORTED
     bad = _p(kda)
     bad.flags = 1 << 5
     assert _call_fwd(kda, bad) == kda.KDA_ERR_INVALID_ARG
