@@ -30,7 +30,11 @@
 #include "common.cuh"
 #include "tc.cuh"
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_fp16.h>
+
+#include <mutex>
 
 namespace kda {
 namespace {
@@ -105,6 +109,15 @@ __device__ __forceinline__ uint32_t tmem_at(uint32_t base, int lane0, int col) {
   return base + ((uint32_t)lane0 << 16) + (uint32_t)col;
 }
 
+// Waits for a TMA load counted on `bar`; on timeout records the status.  Returns false on timeout.
+__device__ __forceinline__ bool wait_tma(uint64_t* bar, uint32_t& phase, uint32_t* status, bool alive) {
+  if (!alive) return false;
+  const bool ok = mbar_wait(bar, phase);
+  if (ok) phase ^= 1u;
+  else set_status(status, KDA_ERR_TIMEOUT);
+  return ok;
+}
+
 // Waits on the MMA barrier; on timeout records the status.  Returns false on timeout.
 __device__ __forceinline__ bool wait_mma(uint64_t* bar, uint32_t& phase, uint32_t* status, bool alive) {
   if (!alive) return false;   // nothing was issued
@@ -128,14 +141,21 @@ constexpr uint32_t OFF_B1 = 114688;     // [128][128] fp16: B_1 (MN-major operan
 constexpr uint32_t OFF_AS = 147456;     // fp32 [64][65]: A (strictly lower, beta applied)
 constexpr uint32_t OFF_XS = 164096;     // fp32 [64][65]: (I + A)^{-1}
 constexpr uint32_t OFF_YS = 180736;     // fp32 [32][33]: merge scratch / quarter totals
-constexpr uint32_t OFF_MISC = 184960;   // beta[64], egm, egl, ekt, gm, tot [128 each], barrier, tmem slot, flag
-constexpr uint32_t PREP_SMEM = OFF_MISC + 4096 + 1024;   // + alignment slack
+constexpr uint32_t OFF_MISC = 184960;   // beta[64], egm, egl, ekt, gm, tot [128 each], barriers, tmem slot, flag
+constexpr uint32_t OFF_LA = 189440;     // fp32 [64 tokens][128]: log alpha of the current sub-chunk (TMA)
+constexpr uint32_t PREP_SMEM = OFF_LA + 32768 + 1024;   // + alignment slack
 
 constexpr int LDX = 65;
 
 // TMEM columns
 constexpr int C_AP = 0, C_W = 64, C_U = 192;
 constexpr int C_MK = 0, C_BK = 128, C_PW = 256, C_PU = 384;
+
+// TMA descriptors of the [B][N][H][128] inputs, box [1][64 tokens][1][64 or 128 channels]
+struct PrepMaps {
+  CUtensorMap q, k, v;   // 64-channel boxes, 128-byte swizzle: one operand panel each
+  CUtensorMap la;        // 128-channel box, no swizzle
+};
 
 struct PrepArgs {
   const void* q; const void* k; const void* v;
@@ -227,7 +247,7 @@ __device__ void unit_lower_inverse64(const float* As, float* Xs, float* Ys) {
 }
 
 template <typename TIn>
-__global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a) {
+__global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_constant__ PrepMaps mp) {
   extern __shared__ uint8_t dyn[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn) + 1023) & ~uintptr_t(1023));
   uint8_t* KQ = sm + OFF_KQ;
@@ -246,8 +266,11 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a) {
   float* ekt = egl + 128;                                       // 128: e^{g_l - g_m}
   float* gm_s = ekt + 128;                                      // 128
   float* tot_s = gm_s + 128;                                    // 128
-  uint64_t* bar = reinterpret_cast<uint64_t*>(tot_s + 128);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 2);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(tot_s + 128);    // [0] MMA, [1] k/q/v tiles, [2] log alpha
+  uint64_t* kqv_bar = bar + 1;
+  uint64_t* la_bar = bar + 2;
+  const float* LAs = reinterpret_cast<const float*>(sm + OFF_LA);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 4);
   int* range_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -256,13 +279,30 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a) {
 
   if (*(volatile uint32_t*)a.status == KDA_ERR_TIMEOUT) return;   // an earlier CTA gave up: skip the work
   if (warp == 0) { tmem_alloc(tmem_slot, 512); tmem_relinquish(); }
-  if (tid == 0) { mbar_init(bar, 1); fence_mbar_init(); *range_flag = 0; }
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    mbar_init(kqv_bar, 1);
+    mbar_init(la_bar, 1);
+    fence_mbar_init();
+    *range_flag = 0;
+  }
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
   const uint32_t tm = *tmem_slot;
-  uint32_t phase = 0;
+  uint32_t phase = 0, kqv_phase = 0, la_phase = 0;
   bool alive = true;
+  bool la_inflight = false, kqv_inflight = false;   // thread 0's view: TMA loads not yet waited for
+  auto issue_la = [&](int u, int s_) {   // log alpha of sub-chunk s_ of unit u -> LAs (thread 0)
+    const int blk_ = u / a.BH, bh_ = u - blk_ * a.BH;
+    const int b_ = bh_ / a.H, h_ = bh_ - b_ * a.H;
+    mbar_arrive_expect_tx(la_bar, 32768);
+    tma_load_4d(sm + OFF_LA, &mp.la, 0, h_, blk_ * BLK + s_ * SUB, b_, la_bar);
+  };
+  if (tid == 0 && (int)blockIdx.x < a.n_units) {
+    issue_la(blockIdx.x, 0);
+    la_inflight = true;
+  }
 
   // operand descriptors of the fixed tiles (stepped along K by kstep / mstep)
   const uint64_t dKQk = kdesc0(smem_u32(KQ)), dKQm = mdesc0(smem_u32(KQ), 16384);
@@ -314,43 +354,44 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a) {
         }
       }
       // ---------------- inputs ----------------
-      // raw k, q, v rows copied straight into their swizzled tile slots
-      // (k -> KQ rows 0-63, q -> KQ rows 64-127, v -> VV); padding rows zeroed
-      for (int e = tid; e < SUB * 16; e += 256) {
-        const int r = e >> 4, ch = (e & 15) * 8, pnl = ch >> 6, cc = ch & 63;
-        uint8_t* dk = KQ + pnl * 16384 + swz_off(r, cc);
-        uint8_t* dq = KQ + pnl * 16384 + swz_off(64 + r, cc);
-        uint8_t* dv = VV + pnl * 8192 + swz_off(r, cc);
-        if (r < nv) {
-          const int64_t go = (t0 + r) * tok_stride + ch;
-          cp_async16(dk, kb + go);
-          cp_async16(dq, qb + go);
-          cp_async16(dv, vb + go);
-        } else {
-          const uint4 z = make_uint4(0, 0, 0, 0);
-          *reinterpret_cast<uint4*>(dk) = z;
-          *reinterpret_cast<uint4*>(dq) = z;
-          *reinterpret_cast<uint4*>(dv) = z;
+      // k -> KQ rows 0-63, q -> KQ rows 64-127, v -> VV: 128-byte-swizzled operand panels
+      // written by TMA; rows past the sequence end read as zero
+      if (tid == 0 && alive) {
+        mbar_arrive_expect_tx(kqv_bar, 6 * 8192);
+#pragma unroll
+        for (int pnl = 0; pnl < 2; ++pnl) {
+          tma_load_4d(KQ + pnl * 16384, &mp.k, 64 * pnl, h, (int)t0, b, kqv_bar);
+          tma_load_4d(KQ + pnl * 16384 + 8192, &mp.q, 64 * pnl, h, (int)t0, b, kqv_bar);
+          tma_load_4d(VV + pnl * 8192, &mp.v, 64 * pnl, h, (int)t0, b, kqv_bar);
         }
+        kqv_inflight = true;
       }
-      cp_async_commit();
-      // thread: channels 2cp, 2cp+1 and tokens 16*qt .. 16*qt+15 of the sub-chunk
+      if (tid < SUB) beta_s[tid] = tid < nv ? __bfloat162float(bb[(t0 + tid) * a.H]) : 0.f;
+      // thread: channels 2cp, 2cp+1 and tokens 16*qt .. 16*qt+15 of the sub-chunk; log alpha
+      // arrived in LAs during the previous sub-chunk (zero past the sequence end)
       const int cp = (tid & 31) + 32 * ((tid >> 5) & 1);
       const int qt = tid >> 6;
       const int c = 2 * cp;
+      bool ok_in = wait_tma(la_bar, la_phase, a.status, alive);
       float2 gl[16];
 #pragma unroll
-      for (int t = 0; t < 16; ++t) {
-        const int tok = 16 * qt + t;
-        gl[t] = tok < nv ? *reinterpret_cast<const float2*>(lab + (t0 + tok) * tok_stride + c) : make_float2(0.f, 0.f);
-      }
+      for (int t = 0; t < 16; ++t) gl[t] = *reinterpret_cast<const float2*>(LAs + (16 * qt + t) * D + c);
 #pragma unroll
       for (int t = 1; t < 16; ++t) { gl[t].x += gl[t - 1].x; gl[t].y += gl[t - 1].y; }
       float2* qtot = reinterpret_cast<float2*>(Ys);      // [4][64] quarter totals
       qtot[qt * 64 + cp] = gl[15];
-      if (tid < SUB) beta_s[tid] = tid < nv ? __bfloat162float(bb[(t0 + tid) * a.H]) : 0.f;
-      cp_async_wait_all();
-      __syncthreads();
+      ok_in = wait_tma(kqv_bar, kqv_phase, a.status, ok_in);
+      alive = __syncthreads_and(ok_in);
+      if (tid == 0 && alive) {
+        la_inflight = false;
+        kqv_inflight = false;
+        // LAs consumed: fetch the log alpha of this CTA's next sub-chunk
+        const int nunit = s == 0 ? unit : unit + (int)gridDim.x;
+        if (alive && nunit < a.n_units) {
+          issue_la(nunit, s ^ 1);
+          la_inflight = true;
+        }
+      }
       float2 pre = make_float2(0.f, 0.f), gmv = make_float2(0.f, 0.f), tot = make_float2(0.f, 0.f);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -641,7 +682,12 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a) {
       }
     }
   }
-  if (tid == 0) bulk_wait_all();
+  if (tid == 0) {
+    // loads still in flight after a timeout land before the CTA exits
+    if (la_inflight) mbar_wait(la_bar, la_phase, 100000000ull);
+    if (kqv_inflight) mbar_wait(kqv_bar, kqv_phase, 100000000ull);
+    bulk_wait_all();
+  }
   if (tid == 0 && *range_flag) set_status(a.status, KDA_ERR_RANGE);
   fence_before_sync();
   __syncthreads();
@@ -884,6 +930,35 @@ __global__ void __launch_bounds__(256, 1) kda_tc_chain(ChainArgs a) {
   if (warp == 0) tmem_dealloc(tm, 256);
 }
 
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// [B][N][H][128] activations seen as a 4D tensor (channel, head, token, item);
+// box: box_c channels x 1 head x 64 tokens x 1 item.  Tokens past N read as zero.
+bool encode_act_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int es, const Dims& d, int box_c,
+                    bool swizzle128) {
+  const PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)d.H, (cuuint64_t)d.N, (cuuint64_t)d.B};
+  const cuuint64_t strides[3] = {(cuuint64_t)D * es, (cuuint64_t)d.H * D * es, (cuuint64_t)d.N * d.H * D * es};
+  const cuuint32_t box[4] = {(cuuint32_t)box_c, 1u, (cuuint32_t)SUB, 1u};
+  const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  return enc(m, dt, 4, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <typename TIn>
 cudaError_t launch_all(const Dims& d, const void* q, const void* k, const void* v, const float* la,
                        const void* beta, const float* S0, void* o, float* SN, uint8_t* ws, uint32_t* status,
@@ -900,7 +975,13 @@ cudaError_t launch_all(const Dims& d, const void* q, const void* k, const void* 
   const int BH = d.B * d.H;
   const int n_units = BH * n_blocks;
   PrepArgs pa{q, k, v, la, beta, ws, d.N, d.H, BH, n_blocks, n_units, status};
-  kda_tc_prep<TIn><<<dim3((unsigned)min(n_units, n_sm)), 256, PREP_SMEM, s>>>(pa);
+  PrepMaps mp;
+  const CUtensorMapDataType adt = kIsHalf<TIn> ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  if (!encode_act_map(&mp.q, q, adt, 2, d, 64, true) || !encode_act_map(&mp.k, k, adt, 2, d, 64, true) ||
+      !encode_act_map(&mp.v, v, adt, 2, d, 64, true) ||
+      !encode_act_map(&mp.la, la, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, d, 128, false))
+    return cudaErrorInvalidValue;
+  kda_tc_prep<TIn><<<dim3((unsigned)min(n_units, n_sm)), 256, PREP_SMEM, s>>>(pa, mp);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   ChainArgs ca{ws, S0, SN, static_cast<__nv_bfloat16*>(o), d.N, d.H, n_blocks, status};
   kda_tc_chain<<<dim3(2, d.H, d.B), 256, CHAIN_SMEM, s>>>(ca);
