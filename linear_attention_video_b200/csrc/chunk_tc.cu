@@ -87,17 +87,11 @@ __device__ __forceinline__ void unpack8(uint4 u, float* v) {
 }
 
 // 32 consecutive fp32 values -> fp16 at (row, col0..col0+31) of a swizzled
-// panel (col0 a multiple of 32).  The four 16-byte chunks are written in an
-// order rotated by `rot`, so rows that share a bank group (row, row+8, ...)
-// write different chunks at the same time.
-__device__ __forceinline__ void st_row32_h(uint8_t* panel, int row, int col0, const float (&v)[32], int rot) {
-  const uint4 p0 = pack8(v), p1 = pack8(v + 8), p2 = pack8(v + 16), p3 = pack8(v + 24);
+// panel (col0 a multiple of 32).  Eight consecutive rows writing the same chunk
+// land in eight different bank groups (the swizzle), so stores need no reordering.
+__device__ __forceinline__ void st_row32_h(uint8_t* panel, int row, int col0, const float (&v)[32]) {
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int c = (i + rot) & 3;
-    const uint4 d = c == 0 ? p0 : c == 1 ? p1 : c == 2 ? p2 : p3;
-    *reinterpret_cast<uint4*>(panel + swz_off(row, col0 + 8 * c)) = d;
-  }
+  for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4*>(panel + swz_off(row, col0 + 8 * c)) = pack8(v + 8 * c);
 }
 // 16 consecutive fp16 values at (row, col0..) of a swizzled panel -> fp32
 __device__ __forceinline__ void ld_row16_h(const uint8_t* panel, int row, int col0, float* v) {
@@ -275,7 +269,6 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int sub = warp & 3, chalf = warp >> 2;
-  const int64_t tok_stride = (int64_t)a.H * D;
 
   if (*(volatile uint32_t*)a.status == KDA_ERR_TIMEOUT) return;   // an earlier CTA gave up: skip the work
   if (warp == 0) { tmem_alloc(tmem_slot, 512); tmem_relinquish(); }
@@ -293,6 +286,25 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
   uint32_t phase = 0, kqv_phase = 0, la_phase = 0;
   bool alive = true;
   bool la_inflight = false, kqv_inflight = false;   // thread 0's view: TMA loads not yet waited for
+  // batch item, head and first token of the sub-chunk this CTA processes after (u, s_)
+  auto next_sub = [&](int u, int s_, int& nb_, int& nh_, int& nt0_) -> bool {
+    const int nu = s_ == 0 ? u : u + (int)gridDim.x;
+    if (nu >= a.n_units) return false;
+    const int blk_ = nu / a.BH, bh_ = nu - blk_ * a.BH;
+    nb_ = bh_ / a.H;
+    nh_ = bh_ - nb_ * a.H;
+    nt0_ = blk_ * BLK + (s_ ^ 1) * SUB;
+    return true;
+  };
+  auto load_beta = [&](int b_, int h_, int t_) -> float {   // 0 past the sequence end
+    return t_ < a.N ? __bfloat162float(static_cast<const __nv_bfloat16*>(a.beta)[((int64_t)b_ * a.N + t_) * a.H + h_])
+                    : 0.f;
+  };
+  float beta_next = 0.f;
+  if (tid < SUB && (int)blockIdx.x < a.n_units) {
+    const int bh_ = (int)blockIdx.x % a.BH;   // unit blockIdx.x: block blockIdx.x / BH, sub-chunk 0
+    beta_next = load_beta(bh_ / a.H, bh_ % a.H, ((int)blockIdx.x / a.BH) * BLK + tid);
+  }
   auto issue_la = [&](int u, int s_) {   // log alpha of sub-chunk s_ of unit u -> LAs (thread 0)
     const int blk_ = u / a.BH, bh_ = u - blk_ * a.BH;
     const int b_ = bh_ / a.H, h_ = bh_ - b_ * a.H;
@@ -318,11 +330,6 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
   for (int unit = blockIdx.x; unit < a.n_units && alive; unit += gridDim.x) {
     const int blk = unit / a.BH, bh = unit - blk * a.BH;
     const int b = bh / a.H, h = bh - b * a.H;
-    const TIn* qb = static_cast<const TIn*>(a.q) + (int64_t)b * a.N * tok_stride + (int64_t)h * D;
-    const TIn* kb = static_cast<const TIn*>(a.k) + (int64_t)b * a.N * tok_stride + (int64_t)h * D;
-    const TIn* vb = static_cast<const TIn*>(a.v) + (int64_t)b * a.N * tok_stride + (int64_t)h * D;
-    const float* lab = a.la + (int64_t)b * a.N * tok_stride + (int64_t)h * D;
-    const __nv_bfloat16* bb = static_cast<const __nv_bfloat16*>(a.beta) + (int64_t)b * a.N * a.H + h;
     uint8_t* rec = a.ws + (((int64_t)b * a.H + h) * a.n_blocks + blk) * kBlockBytes;
     uint8_t* gM = rec + kMOff;
     uint8_t* gB = rec + kBOff;
@@ -332,27 +339,6 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
     for (int s = 0; s < 2; ++s) {
       const int64_t t0 = (int64_t)blk * BLK + s * SUB;
       const int nv = (int)max((int64_t)0, min((int64_t)SUB, a.N - t0));
-      {
-        // bring the rows of this CTA's next sub-chunk into L2 while this one is processed
-        int64_t nt0 = t0 + SUB, noff = 0;
-        bool have = s == 0;
-        if (s == 1 && unit + (int)gridDim.x < a.n_units) {
-          const int nunit = unit + (int)gridDim.x;
-          const int nblk = nunit / a.BH, nbh = nunit - nblk * a.BH;
-          const int nb_ = nbh / a.H, nh = nbh - nb_ * a.H;
-          nt0 = (int64_t)nblk * BLK;
-          noff = ((int64_t)nb_ - b) * a.N * tok_stride + (int64_t)(nh - h) * D;
-          have = true;
-        }
-        const int r = tid & 63, which = tid >> 6;
-        if (have && nt0 + r < a.N) {
-          const int64_t go = (nt0 + r) * tok_stride + noff;
-          if (which == 0) prefetch_l2(kb + go, D * sizeof(TIn));
-          else if (which == 1) prefetch_l2(qb + go, D * sizeof(TIn));
-          else if (which == 2) prefetch_l2(vb + go, D * sizeof(TIn));
-          else prefetch_l2(lab + go, D * sizeof(float));
-        }
-      }
       // ---------------- inputs ----------------
       // k -> KQ rows 0-63, q -> KQ rows 64-127, v -> VV: 128-byte-swizzled operand panels
       // written by TMA; rows past the sequence end read as zero
@@ -365,8 +351,23 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
           tma_load_4d(VV + pnl * 8192, &mp.v, 64 * pnl, h, (int)t0, b, kqv_bar);
         }
         kqv_inflight = true;
+        // and the next sub-chunk's tiles into L2 meanwhile
+        int nb_, nh_, nt0_;
+        if (next_sub(unit, s, nb_, nh_, nt0_)) {
+#pragma unroll
+          for (int pnl = 0; pnl < 2; ++pnl) {
+            tma_prefetch_4d(&mp.k, 64 * pnl, nh_, nt0_, nb_);
+            tma_prefetch_4d(&mp.q, 64 * pnl, nh_, nt0_, nb_);
+            tma_prefetch_4d(&mp.v, 64 * pnl, nh_, nt0_, nb_);
+          }
+        }
       }
-      if (tid < SUB) beta_s[tid] = tid < nv ? __bfloat162float(bb[(t0 + tid) * a.H]) : 0.f;
+      if (tid < SUB) {
+        // beta of this sub-chunk was read one sub-chunk ago; read the next one now
+        beta_s[tid] = beta_next;
+        int nb_, nh_, nt0_;
+        beta_next = next_sub(unit, s, nb_, nh_, nt0_) ? load_beta(nb_, nh_, nt0_ + tid) : 0.f;
+      }
       // thread: channels 2cp, 2cp+1 and tokens 16*qt .. 16*qt+15 of the sub-chunk; log alpha
       // arrived in LAs during the previous sub-chunk (zero past the sequence end)
       const int cp = (tid & 31) + 32 * ((tid >> 5) & 1);
@@ -462,7 +463,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
           const int r = row - 64;
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = (col0 + j <= r) ? v[j] : 0.f;
-          st_row32_h(PP, r, col0, v, (r >> 3) & 3);
+          st_row32_h(PP, r, col0, v);
         }
       }
       fence_before_sync();
@@ -506,7 +507,6 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
       // W' -> KQ rows 0-63, U~ -> VV (fp16); M=64 accumulator layout: rows 16*sub + lane (lane < 16)
       {
         const int r = 16 * sub + lane;
-        const int rot = 2 * ((lane >> 3) & 1);
         for (int cb = 0; cb < 2; ++cb) {
           const int col0 = 64 * chalf + 32 * cb;
           float w[32], u[32];
@@ -514,8 +514,8 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
           tmem_ld32(tmem_at(tm, 32 * sub, C_U + col0), u);
           tmem_wait_ld();
           if (lane < 16) {
-            st_row32_h(KQ + chalf * 16384, r, col0 & 63, w, rot);
-            st_row32_h(VV + chalf * 8192, r, col0 & 63, u, rot);
+            st_row32_h(KQ + chalf * 16384, r, col0 & 63, w);
+            st_row32_h(VV + chalf * 8192, r, col0 & 63, u);
           }
         }
       }
@@ -542,9 +542,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
       alive = __syncthreads_and(wait_mma(bar, phase, a.status, alive));
       fence_after_sync();
       const int row = 32 * sub + lane;        // M=128 layout row
-      const int rot128 = (row >> 3) & 3;
       const int r64 = 16 * sub + lane;        // M=64 layout row (lane < 16)
-      const int rot64 = 2 * ((lane >> 3) & 1);
       if (s == 0) {
         // M_1 = Diag(e^{g_l}) - MK Diag(e^{g_m}) -> M1 tile;  B_1 -> B1 tile
         for (int cb = 0; cb < 2; ++cb) {
@@ -555,8 +553,8 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
           tmem_wait_ld();
 #pragma unroll
           for (int j = 0; j < 32; ++j) m[j] = (row == col0 + j ? egl[row] : 0.f) - m[j] * egm[col0 + j];
-          st_row32_h(M1 + chalf * 16384, row, col0 & 63, m, rot128);
-          st_row32_h(B1 + chalf * 16384, row, col0 & 63, bv, rot128);
+          st_row32_h(M1 + chalf * 16384, row, col0 & 63, m);
+          st_row32_h(B1 + chalf * 16384, row, col0 & 63, bv);
         }
         // R_1 = (QG - P W') Diag(e^{g_m}) and O'_1, staged for the record (R rows 0-63, O'' rows 0-63)
         uint8_t* stR = reinterpret_cast<uint8_t*>(Xs);   // [panel][64 rows][128 B], swizzled
@@ -573,7 +571,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
             ld_row16_h(KQ + chalf * 16384, 64 + r64, (col0 & 63) + 16, qg + 16);
 #pragma unroll
             for (int j = 0; j < 32; ++j) qg[j] = (qg[j] - pw[j]) * egm[col0 + j];
-            st_row32_h(stR + chalf * 8192, r64, col0 & 63, qg, rot64);
+            st_row32_h(stR + chalf * 8192, r64, col0 & 63, qg);
 #pragma unroll
             for (int i = 0; i < 4; ++i) stO[((col0 >> 3) + i) * 64 + r64] = pack8(pu + 8 * i);
           }
@@ -600,7 +598,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
             ld_row16_h(KQ + chalf * 16384, 64 + r64, (col0 & 63) + 16, qg + 16);
 #pragma unroll
             for (int j = 0; j < 32; ++j) qg[j] = (qg[j] - pw[j]) * egm[col0 + j];
-            st_row32_h(VV + chalf * 8192, r64, col0 & 63, qg, rot64);
+            st_row32_h(VV + chalf * 8192, r64, col0 & 63, qg);
           }
         }
         __syncthreads();
@@ -612,7 +610,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
           tmem_wait_ld();
 #pragma unroll
           for (int j = 0; j < 32; ++j) m[j] = (row == col0 + j ? egl[row] : 0.f) - m[j] * egm[col0 + j];
-          st_row32_h(KQ + chalf * 16384, row, col0 & 63, m, rot128);
+          st_row32_h(KQ + chalf * 16384, row, col0 & 63, m);
         }
         fence_proxy_async();
         fence_before_sync();
@@ -647,7 +645,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
           tmem_ld32(tmem_at(tm, 32 * sub, C_MK + col0), m);
           tmem_ld32(tmem_at(tm, 32 * sub, C_BK + col0), bv);
           tmem_wait_ld();
-          st_row32_h(M1 + chalf * 16384, row, col0 & 63, m, rot128);
+          st_row32_h(M1 + chalf * 16384, row, col0 & 63, m);
           // B: [c/8][row][8]
           uint4* b16 = reinterpret_cast<uint4*>(B1);
 #pragma unroll
@@ -660,7 +658,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
           tmem_ld32(tmem_at(tm, 32 * sub, C_PU + col0), oo);
           tmem_wait_ld();
           if (lane < 16) {
-            st_row32_h(stR + chalf * 8192, r64, col0 & 63, rr, rot64);
+            st_row32_h(stR + chalf * 8192, r64, col0 & 63, rr);
 #pragma unroll
             for (int i = 0; i < 4; ++i) stO[((col0 >> 3) + i) * 64 + r64] = pack8(oo + 8 * i);
           }
