@@ -23,7 +23,7 @@
 //   kda_tc_prep   persistent, one CTA per SM, looping over (block, batch item,
 //                 head) units: everything above, written to the workspace as one
 //                 record per unit (M, B, R, O'' in fp16 operand images).
-//   kda_tc_chain  one CTA per (batch item, head, half of the value columns):
+//   kda_tc_chain  one CTA per (batch item, head, 32 of the value columns):
 //                 the serial pass S <- M S + B, state kept in registers (fp32),
 //                 and beside it the block outputs O = R S + O''.
 // Padding tokens of the last block carry k = q = v = 0, beta = 0, log alpha = 0.
@@ -48,7 +48,7 @@ constexpr float kRange = 9.f;     // max |g - g_m| allowed for the fp16 factors
 
 // Record per (batch item, head, block), all fp16:
 //   M   K-major operand image: 2 panels [128 rows][64 cols]            32 KB
-//   B   [half][c/8][row a][8]  (16-byte units)                         32 KB
+//   B   [c/8][row a][8]  (16-byte units)                               32 KB
 //   R   K-major operand image: 2 panels [128 rows][64 cols]            32 KB
 //   O'' [row half][c/8][row r % 64][8]  (16-byte units)                32 KB
 constexpr size_t kMOff = 0, kBOff = 32768, kROff = 65536, kOOff = 98304;
@@ -132,14 +132,16 @@ constexpr uint32_t OFF_TT = 65536;      // [64][64] fp16: T
 constexpr uint32_t OFF_PP = 73728;      // [64][64] fp16: P
 constexpr uint32_t OFF_M1 = 81920;      // [128][128] fp16: M_1 (MN-major operand image)
 constexpr uint32_t OFF_B1 = 114688;     // [128][128] fp16: B_1 (MN-major operand image)
-constexpr uint32_t OFF_AS = 147456;     // fp32 [64][65]: A (strictly lower, beta applied)
-constexpr uint32_t OFF_XS = 164096;     // fp32 [64][65]: (I + A)^{-1}
-constexpr uint32_t OFF_YS = 180736;     // fp32 [32][33]: merge scratch / quarter totals
-constexpr uint32_t OFF_MISC = 184960;   // beta[64], egm, egl, ekt, gm, tot [128 each], barriers, tmem slot, flag
-constexpr uint32_t OFF_LA = 189440;     // fp32 [64 tokens][128]: log alpha of the current sub-chunk (TMA)
+constexpr uint32_t OFF_AS = 147456;     // fp32 [64][LDA]: A (strictly lower, beta applied)
+constexpr uint32_t OFF_XS = 164096;     // fp32 [64][LDXS]: (I + A)^{-1}
+constexpr uint32_t OFF_YS = 181504;     // fp32 [32][36]: merge scratch / quarter totals
+constexpr uint32_t OFF_MISC = 186112;   // beta[64], egm, egl, ekt, gm, tot [128 each], barriers, tmem slot, flag
+constexpr uint32_t OFF_LA = 190464;     // fp32 [64 tokens][128]: log alpha of the current sub-chunk (TMA)
 constexpr uint32_t PREP_SMEM = OFF_LA + 32768 + 1024;   // + alignment slack
 
-constexpr int LDX = 65;
+constexpr int LDA = 65;    // row stride of A: rows written by consecutive lanes hit consecutive banks
+constexpr int LDXS = 68;   // row stride of X: rows 16-byte aligned for 4-wide loads
+constexpr int LDY = 36;    // row stride of the merge scratch
 
 // TMEM columns
 constexpr int C_AP = 0, C_W = 64, C_U = 192;
@@ -175,17 +177,17 @@ __device__ void unit_lower_inverse64(const float* As, float* Xs, float* Ys) {
 #pragma unroll
     for (int m = 0; m < 15; ++m) {
 #pragma unroll
-      for (int r = m + 1; r < 16; ++r) x[r] -= As[(o + r) * LDX + o + m] * x[m];
+      for (int r = m + 1; r < 16; ++r) x[r] -= As[(o + r) * LDA + o + m] * x[m];
     }
 #pragma unroll
-    for (int r = 0; r < 16; ++r) Xs[(o + r) * LDX + o + l] = x[r];
+    for (int r = 0; r < 16; ++r) Xs[(o + r) * LDXS + o + l] = x[r];
   } else if (warp >= 4) {
     // zero blocks (0,1) and (2,3)
     const int e = tid - 128, r = e >> 3, c = 2 * (e & 7);   // 16 rows x 8 column pairs
-    Xs[r * LDX + 16 + c] = 0.f;
-    Xs[r * LDX + 17 + c] = 0.f;
-    Xs[(32 + r) * LDX + 48 + c] = 0.f;
-    Xs[(32 + r) * LDX + 49 + c] = 0.f;
+    Xs[r * LDXS + 16 + c] = 0.f;
+    Xs[r * LDXS + 17 + c] = 0.f;
+    Xs[(32 + r) * LDXS + 48 + c] = 0.f;
+    Xs[(32 + r) * LDXS + 49 + c] = 0.f;
   }
   __syncthreads();
   {
@@ -196,9 +198,9 @@ __device__ void unit_lower_inverse64(const float* As, float* Xs, float* Ys) {
     float y0 = 0.f, y1 = 0.f;
 #pragma unroll
     for (int m = 0; m < 16; ++m) {
-      const float d = Xs[(o + m) * LDX + o + j];
-      y0 += As[(o + 16 + i0) * LDX + o + m] * d;
-      y1 += As[(o + 17 + i0) * LDX + o + m] * d;
+      const float d = Xs[(o + m) * LDXS + o + j];
+      y0 += As[(o + 16 + i0) * LDA + o + m] * d;
+      y1 += As[(o + 17 + i0) * LDA + o + m] * d;
     }
     Y[i0 * 17 + j] = y0;
     Y[(i0 + 1) * 17 + j] = y1;
@@ -207,35 +209,70 @@ __device__ void unit_lower_inverse64(const float* As, float* Xs, float* Ys) {
 #pragma unroll
     for (int k = 0; k < 16; ++k) {
       const float y = Y[k * 17 + j];
-      z0 += Xs[(o + 16 + i0) * LDX + o + 16 + k] * y;
-      z1 += Xs[(o + 17 + i0) * LDX + o + 16 + k] * y;
+      z0 += Xs[(o + 16 + i0) * LDXS + o + 16 + k] * y;
+      z1 += Xs[(o + 17 + i0) * LDXS + o + 16 + k] * y;
     }
-    Xs[(o + 16 + i0) * LDX + o + j] = -z0;
-    Xs[(o + 17 + i0) * LDX + o + j] = -z1;
+    Xs[(o + 16 + i0) * LDXS + o + j] = -z0;
+    Xs[(o + 17 + i0) * LDXS + o + j] = -z1;
   }
   __syncthreads();
   {
-    // 64-merge: X[32.., 0..31] = -X_22 (A_21 X_11); 2x2 outputs per thread
-    const int r0 = 2 * (tid >> 4), c0 = 2 * (tid & 15);
-    float a00 = 0.f, a01 = 0.f, a10 = 0.f, a11 = 0.f;
+    // 64-merge: X[32.., 0..31] = -X_22 (A_21 X_11), two 32x32x32 products.  Warp w
+    // owns output rows 4w..4w+3; lane = (tile column tc, K quarter g): a 4x4 tile
+    // over 8 of the 32 K indices, then the four quarters are summed across lanes.
+    const int tc = lane & 7, g = lane >> 3;
+    const int r0 = 4 * warp, c0 = 4 * tc;
+    float acc[4][4];
 #pragma unroll
-    for (int m = 0; m < 32; ++m) {
-      const float x0 = Xs[m * LDX + c0], x1 = Xs[m * LDX + c0 + 1];
-      const float u0 = As[(32 + r0) * LDX + m], u1 = As[(33 + r0) * LDX + m];
-      a00 += u0 * x0; a01 += u0 * x1; a10 += u1 * x0; a11 += u1 * x1;
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+      const int m = 8 * g + it;
+      const float4 x = *reinterpret_cast<const float4*>(Xs + m * LDXS + c0);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float u = As[(32 + r0 + i) * LDA + m];
+        acc[i][0] += u * x.x; acc[i][1] += u * x.y; acc[i][2] += u * x.z; acc[i][3] += u * x.w;
+      }
     }
-    Ys[r0 * 33 + c0] = a00; Ys[r0 * 33 + c0 + 1] = a01;
-    Ys[(r0 + 1) * 33 + c0] = a10; Ys[(r0 + 1) * 33 + c0 + 1] = a11;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        acc[i][j] += __shfl_xor_sync(0xffffffffu, acc[i][j], 8);
+        acc[i][j] += __shfl_xor_sync(0xffffffffu, acc[i][j], 16);
+      }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)   // lane quarter g writes row g of the tile
+      if (i == g) *reinterpret_cast<float4*>(Ys + (r0 + i) * LDY + c0) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
     __syncthreads();
-    a00 = a01 = a10 = a11 = 0.f;
 #pragma unroll
-    for (int m = 0; m < 32; ++m) {
-      const float y0 = Ys[m * 33 + c0], y1 = Ys[m * 33 + c0 + 1];
-      const float u0 = Xs[(32 + r0) * LDX + 32 + m], u1 = Xs[(33 + r0) * LDX + 32 + m];
-      a00 += u0 * y0; a01 += u0 * y1; a10 += u1 * y0; a11 += u1 * y1;
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+#pragma unroll
+    for (int it = 0; it < 8; ++it) {
+      const int m = 8 * g + it;
+      const float4 y = *reinterpret_cast<const float4*>(Ys + m * LDY + c0);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float u = Xs[(32 + r0 + i) * LDXS + 32 + m];
+        acc[i][0] += u * y.x; acc[i][1] += u * y.y; acc[i][2] += u * y.z; acc[i][3] += u * y.w;
+      }
     }
-    Xs[(32 + r0) * LDX + c0] = -a00; Xs[(32 + r0) * LDX + c0 + 1] = -a01;
-    Xs[(33 + r0) * LDX + c0] = -a10; Xs[(33 + r0) * LDX + c0 + 1] = -a11;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        acc[i][j] += __shfl_xor_sync(0xffffffffu, acc[i][j], 8);
+        acc[i][j] += __shfl_xor_sync(0xffffffffu, acc[i][j], 16);
+      }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (i == g)
+        *reinterpret_cast<float4*>(Xs + (32 + r0 + i) * LDXS + c0) = make_float4(-acc[i][0], -acc[i][1], -acc[i][2], -acc[i][3]);
     __syncthreads();
   }
 }
@@ -458,7 +495,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
         if (sub < 2) {
           const float bt = beta_s[row];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) As[row * LDX + col0 + j] = (col0 + j < row) ? bt * v[j] : 0.f;
+          for (int j = 0; j < 32; ++j) As[row * LDA + col0 + j] = (col0 + j < row) ? bt * v[j] : 0.f;
         } else {
           const int r = row - 64;
 #pragma unroll
@@ -474,7 +511,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
         const int r = e >> 3, c0 = (e & 7) * 8;
         float v[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) v[j] = c0 + j <= r ? Xs[r * LDX + c0 + j] * beta_s[c0 + j] : 0.f;
+        for (int j = 0; j < 8; ++j) v[j] = c0 + j <= r ? Xs[r * LDXS + c0 + j] * beta_s[c0 + j] : 0.f;
         *reinterpret_cast<uint4*>(TT + swz_off(r, c0)) = pack8(v);
       }
       fence_proxy_async();
@@ -694,7 +731,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
 }
 
 // ---------------------------------------------------------------------------
-// kda_tc_chain: per (batch item, head, half of the value columns) the serial
+// kda_tc_chain: per (batch item, head, CW value columns) the serial
 // pass S <- M S + B over the blocks, fused with the block outputs O = R S + O''.
 //   warps 0-3, the state group: thread t owns row t of S (fp32, in registers);
 //     thread 0 loads M, B and issues M S.
@@ -703,7 +740,11 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
 // Both products read the fp16 image of S_j; two images alternate so the next
 // state is written while R S_j may still be reading the current one.
 // ---------------------------------------------------------------------------
-constexpr uint32_t CH_SLOT = 49152;                  // 32 KB operand image + 16 KB fp16 half-width tile
+constexpr int CW = 32;                               // value columns per CTA
+constexpr int NQ = D / CW;                           // CTAs per (batch item, head)
+constexpr uint32_t CW_BYTES = 128 * CW * 2;          // fp16 [128 rows][CW columns]
+constexpr uint32_t CH_SLOT = 32768 + CW_BYTES;       // 32 KB operand image + the CTA's columns of B or O''
+constexpr uint32_t CT_O = CW;                        // TMEM: M S at column 0, R S buffers at CW and 2 CW
 constexpr uint32_t CH_OFF_A = 0;                     // ring A: M_j, B_j   (2 slots)
 constexpr uint32_t CH_OFF_B = 2 * CH_SLOT;           // ring B: R_j, O''_j (2 slots)
 constexpr uint32_t CH_OFF_S = 4 * CH_SLOT;           // S_j fp16 MN-major images (2 x 16 KB)
@@ -743,12 +784,12 @@ __global__ void __launch_bounds__(256, 1) kda_tc_chain(ChainArgs a) {
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int tid = threadIdx.x, warp = tid >> 5;
-  const int half = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int qtr = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int nb = a.n_blocks;
   const int64_t rec0 = ((int64_t)b * a.H + h) * nb;
   if (*(volatile uint32_t*)a.status == KDA_ERR_TIMEOUT) return;   // an earlier kernel gave up
 
-  if (warp == 0) { tmem_alloc(tmem_slot, 256); tmem_relinquish(); }
+  if (warp == 0) { tmem_alloc(tmem_slot, 128); tmem_relinquish(); }
   if (tid == 0) {
     for (int i = 0; i < 11; ++i) mbar_init(&bars[i], (i == 7 || i == 8) ? 128 : 1);
     *abort_flag = 0;
@@ -758,7 +799,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_chain(ChainArgs a) {
   __syncthreads();
   fence_after_sync();
   const uint32_t tm = *tmem_slot;
-  const uint32_t idesc = idesc_f16(128, 64, false, true);
+  const uint32_t idesc = idesc_f16(128, CW, false, true);
   const uint64_t dS = mdesc0(smem_u32(sm + CH_OFF_S), 16384);
   const int lane_base = 32 * (warp & 3);
   bool ok = true;
@@ -771,19 +812,19 @@ __global__ void __launch_bounds__(256, 1) kda_tc_chain(ChainArgs a) {
       const uint8_t* rec = a.ws + (rec0 + j) * kBlockBytes;
       mbar_arrive_expect_tx(&fullA[j & 1], CH_SLOT);
       bulk_g2s(dst, rec + kMOff, 32768, &fullA[j & 1]);
-      bulk_g2s(dst + 32768, rec + kBOff + half * 16384, 16384, &fullA[j & 1]);
+      bulk_g2s(dst + 32768, rec + kBOff + qtr * CW_BYTES, CW_BYTES, &fullA[j & 1]);
     };
     int issuedA = 0, seenA = 0, mma_pending = 0;
     if (tid == 0)
       for (; issuedA < 2 && issuedA < nb; ++issuedA) load_A(issuedA);
-    float S[64];
+    float S[CW];
 #pragma unroll
-    for (int c = 0; c < 64; ++c)
-      S[c] = a.S0 ? a.S0[(((int64_t)b * a.H + h) * D + row) * D + 64 * half + c] : 0.f;
+    for (int c = 0; c < CW; ++c)
+      S[c] = a.S0 ? a.S0[(((int64_t)b * a.H + h) * D + row) * D + CW * qtr + c] : 0.f;
     auto store_S = [&](int slot) {
       uint8_t* img = sm + CH_OFF_S + slot * 16384;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) *reinterpret_cast<uint4*>(img + swz_off(row, 8 * i)) = pack8(S + 8 * i);
+      for (int i = 0; i < CW / 8; ++i) *reinterpret_cast<uint4*>(img + swz_off(row, 8 * i)) = pack8(S + 8 * i);
       fence_proxy_async();
       mbar_arrive(&sReady[slot]);
     };
@@ -812,7 +853,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_chain(ChainArgs a) {
         fence_after_sync();
         const uint4* Bs = reinterpret_cast<const uint4*>(sm + CH_OFF_A + (j & 1) * CH_SLOT + 32768);
 #pragma unroll
-        for (int c0 = 0; c0 < 64; c0 += 32) {
+        for (int c0 = 0; c0 < CW; c0 += 32) {
           float v[32];
           tmem_ld32(tmem_at(tm, lane_base, c0), v);
           uint4 bu[4];
@@ -839,7 +880,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_chain(ChainArgs a) {
     }
     if (ok && a.SN) {
 #pragma unroll
-      for (int c = 0; c < 64; ++c) a.SN[(((int64_t)b * a.H + h) * D + row) * D + 64 * half + c] = S[c];
+      for (int c = 0; c < CW; ++c) a.SN[(((int64_t)b * a.H + h) * D + row) * D + CW * qtr + c] = S[c];
     }
     if (tid == 0) {
       if (mma_pending) mbar_wait(msDone, (uint32_t)(j - 1) & 1u, 100000000ull);
@@ -854,15 +895,15 @@ __global__ void __launch_bounds__(256, 1) kda_tc_chain(ChainArgs a) {
       const uint8_t* rec = a.ws + (rec0 + j) * kBlockBytes;
       mbar_arrive_expect_tx(&fullB[j & 1], CH_SLOT);
       bulk_g2s(dst, rec + kROff, 32768, &fullB[j & 1]);
-      bulk_g2s(dst + 32768, rec + kOOff + half * 8192, 8192, &fullB[j & 1]);
-      bulk_g2s(dst + 40960, rec + kOOff + 16384 + half * 8192, 8192, &fullB[j & 1]);
+      bulk_g2s(dst + 32768, rec + kOOff + qtr * (CW_BYTES / 2), CW_BYTES / 2, &fullB[j & 1]);
+      bulk_g2s(dst + 32768 + CW_BYTES / 2, rec + kOOff + 16384 + qtr * (CW_BYTES / 2), CW_BYTES / 2, &fullB[j & 1]);
     };
     int issuedB = 0, seenB = 0, o_pending = -1;
     if (leader)
       for (; issuedB < 2 && issuedB < nb; ++issuedB) load_B(issuedB);
     const uint64_t dR = kdesc0(smem_u32(sm + CH_OFF_B));
     const int64_t tok_stride = (int64_t)a.H * D;
-    __nv_bfloat16* obase = a.o + (int64_t)b * a.N * tok_stride + (int64_t)h * D + 64 * half;
+    __nv_bfloat16* obase = a.o + (int64_t)b * a.N * tok_stride + (int64_t)h * D + CW * qtr;
     for (int j = 0; j < nb && ok; ++j) {
       if (leader) {
         bool go = wait_or_abort(&sReady[j & 1], (uint32_t)(j >> 1) & 1u, abort_flag);
@@ -872,7 +913,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_chain(ChainArgs a) {
           fence_after_sync();
           const uint64_t da = dR + (uint32_t)(j & 1) * (CH_SLOT >> 4);
           const uint64_t db = dS + (uint32_t)(j & 1) * (16384u >> 4);
-          const uint32_t d = tm + 64 + 64 * (uint32_t)(j & 1);
+          const uint32_t d = tm + CT_O + CW * (uint32_t)(j & 1);
 #pragma unroll
           for (int k16 = 0; k16 < 8; ++k16) mma_ss(d, da + kstep(k16, 16384), db + mstep(k16), idesc, k16 > 0);
           mma_commit(&oDone[j & 1]);
@@ -889,12 +930,12 @@ __global__ void __launch_bounds__(256, 1) kda_tc_chain(ChainArgs a) {
         const int64_t tok = (int64_t)j * BLK + r;
         __nv_bfloat16* orow = obase + tok * tok_stride;
 #pragma unroll
-        for (int c0 = 0; c0 < 64; c0 += 32) {
+        for (int c0 = 0; c0 < CW; c0 += 32) {
           float v[32];
-          tmem_ld32(tmem_at(tm, lane_base, 64 + 64 * (j & 1) + c0), v);
+          tmem_ld32(tmem_at(tm, lane_base, CT_O + CW * (j & 1) + c0), v);
           uint4 ou[4];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) ou[i] = Oo[((r >> 6) * 8 + (c0 >> 3) + i) * 64 + (r & 63)];
+          for (int i = 0; i < 4; ++i) ou[i] = Oo[((r >> 6) * (CW / 8) + (c0 >> 3) + i) * 64 + (r & 63)];
           tmem_wait_ld();
           if (tok < a.N) {
 #pragma unroll
@@ -925,7 +966,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_chain(ChainArgs a) {
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
-  if (warp == 0) tmem_dealloc(tm, 256);
+  if (warp == 0) tmem_dealloc(tm, 128);
 }
 
 // cuTensorMapEncodeTiled from the driver, looked up once through the runtime
@@ -982,7 +1023,7 @@ cudaError_t launch_all(const Dims& d, const void* q, const void* k, const void* 
   kda_tc_prep<TIn><<<dim3((unsigned)min(n_units, n_sm)), 256, PREP_SMEM, s>>>(pa, mp);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   ChainArgs ca{ws, S0, SN, static_cast<__nv_bfloat16*>(o), d.N, d.H, n_blocks, status};
-  kda_tc_chain<<<dim3(2, d.H, d.B), 256, CHAIN_SMEM, s>>>(ca);
+  kda_tc_chain<<<dim3(NQ, d.H, d.B), 256, CHAIN_SMEM, s>>>(ca);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (launches) *launches += 2;
   return cudaSuccess;
