@@ -23,7 +23,7 @@
 //   kda_tc_prep   persistent, one CTA per SM, looping over (block, batch item,
 //                 head) units: everything above, written to the workspace as one
 //                 record per unit (M, B, R, O'' in fp16 operand images).
-//   kda_tc_chain  one CTA per (batch item, head, 32 of the value columns):
+//   kda_tc_chain  one CTA per (batch item, head, 16, 32 or 64 value columns):
 //                 the serial pass S <- M S + B, state kept in registers (fp32),
 //                 and beside it the block outputs O = R S + O''.
 // Padding tokens of the last block carry k = q = v = 0, beta = 0, log alpha = 0.
@@ -97,6 +97,13 @@ __device__ __forceinline__ void st_row32_h(uint8_t* panel, int row, int col0, co
 __device__ __forceinline__ void ld_row16_h(const uint8_t* panel, int row, int col0, float* v) {
   unpack8(*reinterpret_cast<const uint4*>(panel + swz_off(row, col0)), v);
   unpack8(*reinterpret_cast<const uint4*>(panel + swz_off(row, col0 + 8)), v + 8);
+}
+
+// 16 or 32 consecutive TMEM columns of this warp's lanes
+template <int N>
+__device__ __forceinline__ void tmem_ld_n(uint32_t taddr, float (&v)[N]) {
+  static_assert(N == 16 || N == 32, "16 or 32 columns");
+  if constexpr (N == 16) tmem_ld16(taddr, v); else tmem_ld32(taddr, v);
 }
 
 __device__ __forceinline__ uint32_t tmem_at(uint32_t base, int lane0, int col) {
@@ -740,16 +747,19 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
 // Both products read the fp16 image of S_j; two images alternate so the next
 // state is written while R S_j may still be reading the current one.
 // ---------------------------------------------------------------------------
-constexpr int CW = 32;                               // value columns per CTA
-constexpr int NQ = D / CW;                           // CTAs per (batch item, head)
-constexpr uint32_t CW_BYTES = 128 * CW * 2;          // fp16 [128 rows][CW columns]
-constexpr uint32_t CH_SLOT = 32768 + CW_BYTES;       // 32 KB operand image + the CTA's columns of B or O''
-constexpr uint32_t CT_O = CW;                        // TMEM: M S at column 0, R S buffers at CW and 2 CW
-constexpr uint32_t CH_OFF_A = 0;                     // ring A: M_j, B_j   (2 slots)
-constexpr uint32_t CH_OFF_B = 2 * CH_SLOT;           // ring B: R_j, O''_j (2 slots)
-constexpr uint32_t CH_OFF_S = 4 * CH_SLOT;           // S_j fp16 MN-major images (2 x 16 KB)
-constexpr uint32_t CH_OFF_BAR = CH_OFF_S + 32768;
-constexpr uint32_t CHAIN_SMEM = CH_OFF_BAR + 256 + 1024;
+// Layout for CW value columns per CTA (16, 32 or 64; the MMA N is CW).
+template <int CW>
+struct ChainLayout {
+  static constexpr int NQ = D / CW;                           // CTAs per (batch item, head)
+  static constexpr uint32_t CW_BYTES = 128 * CW * 2;          // fp16 [128 rows][CW columns]
+  static constexpr uint32_t SLOT = 32768 + CW_BYTES;          // 32 KB operand image + the CTA's columns of B or O''
+  static constexpr uint32_t CT_O = CW;                        // TMEM: M S at column 0, R S buffers at CW and 2 CW
+  static constexpr uint32_t OFF_A = 0;                        // ring A: M_j, B_j   (2 slots)
+  static constexpr uint32_t OFF_B = 2 * SLOT;                 // ring B: R_j, O''_j (2 slots)
+  static constexpr uint32_t OFF_S = 4 * SLOT;                 // S_j fp16 MN-major images (2 x 16 KB)
+  static constexpr uint32_t OFF_BAR = OFF_S + 32768;
+  static constexpr uint32_t SMEM = OFF_BAR + 256 + 1024;
+};
 
 struct ChainArgs {
   const uint8_t* ws;
@@ -771,7 +781,13 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
   return true;
 }
 
+template <int CW>
 __global__ void __launch_bounds__(256, 1) kda_tc_chain(ChainArgs a) {
+  using L = ChainLayout<CW>;
+  constexpr uint32_t CW_BYTES = L::CW_BYTES, CH_SLOT = L::SLOT, CT_O = L::CT_O;
+  constexpr uint32_t CH_OFF_A = L::OFF_A, CH_OFF_B = L::OFF_B, CH_OFF_S = L::OFF_S, CH_OFF_BAR = L::OFF_BAR;
+  constexpr int CK = CW < 32 ? CW : 32;   // columns per TMEM load
+  constexpr uint32_t TCOLS = 3 * CW <= 64 ? 64 : (3 * CW <= 128 ? 128 : 256);   // M S and two R S buffers
   extern __shared__ uint8_t dyn[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + CH_OFF_BAR);
@@ -789,7 +805,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_chain(ChainArgs a) {
   const int64_t rec0 = ((int64_t)b * a.H + h) * nb;
   if (*(volatile uint32_t*)a.status == KDA_ERR_TIMEOUT) return;   // an earlier kernel gave up
 
-  if (warp == 0) { tmem_alloc(tmem_slot, 128); tmem_relinquish(); }
+  if (warp == 0) { tmem_alloc(tmem_slot, TCOLS); tmem_relinquish(); }
   if (tid == 0) {
     for (int i = 0; i < 11; ++i) mbar_init(&bars[i], (i == 7 || i == 8) ? 128 : 1);
     *abort_flag = 0;
@@ -853,15 +869,15 @@ __global__ void __launch_bounds__(256, 1) kda_tc_chain(ChainArgs a) {
         fence_after_sync();
         const uint4* Bs = reinterpret_cast<const uint4*>(sm + CH_OFF_A + (j & 1) * CH_SLOT + 32768);
 #pragma unroll
-        for (int c0 = 0; c0 < CW; c0 += 32) {
-          float v[32];
-          tmem_ld32(tmem_at(tm, lane_base, c0), v);
-          uint4 bu[4];
+        for (int c0 = 0; c0 < CW; c0 += CK) {
+          float v[CK];
+          tmem_ld_n(tmem_at(tm, lane_base, c0), v);
+          uint4 bu[CK / 8];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) bu[i] = Bs[((c0 >> 3) + i) * 128 + row];
+          for (int i = 0; i < CK / 8; ++i) bu[i] = Bs[((c0 >> 3) + i) * 128 + row];
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
+          for (int i = 0; i < CK / 8; ++i) {
             float bf[8];
             unpack8(bu[i], bf);
 #pragma unroll
@@ -930,16 +946,16 @@ __global__ void __launch_bounds__(256, 1) kda_tc_chain(ChainArgs a) {
         const int64_t tok = (int64_t)j * BLK + r;
         __nv_bfloat16* orow = obase + tok * tok_stride;
 #pragma unroll
-        for (int c0 = 0; c0 < CW; c0 += 32) {
-          float v[32];
-          tmem_ld32(tmem_at(tm, lane_base, CT_O + CW * (j & 1) + c0), v);
-          uint4 ou[4];
+        for (int c0 = 0; c0 < CW; c0 += CK) {
+          float v[CK];
+          tmem_ld_n(tmem_at(tm, lane_base, CT_O + CW * (j & 1) + c0), v);
+          uint4 ou[CK / 8];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) ou[i] = Oo[((r >> 6) * (CW / 8) + (c0 >> 3) + i) * 64 + (r & 63)];
+          for (int i = 0; i < CK / 8; ++i) ou[i] = Oo[((r >> 6) * (CW / 8) + (c0 >> 3) + i) * 64 + (r & 63)];
           tmem_wait_ld();
           if (tok < a.N) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
+            for (int i = 0; i < CK / 8; ++i) {
               float of[8];
               unpack8(ou[i], of);
               uint32_t w[4];
@@ -966,7 +982,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_chain(ChainArgs a) {
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
-  if (warp == 0) tmem_dealloc(tm, 128);
+  if (warp == 0) tmem_dealloc(tm, TCOLS);
 }
 
 // cuTensorMapEncodeTiled from the driver, looked up once through the runtime
@@ -998,6 +1014,15 @@ bool encode_act_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, in
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+template <int CW>
+cudaError_t launch_chain(const ChainArgs& ca, dim3 grid, cudaStream_t s) {
+  cudaError_t e = cudaFuncSetAttribute(kda_tc_chain<CW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)ChainLayout<CW>::SMEM);
+  if (e != cudaSuccess) return e;
+  kda_tc_chain<CW><<<grid, 256, ChainLayout<CW>::SMEM, s>>>(ca);
+  return cudaGetLastError();
+}
+
 template <typename TIn>
 cudaError_t launch_all(const Dims& d, const void* q, const void* k, const void* v, const float* la,
                        const void* beta, const float* S0, void* o, float* SN, uint8_t* ws, uint32_t* status,
@@ -1009,8 +1034,7 @@ cudaError_t launch_all(const Dims& d, const void* q, const void* k, const void* 
   if ((e = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
   e = cudaFuncSetAttribute(kda_tc_prep<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize, PREP_SMEM);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(kda_tc_chain, cudaFuncAttributeMaxDynamicSharedMemorySize, CHAIN_SMEM);
-  if (e != cudaSuccess) return e;
+
   const int BH = d.B * d.H;
   const int n_units = BH * n_blocks;
   PrepArgs pa{q, k, v, la, beta, ws, d.N, d.H, BH, n_blocks, n_units, status};
@@ -1023,7 +1047,12 @@ cudaError_t launch_all(const Dims& d, const void* q, const void* k, const void* 
   kda_tc_prep<TIn><<<dim3((unsigned)min(n_units, n_sm)), 256, PREP_SMEM, s>>>(pa, mp);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   ChainArgs ca{ws, S0, SN, static_cast<__nv_bfloat16*>(o), d.N, d.H, n_blocks, status};
-  kda_tc_chain<<<dim3(NQ, d.H, d.B), 256, CHAIN_SMEM, s>>>(ca);
+  // the narrowest column split whose grid fits on the SMs (the serial pass is latency bound)
+  const int bh = d.B * d.H;
+  if (ChainLayout<16>::NQ * bh <= n_sm) e = launch_chain<16>(ca, dim3(ChainLayout<16>::NQ, d.H, d.B), s);
+  else if (ChainLayout<32>::NQ * bh <= n_sm) e = launch_chain<32>(ca, dim3(ChainLayout<32>::NQ, d.H, d.B), s);
+  else e = launch_chain<64>(ca, dim3(ChainLayout<64>::NQ, d.H, d.B), s);
+  if (e != cudaSuccess) return e;
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (launches) *launches += 2;
   return cudaSuccess;
