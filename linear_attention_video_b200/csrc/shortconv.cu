@@ -27,9 +27,9 @@ namespace {
 
 constexpr int kVisTaps = 27;
 constexpr int CG = 32;            // channels per CTA, one per lane
-constexpr int TH = 4;             // tile rows, one per warp row
+constexpr int TH = 4;             // tile rows, two per warp
 constexpr int NRUN = 4;           // runs per tile row
-constexpr int kThreads = 32 * TH * NRUN;
+constexpr int kThreads = 32 * (TH / 2) * NRUN;   // a warp: 32 channels x one run of two rows
 constexpr int PH = TH + 2;        // plane rows incl. halo
 
 struct ConvArgs {
@@ -147,38 +147,49 @@ struct VisPlane {
   static constexpr int BYTES = PH * PWr * CG * (int)sizeof(TIn);
 };
 
-// One plane f: FMAs into the three frames it feeds, then the completed frame out.
+// One plane f: FMAs into the three frames it feeds (two output rows each), then
+// the completed frame out.  Plane row ir feeds output row orow through tap
+// tb = ir - orow.
 template <typename TIn, typename TOut, int RUN, int PT>
 __device__ __forceinline__ void vis_plane_step(const TIn* pl, bool compute, const float (&wv)[kVisTaps],
-                                               float (&an)[RUN], float (&ac)[RUN], float (&ap)[RUN],
-                                               TOut* yo, bool emit, int nrun, int64_t C) {
+                                               float (&an)[2][RUN], float (&ac)[2][RUN], float (&ap)[2][RUN],
+                                               TOut* yo, int64_t row_stride, bool emit0, bool emit1, int nrun,
+                                               int64_t C) {
   constexpr int PWr = VisPlane<TIn, RUN>::PWr;
   if (compute) {
 #pragma unroll
-    for (int tb = 0; tb < 3; ++tb) {
-      const TIn* src = pl + tb * PWr * CG;
+    for (int ir = 0; ir < 4; ++ir) {
+      const TIn* src = pl + ir * PWr * CG;
       float in[RUN + 2];
 #pragma unroll
       for (int i = 0; i < RUN + 2; ++i) in[i] = widen1(src[i * CG]);
 #pragma unroll
-      for (int te = 0; te < 3; ++te) {
-        const float c0 = wv[tb * 3 + te], c1 = wv[9 + tb * 3 + te], c2 = wv[18 + tb * 3 + te];
+      for (int orow = 0; orow < 2; ++orow) {
+        const int tb = ir - orow;
+        if (tb < 0 || tb > 2) continue;
 #pragma unroll
-        for (int i = 0; i < RUN; ++i) {
-          an[i] = fmaf(c0, in[i + te], an[i]);
-          ac[i] = fmaf(c1, in[i + te], ac[i]);
-          ap[i] = fmaf(c2, in[i + te], ap[i]);
+        for (int te = 0; te < 3; ++te) {
+          const float c0 = wv[tb * 3 + te], c1 = wv[9 + tb * 3 + te], c2 = wv[18 + tb * 3 + te];
+#pragma unroll
+          for (int i = 0; i < RUN; ++i) {
+            an[orow][i] = fmaf(c0, in[i + te], an[orow][i]);
+            ac[orow][i] = fmaf(c1, in[i + te], ac[orow][i]);
+            ap[orow][i] = fmaf(c2, in[i + te], ap[orow][i]);
+          }
         }
       }
     }
   }
-  if (emit) {
 #pragma unroll
-    for (int i = 0; i < RUN; ++i)
-      if (i < nrun) store1<TOut>(yo + (int64_t)i * C, ap[i]);
+  for (int orow = 0; orow < 2; ++orow) {
+    if (orow == 0 ? emit0 : emit1) {
+#pragma unroll
+      for (int i = 0; i < RUN; ++i)
+        if (i < nrun) store1<TOut>(yo + orow * row_stride + (int64_t)i * C, ap[orow][i]);
+    }
+#pragma unroll
+    for (int i = 0; i < RUN; ++i) ap[orow][i] = 0.f;   // ap becomes the frame three ahead
   }
-#pragma unroll
-  for (int i = 0; i < RUN; ++i) ap[i] = 0.f;   // ap becomes the frame three ahead
 }
 
 template <typename TIn, typename TOut, int RUN, int PT>
@@ -201,10 +212,11 @@ __global__ void __launch_bounds__(kThreads, 1) vis_conv_kernel(ConvArgs a) {
   const TIn* x = static_cast<const TIn*>(xs) + ((int64_t)b * a.N + a.L) * C + cg0;
   TOut* y = static_cast<TOut*>(ys) + ((int64_t)b * a.N + a.L) * C + cg0;
 
-  const int row = warp % TH, run = warp / TH;
+  const int row = 2 * (warp % (TH / 2)), run = warp / (TH / 2);   // output rows row, row + 1
   const int w0 = run * RUN;
   const int nrun = max(0, min(RUN, TW - w0));
   const bool active = row < THh && nrun > 0;
+  const bool active1 = row + 1 < THh && nrun > 0;
 
   float wv[kVisTaps];
   {
@@ -242,9 +254,11 @@ __global__ void __launch_bounds__(kThreads, 1) vis_conv_kernel(ConvArgs a) {
     asm volatile("cp.async.commit_group;" ::: "memory");
   };
 
-  float s0[RUN], s1[RUN], s2[RUN];
+  float s0[2][RUN], s1[2][RUN], s2[2][RUN];
 #pragma unroll
-  for (int i = 0; i < RUN; ++i) { s0[i] = 0.f; s1[i] = 0.f; s2[i] = 0.f; }
+  for (int r = 0; r < 2; ++r)
+#pragma unroll
+    for (int i = 0; i < RUN; ++i) { s0[r][i] = 0.f; s1[r][i] = 0.f; s2[r][i] = 0.f; }
   for (int f = 0; f < NSLOT - 1; ++f) issue(f);
 
   // after plane f, frame f+PT-2 is complete; with PT = 1 one step past the last
@@ -252,14 +266,15 @@ __global__ void __launch_bounds__(kThreads, 1) vis_conv_kernel(ConvArgs a) {
   const int f_end = a.T + (PT == 1 ? 1 : 0);
   const TIn* pl_base = reinterpret_cast<const TIn*>(slots) + (row * PWr + w0) * CG + lane;
   TOut* y_base = y + ((int64_t)(th0 + row) * a.Wg + tw0 + w0) * C + lane;
-  auto step = [&](int f, float (&an)[RUN], float (&ac)[RUN], float (&ap)[RUN]) {
+  auto step = [&](int f, float (&an)[2][RUN], float (&ac)[2][RUN], float (&ap)[2][RUN]) {
     asm volatile("cp.async.wait_group %0;" :: "n"(NSLOT - 2) : "memory");
     __syncthreads();   // plane f in place everywhere; slot (f-1) % NSLOT no longer read
     issue(f + NSLOT - 1);
     const int t = f + PT - 2;
+    const bool tv = t >= 0 && t < a.T;
     vis_plane_step<TIn, TOut, RUN, PT>(pl_base + (f % NSLOT) * (VP::BYTES / (int)sizeof(TIn)),
                                        active && f < a.T, wv, an, ac, ap, y_base + (int64_t)t * HW * C,
-                                       active && t >= 0 && t < a.T, nrun, C);
+                                       (int64_t)a.Wg * C, active && tv, active1 && tv, nrun, C);
   };
   // roles rotate with f % 3: (frame f+PT, f+PT-1, f+PT-2) live in sets ((f+PT)%3, ...)
   for (int f = 0; f < f_end; f += 3) {
