@@ -349,6 +349,17 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
     const int bh_ = (int)blockIdx.x % a.BH;   // unit blockIdx.x: block blockIdx.x / BH, sub-chunk 0
     beta_next = load_beta(bh_ / a.H, bh_ % a.H, ((int)blockIdx.x / a.BH) * BLK + tid);
   }
+  // k, q, v of the sub-chunk starting at token t0_ -> KQ rows 0-63 / 64-127 and VV (thread 0)
+  auto issue_kqv = [&](int b_, int h_, int t0_) {
+    mbar_arrive_expect_tx(kqv_bar, 6 * 8192);
+#pragma unroll
+    for (int pnl = 0; pnl < 2; ++pnl) {
+      tma_load_4d(KQ + pnl * 16384, &mp.k, 64 * pnl, h_, t0_, b_, kqv_bar);
+      tma_load_4d(KQ + pnl * 16384 + 8192, &mp.q, 64 * pnl, h_, t0_, b_, kqv_bar);
+      tma_load_4d(VV + pnl * 8192, &mp.v, 64 * pnl, h_, t0_, b_, kqv_bar);
+    }
+  };
+  bool kqv_early = false;   // thread 0: the next sub-chunk's tiles are already on their way
   auto issue_la = [&](int u, int s_) {   // log alpha of sub-chunk s_ of unit u -> LAs (thread 0)
     const int blk_ = u / a.BH, bh_ = u - blk_ * a.BH;
     const int b_ = bh_ / a.H, h_ = bh_ - b_ * a.H;
@@ -387,13 +398,8 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
       // k -> KQ rows 0-63, q -> KQ rows 64-127, v -> VV: 128-byte-swizzled operand panels
       // written by TMA; rows past the sequence end read as zero
       if (tid == 0 && alive) {
-        mbar_arrive_expect_tx(kqv_bar, 6 * 8192);
-#pragma unroll
-        for (int pnl = 0; pnl < 2; ++pnl) {
-          tma_load_4d(KQ + pnl * 16384, &mp.k, 64 * pnl, h, (int)t0, b, kqv_bar);
-          tma_load_4d(KQ + pnl * 16384 + 8192, &mp.q, 64 * pnl, h, (int)t0, b, kqv_bar);
-          tma_load_4d(VV + pnl * 8192, &mp.v, 64 * pnl, h, (int)t0, b, kqv_bar);
-        }
+        if (!kqv_early) issue_kqv(b, h, (int)t0);   // else issued while the previous unit finished
+        kqv_early = false;
         kqv_inflight = true;
         // and the next sub-chunk's tiles into L2 meanwhile
         int nb_, nh_, nt0_;
@@ -679,6 +685,15 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
         if (tid == 0) bulk_wait_read();   // staged records read: their tiles may be rewritten
         alive = __syncthreads_and(wait_mma(bar, phase, a.status, alive));
         fence_after_sync();
+        if (tid == 0 && alive) {
+          // KQ and VV are free now: start the next unit's tiles before this unit's stores
+          int nb_, nh_, nt0_;
+          if (next_sub(unit, 1, nb_, nh_, nt0_)) {
+            issue_kqv(nb_, nh_, nt0_);
+            kqv_early = true;
+            kqv_inflight = true;
+          }
+        }
         // records staged in tiles the combine products no longer read:
         //   M -> M1 region, B -> B1 region, R_2 -> TT/PP region, O''_2 -> Xs region
         uint8_t* stR = TT;                               // [panel][64 rows][128 B], swizzled
