@@ -630,6 +630,12 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
         fence_before_sync();
         __syncthreads();
         if (tid == 0) {
+          // KQ (QG read above) and VV are free: sub-chunk 1's tiles first, then the stores
+          if (alive) {
+            issue_kqv(b, h, (int)t0 + SUB);
+            kqv_early = true;
+            kqv_inflight = true;
+          }
           bulk_s2g(gR, stR, 8192);
           bulk_s2g(gR + 16384, stR + 8192, 8192);
           bulk_s2g(gO, stO, 16384);
