@@ -818,7 +818,8 @@ __global__ void __launch_bounds__(256, 1) kda_tc_chain(ChainArgs a) {
   uint64_t* oDone = bars + 5;    // [2] R S_j complete (TMEM buffer j&1)
   uint64_t* sReady = bars + 7;   // [2] S_j image written (128 arrivals)
   uint64_t* sFree = bars + 9;    // [2] R S_j no longer reads S image j&1
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
+  uint64_t* oGo = bars + 11;     // [2] M S_j complete: R S_j may take the tensor pipe
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int tid = threadIdx.x, warp = tid >> 5;
   const int qtr = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -828,7 +829,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_chain(ChainArgs a) {
 
   if (warp == 0) { tmem_alloc(tmem_slot, TCOLS); tmem_relinquish(); }
   if (tid == 0) {
-    for (int i = 0; i < 11; ++i) mbar_init(&bars[i], (i == 7 || i == 8) ? 128 : 1);
+    for (int i = 0; i < 13; ++i) mbar_init(&bars[i], (i == 7 || i == 8) ? 128 : 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -851,8 +852,10 @@ __global__ void __launch_bounds__(256, 1) kda_tc_chain(ChainArgs a) {
       bulk_g2s(dst, rec + kMOff, 32768, &fullA[j & 1]);
       bulk_g2s(dst + 32768, rec + kBOff + qtr * CW_BYTES, CW_BYTES, &fullA[j & 1]);
     };
-    int issuedA = 0, seenA = 0, mma_pending = 0;
-    if (tid == 0)
+    // thread 32 refills ring A, so thread 0 goes from the barrier straight to the next product
+    const bool loaderA = tid == 32;
+    int issuedA = 0, mma_pending = 0;
+    if (loaderA)
       for (; issuedA < 2 && issuedA < nb; ++issuedA) load_A(issuedA);
     float S[CW];
 #pragma unroll
@@ -873,13 +876,13 @@ __global__ void __launch_bounds__(256, 1) kda_tc_chain(ChainArgs a) {
       if (tid == 0) {
         const bool landed = wait_or_abort(&fullA[j & 1], (uint32_t)(j >> 1) & 1u, abort_flag);
         if (landed) {
-          ++seenA;
           fence_after_sync();
           const uint64_t da = dA + (uint32_t)(j & 1) * (CH_SLOT >> 4);
           const uint64_t db = dS + (uint32_t)(j & 1) * (16384u >> 4);
 #pragma unroll
           for (int k16 = 0; k16 < 8; ++k16) mma_ss(tm, da + kstep(k16, 16384), db + mstep(k16), idesc, k16 > 0);
           mma_commit(msDone);
+          mma_commit(&oGo[j & 1]);
           mma_pending = 1;
         }
       }
@@ -913,16 +916,16 @@ __global__ void __launch_bounds__(256, 1) kda_tc_chain(ChainArgs a) {
       }
       fence_before_sync();
       ok = named_sync_and(1, 128, mine);   // ring A slot j consumed, S_{j+1} image written
-      if (ok && tid == 0 && issuedA < nb) { load_A(issuedA); ++issuedA; }
+      if (ok && loaderA && issuedA < nb) { load_A(issuedA); ++issuedA; }
     }
     if (ok && a.SN) {
 #pragma unroll
       for (int c = 0; c < CW; ++c) a.SN[(((int64_t)b * a.H + h) * D + row) * D + CW * qtr + c] = S[c];
     }
-    if (tid == 0) {
-      if (mma_pending) mbar_wait(msDone, (uint32_t)(j - 1) & 1u, 100000000ull);
-      for (int jj = seenA; jj < issuedA; ++jj) mbar_wait(&fullA[jj & 1], (uint32_t)(jj >> 1) & 1u, 100000000ull);
-    }
+    if (tid == 0 && mma_pending) mbar_wait(msDone, (uint32_t)(j - 1) & 1u, 100000000ull);
+    if (loaderA)   // each slot's latest load lands before the CTA exits (consumed ones return at once)
+      for (int jj = max(0, issuedA - 2); jj < issuedA; ++jj)
+        mbar_wait(&fullA[jj & 1], (uint32_t)(jj >> 1) & 1u, 100000000ull);
   } else {
     // ---------------- output group ----------------
     const int r = tid - 128;   // token row of the block = TMEM lane
@@ -935,8 +938,10 @@ __global__ void __launch_bounds__(256, 1) kda_tc_chain(ChainArgs a) {
       bulk_g2s(dst + 32768, rec + kOOff + qtr * (CW_BYTES / 2), CW_BYTES / 2, &fullB[j & 1]);
       bulk_g2s(dst + 32768 + CW_BYTES / 2, rec + kOOff + 16384 + qtr * (CW_BYTES / 2), CW_BYTES / 2, &fullB[j & 1]);
     };
-    int issuedB = 0, seenB = 0, o_pending = -1;
-    if (leader)
+    // thread 160 refills ring B, so the leader goes from the barrier straight to the next product
+    const bool loaderB = r == 32;
+    int issuedB = 0, o_pending = -1;
+    if (loaderB)
       for (; issuedB < 2 && issuedB < nb; ++issuedB) load_B(issuedB);
     const uint64_t dR = kdesc0(smem_u32(sm + CH_OFF_B));
     const int64_t tok_stride = (int64_t)a.H * D;
@@ -944,9 +949,10 @@ __global__ void __launch_bounds__(256, 1) kda_tc_chain(ChainArgs a) {
     for (int j = 0; j < nb && ok; ++j) {
       if (leader) {
         bool go = wait_or_abort(&sReady[j & 1], (uint32_t)(j >> 1) & 1u, abort_flag);
+        // issued once M S_j is done, so it does not share the tensor pipe with the serial product
+        go = go && wait_or_abort(&oGo[j & 1], (uint32_t)(j >> 1) & 1u, abort_flag);
         go = go && wait_or_abort(&fullB[j & 1], (uint32_t)(j >> 1) & 1u, abort_flag);
         if (go) {
-          ++seenB;
           fence_after_sync();
           const uint64_t da = dR + (uint32_t)(j & 1) * (CH_SLOT >> 4);
           const uint64_t db = dS + (uint32_t)(j & 1) * (16384u >> 4);
@@ -992,12 +998,12 @@ __global__ void __launch_bounds__(256, 1) kda_tc_chain(ChainArgs a) {
       }
       fence_before_sync();
       ok = named_sync_and(2, 128, mine);   // TMEM buffer j&1 read, ring B slot j consumed
-      if (ok && leader && issuedB < nb) { load_B(issuedB); ++issuedB; }
+      if (ok && loaderB && issuedB < nb) { load_B(issuedB); ++issuedB; }
     }
-    if (leader) {
-      if (o_pending >= 0) mbar_wait(&oDone[o_pending & 1], (uint32_t)(o_pending >> 1) & 1u, 100000000ull);
-      for (int jj = seenB; jj < issuedB; ++jj) mbar_wait(&fullB[jj & 1], (uint32_t)(jj >> 1) & 1u, 100000000ull);
-    }
+    if (leader && o_pending >= 0) mbar_wait(&oDone[o_pending & 1], (uint32_t)(o_pending >> 1) & 1u, 100000000ull);
+    if (loaderB)
+      for (int jj = max(0, issuedB - 2); jj < issuedB; ++jj)
+        mbar_wait(&fullB[jj & 1], (uint32_t)(jj >> 1) & 1u, 100000000ull);
   }
   if (tid == 0 && *abort_flag) set_status(a.status, KDA_ERR_TIMEOUT);
   fence_before_sync();
