@@ -139,6 +139,20 @@ def test_bf16_tensor_core_state_io(kda):
         assert rel_l2(s[:, h], ref_s[:, h]) < 5e-3
 
 
+@pytest.mark.parametrize("B,H", [(1, 40), (3, 12)])
+def test_bf16_tensor_core_many_heads(kda, B, H):
+    """More (batch item, head) pairs than fit 16- or 32-column chain CTAs on the SMs: the serial pass
+    runs with 64 value columns per CTA (40 pairs) or 32 (36 pairs); parity on a few heads."""
+    import dataclasses
+    w = dataclasses.replace(kda_synth.WORKLOADS[1], B=B, H=H, text_len=70, grid=(2, 11, 13))
+    inp = kda_synth.generate(w, 41 + H)
+    heads = [0, H // 2, H - 1]
+    ref, _ = oracle.forward(inp, w.text_len, w.grid, heads=heads)
+    o, _ = run_fwd(kda, w, inp)
+    for h in heads:
+        assert_parity(o[:, :, h], ref[:, :, h], "bf16", f"head {h}")
+
+
 def test_bf16_tensor_core_continuation(kda):
     """Two kda_chunk_fwd calls chained through the state equal one call (bf16, d = 128)."""
     w = kda_synth.WORKLOADS[1]
