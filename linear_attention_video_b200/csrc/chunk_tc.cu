@@ -168,6 +168,47 @@ struct PrepArgs {
   uint32_t* status;
 };
 
+// One 16x8 tile of C = A B with fp32 operands in shared memory (A row-major with
+// leading dimension lda, 16 rows; B row-major [k][n] with leading dimension ldb,
+// 8 columns), K = 8 * ksteps, on mma.sync m16n8k8 tf32 with the operands split
+// as x = hi + lo (both tf32): C = A_hi B_hi + A_hi B_lo + A_lo B_hi.  Fragment
+// coordinates: g = lane / 4, t = lane % 4; d[0..3] = C[g][2t], C[g][2t+1],
+// C[g+8][2t], C[g+8][2t+1].
+__device__ __forceinline__ uint32_t tf32_hi(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+  asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+               : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+               : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+__device__ __forceinline__ void mma_tile_3xtf32(const float* A, int lda, const float* B, int ldb, int ksteps, int g,
+                                                int t, float (&d)[4]) {
+  d[0] = d[1] = d[2] = d[3] = 0.f;
+#pragma unroll
+  for (int kk = 0; kk < ksteps; ++kk) {
+    const float af[4] = {A[g * lda + 8 * kk + t], A[(g + 8) * lda + 8 * kk + t], A[g * lda + 8 * kk + t + 4],
+                         A[(g + 8) * lda + 8 * kk + t + 4]};
+    const float bf[2] = {B[(8 * kk + t) * ldb + g], B[(8 * kk + t + 4) * ldb + g]};
+    uint32_t ah[4], al[4], bh[2], bl[2];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      ah[i] = tf32_hi(af[i]);
+      al[i] = tf32_hi(af[i] - __uint_as_float(ah[i]));
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      bh[i] = tf32_hi(bf[i]);
+      bl[i] = tf32_hi(bf[i] - __uint_as_float(bh[i]));
+    }
+    mma_tf32(d, al, bh);
+    mma_tf32(d, ah, bl);
+    mma_tf32(d, ah, bh);
+  }
+}
+
 // Blocked inverse X = (I + A)^{-1} of the unit lower-triangular 64x64 matrix,
 // A strictly lower in As.  16x16 diagonal blocks by forward substitution, then
 // two doubling merges (X_21 = -X_22 A_21 X_11) at 32 and 64.  Every loop has a
@@ -224,62 +265,27 @@ __device__ void unit_lower_inverse64(const float* As, float* Xs, float* Ys) {
   }
   __syncthreads();
   {
-    // 64-merge: X[32.., 0..31] = -X_22 (A_21 X_11), two 32x32x32 products.  Warp w
-    // owns output rows 4w..4w+3; lane = (tile column tc, K quarter g): a 4x4 tile
-    // over 8 of the 32 K indices, then the four quarters are summed across lanes.
-    const int tc = lane & 7, g = lane >> 3;
-    const int r0 = 4 * warp, c0 = 4 * tc;
-    float acc[4][4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-#pragma unroll
-    for (int it = 0; it < 8; ++it) {
-      const int m = 8 * g + it;
-      const float4 x = *reinterpret_cast<const float4*>(Xs + m * LDXS + c0);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float u = As[(32 + r0 + i) * LDA + m];
-        acc[i][0] += u * x.x; acc[i][1] += u * x.y; acc[i][2] += u * x.z; acc[i][3] += u * x.w;
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        acc[i][j] += __shfl_xor_sync(0xffffffffu, acc[i][j], 8);
-        acc[i][j] += __shfl_xor_sync(0xffffffffu, acc[i][j], 16);
-      }
-#pragma unroll
-    for (int i = 0; i < 4; ++i)   // lane quarter g writes row g of the tile
-      if (i == g) *reinterpret_cast<float4*>(Ys + (r0 + i) * LDY + c0) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+    // 64-merge: X[32.., 0..31] = -X_22 (A_21 X_11), two 32x32x32 products on the
+    // warp-level tensor cores (m16n8k8, tf32).  Each operand is split into a tf32
+    // high part and a tf32 remainder and the product is formed as hi*hi + hi*lo +
+    // lo*hi, which keeps it at about fp32 accuracy.  Warp w owns the 16x8 output
+    // tile (rows 16*(w>>2), columns 8*(w&3)).
+    const int g = lane >> 2, t4 = lane & 3;
+    const int tm = warp >> 2, tn = warp & 3;
+    float d[4];
+    // Y = A_21 X_11 -> Ys
+    mma_tile_3xtf32(As + (32 + 16 * tm) * LDA, LDA, Xs + 8 * tn, LDXS, 4, g, t4, d);
+    Ys[(16 * tm + g) * LDY + 8 * tn + 2 * t4] = d[0];
+    Ys[(16 * tm + g) * LDY + 8 * tn + 2 * t4 + 1] = d[1];
+    Ys[(16 * tm + g + 8) * LDY + 8 * tn + 2 * t4] = d[2];
+    Ys[(16 * tm + g + 8) * LDY + 8 * tn + 2 * t4 + 1] = d[3];
     __syncthreads();
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-#pragma unroll
-    for (int it = 0; it < 8; ++it) {
-      const int m = 8 * g + it;
-      const float4 y = *reinterpret_cast<const float4*>(Ys + m * LDY + c0);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float u = Xs[(32 + r0 + i) * LDXS + 32 + m];
-        acc[i][0] += u * y.x; acc[i][1] += u * y.y; acc[i][2] += u * y.z; acc[i][3] += u * y.w;
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        acc[i][j] += __shfl_xor_sync(0xffffffffu, acc[i][j], 8);
-        acc[i][j] += __shfl_xor_sync(0xffffffffu, acc[i][j], 16);
-      }
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-      if (i == g)
-        *reinterpret_cast<float4*>(Xs + (32 + r0 + i) * LDXS + c0) = make_float4(-acc[i][0], -acc[i][1], -acc[i][2], -acc[i][3]);
+    // X_21 = -X_22 Y
+    mma_tile_3xtf32(Xs + (32 + 16 * tm) * LDXS + 32, LDXS, Ys + 8 * tn, LDY, 4, g, t4, d);
+    Xs[(32 + 16 * tm + g) * LDXS + 8 * tn + 2 * t4] = -d[0];
+    Xs[(32 + 16 * tm + g) * LDXS + 8 * tn + 2 * t4 + 1] = -d[1];
+    Xs[(32 + 16 * tm + g + 8) * LDXS + 8 * tn + 2 * t4] = -d[2];
+    Xs[(32 + 16 * tm + g + 8) * LDXS + 8 * tn + 2 * t4 + 1] = -d[3];
     __syncthreads();
   }
 }
