@@ -133,13 +133,13 @@ def oracle_sample_workload(w, frames):
     return dataclasses.replace(w, grid=(min(frames, T), Hg, Wg), B=1)
 
 
-def run_oracle_sample(w, idx, frames, heads):
+def run_oracle_sample(w, idx, frames, heads, causal_t=False):
     import oracle
     ws = oracle_sample_workload(w, frames)
     inp = kda_synth.generate(ws, kda_synth.seed_for(idx))
     oracle.build()
     t0 = time.perf_counter()
-    oracle.forward(inp, ws.text_len, ws.grid, heads=list(range(heads)))
+    oracle.forward(inp, ws.text_len, ws.grid, heads=list(range(heads)), vis_causal_t=causal_t)
     dt = time.perf_counter() - t0
     # throughput in full-width tokens: the sample covers `heads` of H heads
     tokens_equiv = ws.N * heads / w.H
@@ -161,7 +161,7 @@ def reference_arm(args, w, idx, rank):
     heads = 1
     vals = []
     for i in range(args.warmup + args.steps):
-        v, dt, sample = run_oracle_sample(w, idx, frames, heads)
+        v, dt, sample = run_oracle_sample(w, idx, frames, heads, args.causal_t)
         if i >= args.warmup:
             vals.append(v)
     value = statistics.mean(vals)
@@ -170,6 +170,7 @@ def reference_arm(args, w, idx, rank):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * w.tokens / value,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "N": w.N, "H": w.H, "d": w.d, "text_len": w.text_len,
+                       "vis_conv_t": "causal" if args.causal_t else "centred",
                    "grid": list(w.grid), "chunk": w.chunk},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -207,7 +208,7 @@ def ours_arm(args, w, idx, rank, world, local_rank):
     B, N, H, d = inp["shape"]
     t = to_device(inp, dev)
     dt = t["q"].dtype
-    p = kda.problem(B, H, d, w.text_len, w.grid, chunk=w.chunk)
+    p = kda.problem(B, H, d, w.text_len, w.grid, chunk=w.chunk, vis_causal_t=args.causal_t)
     o = torch.empty(B, N, H, d, dtype=dt, device=dev)
     ws = kda.alloc_workspace(p, dt, dev)
 
@@ -299,7 +300,7 @@ def ours_arm(args, w, idx, rank, world, local_rank):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
         frames = sample_frames(w)
-        v, secs, sample = run_oracle_sample(w, idx, frames, args.cpu_heads)
+        v, secs, sample = run_oracle_sample(w, idx, frames, args.cpu_heads, args.causal_t)
         cpu = {"value": v, "unit": "tokens/s", "cores": os.cpu_count(), "kind": "oracle", "sample": sample,
                "seconds": secs}
 
@@ -309,6 +310,7 @@ def ours_arm(args, w, idx, rank, world, local_rank):
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f16" if w.dtype == "bf16" else "f32", "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "N": w.N, "H": w.H, "d": w.d, "text_len": w.text_len,
+                       "vis_conv_t": "causal" if args.causal_t else "centred",
                        "grid": list(w.grid), "chunk": w.chunk, "parallelism": f"replicas{world}",
                        "l2": "inputs larger than L2 (no flush)"},
             "roofline": roofline,
@@ -331,6 +333,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-heads", type=int, default=4, help="heads in the CPU-baseline sample")
+    ap.add_argument("--causal-t", action="store_true",
+                    help="temporal taps of the 3D conv cover frames t-2..t instead of t-1..t+1")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     idx, w = workload_by_name(args.workload)

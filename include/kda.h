@@ -26,6 +26,13 @@
  *    `chunk` tokens (the chunked KDA form named in section 复现评估); the result
  *    does not depend on the chunk length beyond rounding.
  *
+ *  - Batch items with fewer text tokens than text_len: place an item's text at
+ *    the end of the text span and fill the leading positions with zero tokens
+ *    (q = k = v = 0, log_alpha = 0, beta = 0).  A zero token leaves the state
+ *    unchanged and is what the causal text conv reads before the first token,
+ *    so the real tokens' outputs and the final state are exactly those of the
+ *    unpadded item; the padding positions' outputs are zero.
+ *
  * Layouts (row-major, contiguous):
  *    q, k, log_alpha : [B, N, H, dk]      v, o : [B, N, H, dv]      beta : [B, N, H]
  *    w_text : [3][H*dk][text_k]           w_vis : [3][H*dk][vis_kt*vis_kh*vis_kw]

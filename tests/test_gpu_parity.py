@@ -153,6 +153,30 @@ def test_bf16_tensor_core_many_heads(kda, B, H):
         assert_parity(o[:, :, h], ref[:, :, h], "bf16", f"head {h}")
 
 
+def test_bf16_left_padded_text_item(kda):
+    """An item with 20 fewer text tokens, padded with zero tokens at the front of its text
+    span, gives the unpadded item's outputs at its real tokens (tensor-core path)."""
+    import dataclasses
+    from tests.test_oracle_kda import _left_padded_pair
+    w, padded, single, pad = _left_padded_pair()
+    w = dataclasses.replace(w, H=padded["shape"][2])
+    ref, _ = oracle.forward(single, w.text_len - pad, w.grid)
+    o, _ = run_fwd(kda, w, padded)
+    for h in range(w.H):
+        assert_parity(o[1, pad:, h], ref[0, :, h], "bf16", f"head {h}")
+
+
+def test_bf16_causal_t_conv(kda):
+    """Temporal-causal 3D conv (taps on frames t-2..t) through the bf16 tensor-core path."""
+    import dataclasses
+    w = dataclasses.replace(kda_synth.WORKLOADS[1], H=4, text_len=30, grid=(4, 9, 13))
+    inp = kda_synth.generate(w, 77)
+    ref, _ = oracle.forward(inp, w.text_len, w.grid, vis_causal_t=True)
+    o, _ = run_fwd(kda, w, inp, vis_causal_t=True)
+    for h in range(w.H):
+        assert_parity(o[:, :, h], ref[:, :, h], "bf16", f"head {h}")
+
+
 def test_bf16_tensor_core_continuation(kda):
     """Two kda_chunk_fwd calls chained through the state equal one call (bf16, d = 128)."""
     w = kda_synth.WORKLOADS[1]

@@ -12,6 +12,7 @@ import os
 import numpy as np
 import pytest
 
+import kda_synth
 import oracle
 
 
@@ -231,3 +232,33 @@ def test_planted_mistakes_are_caught(mistake):
     o, _ = _scan1(q, k, v, la, beta)
     bad = _chunked_with(mistake, q, k, v, la, beta, 32)
     assert np.max(np.abs(bad - o)) > 1e-3
+
+
+def _left_padded_pair(pad=20):
+    """A two-item batch whose second item has `pad` fewer text tokens, stored as zero
+    tokens (q = k = v = 0, log alpha = 0, beta = 0) at the front of its text span, and
+    the same second item as a batch of one with the shorter text."""
+    import dataclasses
+    w = dataclasses.replace(kda_synth.WORKLOADS[1], B=2, H=2, text_len=60, grid=(2, 5, 7))
+    inp = kda_synth.generate(w, 5)
+    B, N, H, d = inp["shape"]
+    padded = {k: (v.copy() if isinstance(v, np.ndarray) else v) for k, v in inp.items()}
+    for name in ("q", "k", "v", "log_alpha"):
+        a = padded[name].reshape(B, N, H, d)
+        a[1, :pad] = 0
+    padded["beta"].reshape(B, N, H)[1, :pad] = 0
+    single = dict(inp, shape=(1, N - pad, H, d))
+    for name in ("q", "k", "v", "log_alpha"):
+        single[name] = np.ascontiguousarray(inp[name].reshape(B, N, H, d)[1, pad:]).reshape(-1)
+    single["beta"] = np.ascontiguousarray(inp["beta"].reshape(B, N, H)[1, pad:]).reshape(-1)
+    return w, padded, single, pad
+
+
+def test_left_padded_text_is_exact():
+    """Items with fewer text tokens: leading zero tokens leave the state and the causal text
+    conv untouched, so the real tokens' outputs equal those of the unpadded item."""
+    w, padded, single, pad = _left_padded_pair()
+    o_pad, s_pad = oracle.forward(padded, w.text_len, w.grid)
+    o_one, s_one = oracle.forward(single, w.text_len - pad, w.grid)
+    np.testing.assert_allclose(o_pad[1, pad:], o_one[0], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(s_pad[1], s_one[0], rtol=0, atol=1e-12)
