@@ -140,14 +140,16 @@ constexpr uint32_t OFF_PP = 73728;      // [64][64] fp16: P
 constexpr uint32_t OFF_M1 = 81920;      // [128][128] fp16: M_1 (MN-major operand image)
 constexpr uint32_t OFF_B1 = 114688;     // [128][128] fp16: B_1 (MN-major operand image)
 constexpr uint32_t OFF_AS = 147456;     // fp32 [64][LDA]: A (strictly lower, beta applied)
-constexpr uint32_t OFF_XS = 164096;     // fp32 [64][LDXS]: (I + A)^{-1}
-constexpr uint32_t OFF_YS = 181504;     // fp32 [32][36]: merge scratch / quarter totals
-constexpr uint32_t OFF_MISC = 186112;   // beta[64], egm, egl, ekt, gm, tot [128 each], barriers, tmem slot, flag
-constexpr uint32_t OFF_LA = 190464;     // fp32 [64 tokens][128]: log alpha of the current sub-chunk (TMA)
+constexpr uint32_t OFF_XS = 164864;     // fp32 [64][LDXS]: (I + A)^{-1}
+constexpr uint32_t OFF_YS = 182272;     // fp32 [32][36]: merge scratch / quarter totals
+constexpr uint32_t OFF_MISC = 186880;   // beta[64], egm, egl, ekt, gm, tot [128 each], barriers, tmem slot, flag
+constexpr uint32_t OFF_LA = 191232;     // fp32 [64 tokens][128]: log alpha of a sub-chunk (TMA), then x = g - g_m
 constexpr uint32_t PREP_SMEM = OFF_LA + 32768 + 1024;   // + alignment slack
 
-constexpr int LDA = 65;    // row stride of A: rows written by consecutive lanes hit consecutive banks
+constexpr int LDA = 68;    // row stride of A: rows 16-byte aligned (4-wide stores and loads)
 constexpr int LDXS = 68;   // row stride of X: rows 16-byte aligned for 4-wide loads
+static_assert(OFF_XS >= OFF_AS + 64 * LDA * 4 && OFF_YS >= OFF_XS + 64 * LDXS * 4, "prep shared-memory map");
+static_assert(OFF_LA % 128 == 0 && OFF_LA >= OFF_MISC + 4096, "prep shared-memory map");
 constexpr int LDY = 36;    // row stride of the merge scratch
 
 // TMEM columns
@@ -186,7 +188,9 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], 
 }
 __device__ __forceinline__ void mma_tile_3xtf32(const float* A, int lda, const float* B, int ldb, int ksteps, int g,
                                                 int t, float (&d)[4]) {
-  d[0] = d[1] = d[2] = d[3] = 0.f;
+  // four independent accumulation chains (even / odd k-steps, main / correction terms),
+  // summed at the end, so consecutive products do not wait on each other
+  float dh[2][4] = {}, dl[2][4] = {};
 #pragma unroll
   for (int kk = 0; kk < ksteps; ++kk) {
     const float af[4] = {A[g * lda + 8 * kk + t], A[(g + 8) * lda + 8 * kk + t], A[g * lda + 8 * kk + t + 4],
@@ -203,18 +207,24 @@ __device__ __forceinline__ void mma_tile_3xtf32(const float* A, int lda, const f
       bh[i] = tf32_hi(bf[i]);
       bl[i] = tf32_hi(bf[i] - __uint_as_float(bh[i]));
     }
-    mma_tf32(d, al, bh);
-    mma_tf32(d, ah, bl);
-    mma_tf32(d, ah, bh);
+    mma_tf32(dl[kk & 1], al, bh);
+    mma_tf32(dl[kk & 1], ah, bl);
+    mma_tf32(dh[kk & 1], ah, bh);
   }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) d[i] = (dl[0][i] + dl[1][i]) + (dh[0][i] + dh[1][i]);
 }
 
 // Blocked inverse X = (I + A)^{-1} of the unit lower-triangular 64x64 matrix,
-// A strictly lower in As.  16x16 diagonal blocks by forward substitution, then
+// A strictly lower in As, delivered as T = X Diag(beta) in fp16 (TT, one
+// swizzled K-major panel).  16x16 diagonal blocks by forward substitution, then
 // two doubling merges (X_21 = -X_22 A_21 X_11) at 32 and 64.  Every loop has a
 // fixed trip count; the zero blocks above the diagonal of X_11 and X_22 are
 // written here, the rest of the upper triangle is never read.
-__device__ void unit_lower_inverse64(const float* As, float* Xs, float* Ys) {
+// Step 1 (inverse_diag32) leaves the two diagonal 32x32 blocks of X in Xs and
+// writes every part of T but its lower-left block, so products over T's
+// columns 32-63 can start while step 2 (inverse_merge64) forms that block.
+__device__ void inverse_diag32(const float* As, float* Xs, float* Ys, uint8_t* TT, const float* beta) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (warp < 4 && lane < 16) {
     // diagonal block `warp`, column `lane`: right-looking substitution
@@ -222,10 +232,18 @@ __device__ void unit_lower_inverse64(const float* As, float* Xs, float* Ys) {
     float x[16];
 #pragma unroll
     for (int r = 0; r < 16; ++r) x[r] = r == l ? 1.f : 0.f;
+    // row r: x[r] -= A[r][m] x[m] for m = 0 .. r-1 in that order, A's row read 4 wide
 #pragma unroll
-    for (int m = 0; m < 15; ++m) {
+    for (int r = 1; r < 16; ++r) {
+      const float4* arow = reinterpret_cast<const float4*>(As + (o + r) * LDA + o);
 #pragma unroll
-      for (int r = m + 1; r < 16; ++r) x[r] -= As[(o + r) * LDA + o + m] * x[m];
+      for (int q = 0; q < (r + 3) / 4; ++q) {
+        const float4 a4 = arow[q];
+        const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (4 * q + u < r) x[r] -= av[u] * x[4 * q + u];
+      }
     }
 #pragma unroll
     for (int r = 0; r < 16; ++r) Xs[(o + r) * LDXS + o + l] = x[r];
@@ -264,6 +282,28 @@ __device__ void unit_lower_inverse64(const float* As, float* Xs, float* Ys) {
     Xs[(o + 17 + i0) * LDXS + o + j] = -z1;
   }
   __syncthreads();
+  // T = X Diag(beta) for rows 0-31 (X_11, then zeros) and the X_22 block of rows 32-63
+  for (int e = tid; e < 384; e += 256) {
+    const int r = e < 256 ? e >> 3 : 32 + ((e - 256) >> 2);
+    const int c0 = e < 256 ? (e & 7) * 8 : 32 + ((e - 256) & 3) * 8;
+    float v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int cj = c0 + j;
+      v[j] = (cj <= r && (r < 32) == (cj < 32)) ? Xs[r * LDXS + cj] * beta[cj] : 0.f;
+    }
+    *reinterpret_cast<uint4*>(TT + swz_off(r, c0)) = pack8(v);
+  }
+  fence_proxy_async();
+}
+
+// Step 2: X_21 = -X_22 (A_21 X_11) -> T rows 32-63, columns 0-31.  `between`
+// runs on every thread after the barrier that follows the first product; the
+// caller's next barrier publishes the block.
+template <typename F>
+__device__ __forceinline__ void inverse_merge64(const float* As, const float* Xs, float* Ys, uint8_t* TT,
+                                                const float* beta, F&& between) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   {
     // 64-merge: X[32.., 0..31] = -X_22 (A_21 X_11), two 32x32x32 products on the
     // warp-level tensor cores (m16n8k8, tf32).  Each operand is split into a tf32
@@ -280,13 +320,14 @@ __device__ void unit_lower_inverse64(const float* As, float* Xs, float* Ys) {
     Ys[(16 * tm + g + 8) * LDY + 8 * tn + 2 * t4] = d[2];
     Ys[(16 * tm + g + 8) * LDY + 8 * tn + 2 * t4 + 1] = d[3];
     __syncthreads();
-    // X_21 = -X_22 Y
+    between();
+    // X_21 = -X_22 Y, times beta of its column, into T
     mma_tile_3xtf32(Xs + (32 + 16 * tm) * LDXS + 32, LDXS, Ys + 8 * tn, LDY, 4, g, t4, d);
-    Xs[(32 + 16 * tm + g) * LDXS + 8 * tn + 2 * t4] = -d[0];
-    Xs[(32 + 16 * tm + g) * LDXS + 8 * tn + 2 * t4 + 1] = -d[1];
-    Xs[(32 + 16 * tm + g + 8) * LDXS + 8 * tn + 2 * t4] = -d[2];
-    Xs[(32 + 16 * tm + g + 8) * LDXS + 8 * tn + 2 * t4 + 1] = -d[3];
-    __syncthreads();
+    const int r0 = 32 + 16 * tm + g, c = 8 * tn + 2 * t4;
+    const float b0 = beta[c], b1 = beta[c + 1];
+    st_h2(TT + swz_off(r0, c), -d[0] * b0, -d[1] * b1);
+    st_h2(TT + swz_off(r0 + 8, c), -d[2] * b0, -d[3] * b1);
+    fence_proxy_async();
   }
 }
 
@@ -313,7 +354,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
   uint64_t* bar = reinterpret_cast<uint64_t*>(tot_s + 128);    // [0] MMA, [1] k/q/v tiles, [2] log alpha
   uint64_t* kqv_bar = bar + 1;
   uint64_t* la_bar = bar + 2;
-  const float* LAs = reinterpret_cast<const float*>(sm + OFF_LA);
+  float* LAx = reinterpret_cast<float*>(sm + OFF_LA);   // log alpha, turned in place into x = g - g_m
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 4);
   int* range_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
@@ -376,6 +417,52 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
     issue_la(blockIdx.x, 0);
     la_inflight = true;
   }
+  // Decay exponents of a sub-chunk, in place in LAx (zero log alpha past the sequence end).
+  // Thread: channels 2 dp, 2 dp + 1 and tokens 16 dq .. 16 dq + 15.  Part 1 forms the running
+  // sums within the thread's 16 tokens and publishes their totals; part 2 (after a barrier)
+  // turns them into x = g - g_m, g_m = g_31, and records g_m and the decay over tokens 32..63.
+  const int dp = (tid & 31) + 32 * ((tid >> 5) & 1), dq = tid >> 6, dc = 2 * dp;
+  float2* qtot = reinterpret_cast<float2*>(Ys);   // [4][64] quarter totals
+  auto decay_part1 = [&](bool ok) -> bool {
+    ok = wait_tma(la_bar, la_phase, a.status, ok);
+    if (tid == 0) la_inflight = !ok && la_inflight;
+    if (!ok) return false;
+    float2 gl[16];
+#pragma unroll
+    for (int t = 0; t < 16; ++t) gl[t] = *reinterpret_cast<const float2*>(LAx + (16 * dq + t) * D + dc);
+#pragma unroll
+    for (int t = 1; t < 16; ++t) { gl[t].x += gl[t - 1].x; gl[t].y += gl[t - 1].y; }
+#pragma unroll
+    for (int t = 0; t < 16; ++t) *reinterpret_cast<float2*>(LAx + (16 * dq + t) * D + dc) = gl[t];
+    qtot[dq * 64 + dp] = gl[15];
+    return true;
+  };
+  auto decay_part2 = [&]() {
+    float2 pre = make_float2(0.f, 0.f), gmv = make_float2(0.f, 0.f), tot = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 v = qtot[j * 64 + dp];
+      if (j < dq) { pre.x += v.x; pre.y += v.y; }
+      if (j < 2) { gmv.x += v.x; gmv.y += v.y; } else { tot.x += v.x; tot.y += v.y; }
+    }
+    if (dq == 0) {
+      gm_s[dc] = gmv.x; gm_s[dc + 1] = gmv.y;       // g_m: decay through token 31
+      tot_s[dc] = tot.x; tot_s[dc + 1] = tot.y;     // decay over tokens 32..63
+    }
+    float2 x0 = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int t = 0; t < 16; ++t) {
+      float2* p = reinterpret_cast<float2*>(LAx + (16 * dq + t) * D + dc);
+      const float2 g = *p;
+      const float2 x = make_float2(pre.x + g.x - gmv.x, pre.y + g.y - gmv.y);
+      if (t == 0) x0 = x;
+      *p = x;
+    }
+    // x is largest at token 0 and smallest (-tot) at token 63
+    if (dq == 0 && (x0.x > kRange || x0.y > kRange)) *range_flag = 1;
+    if (dq == 3 && (-tot.x > kRange || -tot.y > kRange)) *range_flag = 1;
+  };
+  bool x_ready = false;   // the current sub-chunk's exponents were formed during the previous one
 
   // operand descriptors of the fixed tiles (stepped along K by kstep / mstep)
   const uint64_t dKQk = kdesc0(smem_u32(KQ)), dKQm = mdesc0(smem_u32(KQ), 16384);
@@ -407,7 +494,9 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
         if (!kqv_early) issue_kqv(b, h, (int)t0);   // else issued while the previous unit finished
         kqv_early = false;
         kqv_inflight = true;
-        // and the next sub-chunk's tiles into L2 meanwhile
+      }
+      if (tid == 128 && alive) {
+        // the next sub-chunk's tiles and log alpha into L2 meanwhile
         int nb_, nh_, nt0_;
         if (next_sub(unit, s, nb_, nh_, nt0_)) {
 #pragma unroll
@@ -416,6 +505,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
             tma_prefetch_4d(&mp.q, 64 * pnl, nh_, nt0_, nb_);
             tma_prefetch_4d(&mp.v, 64 * pnl, nh_, nt0_, nb_);
           }
+          tma_prefetch_4d(&mp.la, 0, nh_, nt0_, nb_);
         }
       }
       if (tid < SUB) {
@@ -424,46 +514,24 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
         int nb_, nh_, nt0_;
         beta_next = next_sub(unit, s, nb_, nh_, nt0_) ? load_beta(nb_, nh_, nt0_ + tid) : 0.f;
       }
-      // thread: channels 2cp, 2cp+1 and tokens 16*qt .. 16*qt+15 of the sub-chunk; log alpha
-      // arrived in LAs during the previous sub-chunk (zero past the sequence end)
-      const int cp = (tid & 31) + 32 * ((tid >> 5) & 1);
-      const int qt = tid >> 6;
-      const int c = 2 * cp;
-      bool ok_in = wait_tma(la_bar, la_phase, a.status, alive);
-      float2 gl[16];
-#pragma unroll
-      for (int t = 0; t < 16; ++t) gl[t] = *reinterpret_cast<const float2*>(LAs + (16 * qt + t) * D + c);
-#pragma unroll
-      for (int t = 1; t < 16; ++t) { gl[t].x += gl[t - 1].x; gl[t].y += gl[t - 1].y; }
-      float2* qtot = reinterpret_cast<float2*>(Ys);      // [4][64] quarter totals
-      qtot[qt * 64 + cp] = gl[15];
+      bool ok_in = alive;
+      if (!x_ready) {
+        // first sub-chunk of this CTA: its decay exponents are formed here (later ones are
+        // formed while the previous sub-chunk waits for its products)
+        ok_in = decay_part1(ok_in);
+        fence_before_sync();
+        __syncthreads();
+        decay_part2();
+      }
+      x_ready = false;
       ok_in = wait_tma(kqv_bar, kqv_phase, a.status, ok_in);
       alive = __syncthreads_and(ok_in);
-      if (tid == 0 && alive) {
-        la_inflight = false;
-        kqv_inflight = false;
-        // LAs consumed: fetch the log alpha of this CTA's next sub-chunk
-        const int nunit = s == 0 ? unit : unit + (int)gridDim.x;
-        if (alive && nunit < a.n_units) {
-          issue_la(nunit, s ^ 1);
-          la_inflight = true;
-        }
-      }
-      float2 pre = make_float2(0.f, 0.f), gmv = make_float2(0.f, 0.f), tot = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float2 v = qtot[j * 64 + cp];
-        if (j < qt) { pre.x += v.x; pre.y += v.y; }
-        if (j < 2) { gmv.x += v.x; gmv.y += v.y; } else { tot.x += v.x; tot.y += v.y; }
-      }
-      if (qt == 0) {
-        gm_s[c] = gmv.x; gm_s[c + 1] = gmv.y;       // g_m: decay through token 31
-        tot_s[c] = tot.x; tot_s[c + 1] = tot.y;     // decay over tokens 32..63
-      }
-      // exponent x = g - g_m; its extremes sit at token 0 and token 63
-      if (qt == 0 && (pre.x + gl[0].x - gmv.x > kRange || pre.y + gl[0].y - gmv.y > kRange)) *range_flag = 1;
-      if (qt == 3 && (-tot.x > kRange || -tot.y > kRange)) *range_flag = 1;
+      if (tid == 0) kqv_inflight = false;
       {
+        // thread: channels 2cp, 2cp+1 and tokens 16*qt .. 16*qt+15; X holds x = g - g_m
+        const int cp = (tid & 31) + 32 * ((tid >> 5) & 1);
+        const int qt = tid >> 6;
+        const int c = 2 * cp;
         const int pnl = c >> 6, cc = c & 63;
         uint8_t* kq = KQ + pnl * 16384;
         uint8_t* kn = KN + pnl * 8192;
@@ -474,8 +542,8 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
           const uint32_t off = swz_off(tok, cc), offq = swz_off(64 + tok, cc);
           const float2 kv = ld_act2(kq + off, (TIn*)nullptr);
           const float2 qv = ld_act2(kq + offq, (TIn*)nullptr);
-          const float x0 = pre.x + gl[t].x - gmv.x, x1 = pre.y + gl[t].y - gmv.y;
-          const float ep0 = __expf(x0), ep1 = __expf(x1), en0 = __expf(-x0), en1 = __expf(-x1);
+          const float2 x = *reinterpret_cast<const float2*>(LAx + tok * D + c);
+          const float ep0 = __expf(x.x), ep1 = __expf(x.y), en0 = __expf(-x.x), en1 = __expf(-x.y);
           st_h2(kq + off, kv.x * ep0, kv.y * ep1);
           st_h2(kq + offq, qv.x * ep0, qv.y * ep1);
           st_h2(kn + off, kv.x * en0, kv.y * en1);
@@ -492,6 +560,14 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
         egm[tid] = __expf(gmx);
         egl[tid] = __expf(gmx + totx);
         ekt[tid] = __expf(totx);
+      }
+      if (tid == 0 && alive) {
+        // X consumed: fetch the log alpha of this CTA's next sub-chunk
+        const int nunit = s == 0 ? unit : unit + (int)gridDim.x;
+        if (nunit < a.n_units) {
+          issue_la(nunit, s ^ 1);
+          la_inflight = true;
+        }
       }
       // ---------------- A, P = [KG; QG] KN^T ----------------
       if (tid == 0 && alive) {
@@ -514,7 +590,10 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
         if (sub < 2) {
           const float bt = beta_s[row];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) As[row * LDA + col0 + j] = (col0 + j < row) ? bt * v[j] : 0.f;
+          for (int j = 0; j < 32; j += 4)
+            *reinterpret_cast<float4*>(As + row * LDA + col0 + j) =
+                make_float4(col0 + j < row ? bt * v[j] : 0.f, col0 + j + 1 < row ? bt * v[j + 1] : 0.f,
+                            col0 + j + 2 < row ? bt * v[j + 2] : 0.f, col0 + j + 3 < row ? bt * v[j + 3] : 0.f);
         } else {
           const int r = row - 64;
 #pragma unroll
@@ -524,25 +603,28 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
       }
       fence_before_sync();
       __syncthreads();
-      unit_lower_inverse64(As, Xs, Ys);
-      // T = X Diag(beta) -> TT (fp16, [r][i]); X is lower triangular
-      for (int e = tid; e < SUB * 8; e += 256) {
-        const int r = e >> 3, c0 = (e & 7) * 8;
-        float v[8];
+      // T = (I + A)^{-1} Diag(beta) -> TT; W' = T KG, U~ = T V over T's columns 32-63 first,
+      // issued as soon as they are written, then over columns 0-31
+      inverse_diag32(As, Xs, Ys, TT, beta_s);
+      inverse_merge64(As, Xs, Ys, TT, beta_s, [&]() {
+        if (tid == 0 && alive) {
+          fence_after_sync();
 #pragma unroll
-        for (int j = 0; j < 8; ++j) v[j] = c0 + j <= r ? Xs[r * LDXS + c0 + j] * beta_s[c0 + j] : 0.f;
-        *reinterpret_cast<uint4*>(TT + swz_off(r, c0)) = pack8(v);
-      }
-      fence_proxy_async();
+          for (int k16 = 2; k16 < 4; ++k16) {
+            const uint64_t ad = dTTk + kstep(k16, 8192);
+            mma_ss(tmem_at(tm, 0, C_W), ad, dKQm + mstep(k16), id_64x128_kmn, k16 > 2);
+            mma_ss(tmem_at(tm, 0, C_U), ad, dVVm + mstep(k16), id_64x128_kmn, k16 > 2);
+          }
+        }
+      });
       __syncthreads();
-      // ---------------- W' = T KG, U~ = T V ----------------
       if (tid == 0 && alive) {
         fence_after_sync();
 #pragma unroll
-        for (int k16 = 0; k16 < 4; ++k16) {
+        for (int k16 = 0; k16 < 2; ++k16) {
           const uint64_t ad = dTTk + kstep(k16, 8192);
-          mma_ss(tmem_at(tm, 0, C_W), ad, dKQm + mstep(k16), id_64x128_kmn, k16 > 0);
-          mma_ss(tmem_at(tm, 0, C_U), ad, dVVm + mstep(k16), id_64x128_kmn, k16 > 0);
+          mma_ss(tmem_at(tm, 0, C_W), ad, dKQm + mstep(k16), id_64x128_kmn, 1);
+          mma_ss(tmem_at(tm, 0, C_U), ad, dVVm + mstep(k16), id_64x128_kmn, 1);
         }
         mma_commit(bar);
       }
@@ -556,9 +638,13 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
         for (int j = 0; j < 8; ++j) f[j] *= ekt[ch + j];
         *p = pack8(f);
       }
+      // meanwhile the next sub-chunk's decay exponents, part 1 (its log alpha has landed by now)
+      const bool have_next = (s == 0 ? unit : unit + (int)gridDim.x) < a.n_units;
+      bool ok_next = true;
+      if (have_next) ok_next = decay_part1(alive);
       fence_proxy_async();
       if (tid == 0) bulk_wait_read();   // staged records read: their tiles may be rewritten
-      alive = __syncthreads_and(wait_mma(bar, phase, a.status, alive));
+      alive = __syncthreads_and(wait_mma(bar, phase, a.status, alive) && ok_next);
       fence_after_sync();
       // W' -> KQ rows 0-63, U~ -> VV (fp16); M=64 accumulator layout: rows 16*sub + lane (lane < 16)
       {
@@ -593,6 +679,10 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
           mma_ss(tmem_at(tm, 0, C_PU), pd, ud, id_64x128_kmn, k16 > 0);
         }
         mma_commit(bar);
+      }
+      if (have_next && alive) {
+        decay_part2();   // part 2 of the next sub-chunk's exponents
+        x_ready = true;
       }
       if (tid == 0) bulk_wait_read();   // staged records read: their tiles may be rewritten
       alive = __syncthreads_and(wait_mma(bar, phase, a.status, alive));

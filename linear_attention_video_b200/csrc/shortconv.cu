@@ -96,33 +96,6 @@ template <> __device__ __forceinline__ void store1<__nv_bfloat16>(__nv_bfloat16*
 template <> __device__ __forceinline__ void store1<__half>(__half* p, float a) { *p = __float2half_rn(a); }
 template <> __device__ __forceinline__ void store1<float>(float* p, float a) { *p = a; }
 
-// raw 16-byte chunk holding 8 channels (bf16: one uint4; fp32: two float4 -> handled separately)
-template <typename T> struct Chunk { uint4 a; };
-template <> struct Chunk<float> { float4 a, b; };
-
-template <typename T> __device__ __forceinline__ void chunk_load(const T* p, Chunk<T>& c) {
-  c.a = __ldg(reinterpret_cast<const uint4*>(p));
-}
-template <> __device__ __forceinline__ void chunk_load<float>(const float* p, Chunk<float>& c) {
-  c.a = __ldg(reinterpret_cast<const float4*>(p));
-  c.b = __ldg(reinterpret_cast<const float4*>(p) + 1);
-}
-template <typename T> __device__ __forceinline__ void chunk_zero(Chunk<T>& c) { c.a = make_uint4(0, 0, 0, 0); }
-template <> __device__ __forceinline__ void chunk_zero<float>(Chunk<float>& c) {
-  c.a = make_float4(0.f, 0.f, 0.f, 0.f);
-  c.b = c.a;
-}
-template <typename T> __device__ __forceinline__ void chunk_store(float* dst, const Chunk<T>& c) {
-  float v[8];
-  Act<__nv_bfloat16>::widen8(c.a, v);
-  reinterpret_cast<float4*>(dst)[0] = make_float4(v[0], v[1], v[2], v[3]);
-  reinterpret_cast<float4*>(dst)[1] = make_float4(v[4], v[5], v[6], v[7]);
-}
-template <> __device__ __forceinline__ void chunk_store<float>(float* dst, const Chunk<float>& c) {
-  reinterpret_cast<float4*>(dst)[0] = c.a;
-  reinterpret_cast<float4*>(dst)[1] = c.b;
-}
-
 // ---- visual kernel -----------------------------------------------------------
 // RUN: pixels per thread along a row (compile-time, so the FMA loop carries no
 // predicates); a tile is NRUN runs wide.  Columns past the grid edge read the
