@@ -11,6 +11,12 @@ HBM.  Default workload: the 30-second 480x832 video (512 text tokens + a
 Prints one JSON line (rank 0).  Under torchrun every rank runs its own copy of
 the workload (weak scaling, no collective on the data path); the value is the
 tokens of all ranks divided by the slowest rank's device time.
+
+  python bench.py --shard seq [--seq-ranks R]        (torchrun for N > 1)
+
+times the sequence-sharded pass instead: the workload's frames split over the
+ranks (conv halo exchange, per-rank state maps composed across ranks), total
+work fixed (strong scaling).  On one GPU, --seq-ranks R runs R ranks as threads.
 """
 from __future__ import annotations
 
@@ -193,6 +199,106 @@ def time_calls(fn, steps, stream):
     return ev0.elapsed_time(ev1) / steps
 
 
+def reduce_max(value: float, device, world: int) -> float:
+    """The largest of the ranks' values (every rank gets it); the identity on one rank."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def seq_arm(args, w, idx, rank, world, local_rank):
+    """Sequence-sharded pass: rank r owns an even share of the frames (rank 0 the text too)."""
+    import torch
+    import linear_attention_video_b200 as kda
+    from linear_attention_video_b200 import seqshard
+    from tests._util import to_device
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.current_stream(dev)
+    ranks = world if world > 1 else max(1, args.seq_ranks)
+    segs = seqshard.partition(w.text_len, w.grid, ranks, args.causal_t)
+    mine = [rank] if world > 1 else list(range(ranks))
+    inp = kda_synth.generate(w, kda_synth.seed_for(idx))
+    B, N, H, d = inp["shape"]
+    full = to_device(inp, "cpu")
+    host = {}
+    for r in mine:
+        sg = segs[r]
+        host[r] = {n: full[n][:, sg.t0:sg.t1].contiguous().pin_memory() for n in ("q", "k", "v", "log_alpha", "beta")}
+    weights = {n: full[n].to(dev) for n in ("w_text", "w_vis")}
+    dev_in = {r: {n: x.to(dev) for n, x in host[r].items()} for r in mine}
+    backends = {r: seqshard.GpuBackend(B, H, d, w.chunk, args.causal_t) for r in mine}
+    outs = {}
+
+    def rank_step(comm, src):
+        r = comm.rank
+        x = src[r]
+        outs[r] = seqshard.seqshard_fwd(backends[r], comm, (x["q"], x["k"], x["v"]), x["log_alpha"], x["beta"],
+                                        weights["w_text"], weights["w_vis"], w.text_len, w.grid)
+
+    if world > 1:
+        comm = seqshard.DistComm()
+        step = lambda src=dev_in: rank_step(comm, src)   # noqa: E731
+    else:
+        group = seqshard.LocalGroup(ranks)
+        step = lambda src=dev_in: group.run(lambda c: rank_step(c, src))   # noqa: E731
+
+    with ClockSampler(local_rank) as clk:
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        torch.cuda.synchronize()
+        ms = time_calls(step, args.steps, stream)
+    clocks = clk.summary()
+    ms = reduce_max(ms, dev, world)
+    value = w.tokens / (ms * 1e-3)
+
+    # end to end: this rank's inputs from pinned host memory, the pass, its outputs back
+    e2e = None
+    if not args.no_e2e:
+        o_host = {r: torch.empty((B, segs[r].t1 - segs[r].t0, H, d), dtype=dev_in[r]["q"].dtype).pin_memory()
+                  for r in mine}
+        h2d = sum(x.numel() * x.element_size() for r in mine for x in host[r].values())
+        d2h = sum(x.numel() * x.element_size() for x in o_host.values())
+
+        def e2e_step():
+            for r in mine:
+                for n in host[r]:
+                    dev_in[r][n].copy_(host[r][n], non_blocking=True)
+            step()
+            for r in mine:
+                o_host[r].copy_(outs[r][0], non_blocking=True)
+        e2e_step()
+        ms_e2e = reduce_max(time_calls(e2e_step, max(3, min(args.steps, 10)), stream), dev, world)
+        e2e = {"value": w.tokens / (ms_e2e * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h}
+    # launches per step on this process: conv (text + visual) and three scans per rank
+    launches = 0
+    for r in mine:
+        sg = segs[r]
+        launches += (1 if r == 0 and w.text_len else 0) + 1 + 2 + 1 + 1
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "strong",
+            "vs_baseline": None, "dtype": "f16" if w.dtype == "bf16" else "f32", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "N": w.N, "H": w.H, "d": w.d, "text_len": w.text_len,
+                       "vis_conv_t": "causal" if args.causal_t else "centred", "grid": list(w.grid),
+                       "chunk": w.chunk, "parallelism": f"sequence{ranks}" + ("" if world > 1 else " (threads on 1 GPU)"),
+                       "l2": "inputs larger than L2 (no flush)"},
+            "e2e": e2e, "gpu_launches": launches * args.steps, "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+
+
 def ours_arm(args, w, idx, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -230,10 +336,7 @@ def ours_arm(args, w, idx, rank, world, local_rank):
         torch.cuda.synchronize()
         ms = time_calls(step, args.steps, stream)
     clocks = clk.summary()
-    ms_t = torch.tensor([ms], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-    ms = float(ms_t.item())
+    ms = reduce_max(ms, dev, world)
     tokens_all = w.tokens * world
     value = tokens_all / (ms * 1e-3)
 
@@ -290,10 +393,8 @@ def ours_arm(args, w, idx, rank, world, local_rank):
         e2e_step()
         e2e_steps = max(3, min(args.steps, 10))
         ms_e2e = time_calls(e2e_step, e2e_steps, stream)
-        e2e_t = torch.tensor([ms_e2e], device=dev, dtype=torch.float64)
-        if world > 1:
-            dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
-        e2e = {"value": tokens_all / (float(e2e_t.item()) * 1e-3), "unit": "tokens/s",
+        ms_e2e = reduce_max(ms_e2e, dev, world)
+        e2e = {"value": tokens_all / (ms_e2e * 1e-3), "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
         del host, dev_in
 
@@ -333,6 +434,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-heads", type=int, default=4, help="heads in the CPU-baseline sample")
+    ap.add_argument("--shard", default="replicas", choices=["replicas", "seq"],
+                    help="replicas: every rank runs the whole workload; seq: the frames are split over the ranks")
+    ap.add_argument("--seq-ranks", type=int, default=2, help="--shard seq on one GPU: ranks run as threads")
     ap.add_argument("--causal-t", action="store_true",
                     help="temporal taps of the 3D conv cover frames t-2..t instead of t-1..t+1")
     args = ap.parse_args()
@@ -351,7 +455,7 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     try:
-        ours_arm(args, w, idx, rank, world, local_rank)
+        (seq_arm if args.shard == "seq" else ours_arm)(args, w, idx, rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist

@@ -82,6 +82,21 @@ typedef enum { KDA_DT_BF16 = 0, KDA_DT_F32 = 1 } kda_dtype;
 
 /* Temporal taps of the 3D conv cover frames t-kt+1..t instead of being centred. */
 #define KDA_FLAG_VIS_CAUSAL_T 1u
+/* kda_chunk_fwd only (the other entry points reject it): the workspace still holds the
+ * intermediate block records that the previous kda_chunk_fwd call on it computed from the
+ * same q, k, v, log_alpha, beta, problem and dtype, on the same stream, with no other call on
+ * this workspace in between.  Only the serial state pass runs again, from the new
+ * initial_state: the map from initial to final state is affine, so a caller can evaluate it
+ * at several initial states (sequence sharding) for the price of one full pass.  Paths that
+ * keep no records (fp32, d = 64) recompute everything; the result is the same. */
+#define KDA_FLAG_REUSE_RECORDS 2u
+/* bf16 problems with d = 128 only (otherwise KDA_ERR_UNSUPPORTED): the convolved q', k', v'
+ * are fp16 instead of bf16 -- the outputs of kda_shortconv_fwd and the q, k, v inputs of
+ * kda_chunk_fwd / kda_chunk_fwd_noalloc.  fp16 is the operand type of the tensor-core scan
+ * and keeps three more mantissa bits than bf16 (kda_fwd keeps its intermediates in fp16
+ * anyway and rejects the flag); callers that split the pass into the two calls use it to
+ * get kda_fwd's accuracy.  beta and o stay bf16. */
+#define KDA_FLAG_QKV_F16 4u
 
 typedef struct {
   int32_t B, H, dk, dv;             /* batch items, heads, key and value head dims */

@@ -28,6 +28,8 @@ KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_MISALIGNED = 0, 1, 2, 
 KDA_ERR_WORKSPACE, KDA_ERR_CUDA, KDA_ERR_TIMEOUT, KDA_ERR_DEVICE_ASSERT, KDA_ERR_RANGE = 4, 5, 6, 7, 8
 KDA_DT_BF16, KDA_DT_F32 = 0, 1
 KDA_FLAG_VIS_CAUSAL_T = 1
+KDA_FLAG_REUSE_RECORDS = 2
+KDA_FLAG_QKV_F16 = 4
 
 EXPORTS = ("kda_tokens", "kda_workspace_bytes", "kda_shortconv_fwd", "kda_chunk_fwd", "kda_fwd",
            "kda_chunk_fwd_noalloc", "kda_read_status", "kda_status_str", "kda_last_launch_count")
@@ -70,10 +72,12 @@ class KdaError(RuntimeError):
 
 
 def problem(B, H, d, text_len, grid, text_k=4, vis_k=(3, 3, 3), chunk=64, vis_causal_t=False,
-            dv=None) -> kda_problem:
+            dv=None, reuse_records=False, qkv_f16=False) -> kda_problem:
     T, Hg, Wg = grid
+    flags = ((KDA_FLAG_VIS_CAUSAL_T if vis_causal_t else 0) | (KDA_FLAG_REUSE_RECORDS if reuse_records else 0)
+             | (KDA_FLAG_QKV_F16 if qkv_f16 else 0))
     return kda_problem(B, H, d, d if dv is None else dv, text_len, T, Hg, Wg, text_k,
-                       vis_k[0], vis_k[1], vis_k[2], chunk, KDA_FLAG_VIS_CAUSAL_T if vis_causal_t else 0)
+                       vis_k[0], vis_k[1], vis_k[2], chunk, flags)
 
 
 def _dt(dtype) -> int:
@@ -139,7 +143,8 @@ def kda_shortconv_fwd(p, q, k, v, w_text, w_vis, q_out, k_out, v_out, stream=Non
 def kda_chunk_fwd(p, q, k, v, log_alpha, beta, o, workspace, initial_state=None, final_state=None,
                   stream=None, workspace_bytes=None):
     nbytes = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
-    _check(_lib.kda_chunk_fwd(ctypes.byref(p), _dt(q.dtype), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
+    # the problem dtype is o's (q, k, v may be fp16 under KDA_FLAG_QKV_F16)
+    _check(_lib.kda_chunk_fwd(ctypes.byref(p), _dt(o.dtype), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
                               _ptr(beta), _ptr(initial_state), _ptr(o), _ptr(final_state), _ptr(workspace),
                               nbytes, _stream(stream)),
            "kda_chunk_fwd")
@@ -158,7 +163,7 @@ def kda_chunk_fwd_noalloc(p, q, k, v, log_alpha, beta, o, initial_state=None, fi
                           device_status=None, stream=None):
     """kda_chunk_fwd without a workspace: scratch is the library's static device
     array (see include/kda.h for its limit and sharing rules)."""
-    _check(_lib.kda_chunk_fwd_noalloc(ctypes.byref(p), _dt(q.dtype), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
+    _check(_lib.kda_chunk_fwd_noalloc(ctypes.byref(p), _dt(o.dtype), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
                                       _ptr(beta), _ptr(initial_state), _ptr(o), _ptr(final_state),
                                       _ptr(device_status), _stream(stream)),
            "kda_chunk_fwd_noalloc")

@@ -1167,8 +1167,12 @@ cudaError_t launch_all(const Dims& d, const void* q, const void* k, const void* 
       !encode_act_map(&mp.v, v, adt, 2, d, 64, true) ||
       !encode_act_map(&mp.la, la, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, d, 128, false))
     return cudaErrorInvalidValue;
-  kda_tc_prep<TIn><<<dim3((unsigned)min(n_units, n_sm)), 256, PREP_SMEM, s>>>(pa, mp);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // the records depend on q, k, v, log alpha and beta only: a caller that kept them (same inputs,
+  // same workspace) runs the state pass alone
+  if (!d.reuse_records) {
+    kda_tc_prep<TIn><<<dim3((unsigned)min(n_units, n_sm)), 256, PREP_SMEM, s>>>(pa, mp);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
   ChainArgs ca{ws, S0, SN, static_cast<__nv_bfloat16*>(o), d.N, d.H, n_blocks, status};
   // the narrowest column split whose grid fits on the SMs (the serial pass is latency bound)
   const int bh = d.B * d.H;
@@ -1177,7 +1181,7 @@ cudaError_t launch_all(const Dims& d, const void* q, const void* k, const void* 
   else e = launch_chain<64>(ca, dim3(ChainLayout<64>::NQ, d.H, d.B), s);
   if (e != cudaSuccess) return e;
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  if (launches) *launches += 2;
+  if (launches) *launches += d.reuse_records ? 1 : 2;
   return cudaSuccess;
 }
 

@@ -17,6 +17,8 @@ struct Dims {
   int text_k;
   int pt, ph, pw;        // 3D conv padding (tap offsets are a - pt etc.)
   int chunk;
+  bool reuse_records;    // KDA_FLAG_REUSE_RECORDS: the workspace holds this problem's block records
+  bool qkv_f16;          // KDA_FLAG_QKV_F16: convolved q', k', v' are fp16
 };
 
 // Device status word: the first uint32 of the workspace.

@@ -25,7 +25,7 @@ int make_dims(const kda_problem* p, kda_dtype dt, kda::Dims* d) {
   if (any_grid && !all_grid) return KDA_ERR_INVALID_ARG;
   if (p->text_k < 1 || p->vis_kt < 1 || p->vis_kh < 1 || p->vis_kw < 1 || p->chunk < 1)
     return KDA_ERR_INVALID_ARG;
-  if (p->flags & ~KDA_FLAG_VIS_CAUSAL_T) return KDA_ERR_INVALID_ARG;
+  if (p->flags & ~(KDA_FLAG_VIS_CAUSAL_T | KDA_FLAG_REUSE_RECORDS | KDA_FLAG_QKV_F16)) return KDA_ERR_INVALID_ARG;
   if (p->dk != p->dv || (p->dk != 64 && p->dk != 128)) return KDA_ERR_UNSUPPORTED;
   if (p->text_k > 8) return KDA_ERR_UNSUPPORTED;
   if (p->vis_kt != 3 || p->vis_kh != 3 || p->vis_kw != 3) return KDA_ERR_UNSUPPORTED;
@@ -45,6 +45,10 @@ int make_dims(const kda_problem* p, kda_dtype dt, kda::Dims* d) {
   d->ph = (p->vis_kh - 1) / 2;
   d->pw = (p->vis_kw - 1) / 2;
   d->chunk = p->chunk;
+  d->reuse_records = (p->flags & KDA_FLAG_REUSE_RECORDS) != 0;
+  d->qkv_f16 = (p->flags & KDA_FLAG_QKV_F16) != 0;
+  // fp16 activations exist only where the tensor-core scan reads them (bf16, d = 128)
+  if (d->qkv_f16 && !(dt == KDA_DT_BF16 && kda::chunk_tc_supported(*d))) return KDA_ERR_UNSUPPORTED;
   return KDA_OK;
 }
 
@@ -137,10 +141,11 @@ int kda_shortconv_fwd(const kda_problem* p, kda_dtype dtype, const void* q, cons
   kda::Dims d;
   int st = make_dims(p, dtype, &d);
   if (st) return st;
+  if (d.reuse_records) return KDA_ERR_INVALID_ARG;
   if ((st = check_ptrs({q, k, v, w_text, w_vis, q_out, k_out, v_out}, {}))) return st;
   int launches = 0;
   st = cuda_status(kda::launch_shortconv(d, dtype, q, k, v, w_text, w_vis, q_out, k_out, v_out,
-                                         static_cast<cudaStream_t>(stream), &launches));
+                                         static_cast<cudaStream_t>(stream), &launches, d.qkv_f16));
   if (!st) g_last_launches = launches;
   return st;
 }
@@ -159,7 +164,7 @@ int kda_chunk_fwd(const kda_problem* p, kda_dtype dtype, const void* q, const vo
   if ((st = cuda_status(cudaMemsetAsync(status, 0, sizeof(uint32_t), s)))) return st;
   int launches = 0;
   st = run_scan(d, dtype, q, k, v, log_alpha, beta, initial_state, o, final_state, workspace, s, &launches,
-                false);
+                d.qkv_f16);
   if (!st) g_last_launches = launches;
   return st;
 }
@@ -172,6 +177,7 @@ int kda_fwd(const kda_problem* p, kda_dtype dtype, const void* q, const void* k,
   kda::Dims d;
   int st = make_dims(p, dtype, &d);
   if (st) return st;
+  if (d.reuse_records || d.qkv_f16) return KDA_ERR_INVALID_ARG;
   if ((st = check_ptrs({q, k, v, log_alpha, beta, w_text, w_vis, o}, {initial_state, final_state})))
     return st;
   if ((st = check_workspace(d, dtype, workspace, workspace_bytes_))) return st;

@@ -54,6 +54,7 @@ extern "C" int kda_chunk_fwd_noalloc(const kda_problem* p, kda_dtype dtype, cons
   kda::Dims d;
   int st = kda::validate_problem(p, dtype, &d);
   if (st) return st;
+  if (d.reuse_records) return KDA_ERR_INVALID_ARG;   // the shared scratch keeps no records between calls
   if ((st = kda::validate_scan_pointers(q, k, v, log_alpha, beta, o, initial_state, final_state))) return st;
   if (device_status && (reinterpret_cast<uintptr_t>(device_status) & 3u)) return KDA_ERR_MISALIGNED;
   const bool tc = dtype == KDA_DT_BF16 && kda::chunk_tc_supported(d);
@@ -73,7 +74,7 @@ extern "C" int kda_chunk_fwd_noalloc(const kda_problem* p, kda_dtype dtype, cons
                         : cudaMemsetAsync(final_state, 0, bytes, s);
     }
   } else if (tc) {
-    e = kda::launch_chunk_tc(d, false, q, k, v, log_alpha, beta, initial_state, o, final_state,
+    e = kda::launch_chunk_tc(d, d.qkv_f16, q, k, v, log_alpha, beta, initial_state, o, final_state,
                              static_cast<char*>(scratch) + kStatusBytes, status, s, &launches);
   } else {
     e = kda::launch_chunk_simt(d, dtype, q, k, v, log_alpha, beta, initial_state, o, final_state, status, s,

@@ -86,6 +86,22 @@ def test_host_side_rejections_launch_nothing(kda):
     bad = _p(kda)
     bad.flags = 1 << 5
     assert _call_fwd(kda, bad) == kda.KDA_ERR_INVALID_ARG
+    # record reuse is a kda_chunk_fwd option: the conv and fused entry points reject it
+    reuse = _p(kda)
+    reuse.flags = kda.KDA_FLAG_REUSE_RECORDS
+    assert _call_fwd(kda, reuse) == kda.KDA_ERR_INVALID_ARG
+    assert kda._lib.kda_shortconv_fwd(ctypes.byref(reuse), 0, 256, 256, 256, 256, 256, 256, 256, 256, None) == \
+        kda.KDA_ERR_INVALID_ARG
+    assert kda._lib.kda_chunk_fwd_noalloc(ctypes.byref(reuse), 0, 256, 256, 256, 256, 256, None, 256, None, None,
+                                          None) == kda.KDA_ERR_INVALID_ARG
+    # fp16 activations: bf16 problems with d = 128 only; kda_fwd keeps its own and rejects the flag
+    f16 = _p(kda, d=128)
+    f16.flags = kda.KDA_FLAG_QKV_F16
+    assert _call_fwd(kda, f16) == kda.KDA_ERR_INVALID_ARG
+    assert _call_fwd(kda, f16, dt=1) == kda.KDA_ERR_UNSUPPORTED
+    f16_64 = _p(kda, d=64)
+    f16_64.flags = kda.KDA_FLAG_QKV_F16
+    assert _call_fwd(kda, f16_64) == kda.KDA_ERR_UNSUPPORTED
     lib = kda._lib
     assert lib.kda_shortconv_fwd(ctypes.byref(p), 0, 256, 256, 256, 256, 256, 256, 256, 0x1002, None) == \
         kda.KDA_ERR_MISALIGNED

@@ -306,3 +306,79 @@ def test_strong_decay_takes_exact_branch(kda):
     ref, _ = oracle.forward(inp, w.text_len, w.grid)
     o, _ = run_fwd(kda, w, inp, chunk=64)
     assert_parity(o, ref, "f32", "strong decay")
+
+
+def test_bf16_record_reuse_reruns_only_the_state_pass(kda):
+    """KDA_FLAG_REUSE_RECORDS: a second kda_chunk_fwd on the same inputs and workspace, from
+    another initial state, launches the state pass alone and equals a fresh call bit for bit."""
+    w = kda_synth.WORKLOADS[1]
+    inp = workload_inputs(1)
+    B, N, H, d = inp["shape"]
+    t = to_device(inp)
+    args = [t[n] for n in ("q", "k", "v", "log_alpha", "beta")]
+    s_a, s_b = (torch.from_numpy(kda_synth.initial_state(s, B, H, d, d)).cuda() for s in (3, 4))
+    p = kda.problem(B, H, d, w.text_len, w.grid)
+    p_reuse = kda.problem(B, H, d, w.text_len, w.grid, reuse_records=True)
+
+    def out():
+        return (torch.empty(B, N, H, d, dtype=t["q"].dtype, device="cuda"),
+                torch.empty(B, H, d, d, dtype=torch.float32, device="cuda"))
+    (o1, n1), (o2, n2), (o3, n3) = out(), out(), out()
+    ws1, ws2 = kda.alloc_workspace(p, t["q"].dtype), kda.alloc_workspace(p, t["q"].dtype)
+    kda.kda_chunk_fwd(p, *args, o1, ws1, initial_state=s_b, final_state=n1)
+    kda.kda_chunk_fwd(p, *args, o2, ws2, initial_state=s_a, final_state=n2)
+    kda.kda_chunk_fwd(p_reuse, *args, o3, ws2, initial_state=s_b, final_state=n3)
+    assert kda.kda_last_launch_count() == 1
+    assert kda.kda_read_status(ws2) == kda.KDA_OK
+    assert torch.equal(o3, o1) and torch.equal(n3, n1)
+    assert not torch.equal(o2, o1)
+
+
+@pytest.mark.parametrize("world,causal", [(3, False), (2, True)])
+def test_bf16_sequence_sharded_on_thread_ranks(kda, world, causal):
+    """The sequence-sharded pass (frames split over ranks, conv halo exchange, per-rank state maps
+    composed across ranks) with every rank a thread on this GPU: same result as the unsharded pass,
+    and oracle parity on sampled value columns."""
+    from linear_attention_video_b200 import seqshard
+    w = kda_synth.WORKLOADS[2]
+    inp = workload_inputs(2)
+    B, N, H, d = inp["shape"]
+    t = to_device(inp)
+    S0 = kda_synth.initial_state(9, B, H, d, d)
+    s0 = torch.from_numpy(S0).cuda()
+
+    def rank_pass(comm):
+        seg = seqshard.partition(w.text_len, w.grid, comm.world, causal)[comm.rank]
+        x = tuple(t[n][:, seg.t0:seg.t1].contiguous() for n in ("q", "k", "v"))
+        be = seqshard.GpuBackend(B, H, d, vis_causal_t=causal)
+        return seqshard.seqshard_fwd(be, comm, x, t["log_alpha"][:, seg.t0:seg.t1].contiguous(),
+                                     t["beta"][:, seg.t0:seg.t1].contiguous(), t["w_text"], t["w_vis"],
+                                     w.text_len, w.grid, s0)
+    outs = seqshard.LocalGroup(world, timeout_s=300).run(rank_pass)
+    torch.cuda.synchronize()
+    o = torch.cat([o_r for o_r, _ in outs], dim=1).float().cpu().numpy()
+    s_last = outs[-1][1].cpu().numpy()
+    o_full, s_full = run_fwd(kda, w, inp, S0=S0, want_state=True, vis_causal_t=causal)
+    assert rel_l2(o, o_full) < 3e-3 and rel_l2(s_last, s_full) < 3e-3
+    items = [(0, 0), (7, 77), (15, 127)]
+    ref = oracle.forward_columns(inp, w.text_len, w.grid, items, S0=S0, vis_causal_t=causal)
+    got = np.stack([o[:, :, h, j] for h, j in items])
+    assert_parity(got, ref, "bf16", f"sharded over {world}")
+
+
+def test_bf16_split_pass_with_fp16_activations_equals_fused(kda):
+    """KDA_FLAG_QKV_F16: kda_shortconv_fwd writing fp16 q', k', v' and kda_chunk_fwd reading them
+    reproduce kda_fwd (which keeps the same fp16 intermediates) bit for bit."""
+    w = kda_synth.WORKLOADS[1]
+    inp = workload_inputs(1)
+    B, N, H, d = inp["shape"]
+    t = to_device(inp)
+    p = kda.problem(B, H, d, w.text_len, w.grid, qkv_f16=True)
+    conv = [torch.empty(B, N, H, d, dtype=torch.float16, device="cuda") for _ in range(3)]
+    kda.kda_shortconv_fwd(p, t["q"], t["k"], t["v"], t["w_text"], t["w_vis"], *conv)
+    o_split = torch.empty_like(t["q"])
+    ws = kda.alloc_workspace(p, t["q"].dtype)
+    kda.kda_chunk_fwd(p, *conv, t["log_alpha"], t["beta"], o_split, ws)
+    assert kda.kda_read_status(ws) == kda.KDA_OK
+    o_fused, _ = run_fwd(kda, w, inp)
+    assert np.array_equal(o_split.float().cpu().numpy(), o_fused)
