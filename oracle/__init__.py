@@ -10,6 +10,9 @@ Two independent formulations live here, both in fp64:
   out tap by tap, and the token-by-token KDA recurrence
   (paper.rainbus.top, section 方法步骤详情, step (5);
   genai-atlas, section "How it works").
+* ``kda_oracle.c`` also holds the backward pass: the chain rule written out
+  through the recurrence (token by token, in reverse, every state kept) and the
+  transpose of the convolution; pinned by finite differences of the forward.
 * this module's numpy code -- the chunked (UT/WY) form for any chunk length,
   the dense lower-triangular form, and the update exactly as printed on the
   page (explicit (I - beta k k^T) Diag(alpha) products), used only to
@@ -66,6 +69,10 @@ def _load():
             lib.kdao_shortconv.restype = i32
             lib.kdao_scan.argtypes = [i64, i64, i64, i64, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i32]
             lib.kdao_scan.restype = i32
+            lib.kdao_scan_bwd.argtypes = [i64, i64, i64, i64] + [vp] * 14 + [i32]
+            lib.kdao_scan_bwd.restype = i32
+            lib.kdao_shortconv_bwd.argtypes = [ctypes.POINTER(ConvShape), i64] + [vp] * 7 + [i32]
+            lib.kdao_shortconv_bwd.restype = i32
             _lib = lib
     return _lib
 
@@ -201,6 +208,90 @@ def forward_columns(inp: dict, text_len: int, grid, items, S0=None, text_k=4, vi
             oh, _ = scan(qh, kh, vfull, la, bt, s0, j0=j, j1=j + 1, nthreads=nthreads)
             res[i] = oh[:, :, j]
     return res
+
+
+# ---------------------------------------------------------------------------
+# Backward pass (fp64): the chain rule through the steps above, in kda_oracle.c.
+# ---------------------------------------------------------------------------
+
+def scan_bwd(q, k, v, log_alpha, beta, dO, S0=None, dSN=None, nthreads=None):
+    """Gradients of one head's recurrence for the loss sum(dO * o) + sum(dSN * S_N).
+
+    Shapes as in ``scan``; dO [B, N, dv], dSN [B, dk, dv] or None.  Returns a dict with
+    dq, dk, dla [B, N, dk], dv [B, N, dv], dbeta [B, N] and dS0 [B, dk, dv].  Every state
+    is kept: small problems only."""
+    q, k, v, la, bt, dO = (np.ascontiguousarray(a, dtype=np.float64) for a in (q, k, v, log_alpha, beta, dO))
+    B, N, dk = q.shape
+    dv = v.shape[-1]
+    out = {"dq": np.zeros((B, N, dk)), "dk": np.zeros((B, N, dk)), "dv": np.zeros((B, N, dv)),
+           "dla": np.zeros((B, N, dk)), "dbeta": np.zeros((B, N)), "dS0": np.zeros((B, dk, dv))}
+    s0 = None if S0 is None else np.ascontiguousarray(S0, dtype=np.float64)
+    dsn = None if dSN is None else np.ascontiguousarray(dSN, dtype=np.float64)
+    ptr = lambda a: None if a is None else a.ctypes.data   # noqa: E731
+    rc = _load().kdao_scan_bwd(B, N, dk, dv, ptr(q), ptr(k), ptr(v), ptr(la), ptr(bt), ptr(s0), ptr(dO), ptr(dsn),
+                               ptr(out["dq"]), ptr(out["dk"]), ptr(out["dv"]), ptr(out["dla"]), ptr(out["dbeta"]),
+                               ptr(out["dS0"]), nthreads or default_threads())
+    if rc:
+        raise ValueError(f"kdao_scan_bwd failed ({rc})")
+    return out
+
+
+def shortconv_bwd(shape: ConvShape, x: np.ndarray, w_text: np.ndarray, w_vis: np.ndarray, dy: np.ndarray,
+                  nthreads: int | None = None):
+    """Gradients of sum(dy * shortconv(x)) w.r.t. x [B, N, C] and the weights.
+
+    Returns (dx [B, N, C], dw_text [C, text_k], dw_vis [C, kt*kh*kw]), float64."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    B, N, C = x.shape
+    wt = np.ascontiguousarray(w_text, dtype=np.float32)
+    wv = np.ascontiguousarray(w_vis, dtype=np.float32)
+    dy = np.ascontiguousarray(dy, dtype=np.float64)
+    dx = np.empty((B, N, C))
+    dwt = np.empty(wt.shape)
+    dwv = np.empty(wv.shape)
+    rc = _load().kdao_shortconv_bwd(ctypes.byref(shape), C, x.ctypes.data, wt.ctypes.data, wv.ctypes.data,
+                                    dy.ctypes.data, dx.ctypes.data, dwt.ctypes.data, dwv.ctypes.data,
+                                    nthreads or default_threads())
+    if rc:
+        raise ValueError(f"kdao_shortconv_bwd failed ({rc})")
+    return dx, dwt, dwv
+
+
+def backward(inp: dict, text_len: int, grid, dO, S0=None, dSN=None, text_k=4, vis_k=(3, 3, 3),
+             vis_causal_t=False, nthreads=None):
+    """Gradients of the whole forward (conv on q, k, v, then the recurrence, every head) for the
+    loss sum(dO * o) + sum(dSN * S_N).
+
+    dO [B, N, H, d]; S0, dSN [B, H, d, d] or None.  Returns a dict with dq, dk, dv, dla
+    [B, N, H, d], dbeta [B, N, H], dS0 [B, H, d, d] and dw_text, dw_vis [3][C][...] (float64)."""
+    B, N, H, d = inp["shape"]
+    shape = conv_shape(B, N, text_len, grid, text_k, vis_k, vis_causal_t)
+    xs = _widened(inp)
+    conv = [shortconv(shape, xs[i], inp["w_text"][i], inp["w_vis"][i], nthreads=nthreads).reshape(B, N, H, d)
+            for i in range(3)]
+    la = inp["log_alpha"].reshape(B, N, H, d).astype(np.float64)
+    bt = widen(inp["beta"], inp["dtype"]).reshape(B, N, H).astype(np.float64)
+    dO = np.asarray(dO, dtype=np.float64).reshape(B, N, H, d)
+    dconv = [np.zeros((B, N, H, d)) for _ in range(3)]
+    g = {"dla": np.zeros((B, N, H, d)), "dbeta": np.zeros((B, N, H)), "dS0": np.zeros((B, H, d, d))}
+    for h in range(H):
+        r = scan_bwd(conv[0][:, :, h], conv[1][:, :, h], conv[2][:, :, h], la[:, :, h], bt[:, :, h],
+                     dO[:, :, h], None if S0 is None else np.asarray(S0)[:, h],
+                     None if dSN is None else np.asarray(dSN)[:, h], nthreads)
+        for i, n in enumerate(("dq", "dk", "dv")):
+            dconv[i][:, :, h] = r[n]
+        g["dla"][:, :, h] = r["dla"]
+        g["dbeta"][:, :, h] = r["dbeta"]
+        g["dS0"][:, h] = r["dS0"]
+    g["dw_text"], g["dw_vis"] = [], []
+    for i, n in enumerate(("dq", "dk", "dv")):
+        dx, dwt, dwv = shortconv_bwd(shape, xs[i], inp["w_text"][i], inp["w_vis"][i],
+                                     dconv[i].reshape(B, N, H * d), nthreads)
+        g[n] = dx.reshape(B, N, H, d)
+        g["dw_text"].append(dwt)
+        g["dw_vis"].append(dwv)
+    g["dw_text"], g["dw_vis"] = np.stack(g["dw_text"]), np.stack(g["dw_vis"])
+    return g
 
 
 # ---------------------------------------------------------------------------
