@@ -141,6 +141,31 @@ int kda_fwd(const kda_problem* p, kda_dtype dtype,
             const float* initial_state, void* o, float* final_state,
             void* workspace, size_t workspace_bytes, void* stream);
 
+/* Backward pass of kda_fwd: the gradients of the loss sum(d_o * o) + sum(d_final_state * S_N)
+ * (o and S_N as kda_fwd computes them from the same arguments) with respect to every input.
+ * The pages describe only the forward pass; the gradients are the chain rule applied to it
+ * (the conv is linear, its adjoint is its transpose; the recurrence is run in reverse from
+ * states recomputed from a copy stored every 16 tokens).  fp32 on the CUDA cores.
+ *   d_o                    [B, N, H, d] of dtype; d_final_state [B, H, d, d] fp32 or NULL (zero)
+ *   dq, dk, dv             [B, N, H, d] of dtype: gradients of the raw (unconvolved) q, k, v
+ *   d_log_alpha            [B, N, H, d] fp32;  d_beta [B, N, H] of dtype
+ *   d_w_text, d_w_vis      [3][H*d][text_k], [3][H*d][kt*kh*kw] fp32
+ *   d_initial_state        [B, H, d, d] fp32 or NULL (not written)
+ * The workspace is kda_bwd_workspace_bytes(p, dtype) bytes, 256-byte aligned.  Flags:
+ * KDA_FLAG_VIS_CAUSAL_T as in kda_fwd; the other flags are rejected.  fp32 gradients that
+ * several CTAs add into (dq, dk, d_log_alpha, d_beta before rounding, the weights) are summed
+ * with atomic adds, so their last bits depend on the order of the additions.  Returns a
+ * kda_status. */
+size_t kda_bwd_workspace_bytes(const kda_problem* p, kda_dtype dtype);
+int kda_bwd(const kda_problem* p, kda_dtype dtype,
+            const void* q, const void* k, const void* v,
+            const float* log_alpha, const void* beta,
+            const float* w_text, const float* w_vis, const float* initial_state,
+            const void* d_o, const float* d_final_state,
+            void* dq, void* dk, void* dv, float* d_log_alpha, void* d_beta,
+            float* d_w_text, float* d_w_vis, float* d_initial_state,
+            void* workspace, size_t workspace_bytes, void* stream);
+
 /* kda_chunk_fwd without a workspace, for callers that cannot allocate device
  * memory (code running inside an allocator or memory-pool callback, runtimes
  * that forbid allocation after start-up, plugins handed only their input and

@@ -32,7 +32,8 @@ KDA_FLAG_REUSE_RECORDS = 2
 KDA_FLAG_QKV_F16 = 4
 
 EXPORTS = ("kda_tokens", "kda_workspace_bytes", "kda_shortconv_fwd", "kda_chunk_fwd", "kda_fwd",
-           "kda_chunk_fwd_noalloc", "kda_read_status", "kda_status_str", "kda_last_launch_count")
+           "kda_chunk_fwd_noalloc", "kda_bwd_workspace_bytes", "kda_bwd", "kda_read_status", "kda_status_str",
+           "kda_last_launch_count")
 
 
 class kda_problem(ctypes.Structure):
@@ -57,6 +58,10 @@ _lib.kda_fwd.argtypes = [_pp, _i] + [_vp] * 11 + [_sz, _vp]
 _lib.kda_fwd.restype = _i
 _lib.kda_chunk_fwd_noalloc.argtypes = [_pp, _i] + [_vp] * 10
 _lib.kda_chunk_fwd_noalloc.restype = _i
+_lib.kda_bwd_workspace_bytes.argtypes = [_pp, _i]
+_lib.kda_bwd_workspace_bytes.restype = _sz
+_lib.kda_bwd.argtypes = [_pp, _i] + [_vp] * 19 + [_sz, _vp]
+_lib.kda_bwd.restype = _i
 _lib.kda_read_status.argtypes = [_vp, _vp]
 _lib.kda_read_status.restype = _i
 _lib.kda_status_str.argtypes = [_i]
@@ -167,6 +172,28 @@ def kda_chunk_fwd_noalloc(p, q, k, v, log_alpha, beta, o, initial_state=None, fi
                                       _ptr(beta), _ptr(initial_state), _ptr(o), _ptr(final_state),
                                       _ptr(device_status), _stream(stream)),
            "kda_chunk_fwd_noalloc")
+
+
+def kda_bwd_workspace_bytes(p: kda_problem, dtype) -> int:
+    return _lib.kda_bwd_workspace_bytes(ctypes.byref(p), _dt(dtype))
+
+
+def alloc_bwd_workspace(p: kda_problem, dtype, device="cuda") -> torch.Tensor:
+    n = kda_bwd_workspace_bytes(p, dtype)
+    if n == 0:
+        raise KdaError(KDA_ERR_INVALID_ARG, "kda_bwd_workspace_bytes")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def kda_bwd(p, q, k, v, log_alpha, beta, w_text, w_vis, d_o, dq, dk, dv, d_log_alpha, d_beta, d_w_text, d_w_vis,
+            workspace, initial_state=None, d_final_state=None, d_initial_state=None, stream=None,
+            workspace_bytes=None):
+    nbytes = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    _check(_lib.kda_bwd(ctypes.byref(p), _dt(q.dtype), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                        _ptr(w_text), _ptr(w_vis), _ptr(initial_state), _ptr(d_o), _ptr(d_final_state), _ptr(dq),
+                        _ptr(dk), _ptr(dv), _ptr(d_log_alpha), _ptr(d_beta), _ptr(d_w_text), _ptr(d_w_vis),
+                        _ptr(d_initial_state), _ptr(workspace), nbytes, _stream(stream)),
+           "kda_bwd")
 
 
 def kda_read_status(workspace, stream=None) -> int:

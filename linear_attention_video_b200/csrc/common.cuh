@@ -36,10 +36,20 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 }
 
 // Launchers (defined in the .cu files).
-// out_f16: write fp16 outputs (the internal format the tensor-core scan reads) instead of dtype.
+// out_f16: write fp16 outputs (the internal format the tensor-core scan reads) instead of dtype;
+// out_f32: write fp32 outputs (what the backward pass recomputes).
 cudaError_t launch_shortconv(const Dims& d, kda_dtype dt, const void* q, const void* k, const void* v,
                              const float* w_text, const float* w_vis, void* qo, void* ko, void* vo,
-                             cudaStream_t s, int* launches, bool out_f16 = false);
+                             cudaStream_t s, int* launches, bool out_f16 = false, bool out_f32 = false);
+
+// Backward pass (bwd.cu): gradients of kda_fwd.  Buffers as in kda_bwd (include/kda.h); ws holds
+// bwd_workspace_bytes(d, dt) bytes, 256-byte aligned, its first word the status word.
+size_t bwd_workspace_bytes(const Dims& d, kda_dtype dt);
+cudaError_t launch_bwd(const Dims& d, kda_dtype dt, const void* q, const void* k, const void* v,
+                       const float* log_alpha, const void* beta, const float* w_text, const float* w_vis,
+                       const float* S0, const void* d_o, const float* dSN, void* dq, void* dk, void* dv,
+                       float* dla, void* dbeta, float* dw_text, float* dw_vis, float* dS0, void* ws,
+                       cudaStream_t s, int* launches);
 
 cudaError_t launch_chunk_simt(const Dims& d, kda_dtype dt, const void* q, const void* k, const void* v,
                               const float* log_alpha, const void* beta, const float* S0, void* o,

@@ -200,6 +200,38 @@ int kda_fwd(const kda_problem* p, kda_dtype dtype, const void* q, const void* k,
   return st;
 }
 
+size_t kda_bwd_workspace_bytes(const kda_problem* p, kda_dtype dtype) {
+  kda::Dims d;
+  if (make_dims(p, dtype, &d) || d.reuse_records || d.qkv_f16) return 0;
+  return kda::bwd_workspace_bytes(d, dtype);
+}
+
+int kda_bwd(const kda_problem* p, kda_dtype dtype, const void* q, const void* k, const void* v,
+            const float* log_alpha, const void* beta, const float* w_text, const float* w_vis,
+            const float* initial_state, const void* d_o, const float* d_final_state, void* dq, void* dk, void* dv,
+            float* d_log_alpha, void* d_beta, float* d_w_text, float* d_w_vis, float* d_initial_state,
+            void* workspace, size_t workspace_bytes_, void* stream) {
+  g_last_launches = 0;
+  kda::Dims d;
+  int st = make_dims(p, dtype, &d);
+  if (st) return st;
+  if (d.reuse_records || d.qkv_f16) return KDA_ERR_INVALID_ARG;
+  if ((st = check_ptrs({q, k, v, log_alpha, beta, w_text, w_vis, d_o, dq, dk, dv, d_log_alpha, d_beta, d_w_text,
+                        d_w_vis},
+                       {initial_state, d_final_state, d_initial_state})))
+    return st;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return KDA_ERR_WORKSPACE;
+  if (workspace_bytes_ < kda::bwd_workspace_bytes(d, dtype)) return KDA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = cuda_status(cudaMemsetAsync(workspace, 0, sizeof(uint32_t), s)))) return st;
+  int launches = 0;
+  st = cuda_status(kda::launch_bwd(d, dtype, q, k, v, log_alpha, beta, w_text, w_vis, initial_state, d_o,
+                                   d_final_state, dq, dk, dv, d_log_alpha, d_beta, d_w_text, d_w_vis,
+                                   d_initial_state, workspace, s, &launches));
+  if (!st) g_last_launches = launches;
+  return st;
+}
+
 int kda_read_status(void* workspace, void* stream) {
   if (!workspace) return KDA_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -328,7 +328,7 @@ cudaError_t launch_t(const ConvArgs& a, cudaStream_t s) {
 
 cudaError_t launch_shortconv(const Dims& d, kda_dtype dt, const void* q, const void* k, const void* v,
                              const float* w_text, const float* w_vis, void* qo, void* ko, void* vo,
-                             cudaStream_t s, int* launches, bool out_f16) {
+                             cudaStream_t s, int* launches, bool out_f16, bool out_f32) {
   ConvArgs a;
   a.x[0] = q; a.x[1] = k; a.x[2] = v;
   a.y[0] = qo; a.y[1] = ko; a.y[2] = vo;
@@ -341,7 +341,8 @@ cudaError_t launch_shortconv(const Dims& d, kda_dtype dt, const void* q, const v
   a.n_hbands = d.T > 0 ? (d.Hg + TH - 1) / TH : 0;
   if ((int64_t)d.B * d.N == 0) return cudaSuccess;
   cudaError_t e;
-  if (dt == KDA_DT_BF16 && out_f16) e = launch_t<__nv_bfloat16, __half>(a, s);
+  if (dt == KDA_DT_BF16 && out_f32) e = launch_t<__nv_bfloat16, float>(a, s);
+  else if (dt == KDA_DT_BF16 && out_f16) e = launch_t<__nv_bfloat16, __half>(a, s);
   else if (dt == KDA_DT_BF16) e = launch_t<__nv_bfloat16, __nv_bfloat16>(a, s);
   else e = launch_t<float, float>(a, s);
   if (e == cudaSuccess && launches) *launches += (a.L > 0) + (a.T > 0);

@@ -5,6 +5,7 @@ import os
 import re
 
 import pytest
+import torch
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "kda.h")
@@ -107,4 +108,17 @@ def test_host_side_rejections_launch_nothing(kda):
         kda.KDA_ERR_MISALIGNED
     assert lib.kda_chunk_fwd(ctypes.byref(p), 0, 256, 256, 256, 256, None, None, 256, None, 512, 1 << 40, None) == \
         kda.KDA_ERR_INVALID_ARG
+    # backward entry point: host-side checks before any CUDA call
+    lib.kda_bwd.restype = ctypes.c_int
+    bwd = lambda pp, **kw: lib.kda_bwd(ctypes.byref(pp), kw.get("dt", 0), *[kw.get(n, 256) for n in (   # noqa: E731
+        "q", "k", "v", "la", "beta", "wt", "wv", "s0", "do", "dsn", "dq", "dk", "dv", "dla", "dbeta", "dwt", "dwv",
+        "ds0")], kw.get("ws", 512), kw.get("ws_bytes", 1 << 40), None)
+    for n in ("q", "do", "dq", "dla", "dwv"):
+        assert bwd(p, **{n: None}) == kda.KDA_ERR_INVALID_ARG, n
+    assert bwd(p, dv=0x1008) == kda.KDA_ERR_MISALIGNED
+    assert bwd(p, ds0=0x1004) == kda.KDA_ERR_MISALIGNED
+    assert bwd(p, ws=0x1010) == kda.KDA_ERR_WORKSPACE
+    assert bwd(p, ws_bytes=1000) == kda.KDA_ERR_WORKSPACE
+    assert bwd(reuse) == kda.KDA_ERR_INVALID_ARG
+    assert kda.kda_bwd_workspace_bytes(p, torch.bfloat16) > kda.kda_workspace_bytes(p, torch.bfloat16)
     assert kda.kda_last_launch_count() == 0

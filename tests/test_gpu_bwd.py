@@ -1,0 +1,103 @@
+"""Backward pass (kda_bwd) vs the oracle's adjoint, through the C ABI (needs a B200).
+
+The oracle's backward is pinned by finite differences (tests/test_oracle_bwd.py).
+Each gradient is compared element by element: relative L2 error within the
+fp32 bound (1e-5) for fp32 problems; for bf16 problems within the bf16 bounds
+(relative L2 5e-3, and max-abs 2e-2 taken relative to the gradient's largest
+magnitude, since gradients carry the scale of d_o rather than of o).
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import kda_synth
+import oracle
+from tests._util import rel_l2, to_device
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def kda():
+    import linear_attention_video_b200 as kda
+    assert torch.cuda.is_available()
+    return kda
+
+
+def run_bwd(kda, w, inp, dO, S0=None, dSN=None, causal=False):
+    B, N, H, d = inp["shape"]
+    t = to_device(inp)
+    dt = t["q"].dtype
+    p = kda.problem(B, H, d, w.text_len, w.grid, vis_causal_t=causal)
+    f32 = lambda a: None if a is None else torch.from_numpy(np.ascontiguousarray(a, np.float32)).cuda()   # noqa: E731
+    d_o = torch.from_numpy(np.ascontiguousarray(dO, np.float32)).reshape(B, N, H, d).cuda().to(dt)
+    g = {n: torch.empty(B, N, H, d, dtype=dt, device="cuda") for n in ("dq", "dk", "dv")}
+    g["dla"] = torch.empty(B, N, H, d, dtype=torch.float32, device="cuda")
+    g["dbeta"] = torch.empty(B, N, H, dtype=dt, device="cuda")
+    g["dw_text"] = torch.empty(3, H * d, w.text_k, dtype=torch.float32, device="cuda")
+    g["dw_vis"] = torch.empty(3, H * d, 27, dtype=torch.float32, device="cuda")
+    g["dS0"] = torch.empty(B, H, d, d, dtype=torch.float32, device="cuda")
+    ws = kda.alloc_bwd_workspace(p, dt)
+    kda.kda_bwd(p, t["q"], t["k"], t["v"], t["log_alpha"], t["beta"], t["w_text"], t["w_vis"], d_o, g["dq"], g["dk"],
+                g["dv"], g["dla"], g["dbeta"], g["dw_text"], g["dw_vis"], ws, initial_state=f32(S0),
+                d_final_state=f32(dSN), d_initial_state=g["dS0"])
+    torch.cuda.synchronize()
+    assert kda.kda_read_status(ws) == kda.KDA_OK
+    # the gradient the oracle sees for d_o is the value actually passed (rounded to dtype)
+    return {n: v.float().cpu().numpy() for n, v in g.items()}, d_o.float().cpu().numpy()
+
+
+def check(got, ref, dtype):
+    for n in ("dq", "dk", "dv", "dla", "dbeta", "dw_text", "dw_vis", "dS0"):
+        x, r = got[n].reshape(ref[n].shape), ref[n]
+        e = rel_l2(x, r)
+        if dtype == "f32":
+            assert e <= 1e-5, f"{n}: rel_l2={e:.3e}"
+        else:
+            m = float(np.abs(x - r).max() / max(np.abs(r).max(), 1e-30))
+            assert e <= 5e-3 and m <= 2e-2, f"{n}: rel_l2={e:.3e} rel max-abs={m:.3e}"
+
+
+def _case(kda, w, seed, causal=False, with_state=True):
+    inp = kda_synth.generate(w, seed)
+    B, N, H, d = inp["shape"]
+    rng = np.random.default_rng(seed)
+    dO = rng.standard_normal((B, N, H, d))
+    S0 = kda_synth.initial_state(seed + 1, B, H, d, d) if with_state else None
+    dSN = rng.standard_normal((B, H, d, d)) * 0.1 if with_state else None
+    got, dO_used = run_bwd(kda, w, inp, dO, S0, dSN, causal)
+    ref = oracle.backward(inp, w.text_len, w.grid, dO_used, S0=S0, dSN=dSN, vis_causal_t=causal)
+    check(got, ref, w.dtype)
+
+
+def test_bwd_tiny_fp32(kda):
+    _case(kda, kda_synth.WORKLOADS[0], 31)
+
+
+@pytest.mark.parametrize("case", ["causal_t", "text_only", "visual_only", "batch2_ragged"])
+def test_bwd_edge_shapes_fp32(kda, case):
+    w = kda_synth.WORKLOADS[0]
+    if case == "causal_t":
+        _case(kda, w, 32, causal=True)
+    elif case == "text_only":
+        _case(kda, dataclasses.replace(w, text_len=77, grid=(0, 0, 0)), 33)
+    elif case == "visual_only":
+        _case(kda, dataclasses.replace(w, text_len=0, grid=(3, 5, 7)), 34, with_state=False)
+    else:
+        _case(kda, dataclasses.replace(w, B=2, text_len=13, grid=(2, 7, 9)), 35)
+
+
+def test_bwd_bf16_d128(kda):
+    """bf16 inputs and gradients, d = 128, several heads: 64 text tokens + a 3 x 8 x 8 grid."""
+    w = kda_synth.Workload("bwd_bf16", 1, 4, 128, 64, (3, 8, 8), "bf16", 0.1)
+    _case(kda, w, 36)
+
+
+def test_bwd_rejects_scan_only_flags(kda):
+    import ctypes
+    w = kda_synth.WORKLOADS[0]
+    p = kda.problem(1, w.H, w.d, w.text_len, w.grid, reuse_records=True)
+    assert kda.kda_bwd_workspace_bytes(p, torch.float32) == 0
+    assert kda._lib.kda_bwd(ctypes.byref(p), 1, *([256] * 19), 1 << 40, None) == kda.KDA_ERR_INVALID_ARG
