@@ -299,6 +299,66 @@ def seq_arm(args, w, idx, rank, world, local_rank):
         print(json.dumps(line), flush=True)
 
 
+def bwd_bytes(w):
+    """Bytes the backward pass must move once: q, k, v, beta, d_o read and dq, dk, dv, dbeta written in
+    the storage dtype, log alpha read and its gradient written in fp32."""
+    e = 2 if w.dtype == "bf16" else 4
+    per_tok = w.H * w.d * (7 * e + 8) + 2 * w.H * e
+    return w.B * w.N * per_tok
+
+
+def bwd_arm(args, w, idx, rank, world, local_rank):
+    """One step = one kda_bwd call (gradients of the whole forward) over the workload."""
+    import torch
+    import linear_attention_video_b200 as kda
+    from tests._util import to_device
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.current_stream(dev)
+    peaks = load_peaks()
+    inp = kda_synth.generate(w, kda_synth.seed_for(idx))
+    B, N, H, d = inp["shape"]
+    t = to_device(inp, dev)
+    dt = t["q"].dtype
+    p = kda.problem(B, H, d, w.text_len, w.grid, chunk=w.chunk, vis_causal_t=args.causal_t)
+    gen = torch.Generator(device=dev).manual_seed(kda_synth.seed_for(idx))
+    d_o = torch.randn(B, N, H, d, device=dev, generator=gen).to(dt)
+    g = [torch.empty(B, N, H, d, dtype=dt, device=dev) for _ in range(3)]
+    dla = torch.empty(B, N, H, d, dtype=torch.float32, device=dev)
+    dbeta = torch.empty(B, N, H, dtype=dt, device=dev)
+    dwt = torch.empty(3, H * d, w.text_k, device=dev)
+    dwv = torch.empty(3, H * d, 27, device=dev)
+    ws = kda.alloc_bwd_workspace(p, dt, dev)
+
+    def step():
+        kda.kda_bwd(p, t["q"], t["k"], t["v"], t["log_alpha"], t["beta"], t["w_text"], t["w_vis"], d_o, *g, dla,
+                    dbeta, dwt, dwv, ws, stream=stream)
+    with ClockSampler(local_rank) as clk:
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
+        launches = kda.kda_last_launch_count()
+        ms = time_calls(step, args.steps, stream)
+    ms = reduce_max(ms, dev, world)
+    hbm = float(peaks["hbm_gbs"])
+    achieved = bwd_bytes(w) / (ms * 1e-3) / 1e9
+    if rank == 0:
+        print(json.dumps({
+            "metric": "KDA+shortconv bwd tokens/sec on 1 B200", "value": w.tokens * world / (ms * 1e-3),
+            "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32 (bf16 storage)" if w.dtype == "bf16" else "f32", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "N": w.N, "H": w.H, "d": w.d, "text_len": w.text_len,
+                       "grid": list(w.grid), "pass": "backward", "parallelism": f"replicas{world}",
+                       "l2": "inputs larger than L2 (no flush)"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                         "traffic": None, "kernel": "kda_bwd (all its kernels)",
+                         "peak_source": peaks["source"] + " hbm_gbs"},
+            "e2e": None, "gpu_launches": launches * args.steps, "clocks": clk.summary(),
+        }), flush=True)
+
+
 def ours_arm(args, w, idx, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -434,6 +494,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--cpu-heads", type=int, default=4, help="heads in the CPU-baseline sample")
+    ap.add_argument("--pass", dest="which", default="fwd", choices=["fwd", "bwd"],
+                    help="bwd: time the backward pass (kda_bwd) instead of the forward")
     ap.add_argument("--shard", default="replicas", choices=["replicas", "seq"],
                     help="replicas: every rank runs the whole workload; seq: the frames are split over the ranks")
     ap.add_argument("--seq-ranks", type=int, default=2, help="--shard seq on one GPU: ranks run as threads")
@@ -455,7 +517,8 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     try:
-        (seq_arm if args.shard == "seq" else ours_arm)(args, w, idx, rank, world, local_rank)
+        arm = bwd_arm if args.which == "bwd" else (seq_arm if args.shard == "seq" else ours_arm)
+        arm(args, w, idx, rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist
