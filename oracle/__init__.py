@@ -294,6 +294,36 @@ def backward(inp: dict, text_len: int, grid, dO, S0=None, dSN=None, text_k=4, vi
     return g
 
 
+def backward_v_columns(inp: dict, text_len: int, grid, dO, items, S0=None, dSN=None, text_k=4, vis_k=(3, 3, 3),
+                       vis_causal_t=False, nthreads=None):
+    """dv[b, :, h, j] (the gradient of the raw v) for each (h, j) in ``items``, at any length.
+
+    Column j of the state, and so of its gradient, only involves column j of v, d_o, S0 and
+    dSN; the conv is depthwise.  So the gradient of v's channel h*d + j comes from the
+    adjoint of a one-column recurrence followed by the transposed conv of that channel.
+    Returns float64 [len(items), B, N]."""
+    B, N, H, d = inp["shape"]
+    shape = conv_shape(B, N, text_len, grid, text_k, vis_k, vis_causal_t)
+    xs = _widened(inp)
+    dO = np.asarray(dO, dtype=np.float64).reshape(B, N, H, d)
+    res = np.zeros((len(items), B, N))
+    by_head = {}
+    for i, (h, j) in enumerate(items):
+        by_head.setdefault(h, []).append((i, j))
+    for h, lst in by_head.items():
+        qh, kh, _, la, bt = _heads_inputs(inp, h, shape, d, nthreads, v_cols=(0, 1), xs=xs)
+        for i, j in lst:
+            c = h * d + j
+            vj = shortconv(shape, xs[2], inp["w_text"][2], inp["w_vis"][2], c, c + 1, nthreads)
+            s0 = None if S0 is None else np.asarray(S0)[:, h, :, j:j + 1]
+            dsn = None if dSN is None else np.asarray(dSN)[:, h, :, j:j + 1]
+            r = scan_bwd(qh, kh, vj, la, bt, dO[:, :, h, j:j + 1], s0, dsn, nthreads)
+            dx, _, _ = shortconv_bwd(shape, xs[2][:, :, c:c + 1], inp["w_text"][2][c:c + 1],
+                                     inp["w_vis"][2][c:c + 1], r["dv"], nthreads)
+            res[i] = dx[:, :, 0]
+    return res
+
+
 # ---------------------------------------------------------------------------
 # Second formulations (numpy, fp64), for cross-checking the recurrence.
 # ---------------------------------------------------------------------------

@@ -101,3 +101,23 @@ def test_bwd_rejects_scan_only_flags(kda):
     p = kda.problem(1, w.H, w.d, w.text_len, w.grid, reuse_records=True)
     assert kda.kda_bwd_workspace_bytes(p, torch.float32) == 0
     assert kda._lib.kda_bwd(ctypes.byref(p), 1, *([256] * 19), 1 << 40, None) == kda.KDA_ERR_INVALID_ARG
+
+
+def test_bwd_bf16_full_size_sampled_v_columns(kda):
+    """Full 5 s video: the gradient of v on sampled channels, which the oracle computes exactly at
+    any length (one state column at a time; the conv is depthwise)."""
+    idx = 2
+    w = kda_synth.WORKLOADS[idx]
+    inp = kda_synth.generate(w, kda_synth.seed_for(idx))
+    B, N, H, d = inp["shape"]
+    rng = np.random.default_rng(5)
+    dO = rng.standard_normal((B, N, H, d)).astype(np.float32)
+    S0 = kda_synth.initial_state(6, B, H, d, d)
+    dSN = (rng.standard_normal((B, H, d, d)) * 0.1).astype(np.float32)
+    got, dO_used = run_bwd(kda, w, inp, dO, S0, dSN)
+    items = [(0, 0), (9, 64), (15, 127)]
+    ref = oracle.backward_v_columns(inp, w.text_len, w.grid, dO_used, items, S0=S0, dSN=dSN)
+    x = np.stack([got["dv"][:, :, h, j] for h, j in items])
+    e = rel_l2(x, ref)
+    m = float(np.abs(x - ref).max() / np.abs(ref).max())
+    assert e <= 5e-3 and m <= 2e-2, f"dv columns: rel_l2={e:.3e} rel max-abs={m:.3e}"

@@ -95,8 +95,8 @@ def test_pipeline_adjoint_matches_directional_derivatives(causal):
     dO, dSN = rng.standard_normal((B, N, H, d)), rng.standard_normal((B, H, d, d))
     S0 = rng.standard_normal((B, H, d, d)) * 0.1
     g = oracle.backward(inp, w.text_len, w.grid, dO, S0=S0, dSN=dSN, vis_causal_t=causal)
-    # inputs are float32 arrays; step along a random direction in fp64 through a float32 copy is
-    # too coarse, so the direction is applied to float64-exact perturbations of a scaled size
+    # the inputs are stored in float32: the perturbed inputs are rounded to float32 and the
+    # step actually taken is measured from the rounded values
     for name, gkey, shape in [("q", "dq", (B, N, H, d)), ("k", "dk", (B, N, H, d)), ("v", "dv", (B, N, H, d)),
                               ("log_alpha", "dla", (B, N, H, d)), ("beta", "dbeta", (B, N, H))]:
         r = rng.standard_normal(shape)
@@ -122,3 +122,19 @@ def test_pipeline_adjoint_matches_directional_derivatives(causal):
     r = rng.standard_normal(S0.shape)
     fd = _pipeline_loss(inp, w, dO, dSN, S0 + 1e-6 * r, causal) - _pipeline_loss(inp, w, dO, dSN, S0 - 1e-6 * r, causal)
     assert abs(fd - 2e-6 * float((g["dS0"] * r).sum())) <= 1e-8 * max(1.0, abs(fd))
+
+
+def test_v_columns_equal_the_full_backward():
+    """The one-column route to dv gives the full backward's dv (the column property the GPU
+    tests rely on at full length)."""
+    w = kda_synth.Workload("bwd_cols", 1, 2, 8, 4, (3, 3, 4), "f32", 0.1)
+    inp = kda_synth.generate(w, 23)
+    B, N, H, d = inp["shape"]
+    rng = np.random.default_rng(4)
+    dO, dSN = rng.standard_normal((B, N, H, d)), rng.standard_normal((B, H, d, d))
+    S0 = rng.standard_normal((B, H, d, d)) * 0.1
+    g = oracle.backward(inp, w.text_len, w.grid, dO, S0=S0, dSN=dSN)
+    items = [(0, 0), (1, 5), (1, 7)]
+    cols = oracle.backward_v_columns(inp, w.text_len, w.grid, dO, items, S0=S0, dSN=dSN)
+    for i, (h, j) in enumerate(items):
+        assert np.allclose(cols[i], g["dv"][:, :, h, j], rtol=1e-12, atol=1e-12)
