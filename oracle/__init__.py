@@ -388,6 +388,75 @@ def chunked_scan(q, k, v, log_alpha, beta, S0=None, chunk=64):
     return o, S
 
 
+def _chunk_terms_bwd(q, k, v, la, beta, S0):
+    """Forward quantities of one chunk in the chunked (UT/WY) form, every pairwise decay
+    exp(g_r - g_i) formed exactly.  Shapes: q, k, la [n, dk], v [n, dv], beta [n], S0 [dk, dv]."""
+    n = k.shape[0]
+    g = np.cumsum(la, axis=0)
+    gl = g[-1]
+    E = np.exp(g[:, None, :] - g[None, :, :])                         # [r, i, c]
+    strict, incl = np.tril(np.ones((n, n)), -1), np.tril(np.ones((n, n)))
+    Ab = np.einsum("rc,ic,ric->ri", k, k, E) * strict                 # A without its beta_r factor
+    P = np.einsum("rc,ic,ric->ri", q, k, E) * incl
+    X = np.linalg.inv(np.eye(n) + beta[:, None] * Ab)                  # (I + A)^{-1}
+    T = X * beta[None, :]
+    KG, QG, Kt = k * np.exp(g), q * np.exp(g), k * np.exp(gl - g)
+    W = T @ KG
+    U = T @ v - W @ S0
+    return dict(g=g, gl=gl, E=E, strict=strict, incl=incl, Ab=Ab, P=P, X=X, T=T, KG=KG, QG=QG, Kt=Kt, W=W, U=U)
+
+
+def chunked_scan_bwd(q, k, v, log_alpha, beta, dO, S0=None, dSN=None, chunk=16):
+    """The backward pass in the chunked form, one head and one batch item, fp64: a second
+    formulation, cross-checked against the token-by-token adjoint (scan_bwd).
+
+    Per chunk, entering with S0: U = T V - W S0, O = QG S0 + P U,
+    S_out = Diag(e^{g_last}) S0 + Kt^T U (the chunked_scan quantities); the chain rule through
+    these, then through T = (I + A)^{-1} Diag(beta), A, P and the exponential factors, gives
+    the chunk's gradients and dS0, which is the gradient reaching the previous chunk's exit.
+    q, k, log_alpha [N, dk]; v, dO [N, dv]; beta [N]; S0, dSN [dk, dv] or None."""
+    q, k, v, la, beta, dO = (np.asarray(a, dtype=np.float64) for a in (q, k, v, log_alpha, beta, dO))
+    N, dk = q.shape
+    dv = v.shape[1]
+    S = [np.zeros((dk, dv)) if S0 is None else np.asarray(S0, dtype=np.float64)]
+    starts = list(range(0, N, chunk))
+    for s in starts:                                                   # entry state of every chunk
+        c = _chunk_terms_bwd(q[s:s + chunk], k[s:s + chunk], v[s:s + chunk], la[s:s + chunk], beta[s:s + chunk],
+                             S[-1])
+        S.append(np.exp(c["gl"])[:, None] * S[-1] + c["Kt"].T @ c["U"])
+    out = {"dq": np.zeros((N, dk)), "dk": np.zeros((N, dk)), "dv": np.zeros((N, dv)), "dla": np.zeros((N, dk)),
+           "dbeta": np.zeros(N)}
+    dS = np.zeros((dk, dv)) if dSN is None else np.asarray(dSN, dtype=np.float64)
+    for ci in range(len(starts) - 1, -1, -1):
+        s = starts[ci]
+        sl = slice(s, s + chunk)
+        Kc, Qc, Vc, bc, dOc, S0c = k[sl], q[sl], v[sl], beta[sl], dO[sl], S[ci]
+        c = _chunk_terms_bwd(Qc, Kc, Vc, la[sl], bc, S0c)
+        g, gl, E, X, T, W, U, P = c["g"], c["gl"], c["E"], c["X"], c["T"], c["W"], c["U"], c["P"]
+        dU = P.T @ dOc + c["Kt"] @ dS
+        dS0 = np.exp(gl)[:, None] * dS + c["QG"].T @ dOc - W.T @ dU
+        dP = (dOc @ U.T) * c["incl"]
+        dQG, dKt, dW = dOc @ S0c.T, U @ dS.T, -dU @ S0c.T
+        dT = dW @ c["KG"].T + dU @ Vc.T
+        dKG = T.T @ dW
+        out["dv"][sl] = T.T @ dU
+        dA = -(X.T @ (dT * bc[None, :]) @ X.T) * c["strict"]
+        out["dbeta"][sl] = np.einsum("ri,ri->i", X, dT) + np.einsum("ri,ri->r", dA, c["Ab"])
+        dAb = dA * bc[:, None]
+        dq = dQG * np.exp(g) + np.einsum("ri,ic,ric->rc", dP, Kc, E)
+        dkk = dKG * np.exp(g) + dKt * np.exp(gl - g)
+        dkk += np.einsum("ri,ic,ric->rc", dAb, Kc, E) + np.einsum("ri,rc,ric->ic", dAb, Kc, E)
+        dkk += np.einsum("ri,rc,ric->ic", dP, Qc, E)
+        dEE = (np.einsum("ri,rc,ic->ric", dAb, Kc, Kc) + np.einsum("ri,rc,ic->ric", dP, Qc, Kc)) * E
+        dg = dEE.sum(axis=1) - dEE.sum(axis=0) + dKG * c["KG"] + dQG * c["QG"] - dKt * c["Kt"]
+        dg[-1] += (dKt * c["Kt"]).sum(axis=0) + (dS * np.exp(gl)[:, None] * S0c).sum(axis=1)
+        out["dla"][sl] = np.cumsum(dg[::-1], axis=0)[::-1]             # g is the running sum of log alpha
+        out["dq"][sl], out["dk"][sl] = dq, dkk
+        dS = dS0
+    out["dS0"] = dS
+    return out
+
+
 def dense_scan(q, k, v, log_alpha, beta):
     """Dense lower-triangular form from a zero state, one head, one batch item.
 

@@ -138,3 +138,19 @@ def test_v_columns_equal_the_full_backward():
     cols = oracle.backward_v_columns(inp, w.text_len, w.grid, dO, items, S0=S0, dSN=dSN)
     for i, (h, j) in enumerate(items):
         assert np.allclose(cols[i], g["dv"][:, :, h, j], rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("chunk", [1, 4, 16, 64])
+def test_chunked_backward_equals_the_token_adjoint(chunk):
+    """A second formulation of the backward (the chain rule through the chunked UT/WY form)
+    agrees with the token-by-token adjoint for any chunk length, ragged last chunk included."""
+    rng = np.random.default_rng(6)
+    N, dk, dv = 37, 6, 5
+    a = _scan_problem(rng, B=1, N=N, dk=dk, dv=dv)
+    dO, dSN = rng.standard_normal((1, N, dv)), rng.standard_normal((1, dk, dv))
+    ref = oracle.scan_bwd(a["q"], a["k"], a["v"], a["la"], a["beta"], dO, a["S0"], dSN)
+    got = oracle.chunked_scan_bwd(a["q"][0], a["k"][0], a["v"][0], a["la"][0], a["beta"][0], dO[0], a["S0"][0],
+                                  dSN[0], chunk=chunk)
+    for n in ("dq", "dk", "dv", "dla", "dbeta", "dS0"):
+        r = ref[n][0]
+        assert np.abs(got[n] - r).max() <= 1e-12 * max(1.0, np.abs(r).max()), n
