@@ -281,10 +281,12 @@ def seq_arm(args, w, idx, rank, world, local_rank):
         e2e = {"value": w.tokens / (ms_e2e * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h}
     # launches per step on this process: conv (text + visual) and three scans per rank
-    launches = 0
-    for r in mine:
-        sg = segs[r]
-        launches += (1 if r == 0 and w.text_len else 0) + 1 + 2 + 1 + 1
+    # kernels one step launches on this process (every rank's backend counts its own)
+    for be in backends.values():
+        be.launches = 0
+    step()
+    torch.cuda.synchronize()
+    launches = sum(be.launches for be in backends.values())
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,

@@ -34,7 +34,8 @@ from dataclasses import dataclass
 
 import torch
 
-from . import (kda_chunk_fwd, kda_shortconv_fwd, problem, alloc_workspace, KdaError, KDA_ERR_INVALID_ARG)
+from . import (kda_chunk_fwd, kda_shortconv_fwd, kda_last_launch_count, problem, alloc_workspace, KdaError,
+               KDA_ERR_INVALID_ARG)
 
 
 # ---------------------------------------------------------------------------
@@ -195,6 +196,7 @@ class GpuBackend:
         self.B, self.H, self.d, self.chunk, self.causal = B, H, d, chunk, vis_causal_t
         self.stream = stream
         self._ws = {}
+        self.launches = 0   # kernels this backend has launched
 
     def _f16(self, dtype):
         return dtype == torch.bfloat16 and self.d == 128
@@ -208,6 +210,7 @@ class GpuBackend:
         out_dtype = torch.float16 if self._f16(q.dtype) else q.dtype
         outs = [torch.empty(q.shape, dtype=out_dtype, device=q.device) for _ in range(3)]
         kda_shortconv_fwd(p, q, k, v, w_text, w_vis, *outs, stream=self.stream)
+        self.launches += kda_last_launch_count()
         return outs
 
     def scan(self, q, k, v, log_alpha, beta, S0, text_len, grid, reuse):
@@ -221,6 +224,7 @@ class GpuBackend:
         SN = torch.empty(self.B, self.H, self.d, self.d, dtype=torch.float32, device=q.device)
         kda_chunk_fwd(self._problem(text_len, grid, dtype, reuse), q, k, v, log_alpha, beta, o, ws, S0, SN,
                       stream=self.stream)
+        self.launches += kda_last_launch_count()
         return o, SN
 
 
