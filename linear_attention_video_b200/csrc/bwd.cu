@@ -333,6 +333,7 @@ __global__ void __launch_bounds__(256) conv_bwd_dx_kernel(ConvBwdArgs a) {
   for (int i = 0; i < 8; ++i) wt[i] = i < a.text_k ? a.w_text[((int64_t)tensor * a.C + c) * a.text_k + i] : 0.f;
   const float* dy = (tensor == 0 ? a.dy[0] : tensor == 1 ? a.dy[1] : a.dy[2]) + b * a.N * a.C + c;
   T* dx = static_cast<T*>(tensor == 0 ? a.dx[0] : tensor == 1 ? a.dx[1] : a.dx[2]) + b * a.N * a.C + c;
+  const int64_t wc = (int64_t)a.Wg * a.C, hwc = wc * a.Hg;   // one grid row, one frame
   const int64_t n1 = min(n0 + CB_TOK, a.N);
   for (int64_t n = n0 + warp; n < n1; n += 8) {
     float acc = 0.f;
@@ -344,18 +345,24 @@ __global__ void __launch_bounds__(256) conv_bwd_dx_kernel(ConvBwdArgs a) {
         if (j < a.text_k && m < a.L) acc += wt[j] * dy[m * a.C];
       }
     } else {
+      // the output at (tt - ta + pt, hh - tb + 1, ww - te + 1) reads this token through tap (ta, tb, te);
+      // its address is this token's plus fixed per-axis offsets
       const TokenPos t = grid_pos(a, n);
+      const float* p = dy + n * a.C;
 #pragma unroll
       for (int ta = 0; ta < 3; ++ta) {
-        const int t2 = t.tt - ta + a.pt;   // output frame that reads this frame through tap ta
+        const int t2 = t.tt - ta + a.pt;
+        if (t2 < 0 || t2 >= a.T) continue;
+        const float* pa = p + (int64_t)(a.pt - ta) * hwc;
 #pragma unroll
         for (int tb = 0; tb < 3; ++tb) {
           const int h2 = t.hh - tb + 1;
+          if (h2 < 0 || h2 >= a.Hg) continue;
+          const float* pb = pa + (int64_t)(1 - tb) * wc;
 #pragma unroll
           for (int te = 0; te < 3; ++te) {
             const int w2 = t.ww - te + 1;
-            if (t2 >= 0 && t2 < a.T && h2 >= 0 && h2 < a.Hg && w2 >= 0 && w2 < a.Wg)
-              acc += wv[(ta * 3 + tb) * 3 + te] * dy[(a.L + ((int64_t)t2 * a.Hg + h2) * a.Wg + w2) * a.C];
+            if (w2 >= 0 && w2 < a.Wg) acc += wv[(ta * 3 + tb) * 3 + te] * pb[(1 - te) * a.C];
           }
         }
       }
@@ -375,6 +382,7 @@ __global__ void __launch_bounds__(256) conv_bwd_dw_kernel(ConvBwdArgs a) {
   const int64_t b = blockIdx.x / bpi, n0 = (blockIdx.x % bpi) * CB_TOK;
   const TIn* x = static_cast<const TIn*>(tensor == 0 ? a.x[0] : tensor == 1 ? a.x[1] : a.x[2]) + b * a.N * a.C + c;
   const float* dy = (tensor == 0 ? a.dy[0] : tensor == 1 ? a.dy[1] : a.dy[2]) + b * a.N * a.C + c;
+  const int64_t wc = (int64_t)a.Wg * a.C, hwc = wc * a.Hg;   // one grid row, one frame
   float av[27], at[8];
 #pragma unroll
   for (int i = 0; i < 27; ++i) av[i] = 0.f;
@@ -390,18 +398,23 @@ __global__ void __launch_bounds__(256) conv_bwd_dw_kernel(ConvBwdArgs a) {
         if (j < a.text_k && s >= 0) at[j] += to_f32(x[s * a.C]) * gv;
       }
     } else {
+      // tap (ta, tb, te) of this output read x at (tt + ta - pt, hh + tb - 1, ww + te - 1)
       const TokenPos t = grid_pos(a, n);
+      const TIn* p = x + n * a.C;
 #pragma unroll
       for (int ta = 0; ta < 3; ++ta) {
         const int t2 = t.tt + ta - a.pt;
+        if (t2 < 0 || t2 >= a.T) continue;
+        const TIn* pa = p + (int64_t)(ta - a.pt) * hwc;
 #pragma unroll
         for (int tb = 0; tb < 3; ++tb) {
           const int h2 = t.hh + tb - 1;
+          if (h2 < 0 || h2 >= a.Hg) continue;
+          const TIn* pb = pa + (int64_t)(tb - 1) * wc;
 #pragma unroll
           for (int te = 0; te < 3; ++te) {
             const int w2 = t.ww + te - 1;
-            if (t2 >= 0 && t2 < a.T && h2 >= 0 && h2 < a.Hg && w2 >= 0 && w2 < a.Wg)
-              av[(ta * 3 + tb) * 3 + te] += to_f32(x[(a.L + ((int64_t)t2 * a.Hg + h2) * a.Wg + w2) * a.C]) * gv;
+            if (w2 >= 0 && w2 < a.Wg) av[(ta * 3 + tb) * 3 + te] += to_f32(pb[(te - 1) * a.C]) * gv;
           }
         }
       }
