@@ -260,11 +260,12 @@ __global__ void __launch_bounds__(DK, 2) bwd_scan_kernel(ScanBwdArgs a) {
       if (i == 0) {
         float db = 0.f;
 #pragma unroll
-        for (int j = 0; j < CWB; ++j) {
-          a.dv[tok * DK + c0 + j] = bt * du[j];
-          db += du[j] * rb[tau * CWB + j];
-        }
+        for (int j = 0; j < CWB; ++j) db += du[j] * rb[tau * CWB + j];
         atomicAdd(a.dbeta + tok, db);
+        float4* dvp = reinterpret_cast<float4*>(a.dv + tok * DK + c0);   // 32-byte aligned: c0 = 8 g
+#pragma unroll
+        for (int q4 = 0; q4 < CWB / 4; ++q4)
+          dvp[q4] = make_float4(bt * du[4 * q4], bt * du[4 * q4 + 1], bt * du[4 * q4 + 2], bt * du[4 * q4 + 3]);
       }
       float dki = 0.f, dlai = 0.f;
 #pragma unroll
