@@ -32,7 +32,7 @@ namespace kda {
 namespace {
 
 constexpr int CWB = 8;    // value columns per CTA of the scan kernels (two CTAs share an SM)
-constexpr int KC = 16;    // tokens between stored states
+constexpr int KC = 8;     // tokens between stored states (and per pipelined chunk of the adjoint kernel)
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -55,13 +55,20 @@ struct ScanBwdArgs {
   int64_t N; int H; int n_ck; bool bf16;
 };
 
-// out[j] = sum over the CTA's DK threads (rows) of x[j], for the CWB columns; every thread gets all
+// Barrier over the DK threads of one row group: the whole CTA (id 0) or a named barrier.
 template <int DK>
-__device__ __forceinline__ void colsum(const float (&x)[CWB], float* red, float* red2, float (&out)[CWB]) {
-  const int i = threadIdx.x;
+__device__ __forceinline__ void group_sync(int id) {
+  if (id == 0) __syncthreads();
+  else asm volatile("bar.sync %0, %1;" :: "r"(id), "r"(DK) : "memory");
+}
+
+// out[j] = sum over a row group's DK threads (row i) of x[j], for the CWB columns; every thread gets all
+template <int DK>
+__device__ __forceinline__ void colsum(const float (&x)[CWB], float* red, float* red2, float (&out)[CWB], int i,
+                                       int bar) {
 #pragma unroll
   for (int j = 0; j < CWB; ++j) red[i * (CWB + 1) + j] = x[j];
-  __syncthreads();
+  group_sync<DK>(bar);
   const int j = i % CWB, part = i / CWB;   // DK / CWB parts of CWB rows
   float s = 0.f;
 #pragma unroll
@@ -69,7 +76,7 @@ __device__ __forceinline__ void colsum(const float (&x)[CWB], float* red, float*
 #pragma unroll
   for (int off = CWB; off < 32; off <<= 1) s += __shfl_xor_sync(0xffffffffu, s, off);   // parts of one warp
   if ((i & 31) < CWB) red2[(i >> 5) * CWB + j] = s;
-  __syncthreads();
+  group_sync<DK>(bar);
 #pragma unroll
   for (int jj = 0; jj < CWB; ++jj) {
     float acc = 0.f;
@@ -83,24 +90,24 @@ __device__ __forceinline__ void colsum(const float (&x)[CWB], float* red, float*
 // each key channel (thread i loads element i of every token) and the CTA's
 // value columns.  Loads for the next chunk are issued into registers before
 // the current chunk is processed, so their latency overlaps its work.
-template <int DK>
+template <int DK, int L = KC>
 struct ChunkIn {
-  float la[KC][DK], k[KC][DK], q[KC][DK];
-  float v[KC][CWB], dout[KC][CWB], beta[KC];
+  float la[L][DK], k[L][DK], q[L][DK];
+  float v[L][CWB], dout[L][CWB], beta[L];
 };
 
-template <int DK>
+template <int DK, int L = KC>
 struct ChunkRegs {
-  float la[KC], k[KC], q[KC], v[KC], dout[KC], beta;
+  float la[L], k[L], q[L], v[L], dout[L], beta;
 };
 
 // thread i: element i of the chunk's rows (zero past the sequence end); threads < CWB also
 // the CTA's value columns, threads < KC the gates
-template <int DK, bool BWD>
-__device__ __forceinline__ void load_chunk(const ScanBwdArgs& a, int b, int h, int c0, int64_t t0, ChunkRegs<DK>& r) {
-  const int i = threadIdx.x;
+template <int DK, bool BWD, int L = KC>
+__device__ __forceinline__ void load_chunk(const ScanBwdArgs& a, int b, int h, int c0, int64_t t0,
+                                           ChunkRegs<DK, L>& r, int i) {
 #pragma unroll
-  for (int tau = 0; tau < KC; ++tau) {
+  for (int tau = 0; tau < L; ++tau) {
     const bool in = t0 + tau < a.N;
     const int64_t tok = ((int64_t)b * a.N + (in ? t0 + tau : 0)) * a.H + h;
     r.la[tau] = in ? a.la[tok * DK + i] : 0.f;
@@ -111,17 +118,16 @@ __device__ __forceinline__ void load_chunk(const ScanBwdArgs& a, int b, int h, i
       if (BWD) r.dout[tau] = in ? ld_act(a.d_o, tok * DK + c0 + i, a.bf16) : 0.f;
     }
   }
-  if (i < KC) {
+  if (i < L) {
     const bool in = t0 + i < a.N;
     r.beta = in ? ld_act(a.beta, ((int64_t)b * a.N + t0 + i) * a.H + h, a.bf16) : 0.f;
   }
 }
 
-template <int DK, bool BWD>
-__device__ __forceinline__ void store_chunk(const ChunkRegs<DK>& r, ChunkIn<DK>& c) {
-  const int i = threadIdx.x;
+template <int DK, bool BWD, int L = KC>
+__device__ __forceinline__ void store_chunk(const ChunkRegs<DK, L>& r, ChunkIn<DK, L>& c, int i) {
 #pragma unroll
-  for (int tau = 0; tau < KC; ++tau) {
+  for (int tau = 0; tau < L; ++tau) {
     c.la[tau][i] = r.la[tau];
     c.k[tau][i] = r.k[tau];
     if (BWD) c.q[tau][i] = r.q[tau];
@@ -130,12 +136,13 @@ __device__ __forceinline__ void store_chunk(const ChunkRegs<DK>& r, ChunkIn<DK>&
       if (BWD) c.dout[tau][i] = r.dout[tau];
     }
   }
-  if (i < KC) c.beta[i] = r.beta;
+  if (i < L) c.beta[i] = r.beta;
 }
 
 template <int DK>
 __global__ void __launch_bounds__(DK) bwd_states_kernel(ScanBwdArgs a) {
-  __shared__ ChunkIn<DK> cin;
+  constexpr int SL = 2 * KC;   // tokens staged per step (two stored states per step)
+  __shared__ ChunkIn<DK, SL> cin;
   __shared__ float red[DK * (CWB + 1)];
   __shared__ float red2[(DK / 32) * CWB];
   const int g = blockIdx.x, h = blockIdx.y, b = blockIdx.z, i = threadIdx.x;
@@ -145,19 +152,22 @@ __global__ void __launch_bounds__(DK) bwd_states_kernel(ScanBwdArgs a) {
 #pragma unroll
   for (int j = 0; j < CWB; ++j) S[j] = a.S0 ? a.S0[srow + j] : 0.f;
   float* ck = a.ckpt + ((int64_t)b * a.H + h) * a.n_ck * DK * DK;
-  ChunkRegs<DK> nxt;
-  load_chunk<DK, false>(a, b, h, c0, 0, nxt);
-  for (int c = 0; c < a.n_ck; ++c) {
-    const int64_t t0 = (int64_t)c * KC;
-    const int nt = (int)min((int64_t)KC, a.N - t0);
-    __syncthreads();   // the previous chunk's inputs are no longer read
-    store_chunk<DK, false>(nxt, cin);
+  const int n_steps = (int)((a.N + SL - 1) / SL);
+  ChunkRegs<DK, SL> nxt;
+  load_chunk<DK, false, SL>(a, b, h, c0, 0, nxt, i);
+  for (int c = 0; c < n_steps; ++c) {
+    const int64_t t0 = (int64_t)c * SL;
+    const int nt = (int)min((int64_t)SL, a.N - t0);
+    __syncthreads();   // the previous step's inputs are no longer read
+    store_chunk<DK, false, SL>(nxt, cin, i);
     __syncthreads();
-    if (c + 1 < a.n_ck) load_chunk<DK, false>(a, b, h, c0, t0 + KC, nxt);
-    float* dst = ck + ((int64_t)c * DK + i) * DK + c0;
-#pragma unroll
-    for (int j = 0; j < CWB; ++j) dst[j] = S[j];
+    if (c + 1 < n_steps) load_chunk<DK, false, SL>(a, b, h, c0, t0 + SL, nxt, i);
     for (int tau = 0; tau < nt; ++tau) {
+      if (tau % KC == 0) {   // the state entering tokens t0 + tau ..
+        float4* dst = reinterpret_cast<float4*>(ck + (((t0 + tau) / KC) * DK + i) * DK + c0);
+#pragma unroll
+        for (int q4 = 0; q4 < CWB / 4; ++q4) dst[q4] = make_float4(S[4 * q4], S[4 * q4 + 1], S[4 * q4 + 2], S[4 * q4 + 3]);
+      }
       const float al = expf(cin.la[tau][i]);
       const float ki = cin.k[tau][i];
       const float bt = cin.beta[tau];
@@ -167,119 +177,147 @@ __global__ void __launch_bounds__(DK) bwd_states_kernel(ScanBwdArgs a) {
         S[j] *= al;
         x[j] = S[j] * ki;
       }
-      colsum<DK>(x, red, red2, sk);
+      colsum<DK>(x, red, red2, sk, i, 0);
 #pragma unroll
       for (int j = 0; j < CWB; ++j) S[j] += ki * (bt * (cin.v[tau][j] - sk[j]));
     }
   }
 }
 
+// The adjoint kernel runs two row groups of DK threads: group 0 recomputes the states (and u, r)
+// of chunk c - 1 from its stored entry state while group 1 applies the adjoint to chunk c, whose
+// states group 0 recomputed in the previous step; the groups meet at one CTA barrier per chunk.
 template <int DK>
-constexpr size_t scan_bwd_smem() {
-  return sizeof(float) * ((size_t)(KC + 1) * DK * CWB + 2 * KC * CWB + DK * (CWB + 1) + (DK / 32) * CWB) +
-         sizeof(ChunkIn<DK>);
-}
+struct ScanBwdSmem {
+  float st[2][KC + 1][DK][CWB];   // per buffer: entry state, then the state after each token
+  float ub[2][KC][CWB];           // u = beta (v - S~^T k)
+  float rb[2][KC][CWB];           // v - S~^T k
+  ChunkIn<DK> in[2];              // inputs of each group's current chunk
+  float red[2][DK * (CWB + 1)];
+  float red2[2][(DK / 32) * CWB];
+};
 
 template <int DK>
-__global__ void __launch_bounds__(DK, 2) bwd_scan_kernel(ScanBwdArgs a) {
-  extern __shared__ float sm[];
-  float* st = sm;                                // [KC + 1][DK][CWB]: st[0] entry state, st[1 + tau] after token tau
-  float* ub = st + (size_t)(KC + 1) * DK * CWB;  // [KC][CWB]: u
-  float* rb = ub + KC * CWB;                     // [KC][CWB]: v - S~^T k
-  float* red = rb + KC * CWB;                    // [DK][CWB + 1]
-  float* red2 = red + DK * (CWB + 1);            // [DK / 32][CWB]
-  ChunkIn<DK>& cin = *reinterpret_cast<ChunkIn<DK>*>(red2 + (DK / 32) * CWB);
-  const int g = blockIdx.x, h = blockIdx.y, b = blockIdx.z, i = threadIdx.x;
+constexpr size_t scan_bwd_smem() { return sizeof(ScanBwdSmem<DK>); }
+
+template <int DK>
+__global__ void __launch_bounds__(2 * DK, 2) bwd_scan_kernel(ScanBwdArgs a) {
+  extern __shared__ __align__(16) unsigned char smraw[];
+  ScanBwdSmem<DK>& sm = *reinterpret_cast<ScanBwdSmem<DK>*>(smraw);
+  const int grp = threadIdx.x / DK, i = threadIdx.x % DK;
+  const int bar = 1 + grp;   // named barrier of the row group
+  const int g = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int c0 = g * CWB;
   const int64_t srow = (((int64_t)b * a.H + h) * DK + i) * DK + c0;
   const float* ck = a.ckpt + ((int64_t)b * a.H + h) * a.n_ck * DK * DK;
-  float dS[CWB];
+  ChunkIn<DK>& cin = sm.in[grp];
+  float* red = sm.red[grp];
+  float* red2 = sm.red2[grp];
+  float dS[CWB];   // group 1: gradient reaching the current chunk's exit state
 #pragma unroll
-  for (int j = 0; j < CWB; ++j) dS[j] = a.dSN ? a.dSN[srow + j] : 0.f;
-  ChunkRegs<DK> nxt;
-  load_chunk<DK, true>(a, b, h, c0, (int64_t)(a.n_ck - 1) * KC, nxt);
-  for (int c = a.n_ck - 1; c >= 0; --c) {
-    const int64_t t0 = (int64_t)c * KC;
-    const int nt = (int)min((int64_t)KC, a.N - t0);
-    __syncthreads();   // the previous chunk's inputs, u and r are no longer read
-    store_chunk<DK, true>(nxt, cin);
-    __syncthreads();
-    if (c > 0) load_chunk<DK, true>(a, b, h, c0, t0 - KC, nxt);
-    // states of the chunk, recomputed from the stored entry state
-    float S[CWB];
-    const float* src = ck + ((int64_t)c * DK + i) * DK + c0;
-#pragma unroll
-    for (int j = 0; j < CWB; ++j) {
-      S[j] = src[j];
-      st[i * CWB + j] = S[j];
-    }
-    for (int tau = 0; tau < nt; ++tau) {
-      const float al = expf(cin.la[tau][i]);
-      const float ki = cin.k[tau][i];
-      const float bt = cin.beta[tau];
-      float x[CWB], sk[CWB];
-#pragma unroll
-      for (int j = 0; j < CWB; ++j) {
-        S[j] *= al;
-        x[j] = S[j] * ki;
+  for (int j = 0; j < CWB; ++j) dS[j] = (grp == 1 && a.dSN) ? a.dSN[srow + j] : 0.f;
+  // step it: group 0 recomputes chunk n_ck - 1 - it, group 1 differentiates chunk n_ck - it
+  ChunkRegs<DK> nxt;   // both groups start with chunk n_ck - 1 (group 1 one step later)
+  if (grp == 0) load_chunk<DK, false>(a, b, h, c0, (int64_t)(a.n_ck - 1) * KC, nxt, i);
+  else load_chunk<DK, true>(a, b, h, c0, (int64_t)(a.n_ck - 1) * KC, nxt, i);
+  for (int it = 0; it <= a.n_ck; ++it) {
+    const int c = grp == 0 ? a.n_ck - 1 - it : a.n_ck - it;
+    const bool active = grp == 0 ? it < a.n_ck : it >= 1;
+    const int buf = grp == 0 ? (it & 1) : ((it - 1) & 1);
+    if (active) {
+      const int64_t t0 = (int64_t)c * KC;
+      const int nt = (int)min((int64_t)KC, a.N - t0);
+      group_sync<DK>(bar);   // the group's previous inputs are no longer read
+      if (grp == 0) store_chunk<DK, false>(nxt, cin, i);
+      else store_chunk<DK, true>(nxt, cin, i);
+      group_sync<DK>(bar);
+      if (c > 0) {
+        if (grp == 0) load_chunk<DK, false>(a, b, h, c0, t0 - KC, nxt, i);
+        else load_chunk<DK, true>(a, b, h, c0, t0 - KC, nxt, i);
       }
-      colsum<DK>(x, red, red2, sk);
-      float* dst = st + ((size_t)(1 + tau) * DK + i) * CWB;
+      float* st = &sm.st[buf][0][0][0];
+      float* ub = &sm.ub[buf][0][0];
+      float* rb = &sm.rb[buf][0][0];
+      if (grp == 0) {
+        // states of chunk c, recomputed from the stored entry state
+        float S[CWB];
+        const float* src = ck + ((int64_t)c * DK + i) * DK + c0;
 #pragma unroll
-      for (int j = 0; j < CWB; ++j) {
-        const float r = cin.v[tau][j] - sk[j];
-        S[j] += ki * (bt * r);
-        dst[j] = S[j];
-        if (i == 0) {
-          ub[tau * CWB + j] = bt * r;
-          rb[tau * CWB + j] = r;
+        for (int j = 0; j < CWB; ++j) {
+          S[j] = src[j];
+          st[i * CWB + j] = S[j];
+        }
+        for (int tau = 0; tau < nt; ++tau) {
+          const float al = expf(cin.la[tau][i]);
+          const float ki = cin.k[tau][i];
+          const float bt = cin.beta[tau];
+          float x[CWB], sk[CWB];
+#pragma unroll
+          for (int j = 0; j < CWB; ++j) {
+            S[j] *= al;
+            x[j] = S[j] * ki;
+          }
+          colsum<DK>(x, red, red2, sk, i, bar);
+          float* dst = st + ((size_t)(1 + tau) * DK + i) * CWB;
+#pragma unroll
+          for (int j = 0; j < CWB; ++j) {
+            const float r = cin.v[tau][j] - sk[j];
+            S[j] += ki * (bt * r);
+            dst[j] = S[j];
+            if (i == 0) {
+              ub[tau * CWB + j] = bt * r;
+              rb[tau * CWB + j] = r;
+            }
+          }
+        }
+      } else {
+        // the adjoint over chunk c, token by token in reverse
+        for (int tau = nt - 1; tau >= 0; --tau) {
+          const int64_t tok = ((int64_t)b * a.N + t0 + tau) * a.H + h;
+          const float al = expf(cin.la[tau][i]);
+          const float ki = cin.k[tau][i];
+          const float qi = cin.q[tau][i];
+          const float bt = cin.beta[tau];
+          const float* sp = st + ((size_t)tau * DK + i) * CWB;         // S_{t-1}
+          const float* sc = st + ((size_t)(tau + 1) * DK + i) * CWB;   // S_t
+          float sv[CWB], G[CWB], x[CWB], du[CWB];
+          float dqi = 0.f;
+#pragma unroll
+          for (int j = 0; j < CWB; ++j) {
+            const float doj = cin.dout[tau][j];
+            sv[j] = al * sp[j];                 // S~
+            G[j] = dS[j] + qi * doj;
+            dqi += sc[j] * doj;
+            x[j] = G[j] * ki;
+          }
+          atomicAdd(a.dq + tok * DK + i, dqi);
+          colsum<DK>(x, red, red2, du, i, bar);
+          if (i == 0) {
+            float db = 0.f;
+#pragma unroll
+            for (int j = 0; j < CWB; ++j) db += du[j] * rb[tau * CWB + j];
+            atomicAdd(a.dbeta + tok, db);
+            float4* dvp = reinterpret_cast<float4*>(a.dv + tok * DK + c0);   // 32-byte aligned: c0 = 8 g
+#pragma unroll
+            for (int q4 = 0; q4 < CWB / 4; ++q4)
+              dvp[q4] = make_float4(bt * du[4 * q4], bt * du[4 * q4 + 1], bt * du[4 * q4 + 2], bt * du[4 * q4 + 3]);
+          }
+          float dki = 0.f, dlai = 0.f;
+#pragma unroll
+          for (int j = 0; j < CWB; ++j) {
+            const float dst = G[j] - bt * ki * du[j];   // dS~
+            dki += G[j] * ub[tau * CWB + j] - bt * sv[j] * du[j];
+            dlai += dst * sv[j];
+            dS[j] = al * dst;
+          }
+          atomicAdd(a.dk + tok * DK + i, dki);
+          atomicAdd(a.dla + tok * DK + i, dlai);
         }
       }
     }
-    __syncthreads();   // u, r of the chunk visible to every thread
-    for (int tau = nt - 1; tau >= 0; --tau) {
-      const int64_t tok = ((int64_t)b * a.N + t0 + tau) * a.H + h;
-      const float al = expf(cin.la[tau][i]);
-      const float ki = cin.k[tau][i];
-      const float qi = cin.q[tau][i];
-      const float bt = cin.beta[tau];
-      const float* sp = st + ((size_t)tau * DK + i) * CWB;         // S_{t-1}
-      const float* sc = st + ((size_t)(tau + 1) * DK + i) * CWB;   // S_t
-      float sv[CWB], G[CWB], x[CWB], du[CWB];
-      float dqi = 0.f;
-#pragma unroll
-      for (int j = 0; j < CWB; ++j) {
-        const float doj = cin.dout[tau][j];
-        sv[j] = al * sp[j];                 // S~
-        G[j] = dS[j] + qi * doj;
-        dqi += sc[j] * doj;
-        x[j] = G[j] * ki;
-      }
-      atomicAdd(a.dq + tok * DK + i, dqi);
-      colsum<DK>(x, red, red2, du);
-      if (i == 0) {
-        float db = 0.f;
-#pragma unroll
-        for (int j = 0; j < CWB; ++j) db += du[j] * rb[tau * CWB + j];
-        atomicAdd(a.dbeta + tok, db);
-        float4* dvp = reinterpret_cast<float4*>(a.dv + tok * DK + c0);   // 32-byte aligned: c0 = 8 g
-#pragma unroll
-        for (int q4 = 0; q4 < CWB / 4; ++q4)
-          dvp[q4] = make_float4(bt * du[4 * q4], bt * du[4 * q4 + 1], bt * du[4 * q4 + 2], bt * du[4 * q4 + 3]);
-      }
-      float dki = 0.f, dlai = 0.f;
-#pragma unroll
-      for (int j = 0; j < CWB; ++j) {
-        const float dst = G[j] - bt * ki * du[j];   // dS~
-        dki += G[j] * ub[tau * CWB + j] - bt * sv[j] * du[j];
-        dlai += dst * sv[j];
-        dS[j] = al * dst;
-      }
-      atomicAdd(a.dk + tok * DK + i, dki);
-      atomicAdd(a.dla + tok * DK + i, dlai);
-    }
+    __syncthreads();   // group 0's states of this step are complete; group 1 is done with the other buffer
   }
-  if (a.dS0)
+  if (grp == 1 && a.dS0)
 #pragma unroll
     for (int j = 0; j < CWB; ++j) a.dS0[srow + j] = dS[j];
 }
@@ -463,7 +501,7 @@ cudaError_t launch_scan_bwd(const ScanBwdArgs& a, const Dims& d, cudaStream_t s)
   if ((e = cudaFuncSetAttribute(bwd_scan_kernel<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
       cudaSuccess)
     return e;
-  bwd_scan_kernel<DK><<<grid, DK, smem, s>>>(a);
+  bwd_scan_kernel<DK><<<grid, 2 * DK, smem, s>>>(a);
   return cudaGetLastError();
 }
 
