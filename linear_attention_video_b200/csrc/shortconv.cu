@@ -27,9 +27,14 @@ namespace {
 
 constexpr int kVisTaps = 27;
 constexpr int CG = 32;            // channels per CTA, one per lane
-constexpr int TH = 4;             // tile rows, two per warp
-constexpr int NRUN = 4;           // runs per tile row
-constexpr int kThreads = 32 * (TH / 2) * NRUN;   // a warp: 32 channels x one run of two rows
+// Small CTAs (two warps) with eight resident per SM measured fastest: 124
+// registers a thread keeps one row of three frames in flight, and many small
+// tiles hide the plane loads better than a few large ones.
+constexpr int TH = 2;             // tile rows
+constexpr int RPT = 1;            // output rows per thread
+constexpr int NRUN = 1;           // runs per tile row
+constexpr int kMinBlocks = 8;     // resident CTAs per SM the register budget is sized for
+constexpr int kThreads = 32 * (TH / RPT) * NRUN;   // a warp: 32 channels x one run of RPT rows
 constexpr int PH = TH + 2;        // plane rows incl. halo
 
 struct ConvArgs {
@@ -101,7 +106,7 @@ template <> __device__ __forceinline__ void store1<float>(float* p, float a) { *
 // predicates); a tile is NRUN runs wide.  Columns past the grid edge read the
 // zero padding of the plane and their outputs are not stored.  PT: temporal
 // offset of the first tap (1 centred, 2 causal).
-constexpr int NSLOT = 4;   // plane slots in shared memory (3 planes in flight)
+constexpr int NSLOT = 3;   // plane slots in shared memory (2 planes in flight)
 
 __device__ __forceinline__ float widen1(__nv_bfloat16 h) { return __bfloat162float(h); }
 __device__ __forceinline__ float widen1(float v) { return v; }
@@ -120,24 +125,24 @@ struct VisPlane {
   static constexpr int BYTES = PH * PWr * CG * (int)sizeof(TIn);
 };
 
-// One plane f: FMAs into the three frames it feeds (two output rows each), then
+// One plane f: FMAs into the three frames it feeds (RPT output rows each), then
 // the completed frame out.  Plane row ir feeds output row orow through tap
 // tb = ir - orow.
 template <typename TIn, typename TOut, int RUN, int PT>
 __device__ __forceinline__ void vis_plane_step(const TIn* pl, bool compute, const float (&wv)[kVisTaps],
-                                               float (&an)[2][RUN], float (&ac)[2][RUN], float (&ap)[2][RUN],
-                                               TOut* yo, int64_t row_stride, bool emit0, bool emit1, int nrun,
+                                               float (&an)[RPT][RUN], float (&ac)[RPT][RUN], float (&ap)[RPT][RUN],
+                                               TOut* yo, int64_t row_stride, bool emit, int nrow, int nrun,
                                                int64_t C) {
   constexpr int PWr = VisPlane<TIn, RUN>::PWr;
   if (compute) {
 #pragma unroll
-    for (int ir = 0; ir < 4; ++ir) {
+    for (int ir = 0; ir < RPT + 2; ++ir) {
       const TIn* src = pl + ir * PWr * CG;
       float in[RUN + 2];
 #pragma unroll
       for (int i = 0; i < RUN + 2; ++i) in[i] = widen1(src[i * CG]);
 #pragma unroll
-      for (int orow = 0; orow < 2; ++orow) {
+      for (int orow = 0; orow < RPT; ++orow) {
         const int tb = ir - orow;
         if (tb < 0 || tb > 2) continue;
 #pragma unroll
@@ -154,8 +159,8 @@ __device__ __forceinline__ void vis_plane_step(const TIn* pl, bool compute, cons
     }
   }
 #pragma unroll
-  for (int orow = 0; orow < 2; ++orow) {
-    if (orow == 0 ? emit0 : emit1) {
+  for (int orow = 0; orow < RPT; ++orow) {
+    if (emit && orow < nrow) {
 #pragma unroll
       for (int i = 0; i < RUN; ++i)
         if (i < nrun) store1<TOut>(yo + orow * row_stride + (int64_t)i * C, ap[orow][i]);
@@ -166,7 +171,7 @@ __device__ __forceinline__ void vis_plane_step(const TIn* pl, bool compute, cons
 }
 
 template <typename TIn, typename TOut, int RUN, int PT>
-__global__ void __launch_bounds__(kThreads, 1) vis_conv_kernel(ConvArgs a) {
+__global__ void __launch_bounds__(kThreads, kMinBlocks) vis_conv_kernel(ConvArgs a) {
   using VP = VisPlane<TIn, RUN>;
   constexpr int PWr = VP::PWr;
   extern __shared__ __align__(128) uint8_t slots[];   // [NSLOT][PH][PWr][CG] of TIn
@@ -185,11 +190,11 @@ __global__ void __launch_bounds__(kThreads, 1) vis_conv_kernel(ConvArgs a) {
   const TIn* x = static_cast<const TIn*>(xs) + ((int64_t)b * a.N + a.L) * C + cg0;
   TOut* y = static_cast<TOut*>(ys) + ((int64_t)b * a.N + a.L) * C + cg0;
 
-  const int row = 2 * (warp % (TH / 2)), run = warp / (TH / 2);   // output rows row, row + 1
+  const int row = RPT * (warp % (TH / RPT)), run = warp / (TH / RPT);   // output rows row .. row + RPT - 1
   const int w0 = run * RUN;
   const int nrun = max(0, min(RUN, TW - w0));
-  const bool active = row < THh && nrun > 0;
-  const bool active1 = row + 1 < THh && nrun > 0;
+  const int nrow = nrun > 0 ? max(0, min(RPT, THh - row)) : 0;   // rows of this thread inside the grid
+  const bool active = nrow > 0;
 
   float wv[kVisTaps];
   {
@@ -227,9 +232,9 @@ __global__ void __launch_bounds__(kThreads, 1) vis_conv_kernel(ConvArgs a) {
     asm volatile("cp.async.commit_group;" ::: "memory");
   };
 
-  float s0[2][RUN], s1[2][RUN], s2[2][RUN];
+  float s0[RPT][RUN], s1[RPT][RUN], s2[RPT][RUN];
 #pragma unroll
-  for (int r = 0; r < 2; ++r)
+  for (int r = 0; r < RPT; ++r)
 #pragma unroll
     for (int i = 0; i < RUN; ++i) { s0[r][i] = 0.f; s1[r][i] = 0.f; s2[r][i] = 0.f; }
   for (int f = 0; f < NSLOT - 1; ++f) issue(f);
@@ -239,7 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1) vis_conv_kernel(ConvArgs a) {
   const int f_end = a.T + (PT == 1 ? 1 : 0);
   const TIn* pl_base = reinterpret_cast<const TIn*>(slots) + (row * PWr + w0) * CG + lane;
   TOut* y_base = y + ((int64_t)(th0 + row) * a.Wg + tw0 + w0) * C + lane;
-  auto step = [&](int f, float (&an)[2][RUN], float (&ac)[2][RUN], float (&ap)[2][RUN]) {
+  auto step = [&](int f, float (&an)[RPT][RUN], float (&ac)[RPT][RUN], float (&ap)[RPT][RUN]) {
     asm volatile("cp.async.wait_group %0;" :: "n"(NSLOT - 2) : "memory");
     __syncthreads();   // plane f in place everywhere; slot (f-1) % NSLOT no longer read
     issue(f + NSLOT - 1);
@@ -247,7 +252,7 @@ __global__ void __launch_bounds__(kThreads, 1) vis_conv_kernel(ConvArgs a) {
     const bool tv = t >= 0 && t < a.T;
     vis_plane_step<TIn, TOut, RUN, PT>(pl_base + (f % NSLOT) * (VP::BYTES / (int)sizeof(TIn)),
                                        active && f < a.T, wv, an, ac, ap, y_base + (int64_t)t * HW * C,
-                                       (int64_t)a.Wg * C, active && tv, active1 && tv, nrun, C);
+                                       (int64_t)a.Wg * C, active && tv, nrow, nrun, C);
   };
   // roles rotate with f % 3: (frame f+PT, f+PT-1, f+PT-2) live in sets ((f+PT)%3, ...)
   for (int f = 0; f < f_end; f += 3) {
