@@ -3,27 +3,34 @@
 // v, log alpha, beta, the conv weights and the initial state.  fp32 on the CUDA
 // cores.
 //
-// Forward step per head (paper.rainbus.top, section 方法步骤详情, step (5)),
-// with S~ = Diag(alpha_t) S_{t-1}:
-//     u = beta_t (v_t - S~^T k_t),   S_t = S~ + k_t u^T,   o_t = S_t^T q_t.
-// Its adjoint, with dS the gradient reaching S_t from later tokens and
-// G = dS + q_t do_t^T:
-//     dq_t = S_t do_t,  du = G^T k_t,  dv_t = beta_t du,  dbeta_t = du . (v_t - S~^T k_t),
-//     dk_t = G u - beta_t S~ du,  dS~ = G - beta_t k_t du^T,
-//     dlog_alpha_t = rowsum(dS~ o S~),  dS_{t-1} = Diag(alpha_t) dS~.
-// Column j of S only sees column j of v, so a CTA owns CWB value columns of
-// one (batch item, head); the column sums of dq, dk, dlog alpha and dbeta are
-// accumulated across CTAs with fp32 reductions in global memory.
+// Forward step per head (paper.rainbus.top, section 方法步骤详情, step (5)):
+//     S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T,   o_t = S_t^T q_t.
+// The backward runs in the chunked (UT/WY) form over CH-token chunks.  With g
+// the running sum of log alpha from the chunk start, gl its last row,
+// KG = k e^g, QG = q e^g, Kt = k e^{gl - g}, A = strict-lower(Diag(beta) (k k^T o e^{g_r - g_i})),
+// P = lower(q k^T o e^{g_r - g_i}), X = (I + A)^{-1}, T = X Diag(beta), W = T KG:
+//     U = T V - W S_in,   O = QG S_in + P U,   S_out = Diag(e^{gl}) S_in + Kt^T U.
+// Its adjoint, chunk by chunk in reverse with dS the gradient reaching S_out:
+//     dU = P^T dO + Kt dS,   dS_in = Diag(e^{gl}) dS + QG^T dO - W^T dU,
+// then the chain rule through U, O, S_out, T, A, P and the exponential factors
+// gives the chunk's dq, dk, dv, dlog alpha and dbeta (no term crosses the
+// chunk boundary except dS).  The pairwise decays e^{g_r - g_i} are split as
+// e^{g_r - g_m} e^{g_m - g_i} around g_m, the running sum at token CH/2 - 1;
+// a chunk whose |g - g_m| exceeds kRange nats sets KDA_ERR_RANGE.
 //
 // Kernels, in launch order:
-//   conv (forward, fp32 out)  q', k', v' recomputed from the raw inputs
-//   bwd_states_kernel         forward recurrence, the state stored every KC tokens
-//   bwd_scan_kernel           per KC-token chunk in reverse: its states recomputed
-//                             from the stored one into shared memory, then the
-//                             adjoint token by token
-//   bwd_beta_kernel           dbeta fp32 -> dtype
-//   conv_bwd_dx_kernel        dx = transpose of the conv applied to dq', dk', dv'
-//   conv_bwd_dw_kernel        dw = sum over tokens of x * dy, per channel and tap
+//   conv (forward, fp32 out)   q', k', v' recomputed from the raw inputs
+//   cbwd_prep_kernel           per chunk: W, U~ = T V, Kt, X, A/beta, e^{gl}, and
+//                              the dO terms Z = P^T dO, Y = QG^T dO
+//   cbwd_fwd_chain_kernel      per CW value columns: S_in of every chunk, U
+//   cbwd_bwd_chain_kernel      per CW value columns, in reverse: dS of every chunk, dU, dS0
+//   cbwd_state_grad_kernel     per chunk: the contractions with S_in and dS
+//                              (dQG, dW, dKt), dP, dU V^T
+//   cbwd_local_grad_kernel     per chunk: dT, the inverse's adjoint, dq, dk, dv,
+//                              dlog alpha, dbeta
+//   bwd_beta_kernel            dbeta fp32 -> dtype
+//   conv_bwd_dx_kernel         dx = transpose of the conv applied to dq', dk', dv'
+//   conv_bwd_dw_kernel         dw = sum over tokens of x * dy, per channel and tap
 #include "common.cuh"
 
 #include <cuda_fp16.h>
@@ -31,8 +38,13 @@
 namespace kda {
 namespace {
 
-constexpr int CWB = 8;    // value columns per CTA of the scan kernels (two CTAs share an SM)
-constexpr int KC = 8;     // tokens between stored states (and per pipelined chunk of the adjoint kernel)
+constexpr int CH = 64;          // tokens per chunk
+constexpr int NT = 256;         // threads of every scan kernel: a 16 x 16 grid (ty, tx)
+constexpr int LDC = CH + 1;     // row stride of CH x CH tiles in shared memory
+constexpr int CW = 16;          // value columns per CTA of the two chains
+constexpr int JB = 32;          // value columns per stage of the state-gradient kernel
+constexpr int LDJ = JB + 1;
+constexpr float kRange = 60.f;  // largest |g - g_m| (nats) of the fp32 factorised decays
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -40,288 +52,674 @@ __device__ __forceinline__ float ld_act(const void* p, int64_t i, bool bf16) {
   return bf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(p)[i]) : static_cast<const float*>(p)[i];
 }
 
-struct ScanBwdArgs {
+__device__ __forceinline__ void cp_async16(float* dst, const float* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" :: "r"((uint32_t)__cvta_generic_to_shared(dst)),
+               "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+// Per chunk-head arrays in the workspace, fp32, chunk-head index (b * H + h) * nc + c.
+struct CbwdBufs {
+  float* W;    // [CH][D]  T KG
+  float* Ut;   // [CH][D]  T V
+  float* Kt;   // [CH][D]  k e^{gl - g}
+  float* Z;    // [CH][D]  P^T dO
+  float* Y;    // [D][D]   QG^T dO
+  float* X;    // [CH][CH] (I + A)^{-1}
+  float* Ab;   // [CH][CH] A / beta_r
+  float* egl;  // [D]      e^{gl}
+  float* S;    // [D][D]   state entering the chunk
+  float* U;    // [CH][D]  U~ - W S
+  float* dS;   // [D][D]   gradient reaching the chunk's exit state
+  float* dU;   // [CH][D]
+  float* dQG;  // [CH][D]  dO S^T
+  float* dW;   // [CH][D]  -dU S^T
+  float* dKt;  // [CH][D]  U dS^T
+  float* dP;   // [CH][CH] lower(dO U^T)
+  float* dUV;  // [CH][CH] dU V^T
+  float* last; // [D]      e^{gl} rowsum(dS o S)
+};
+
+struct CbwdArgs {
   const float* q; const float* k; const float* v;   // convolved activations, fp32 [B][N][H][D]
   const float* la;                                   // [B][N][H][D]
   const void* beta;                                  // [B][N][H], dtype
-  const float* S0;                                   // [B][H][D][D] or null
   const void* d_o;                                   // [B][N][H][D], dtype
+  const float* S0;                                   // [B][H][D][D] or null
   const float* dSN;                                  // [B][H][D][D] or null
-  float* ckpt;                                       // [B][H][n_ck][D][D]: state before token KC c
-  float* dq; float* dk; float* dv;                   // fp32 [B][N][H][D]; dq, dk accumulated
-  float* dla;                                        // fp32 [B][N][H][D], accumulated
-  float* dbeta;                                      // fp32 [B][N][H], accumulated
+  float* dq; float* dk; float* dv;                   // fp32 [B][N][H][D]
+  float* dla;                                        // fp32 [B][N][H][D]
+  float* dbeta;                                      // fp32 [B][N][H]
   float* dS0;                                        // [B][H][D][D] or null
-  int64_t N; int H; int n_ck; bool bf16;
+  CbwdBufs w;
+  int64_t N; int H; int nc; bool bf16;
+  uint32_t* status;
 };
 
-// Barrier over the DK threads of one row group: the whole CTA (id 0) or a named barrier.
-template <int DK>
-__device__ __forceinline__ void group_sync(int id) {
-  if (id == 0) __syncthreads();
-  else asm volatile("bar.sync %0, %1;" :: "r"(id), "r"(DK) : "memory");
-}
-
-// out[j] = sum over a row group's DK threads (row i) of x[j], for the CWB columns; every thread gets all
-template <int DK>
-__device__ __forceinline__ void colsum(const float (&x)[CWB], float* red, float* red2, float (&out)[CWB], int i,
-                                       int bar) {
+// acc[i][j] += sum_{kk < K} A(m_i, kk) B(kk, n_j), m_i = ty + 16 i, n_j = tx + 16 j, with
+// A(m, k) = A[m * am + k * ak] and B(k, n) = B[k * bk + n * bn] in shared memory.  The
+// tiles' odd row strides keep both the row and the column reads free of bank conflicts.
+template <int TM, int TN>
+__device__ __forceinline__ void gemm_acc(float (&acc)[TM][TN], const float* A, int am, int ak, const float* B,
+                                         int bk, int bn, int K, int ty, int tx) {
+  const float* a0 = A + ty * am;
+  const float* b0 = B + tx * bn;
+#pragma unroll 4
+  for (int kk = 0; kk < K; ++kk) {
+    float av[TM], bv[TN];
 #pragma unroll
-  for (int j = 0; j < CWB; ++j) red[i * (CWB + 1) + j] = x[j];
-  group_sync<DK>(bar);
-  const int j = i % CWB, part = i / CWB;   // DK / CWB parts of CWB rows
-  float s = 0.f;
+    for (int i = 0; i < TM; ++i) av[i] = a0[i * 16 * am + kk * ak];
 #pragma unroll
-  for (int r = 0; r < CWB; ++r) s += red[(part * CWB + r) * (CWB + 1) + j];
+    for (int j = 0; j < TN; ++j) bv[j] = b0[kk * bk + j * 16 * bn];
 #pragma unroll
-  for (int off = CWB; off < 32; off <<= 1) s += __shfl_xor_sync(0xffffffffu, s, off);   // parts of one warp
-  if ((i & 31) < CWB) red2[(i >> 5) * CWB + j] = s;
-  group_sync<DK>(bar);
+    for (int i = 0; i < TM; ++i)
 #pragma unroll
-  for (int jj = 0; jj < CWB; ++jj) {
-    float acc = 0.f;
-#pragma unroll
-    for (int w = 0; w < DK / 32; ++w) acc += red2[w * CWB + jj];
-    out[jj] = acc;
+      for (int j = 0; j < TN; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
   }
 }
 
-// Per-token inputs of one KC-token chunk, staged in shared memory: the row of
-// each key channel (thread i loads element i of every token) and the CTA's
-// value columns.  Loads for the next chunk are issued into registers before
-// the current chunk is processed, so their latency overlaps its work.
-template <int DK, int L = KC>
-struct ChunkIn {
-  float la[L][DK], k[L][DK], q[L][DK];
-  float v[L][CWB], dout[L][CWB], beta[L];
-};
-
-template <int DK, int L = KC>
-struct ChunkRegs {
-  float la[L], k[L], q[L], v[L], dout[L], beta;
-};
-
-// thread i: element i of the chunk's rows (zero past the sequence end); threads < CWB also
-// the CTA's value columns, threads < KC the gates
-template <int DK, bool BWD, int L = KC>
-__device__ __forceinline__ void load_chunk(const ScanBwdArgs& a, int b, int h, int c0, int64_t t0,
-                                           ChunkRegs<DK, L>& r, int i) {
+template <int TM, int TN>
+__device__ __forceinline__ void zero(float (&acc)[TM][TN]) {
 #pragma unroll
-  for (int tau = 0; tau < L; ++tau) {
-    const bool in = t0 + tau < a.N;
-    const int64_t tok = ((int64_t)b * a.N + (in ? t0 + tau : 0)) * a.H + h;
-    r.la[tau] = in ? a.la[tok * DK + i] : 0.f;
-    r.k[tau] = in ? a.k[tok * DK + i] : 0.f;
-    if (BWD) r.q[tau] = in ? a.q[tok * DK + i] : 0.f;
-    if (i < CWB) {
-      r.v[tau] = in ? a.v[tok * DK + c0 + i] : 0.f;
-      if (BWD) r.dout[tau] = in ? ld_act(a.d_o, tok * DK + c0 + i, a.bf16) : 0.f;
+  for (int i = 0; i < TM; ++i)
+#pragma unroll
+    for (int j = 0; j < TN; ++j) acc[i][j] = 0.f;
+}
+
+// rows [0, CH) of a [.][D] fp32 matrix whose row r starts at src + r * rs, zero from row n on
+template <int D>
+__device__ __forceinline__ void load_rows(float* dst, int ld, const float* src, int64_t rs, int n, int tid) {
+  for (int idx = tid; idx < CH * D / 4; idx += NT) {
+    const int r = idx / (D / 4), c4 = (idx % (D / 4)) * 4;
+    const float4 x = r < n ? *reinterpret_cast<const float4*>(src + r * rs + c4) : make_float4(0.f, 0.f, 0.f, 0.f);
+    float* d = dst + r * ld + c4;
+    d[0] = x.x; d[1] = x.y; d[2] = x.z; d[3] = x.w;
+  }
+}
+
+// running sum over the chunk's rows, per key channel (threads < D); g_m and g_l per channel
+template <int D>
+__device__ __forceinline__ void chunk_cumsum(float* Gs, float* gm, float* gl, int tid) {
+  constexpr int LDD = D + 1;
+  if (tid < D) {
+    float s = 0.f;
+    for (int r = 0; r < CH; ++r) {
+      s += Gs[r * LDD + tid];
+      Gs[r * LDD + tid] = s;
+      if (r == CH / 2 - 1) gm[tid] = s;
+    }
+    gl[tid] = s;
+  }
+}
+
+struct ChunkPos {
+  int64_t ch;     // chunk-head index
+  int64_t tok0;   // (b * N + n0) * H + h: token row index of the chunk's first token
+  int n;          // tokens in the chunk
+};
+
+__device__ __forceinline__ ChunkPos chunk_pos(const CbwdArgs& a) {
+  const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int64_t n0 = (int64_t)c * CH;
+  ChunkPos p;
+  p.ch = ((int64_t)b * a.H + h) * a.nc + c;
+  p.tok0 = ((int64_t)b * a.N + n0) * a.H + h;
+  p.n = (int)(a.N - n0 < CH ? a.N - n0 : CH);
+  return p;
+}
+
+// ---- per-chunk forward quantities and dO terms ------------------------------------
+template <int D>
+constexpr size_t prep_smem() { return sizeof(float) * (4 * CH * (D + 1) + 2 * CH * LDC + 2 * D + CH); }
+
+template <int D>
+__global__ void __launch_bounds__(NT, 1) cbwd_prep_kernel(CbwdArgs a) {
+  constexpr int LDD = D + 1, TN = D / 16;
+  extern __shared__ float sm[];
+  float* Gs = sm;                 // [CH][LDD] g, later dO
+  float* Kx = Gs + CH * LDD;      // k e^{g - g_m}
+  float* KN = Kx + CH * LDD;      // k e^{g_m - g}, later v
+  float* Qx = KN + CH * LDD;      // q e^{g - g_m}
+  float* As = Qx + CH * LDD;      // [CH][LDC] A, later T
+  float* Ps = As + CH * LDC;      // P
+  float* gm = Ps + CH * LDC;      // [D]
+  float* gl = gm + D;             // [D]
+  float* bs = gl + D;             // [CH] beta
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  const ChunkPos p = chunk_pos(a);
+  const int64_t rs = (int64_t)a.H * D;
+  const float* q = a.q + p.tok0 * D;
+  const float* k = a.k + p.tok0 * D;
+
+  load_rows<D>(Gs, LDD, a.la + p.tok0 * D, rs, p.n, tid);
+  if (tid < CH) bs[tid] = tid < p.n ? ld_act(a.beta, p.tok0 + (int64_t)tid * a.H, a.bf16) : 0.f;
+  __syncthreads();
+  chunk_cumsum<D>(Gs, gm, gl, tid);
+  __syncthreads();
+  bool bad = false;
+  float* Kt = a.w.Kt + p.ch * CH * D;
+  for (int idx = tid; idx < CH * D; idx += NT) {
+    const int r = idx / D, c = idx % D;
+    const float g = Gs[r * LDD + c], x = g - gm[c];
+    bad |= fabsf(x) > kRange;
+    const float kv = r < p.n ? k[r * rs + c] : 0.f, qv = r < p.n ? q[r * rs + c] : 0.f;
+    const float ep = expf(x), en = expf(-x);
+    Kx[r * LDD + c] = kv * ep;
+    KN[r * LDD + c] = kv * en;
+    Qx[r * LDD + c] = qv * ep;
+    Kt[idx] = kv * expf(gl[c] - g);
+  }
+  if (tid < D) a.w.egl[p.ch * D + tid] = expf(gl[tid]);
+  if (__syncthreads_or(bad) && tid == 0) set_status(a.status, KDA_ERR_RANGE);
+
+  {  // A = Diag(beta) strict(Kx KN^T), P = lower(Qx KN^T)
+    float ab[4][4], pp[4][4];
+    zero(ab);
+    zero(pp);
+    gemm_acc<4, 4>(ab, Kx, LDD, 1, KN, 1, LDD, D, ty, tx);
+    gemm_acc<4, 4>(pp, Qx, LDD, 1, KN, 1, LDD, D, ty, tx);
+    float* Abg = a.w.Ab + p.ch * CH * CH;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int r = ty + 16 * i, c = tx + 16 * j;
+        const float abv = c < r ? ab[i][j] : 0.f;
+        As[r * LDC + c] = bs[r] * abv;
+        Abg[r * CH + c] = abv;
+        Ps[r * LDC + c] = c <= r ? pp[i][j] : 0.f;
+      }
+  }
+  __syncthreads();
+  // X = (I + A)^{-1} by forward substitution, one column per thread (threads < CH); the other
+  // threads meanwhile stage v and dO into the tiles the products above no longer read
+  float x[CH];
+  if (tid < CH) {
+#pragma unroll
+    for (int r = 0; r < CH; ++r) {
+      float s0 = r == tid ? 1.f : 0.f, s1 = 0.f;
+#pragma unroll
+      for (int i = 0; i + 1 < r; i += 2) {
+        s0 = fmaf(-As[r * LDC + i], x[i], s0);
+        s1 = fmaf(-As[r * LDC + i + 1], x[i + 1], s1);
+      }
+      if (r & 1) s0 = fmaf(-As[r * LDC + r - 1], x[r - 1], s0);
+      x[r] = s0 + s1;
+    }
+    float* Xg = a.w.X + p.ch * CH * CH;
+#pragma unroll
+    for (int r = 0; r < CH; ++r) Xg[r * CH + tid] = x[r];
+  } else {
+    const int t2 = tid - CH;
+    for (int idx = t2; idx < CH * D; idx += NT - CH) {
+      const int r = idx / D, c = idx % D;
+      const bool in = r < p.n;
+      KN[r * LDD + c] = in ? a.v[(p.tok0 + (int64_t)r * a.H) * D + c] : 0.f;
+      Gs[r * LDD + c] = in ? ld_act(a.d_o, (p.tok0 + (int64_t)r * a.H) * D + c, a.bf16) : 0.f;
     }
   }
-  if (i < L) {
-    const bool in = t0 + i < a.N;
-    r.beta = in ? ld_act(a.beta, ((int64_t)b * a.N + t0 + i) * a.H + h, a.bf16) : 0.f;
-  }
-}
-
-template <int DK, bool BWD, int L = KC>
-__device__ __forceinline__ void store_chunk(const ChunkRegs<DK, L>& r, ChunkIn<DK, L>& c, int i) {
+  __syncthreads();
+  if (tid < CH) {
 #pragma unroll
-  for (int tau = 0; tau < L; ++tau) {
-    c.la[tau][i] = r.la[tau];
-    c.k[tau][i] = r.k[tau];
-    if (BWD) c.q[tau][i] = r.q[tau];
-    if (i < CWB) {
-      c.v[tau][i] = r.v[tau];
-      if (BWD) c.dout[tau][i] = r.dout[tau];
+    for (int r = 0; r < CH; ++r) As[r * LDC + tid] = x[r] * bs[tid];   // T = X Diag(beta)
+  }
+  __syncthreads();
+  {  // W = T Kx Diag(e^{g_m}),  U~ = T V,  Z = P^T dO
+    float acc[4][TN];
+    zero(acc);
+    gemm_acc<4, TN>(acc, As, LDC, 1, Kx, LDD, 1, CH, ty, tx);
+    float* W = a.w.W + p.ch * CH * D;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < TN; ++j) {
+        const int r = ty + 16 * i, c = tx + 16 * j;
+        W[r * D + c] = acc[i][j] * expf(gm[c]);
+      }
+    zero(acc);
+    gemm_acc<4, TN>(acc, As, LDC, 1, KN, LDD, 1, CH, ty, tx);
+    float* Ut = a.w.Ut + p.ch * CH * D;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < TN; ++j) Ut[(ty + 16 * i) * D + tx + 16 * j] = acc[i][j];
+    zero(acc);
+    gemm_acc<4, TN>(acc, Ps, 1, LDC, Gs, LDD, 1, CH, ty, tx);
+    float* Z = a.w.Z + p.ch * CH * D;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < TN; ++j) Z[(ty + 16 * i) * D + tx + 16 * j] = acc[i][j];
+  }
+  {  // Y = QG^T dO = Diag(e^{g_m}) Qx^T dO
+    float acc[D / 16][TN];
+    zero(acc);
+    gemm_acc<D / 16, TN>(acc, Qx, 1, LDD, Gs, LDD, 1, CH, ty, tx);
+    float* Y = a.w.Y + p.ch * D * D;
+#pragma unroll
+    for (int i = 0; i < D / 16; ++i) {
+      const int r = ty + 16 * i;
+      const float e = expf(gm[r]);
+#pragma unroll
+      for (int j = 0; j < TN; ++j) Y[r * D + tx + 16 * j] = acc[i][j] * e;
     }
   }
-  if (i < L) c.beta[i] = r.beta;
 }
 
-template <int DK>
-__global__ void __launch_bounds__(DK) bwd_states_kernel(ScanBwdArgs a) {
-  constexpr int SL = 2 * KC;   // tokens staged per step (two stored states per step)
-  __shared__ ChunkIn<DK, SL> cin;
-  __shared__ float red[DK * (CWB + 1)];
-  __shared__ float red2[(DK / 32) * CWB];
-  const int g = blockIdx.x, h = blockIdx.y, b = blockIdx.z, i = threadIdx.x;
-  const int c0 = g * CWB;
-  const int64_t srow = (((int64_t)b * a.H + h) * DK + i) * DK + c0;
-  float S[CWB];
+// ---- the two serial passes over chunks, CW value columns per CTA ------------------------
+// Column j of the state (and of its gradient) only meets column j of v and dO, so the
+// (b, h) chains split into D / CW independent CTAs.  The next chunk's tiles are copied by
+// cp.async into the other half of a double buffer while the current chunk is processed.
+template <int D, bool BWD>
+constexpr size_t chain_smem() {
+  return sizeof(float) * (2 * 2 * CH * (D + 4) + 2 * CH * CW + (BWD ? 2 * D * CW : 0) + 2 * D + D * (CW + 1) +
+                          CH * (CW + 1));
+}
+
+template <int D, bool BWD>
+__global__ void __launch_bounds__(NT, 1) cbwd_chain_kernel(CbwdArgs a) {
+  constexpr int LDW = D + 4, LDS = CW + 1;
+  extern __shared__ __align__(16) float sm[];
+  float* Wb = sm;                            // [2][CH][LDW] W
+  float* Kb = Wb + 2 * CH * LDW;             // [2][CH][LDW] Kt
+  float* Vb = Kb + 2 * CH * LDW;             // [2][CH][CW]  U~ (forward) or Z (backward) columns
+  float* Yb = Vb + 2 * CH * CW;              // [2][D][CW]   Y columns (backward)
+  float* eb = Yb + (BWD ? 2 * D * CW : 0);   // [2][D]       e^{gl}
+  float* S = eb + 2 * D;                     // [D][LDS]     state (forward) or its gradient (backward)
+  float* Us = S + D * LDS;                   // [CH][LDS]    U or dU
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  const int c0 = blockIdx.x * CW, h = blockIdx.y, b = blockIdx.z;
+  const int64_t bh = (int64_t)b * a.H + h, ch0 = bh * a.nc;
+  const float* init = BWD ? a.dSN : a.S0;
+  for (int idx = tid; idx < D * CW; idx += NT) {
+    const int r = idx / CW, j = idx % CW;
+    S[r * LDS + j] = init ? init[(bh * D + r) * D + c0 + j] : 0.f;
+  }
+  auto issue = [&](int c) {
+    if (c >= 0 && c < a.nc) {
+      const int s = c & 1;
+      const int64_t ch = ch0 + c;
+      const float* W = a.w.W + ch * CH * D;
+      const float* K = a.w.Kt + ch * CH * D;
+      const float* V = (BWD ? a.w.Z : a.w.Ut) + ch * CH * D;
+      for (int i = tid; i < CH * D / 4; i += NT) {
+        const int r = i / (D / 4), c4 = (i % (D / 4)) * 4;
+        cp_async16(Wb + (s * CH + r) * LDW + c4, W + r * D + c4);
+        cp_async16(Kb + (s * CH + r) * LDW + c4, K + r * D + c4);
+      }
+      for (int i = tid; i < CH * CW / 4; i += NT) {
+        const int r = i / (CW / 4), c4 = (i % (CW / 4)) * 4;
+        cp_async16(Vb + (s * CH + r) * CW + c4, V + r * D + c0 + c4);
+      }
+      if (BWD) {
+        const float* Y = a.w.Y + ch * D * D;
+        for (int i = tid; i < D * CW / 4; i += NT) {
+          const int r = i / (CW / 4), c4 = (i % (CW / 4)) * 4;
+          cp_async16(Yb + (s * D + r) * CW + c4, Y + r * D + c0 + c4);
+        }
+      }
+      for (int i = tid; i < D / 4; i += NT) cp_async16(eb + s * D + 4 * i, a.w.egl + ch * D + 4 * i);
+    }
+    cp_async_commit();
+  };
+  issue(BWD ? a.nc - 1 : 0);
+  for (int step = 0; step < a.nc; ++step) {
+    const int c = BWD ? a.nc - 1 - step : step;
+    const int s = c & 1;
+    const int64_t ch = ch0 + c;
+    cp_async_wait_all();
+    __syncthreads();   // chunk c's tiles in place; every thread is done with the other buffer
+    issue(BWD ? c - 1 : c + 1);
+    {  // the state entering the chunk (forward) or the gradient reaching its exit (backward)
+      float* out = (BWD ? a.w.dS : a.w.S) + ch * D * D;
+      for (int idx = tid; idx < D * CW; idx += NT) {
+        const int r = idx / CW, j = idx % CW;
+        out[r * D + c0 + j] = S[r * LDS + j];
+      }
+    }
+    {  // forward: U = U~ - W S;  backward: dU = Z + Kt dS
+      float u[4][1];
+      zero(u);
+      gemm_acc<4, 1>(u, (BWD ? Kb : Wb) + s * CH * LDW, LDW, 1, S, LDS, 1, D, ty, tx);
+      float* out = (BWD ? a.w.dU : a.w.U) + ch * CH * D;
 #pragma unroll
-  for (int j = 0; j < CWB; ++j) S[j] = a.S0 ? a.S0[srow + j] : 0.f;
-  float* ck = a.ckpt + ((int64_t)b * a.H + h) * a.n_ck * DK * DK;
-  const int n_steps = (int)((a.N + SL - 1) / SL);
-  ChunkRegs<DK, SL> nxt;
-  load_chunk<DK, false, SL>(a, b, h, c0, 0, nxt, i);
-  for (int c = 0; c < n_steps; ++c) {
-    const int64_t t0 = (int64_t)c * SL;
-    const int nt = (int)min((int64_t)SL, a.N - t0);
-    __syncthreads();   // the previous step's inputs are no longer read
-    store_chunk<DK, false, SL>(nxt, cin, i);
+      for (int i = 0; i < 4; ++i) {
+        const int r = ty + 16 * i;
+        const float val = BWD ? Vb[(s * CH + r) * CW + tx] + u[i][0] : Vb[(s * CH + r) * CW + tx] - u[i][0];
+        Us[r * LDS + tx] = val;
+        out[r * D + c0 + tx] = val;
+      }
+    }
     __syncthreads();
-    if (c + 1 < n_steps) load_chunk<DK, false, SL>(a, b, h, c0, t0 + SL, nxt, i);
-    for (int tau = 0; tau < nt; ++tau) {
-      if (tau % KC == 0) {   // the state entering tokens t0 + tau ..
-        float4* dst = reinterpret_cast<float4*>(ck + (((t0 + tau) / KC) * DK + i) * DK + c0);
+    {  // forward: S = Diag(e^{gl}) S + Kt^T U;  backward: dS = Diag(e^{gl}) dS - W^T dU + Y
+      float sv[D / 16][1];
+      zero(sv);
+      gemm_acc<D / 16, 1>(sv, (BWD ? Wb : Kb) + s * CH * LDW, 1, LDW, Us, LDS, 1, CH, ty, tx);
 #pragma unroll
-        for (int q4 = 0; q4 < CWB / 4; ++q4) dst[q4] = make_float4(S[4 * q4], S[4 * q4 + 1], S[4 * q4 + 2], S[4 * q4 + 3]);
+      for (int i = 0; i < D / 16; ++i) {
+        const int r = ty + 16 * i;
+        const float prev = eb[s * D + r] * S[r * LDS + tx];
+        S[r * LDS + tx] = BWD ? prev - sv[i][0] + Yb[(s * D + r) * CW + tx] : prev + sv[i][0];
       }
-      const float al = expf(cin.la[tau][i]);
-      const float ki = cin.k[tau][i];
-      const float bt = cin.beta[tau];
-      float x[CWB], sk[CWB];
-#pragma unroll
-      for (int j = 0; j < CWB; ++j) {
-        S[j] *= al;
-        x[j] = S[j] * ki;
-      }
-      colsum<DK>(x, red, red2, sk, i, 0);
-#pragma unroll
-      for (int j = 0; j < CWB; ++j) S[j] += ki * (bt * (cin.v[tau][j] - sk[j]));
+    }
+  }
+  if (BWD && a.dS0) {
+    __syncthreads();
+    for (int idx = tid; idx < D * CW; idx += NT) {
+      const int r = idx / CW, j = idx % CW;
+      a.dS0[(bh * D + r) * D + c0 + j] = S[r * LDS + j];
     }
   }
 }
 
-// The adjoint kernel runs two row groups of DK threads: group 0 recomputes the states (and u, r)
-// of chunk c - 1 from its stored entry state while group 1 applies the adjoint to chunk c, whose
-// states group 0 recomputed in the previous step; the groups meet at one CTA barrier per chunk.
-template <int DK>
-struct ScanBwdSmem {
-  float st[2][KC + 1][DK][CWB];   // per buffer: entry state, then the state after each token
-  float ub[2][KC][CWB];           // u = beta (v - S~^T k)
-  float rb[2][KC][CWB];           // v - S~^T k
-  ChunkIn<DK> in[2];              // inputs of each group's current chunk
-  float red[2][DK * (CWB + 1)];
-  float red2[2][(DK / 32) * CWB];
-};
+// ---- contractions with the chunk's entry state and exit gradient -------------------------
+template <int D>
+constexpr size_t state_grad_smem() { return sizeof(float) * (2 * D * LDJ + 4 * CH * LDJ); }
 
-template <int DK>
-constexpr size_t scan_bwd_smem() { return sizeof(ScanBwdSmem<DK>); }
-
-template <int DK>
-__global__ void __launch_bounds__(2 * DK, 2) bwd_scan_kernel(ScanBwdArgs a) {
-  extern __shared__ __align__(16) unsigned char smraw[];
-  ScanBwdSmem<DK>& sm = *reinterpret_cast<ScanBwdSmem<DK>*>(smraw);
-  const int grp = threadIdx.x / DK, i = threadIdx.x % DK;
-  const int bar = 1 + grp;   // named barrier of the row group
-  const int g = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int c0 = g * CWB;
-  const int64_t srow = (((int64_t)b * a.H + h) * DK + i) * DK + c0;
-  const float* ck = a.ckpt + ((int64_t)b * a.H + h) * a.n_ck * DK * DK;
-  ChunkIn<DK>& cin = sm.in[grp];
-  float* red = sm.red[grp];
-  float* red2 = sm.red2[grp];
-  float dS[CWB];   // group 1: gradient reaching the current chunk's exit state
-#pragma unroll
-  for (int j = 0; j < CWB; ++j) dS[j] = (grp == 1 && a.dSN) ? a.dSN[srow + j] : 0.f;
-  // step it: group 0 recomputes chunk n_ck - 1 - it, group 1 differentiates chunk n_ck - it
-  ChunkRegs<DK> nxt;   // both groups start with chunk n_ck - 1 (group 1 one step later)
-  if (grp == 0) load_chunk<DK, false>(a, b, h, c0, (int64_t)(a.n_ck - 1) * KC, nxt, i);
-  else load_chunk<DK, true>(a, b, h, c0, (int64_t)(a.n_ck - 1) * KC, nxt, i);
-  for (int it = 0; it <= a.n_ck; ++it) {
-    const int c = grp == 0 ? a.n_ck - 1 - it : a.n_ck - it;
-    const bool active = grp == 0 ? it < a.n_ck : it >= 1;
-    const int buf = grp == 0 ? (it & 1) : ((it - 1) & 1);
-    if (active) {
-      const int64_t t0 = (int64_t)c * KC;
-      const int nt = (int)min((int64_t)KC, a.N - t0);
-      group_sync<DK>(bar);   // the group's previous inputs are no longer read
-      if (grp == 0) store_chunk<DK, false>(nxt, cin, i);
-      else store_chunk<DK, true>(nxt, cin, i);
-      group_sync<DK>(bar);
-      if (c > 0) {
-        if (grp == 0) load_chunk<DK, false>(a, b, h, c0, t0 - KC, nxt, i);
-        else load_chunk<DK, true>(a, b, h, c0, t0 - KC, nxt, i);
+template <int D>
+__global__ void __launch_bounds__(NT) cbwd_state_grad_kernel(CbwdArgs a) {
+  constexpr int TN = D / 16;
+  extern __shared__ float sm[];
+  float* S0b = sm;              // [D][LDJ]  S columns j0 .. j0 + JB
+  float* dSb = S0b + D * LDJ;   // [D][LDJ]  dS columns
+  float* dOb = dSb + D * LDJ;   // [CH][LDJ]
+  float* dUb = dOb + CH * LDJ;
+  float* Ub = dUb + CH * LDJ;
+  float* Vb = Ub + CH * LDJ;
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  const ChunkPos p = chunk_pos(a);
+  const float* S = a.w.S + p.ch * D * D;
+  const float* dS = a.w.dS + p.ch * D * D;
+  const float* dU = a.w.dU + p.ch * CH * D;
+  const float* U = a.w.U + p.ch * CH * D;
+  // stage columns [j0, j0 + JB) of the chunk's operands; which ones per pass
+  auto stage = [&](int j0, bool pass2) {
+    __syncthreads();
+    for (int idx = tid; idx < D * JB; idx += NT) {
+      const int r = idx / JB, j = idx % JB;
+      if (!pass2) S0b[r * LDJ + j] = S[r * D + j0 + j];
+      dSb[r * LDJ + j] = dS[r * D + j0 + j];
+    }
+    for (int idx = tid; idx < CH * JB; idx += NT) {
+      const int r = idx / JB, j = idx % JB;
+      const bool in = r < p.n;
+      const int64_t t = (p.tok0 + (int64_t)r * a.H) * D + j0 + j;
+      dOb[r * LDJ + j] = in ? ld_act(a.d_o, t, a.bf16) : 0.f;
+      dUb[r * LDJ + j] = dU[r * D + j0 + j];
+      if (pass2) {
+        Ub[r * LDJ + j] = U[r * D + j0 + j];
+        Vb[r * LDJ + j] = in ? a.v[t] : 0.f;
       }
-      float* st = &sm.st[buf][0][0][0];
-      float* ub = &sm.ub[buf][0][0];
-      float* rb = &sm.rb[buf][0][0];
-      if (grp == 0) {
-        // states of chunk c, recomputed from the stored entry state
-        float S[CWB];
-        const float* src = ck + ((int64_t)c * DK + i) * DK + c0;
+    }
+    __syncthreads();
+  };
+  {  // dQG = dO S^T, dW = -dU S^T, and rowsum(dS o S)
+    float aq[4][TN], aw[4][TN];
+    zero(aq);
+    zero(aw);
+    float lastp = 0.f;
+    for (int j0 = 0; j0 < D; j0 += JB) {
+      stage(j0, false);
+      gemm_acc<4, TN>(aq, dOb, LDJ, 1, S0b, 1, LDJ, JB, ty, tx);
+      gemm_acc<4, TN>(aw, dUb, LDJ, 1, S0b, 1, LDJ, JB, ty, tx);
+      if (tid < D)
+#pragma unroll 8
+        for (int j = 0; j < JB; ++j) lastp = fmaf(dSb[tid * LDJ + j], S0b[tid * LDJ + j], lastp);
+    }
+    float* dQG = a.w.dQG + p.ch * CH * D;
+    float* dW = a.w.dW + p.ch * CH * D;
 #pragma unroll
-        for (int j = 0; j < CWB; ++j) {
-          S[j] = src[j];
-          st[i * CWB + j] = S[j];
-        }
-        for (int tau = 0; tau < nt; ++tau) {
-          const float al = expf(cin.la[tau][i]);
-          const float ki = cin.k[tau][i];
-          const float bt = cin.beta[tau];
-          float x[CWB], sk[CWB];
+    for (int i = 0; i < 4; ++i)
 #pragma unroll
-          for (int j = 0; j < CWB; ++j) {
-            S[j] *= al;
-            x[j] = S[j] * ki;
-          }
-          colsum<DK>(x, red, red2, sk, i, bar);
-          float* dst = st + ((size_t)(1 + tau) * DK + i) * CWB;
+      for (int j = 0; j < TN; ++j) {
+        const int r = ty + 16 * i, c = tx + 16 * j;
+        dQG[r * D + c] = aq[i][j];
+        dW[r * D + c] = -aw[i][j];
+      }
+    if (tid < D) a.w.last[p.ch * D + tid] = lastp * a.w.egl[p.ch * D + tid];
+  }
+  {  // dKt = U dS^T, dP = lower(dO U^T), dU V^T
+    float ak[4][TN], ap[4][4], auv[4][4];
+    zero(ak);
+    zero(ap);
+    zero(auv);
+    for (int j0 = 0; j0 < D; j0 += JB) {
+      stage(j0, true);
+      gemm_acc<4, TN>(ak, Ub, LDJ, 1, dSb, 1, LDJ, JB, ty, tx);
+      gemm_acc<4, 4>(ap, dOb, LDJ, 1, Ub, 1, LDJ, JB, ty, tx);
+      gemm_acc<4, 4>(auv, dUb, LDJ, 1, Vb, 1, LDJ, JB, ty, tx);
+    }
+    float* dKt = a.w.dKt + p.ch * CH * D;
+    float* dP = a.w.dP + p.ch * CH * CH;
+    float* dUV = a.w.dUV + p.ch * CH * CH;
 #pragma unroll
-          for (int j = 0; j < CWB; ++j) {
-            const float r = cin.v[tau][j] - sk[j];
-            S[j] += ki * (bt * r);
-            dst[j] = S[j];
-            if (i == 0) {
-              ub[tau * CWB + j] = bt * r;
-              rb[tau * CWB + j] = r;
-            }
-          }
-        }
-      } else {
-        // the adjoint over chunk c, token by token in reverse
-        for (int tau = nt - 1; tau >= 0; --tau) {
-          const int64_t tok = ((int64_t)b * a.N + t0 + tau) * a.H + h;
-          const float al = expf(cin.la[tau][i]);
-          const float ki = cin.k[tau][i];
-          const float qi = cin.q[tau][i];
-          const float bt = cin.beta[tau];
-          const float* sp = st + ((size_t)tau * DK + i) * CWB;         // S_{t-1}
-          const float* sc = st + ((size_t)(tau + 1) * DK + i) * CWB;   // S_t
-          float sv[CWB], G[CWB], x[CWB], du[CWB];
-          float dqi = 0.f;
+    for (int i = 0; i < 4; ++i) {
+      const int r = ty + 16 * i;
 #pragma unroll
-          for (int j = 0; j < CWB; ++j) {
-            const float doj = cin.dout[tau][j];
-            sv[j] = al * sp[j];                 // S~
-            G[j] = dS[j] + qi * doj;
-            dqi += sc[j] * doj;
-            x[j] = G[j] * ki;
-          }
-          atomicAdd(a.dq + tok * DK + i, dqi);
-          colsum<DK>(x, red, red2, du, i, bar);
-          if (i == 0) {
-            float db = 0.f;
+      for (int j = 0; j < TN; ++j) dKt[r * D + tx + 16 * j] = ak[i][j];
 #pragma unroll
-            for (int j = 0; j < CWB; ++j) db += du[j] * rb[tau * CWB + j];
-            atomicAdd(a.dbeta + tok, db);
-            float4* dvp = reinterpret_cast<float4*>(a.dv + tok * DK + c0);   // 32-byte aligned: c0 = 8 g
+      for (int j = 0; j < 4; ++j) {
+        const int c = tx + 16 * j;
+        dP[r * CH + c] = c <= r ? ap[i][j] : 0.f;
+        dUV[r * CH + c] = auv[i][j];
+      }
+    }
+  }
+}
+
+// ---- the chunk-local part of the adjoint ---------------------------------------------
+template <int D>
+constexpr size_t local_grad_smem() { return sizeof(float) * (4 * CH * (D + 1) + 5 * CH * LDC + 3 * D + 2 * CH); }
+
+template <int D>
+__global__ void __launch_bounds__(NT, 1) cbwd_local_grad_kernel(CbwdArgs a) {
+  constexpr int LDD = D + 1, TN = D / 16;
+  extern __shared__ float sm[];
+  float* Gs = sm;                 // [CH][LDD] g, at the end dg
+  float* Kx = Gs + CH * LDD;      // k e^{g - g_m}
+  float* Fs = Kx + CH * LDD;      // dW e^{g_m}, later q e^{g - g_m}
+  float* Bs = Fs + CH * LDD;      // dU, later k e^{g_m - g}
+  float* Xs = Bs + CH * LDD;      // [CH][LDC] X
+  float* dTs = Xs + CH * LDC;     // dT
+  float* Ms = dTs + CH * LDC;     // X^T dT Diag(beta)
+  float* dPs = Ms + CH * LDC;     // dP
+  float* Abs = dPs + CH * LDC;    // A / beta, later dA Diag... (dAb)
+  float* gm = Abs + CH * LDC;     // [D]
+  float* gl = gm + D;             // [D]
+  float* colk = gl + D;           // [D] column sums of dKt o Kt
+  float* bs = colk + D;           // [CH]
+  float* db = bs + CH;            // [CH] dbeta
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  const ChunkPos p = chunk_pos(a);
+  const int64_t rs = (int64_t)a.H * D;
+  const float* q = a.q + p.tok0 * D;
+  const float* k = a.k + p.tok0 * D;
+  const int64_t cd = p.ch * CH * D, cc = p.ch * CH * CH;
+
+  load_rows<D>(Gs, LDD, a.la + p.tok0 * D, rs, p.n, tid);
+  if (tid < CH) bs[tid] = tid < p.n ? ld_act(a.beta, p.tok0 + (int64_t)tid * a.H, a.bf16) : 0.f;
+  if (tid < D) colk[tid] = 0.f;
+  __syncthreads();
+  chunk_cumsum<D>(Gs, gm, gl, tid);
+  __syncthreads();
+  for (int idx = tid; idx < CH * D; idx += NT) {
+    const int r = idx / D, c = idx % D;
+    const float kv = r < p.n ? k[r * rs + c] : 0.f;
+    Kx[r * LDD + c] = kv * expf(Gs[r * LDD + c] - gm[c]);
+    Fs[r * LDD + c] = a.w.dW[cd + idx] * expf(gm[c]);
+    Bs[r * LDD + c] = a.w.dU[cd + idx];
+  }
+  for (int idx = tid; idx < CH * CH; idx += NT) {
+    const int r = idx / CH, c = idx % CH;
+    Xs[r * LDC + c] = a.w.X[cc + idx];
+    dTs[r * LDC + c] = a.w.dUV[cc + idx];
+    dPs[r * LDC + c] = a.w.dP[cc + idx];
+    Abs[r * LDC + c] = a.w.Ab[cc + idx];
+  }
+  __syncthreads();
+  {  // dT = dW KG^T + dU V^T
+    float t[4][4];
+    zero(t);
+    gemm_acc<4, 4>(t, Fs, LDD, 1, Kx, 1, LDD, D, ty, tx);
 #pragma unroll
-            for (int q4 = 0; q4 < CWB / 4; ++q4)
-              dvp[q4] = make_float4(bt * du[4 * q4], bt * du[4 * q4 + 1], bt * du[4 * q4 + 2], bt * du[4 * q4 + 3]);
-          }
-          float dki = 0.f, dlai = 0.f;
+    for (int i = 0; i < 4; ++i)
 #pragma unroll
-          for (int j = 0; j < CWB; ++j) {
-            const float dst = G[j] - bt * ki * du[j];   // dS~
-            dki += G[j] * ub[tau * CWB + j] - bt * sv[j] * du[j];
-            dlai += dst * sv[j];
-            dS[j] = al * dst;
-          }
-          atomicAdd(a.dk + tok * DK + i, dki);
-          atomicAdd(a.dla + tok * DK + i, dlai);
+      for (int j = 0; j < 4; ++j) dTs[(ty + 16 * i) * LDC + tx + 16 * j] += t[i][j];
+  }
+  // per-thread elements (row ty + 16 i, key channel tx + 16 j) of dq, dk and dg
+  float dq[4][TN], dk[4][TN], dg[4][TN];
+  {  // dv = Diag(beta) X^T dU
+    float acc[4][TN];
+    zero(acc);
+    gemm_acc<4, TN>(acc, Xs, 1, LDC, Bs, LDD, 1, CH, ty, tx);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = ty + 16 * i;
+      if (r < p.n)
+#pragma unroll
+        for (int j = 0; j < TN; ++j) a.dv[(p.tok0 + (int64_t)r * a.H) * D + tx + 16 * j] = bs[r] * acc[i][j];
+    }
+  }
+  {  // dKG = Diag(beta) X^T dW; the dq, dk, dg terms of KG, QG and Kt
+    float acc[4][TN];
+    zero(acc);
+    gemm_acc<4, TN>(acc, Xs, 1, LDC, Fs, LDD, 1, CH, ty, tx);
+    const float* dKt = a.w.dKt + cd;
+    const float* dQG = a.w.dQG + cd;
+#pragma unroll
+    for (int j = 0; j < TN; ++j) {
+      const int c = tx + 16 * j;
+      float ck = 0.f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = ty + 16 * i;
+        const bool in = r < p.n;
+        const float g = Gs[r * LDD + c];
+        const float e1 = expf(g - gm[c]), e2 = expf(gl[c] - g), eg = expf(g);
+        const float kv = in ? k[r * rs + c] : 0.f, qv = in ? q[r * rs + c] : 0.f;
+        const float dkt = dKt[r * D + c], dqg = dQG[r * D + c];
+        const float av = bs[r] * acc[i][j] * e1;   // dKG o e^g
+        dk[i][j] = av + dkt * e2;
+        dq[i][j] = dqg * eg;
+        dg[i][j] = kv * av - kv * e2 * dkt + qv * eg * dqg;
+        ck = fmaf(kv * e2, dkt, ck);
+      }
+      atomicAdd(&colk[c], ck);
+    }
+  }
+  __syncthreads();   // dT complete
+  {  // M = X^T dT Diag(beta); the first dbeta term, colsum(X o dT)
+    float m[4][4];
+    zero(m);
+    gemm_acc<4, 4>(m, Xs, 1, LDC, dTs, LDC, 1, CH, ty, tx);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int c = tx + 16 * j;
+        Ms[(ty + 16 * i) * LDC + c] = m[i][j] * bs[c];
+      }
+    if (tid < CH) {
+      float s = 0.f;
+      for (int r = 0; r < CH; ++r) s = fmaf(Xs[r * LDC + tid], dTs[r * LDC + tid], s);
+      db[tid] = s;
+    }
+  }
+  // q e^{g - g_m} and k e^{g_m - g} replace dW e^{g_m} and dU, whose products are done
+  for (int idx = tid; idx < CH * D; idx += NT) {
+    const int r = idx / D, c = idx % D;
+    const bool in = r < p.n;
+    const float x = Gs[r * LDD + c] - gm[c];
+    Fs[r * LDD + c] = in ? q[r * rs + c] * expf(x) : 0.f;
+    Bs[r * LDD + c] = in ? k[r * rs + c] * expf(-x) : 0.f;
+  }
+  __syncthreads();
+  {  // dA = -strict(M X^T); the second dbeta term, rowsum(dA o A/beta); dAb = Diag(beta) dA
+    float m[4][4];
+    zero(m);
+    gemm_acc<4, 4>(m, Ms, LDC, 1, Xs, 1, LDC, CH, ty, tx);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = ty + 16 * i;
+      float part = 0.f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int c = tx + 16 * j;
+        const float dA = c < r ? -m[i][j] : 0.f;
+        part = fmaf(dA, Abs[r * LDC + c], part);
+        Abs[r * LDC + c] = dA * bs[r];
+      }
+      atomicAdd(&db[r], part);
+    }
+  }
+  __syncthreads();
+  if (tid < p.n) a.dbeta[p.tok0 + (int64_t)tid * a.H] = db[tid];
+  {  // R2 = e^{g - g_m} o (dP KN): dq, and R1 = e^{g - g_m} o (dAb KN): dk
+    float acc[4][TN];
+    zero(acc);
+    gemm_acc<4, TN>(acc, dPs, LDC, 1, Bs, LDD, 1, CH, ty, tx);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < TN; ++j) {
+        const int r = ty + 16 * i, c = tx + 16 * j;
+        const float r2 = acc[i][j] * expf(Gs[r * LDD + c] - gm[c]);
+        const float qv = r < p.n ? q[r * rs + c] : 0.f;
+        dq[i][j] += r2;
+        dg[i][j] = fmaf(qv, r2, dg[i][j]);
+      }
+    zero(acc);
+    gemm_acc<4, TN>(acc, Abs, LDC, 1, Bs, LDD, 1, CH, ty, tx);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < TN; ++j) {
+        const int r = ty + 16 * i, c = tx + 16 * j;
+        const float r1 = acc[i][j] * expf(Gs[r * LDD + c] - gm[c]);
+        const float kv = r < p.n ? k[r * rs + c] : 0.f;
+        dk[i][j] += r1;
+        dg[i][j] = fmaf(kv, r1, dg[i][j]);
+      }
+  }
+  {  // R3 = e^{g_m - g} o (dAb^T Kx + dP^T Qx): dk
+    float acc[4][TN];
+    zero(acc);
+    gemm_acc<4, TN>(acc, Abs, 1, LDC, Kx, LDD, 1, CH, ty, tx);
+    gemm_acc<4, TN>(acc, dPs, 1, LDC, Fs, LDD, 1, CH, ty, tx);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = ty + 16 * i;
+      const bool in = r < p.n;
+#pragma unroll
+      for (int j = 0; j < TN; ++j) {
+        const int c = tx + 16 * j;
+        const float r3 = acc[i][j] * expf(gm[c] - Gs[r * LDD + c]);
+        const float kv = in ? k[r * rs + c] : 0.f;
+        dk[i][j] += r3;
+        dg[i][j] = fmaf(-kv, r3, dg[i][j]);
+        if (in) {
+          const int64_t t = (p.tok0 + (int64_t)r * a.H) * D + c;
+          a.dq[t] = dq[i][j];
+          a.dk[t] = dk[i][j];
         }
       }
     }
-    __syncthreads();   // group 0's states of this step are complete; group 1 is done with the other buffer
   }
-  if (grp == 1 && a.dS0)
+  __syncthreads();   // every read of g is done: Gs takes dg
 #pragma unroll
-    for (int j = 0; j < CWB; ++j) a.dS0[srow + j] = dS[j];
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < TN; ++j) Gs[(ty + 16 * i) * LDD + tx + 16 * j] = dg[i][j];
+  __syncthreads();
+  if (tid < D) {   // dlog alpha = reverse running sum of dg; the exit terms enter at the last row
+    float s = colk[tid] + a.w.last[p.ch * D + tid];
+    for (int r = CH - 1; r >= 0; --r) {
+      s += Gs[r * LDD + tid];
+      if (r < p.n) a.dla[(p.tok0 + (int64_t)r * a.H) * D + tid] = s;
+    }
+  }
 }
-
 template <typename T>
 __global__ void bwd_beta_kernel(const float* src, T* dst, int64_t n) {
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -476,32 +874,60 @@ __global__ void __launch_bounds__(256) conv_bwd_dw_kernel(ConvBwdArgs a) {
 }
 
 struct BwdLayout {
-  size_t act32, dbeta, ckpt, total;
-  int n_ck;
+  size_t act32, dbeta, cd, cc, dd, d1, total;
+  int nc;
 };
 
+// workspace: status word, q', k', v', dq', dk', dv' (fp32), dbeta (fp32), then the per
+// chunk-head arrays of CbwdBufs
 BwdLayout bwd_layout(const Dims& d) {
   BwdLayout l;
   const size_t elems = (size_t)d.B * d.N * d.H * d.dk;
   l.act32 = align256(elems * sizeof(float));
   l.dbeta = align256((size_t)d.B * d.N * d.H * sizeof(float));
-  l.n_ck = (int)((d.N + KC - 1) / KC);
-  l.ckpt = align256((size_t)d.B * d.H * l.n_ck * d.dk * d.dk * sizeof(float));
-  l.total = 256 + 6 * l.act32 + l.dbeta + l.ckpt;
+  l.nc = (int)((d.N + CH - 1) / CH);
+  const size_t nch = (size_t)d.B * d.H * l.nc;
+  l.cd = align256(nch * CH * d.dk * sizeof(float));
+  l.cc = align256(nch * CH * CH * sizeof(float));
+  l.dd = align256(nch * d.dk * d.dk * sizeof(float));
+  l.d1 = align256(nch * d.dk * sizeof(float));
+  l.total = 256 + 6 * l.act32 + l.dbeta + 9 * l.cd + 4 * l.cc + 3 * l.dd + 2 * l.d1;
   return l;
 }
 
-template <int DK>
-cudaError_t launch_scan_bwd(const ScanBwdArgs& a, const Dims& d, cudaStream_t s) {
-  const dim3 grid((unsigned)(DK / CWB), (unsigned)d.H, (unsigned)d.B);
-  bwd_states_kernel<DK><<<grid, DK, 0, s>>>(a);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  constexpr size_t smem = scan_bwd_smem<DK>();
-  if ((e = cudaFuncSetAttribute(bwd_scan_kernel<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
-      cudaSuccess)
-    return e;
-  bwd_scan_kernel<DK><<<grid, 2 * DK, smem, s>>>(a);
+CbwdBufs carve(const BwdLayout& l, char* p) {
+  CbwdBufs w;
+  float** cd[] = {&w.W, &w.Ut, &w.Kt, &w.Z, &w.U, &w.dU, &w.dQG, &w.dW, &w.dKt};
+  for (float** x : cd) { *x = reinterpret_cast<float*>(p); p += l.cd; }
+  float** cc[] = {&w.X, &w.Ab, &w.dP, &w.dUV};
+  for (float** x : cc) { *x = reinterpret_cast<float*>(p); p += l.cc; }
+  float** dd[] = {&w.Y, &w.S, &w.dS};
+  for (float** x : dd) { *x = reinterpret_cast<float*>(p); p += l.dd; }
+  w.egl = reinterpret_cast<float*>(p); p += l.d1;
+  w.last = reinterpret_cast<float*>(p);
+  return w;
+}
+
+template <typename K>
+cudaError_t set_smem(K kernel, size_t bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+template <int D>
+cudaError_t launch_scan_bwd(const CbwdArgs& a, const Dims& d, cudaStream_t s) {
+  cudaError_t e;
+  const dim3 chunks((unsigned)a.nc, (unsigned)d.H, (unsigned)d.B);
+  const dim3 cols((unsigned)(D / CW), (unsigned)d.H, (unsigned)d.B);
+  if ((e = set_smem(cbwd_prep_kernel<D>, prep_smem<D>())) != cudaSuccess) return e;
+  cbwd_prep_kernel<D><<<chunks, NT, prep_smem<D>(), s>>>(a);
+  if ((e = set_smem(cbwd_chain_kernel<D, false>, chain_smem<D, false>())) != cudaSuccess) return e;
+  cbwd_chain_kernel<D, false><<<cols, NT, chain_smem<D, false>(), s>>>(a);
+  if ((e = set_smem(cbwd_chain_kernel<D, true>, chain_smem<D, true>())) != cudaSuccess) return e;
+  cbwd_chain_kernel<D, true><<<cols, NT, chain_smem<D, true>(), s>>>(a);
+  if ((e = set_smem(cbwd_state_grad_kernel<D>, state_grad_smem<D>())) != cudaSuccess) return e;
+  cbwd_state_grad_kernel<D><<<chunks, NT, state_grad_smem<D>(), s>>>(a);
+  if ((e = set_smem(cbwd_local_grad_kernel<D>, local_grad_smem<D>())) != cudaSuccess) return e;
+  cbwd_local_grad_kernel<D><<<chunks, NT, local_grad_smem<D>(), s>>>(a);
   return cudaGetLastError();
 }
 
@@ -529,9 +955,7 @@ cudaError_t launch_bwd(const Dims& d, kda_dtype dt, const void* q, const void* k
   float* act[6];
   for (int i = 0; i < 6; ++i) act[i] = reinterpret_cast<float*>(base + i * l.act32);   // q', k', v', dq', dk', dv'
   float* dbeta32 = reinterpret_cast<float*>(base + 6 * l.act32);
-  float* ckpt = reinterpret_cast<float*>(base + 6 * l.act32 + l.dbeta);
   const int C = d.H * d.dk;
-  const size_t elems = (size_t)d.B * d.N * d.H * d.dk;
   cudaError_t e;
   if ((e = cudaMemsetAsync(dw_text, 0, sizeof(float) * 3 * C * d.text_k, s)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(dw_vis, 0, sizeof(float) * 3 * C * 27, s)) != cudaSuccess) return e;
@@ -540,17 +964,17 @@ cudaError_t launch_bwd(const Dims& d, kda_dtype dt, const void* q, const void* k
     const size_t bytes = (size_t)d.B * d.H * d.dk * d.dv * sizeof(float);
     return dSN ? cudaMemcpyAsync(dS0, dSN, bytes, cudaMemcpyDeviceToDevice, s) : cudaMemsetAsync(dS0, 0, bytes, s);
   }
-  for (int i = 3; i < 5; ++i)
-    if ((e = cudaMemsetAsync(act[i], 0, elems * sizeof(float), s)) != cudaSuccess) return e;   // dq', dk'
-  if ((e = cudaMemsetAsync(dla, 0, elems * sizeof(float), s)) != cudaSuccess) return e;
-  if ((e = cudaMemsetAsync(dbeta32, 0, (size_t)d.B * d.N * d.H * sizeof(float), s)) != cudaSuccess) return e;
   // 1. the convolved activations, fp32
   if ((e = launch_shortconv(d, dt, q, k, v, w_text, w_vis, act[0], act[1], act[2], s, launches, false, true)) !=
       cudaSuccess)
     return e;
-  // 2. scan backward
-  ScanBwdArgs a{act[0], act[1], act[2], log_alpha, beta, S0, d_o, dSN, ckpt, act[3], act[4], act[5], dla, dbeta32,
-                dS0, d.N, d.H, l.n_ck, dt == KDA_DT_BF16};
+  // 2. scan backward, chunked
+  CbwdArgs a;
+  a.q = act[0]; a.k = act[1]; a.v = act[2]; a.la = log_alpha; a.beta = beta; a.d_o = d_o; a.S0 = S0; a.dSN = dSN;
+  a.dq = act[3]; a.dk = act[4]; a.dv = act[5]; a.dla = dla; a.dbeta = dbeta32; a.dS0 = dS0;
+  a.w = carve(l, base + 6 * l.act32 + l.dbeta);
+  a.N = d.N; a.H = d.H; a.nc = l.nc; a.bf16 = dt == KDA_DT_BF16;
+  a.status = static_cast<uint32_t*>(ws);
   e = d.dk == 128 ? launch_scan_bwd<128>(a, d, s) : launch_scan_bwd<64>(a, d, s);
   if (e != cudaSuccess) return e;
   const int64_t nb = (int64_t)d.B * d.N * d.H;
@@ -568,7 +992,7 @@ cudaError_t launch_bwd(const Dims& d, kda_dtype dt, const void* q, const void* k
   c.N = d.N; c.L = d.L; c.B = d.B; c.C = C; c.text_k = d.text_k; c.T = d.T; c.Hg = d.Hg; c.Wg = d.Wg; c.pt = d.pt;
   e = dt == KDA_DT_BF16 ? launch_conv_bwd<__nv_bfloat16>(c, d, s) : launch_conv_bwd<float>(c, d, s);
   if (e != cudaSuccess) return e;
-  if (launches) *launches += 2 + 1 + 2;
+  if (launches) *launches += 5 + 1 + 2;
   return cudaSuccess;
 }
 
