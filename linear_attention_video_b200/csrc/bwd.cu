@@ -29,8 +29,10 @@
 //   cbwd_local_grad_kernel     per chunk: dT, the inverse's adjoint, dq, dk, dv,
 //                              dlog alpha, dbeta
 //   bwd_beta_kernel            dbeta fp32 -> dtype
-//   conv_bwd_dx_kernel         dx = transpose of the conv applied to dq', dk', dv'
-//   conv_bwd_dw_kernel         dw = sum over tokens of x * dy, per channel and tap
+//   conv_bwd_dx_kernel         text tokens: dx = transpose of the causal 1D conv
+//   conv_bwd_dw_kernel         text tokens: dw = sum over tokens of x * dy per tap
+//   vis_conv_kernel (FLIP)     visual tokens: dx = the conv with reversed taps
+//   vis_dw_kernel              visual tokens: dw, on the forward conv's tiles
 #include "common.cuh"
 
 #include <cuda_fp16.h>
@@ -726,150 +728,78 @@ __global__ void bwd_beta_kernel(const float* src, T* dst, int64_t n) {
   if (i < n) dst[i] = from_f32<T>(src[i]);
 }
 
-// ---- conv backward ------------------------------------------------------------
+// ---- conv backward, text tokens --------------------------------------------------
+// (the visual tokens' dx and dw run on the forward conv's tiles: launch_shortconv_bwd_vis)
 struct ConvBwdArgs {
   const void* x[3];          // raw inputs, dtype [B][N][C]
   const float* dy[3];        // gradients of the conv outputs, fp32 [B][N][C]
   void* dx[3];               // dtype [B][N][C]
   const float* w_text;       // [3][C][text_k]
-  const float* w_vis;        // [3][C][27]
   float* dw_text;            // [3][C][text_k], accumulated
-  float* dw_vis;             // [3][C][27], accumulated
   int64_t N, L;
-  int B, C, text_k, T, Hg, Wg, pt;
+  int B, C, text_k;
 };
 
-// Both conv backward kernels: a CTA covers CB_TOK tokens of one batch item and 32 channels of
-// one tensor (one per lane; 8 warps split the tokens), the channel's taps in registers.
+// A CTA covers CB_TOK text tokens of one batch item and 32 channels of one tensor (one per
+// lane; 8 warps split the tokens), the channel's taps in registers.
 constexpr int CB_TOK = 256;
 
-struct TokenPos {   // visual token n >= L of a batch item: its grid position
-  int tt, hh, ww;
-};
-__device__ __forceinline__ TokenPos grid_pos(const ConvBwdArgs& a, int64_t n) {
-  const int p = (int)(n - a.L), hw = a.Hg * a.Wg;
-  TokenPos t;
-  t.tt = p / hw;
-  const int rem = p - t.tt * hw;
-  t.hh = rem / a.Wg;
-  t.ww = rem - t.hh * a.Wg;
-  return t;
-}
-
-// dx = every output that read x, times its tap weight (the transpose of the conv)
+// dx = every text output that read x, times its tap weight (the transpose of the causal conv)
 template <typename T>
 __global__ void __launch_bounds__(256) conv_bwd_dx_kernel(ConvBwdArgs a) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, tensor = blockIdx.z;
   const int c = blockIdx.y * 32 + lane;
-  const int64_t bpi = (a.N + CB_TOK - 1) / CB_TOK;
+  const int64_t bpi = (a.L + CB_TOK - 1) / CB_TOK;
   const int64_t b = blockIdx.x / bpi, n0 = (blockIdx.x % bpi) * CB_TOK;
-  float wv[27], wt[8];
-#pragma unroll
-  for (int i = 0; i < 27; ++i) wv[i] = a.w_vis[((int64_t)tensor * a.C + c) * 27 + i];
+  float wt[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) wt[i] = i < a.text_k ? a.w_text[((int64_t)tensor * a.C + c) * a.text_k + i] : 0.f;
   const float* dy = (tensor == 0 ? a.dy[0] : tensor == 1 ? a.dy[1] : a.dy[2]) + b * a.N * a.C + c;
   T* dx = static_cast<T*>(tensor == 0 ? a.dx[0] : tensor == 1 ? a.dx[1] : a.dx[2]) + b * a.N * a.C + c;
-  const int64_t wc = (int64_t)a.Wg * a.C, hwc = wc * a.Hg;   // one grid row, one frame
-  const int64_t n1 = min(n0 + CB_TOK, a.N);
+  const int64_t n1 = min(n0 + CB_TOK, a.L);
   for (int64_t n = n0 + warp; n < n1; n += 8) {
+    // y[m] reads x[m - (K-1) + j]: x[n] feeds the text outputs m = n + K-1-j < L
     float acc = 0.f;
-    if (n < a.L) {
-      // y[m] reads x[m - (K-1) + j]: x[n] feeds the text outputs m = n + K-1-j < L
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int64_t m = n + (a.text_k - 1) - j;
-        if (j < a.text_k && m < a.L) acc += wt[j] * dy[m * a.C];
-      }
-    } else {
-      // the output at (tt - ta + pt, hh - tb + 1, ww - te + 1) reads this token through tap (ta, tb, te);
-      // its address is this token's plus fixed per-axis offsets
-      const TokenPos t = grid_pos(a, n);
-      const float* p = dy + n * a.C;
-#pragma unroll
-      for (int ta = 0; ta < 3; ++ta) {
-        const int t2 = t.tt - ta + a.pt;
-        if (t2 < 0 || t2 >= a.T) continue;
-        const float* pa = p + (int64_t)(a.pt - ta) * hwc;
-#pragma unroll
-        for (int tb = 0; tb < 3; ++tb) {
-          const int h2 = t.hh - tb + 1;
-          if (h2 < 0 || h2 >= a.Hg) continue;
-          const float* pb = pa + (int64_t)(1 - tb) * wc;
-#pragma unroll
-          for (int te = 0; te < 3; ++te) {
-            const int w2 = t.ww - te + 1;
-            if (w2 >= 0 && w2 < a.Wg) acc += wv[(ta * 3 + tb) * 3 + te] * pb[(1 - te) * a.C];
-          }
-        }
-      }
+    for (int j = 0; j < 8; ++j) {
+      const int64_t m = n + (a.text_k - 1) - j;
+      if (j < a.text_k && m < a.L) acc += wt[j] * dy[m * a.C];
     }
     dx[n * a.C] = from_f32<T>(acc);
   }
 }
 
-// dw = sum over tokens of x * dy per channel and tap: per-warp sums meet in shared memory, then
-// one atomic add per (channel, tap) and CTA
+// dw_text = sum over text tokens of x * dy per channel and tap: per-warp sums meet in shared
+// memory, then one atomic add per (channel, tap) and CTA
 template <typename TIn>
 __global__ void __launch_bounds__(256) conv_bwd_dw_kernel(ConvBwdArgs a) {
-  __shared__ float part[8][35][32];
+  __shared__ float part[8][8][32];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, tensor = blockIdx.z;
   const int c = blockIdx.y * 32 + lane;
-  const int64_t bpi = (a.N + CB_TOK - 1) / CB_TOK;
+  const int64_t bpi = (a.L + CB_TOK - 1) / CB_TOK;
   const int64_t b = blockIdx.x / bpi, n0 = (blockIdx.x % bpi) * CB_TOK;
   const TIn* x = static_cast<const TIn*>(tensor == 0 ? a.x[0] : tensor == 1 ? a.x[1] : a.x[2]) + b * a.N * a.C + c;
   const float* dy = (tensor == 0 ? a.dy[0] : tensor == 1 ? a.dy[1] : a.dy[2]) + b * a.N * a.C + c;
-  const int64_t wc = (int64_t)a.Wg * a.C, hwc = wc * a.Hg;   // one grid row, one frame
-  float av[27], at[8];
-#pragma unroll
-  for (int i = 0; i < 27; ++i) av[i] = 0.f;
+  float at[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) at[i] = 0.f;
-  const int64_t n1 = min(n0 + CB_TOK, a.N);
+  const int64_t n1 = min(n0 + CB_TOK, a.L);
   for (int64_t n = n0 + warp; n < n1; n += 8) {
     const float gv = dy[n * a.C];
-    if (n < a.L) {
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int64_t s = n - (a.text_k - 1) + j;
-        if (j < a.text_k && s >= 0) at[j] += to_f32(x[s * a.C]) * gv;
-      }
-    } else {
-      // tap (ta, tb, te) of this output read x at (tt + ta - pt, hh + tb - 1, ww + te - 1)
-      const TokenPos t = grid_pos(a, n);
-      const TIn* p = x + n * a.C;
-#pragma unroll
-      for (int ta = 0; ta < 3; ++ta) {
-        const int t2 = t.tt + ta - a.pt;
-        if (t2 < 0 || t2 >= a.T) continue;
-        const TIn* pa = p + (int64_t)(ta - a.pt) * hwc;
-#pragma unroll
-        for (int tb = 0; tb < 3; ++tb) {
-          const int h2 = t.hh + tb - 1;
-          if (h2 < 0 || h2 >= a.Hg) continue;
-          const TIn* pb = pa + (int64_t)(tb - 1) * wc;
-#pragma unroll
-          for (int te = 0; te < 3; ++te) {
-            const int w2 = t.ww + te - 1;
-            if (w2 >= 0 && w2 < a.Wg) av[(ta * 3 + tb) * 3 + te] += to_f32(pb[(te - 1) * a.C]) * gv;
-          }
-        }
-      }
+    for (int j = 0; j < 8; ++j) {
+      const int64_t s = n - (a.text_k - 1) + j;
+      if (j < a.text_k && s >= 0) at[j] += to_f32(x[s * a.C]) * gv;
     }
   }
 #pragma unroll
-  for (int i = 0; i < 27; ++i) part[warp][i][lane] = av[i];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) part[warp][27 + i][lane] = at[i];
+  for (int i = 0; i < 8; ++i) part[warp][i][lane] = at[i];
   __syncthreads();
-  for (int e = threadIdx.x; e < 35 * 32; e += 256) {
-    const int i = e / 32, l = e % 32;
+  if (warp < a.text_k) {
     float s = 0.f;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) s += part[w][i][l];
-    const int cc = blockIdx.y * 32 + l;
-    if (i < 27) atomicAdd(a.dw_vis + ((int64_t)tensor * a.C + cc) * 27 + i, s);
-    else if (i - 27 < a.text_k) atomicAdd(a.dw_text + ((int64_t)tensor * a.C + cc) * a.text_k + (i - 27), s);
+    for (int w = 0; w < 8; ++w) s += part[w][warp][lane];
+    atomicAdd(a.dw_text + ((int64_t)tensor * a.C + c) * a.text_k + warp, s);
   }
 }
 
@@ -933,7 +863,8 @@ cudaError_t launch_scan_bwd(const CbwdArgs& a, const Dims& d, cudaStream_t s) {
 
 template <typename T>
 cudaError_t launch_conv_bwd(const ConvBwdArgs& c, const Dims& d, cudaStream_t s) {
-  const dim3 grid((unsigned)(d.B * ((d.N + CB_TOK - 1) / CB_TOK)), (unsigned)(c.C / 32), 3);
+  if (d.L <= 0) return cudaSuccess;
+  const dim3 grid((unsigned)(d.B * ((d.L + CB_TOK - 1) / CB_TOK)), (unsigned)(c.C / 32), 3);
   conv_bwd_dx_kernel<T><<<grid, 256, 0, s>>>(c);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -983,16 +914,17 @@ cudaError_t launch_bwd(const Dims& d, kda_dtype dt, const void* q, const void* k
   else
     bwd_beta_kernel<float><<<(unsigned)((nb + 255) / 256), 256, 0, s>>>(dbeta32, static_cast<float*>(dbeta), nb);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  // 3. conv backward
+  // 3. conv backward: text tokens here, visual tokens on the forward conv's tiles
   ConvBwdArgs c;
   c.x[0] = q; c.x[1] = k; c.x[2] = v;
   c.dy[0] = act[3]; c.dy[1] = act[4]; c.dy[2] = act[5];
   c.dx[0] = dq; c.dx[1] = dk; c.dx[2] = dv;
-  c.w_text = w_text; c.w_vis = w_vis; c.dw_text = dw_text; c.dw_vis = dw_vis;
-  c.N = d.N; c.L = d.L; c.B = d.B; c.C = C; c.text_k = d.text_k; c.T = d.T; c.Hg = d.Hg; c.Wg = d.Wg; c.pt = d.pt;
+  c.w_text = w_text; c.dw_text = dw_text;
+  c.N = d.N; c.L = d.L; c.B = d.B; c.C = C; c.text_k = d.text_k;
   e = dt == KDA_DT_BF16 ? launch_conv_bwd<__nv_bfloat16>(c, d, s) : launch_conv_bwd<float>(c, d, s);
   if (e != cudaSuccess) return e;
-  if (launches) *launches += 5 + 1 + 2;
+  if ((e = launch_shortconv_bwd_vis(d, dt, c.x, c.dy, c.dx, w_vis, dw_vis, s, launches)) != cudaSuccess) return e;
+  if (launches) *launches += 5 + 1 + (d.L > 0 ? 2 : 0);
   return cudaSuccess;
 }
 

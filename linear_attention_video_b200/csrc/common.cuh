@@ -41,6 +41,11 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 cudaError_t launch_shortconv(const Dims& d, kda_dtype dt, const void* q, const void* k, const void* v,
                              const float* w_text, const float* w_vis, void* qo, void* ko, void* vo,
                              cudaStream_t s, int* launches, bool out_f16 = false, bool out_f32 = false);
+// Backward of the visual conv: dx of the visual tokens (the transposed conv of dy,
+// written as dtype) and dw_vis += the weight gradient (fp32, accumulated).
+cudaError_t launch_shortconv_bwd_vis(const Dims& d, kda_dtype dt, const void* const x[3], const float* const dy[3],
+                                     void* const dx[3], const float* w_vis, float* dw_vis, cudaStream_t s,
+                                     int* launches);
 
 // Backward pass (bwd.cu): gradients of kda_fwd.  Buffers as in kda_bwd (include/kda.h); ws holds
 // bwd_workspace_bytes(d, dt) bytes, 256-byte aligned, its first word the status word.

@@ -46,6 +46,7 @@ struct ConvArgs {
   int B, C, text_k;
   int T, Hg, Wg, pt;
   int n_wtiles, n_hbands;
+  float* dw_vis;        // [3][C][27], accumulated (weight-gradient kernel only)
 };
 
 // ---- type helpers ----------------------------------------------------------
@@ -105,7 +106,9 @@ template <> __device__ __forceinline__ void store1<float>(float* p, float a) { *
 // RUN: pixels per thread along a row (compile-time, so the FMA loop carries no
 // predicates); a tile is NRUN runs wide.  Columns past the grid edge read the
 // zero padding of the plane and their outputs are not stored.  PT: temporal
-// offset of the first tap (1 centred, 2 causal).
+// offset of the first tap (1 centred, 2 causal, 0 anti-causal: the transpose of
+// the causal conv).  FLIP reverses the 27 taps, which turns the kernel into the
+// transpose of the conv with the unflipped taps and offset 2 - PT.
 constexpr int NSLOT = 3;   // plane slots in shared memory (2 planes in flight)
 
 __device__ __forceinline__ float widen1(__nv_bfloat16 h) { return __bfloat162float(h); }
@@ -170,7 +173,7 @@ __device__ __forceinline__ void vis_plane_step(const TIn* pl, bool compute, cons
   }
 }
 
-template <typename TIn, typename TOut, int RUN, int PT>
+template <typename TIn, typename TOut, int RUN, int PT, bool FLIP>
 __global__ void __launch_bounds__(kThreads, kMinBlocks) vis_conv_kernel(ConvArgs a) {
   using VP = VisPlane<TIn, RUN>;
   constexpr int PWr = VP::PWr;
@@ -200,7 +203,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) vis_conv_kernel(ConvArgs
   {
     const float* wbase = a.w_vis + ((int64_t)tensor * C + cg0 + lane) * kVisTaps;
 #pragma unroll
-    for (int i = 0; i < kVisTaps; ++i) wv[i] = wbase[i];
+    for (int i = 0; i < kVisTaps; ++i) wv[i] = wbase[FLIP ? kVisTaps - 1 - i : i];
   }
 
   // this thread's chunks of a plane: element offset inside a frame (-1: outside the grid)
@@ -239,9 +242,9 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) vis_conv_kernel(ConvArgs
     for (int i = 0; i < RUN; ++i) { s0[r][i] = 0.f; s1[r][i] = 0.f; s2[r][i] = 0.f; }
   for (int f = 0; f < NSLOT - 1; ++f) issue(f);
 
-  // after plane f, frame f+PT-2 is complete; with PT = 1 one step past the last
-  // plane (no data) flushes frame T-1
-  const int f_end = a.T + (PT == 1 ? 1 : 0);
+  // after plane f, frame f+PT-2 is complete; 2 - PT steps past the last plane
+  // (no data) flush the frames up to T-1
+  const int f_end = a.T + 2 - PT;
   const TIn* pl_base = reinterpret_cast<const TIn*>(slots) + (row * PWr + w0) * CG + lane;
   TOut* y_base = y + ((int64_t)(th0 + row) * a.Wg + tw0 + w0) * C + lane;
   auto step = [&](int f, float (&an)[RPT][RUN], float (&ac)[RPT][RUN], float (&ap)[RPT][RUN]) {
@@ -260,13 +263,164 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) vis_conv_kernel(ConvArgs
       step(f, s1, s0, s2);
       if (f + 1 < f_end) step(f + 1, s2, s1, s0);
       if (f + 2 < f_end) step(f + 2, s0, s2, s1);
-    } else {
+    } else if (PT == 2) {
       step(f, s2, s1, s0);
       if (f + 1 < f_end) step(f + 1, s0, s2, s1);
       if (f + 2 < f_end) step(f + 2, s1, s0, s2);
+    } else {
+      step(f, s0, s2, s1);
+      if (f + 1 < f_end) step(f + 1, s1, s0, s2);
+      if (f + 2 < f_end) step(f + 2, s2, s1, s0);
     }
   }
   asm volatile("cp.async.wait_group 0;" ::: "memory");
+}
+
+// ---- visual weight gradient ------------------------------------------------------
+// dw[c][a][b][e] = sum over t, h, w of dy[t, h, w, c] x[t + a - PT, h + b - 1, w + e - 1, c].
+// Same tiles and plane ring as the forward kernel: plane f of x meets the dy frames
+// f + PT - a (a = 0, 1, 2) of the thread's pixels, which sit in three register sets
+// rotating like the forward's accumulators (the next frame is loaded into the set
+// just used, so its latency overlaps the next barrier).  Each thread sums the 27 taps
+// of its channel over its pixels; the CTA's warps meet in shared memory and add
+// their totals to dw with one atomic per (channel, tap).
+template <typename TIn, int RUN, int PT>
+__global__ void __launch_bounds__(kThreads, kMinBlocks) vis_dw_kernel(ConvArgs a) {
+  using VP = VisPlane<TIn, RUN>;
+  constexpr int PWr = VP::PWr;
+  constexpr int NW = kThreads / 32;
+  extern __shared__ __align__(128) uint8_t slots[];   // [NSLOT][PH][PWr][CG] of TIn
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tile = blockIdx.x;
+  const int wt = tile % a.n_wtiles, hb = tile / a.n_wtiles;
+  const int cg0 = blockIdx.y * CG;
+  const int tensor = blockIdx.z % 3, b = blockIdx.z / 3;
+  const int C = a.C;
+  const int tw0 = wt * (NRUN * RUN), th0 = hb * TH;
+  const int TW = min(NRUN * RUN, a.Wg - tw0), THh = min(TH, a.Hg - th0);
+  const int64_t HW = (int64_t)a.Hg * a.Wg;
+  const void* xs = tensor == 0 ? a.x[0] : (tensor == 1 ? a.x[1] : a.x[2]);
+  const void* ys = tensor == 0 ? a.y[0] : (tensor == 1 ? a.y[1] : a.y[2]);
+  const TIn* x = static_cast<const TIn*>(xs) + ((int64_t)b * a.N + a.L) * C + cg0;
+  const float* dy = static_cast<const float*>(ys) + ((int64_t)b * a.N + a.L) * C + cg0;
+
+  const int row = RPT * (warp % (TH / RPT)), run = warp / (TH / RPT);
+  const int w0 = run * RUN;
+  const int nrun = max(0, min(RUN, TW - w0));
+  const int nrow = nrun > 0 ? max(0, min(RPT, THh - row)) : 0;
+
+  int goff[VP::NPF];
+#pragma unroll
+  for (int i = 0; i < VP::NPF; ++i) {
+    const int e = tid + i * kThreads;
+    goff[i] = -2;
+    if (e < VP::NCHUNK) {
+      const int cb = e % VP::PIX_CHUNKS, pix = e / VP::PIX_CHUNKS;
+      const int pr = pix / PWr, pc = pix - pr * PWr;
+      const int hh = th0 + pr - 1, ww = tw0 + pc - 1;
+      goff[i] = (hh >= 0 && hh < a.Hg && ww >= 0 && ww < a.Wg)
+                    ? (hh * a.Wg + ww) * C + cb * (16 / (int)sizeof(TIn)) : -1;
+    }
+  }
+  const uint32_t slot0 = (uint32_t)__cvta_generic_to_shared(slots);
+  auto issue = [&](int f) {
+    if (f < a.T) {
+      const TIn* xf = x + (int64_t)f * HW * C;
+      const uint32_t dst = slot0 + (uint32_t)(f % NSLOT) * VP::BYTES;
+#pragma unroll
+      for (int i = 0; i < VP::NPF; ++i) {
+        if (goff[i] >= -1)
+          cp_async16_zfill(dst + (uint32_t)(tid + i * kThreads) * 16u, goff[i] >= 0 ? xf + goff[i] : x,
+                           goff[i] >= 0 ? 16u : 0u);
+      }
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+
+  const float* dy_base = dy + ((int64_t)(th0 + row) * a.Wg + tw0 + w0) * C + lane;
+  auto load_dy = [&](int t, float (&d)[RPT][RUN]) {   // frame t of this thread's pixels, zero outside
+    const bool tv = t >= 0 && t < a.T;
+#pragma unroll
+    for (int r = 0; r < RPT; ++r)
+#pragma unroll
+      for (int i = 0; i < RUN; ++i)
+        d[r][i] = (tv && r < nrow && i < nrun) ? dy_base[(int64_t)t * HW * C + ((int64_t)r * a.Wg + i) * C] : 0.f;
+  };
+  float acc[kVisTaps];
+#pragma unroll
+  for (int i = 0; i < kVisTaps; ++i) acc[i] = 0.f;
+  float s0[RPT][RUN], s1[RPT][RUN], s2[RPT][RUN];
+  // frame X of dy lives in set (X + 3) % 3; before plane 0: frames PT - 2, PT - 1, PT
+  if (PT == 1) { load_dy(-1, s2); load_dy(0, s0); load_dy(1, s1); }
+  else if (PT == 2) { load_dy(0, s0); load_dy(1, s1); load_dy(2, s2); }
+  else { load_dy(-2, s1); load_dy(-1, s2); load_dy(0, s0); }
+  for (int f = 0; f < NSLOT - 1; ++f) issue(f);
+
+  const TIn* pl_base = reinterpret_cast<const TIn*>(slots) + (row * PWr + w0) * CG + lane;
+  const bool active = nrow > 0;
+  // plane f with the dy frames f + PT (d0), f + PT - 1 (d1), f + PT - 2 (d2); then frame
+  // f + PT + 1 replaces d2
+  auto step = [&](int f, float (&d0)[RPT][RUN], float (&d1)[RPT][RUN], float (&d2)[RPT][RUN]) {
+    asm volatile("cp.async.wait_group %0;" :: "n"(NSLOT - 2) : "memory");
+    __syncthreads();
+    issue(f + NSLOT - 1);
+    if (active) {
+      const TIn* pl = pl_base + (f % NSLOT) * (VP::BYTES / (int)sizeof(TIn));
+#pragma unroll
+      for (int ir = 0; ir < RPT + 2; ++ir) {
+        const TIn* src = pl + ir * PWr * CG;
+        float in[RUN + 2];
+#pragma unroll
+        for (int i = 0; i < RUN + 2; ++i) in[i] = widen1(src[i * CG]);
+#pragma unroll
+        for (int orow = 0; orow < RPT; ++orow) {
+          const int tb = ir - orow;
+          if (tb < 0 || tb > 2) continue;
+#pragma unroll
+          for (int te = 0; te < 3; ++te) {
+            float p0 = 0.f, p1 = 0.f, p2 = 0.f;
+#pragma unroll
+            for (int i = 0; i < RUN; ++i) {
+              p0 = fmaf(d0[orow][i], in[i + te], p0);
+              p1 = fmaf(d1[orow][i], in[i + te], p1);
+              p2 = fmaf(d2[orow][i], in[i + te], p2);
+            }
+            acc[tb * 3 + te] += p0;
+            acc[9 + tb * 3 + te] += p1;
+            acc[18 + tb * 3 + te] += p2;
+          }
+        }
+      }
+    }
+    load_dy(f + PT + 1, d2);
+  };
+  for (int f = 0; f < a.T; f += 3) {
+    if (PT == 1) {
+      step(f, s1, s0, s2);
+      if (f + 1 < a.T) step(f + 1, s2, s1, s0);
+      if (f + 2 < a.T) step(f + 2, s0, s2, s1);
+    } else if (PT == 2) {
+      step(f, s2, s1, s0);
+      if (f + 1 < a.T) step(f + 1, s0, s2, s1);
+      if (f + 2 < a.T) step(f + 2, s1, s0, s2);
+    } else {
+      step(f, s0, s2, s1);
+      if (f + 1 < a.T) step(f + 1, s1, s0, s2);
+      if (f + 2 < a.T) step(f + 2, s2, s1, s0);
+    }
+  }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+  __syncthreads();   // the ring is free: the warps' tap sums meet there
+  float* red = reinterpret_cast<float*>(slots);   // [NW][27][32]
+#pragma unroll
+  for (int i = 0; i < kVisTaps; ++i) red[(warp * kVisTaps + i) * 32 + lane] = acc[i];
+  __syncthreads();
+  for (int i = warp; i < kVisTaps; i += NW) {
+    float s = 0.f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) s += red[(w * kVisTaps + i) * 32 + lane];
+    atomicAdd(a.dw_vis + ((int64_t)tensor * C + cg0 + lane) * kVisTaps + i, s);
+  }
 }
 
 // ---- text kernel -------------------------------------------------------------
@@ -296,22 +450,42 @@ __global__ void __launch_bounds__(256) text_conv_kernel(ConvArgs a) {
   for (int e = 0; e < 8; e += 2) store2<TOut>(y + n * C + c0 + e, acc[e], acc[e + 1]);
 }
 
-template <typename TIn, typename TOut, int RUN, int PT>
+// MODE 0: the conv; 1: its transpose (taps reversed, offset 2 - pt); 2: the weight gradient
+template <typename TIn, typename TOut, int RUN, int PT, int MODE>
 cudaError_t launch_vis_pt(const ConvArgs& a, cudaStream_t s) {
   const size_t smem = (size_t)NSLOT * VisPlane<TIn, RUN>::BYTES;
-  cudaError_t e = cudaFuncSetAttribute(vis_conv_kernel<TIn, TOut, RUN, PT>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
   dim3 grid((unsigned)(a.n_wtiles * a.n_hbands), (unsigned)(a.C / CG), (unsigned)(3 * a.B));
-  vis_conv_kernel<TIn, TOut, RUN, PT><<<grid, kThreads, smem, s>>>(a);
+  cudaError_t e;
+  if (MODE == 2) {
+    static_assert(kThreads / 32 * kVisTaps * 32 * 4 <= NSLOT * VisPlane<__nv_bfloat16, 8>::BYTES,
+                  "the tap sums fit in the plane ring");
+    e = cudaFuncSetAttribute(vis_dw_kernel<TIn, RUN, PT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    vis_dw_kernel<TIn, RUN, PT><<<grid, kThreads, smem, s>>>(a);
+  } else {
+    e = cudaFuncSetAttribute(vis_conv_kernel<TIn, TOut, RUN, PT, MODE == 1>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    vis_conv_kernel<TIn, TOut, RUN, PT, MODE == 1><<<grid, kThreads, smem, s>>>(a);
+  }
   return cudaGetLastError();
 }
 
-template <typename TIn, typename TOut, int RUN>
+template <typename TIn, typename TOut, int RUN, int MODE>
 cudaError_t launch_vis(const ConvArgs& a0, cudaStream_t s) {
   ConvArgs a = a0;
   a.n_wtiles = (a.Wg + NRUN * RUN - 1) / (NRUN * RUN);
-  return a.pt == 2 ? launch_vis_pt<TIn, TOut, RUN, 2>(a, s) : launch_vis_pt<TIn, TOut, RUN, 1>(a, s);
+  if (MODE == 1)   // transpose: centred stays centred, causal becomes anti-causal
+    return a.pt == 2 ? launch_vis_pt<TIn, TOut, RUN, 0, MODE>(a, s) : launch_vis_pt<TIn, TOut, RUN, 1, MODE>(a, s);
+  return a.pt == 2 ? launch_vis_pt<TIn, TOut, RUN, 2, MODE>(a, s) : launch_vis_pt<TIn, TOut, RUN, 1, MODE>(a, s);
+}
+
+// widest run whose tiles cover the row with the least padding
+template <typename TIn, typename TOut, int MODE>
+cudaError_t launch_vis_any(const ConvArgs& a, cudaStream_t s) {
+  if (a.Wg % 52 == 0 || (a.Wg <= 52 && a.Wg > 48)) return launch_vis<TIn, TOut, 13, MODE>(a, s);
+  if (a.Wg % 64 == 0 || a.Wg > 52) return launch_vis<TIn, TOut, 16, MODE>(a, s);
+  return launch_vis<TIn, TOut, 8, MODE>(a, s);
 }
 
 template <typename TIn, typename TOut>
@@ -320,12 +494,7 @@ cudaError_t launch_t(const ConvArgs& a, cudaStream_t s) {
     const int64_t total = (int64_t)a.B * a.L * (a.C / 8);
     text_conv_kernel<TIn, TOut><<<dim3((unsigned)((total + 255) / 256), 3), 256, 0, s>>>(a);
   }
-  if (a.T > 0) {
-    // widest run whose tiles cover the row with the least padding
-    if (a.Wg % 52 == 0 || (a.Wg <= 52 && a.Wg > 48)) return launch_vis<TIn, TOut, 13>(a, s);
-    if (a.Wg % 64 == 0 || a.Wg > 52) return launch_vis<TIn, TOut, 16>(a, s);
-    return launch_vis<TIn, TOut, 8>(a, s);
-  }
+  if (a.T > 0) return launch_vis_any<TIn, TOut, 0>(a, s);
   return cudaGetLastError();
 }
 
@@ -351,6 +520,29 @@ cudaError_t launch_shortconv(const Dims& d, kda_dtype dt, const void* q, const v
   else if (dt == KDA_DT_BF16) e = launch_t<__nv_bfloat16, __nv_bfloat16>(a, s);
   else e = launch_t<float, float>(a, s);
   if (e == cudaSuccess && launches) *launches += (a.L > 0) + (a.T > 0);
+  return e;
+}
+
+cudaError_t launch_shortconv_bwd_vis(const Dims& d, kda_dtype dt, const void* const x[3], const float* const dy[3],
+                                     void* const dx[3], const float* w_vis, float* dw_vis, cudaStream_t s,
+                                     int* launches) {
+  if (d.T <= 0 || (int64_t)d.B * d.N == 0) return cudaSuccess;
+  ConvArgs a;
+  for (int i = 0; i < 3; ++i) { a.x[i] = dy[i]; a.y[i] = dx[i]; }
+  a.w_text = nullptr; a.w_vis = w_vis; a.dw_vis = dw_vis;
+  a.N = d.N; a.L = d.L; a.B = d.B;
+  a.C = d.H * d.dk;
+  a.text_k = d.text_k;
+  a.T = d.T; a.Hg = d.Hg; a.Wg = d.Wg; a.pt = d.pt;
+  a.n_wtiles = 0;
+  a.n_hbands = (d.Hg + TH - 1) / TH;
+  // dx of the visual tokens: the transposed conv of dy
+  cudaError_t e = dt == KDA_DT_BF16 ? launch_vis_any<float, __nv_bfloat16, 1>(a, s) : launch_vis_any<float, float, 1>(a, s);
+  if (e != cudaSuccess) return e;
+  // dw: the raw inputs against dy
+  for (int i = 0; i < 3; ++i) { a.x[i] = x[i]; a.y[i] = const_cast<float*>(dy[i]); }
+  e = dt == KDA_DT_BF16 ? launch_vis_any<__nv_bfloat16, float, 2>(a, s) : launch_vis_any<float, float, 2>(a, s);
+  if (e == cudaSuccess && launches) *launches += 2;
   return e;
 }
 
