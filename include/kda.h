@@ -75,7 +75,7 @@ typedef enum {
   KDA_ERR_CUDA = 5,           /* a CUDA runtime call failed (launch, copy) */
   KDA_ERR_TIMEOUT = 6,        /* device: a bounded wait gave up */
   KDA_ERR_DEVICE_ASSERT = 7,  /* device: an internal consistency check failed */
-  KDA_ERR_RANGE = 8           /* device: a chunk's gate decay exceeds what the bf16 tensor path handles */
+  KDA_ERR_RANGE = 8           /* device: a chunk's gate decay exceeds what the tensor path (or the backward) handles */
 } kda_status;
 
 typedef enum { KDA_DT_BF16 = 0, KDA_DT_F32 = 1 } kda_dtype;
@@ -144,18 +144,21 @@ int kda_fwd(const kda_problem* p, kda_dtype dtype,
 /* Backward pass of kda_fwd: the gradients of the loss sum(d_o * o) + sum(d_final_state * S_N)
  * (o and S_N as kda_fwd computes them from the same arguments) with respect to every input.
  * The pages describe only the forward pass; the gradients are the chain rule applied to it
- * (the conv is linear, its adjoint is its transpose; the recurrence is run in reverse from
- * states recomputed from a copy stored every 16 tokens).  fp32 on the CUDA cores.
+ * (the conv is linear, its adjoint is its transpose; the recurrence is differentiated in its
+ * chunked form over 64-token chunks: the state entering every chunk is stored by a forward
+ * pass, the gradient reaching every chunk's exit by a reverse pass, and each chunk's token
+ * gradients follow from the two).  fp32 on the CUDA cores.
  *   d_o                    [B, N, H, d] of dtype; d_final_state [B, H, d, d] fp32 or NULL (zero)
  *   dq, dk, dv             [B, N, H, d] of dtype: gradients of the raw (unconvolved) q, k, v
  *   d_log_alpha            [B, N, H, d] fp32;  d_beta [B, N, H] of dtype
  *   d_w_text, d_w_vis      [3][H*d][text_k], [3][H*d][kt*kh*kw] fp32
  *   d_initial_state        [B, H, d, d] fp32 or NULL (not written)
  * The workspace is kda_bwd_workspace_bytes(p, dtype) bytes, 256-byte aligned.  Flags:
- * KDA_FLAG_VIS_CAUSAL_T as in kda_fwd; the other flags are rejected.  fp32 gradients that
- * several CTAs add into (dq, dk, d_log_alpha, d_beta before rounding, the weights) are summed
- * with atomic adds, so their last bits depend on the order of the additions.  Returns a
- * kda_status. */
+ * KDA_FLAG_VIS_CAUSAL_T as in kda_fwd; the other flags are rejected.  The conv weight
+ * gradients are summed over tokens with atomic adds, so their last bits depend on the order of
+ * the additions.  Device status KDA_ERR_RANGE: within a chunk the running log-decay moved more
+ * than 60 nats away from its value at the chunk's token 31 (the fp32 factors of the pairwise
+ * decays would overflow); the gradients are then not valid.  Returns a kda_status. */
 size_t kda_bwd_workspace_bytes(const kda_problem* p, kda_dtype dtype);
 int kda_bwd(const kda_problem* p, kda_dtype dtype,
             const void* q, const void* k, const void* v,

@@ -26,7 +26,7 @@ def kda():
     return kda
 
 
-def run_bwd(kda, w, inp, dO, S0=None, dSN=None, causal=False):
+def run_bwd(kda, w, inp, dO, S0=None, dSN=None, causal=False, status=None):
     B, N, H, d = inp["shape"]
     t = to_device(inp)
     dt = t["q"].dtype
@@ -44,7 +44,7 @@ def run_bwd(kda, w, inp, dO, S0=None, dSN=None, causal=False):
                 g["dv"], g["dla"], g["dbeta"], g["dw_text"], g["dw_vis"], ws, initial_state=f32(S0),
                 d_final_state=f32(dSN), d_initial_state=g["dS0"])
     torch.cuda.synchronize()
-    assert kda.kda_read_status(ws) == kda.KDA_OK
+    assert kda.kda_read_status(ws) == (kda.KDA_OK if status is None else status)
     # the gradient the oracle sees for d_o is the value actually passed (rounded to dtype)
     return {n: v.float().cpu().numpy() for n, v in g.items()}, d_o.float().cpu().numpy()
 
@@ -60,8 +60,8 @@ def check(got, ref, dtype):
             assert e <= 5e-3 and m <= 2e-2, f"{n}: rel_l2={e:.3e} rel max-abs={m:.3e}"
 
 
-def _case(kda, w, seed, causal=False, with_state=True):
-    inp = kda_synth.generate(w, seed)
+def _case(kda, w, seed, causal=False, with_state=True, inp=None):
+    inp = kda_synth.generate(w, seed) if inp is None else inp
     B, N, H, d = inp["shape"]
     rng = np.random.default_rng(seed)
     dO = rng.standard_normal((B, N, H, d))
@@ -121,3 +121,19 @@ def test_bwd_bf16_full_size_sampled_v_columns(kda):
     e = rel_l2(x, ref)
     m = float(np.abs(x - ref).max() / np.abs(ref).max())
     assert e <= 5e-3 and m <= 2e-2, f"dv columns: rel_l2={e:.3e} rel max-abs={m:.3e}"
+
+
+def test_bwd_strong_decay_within_and_beyond_the_range(kda):
+    """The backward splits each pairwise decay e^(g_r - g_i) of a 64-token chunk around the
+    chunk's middle token in fp32: 37 nats of decay inside a chunk (beyond the forward tensor
+    path's fp16 range) is still exact; 70 nats on one side of the middle token is reported
+    (KDA_ERR_RANGE), not returned as wrong values."""
+    w = kda_synth.WORKLOADS[0]
+    inp = kda_synth.generate(w, 37)
+    B, N, H, d = inp["shape"]
+    la = inp["log_alpha"].reshape(B, N, H, d).copy()
+    la[0, 3:40, 1, 5] = -1.0
+    _case(kda, w, 37, inp=dict(inp, log_alpha=la.reshape(inp["log_alpha"].shape)))
+    la[0, 3:31, 1, 5] = -2.5
+    dO = np.random.default_rng(7).standard_normal((B, N, H, d))
+    run_bwd(kda, w, dict(inp, log_alpha=la.reshape(inp["log_alpha"].shape)), dO, status=kda.KDA_ERR_RANGE)
