@@ -42,10 +42,10 @@ namespace {
 
 constexpr int CH = 64;          // tokens per chunk
 constexpr int NT = 256;         // threads of every scan kernel: a 16 x 16 grid (ty, tx)
-constexpr int LDC = CH + 1;     // row stride of CH x CH tiles in shared memory
+constexpr int LDC = CH + 4;     // row stride of CH x CH tiles in shared memory (4 mod 32, see wmma3)
 constexpr int CW = 16;          // value columns per CTA of the two chains
 constexpr int JB = 32;          // value columns per stage of the state-gradient kernel
-constexpr int LDJ = JB + 1;
+constexpr int LDJ = JB + 4;
 constexpr float kRange = 60.f;  // largest |g - g_m| (nats) of the fp32 factorised decays
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -57,6 +57,11 @@ __device__ __forceinline__ float ld_act(const void* p, int64_t i, bool bf16) {
 __device__ __forceinline__ void cp_async16(float* dst, const float* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" :: "r"((uint32_t)__cvta_generic_to_shared(dst)),
                "l"(src) : "memory");
+}
+// 16-byte cp.async reading 16 bytes (valid) or none (zero fill)
+__device__ __forceinline__ void cp_async16z(float* dst, const float* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" :: "r"((uint32_t)__cvta_generic_to_shared(dst)),
+               "l"(src), "r"(valid ? 16u : 0u) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
@@ -99,51 +104,135 @@ struct CbwdArgs {
   uint32_t* status;
 };
 
-// acc[i][j] += sum_{kk < K} A(m_i, kk) B(kk, n_j), m_i = ty + 16 i, n_j = tx + 16 j, with
-// A(m, k) = A[m * am + k * ak] and B(k, n) = B[k * bk + n * bn] in shared memory.  The
-// tiles' odd row strides keep both the row and the column reads free of bank conflicts.
-template <int TM, int TN>
-__device__ __forceinline__ void gemm_acc(float (&acc)[TM][TN], const float* A, int am, int ak, const float* B,
-                                         int bk, int bn, int K, int ty, int tx) {
-  const float* a0 = A + ty * am;
-  const float* b0 = B + tx * bn;
-#pragma unroll 4
-  for (int kk = 0; kk < K; ++kk) {
-    float av[TM], bv[TN];
+// ---- warp-level tensor-core products (mma.sync m16n8k8, tf32) ----------------------
+// Each operand is split as x = hi + lo (both tf32) and a product is formed as
+// hi*hi + hi*lo + lo*hi, which keeps it at about fp32 accuracy.
+__device__ __forceinline__ uint32_t tf32_of(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+__device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
+  hi = tf32_of(x);
+  lo = tf32_of(x - __uint_as_float(hi));
+}
+__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+  asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+               : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+               : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// One warp: c[mt][nt] += the 16 x 8 tile (rows m0 + 16 mt, columns n0 + 8 nt) of A B, K a
+// multiple of 8, A(m, k) = A[m * am + k * ak] and B(k, n) = B[k * bk + n * bn] in shared memory.
+// Fragment coordinates, g = lane / 4, t = lane % 4: c[.][.][0..3] = C[g][2t], C[g][2t+1],
+// C[g+8][2t], C[g+8][2t+1] of the tile.  With CHAINS the hi*hi and the correction products of
+// even and odd k-steps go to four separate accumulators (summed at the end), for warps that
+// own one or two tiles and would otherwise wait on each product.  Shared-memory reads are free
+// of bank conflicts when a row stride along k (am or bn = ld, the other 1) is 4 mod 32 and a
+// row stride across k (ak or bk = ld) is 8 mod 32.
+template <int MT, int NT, bool CHAINS = false>
+__device__ __forceinline__ void wmma3(float (&c)[MT][NT][4], const float* A, int am, int ak, const float* B, int bk,
+                                      int bn, int K, int m0, int n0, int lane) {
+  const int g = lane >> 2, t = lane & 3;
+  const float* a0 = A + (m0 + g) * am + t * ak;
+  const float* b0 = B + t * bk + (n0 + g) * bn;
+  float e[CHAINS ? 3 : 1][MT][NT][4];
+  if (CHAINS) {
 #pragma unroll
-    for (int i = 0; i < TM; ++i) av[i] = a0[i * 16 * am + kk * ak];
+    for (int x = 0; x < (CHAINS ? 3 : 1); ++x)
 #pragma unroll
-    for (int j = 0; j < TN; ++j) bv[j] = b0[kk * bk + j * 16 * bn];
+      for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-    for (int i = 0; i < TM; ++i)
+        for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-      for (int j = 0; j < TN; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+          for (int i = 0; i < 4; ++i) e[x][mt][nt][i] = 0.f;
+  }
+#pragma unroll 2
+  for (int k0 = 0; k0 < K; k0 += 8) {
+    uint32_t ah[MT][4], al[MT][4], bh[NT][2], bl[NT][2];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+      const float* p = a0 + 16 * mt * am + k0 * ak;
+      split_tf32(p[0], ah[mt][0], al[mt][0]);
+      split_tf32(p[8 * am], ah[mt][1], al[mt][1]);
+      split_tf32(p[4 * ak], ah[mt][2], al[mt][2]);
+      split_tf32(p[8 * am + 4 * ak], ah[mt][3], al[mt][3]);
+    }
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const float* p = b0 + k0 * bk + 8 * nt * bn;
+      split_tf32(p[0], bh[nt][0], bl[nt][0]);
+      split_tf32(p[4 * bk], bh[nt][1], bl[nt][1]);
+    }
+    const bool odd = CHAINS && ((k0 >> 3) & 1);
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        if (CHAINS) {
+          mma_tf32(e[odd ? 1 : 0][mt][nt], al[mt], bh[nt]);
+          mma_tf32(e[odd ? 1 : 0][mt][nt], ah[mt], bl[nt]);
+          if (odd) mma_tf32(e[2][mt][nt], ah[mt], bh[nt]);
+          else mma_tf32(c[mt][nt], ah[mt], bh[nt]);
+        } else {
+          mma_tf32(c[mt][nt], al[mt], bh[nt]);
+          mma_tf32(c[mt][nt], ah[mt], bl[nt]);
+          mma_tf32(c[mt][nt], ah[mt], bh[nt]);
+        }
+      }
+  }
+  if (CHAINS) {
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) c[mt][nt][i] += (e[0][mt][nt][i] + e[1][mt][nt][i]) + e[2][mt][nt][i];
   }
 }
 
-template <int TM, int TN>
-__device__ __forceinline__ void zero(float (&acc)[TM][TN]) {
+template <int MT, int NT>
+__device__ __forceinline__ void zero4(float (&c)[MT][NT][4]) {
 #pragma unroll
-  for (int i = 0; i < TM; ++i)
+  for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-    for (int j = 0; j < TN; ++j) acc[i][j] = 0.f;
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) c[mt][nt][i] = 0.f;
 }
 
-// rows [0, CH) of a [.][D] fp32 matrix whose row r starts at src + r * rs, zero from row n on
-template <int D>
-__device__ __forceinline__ void load_rows(float* dst, int ld, const float* src, int64_t rs, int n, int tid) {
-  for (int idx = tid; idx < CH * D / 4; idx += NT) {
-    const int r = idx / (D / 4), c4 = (idx % (D / 4)) * 4;
-    const float4 x = r < n ? *reinterpret_cast<const float4*>(src + r * rs + c4) : make_float4(0.f, 0.f, 0.f, 0.f);
-    float* d = dst + r * ld + c4;
-    d[0] = x.x; d[1] = x.y; d[2] = x.z; d[3] = x.w;
+// rows [0, CH) of a [.][W] fp32 matrix whose row r starts at src + r * rs into shared memory
+// (row stride ld) by cp.async, zero from row n on; the caller commits and waits
+template <int W>
+__device__ __forceinline__ void stage_rows(float* dst, int ld, const float* src, int64_t rs, int n, int tid) {
+  for (int idx = tid; idx < CH * W / 4; idx += NT) {
+    const int r = idx / (W / 4), c4 = (idx % (W / 4)) * 4;
+    cp_async16z(dst + r * ld + c4, r < n ? src + r * rs + c4 : src, r < n);
+  }
+}
+
+// 8 consecutive activations of dtype (bf16 or fp32) from element i (a multiple of 8), as floats
+__device__ __forceinline__ void ld8_act(const void* p, int64_t i, bool bf16, float (&v)[8]) {
+  if (bf16) {
+    const uint4 u = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p) + i);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      v[2 * j] = __uint_as_float(w[j] << 16);
+      v[2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
+    }
+  } else {
+    const float4 x0 = *reinterpret_cast<const float4*>(static_cast<const float*>(p) + i);
+    const float4 x1 = *reinterpret_cast<const float4*>(static_cast<const float*>(p) + i + 4);
+    v[0] = x0.x; v[1] = x0.y; v[2] = x0.z; v[3] = x0.w;
+    v[4] = x1.x; v[5] = x1.y; v[6] = x1.z; v[7] = x1.w;
   }
 }
 
 // running sum over the chunk's rows, per key channel (threads < D); g_m and g_l per channel
 template <int D>
 __device__ __forceinline__ void chunk_cumsum(float* Gs, float* gm, float* gl, int tid) {
-  constexpr int LDD = D + 1;
+  constexpr int LDD = D + 4;
   if (tid < D) {
     float s = 0.f;
     for (int r = 0; r < CH; ++r) {
@@ -172,13 +261,25 @@ __device__ __forceinline__ ChunkPos chunk_pos(const CbwdArgs& a) {
 }
 
 // ---- per-chunk forward quantities and dO terms ------------------------------------
+// Warp tilings of the per-chunk products (8 warps, wmma3 tiles of 16 x 8):
+//   CH x CH: warp block 16 x 32 at (16 (w % 4), 32 (w / 4))
+//   CH x D:  warp block 32 x D/4 at (32 (w % 2), D/4 (w / 2))
+//   D x D:   warp block D/4 x D/2 at (D/4 (w % 4), D/2 (w / 4))
+// A thread's elements of a block: rows m0 + 16 mt + g (+ 8), columns n0 + 8 nt + 2t (+ 1).
+#define FRAG_LOOP(MT, NT_)                    \
+  _Pragma("unroll") for (int mt = 0; mt < (MT); ++mt) \
+  _Pragma("unroll") for (int nt = 0; nt < (NT_); ++nt) \
+  _Pragma("unroll") for (int i = 0; i < 4; ++i)
+#define FRAG_R(m0) ((m0) + 16 * mt + g + 8 * (i >> 1))
+#define FRAG_C(n0) ((n0) + 8 * nt + 2 * t + (i & 1))
+
 template <int D>
-constexpr size_t prep_smem() { return sizeof(float) * (4 * CH * (D + 1) + 2 * CH * LDC + 2 * D + CH); }
+constexpr size_t prep_smem() { return sizeof(float) * (4 * CH * (D + 4) + 2 * CH * LDC + 2 * D + CH); }
 
 template <int D>
 __global__ void __launch_bounds__(NT, 1) cbwd_prep_kernel(CbwdArgs a) {
-  constexpr int LDD = D + 1, TN = D / 16;
-  extern __shared__ float sm[];
+  constexpr int LDD = D + 4, NTD = D / 32;
+  extern __shared__ __align__(16) float sm[];
   float* Gs = sm;                 // [CH][LDD] g, later dO
   float* Kx = Gs + CH * LDD;      // k e^{g - g_m}
   float* KN = Kx + CH * LDD;      // k e^{g_m - g}, later v
@@ -188,79 +289,109 @@ __global__ void __launch_bounds__(NT, 1) cbwd_prep_kernel(CbwdArgs a) {
   float* gm = Ps + CH * LDC;      // [D]
   float* gl = gm + D;             // [D]
   float* bs = gl + D;             // [CH] beta
-  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = lane >> 2, t = lane & 3;
   const ChunkPos p = chunk_pos(a);
   const int64_t rs = (int64_t)a.H * D;
-  const float* q = a.q + p.tok0 * D;
-  const float* k = a.k + p.tok0 * D;
-
-  load_rows<D>(Gs, LDD, a.la + p.tok0 * D, rs, p.n, tid);
+  // log alpha, k and q of the chunk in flight together (k and q land raw in Kx and Qx)
+  stage_rows<D>(Gs, LDD, a.la + p.tok0 * D, rs, p.n, tid);
+  stage_rows<D>(Kx, LDD, a.k + p.tok0 * D, rs, p.n, tid);
+  stage_rows<D>(Qx, LDD, a.q + p.tok0 * D, rs, p.n, tid);
+  cp_async_commit();
   if (tid < CH) bs[tid] = tid < p.n ? ld_act(a.beta, p.tok0 + (int64_t)tid * a.H, a.bf16) : 0.f;
+  cp_async_wait_all();
   __syncthreads();
   chunk_cumsum<D>(Gs, gm, gl, tid);
   __syncthreads();
   bool bad = false;
   float* Kt = a.w.Kt + p.ch * CH * D;
-  for (int idx = tid; idx < CH * D; idx += NT) {
-    const int r = idx / D, c = idx % D;
-    const float g = Gs[r * LDD + c], x = g - gm[c];
-    bad |= fabsf(x) > kRange;
-    const float kv = r < p.n ? k[r * rs + c] : 0.f, qv = r < p.n ? q[r * rs + c] : 0.f;
-    const float ep = expf(x), en = expf(-x);
-    Kx[r * LDD + c] = kv * ep;
-    KN[r * LDD + c] = kv * en;
-    Qx[r * LDD + c] = qv * ep;
-    Kt[idx] = kv * expf(gl[c] - g);
+  for (int idx = tid; idx < CH * D / 4; idx += NT) {   // each thread transforms its own elements in place
+    const int r = idx / (D / 4), c4 = (idx % (D / 4)) * 4;
+    const float4 k4 = *reinterpret_cast<const float4*>(Kx + r * LDD + c4);
+    const float4 q4 = *reinterpret_cast<const float4*>(Qx + r * LDD + c4);
+    const float4 g4 = *reinterpret_cast<const float4*>(Gs + r * LDD + c4);
+    const float kv[4] = {k4.x, k4.y, k4.z, k4.w}, qv[4] = {q4.x, q4.y, q4.z, q4.w}, gv[4] = {g4.x, g4.y, g4.z, g4.w};
+    float kx[4], kn[4], qx[4], kt[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float x = gv[j] - gm[c4 + j];
+      bad |= fabsf(x) > kRange;
+      const float ep = expf(x), en = expf(-x);
+      kx[j] = kv[j] * ep;
+      kn[j] = kv[j] * en;
+      qx[j] = qv[j] * ep;
+      kt[j] = kv[j] * expf(gl[c4 + j] - gv[j]);
+    }
+    *reinterpret_cast<float4*>(Kx + r * LDD + c4) = make_float4(kx[0], kx[1], kx[2], kx[3]);
+    *reinterpret_cast<float4*>(KN + r * LDD + c4) = make_float4(kn[0], kn[1], kn[2], kn[3]);
+    *reinterpret_cast<float4*>(Qx + r * LDD + c4) = make_float4(qx[0], qx[1], qx[2], qx[3]);
+    *reinterpret_cast<float4*>(Kt + r * D + c4) = make_float4(kt[0], kt[1], kt[2], kt[3]);
   }
   if (tid < D) a.w.egl[p.ch * D + tid] = expf(gl[tid]);
   if (__syncthreads_or(bad) && tid == 0) set_status(a.status, KDA_ERR_RANGE);
 
   {  // A = Diag(beta) strict(Kx KN^T), P = lower(Qx KN^T)
-    float ab[4][4], pp[4][4];
-    zero(ab);
-    zero(pp);
-    gemm_acc<4, 4>(ab, Kx, LDD, 1, KN, 1, LDD, D, ty, tx);
-    gemm_acc<4, 4>(pp, Qx, LDD, 1, KN, 1, LDD, D, ty, tx);
+    const int m0 = 16 * (warp & 3), n0 = 32 * (warp >> 2);
+    float ab[1][4][4], pp[1][4][4];
+    zero4(ab);
+    zero4(pp);
+    wmma3<1, 4>(ab, Kx, LDD, 1, KN, 1, LDD, D, m0, n0, lane);
+    wmma3<1, 4>(pp, Qx, LDD, 1, KN, 1, LDD, D, m0, n0, lane);
     float* Abg = a.w.Ab + p.ch * CH * CH;
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int r = ty + 16 * i, c = tx + 16 * j;
-        const float abv = c < r ? ab[i][j] : 0.f;
-        As[r * LDC + c] = bs[r] * abv;
-        Abg[r * CH + c] = abv;
-        Ps[r * LDC + c] = c <= r ? pp[i][j] : 0.f;
-      }
+    FRAG_LOOP(1, 4) {
+      const int r = FRAG_R(m0), c = FRAG_C(n0);
+      const float abv = c < r ? ab[mt][nt][i] : 0.f;
+      As[r * LDC + c] = bs[r] * abv;
+      Abg[r * CH + c] = abv;
+      Ps[r * LDC + c] = c <= r ? pp[mt][nt][i] : 0.f;
+    }
   }
   __syncthreads();
+  // v into the KN tile the products above no longer read, by cp.async
+  stage_rows<D>(KN, LDD, a.v + p.tok0 * D, rs, p.n, tid);
+  cp_async_commit();
   // X = (I + A)^{-1} by forward substitution, one column per thread (threads < CH); the other
-  // threads meanwhile stage v and dO into the tiles the products above no longer read
+  // threads meanwhile convert dO into the g tile
   float x[CH];
   if (tid < CH) {
 #pragma unroll
     for (int r = 0; r < CH; ++r) {
-      float s0 = r == tid ? 1.f : 0.f, s1 = 0.f;
+      float s0 = r == tid ? 1.f : 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
 #pragma unroll
-      for (int i = 0; i + 1 < r; i += 2) {
-        s0 = fmaf(-As[r * LDC + i], x[i], s0);
-        s1 = fmaf(-As[r * LDC + i + 1], x[i + 1], s1);
+      for (int i = 0; i + 3 < r; i += 4) {
+        const float4 a4 = *reinterpret_cast<const float4*>(As + r * LDC + i);
+        s0 = fmaf(-a4.x, x[i], s0);
+        s1 = fmaf(-a4.y, x[i + 1], s1);
+        s2 = fmaf(-a4.z, x[i + 2], s2);
+        s3 = fmaf(-a4.w, x[i + 3], s3);
       }
-      if (r & 1) s0 = fmaf(-As[r * LDC + r - 1], x[r - 1], s0);
-      x[r] = s0 + s1;
+#pragma unroll
+      for (int i = r & ~3; i < r; ++i) s0 = fmaf(-As[r * LDC + i], x[i], s0);
+      x[r] = (s0 + s1) + (s2 + s3);
     }
     float* Xg = a.w.X + p.ch * CH * CH;
 #pragma unroll
     for (int r = 0; r < CH; ++r) Xg[r * CH + tid] = x[r];
   } else {
-    const int t2 = tid - CH;
-    for (int idx = t2; idx < CH * D; idx += NT - CH) {
-      const int r = idx / D, c = idx % D;
-      const bool in = r < p.n;
-      KN[r * LDD + c] = in ? a.v[(p.tok0 + (int64_t)r * a.H) * D + c] : 0.f;
-      Gs[r * LDD + c] = in ? ld_act(a.d_o, (p.tok0 + (int64_t)r * a.H) * D + c, a.bf16) : 0.f;
+    constexpr int N8 = CH * D / 8, PER = (N8 + NT - CH - 1) / (NT - CH);
+    float v8[PER][8];
+#pragma unroll
+    for (int it = 0; it < PER; ++it) {   // all loads first, then the stores
+      const int idx = tid - CH + it * (NT - CH), r = idx / (D / 8), c8 = (idx % (D / 8)) * 8;
+      if (idx < N8 && r < p.n) ld8_act(a.d_o, (p.tok0 + (int64_t)r * a.H) * D + c8, a.bf16, v8[it]);
+      else
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v8[it][j] = 0.f;
+    }
+#pragma unroll
+    for (int it = 0; it < PER; ++it) {
+      const int idx = tid - CH + it * (NT - CH), r = idx / (D / 8), c8 = (idx % (D / 8)) * 8;
+      if (idx < N8) {
+        *reinterpret_cast<float4*>(Gs + r * LDD + c8) = make_float4(v8[it][0], v8[it][1], v8[it][2], v8[it][3]);
+        *reinterpret_cast<float4*>(Gs + r * LDD + c8 + 4) = make_float4(v8[it][4], v8[it][5], v8[it][6], v8[it][7]);
+      }
     }
   }
+  cp_async_wait_all();
   __syncthreads();
   if (tid < CH) {
 #pragma unroll
@@ -268,43 +399,33 @@ __global__ void __launch_bounds__(NT, 1) cbwd_prep_kernel(CbwdArgs a) {
   }
   __syncthreads();
   {  // W = T Kx Diag(e^{g_m}),  U~ = T V,  Z = P^T dO
-    float acc[4][TN];
-    zero(acc);
-    gemm_acc<4, TN>(acc, As, LDC, 1, Kx, LDD, 1, CH, ty, tx);
+    const int m0 = 32 * (warp & 1), n0 = (D / 4) * (warp >> 1);
+    float acc[2][NTD][4];
+    zero4(acc);
+    wmma3<2, NTD>(acc, As, LDC, 1, Kx, LDD, 1, CH, m0, n0, lane);
     float* W = a.w.W + p.ch * CH * D;
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < TN; ++j) {
-        const int r = ty + 16 * i, c = tx + 16 * j;
-        W[r * D + c] = acc[i][j] * expf(gm[c]);
-      }
-    zero(acc);
-    gemm_acc<4, TN>(acc, As, LDC, 1, KN, LDD, 1, CH, ty, tx);
+    FRAG_LOOP(2, NTD) {
+      const int r = FRAG_R(m0), c = FRAG_C(n0);
+      W[r * D + c] = acc[mt][nt][i] * expf(gm[c]);
+    }
+    zero4(acc);
+    wmma3<2, NTD>(acc, As, LDC, 1, KN, LDD, 1, CH, m0, n0, lane);
     float* Ut = a.w.Ut + p.ch * CH * D;
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < TN; ++j) Ut[(ty + 16 * i) * D + tx + 16 * j] = acc[i][j];
-    zero(acc);
-    gemm_acc<4, TN>(acc, Ps, 1, LDC, Gs, LDD, 1, CH, ty, tx);
+    FRAG_LOOP(2, NTD) Ut[FRAG_R(m0) * D + FRAG_C(n0)] = acc[mt][nt][i];
+    zero4(acc);
+    wmma3<2, NTD>(acc, Ps, 1, LDC, Gs, LDD, 1, CH, m0, n0, lane);
     float* Z = a.w.Z + p.ch * CH * D;
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < TN; ++j) Z[(ty + 16 * i) * D + tx + 16 * j] = acc[i][j];
+    FRAG_LOOP(2, NTD) Z[FRAG_R(m0) * D + FRAG_C(n0)] = acc[mt][nt][i];
   }
   {  // Y = QG^T dO = Diag(e^{g_m}) Qx^T dO
-    float acc[D / 16][TN];
-    zero(acc);
-    gemm_acc<D / 16, TN>(acc, Qx, 1, LDD, Gs, LDD, 1, CH, ty, tx);
+    const int m0 = (D / 4) * (warp & 3), n0 = (D / 2) * (warp >> 2);
+    float acc[D / 64][D / 16][4];
+    zero4(acc);
+    wmma3<D / 64, D / 16>(acc, Qx, 1, LDD, Gs, LDD, 1, CH, m0, n0, lane);
     float* Y = a.w.Y + p.ch * D * D;
-#pragma unroll
-    for (int i = 0; i < D / 16; ++i) {
-      const int r = ty + 16 * i;
-      const float e = expf(gm[r]);
-#pragma unroll
-      for (int j = 0; j < TN; ++j) Y[r * D + tx + 16 * j] = acc[i][j] * e;
+    FRAG_LOOP(D / 64, D / 16) {
+      const int r = FRAG_R(m0);
+      Y[r * D + FRAG_C(n0)] = acc[mt][nt][i] * expf(gm[r]);
     }
   }
 }
@@ -313,42 +434,52 @@ __global__ void __launch_bounds__(NT, 1) cbwd_prep_kernel(CbwdArgs a) {
 // Column j of the state (and of its gradient) only meets column j of v and dO, so the
 // (b, h) chains split into D / CW independent CTAs.  The next chunk's tiles are copied by
 // cp.async into the other half of a double buffer while the current chunk is processed.
+// Tile strides: the tile read along k by the first product (W forward, Kt backward) is
+// D + 4 wide, the one read across k by the second (Kt forward, W backward) D + 8, the
+// state and U columns CW + 8 (see wmma3).
+template <int D>
+struct ChainLd {
+  static constexpr int L1 = D + 4, L2 = D + 8, LS = CW + 8;
+};
+
 template <int D, bool BWD>
 constexpr size_t chain_smem() {
-  return sizeof(float) * (2 * 2 * CH * (D + 4) + 2 * CH * CW + (BWD ? 2 * D * CW : 0) + 2 * D + D * (CW + 1) +
-                          CH * (CW + 1));
+  using L = ChainLd<D>;
+  return sizeof(float) * (2 * CH * (L::L1 + L::L2) + 2 * CH * CW + (BWD ? 2 * D * CW : 0) + 2 * D + D * L::LS +
+                          CH * L::LS);
 }
 
 template <int D, bool BWD>
 __global__ void __launch_bounds__(NT, 1) cbwd_chain_kernel(CbwdArgs a) {
-  constexpr int LDW = D + 4, LDS = CW + 1;
+  using L = ChainLd<D>;
+  constexpr int LS = L::LS;
   extern __shared__ __align__(16) float sm[];
-  float* Wb = sm;                            // [2][CH][LDW] W
-  float* Kb = Wb + 2 * CH * LDW;             // [2][CH][LDW] Kt
-  float* Vb = Kb + 2 * CH * LDW;             // [2][CH][CW]  U~ (forward) or Z (backward) columns
+  float* T1 = sm;                            // [2][CH][L1]  W (forward) or Kt (backward): first product
+  float* T2 = T1 + 2 * CH * L::L1;           // [2][CH][L2]  Kt (forward) or W (backward): second product
+  float* Vb = T2 + 2 * CH * L::L2;           // [2][CH][CW]  U~ (forward) or Z (backward) columns
   float* Yb = Vb + 2 * CH * CW;              // [2][D][CW]   Y columns (backward)
   float* eb = Yb + (BWD ? 2 * D * CW : 0);   // [2][D]       e^{gl}
-  float* S = eb + 2 * D;                     // [D][LDS]     state (forward) or its gradient (backward)
-  float* Us = S + D * LDS;                   // [CH][LDS]    U or dU
-  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  float* S = eb + 2 * D;                     // [D][LS]      state (forward) or its gradient (backward)
+  float* Us = S + D * LS;                    // [CH][LS]     U or dU
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int c0 = blockIdx.x * CW, h = blockIdx.y, b = blockIdx.z;
   const int64_t bh = (int64_t)b * a.H + h, ch0 = bh * a.nc;
   const float* init = BWD ? a.dSN : a.S0;
   for (int idx = tid; idx < D * CW; idx += NT) {
     const int r = idx / CW, j = idx % CW;
-    S[r * LDS + j] = init ? init[(bh * D + r) * D + c0 + j] : 0.f;
+    S[r * LS + j] = init ? init[(bh * D + r) * D + c0 + j] : 0.f;
   }
   auto issue = [&](int c) {
     if (c >= 0 && c < a.nc) {
       const int s = c & 1;
       const int64_t ch = ch0 + c;
-      const float* W = a.w.W + ch * CH * D;
-      const float* K = a.w.Kt + ch * CH * D;
+      const float* M1 = (BWD ? a.w.Kt : a.w.W) + ch * CH * D;
+      const float* M2 = (BWD ? a.w.W : a.w.Kt) + ch * CH * D;
       const float* V = (BWD ? a.w.Z : a.w.Ut) + ch * CH * D;
       for (int i = tid; i < CH * D / 4; i += NT) {
         const int r = i / (D / 4), c4 = (i % (D / 4)) * 4;
-        cp_async16(Wb + (s * CH + r) * LDW + c4, W + r * D + c4);
-        cp_async16(Kb + (s * CH + r) * LDW + c4, K + r * D + c4);
+        cp_async16(T1 + (s * CH + r) * L::L1 + c4, M1 + r * D + c4);
+        cp_async16(T2 + (s * CH + r) * L::L2 + c4, M2 + r * D + c4);
       }
       for (int i = tid; i < CH * CW / 4; i += NT) {
         const int r = i / (CW / 4), c4 = (i % (CW / 4)) * 4;
@@ -365,6 +496,12 @@ __global__ void __launch_bounds__(NT, 1) cbwd_chain_kernel(CbwdArgs a) {
     }
     cp_async_commit();
   };
+  // warp tiles: the CH x CW product as 4 x 2 tiles of 16 x 8, one per warp; the D x CW product
+  // as (D / 16) x 2 tiles, D / 64 per warp
+  const int g = lane >> 2, t = lane & 3;
+  const int m1 = 16 * (warp & 3), n1 = 8 * (warp >> 2);
+  constexpr int MT2 = D / 64;
+  const int m2 = 16 * MT2 * (warp & 3), n2 = 8 * (warp >> 2);
   issue(BWD ? a.nc - 1 : 0);
   for (int step = 0; step < a.nc; ++step) {
     const int c = BWD ? a.nc - 1 - step : step;
@@ -377,40 +514,42 @@ __global__ void __launch_bounds__(NT, 1) cbwd_chain_kernel(CbwdArgs a) {
       float* out = (BWD ? a.w.dS : a.w.S) + ch * D * D;
       for (int idx = tid; idx < D * CW; idx += NT) {
         const int r = idx / CW, j = idx % CW;
-        out[r * D + c0 + j] = S[r * LDS + j];
+        out[r * D + c0 + j] = S[r * LS + j];
       }
     }
     {  // forward: U = U~ - W S;  backward: dU = Z + Kt dS
-      float u[4][1];
-      zero(u);
-      gemm_acc<4, 1>(u, (BWD ? Kb : Wb) + s * CH * LDW, LDW, 1, S, LDS, 1, D, ty, tx);
+      float u[1][1][4];
+      zero4(u);
+      wmma3<1, 1, true>(u, T1 + s * CH * L::L1, L::L1, 1, S, LS, 1, D, m1, n1, lane);
       float* out = (BWD ? a.w.dU : a.w.U) + ch * CH * D;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const int r = ty + 16 * i;
-        const float val = BWD ? Vb[(s * CH + r) * CW + tx] + u[i][0] : Vb[(s * CH + r) * CW + tx] - u[i][0];
-        Us[r * LDS + tx] = val;
-        out[r * D + c0 + tx] = val;
+        const int r = m1 + g + 8 * (i >> 1), j = n1 + 2 * t + (i & 1);
+        const float val = BWD ? Vb[(s * CH + r) * CW + j] + u[0][0][i] : Vb[(s * CH + r) * CW + j] - u[0][0][i];
+        Us[r * LS + j] = val;
+        out[r * D + c0 + j] = val;
       }
     }
     __syncthreads();
     {  // forward: S = Diag(e^{gl}) S + Kt^T U;  backward: dS = Diag(e^{gl}) dS - W^T dU + Y
-      float sv[D / 16][1];
-      zero(sv);
-      gemm_acc<D / 16, 1>(sv, (BWD ? Wb : Kb) + s * CH * LDW, 1, LDW, Us, LDS, 1, CH, ty, tx);
+      float sv[MT2][1][4];
+      zero4(sv);
+      wmma3<MT2, 1, true>(sv, T2 + s * CH * L::L2, 1, L::L2, Us, LS, 1, CH, m2, n2, lane);
 #pragma unroll
-      for (int i = 0; i < D / 16; ++i) {
-        const int r = ty + 16 * i;
-        const float prev = eb[s * D + r] * S[r * LDS + tx];
-        S[r * LDS + tx] = BWD ? prev - sv[i][0] + Yb[(s * D + r) * CW + tx] : prev + sv[i][0];
-      }
+      for (int mt = 0; mt < MT2; ++mt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = m2 + 16 * mt + g + 8 * (i >> 1), j = n2 + 2 * t + (i & 1);
+          const float prev = eb[s * D + r] * S[r * LS + j];
+          S[r * LS + j] = BWD ? prev - sv[mt][0][i] + Yb[(s * D + r) * CW + j] : prev + sv[mt][0][i];
+        }
     }
   }
   if (BWD && a.dS0) {
     __syncthreads();
     for (int idx = tid; idx < D * CW; idx += NT) {
       const int r = idx / CW, j = idx % CW;
-      a.dS0[(bh * D + r) * D + c0 + j] = S[r * LDS + j];
+      a.dS0[(bh * D + r) * D + c0 + j] = S[r * LS + j];
     }
   }
 }
@@ -421,15 +560,15 @@ constexpr size_t state_grad_smem() { return sizeof(float) * (2 * D * LDJ + 4 * C
 
 template <int D>
 __global__ void __launch_bounds__(NT) cbwd_state_grad_kernel(CbwdArgs a) {
-  constexpr int TN = D / 16;
-  extern __shared__ float sm[];
+  constexpr int NTD = D / 32;
+  extern __shared__ __align__(16) float sm[];
   float* S0b = sm;              // [D][LDJ]  S columns j0 .. j0 + JB
   float* dSb = S0b + D * LDJ;   // [D][LDJ]  dS columns
   float* dOb = dSb + D * LDJ;   // [CH][LDJ]
   float* dUb = dOb + CH * LDJ;
   float* Ub = dUb + CH * LDJ;
   float* Vb = Ub + CH * LDJ;
-  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = lane >> 2, t = lane & 3;
   const ChunkPos p = chunk_pos(a);
   const float* S = a.w.S + p.ch * D * D;
   const float* dS = a.w.dS + p.ch * D * D;
@@ -438,86 +577,83 @@ __global__ void __launch_bounds__(NT) cbwd_state_grad_kernel(CbwdArgs a) {
   // stage columns [j0, j0 + JB) of the chunk's operands; which ones per pass
   auto stage = [&](int j0, bool pass2) {
     __syncthreads();
-    for (int idx = tid; idx < D * JB; idx += NT) {
-      const int r = idx / JB, j = idx % JB;
-      if (!pass2) S0b[r * LDJ + j] = S[r * D + j0 + j];
-      dSb[r * LDJ + j] = dS[r * D + j0 + j];
+    for (int idx = tid; idx < D * JB / 4; idx += NT) {
+      const int r = idx / (JB / 4), c4 = (idx % (JB / 4)) * 4;
+      if (!pass2) *reinterpret_cast<float4*>(S0b + r * LDJ + c4) = *reinterpret_cast<const float4*>(S + r * D + j0 + c4);
+      *reinterpret_cast<float4*>(dSb + r * LDJ + c4) = *reinterpret_cast<const float4*>(dS + r * D + j0 + c4);
     }
-    for (int idx = tid; idx < CH * JB; idx += NT) {
-      const int r = idx / JB, j = idx % JB;
+    for (int idx = tid; idx < CH * JB / 4; idx += NT) {
+      const int r = idx / (JB / 4), c4 = (idx % (JB / 4)) * 4;
       const bool in = r < p.n;
-      const int64_t t = (p.tok0 + (int64_t)r * a.H) * D + j0 + j;
-      dOb[r * LDJ + j] = in ? ld_act(a.d_o, t, a.bf16) : 0.f;
-      dUb[r * LDJ + j] = dU[r * D + j0 + j];
+      const int64_t tk = (p.tok0 + (int64_t)r * a.H) * D + j0 + c4;
+      float4 o4 = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (in) o4 = make_float4(ld_act(a.d_o, tk, a.bf16), ld_act(a.d_o, tk + 1, a.bf16), ld_act(a.d_o, tk + 2, a.bf16),
+                               ld_act(a.d_o, tk + 3, a.bf16));
+      *reinterpret_cast<float4*>(dOb + r * LDJ + c4) = o4;
+      *reinterpret_cast<float4*>(dUb + r * LDJ + c4) = *reinterpret_cast<const float4*>(dU + r * D + j0 + c4);
       if (pass2) {
-        Ub[r * LDJ + j] = U[r * D + j0 + j];
-        Vb[r * LDJ + j] = in ? a.v[t] : 0.f;
+        *reinterpret_cast<float4*>(Ub + r * LDJ + c4) = *reinterpret_cast<const float4*>(U + r * D + j0 + c4);
+        *reinterpret_cast<float4*>(Vb + r * LDJ + c4) =
+            in ? *reinterpret_cast<const float4*>(a.v + tk) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
     __syncthreads();
   };
+  const int m0 = 32 * (warp & 1), n0 = (D / 4) * (warp >> 1);        // CH x D blocks
+  const int p0 = 16 * (warp & 3), q0 = 32 * (warp >> 2);             // CH x CH blocks
   {  // dQG = dO S^T, dW = -dU S^T, and rowsum(dS o S)
-    float aq[4][TN], aw[4][TN];
-    zero(aq);
-    zero(aw);
+    float aq[2][NTD][4], aw[2][NTD][4];
+    zero4(aq);
+    zero4(aw);
     float lastp = 0.f;
     for (int j0 = 0; j0 < D; j0 += JB) {
       stage(j0, false);
-      gemm_acc<4, TN>(aq, dOb, LDJ, 1, S0b, 1, LDJ, JB, ty, tx);
-      gemm_acc<4, TN>(aw, dUb, LDJ, 1, S0b, 1, LDJ, JB, ty, tx);
+      wmma3<2, NTD>(aq, dOb, LDJ, 1, S0b, 1, LDJ, JB, m0, n0, lane);
+      wmma3<2, NTD>(aw, dUb, LDJ, 1, S0b, 1, LDJ, JB, m0, n0, lane);
       if (tid < D)
 #pragma unroll 8
         for (int j = 0; j < JB; ++j) lastp = fmaf(dSb[tid * LDJ + j], S0b[tid * LDJ + j], lastp);
     }
     float* dQG = a.w.dQG + p.ch * CH * D;
     float* dW = a.w.dW + p.ch * CH * D;
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < TN; ++j) {
-        const int r = ty + 16 * i, c = tx + 16 * j;
-        dQG[r * D + c] = aq[i][j];
-        dW[r * D + c] = -aw[i][j];
-      }
+    FRAG_LOOP(2, NTD) {
+      const int r = FRAG_R(m0), c = FRAG_C(n0);
+      dQG[r * D + c] = aq[mt][nt][i];
+      dW[r * D + c] = -aw[mt][nt][i];
+    }
     if (tid < D) a.w.last[p.ch * D + tid] = lastp * a.w.egl[p.ch * D + tid];
   }
   {  // dKt = U dS^T, dP = lower(dO U^T), dU V^T
-    float ak[4][TN], ap[4][4], auv[4][4];
-    zero(ak);
-    zero(ap);
-    zero(auv);
+    float ak[2][NTD][4], ap[1][4][4], auv[1][4][4];
+    zero4(ak);
+    zero4(ap);
+    zero4(auv);
     for (int j0 = 0; j0 < D; j0 += JB) {
       stage(j0, true);
-      gemm_acc<4, TN>(ak, Ub, LDJ, 1, dSb, 1, LDJ, JB, ty, tx);
-      gemm_acc<4, 4>(ap, dOb, LDJ, 1, Ub, 1, LDJ, JB, ty, tx);
-      gemm_acc<4, 4>(auv, dUb, LDJ, 1, Vb, 1, LDJ, JB, ty, tx);
+      wmma3<2, NTD>(ak, Ub, LDJ, 1, dSb, 1, LDJ, JB, m0, n0, lane);
+      wmma3<1, 4>(ap, dOb, LDJ, 1, Ub, 1, LDJ, JB, p0, q0, lane);
+      wmma3<1, 4>(auv, dUb, LDJ, 1, Vb, 1, LDJ, JB, p0, q0, lane);
     }
     float* dKt = a.w.dKt + p.ch * CH * D;
     float* dP = a.w.dP + p.ch * CH * CH;
     float* dUV = a.w.dUV + p.ch * CH * CH;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int r = ty + 16 * i;
-#pragma unroll
-      for (int j = 0; j < TN; ++j) dKt[r * D + tx + 16 * j] = ak[i][j];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int c = tx + 16 * j;
-        dP[r * CH + c] = c <= r ? ap[i][j] : 0.f;
-        dUV[r * CH + c] = auv[i][j];
-      }
+    FRAG_LOOP(2, NTD) dKt[FRAG_R(m0) * D + FRAG_C(n0)] = ak[mt][nt][i];
+    FRAG_LOOP(1, 4) {
+      const int r = FRAG_R(p0), c = FRAG_C(q0);
+      dP[r * CH + c] = c <= r ? ap[mt][nt][i] : 0.f;
+      dUV[r * CH + c] = auv[mt][nt][i];
     }
   }
 }
 
 // ---- the chunk-local part of the adjoint ---------------------------------------------
 template <int D>
-constexpr size_t local_grad_smem() { return sizeof(float) * (4 * CH * (D + 1) + 5 * CH * LDC + 3 * D + 2 * CH); }
+constexpr size_t local_grad_smem() { return sizeof(float) * (4 * CH * (D + 4) + 5 * CH * LDC + 3 * D + 2 * CH); }
 
 template <int D>
 __global__ void __launch_bounds__(NT, 1) cbwd_local_grad_kernel(CbwdArgs a) {
-  constexpr int LDD = D + 1, TN = D / 16;
-  extern __shared__ float sm[];
+  constexpr int LDD = D + 4, NTD = D / 32;
+  extern __shared__ __align__(16) float sm[];
   float* Gs = sm;                 // [CH][LDD] g, at the end dg
   float* Kx = Gs + CH * LDD;      // k e^{g - g_m}
   float* Fs = Kx + CH * LDD;      // dW e^{g_m}, later q e^{g - g_m}
@@ -526,102 +662,108 @@ __global__ void __launch_bounds__(NT, 1) cbwd_local_grad_kernel(CbwdArgs a) {
   float* dTs = Xs + CH * LDC;     // dT
   float* Ms = dTs + CH * LDC;     // X^T dT Diag(beta)
   float* dPs = Ms + CH * LDC;     // dP
-  float* Abs = dPs + CH * LDC;    // A / beta, later dA Diag... (dAb)
+  float* Abs = dPs + CH * LDC;    // A / beta, later Diag(beta) dA
   float* gm = Abs + CH * LDC;     // [D]
   float* gl = gm + D;             // [D]
   float* colk = gl + D;           // [D] column sums of dKt o Kt
   float* bs = colk + D;           // [CH]
   float* db = bs + CH;            // [CH] dbeta
-  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = lane >> 2, t = lane & 3;
   const ChunkPos p = chunk_pos(a);
   const int64_t rs = (int64_t)a.H * D;
   const float* q = a.q + p.tok0 * D;
   const float* k = a.k + p.tok0 * D;
   const int64_t cd = p.ch * CH * D, cc = p.ch * CH * CH;
+  const int m0 = 32 * (warp & 1), n0 = (D / 4) * (warp >> 1);        // CH x D blocks
+  const int p0 = 16 * (warp & 3), q0 = 32 * (warp >> 2);             // CH x CH blocks
 
-  load_rows<D>(Gs, LDD, a.la + p.tok0 * D, rs, p.n, tid);
+  // every input tile of the chunk in flight together (k lands raw in Kx, dW in Fs)
+  stage_rows<D>(Gs, LDD, a.la + p.tok0 * D, rs, p.n, tid);
+  stage_rows<D>(Kx, LDD, k, rs, p.n, tid);
+  stage_rows<D>(Fs, LDD, a.w.dW + cd, D, CH, tid);
+  stage_rows<D>(Bs, LDD, a.w.dU + cd, D, CH, tid);
+  stage_rows<CH>(Xs, LDC, a.w.X + cc, CH, CH, tid);
+  stage_rows<CH>(dTs, LDC, a.w.dUV + cc, CH, CH, tid);
+  stage_rows<CH>(dPs, LDC, a.w.dP + cc, CH, CH, tid);
+  stage_rows<CH>(Abs, LDC, a.w.Ab + cc, CH, CH, tid);
+  cp_async_commit();
   if (tid < CH) bs[tid] = tid < p.n ? ld_act(a.beta, p.tok0 + (int64_t)tid * a.H, a.bf16) : 0.f;
   if (tid < D) colk[tid] = 0.f;
+  cp_async_wait_all();
   __syncthreads();
   chunk_cumsum<D>(Gs, gm, gl, tid);
   __syncthreads();
-  for (int idx = tid; idx < CH * D; idx += NT) {
-    const int r = idx / D, c = idx % D;
-    const float kv = r < p.n ? k[r * rs + c] : 0.f;
-    Kx[r * LDD + c] = kv * expf(Gs[r * LDD + c] - gm[c]);
-    Fs[r * LDD + c] = a.w.dW[cd + idx] * expf(gm[c]);
-    Bs[r * LDD + c] = a.w.dU[cd + idx];
-  }
-  for (int idx = tid; idx < CH * CH; idx += NT) {
-    const int r = idx / CH, c = idx % CH;
-    Xs[r * LDC + c] = a.w.X[cc + idx];
-    dTs[r * LDC + c] = a.w.dUV[cc + idx];
-    dPs[r * LDC + c] = a.w.dP[cc + idx];
-    Abs[r * LDC + c] = a.w.Ab[cc + idx];
+  for (int idx = tid; idx < CH * D / 4; idx += NT) {   // Kx = k e^{g - g_m}, Fs = dW e^{g_m}, in place
+    const int r = idx / (D / 4), c4 = (idx % (D / 4)) * 4;
+    float* kp = Kx + r * LDD + c4;
+    float* fp = Fs + r * LDD + c4;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      kp[j] *= expf(Gs[r * LDD + c4 + j] - gm[c4 + j]);
+      fp[j] *= expf(gm[c4 + j]);
+    }
   }
   __syncthreads();
   {  // dT = dW KG^T + dU V^T
-    float t[4][4];
-    zero(t);
-    gemm_acc<4, 4>(t, Fs, LDD, 1, Kx, 1, LDD, D, ty, tx);
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) dTs[(ty + 16 * i) * LDC + tx + 16 * j] += t[i][j];
+    float tt[1][4][4];
+    zero4(tt);
+    wmma3<1, 4>(tt, Fs, LDD, 1, Kx, 1, LDD, D, p0, q0, lane);
+    FRAG_LOOP(1, 4) dTs[FRAG_R(p0) * LDC + FRAG_C(q0)] += tt[mt][nt][i];
   }
-  // per-thread elements (row ty + 16 i, key channel tx + 16 j) of dq, dk and dg
-  float dq[4][TN], dk[4][TN], dg[4][TN];
+  // this thread's elements of dq, dk and dg (the CH x D block tiling)
+  float dq[2][NTD][4], dk[2][NTD][4], dg[2][NTD][4];
   {  // dv = Diag(beta) X^T dU
-    float acc[4][TN];
-    zero(acc);
-    gemm_acc<4, TN>(acc, Xs, 1, LDC, Bs, LDD, 1, CH, ty, tx);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int r = ty + 16 * i;
-      if (r < p.n)
-#pragma unroll
-        for (int j = 0; j < TN; ++j) a.dv[(p.tok0 + (int64_t)r * a.H) * D + tx + 16 * j] = bs[r] * acc[i][j];
+    float acc[2][NTD][4];
+    zero4(acc);
+    wmma3<2, NTD>(acc, Xs, 1, LDC, Bs, LDD, 1, CH, m0, n0, lane);
+    FRAG_LOOP(2, NTD) {
+      const int r = FRAG_R(m0);
+      if (r < p.n) a.dv[(p.tok0 + (int64_t)r * a.H) * D + FRAG_C(n0)] = bs[r] * acc[mt][nt][i];
     }
   }
   {  // dKG = Diag(beta) X^T dW; the dq, dk, dg terms of KG, QG and Kt
-    float acc[4][TN];
-    zero(acc);
-    gemm_acc<4, TN>(acc, Xs, 1, LDC, Fs, LDD, 1, CH, ty, tx);
+    float acc[2][NTD][4];
+    zero4(acc);
+    wmma3<2, NTD>(acc, Xs, 1, LDC, Fs, LDD, 1, CH, m0, n0, lane);
     const float* dKt = a.w.dKt + cd;
     const float* dQG = a.w.dQG + cd;
 #pragma unroll
-    for (int j = 0; j < TN; ++j) {
-      const int c = tx + 16 * j;
-      float ck = 0.f;
+    for (int nt = 0; nt < NTD; ++nt)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int r = ty + 16 * i;
-        const bool in = r < p.n;
-        const float g = Gs[r * LDD + c];
-        const float e1 = expf(g - gm[c]), e2 = expf(gl[c] - g), eg = expf(g);
-        const float kv = in ? k[r * rs + c] : 0.f, qv = in ? q[r * rs + c] : 0.f;
-        const float dkt = dKt[r * D + c], dqg = dQG[r * D + c];
-        const float av = bs[r] * acc[i][j] * e1;   // dKG o e^g
-        dk[i][j] = av + dkt * e2;
-        dq[i][j] = dqg * eg;
-        dg[i][j] = kv * av - kv * e2 * dkt + qv * eg * dqg;
-        ck = fmaf(kv * e2, dkt, ck);
+      for (int par = 0; par < 2; ++par) {
+        float ck = 0.f;
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+          for (int hi = 0; hi < 2; ++hi) {
+            const int i = 2 * hi + par;
+            const int r = FRAG_R(m0), c = FRAG_C(n0);
+            const bool in = r < p.n;
+            const float gv = Gs[r * LDD + c];
+            const float e1 = expf(gv - gm[c]), e2 = expf(gl[c] - gv), eg = expf(gv);
+            const float kv = in ? k[r * rs + c] : 0.f, qv = in ? q[r * rs + c] : 0.f;
+            const float dkt = dKt[r * D + c], dqg = dQG[r * D + c];
+            const float av = bs[r] * acc[mt][nt][i] * e1;   // dKG o e^g
+            dk[mt][nt][i] = av + dkt * e2;
+            dq[mt][nt][i] = dqg * eg;
+            dg[mt][nt][i] = kv * av - kv * e2 * dkt + qv * eg * dqg;
+            ck = fmaf(kv * e2, dkt, ck);
+          }
+        atomicAdd(&colk[n0 + 8 * nt + 2 * t + par], ck);
       }
-      atomicAdd(&colk[c], ck);
-    }
   }
-  __syncthreads();   // dT complete
+  __syncthreads();   // dT complete; the products reading Fs and Bs are done
+  stage_rows<D>(Fs, LDD, q, rs, p.n, tid);   // raw q and k, scaled below
+  stage_rows<D>(Bs, LDD, k, rs, p.n, tid);
+  cp_async_commit();
   {  // M = X^T dT Diag(beta); the first dbeta term, colsum(X o dT)
-    float m[4][4];
-    zero(m);
-    gemm_acc<4, 4>(m, Xs, 1, LDC, dTs, LDC, 1, CH, ty, tx);
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int c = tx + 16 * j;
-        Ms[(ty + 16 * i) * LDC + c] = m[i][j] * bs[c];
-      }
+    float m[1][4][4];
+    zero4(m);
+    wmma3<1, 4>(m, Xs, 1, LDC, dTs, LDC, 1, CH, p0, q0, lane);
+    FRAG_LOOP(1, 4) {
+      const int c = FRAG_C(q0);
+      Ms[FRAG_R(p0) * LDC + c] = m[mt][nt][i] * bs[c];
+    }
     if (tid < CH) {
       float s = 0.f;
       for (int r = 0; r < CH; ++r) s = fmaf(Xs[r * LDC + tid], dTs[r * LDC + tid], s);
@@ -629,90 +771,84 @@ __global__ void __launch_bounds__(NT, 1) cbwd_local_grad_kernel(CbwdArgs a) {
     }
   }
   // q e^{g - g_m} and k e^{g_m - g} replace dW e^{g_m} and dU, whose products are done
-  for (int idx = tid; idx < CH * D; idx += NT) {
-    const int r = idx / D, c = idx % D;
-    const bool in = r < p.n;
-    const float x = Gs[r * LDD + c] - gm[c];
-    Fs[r * LDD + c] = in ? q[r * rs + c] * expf(x) : 0.f;
-    Bs[r * LDD + c] = in ? k[r * rs + c] * expf(-x) : 0.f;
+  cp_async_wait_all();
+  __syncthreads();
+  for (int idx = tid; idx < CH * D / 4; idx += NT) {
+    const int r = idx / (D / 4), c4 = (idx % (D / 4)) * 4;
+    float* fp = Fs + r * LDD + c4;
+    float* bp = Bs + r * LDD + c4;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float x = Gs[r * LDD + c4 + j] - gm[c4 + j];
+      fp[j] *= expf(x);
+      bp[j] *= expf(-x);
+    }
   }
   __syncthreads();
   {  // dA = -strict(M X^T); the second dbeta term, rowsum(dA o A/beta); dAb = Diag(beta) dA
-    float m[4][4];
-    zero(m);
-    gemm_acc<4, 4>(m, Ms, LDC, 1, Xs, 1, LDC, CH, ty, tx);
+    float m[1][4][4];
+    zero4(m);
+    wmma3<1, 4>(m, Ms, LDC, 1, Xs, 1, LDC, CH, p0, q0, lane);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int r = ty + 16 * i;
+    for (int hi = 0; hi < 2; ++hi) {
+      const int r = p0 + g + 8 * hi;
       float part = 0.f;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int c = tx + 16 * j;
-        const float dA = c < r ? -m[i][j] : 0.f;
-        part = fmaf(dA, Abs[r * LDC + c], part);
-        Abs[r * LDC + c] = dA * bs[r];
-      }
+      for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+        for (int par = 0; par < 2; ++par) {
+          const int c = q0 + 8 * nt + 2 * t + par;
+          const float dA = c < r ? -m[0][nt][2 * hi + par] : 0.f;
+          part = fmaf(dA, Abs[r * LDC + c], part);
+          Abs[r * LDC + c] = dA * bs[r];
+        }
       atomicAdd(&db[r], part);
     }
   }
   __syncthreads();
   if (tid < p.n) a.dbeta[p.tok0 + (int64_t)tid * a.H] = db[tid];
   {  // R2 = e^{g - g_m} o (dP KN): dq, and R1 = e^{g - g_m} o (dAb KN): dk
-    float acc[4][TN];
-    zero(acc);
-    gemm_acc<4, TN>(acc, dPs, LDC, 1, Bs, LDD, 1, CH, ty, tx);
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < TN; ++j) {
-        const int r = ty + 16 * i, c = tx + 16 * j;
-        const float r2 = acc[i][j] * expf(Gs[r * LDD + c] - gm[c]);
-        const float qv = r < p.n ? q[r * rs + c] : 0.f;
-        dq[i][j] += r2;
-        dg[i][j] = fmaf(qv, r2, dg[i][j]);
-      }
-    zero(acc);
-    gemm_acc<4, TN>(acc, Abs, LDC, 1, Bs, LDD, 1, CH, ty, tx);
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < TN; ++j) {
-        const int r = ty + 16 * i, c = tx + 16 * j;
-        const float r1 = acc[i][j] * expf(Gs[r * LDD + c] - gm[c]);
-        const float kv = r < p.n ? k[r * rs + c] : 0.f;
-        dk[i][j] += r1;
-        dg[i][j] = fmaf(kv, r1, dg[i][j]);
-      }
+    float acc[2][NTD][4];
+    zero4(acc);
+    wmma3<2, NTD>(acc, dPs, LDC, 1, Bs, LDD, 1, CH, m0, n0, lane);
+    FRAG_LOOP(2, NTD) {
+      const int r = FRAG_R(m0), c = FRAG_C(n0);
+      const float r2 = acc[mt][nt][i] * expf(Gs[r * LDD + c] - gm[c]);
+      const float qv = r < p.n ? q[r * rs + c] : 0.f;
+      dq[mt][nt][i] += r2;
+      dg[mt][nt][i] = fmaf(qv, r2, dg[mt][nt][i]);
+    }
+    zero4(acc);
+    wmma3<2, NTD>(acc, Abs, LDC, 1, Bs, LDD, 1, CH, m0, n0, lane);
+    FRAG_LOOP(2, NTD) {
+      const int r = FRAG_R(m0), c = FRAG_C(n0);
+      const float r1 = acc[mt][nt][i] * expf(Gs[r * LDD + c] - gm[c]);
+      const float kv = r < p.n ? k[r * rs + c] : 0.f;
+      dk[mt][nt][i] += r1;
+      dg[mt][nt][i] = fmaf(kv, r1, dg[mt][nt][i]);
+    }
   }
   {  // R3 = e^{g_m - g} o (dAb^T Kx + dP^T Qx): dk
-    float acc[4][TN];
-    zero(acc);
-    gemm_acc<4, TN>(acc, Abs, 1, LDC, Kx, LDD, 1, CH, ty, tx);
-    gemm_acc<4, TN>(acc, dPs, 1, LDC, Fs, LDD, 1, CH, ty, tx);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int r = ty + 16 * i;
+    float acc[2][NTD][4];
+    zero4(acc);
+    wmma3<2, NTD>(acc, Abs, 1, LDC, Kx, LDD, 1, CH, m0, n0, lane);
+    wmma3<2, NTD>(acc, dPs, 1, LDC, Fs, LDD, 1, CH, m0, n0, lane);
+    FRAG_LOOP(2, NTD) {
+      const int r = FRAG_R(m0), c = FRAG_C(n0);
       const bool in = r < p.n;
-#pragma unroll
-      for (int j = 0; j < TN; ++j) {
-        const int c = tx + 16 * j;
-        const float r3 = acc[i][j] * expf(gm[c] - Gs[r * LDD + c]);
-        const float kv = in ? k[r * rs + c] : 0.f;
-        dk[i][j] += r3;
-        dg[i][j] = fmaf(-kv, r3, dg[i][j]);
-        if (in) {
-          const int64_t t = (p.tok0 + (int64_t)r * a.H) * D + c;
-          a.dq[t] = dq[i][j];
-          a.dk[t] = dk[i][j];
-        }
+      const float r3 = acc[mt][nt][i] * expf(gm[c] - Gs[r * LDD + c]);
+      const float kv = in ? k[r * rs + c] : 0.f;
+      dk[mt][nt][i] += r3;
+      dg[mt][nt][i] = fmaf(-kv, r3, dg[mt][nt][i]);
+      if (in) {
+        const int64_t tk = (p.tok0 + (int64_t)r * a.H) * D + c;
+        a.dq[tk] = dq[mt][nt][i];
+        a.dk[tk] = dk[mt][nt][i];
       }
     }
   }
   __syncthreads();   // every read of g is done: Gs takes dg
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < TN; ++j) Gs[(ty + 16 * i) * LDD + tx + 16 * j] = dg[i][j];
+  FRAG_LOOP(2, NTD) Gs[FRAG_R(m0) * LDD + FRAG_C(n0)] = dg[mt][nt][i];
   __syncthreads();
   if (tid < D) {   // dlog alpha = reverse running sum of dg; the exit terms enter at the last row
     float s = colk[tid] + a.w.last[p.ch * D + tid];
@@ -722,6 +858,7 @@ __global__ void __launch_bounds__(NT, 1) cbwd_local_grad_kernel(CbwdArgs a) {
     }
   }
 }
+
 template <typename T>
 __global__ void bwd_beta_kernel(const float* src, T* dst, int64_t n) {
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
