@@ -1,7 +1,7 @@
 // Backward pass of the modality-aware short convolution + KDA scan: the
 // gradients of kda_fwd's outputs (o and the final state) with respect to q, k,
-// v, log alpha, beta, the conv weights and the initial state.  fp32 on the CUDA
-// cores.
+// v, log alpha, beta, the conv weights and the initial state, at fp32 accuracy
+// (products on the tensor cores as split tf32, see wmma3).
 //
 // Forward step per head (paper.rainbus.top, section 方法步骤详情, step (5)):
 //     S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T,   o_t = S_t^T q_t.
