@@ -229,18 +229,22 @@ __device__ __forceinline__ void ld8_act(const void* p, int64_t i, bool bf16, flo
   }
 }
 
-// running sum over the chunk's rows, per key channel (threads < D); g_m and g_l per channel
+// running sum over the chunk's rows, per key channel (threads < D); per channel g_m, g_l,
+// e^{g_m} and e^{g_l - g_m}
 template <int D>
-__device__ __forceinline__ void chunk_cumsum(float* Gs, float* gm, float* gl, int tid) {
+__device__ __forceinline__ void chunk_cumsum(float* Gs, float* gm, float* gl, float* egm, float* eglm, int tid) {
   constexpr int LDD = D + 4;
   if (tid < D) {
-    float s = 0.f;
+    float s = 0.f, m = 0.f;
     for (int r = 0; r < CH; ++r) {
       s += Gs[r * LDD + tid];
       Gs[r * LDD + tid] = s;
-      if (r == CH / 2 - 1) gm[tid] = s;
+      if (r == CH / 2 - 1) m = s;
     }
+    gm[tid] = m;
     gl[tid] = s;
+    egm[tid] = expf(m);
+    eglm[tid] = expf(s - m);
   }
 }
 
@@ -274,7 +278,7 @@ __device__ __forceinline__ ChunkPos chunk_pos(const CbwdArgs& a) {
 #define FRAG_C(n0) ((n0) + 8 * nt + 2 * t + (i & 1))
 
 template <int D>
-constexpr size_t prep_smem() { return sizeof(float) * (4 * CH * (D + 4) + 2 * CH * LDC + 2 * D + CH); }
+constexpr size_t prep_smem() { return sizeof(float) * (4 * CH * (D + 4) + 2 * CH * LDC + 4 * D + CH); }
 
 template <int D>
 __global__ void __launch_bounds__(NT, 1) cbwd_prep_kernel(CbwdArgs a) {
@@ -288,7 +292,9 @@ __global__ void __launch_bounds__(NT, 1) cbwd_prep_kernel(CbwdArgs a) {
   float* Ps = As + CH * LDC;      // P
   float* gm = Ps + CH * LDC;      // [D]
   float* gl = gm + D;             // [D]
-  float* bs = gl + D;             // [CH] beta
+  float* egm = gl + D;            // [D] e^{g_m}
+  float* eglm = egm + D;          // [D] e^{g_l - g_m}
+  float* bs = eglm + D;           // [CH] beta
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = lane >> 2, t = lane & 3;
   const ChunkPos p = chunk_pos(a);
   const int64_t rs = (int64_t)a.H * D;
@@ -300,7 +306,7 @@ __global__ void __launch_bounds__(NT, 1) cbwd_prep_kernel(CbwdArgs a) {
   if (tid < CH) bs[tid] = tid < p.n ? ld_act(a.beta, p.tok0 + (int64_t)tid * a.H, a.bf16) : 0.f;
   cp_async_wait_all();
   __syncthreads();
-  chunk_cumsum<D>(Gs, gm, gl, tid);
+  chunk_cumsum<D>(Gs, gm, gl, egm, eglm, tid);
   __syncthreads();
   bool bad = false;
   float* Kt = a.w.Kt + p.ch * CH * D;
@@ -315,11 +321,11 @@ __global__ void __launch_bounds__(NT, 1) cbwd_prep_kernel(CbwdArgs a) {
     for (int j = 0; j < 4; ++j) {
       const float x = gv[j] - gm[c4 + j];
       bad |= fabsf(x) > kRange;
-      const float ep = expf(x), en = expf(-x);
+      const float ep = expf(x), en = __fdividef(1.f, ep);   // |x| <= kRange: both well inside fp32
       kx[j] = kv[j] * ep;
       kn[j] = kv[j] * en;
       qx[j] = qv[j] * ep;
-      kt[j] = kv[j] * expf(gl[c4 + j] - gv[j]);
+      kt[j] = kv[j] * (eglm[c4 + j] * en);                  // e^{g_l - g}
     }
     *reinterpret_cast<float4*>(Kx + r * LDD + c4) = make_float4(kx[0], kx[1], kx[2], kx[3]);
     *reinterpret_cast<float4*>(KN + r * LDD + c4) = make_float4(kn[0], kn[1], kn[2], kn[3]);
@@ -406,7 +412,7 @@ __global__ void __launch_bounds__(NT, 1) cbwd_prep_kernel(CbwdArgs a) {
     float* W = a.w.W + p.ch * CH * D;
     FRAG_LOOP(2, NTD) {
       const int r = FRAG_R(m0), c = FRAG_C(n0);
-      W[r * D + c] = acc[mt][nt][i] * expf(gm[c]);
+      W[r * D + c] = acc[mt][nt][i] * egm[c];
     }
     zero4(acc);
     wmma3<2, NTD>(acc, As, LDC, 1, KN, LDD, 1, CH, m0, n0, lane);
@@ -425,7 +431,7 @@ __global__ void __launch_bounds__(NT, 1) cbwd_prep_kernel(CbwdArgs a) {
     float* Y = a.w.Y + p.ch * D * D;
     FRAG_LOOP(D / 64, D / 16) {
       const int r = FRAG_R(m0);
-      Y[r * D + FRAG_C(n0)] = acc[mt][nt][i] * expf(gm[r]);
+      Y[r * D + FRAG_C(n0)] = acc[mt][nt][i] * egm[r];
     }
   }
 }
@@ -648,13 +654,13 @@ __global__ void __launch_bounds__(NT) cbwd_state_grad_kernel(CbwdArgs a) {
 
 // ---- the chunk-local part of the adjoint ---------------------------------------------
 template <int D>
-constexpr size_t local_grad_smem() { return sizeof(float) * (4 * CH * (D + 4) + 5 * CH * LDC + 3 * D + 2 * CH); }
+constexpr size_t local_grad_smem() { return sizeof(float) * (4 * CH * (D + 4) + 5 * CH * LDC + 5 * D + 2 * CH); }
 
 template <int D>
 __global__ void __launch_bounds__(NT, 1) cbwd_local_grad_kernel(CbwdArgs a) {
   constexpr int LDD = D + 4, NTD = D / 32;
   extern __shared__ __align__(16) float sm[];
-  float* Gs = sm;                 // [CH][LDD] g, at the end dg
+  float* Gs = sm;                 // [CH][LDD] g, then E = e^{g - g_m}, at the end dg
   float* Kx = Gs + CH * LDD;      // k e^{g - g_m}
   float* Fs = Kx + CH * LDD;      // dW e^{g_m}, later q e^{g - g_m}
   float* Bs = Fs + CH * LDD;      // dU, later k e^{g_m - g}
@@ -665,7 +671,9 @@ __global__ void __launch_bounds__(NT, 1) cbwd_local_grad_kernel(CbwdArgs a) {
   float* Abs = dPs + CH * LDC;    // A / beta, later Diag(beta) dA
   float* gm = Abs + CH * LDC;     // [D]
   float* gl = gm + D;             // [D]
-  float* colk = gl + D;           // [D] column sums of dKt o Kt
+  float* egm = gl + D;            // [D] e^{g_m}
+  float* eglm = egm + D;          // [D] e^{g_l - g_m}
+  float* colk = eglm + D;         // [D] column sums of dKt o Kt
   float* bs = colk + D;           // [CH]
   float* db = bs + CH;            // [CH] dbeta
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, g = lane >> 2, t = lane & 3;
@@ -691,16 +699,21 @@ __global__ void __launch_bounds__(NT, 1) cbwd_local_grad_kernel(CbwdArgs a) {
   if (tid < D) colk[tid] = 0.f;
   cp_async_wait_all();
   __syncthreads();
-  chunk_cumsum<D>(Gs, gm, gl, tid);
+  chunk_cumsum<D>(Gs, gm, gl, egm, eglm, tid);
   __syncthreads();
-  for (int idx = tid; idx < CH * D / 4; idx += NT) {   // Kx = k e^{g - g_m}, Fs = dW e^{g_m}, in place
+  // in place: E = e^{g - g_m} replaces g (every later use of g is through E and 1/E),
+  // Kx = k E, Fs = dW e^{g_m}
+  for (int idx = tid; idx < CH * D / 4; idx += NT) {
     const int r = idx / (D / 4), c4 = (idx % (D / 4)) * 4;
+    float* ep = Gs + r * LDD + c4;
     float* kp = Kx + r * LDD + c4;
     float* fp = Fs + r * LDD + c4;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      kp[j] *= expf(Gs[r * LDD + c4 + j] - gm[c4 + j]);
-      fp[j] *= expf(gm[c4 + j]);
+      const float e = expf(ep[j] - gm[c4 + j]);
+      ep[j] = e;
+      kp[j] *= e;
+      fp[j] *= egm[c4 + j];
     }
   }
   __syncthreads();
@@ -739,8 +752,8 @@ __global__ void __launch_bounds__(NT, 1) cbwd_local_grad_kernel(CbwdArgs a) {
             const int i = 2 * hi + par;
             const int r = FRAG_R(m0), c = FRAG_C(n0);
             const bool in = r < p.n;
-            const float gv = Gs[r * LDD + c];
-            const float e1 = expf(gv - gm[c]), e2 = expf(gl[c] - gv), eg = expf(gv);
+            const float e1 = Gs[r * LDD + c];
+            const float e2 = eglm[c] * __fdividef(1.f, e1), eg = egm[c] * e1;   // e^{g_l - g}, e^{g}
             const float kv = in ? k[r * rs + c] : 0.f, qv = in ? q[r * rs + c] : 0.f;
             const float dkt = dKt[r * D + c], dqg = dQG[r * D + c];
             const float av = bs[r] * acc[mt][nt][i] * e1;   // dKG o e^g
@@ -779,9 +792,9 @@ __global__ void __launch_bounds__(NT, 1) cbwd_local_grad_kernel(CbwdArgs a) {
     float* bp = Bs + r * LDD + c4;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const float x = Gs[r * LDD + c4 + j] - gm[c4 + j];
-      fp[j] *= expf(x);
-      bp[j] *= expf(-x);
+      const float e = Gs[r * LDD + c4 + j];
+      fp[j] *= e;
+      bp[j] *= __fdividef(1.f, e);
     }
   }
   __syncthreads();
@@ -813,7 +826,7 @@ __global__ void __launch_bounds__(NT, 1) cbwd_local_grad_kernel(CbwdArgs a) {
     wmma3<2, NTD>(acc, dPs, LDC, 1, Bs, LDD, 1, CH, m0, n0, lane);
     FRAG_LOOP(2, NTD) {
       const int r = FRAG_R(m0), c = FRAG_C(n0);
-      const float r2 = acc[mt][nt][i] * expf(Gs[r * LDD + c] - gm[c]);
+      const float r2 = acc[mt][nt][i] * Gs[r * LDD + c];
       const float qv = r < p.n ? q[r * rs + c] : 0.f;
       dq[mt][nt][i] += r2;
       dg[mt][nt][i] = fmaf(qv, r2, dg[mt][nt][i]);
@@ -822,7 +835,7 @@ __global__ void __launch_bounds__(NT, 1) cbwd_local_grad_kernel(CbwdArgs a) {
     wmma3<2, NTD>(acc, Abs, LDC, 1, Bs, LDD, 1, CH, m0, n0, lane);
     FRAG_LOOP(2, NTD) {
       const int r = FRAG_R(m0), c = FRAG_C(n0);
-      const float r1 = acc[mt][nt][i] * expf(Gs[r * LDD + c] - gm[c]);
+      const float r1 = acc[mt][nt][i] * Gs[r * LDD + c];
       const float kv = r < p.n ? k[r * rs + c] : 0.f;
       dk[mt][nt][i] += r1;
       dg[mt][nt][i] = fmaf(kv, r1, dg[mt][nt][i]);
@@ -836,7 +849,7 @@ __global__ void __launch_bounds__(NT, 1) cbwd_local_grad_kernel(CbwdArgs a) {
     FRAG_LOOP(2, NTD) {
       const int r = FRAG_R(m0), c = FRAG_C(n0);
       const bool in = r < p.n;
-      const float r3 = acc[mt][nt][i] * expf(gm[c] - Gs[r * LDD + c]);
+      const float r3 = acc[mt][nt][i] * __fdividef(1.f, Gs[r * LDD + c]);
       const float kv = in ? k[r * rs + c] : 0.f;
       dk[mt][nt][i] += r3;
       dg[mt][nt][i] = fmaf(-kv, r3, dg[mt][nt][i]);
