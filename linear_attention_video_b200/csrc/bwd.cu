@@ -106,15 +106,12 @@ struct CbwdArgs {
 
 // ---- warp-level tensor-core products (mma.sync m16n8k8, tf32) ----------------------
 // Each operand is split as x = hi + lo (both tf32) and a product is formed as
-// hi*hi + hi*lo + lo*hi, which keeps it at about fp32 accuracy.
-__device__ __forceinline__ uint32_t tf32_of(float x) {
-  uint32_t r;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-  return r;
-}
+// hi*hi + hi*lo + lo*hi, which keeps it at about fp32 accuracy (relative error near 2^-20).
 __device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) {
-  hi = tf32_of(x);
-  lo = tf32_of(x - __uint_as_float(hi));
+  // hi: x with the 13 low mantissa bits cleared (a tf32 value); lo: the exact remainder x - hi,
+  // cleared the same way (its dropped bits are below 2^-20 of |x|)
+  hi = __float_as_uint(x) & 0xffffe000u;
+  lo = __float_as_uint(x - __uint_as_float(hi)) & 0xffffe000u;
 }
 __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
   asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
