@@ -176,11 +176,9 @@ struct PrepArgs {
 // as x = hi + lo (both tf32): C = A_hi B_hi + A_hi B_lo + A_lo B_hi.  Fragment
 // coordinates: g = lane / 4, t = lane % 4; d[0..3] = C[g][2t], C[g][2t+1],
 // C[g+8][2t], C[g+8][2t+1].
-__device__ __forceinline__ uint32_t tf32_hi(float x) {
-  uint32_t r;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-  return r;
-}
+// x with its 13 low mantissa bits cleared: a tf32 value; applied to x and to the exact
+// remainder x - hi it splits x into two tf32 terms (dropped bits below 2^-20 of |x|)
+__device__ __forceinline__ uint32_t tf32_hi(float x) { return __float_as_uint(x) & 0xffffe000u; }
 __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
   asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
                : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
