@@ -141,6 +141,35 @@ int kda_fwd(const kda_problem* p, kda_dtype dtype,
             const float* initial_state, void* o, float* final_state,
             void* workspace, size_t workspace_bytes, void* stream);
 
+/* kda_fwd on host-resident tensors, with the host<->device copies overlapped with the kernels.
+ * The pages describe no host interface; this is the call for data that lives in host memory.
+ *   q, k, v, log_alpha, beta: host pointers, layouts as in kda_fwd; o: host pointer [B, N, H, d].
+ *     Page-locked (pinned) memory lets the copies run asynchronously; pageable memory works but
+ *     each copy then blocks the calling thread.  They must stay valid and unchanged until the
+ *     stream has passed the call.
+ *   w_text, w_vis, initial_state, final_state: device pointers, as in kda_fwd.
+ *   seg_frames >= 1: visual frames per segment.  Each batch item's token stream is cut into
+ *     segments of seg_frames frames (its text prefix goes with the first); a segment's inputs are
+ *     copied in on copy_in_stream, its conv and scan run on stream (the scan entering with the
+ *     state the previous segment left, so o and final_state equal kda_fwd's up to the rounding
+ *     of the scan's chunking at segment starts), and its o is copied out on copy_out_stream.
+ *     Copies of one segment overlap the kernels of its neighbours.
+ *   stream, copy_in_stream, copy_out_stream: caller-owned streams (three distinct streams for
+ *     the overlap).  The copies in wait for the work enqueued on `stream` before the call; once
+ *     `stream` has passed the call, o is in host memory and final_state is written.
+ * The call creates and releases a few CUDA events; it allocates no memory and does not
+ * synchronise.  Workspace: kda_fwd_host_workspace_bytes(p, dtype, seg_frames) device bytes,
+ * 256-byte aligned (the inputs and o staged in full, the conv outputs, two states and the scan
+ * records of one segment).  Flags as in kda_fwd.  Returns a kda_status. */
+size_t kda_fwd_host_workspace_bytes(const kda_problem* p, kda_dtype dtype, int32_t seg_frames);
+int kda_fwd_host(const kda_problem* p, kda_dtype dtype,
+                 const void* q, const void* k, const void* v,
+                 const float* log_alpha, const void* beta,
+                 const float* w_text, const float* w_vis,
+                 const float* initial_state, void* o, float* final_state, int32_t seg_frames,
+                 void* workspace, size_t workspace_bytes, void* stream,
+                 void* copy_in_stream, void* copy_out_stream);
+
 /* Backward pass of kda_fwd: the gradients of the loss sum(d_o * o) + sum(d_final_state * S_N)
  * (o and S_N as kda_fwd computes them from the same arguments) with respect to every input.
  * The pages describe only the forward pass; the gradients are the chain rule applied to it

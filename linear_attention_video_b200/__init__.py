@@ -32,7 +32,7 @@ KDA_FLAG_REUSE_RECORDS = 2
 KDA_FLAG_QKV_F16 = 4
 
 EXPORTS = ("kda_tokens", "kda_workspace_bytes", "kda_shortconv_fwd", "kda_chunk_fwd", "kda_fwd",
-           "kda_chunk_fwd_noalloc", "kda_bwd_workspace_bytes", "kda_bwd", "kda_read_status", "kda_status_str",
+           "kda_chunk_fwd_noalloc", "kda_fwd_host_workspace_bytes", "kda_fwd_host", "kda_bwd_workspace_bytes", "kda_bwd", "kda_read_status", "kda_status_str",
            "kda_last_launch_count")
 
 
@@ -58,6 +58,10 @@ _lib.kda_fwd.argtypes = [_pp, _i] + [_vp] * 11 + [_sz, _vp]
 _lib.kda_fwd.restype = _i
 _lib.kda_chunk_fwd_noalloc.argtypes = [_pp, _i] + [_vp] * 10
 _lib.kda_chunk_fwd_noalloc.restype = _i
+_lib.kda_fwd_host_workspace_bytes.argtypes = [_pp, _i, ctypes.c_int32]
+_lib.kda_fwd_host_workspace_bytes.restype = _sz
+_lib.kda_fwd_host.argtypes = [_pp, _i] + [_vp] * 10 + [ctypes.c_int32, _vp, _sz, _vp, _vp, _vp]
+_lib.kda_fwd_host.restype = _i
 _lib.kda_bwd_workspace_bytes.argtypes = [_pp, _i]
 _lib.kda_bwd_workspace_bytes.restype = _sz
 _lib.kda_bwd.argtypes = [_pp, _i] + [_vp] * 19 + [_sz, _vp]
@@ -162,6 +166,29 @@ def kda_fwd(p, q, k, v, log_alpha, beta, w_text, w_vis, o, workspace, initial_st
                         _ptr(w_text), _ptr(w_vis), _ptr(initial_state), _ptr(o), _ptr(final_state),
                         _ptr(workspace), nbytes, _stream(stream)),
            "kda_fwd")
+
+
+def kda_fwd_host_workspace_bytes(p: kda_problem, dtype, seg_frames: int) -> int:
+    return _lib.kda_fwd_host_workspace_bytes(ctypes.byref(p), _dt(dtype), int(seg_frames))
+
+
+def alloc_fwd_host_workspace(p: kda_problem, dtype, seg_frames: int, device="cuda") -> torch.Tensor:
+    n = kda_fwd_host_workspace_bytes(p, dtype, seg_frames)
+    if n == 0:
+        raise KdaError(KDA_ERR_INVALID_ARG, "kda_fwd_host_workspace_bytes")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def kda_fwd_host(p, q, k, v, log_alpha, beta, w_text, w_vis, o, workspace, seg_frames, initial_state=None,
+                 final_state=None, stream=None, copy_in_stream=None, copy_out_stream=None, workspace_bytes=None):
+    """kda_fwd on host tensors (q, k, v, log_alpha, beta, o on the CPU, pinned for overlap); the weights,
+    the states and the workspace are on the device."""
+    nbytes = workspace.numel() * workspace.element_size() if workspace_bytes is None else workspace_bytes
+    _check(_lib.kda_fwd_host(ctypes.byref(p), _dt(q.dtype), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                             _ptr(w_text), _ptr(w_vis), _ptr(initial_state), _ptr(o), _ptr(final_state),
+                             int(seg_frames), _ptr(workspace), nbytes, _stream(stream), _stream(copy_in_stream),
+                             _stream(copy_out_stream)),
+           "kda_fwd_host")
 
 
 def kda_chunk_fwd_noalloc(p, q, k, v, log_alpha, beta, o, initial_state=None, final_state=None,

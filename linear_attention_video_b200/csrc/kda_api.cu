@@ -2,6 +2,9 @@
 // The operations and layouts are documented in include/kda.h.
 #include <string.h>
 
+#include <algorithm>
+#include <vector>
+
 #include "common.cuh"
 
 namespace {
@@ -105,6 +108,45 @@ int run_scan(const kda::Dims& d, kda_dtype dt, const void* q, const void* k, con
     return cuda_status(kda::launch_chunk_tc(d, in_f16, q, k, v, la, beta, S0, o, SN, rec, status, s, launches));
   }
   return cuda_status(kda::launch_chunk_simt(d, dt, q, k, v, la, beta, S0, o, SN, status, s, launches));
+}
+
+// ---- kda_fwd on host-resident tensors -------------------------------------------------
+// The token stream of each batch item is cut into segments of seg_frames visual frames (the
+// text prefix goes with the first).  Per segment: its inputs are copied in on the copy-in
+// stream, its conv and scan run on the caller's stream (the scan entering with the state the
+// previous segment left), and its o is copied out on the copy-out stream; events order the
+// three, so copies of neighbouring segments overlap the kernels.  The conv of a segment reads
+// the neighbouring frames its taps reach (pt before, 2 - pt after): its view is that frame range,
+// and the outputs it computes for the halo frames (with zeros beyond the view) are discarded:
+// the earlier segment has already used its own, and the next one recomputes them first.
+struct HostLayout {
+  size_t act, la, beta, state, rec, total;
+};
+
+kda::Dims segment_dims(const kda::Dims& d, int64_t n_tokens) {   // a 1-item, text-only view of n tokens
+  kda::Dims s = d;
+  s.B = 1;
+  s.N = n_tokens;
+  s.L = n_tokens;
+  s.T = s.Hg = s.Wg = 0;
+  return s;
+}
+
+int64_t max_segment_tokens(const kda::Dims& d, int seg_frames) {
+  return d.L + (int64_t)std::min(seg_frames, d.T) * d.Hg * d.Wg;
+}
+
+// status | q, k, v, log alpha, beta, o staged on the device | q', k', v' | two per-item states | scan records
+HostLayout host_layout(const kda::Dims& d, kda_dtype dt, int seg_frames) {
+  HostLayout l;
+  l.act = align256(act_bytes(d, dt));
+  l.la = align256((size_t)d.B * d.N * d.H * d.dk * sizeof(float));
+  l.beta = align256((size_t)d.B * d.N * d.H * elem_size(dt));
+  l.state = align256((size_t)d.H * d.dk * d.dv * sizeof(float));
+  l.rec = use_tc(d, dt) ? align256(kda::chunk_tc_workspace_bytes(segment_dims(d, max_segment_tokens(d, seg_frames))))
+                        : 0;
+  l.total = kStatusBytes + 7 * l.act + l.la + l.beta + 2 * l.state + l.rec;
+  return l;
 }
 
 }  // namespace
@@ -230,6 +272,147 @@ int kda_bwd(const kda_problem* p, kda_dtype dtype, const void* q, const void* k,
                                    d_initial_state, workspace, s, &launches));
   if (!st) g_last_launches = launches;
   return st;
+}
+
+size_t kda_fwd_host_workspace_bytes(const kda_problem* p, kda_dtype dtype, int32_t seg_frames) {
+  kda::Dims d;
+  if (make_dims(p, dtype, &d) != KDA_OK || d.reuse_records || d.qkv_f16 || seg_frames < 1) return 0;
+  return host_layout(d, dtype, seg_frames).total;
+}
+
+int kda_fwd_host(const kda_problem* p, kda_dtype dtype, const void* q, const void* k, const void* v,
+                 const float* log_alpha, const void* beta, const float* w_text, const float* w_vis,
+                 const float* initial_state, void* o, float* final_state, int32_t seg_frames, void* workspace,
+                 size_t workspace_bytes_, void* stream, void* copy_in_stream, void* copy_out_stream) {
+  g_last_launches = 0;
+  kda::Dims d;
+  int st = make_dims(p, dtype, &d);
+  if (st) return st;
+  if (d.reuse_records || d.qkv_f16 || seg_frames < 1) return KDA_ERR_INVALID_ARG;
+  if ((st = check_ptrs({q, k, v, log_alpha, beta, w_text, w_vis, o}, {initial_state, final_state}))) return st;
+  const HostLayout l = host_layout(d, dtype, seg_frames);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes_ < l.total)
+    return KDA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaStream_t cin = static_cast<cudaStream_t>(copy_in_stream), cout = static_cast<cudaStream_t>(copy_out_stream);
+  char* ws = static_cast<char*>(workspace);
+  uint32_t* status = reinterpret_cast<uint32_t*>(ws);
+  char* base = ws + kStatusBytes;
+  char* dq = base;                  // staged inputs and output, layouts as in kda_fwd
+  char* dk = dq + l.act;
+  char* dv = dk + l.act;
+  char* dout = dv + l.act;
+  char* qc = dout + l.act;          // conv outputs (fp16 on the tensor-core path)
+  char* kc = qc + l.act;
+  char* vc = kc + l.act;
+  float* dla = reinterpret_cast<float*>(vc + l.act);
+  char* dbeta = reinterpret_cast<char*>(dla) + l.la;
+  float* state[2] = {reinterpret_cast<float*>(dbeta + l.beta), reinterpret_cast<float*>(dbeta + l.beta + l.state)};
+  void* rec = dbeta + l.beta + 2 * l.state;
+  const bool tc = use_tc(d, dtype);
+  const size_t es = elem_size(dtype), row = (size_t)d.H * d.dk;   // one token of q, k, v, o: row elements
+  const int64_t HW = (int64_t)d.Hg * d.Wg;
+  const int before = d.pt, after = 2 - d.pt;                      // frames the conv taps reach
+  const int nseg_item = d.T > 0 ? (d.T + seg_frames - 1) / seg_frames : 1;
+  const int nseg = d.B * nseg_item;
+  if ((st = cuda_status(cudaMemsetAsync(status, 0, sizeof(uint32_t), s)))) return st;
+
+  std::vector<cudaEvent_t> ev(2 * nseg + 2, nullptr);
+  auto cleanup = [&]() {
+    for (cudaEvent_t e : ev)
+      if (e) cudaEventDestroy(e);   // released once the work they mark completes
+  };
+  for (cudaEvent_t& e : ev)
+    if ((st = cuda_status(cudaEventCreateWithFlags(&e, cudaEventDisableTiming)))) { cleanup(); return st; }
+  cudaEvent_t* ev_in = ev.data();
+  cudaEvent_t* ev_comp = ev.data() + nseg;
+  cudaEvent_t ev_start = ev[2 * nseg], ev_done = ev[2 * nseg + 1];
+  int launches = 0;
+  auto fail = [&](cudaError_t e) { cleanup(); return cuda_status(e); };
+  cudaError_t e;
+  // the copies wait for the caller's stream: earlier work there may still read the workspace
+  if ((e = cudaEventRecord(ev_start, s)) != cudaSuccess || (e = cudaStreamWaitEvent(cin, ev_start, 0)) != cudaSuccess)
+    return fail(e);
+  for (int b = 0; b < d.B; ++b) {
+    const int64_t item = (int64_t)b * d.N;   // first token of the item
+    int64_t copied = 0;                      // q, k, v tokens of the item already copied in
+    const size_t sbytes = (size_t)d.H * d.dk * d.dv * sizeof(float);
+    const float* S_in = initial_state ? initial_state + (size_t)b * d.H * d.dk * d.dv : nullptr;
+    if (d.N == 0) {   // nothing to scan: the state passes through
+      float* SN = final_state ? final_state + (size_t)b * d.H * d.dk * d.dv : nullptr;
+      if (SN && (e = S_in ? cudaMemcpyAsync(SN, S_in, sbytes, cudaMemcpyDeviceToDevice, s)
+                          : cudaMemsetAsync(SN, 0, sbytes, s)) != cudaSuccess)
+        return fail(e);
+      continue;
+    }
+    for (int sg = 0; sg < nseg_item; ++sg) {
+      const int id = b * nseg_item + sg;
+      const int f0 = sg * seg_frames, f1 = std::min(d.T, f0 + seg_frames);
+      const int64_t s_lo = f0 == 0 ? 0 : d.L + f0 * HW, s_hi = d.L + f1 * HW;   // this segment's tokens
+      const int fv0 = std::max(0, f0 - before), fv1 = std::min(d.T, f1 + after);
+      const int64_t v_lo = f0 == 0 ? 0 : d.L + fv0 * HW, v_hi = d.L + fv1 * HW;   // tokens the conv reads
+      // copy in: q, k, v up to the conv's last frame, log alpha and beta of the segment
+      if (v_hi > copied) {
+        const size_t off = (size_t)(item + copied) * row * es, n = (size_t)(v_hi - copied) * row * es;
+        for (int t = 0; t < 3; ++t) {
+          const void* src = t == 0 ? q : (t == 1 ? k : v);
+          char* dst = t == 0 ? dq : (t == 1 ? dk : dv);
+          if ((e = cudaMemcpyAsync(dst + off, static_cast<const char*>(src) + off, n, cudaMemcpyHostToDevice, cin)) !=
+              cudaSuccess)
+            return fail(e);
+        }
+        copied = v_hi;
+      }
+      {
+        const size_t t0 = (size_t)(item + s_lo), nt = (size_t)(s_hi - s_lo);
+        if ((e = cudaMemcpyAsync(dla + t0 * row, log_alpha + t0 * row, nt * row * sizeof(float), cudaMemcpyHostToDevice,
+                                 cin)) != cudaSuccess ||
+            (e = cudaMemcpyAsync(dbeta + t0 * d.H * es, static_cast<const char*>(beta) + t0 * d.H * es, nt * d.H * es,
+                                 cudaMemcpyHostToDevice, cin)) != cudaSuccess ||
+            (e = cudaEventRecord(ev_in[id], cin)) != cudaSuccess)
+          return fail(e);
+      }
+      // compute: the conv over the view, then the scan over the segment's tokens
+      if ((e = cudaStreamWaitEvent(s, ev_in[id], 0)) != cudaSuccess) return fail(e);
+      {
+        kda::Dims dvw = d;
+        dvw.B = 1;
+        dvw.L = f0 == 0 ? d.L : 0;
+        dvw.T = fv1 - fv0;
+        dvw.N = dvw.L + (int64_t)dvw.T * HW;
+        const size_t off = (size_t)(item + v_lo) * row * es;
+        if ((e = kda::launch_shortconv(dvw, dtype, dq + off, dk + off, dv + off, w_text, w_vis, qc + off, kc + off,
+                                       vc + off, s, &launches, tc)) != cudaSuccess)
+          return fail(e);
+      }
+      {
+        const kda::Dims dsg = segment_dims(d, s_hi - s_lo);
+        const size_t t0 = (size_t)(item + s_lo), off = t0 * row * es;
+        const bool last = sg == nseg_item - 1;
+        float* S_out = last ? (final_state ? final_state + (size_t)b * d.H * d.dk * d.dv : nullptr) : state[sg & 1];
+        e = tc ? kda::launch_chunk_tc(dsg, true, qc + off, kc + off, vc + off, dla + t0 * row, dbeta + t0 * d.H * es,
+                                      S_in, dout + off, S_out, rec, status, s, &launches)
+               : kda::launch_chunk_simt(dsg, dtype, qc + off, kc + off, vc + off, dla + t0 * row, dbeta + t0 * d.H * es,
+                                        S_in, dout + off, S_out, status, s, &launches);
+        if (e != cudaSuccess || (e = cudaEventRecord(ev_comp[id], s)) != cudaSuccess) return fail(e);
+        S_in = S_out;
+      }
+      // copy out
+      {
+        const size_t off = (size_t)(item + s_lo) * row * es, n = (size_t)(s_hi - s_lo) * row * es;
+        if ((e = cudaStreamWaitEvent(cout, ev_comp[id], 0)) != cudaSuccess ||
+            (e = cudaMemcpyAsync(static_cast<char*>(o) + off, dout + off, n, cudaMemcpyDeviceToHost, cout)) !=
+                cudaSuccess)
+          return fail(e);
+      }
+    }
+  }
+  // the caller's stream covers everything the call enqueued
+  if ((e = cudaEventRecord(ev_done, cout)) != cudaSuccess || (e = cudaStreamWaitEvent(s, ev_done, 0)) != cudaSuccess)
+    return fail(e);
+  cleanup();
+  g_last_launches = launches;
+  return KDA_OK;
 }
 
 int kda_read_status(void* workspace, void* stream) {
