@@ -108,6 +108,18 @@ def test_host_side_rejections_launch_nothing(kda):
         kda.KDA_ERR_MISALIGNED
     assert lib.kda_chunk_fwd(ctypes.byref(p), 0, 256, 256, 256, 256, None, None, 256, None, 512, 1 << 40, None) == \
         kda.KDA_ERR_INVALID_ARG
+    # host-buffer entry point: host-side checks before any CUDA call (no stream or event is touched)
+    host = lambda pp, **kw: lib.kda_fwd_host(ctypes.byref(pp), kw.get("dt", 0), *[kw.get(n, 256) for n in (   # noqa: E731
+        "q", "k", "v", "la", "beta", "wt", "wv", "s0", "o", "sn")], kw.get("seg", 4), kw.get("ws", 512),
+        kw.get("ws_bytes", 1 << 40), None, None, None)
+    assert host(p, seg=0) == kda.KDA_ERR_INVALID_ARG
+    assert host(p, q=None) == kda.KDA_ERR_INVALID_ARG
+    assert host(p, o=0x1008) == kda.KDA_ERR_MISALIGNED
+    assert host(p, ws=0x1010) == kda.KDA_ERR_WORKSPACE
+    assert host(p, ws_bytes=1000) == kda.KDA_ERR_WORKSPACE
+    assert host(reuse) == kda.KDA_ERR_INVALID_ARG
+    assert kda.kda_fwd_host_workspace_bytes(p, torch.bfloat16, 0) == 0
+    assert kda.kda_fwd_host_workspace_bytes(p, torch.bfloat16, 4) > kda.kda_workspace_bytes(p, torch.bfloat16)
     # backward entry point: host-side checks before any CUDA call
     lib.kda_bwd.restype = ctypes.c_int
     bwd = lambda pp, **kw: lib.kda_bwd(ctypes.byref(pp), kw.get("dt", 0), *[kw.get(n, 256) for n in (   # noqa: E731

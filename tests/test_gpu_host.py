@@ -76,12 +76,3 @@ def test_host_bf16_d128(kda, seg_frames):
     o, s = run_host(kda, w, inp, seg_frames)
     assert_parity(o, ref, "bf16", "o")
     assert rel_l2(s, ref_s) <= 5e-3
-
-
-def test_host_rejects_bad_arguments(kda):
-    import ctypes
-    w = kda_synth.WORKLOADS[0]
-    p = kda.problem(1, w.H, w.d, w.text_len, w.grid)
-    assert kda.kda_fwd_host_workspace_bytes(p, torch.float32, 0) == 0
-    assert kda._lib.kda_fwd_host(ctypes.byref(p), 1, *([256] * 10), 0, 256, 1 << 40, None, None, None) == \
-        kda.KDA_ERR_INVALID_ARG
