@@ -22,8 +22,8 @@
 //   conv (forward, fp32 out)   q', k', v' recomputed from the raw inputs
 //   cbwd_prep_kernel           per chunk: W, U~ = T V, Kt, X, A/beta, e^{gl}, and
 //                              the dO terms Z = P^T dO, Y = QG^T dO
-//   cbwd_fwd_chain_kernel      per CW value columns: S_in of every chunk, U
-//   cbwd_bwd_chain_kernel      per CW value columns, in reverse: dS of every chunk, dU, dS0
+//   cbwd_chain_kernel<D, false>  per CW value columns: S_in of every chunk, U
+//   cbwd_chain_kernel<D, true>   per CW value columns, in reverse: dS of every chunk, dU, dS0
 //   cbwd_state_grad_kernel     per chunk: the contractions with S_in and dS
 //                              (dQG, dW, dKt), dP, dU V^T
 //   cbwd_local_grad_kernel     per chunk: dT, the inverse's adjoint, dq, dk, dv,
