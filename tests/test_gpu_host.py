@@ -76,3 +76,19 @@ def test_host_bf16_d128(kda, seg_frames):
     o, s = run_host(kda, w, inp, seg_frames)
     assert_parity(o, ref, "bf16", "o")
     assert rel_l2(s, ref_s) <= 5e-3
+
+
+def test_host_text_only_and_causal_bf16(kda):
+    """A text-only problem (no frames: one segment per item) and the temporally causal conv on the
+    tensor-core path (halo of two frames before a segment, none after)."""
+    w = dataclasses.replace(kda_synth.WORKLOADS[0], B=2, text_len=77, grid=(0, 0, 0))
+    inp = kda_synth.generate(w, 44)
+    ref, ref_s = oracle.forward(inp, w.text_len, w.grid)
+    o, s = run_host(kda, w, inp, 4)
+    assert_parity(o, ref, "f32", "o")
+    assert rel_l2(s, ref_s) <= 1e-5
+    w = kda_synth.Workload("host_bf16_causal", 1, 4, 128, 64, (5, 8, 8), "bf16", 0.1)
+    inp = kda_synth.generate(w, 45)
+    ref, _ = oracle.forward(inp, w.text_len, w.grid, vis_causal_t=True)
+    o, _ = run_host(kda, w, inp, 2, causal=True)
+    assert_parity(o, ref, "bf16", "o")
