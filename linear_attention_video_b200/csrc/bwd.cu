@@ -113,6 +113,11 @@ __device__ __forceinline__ void split_tf32(float x, uint32_t& hi, uint32_t& lo) 
   hi = __float_as_uint(x) & 0xffffe000u;
   lo = __float_as_uint(x - __uint_as_float(hi)) & 0xffffe000u;
 }
+__device__ __forceinline__ uint32_t tf32_rn(float x) {   // nearest tf32 (single-product mode)
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
 __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
   asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
                : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
@@ -126,10 +131,39 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], 
 // even and odd k-steps go to four separate accumulators (summed at the end), for warps that
 // own one or two tiles and would otherwise wait on each product.  Shared-memory reads are free
 // of bank conflicts when a row stride along k (am or bn = ld, the other 1) is 4 mod 32 and a
-// row stride across k (ak or bk = ld) is 8 mod 32.
-template <int MT, int NT, bool CHAINS = false>
+// row stride across k (ak or bk = ld) is 8 mod 32.  SPLIT = false forms one product of the
+// operands rounded to the nearest tf32 (relative error near 2^-11, as an fp16 operand).
+template <int MT, int NT, bool CHAINS = false, bool SPLIT = true>
 __device__ __forceinline__ void wmma3(float (&c)[MT][NT][4], const float* A, int am, int ak, const float* B, int bk,
                                       int bn, int K, int m0, int n0, int lane) {
+  if (!SPLIT) {
+    const int g = lane >> 2, t = lane & 3;
+    const float* a0 = A + (m0 + g) * am + t * ak;
+    const float* b0 = B + t * bk + (n0 + g) * bn;
+#pragma unroll 2
+    for (int k0 = 0; k0 < K; k0 += 8) {
+      uint32_t ah[MT][4], bh[NT][2];
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) {
+        const float* p = a0 + 16 * mt * am + k0 * ak;
+        ah[mt][0] = tf32_rn(p[0]);
+        ah[mt][1] = tf32_rn(p[8 * am]);
+        ah[mt][2] = tf32_rn(p[4 * ak]);
+        ah[mt][3] = tf32_rn(p[8 * am + 4 * ak]);
+      }
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const float* p = b0 + k0 * bk + 8 * nt * bn;
+        bh[nt][0] = tf32_rn(p[0]);
+        bh[nt][1] = tf32_rn(p[4 * bk]);
+      }
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) mma_tf32(c[mt][nt], ah[mt], bh[nt]);
+    }
+    return;
+  }
   const int g = lane >> 2, t = lane & 3;
   const float* a0 = A + (m0 + g) * am + t * ak;
   const float* b0 = B + t * bk + (n0 + g) * bn;
@@ -277,7 +311,7 @@ __device__ __forceinline__ ChunkPos chunk_pos(const CbwdArgs& a) {
 template <int D>
 constexpr size_t prep_smem() { return sizeof(float) * (4 * CH * (D + 4) + 2 * CH * LDC + 4 * D + CH); }
 
-template <int D>
+template <int D, bool SPLIT>
 __global__ void __launch_bounds__(NT, 1) cbwd_prep_kernel(CbwdArgs a) {
   constexpr int LDD = D + 4, NTD = D / 32;
   extern __shared__ __align__(16) float sm[];
@@ -337,8 +371,8 @@ __global__ void __launch_bounds__(NT, 1) cbwd_prep_kernel(CbwdArgs a) {
     float ab[1][4][4], pp[1][4][4];
     zero4(ab);
     zero4(pp);
-    wmma3<1, 4>(ab, Kx, LDD, 1, KN, 1, LDD, D, m0, n0, lane);
-    wmma3<1, 4>(pp, Qx, LDD, 1, KN, 1, LDD, D, m0, n0, lane);
+    wmma3<1, 4, false, SPLIT>(ab, Kx, LDD, 1, KN, 1, LDD, D, m0, n0, lane);
+    wmma3<1, 4, false, SPLIT>(pp, Qx, LDD, 1, KN, 1, LDD, D, m0, n0, lane);
     float* Abg = a.w.Ab + p.ch * CH * CH;
     FRAG_LOOP(1, 4) {
       const int r = FRAG_R(m0), c = FRAG_C(n0);
@@ -405,18 +439,18 @@ __global__ void __launch_bounds__(NT, 1) cbwd_prep_kernel(CbwdArgs a) {
     const int m0 = 32 * (warp & 1), n0 = (D / 4) * (warp >> 1);
     float acc[2][NTD][4];
     zero4(acc);
-    wmma3<2, NTD>(acc, As, LDC, 1, Kx, LDD, 1, CH, m0, n0, lane);
+    wmma3<2, NTD, false, SPLIT>(acc, As, LDC, 1, Kx, LDD, 1, CH, m0, n0, lane);
     float* W = a.w.W + p.ch * CH * D;
     FRAG_LOOP(2, NTD) {
       const int r = FRAG_R(m0), c = FRAG_C(n0);
       W[r * D + c] = acc[mt][nt][i] * egm[c];
     }
     zero4(acc);
-    wmma3<2, NTD>(acc, As, LDC, 1, KN, LDD, 1, CH, m0, n0, lane);
+    wmma3<2, NTD, false, SPLIT>(acc, As, LDC, 1, KN, LDD, 1, CH, m0, n0, lane);
     float* Ut = a.w.Ut + p.ch * CH * D;
     FRAG_LOOP(2, NTD) Ut[FRAG_R(m0) * D + FRAG_C(n0)] = acc[mt][nt][i];
     zero4(acc);
-    wmma3<2, NTD>(acc, Ps, 1, LDC, Gs, LDD, 1, CH, m0, n0, lane);
+    wmma3<2, NTD, false, SPLIT>(acc, Ps, 1, LDC, Gs, LDD, 1, CH, m0, n0, lane);
     float* Z = a.w.Z + p.ch * CH * D;
     FRAG_LOOP(2, NTD) Z[FRAG_R(m0) * D + FRAG_C(n0)] = acc[mt][nt][i];
   }
@@ -424,7 +458,7 @@ __global__ void __launch_bounds__(NT, 1) cbwd_prep_kernel(CbwdArgs a) {
     const int m0 = (D / 4) * (warp & 3), n0 = (D / 2) * (warp >> 2);
     float acc[D / 64][D / 16][4];
     zero4(acc);
-    wmma3<D / 64, D / 16>(acc, Qx, 1, LDD, Gs, LDD, 1, CH, m0, n0, lane);
+    wmma3<D / 64, D / 16, false, SPLIT>(acc, Qx, 1, LDD, Gs, LDD, 1, CH, m0, n0, lane);
     float* Y = a.w.Y + p.ch * D * D;
     FRAG_LOOP(D / 64, D / 16) {
       const int r = FRAG_R(m0);
@@ -561,7 +595,7 @@ __global__ void __launch_bounds__(NT, 1) cbwd_chain_kernel(CbwdArgs a) {
 template <int D>
 constexpr size_t state_grad_smem() { return sizeof(float) * (2 * D * LDJ + 4 * CH * LDJ); }
 
-template <int D>
+template <int D, bool SPLIT>
 __global__ void __launch_bounds__(NT) cbwd_state_grad_kernel(CbwdArgs a) {
   constexpr int NTD = D / 32;
   extern __shared__ __align__(16) float sm[];
@@ -611,8 +645,8 @@ __global__ void __launch_bounds__(NT) cbwd_state_grad_kernel(CbwdArgs a) {
     float lastp = 0.f;
     for (int j0 = 0; j0 < D; j0 += JB) {
       stage(j0, false);
-      wmma3<2, NTD>(aq, dOb, LDJ, 1, S0b, 1, LDJ, JB, m0, n0, lane);
-      wmma3<2, NTD>(aw, dUb, LDJ, 1, S0b, 1, LDJ, JB, m0, n0, lane);
+      wmma3<2, NTD, false, SPLIT>(aq, dOb, LDJ, 1, S0b, 1, LDJ, JB, m0, n0, lane);
+      wmma3<2, NTD, false, SPLIT>(aw, dUb, LDJ, 1, S0b, 1, LDJ, JB, m0, n0, lane);
       if (tid < D)
 #pragma unroll 8
         for (int j = 0; j < JB; ++j) lastp = fmaf(dSb[tid * LDJ + j], S0b[tid * LDJ + j], lastp);
@@ -633,9 +667,9 @@ __global__ void __launch_bounds__(NT) cbwd_state_grad_kernel(CbwdArgs a) {
     zero4(auv);
     for (int j0 = 0; j0 < D; j0 += JB) {
       stage(j0, true);
-      wmma3<2, NTD>(ak, Ub, LDJ, 1, dSb, 1, LDJ, JB, m0, n0, lane);
-      wmma3<1, 4>(ap, dOb, LDJ, 1, Ub, 1, LDJ, JB, p0, q0, lane);
-      wmma3<1, 4>(auv, dUb, LDJ, 1, Vb, 1, LDJ, JB, p0, q0, lane);
+      wmma3<2, NTD, false, SPLIT>(ak, Ub, LDJ, 1, dSb, 1, LDJ, JB, m0, n0, lane);
+      wmma3<1, 4, false, SPLIT>(ap, dOb, LDJ, 1, Ub, 1, LDJ, JB, p0, q0, lane);
+      wmma3<1, 4, false, SPLIT>(auv, dUb, LDJ, 1, Vb, 1, LDJ, JB, p0, q0, lane);
     }
     float* dKt = a.w.dKt + p.ch * CH * D;
     float* dP = a.w.dP + p.ch * CH * CH;
@@ -653,7 +687,7 @@ __global__ void __launch_bounds__(NT) cbwd_state_grad_kernel(CbwdArgs a) {
 template <int D>
 constexpr size_t local_grad_smem() { return sizeof(float) * (4 * CH * (D + 4) + 5 * CH * LDC + 5 * D + 2 * CH); }
 
-template <int D>
+template <int D, bool SPLIT>
 __global__ void __launch_bounds__(NT, 1) cbwd_local_grad_kernel(CbwdArgs a) {
   constexpr int LDD = D + 4, NTD = D / 32;
   extern __shared__ __align__(16) float sm[];
@@ -717,7 +751,7 @@ __global__ void __launch_bounds__(NT, 1) cbwd_local_grad_kernel(CbwdArgs a) {
   {  // dT = dW KG^T + dU V^T
     float tt[1][4][4];
     zero4(tt);
-    wmma3<1, 4>(tt, Fs, LDD, 1, Kx, 1, LDD, D, p0, q0, lane);
+    wmma3<1, 4, false, SPLIT>(tt, Fs, LDD, 1, Kx, 1, LDD, D, p0, q0, lane);
     FRAG_LOOP(1, 4) dTs[FRAG_R(p0) * LDC + FRAG_C(q0)] += tt[mt][nt][i];
   }
   // this thread's elements of dq, dk and dg (the CH x D block tiling)
@@ -725,7 +759,7 @@ __global__ void __launch_bounds__(NT, 1) cbwd_local_grad_kernel(CbwdArgs a) {
   {  // dv = Diag(beta) X^T dU
     float acc[2][NTD][4];
     zero4(acc);
-    wmma3<2, NTD>(acc, Xs, 1, LDC, Bs, LDD, 1, CH, m0, n0, lane);
+    wmma3<2, NTD, false, SPLIT>(acc, Xs, 1, LDC, Bs, LDD, 1, CH, m0, n0, lane);
     FRAG_LOOP(2, NTD) {
       const int r = FRAG_R(m0);
       if (r < p.n) a.dv[(p.tok0 + (int64_t)r * a.H) * D + FRAG_C(n0)] = bs[r] * acc[mt][nt][i];
@@ -734,7 +768,7 @@ __global__ void __launch_bounds__(NT, 1) cbwd_local_grad_kernel(CbwdArgs a) {
   {  // dKG = Diag(beta) X^T dW; the dq, dk, dg terms of KG, QG and Kt
     float acc[2][NTD][4];
     zero4(acc);
-    wmma3<2, NTD>(acc, Xs, 1, LDC, Fs, LDD, 1, CH, m0, n0, lane);
+    wmma3<2, NTD, false, SPLIT>(acc, Xs, 1, LDC, Fs, LDD, 1, CH, m0, n0, lane);
     const float* dKt = a.w.dKt + cd;
     const float* dQG = a.w.dQG + cd;
 #pragma unroll
@@ -769,7 +803,7 @@ __global__ void __launch_bounds__(NT, 1) cbwd_local_grad_kernel(CbwdArgs a) {
   {  // M = X^T dT Diag(beta); the first dbeta term, colsum(X o dT)
     float m[1][4][4];
     zero4(m);
-    wmma3<1, 4>(m, Xs, 1, LDC, dTs, LDC, 1, CH, p0, q0, lane);
+    wmma3<1, 4, false, SPLIT>(m, Xs, 1, LDC, dTs, LDC, 1, CH, p0, q0, lane);
     FRAG_LOOP(1, 4) {
       const int c = FRAG_C(q0);
       Ms[FRAG_R(p0) * LDC + c] = m[mt][nt][i] * bs[c];
@@ -798,7 +832,7 @@ __global__ void __launch_bounds__(NT, 1) cbwd_local_grad_kernel(CbwdArgs a) {
   {  // dA = -strict(M X^T); the second dbeta term, rowsum(dA o A/beta); dAb = Diag(beta) dA
     float m[1][4][4];
     zero4(m);
-    wmma3<1, 4>(m, Ms, LDC, 1, Xs, 1, LDC, CH, p0, q0, lane);
+    wmma3<1, 4, false, SPLIT>(m, Ms, LDC, 1, Xs, 1, LDC, CH, p0, q0, lane);
 #pragma unroll
     for (int hi = 0; hi < 2; ++hi) {
       const int r = p0 + g + 8 * hi;
@@ -820,7 +854,7 @@ __global__ void __launch_bounds__(NT, 1) cbwd_local_grad_kernel(CbwdArgs a) {
   {  // R2 = e^{g - g_m} o (dP KN): dq, and R1 = e^{g - g_m} o (dAb KN): dk
     float acc[2][NTD][4];
     zero4(acc);
-    wmma3<2, NTD>(acc, dPs, LDC, 1, Bs, LDD, 1, CH, m0, n0, lane);
+    wmma3<2, NTD, false, SPLIT>(acc, dPs, LDC, 1, Bs, LDD, 1, CH, m0, n0, lane);
     FRAG_LOOP(2, NTD) {
       const int r = FRAG_R(m0), c = FRAG_C(n0);
       const float r2 = acc[mt][nt][i] * Gs[r * LDD + c];
@@ -829,7 +863,7 @@ __global__ void __launch_bounds__(NT, 1) cbwd_local_grad_kernel(CbwdArgs a) {
       dg[mt][nt][i] = fmaf(qv, r2, dg[mt][nt][i]);
     }
     zero4(acc);
-    wmma3<2, NTD>(acc, Abs, LDC, 1, Bs, LDD, 1, CH, m0, n0, lane);
+    wmma3<2, NTD, false, SPLIT>(acc, Abs, LDC, 1, Bs, LDD, 1, CH, m0, n0, lane);
     FRAG_LOOP(2, NTD) {
       const int r = FRAG_R(m0), c = FRAG_C(n0);
       const float r1 = acc[mt][nt][i] * Gs[r * LDD + c];
@@ -841,8 +875,8 @@ __global__ void __launch_bounds__(NT, 1) cbwd_local_grad_kernel(CbwdArgs a) {
   {  // R3 = e^{g_m - g} o (dAb^T Kx + dP^T Qx): dk
     float acc[2][NTD][4];
     zero4(acc);
-    wmma3<2, NTD>(acc, Abs, 1, LDC, Kx, LDD, 1, CH, m0, n0, lane);
-    wmma3<2, NTD>(acc, dPs, 1, LDC, Fs, LDD, 1, CH, m0, n0, lane);
+    wmma3<2, NTD, false, SPLIT>(acc, Abs, 1, LDC, Kx, LDD, 1, CH, m0, n0, lane);
+    wmma3<2, NTD, false, SPLIT>(acc, dPs, 1, LDC, Fs, LDD, 1, CH, m0, n0, lane);
     FRAG_LOOP(2, NTD) {
       const int r = FRAG_R(m0), c = FRAG_C(n0);
       const bool in = r < p.n;
@@ -990,21 +1024,23 @@ cudaError_t set_smem(K kernel, size_t bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
-template <int D>
+// SPLIT: the per-chunk kernels' products at fp32 accuracy (fp32 problems); bf16 problems take one
+// tf32 product there.  The chains always split: their error compounds from chunk to chunk.
+template <int D, bool SPLIT>
 cudaError_t launch_scan_bwd(const CbwdArgs& a, const Dims& d, cudaStream_t s) {
   cudaError_t e;
   const dim3 chunks((unsigned)a.nc, (unsigned)d.H, (unsigned)d.B);
   const dim3 cols((unsigned)(D / CW), (unsigned)d.H, (unsigned)d.B);
-  if ((e = set_smem(cbwd_prep_kernel<D>, prep_smem<D>())) != cudaSuccess) return e;
-  cbwd_prep_kernel<D><<<chunks, NT, prep_smem<D>(), s>>>(a);
+  if ((e = set_smem(cbwd_prep_kernel<D, SPLIT>, prep_smem<D>())) != cudaSuccess) return e;
+  cbwd_prep_kernel<D, SPLIT><<<chunks, NT, prep_smem<D>(), s>>>(a);
   if ((e = set_smem(cbwd_chain_kernel<D, false>, chain_smem<D, false>())) != cudaSuccess) return e;
   cbwd_chain_kernel<D, false><<<cols, NT, chain_smem<D, false>(), s>>>(a);
   if ((e = set_smem(cbwd_chain_kernel<D, true>, chain_smem<D, true>())) != cudaSuccess) return e;
   cbwd_chain_kernel<D, true><<<cols, NT, chain_smem<D, true>(), s>>>(a);
-  if ((e = set_smem(cbwd_state_grad_kernel<D>, state_grad_smem<D>())) != cudaSuccess) return e;
-  cbwd_state_grad_kernel<D><<<chunks, NT, state_grad_smem<D>(), s>>>(a);
-  if ((e = set_smem(cbwd_local_grad_kernel<D>, local_grad_smem<D>())) != cudaSuccess) return e;
-  cbwd_local_grad_kernel<D><<<chunks, NT, local_grad_smem<D>(), s>>>(a);
+  if ((e = set_smem(cbwd_state_grad_kernel<D, SPLIT>, state_grad_smem<D>())) != cudaSuccess) return e;
+  cbwd_state_grad_kernel<D, SPLIT><<<chunks, NT, state_grad_smem<D>(), s>>>(a);
+  if ((e = set_smem(cbwd_local_grad_kernel<D, SPLIT>, local_grad_smem<D>())) != cudaSuccess) return e;
+  cbwd_local_grad_kernel<D, SPLIT><<<chunks, NT, local_grad_smem<D>(), s>>>(a);
   return cudaGetLastError();
 }
 
@@ -1053,7 +1089,8 @@ cudaError_t launch_bwd(const Dims& d, kda_dtype dt, const void* q, const void* k
   a.w = carve(l, base + 6 * l.act32 + l.dbeta);
   a.N = d.N; a.H = d.H; a.nc = l.nc; a.bf16 = dt == KDA_DT_BF16;
   a.status = static_cast<uint32_t*>(ws);
-  e = d.dk == 128 ? launch_scan_bwd<128>(a, d, s) : launch_scan_bwd<64>(a, d, s);
+  if (a.bf16) e = d.dk == 128 ? launch_scan_bwd<128, false>(a, d, s) : launch_scan_bwd<64, false>(a, d, s);
+  else e = d.dk == 128 ? launch_scan_bwd<128, true>(a, d, s) : launch_scan_bwd<64, true>(a, d, s);
   if (e != cudaSuccess) return e;
   const int64_t nb = (int64_t)d.B * d.N * d.H;
   if (dt == KDA_DT_BF16)
