@@ -18,7 +18,7 @@ Two independent formulations live here, both in fp64:
   page (explicit (I - beta k k^T) Diag(alpha) products), used only to
   cross-check the recurrence on small inputs.
 
-Readings of points the pages leave open (each also listed in the design doc):
+Readings of points the pages leave open (the kernels implement the same readings):
   * read-out o_t = S_t^T q_t, no scale on q;
   * kernels: causal 4 taps over text, 3x3x3 over the visual grid, applied as a
     cross-correlation (tap j of the text kernel multiplies x[t-(K-1)+j]);
