@@ -1,0 +1,109 @@
+"""The decomposition the backward kernels use, checked against the oracle's token adjoint (CPU only).
+
+The kernels split the chunked backward into a per-chunk pass (factors about g_m, A, P, the inverse,
+W = T KG, U~ = T V, Z = P^T dO, Y = QG^T dO), a forward pass over chunks storing every entry state
+and U, a reverse pass storing every exit gradient (dU = Z + Kt dS, dS <- e^{gl} dS - W^T dU + Y),
+and two per-chunk gradient passes (the contractions with S and dS; then dT, the inverse's adjoint,
+the decay-weighted products for dq and dk, d log alpha as a reverse running sum within the chunk).
+Written here in numpy in exactly that arrangement, with zero-padded ragged last chunks, it must
+reproduce oracle.scan_bwd to rounding.
+"""
+import numpy as np
+import pytest
+
+import oracle
+
+
+def _chunk_prep(q, k, v, la, beta, dO, C, plant=False):
+    G = np.cumsum(la, 0)
+    gm, gl = G[C // 2 - 1], G[-1]
+    Kx, KN, Qx = k * np.exp(G - gm), k * np.exp(gm - G), q * np.exp(G - gm)
+    Ab = np.tril(Kx @ KN.T, -1)
+    P = np.tril(Qx @ KN.T)
+    X = np.linalg.inv(np.eye(C) + beta[:, None] * Ab)
+    T = X * beta[None, :]
+    W = (T @ Kx) * np.exp(gm)[None, :]
+    Y = (Qx * np.exp(gm)).T @ dO
+    if plant:   # a plausible slip: folding -W^T Z into Y although the reverse pass subtracts W^T dU, Z included
+        Y = Y - W.T @ (P.T @ dO)
+    return dict(W=W, Ut=T @ v, Kt=KN * np.exp(gl - gm)[None, :], Z=P.T @ dO, Y=Y, X=X, Ab=Ab, egl=np.exp(gl))
+
+
+def _decomposed_bwd(q, k, v, la, beta, dO, S0, dSN, C, plant=False):
+    N, D = q.shape
+    pad = lambda a, s: np.concatenate([a[s], np.zeros((C - len(a[s]),) + a.shape[1:])])   # noqa: E731
+    chunks = [[pad(a, slice(s, s + C)) for a in (q, k, v, la, beta, dO)] for s in range(0, N, C)]
+    pre = [_chunk_prep(*c, C, plant) for c in chunks]
+    S, U = [S0], []
+    for p in pre:                                   # forward pass over chunks
+        U.append(p["Ut"] - p["W"] @ S[-1])
+        S.append(p["egl"][:, None] * S[-1] + p["Kt"].T @ U[-1])
+    dS, dSx, dU = dSN, [None] * len(pre), [None] * len(pre)
+    for i in range(len(pre) - 1, -1, -1):           # reverse pass
+        p = pre[i]
+        dSx[i] = dS
+        dU[i] = p["Z"] + p["Kt"] @ dS
+        dS = p["egl"][:, None] * dS - p["W"].T @ dU[i] + p["Y"]
+    out = {n: [] for n in ("dq", "dk", "dv", "dla", "dbeta")}
+    for i, (qc, kc, vc, lac, bc, dOc) in enumerate(chunks):
+        p = pre[i]
+        # contractions with the chunk's entry state and exit gradient
+        dQG, dW, dKt = dOc @ S[i].T, -dU[i] @ S[i].T, U[i] @ dSx[i].T
+        dP, dUV = np.tril(dOc @ U[i].T), dU[i] @ vc.T
+        last = (dSx[i] * S[i]).sum(1) * p["egl"]
+        # chunk-local part
+        G = np.cumsum(lac, 0)
+        gm, gl = G[C // 2 - 1], G[-1]
+        E = np.exp(G - gm)
+        Kx, KN, Qx = kc * E, kc / E, qc * E
+        dWs = dW * np.exp(gm)[None, :]
+        dT = dWs @ Kx.T + dUV
+        dv = bc[:, None] * (p["X"].T @ dU[i])
+        a = bc[:, None] * (p["X"].T @ dWs)
+        e2 = np.exp(gl - gm)[None, :] / E
+        dk = E * a + dKt * e2
+        dq = dQG * np.exp(gm)[None, :] * E
+        dg = kc * E * a - kc * e2 * dKt + qc * np.exp(gm)[None, :] * E * dQG
+        colk = (dKt * kc * e2).sum(0)
+        dA = -np.tril((p["X"].T @ (dT * bc[None, :])) @ p["X"].T, -1)
+        dbeta = (p["X"] * dT).sum(0) + (dA * p["Ab"]).sum(1)
+        dAb = dA * bc[:, None]
+        R2, R1 = E * (dP @ KN), E * (dAb @ KN)
+        R3 = (dAb.T @ Kx + dP.T @ Qx) / E
+        dq, dk = dq + R2, dk + R1 + R3
+        dg = dg + qc * R2 + kc * (R1 - R3)
+        dg[-1] += colk + last
+        dla = np.cumsum(dg[::-1], 0)[::-1]
+        n = min(C, N - i * C)
+        for name, val in (("dq", dq), ("dk", dk), ("dv", dv), ("dla", dla), ("dbeta", dbeta)):
+            out[name].append(val[:n])
+    res = {name: np.concatenate(val) for name, val in out.items()}
+    res["dS0"] = dS
+    return res
+
+
+@pytest.mark.parametrize("N, C", [(37, 16), (64, 16), (16, 16), (5, 16), (70, 32)])
+def test_decomposition_matches_the_token_adjoint(N, C):
+    rng = np.random.default_rng(N + C)
+    D = 6
+    q, k, v = (rng.standard_normal((N, D)) for _ in range(3))
+    la = -np.abs(rng.standard_normal((N, D))) * 0.3
+    beta = 1 / (1 + np.exp(-rng.standard_normal(N)))
+    dO, S0, dSN = rng.standard_normal((N, D)), rng.standard_normal((D, D)), rng.standard_normal((D, D))
+    ref = oracle.scan_bwd(q[None], k[None], v[None], la[None], beta[None], dO[None], S0[None], dSN[None])
+    got = _decomposed_bwd(q, k, v, la, beta, dO, S0, dSN, C)
+    for name in ("dq", "dk", "dv", "dla", "dbeta", "dS0"):
+        r = ref[name][0]
+        assert np.abs(got[name] - r).max() <= 1e-10 * max(1.0, np.abs(r).max()), name
+
+
+def test_a_double_counted_chain_term_is_caught():
+    rng = np.random.default_rng(3)
+    N, D, C = 40, 6, 16
+    q, k, v = (rng.standard_normal((N, D)) for _ in range(3))
+    la = -np.abs(rng.standard_normal((N, D))) * 0.3
+    beta = 1 / (1 + np.exp(-rng.standard_normal(N)))
+    dO, S0, dSN = rng.standard_normal((N, D)), rng.standard_normal((D, D)), rng.standard_normal((D, D))
+    ref = oracle.scan_bwd(q[None], k[None], v[None], la[None], beta[None], dO[None], S0[None], dSN[None])
+    got = _decomposed_bwd(q, k, v, la, beta, dO, S0, dSN, C, plant=True)
+    assert np.abs(got["dS0"] - ref["dS0"][0]).max() > 1e-3
