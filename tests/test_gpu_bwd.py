@@ -137,3 +137,9 @@ def test_bwd_strong_decay_within_and_beyond_the_range(kda):
     la[0, 3:31, 1, 5] = -2.5
     dO = np.random.default_rng(7).standard_normal((B, N, H, d))
     run_bwd(kda, w, dict(inp, log_alpha=la.reshape(inp["log_alpha"].shape)), dO, status=kda.KDA_ERR_RANGE)
+
+
+def test_bwd_bf16_d64(kda):
+    """bf16 with d = 64 (the per-chunk kernels' single-product mode at D = 64), 13 text tokens + 3 x 5 x 7."""
+    w = kda_synth.Workload("bwd_bf16_d64", 1, 2, 64, 13, (3, 5, 7), "bf16", 0.1)
+    _case(kda, w, 38)
