@@ -5,17 +5,21 @@
 //   S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T,   o_t = S_t^T q_t.
 //
 // The sequence is cut into blocks of 128 tokens, each made of two 64-token
-// sub-chunks.  For a sub-chunk with g_r = sum_{i<=r} log alpha_i (per key
-// channel, from the sub-chunk start), a reference g_m = g_31 (mid point) keeps
-// every exponential factor within e^{+-9} so fp16 operands cannot overflow:
-//   KG = K e^{g-g_m},  QG = Q e^{g-g_m},  KN = K e^{g_m-g}
-//   A  = strict_lower(Diag(beta) KG KN^T),  P = lower(QG KN^T)
-//   T  = (I + A)^{-1} Diag(beta),  W' = T KG,  U~ = T V
-//   K~ = KN e^{g_l-g_m}  (g_l = last g),   Gamma = e^{g_l}
-//   M_s = Diag(Gamma) - (K~^T W') Diag(e^{g_m}),   B_s = K~^T U~
-//   Q^_s = (QG - P W') Diag(e^{g_m}),   O'_s = P U~
+// sub-chunks.  Within a sub-chunk, with g_r = sum_{i<=r} log alpha_i (per key
+// channel, from the sub-chunk start) and g_l its last value, every factor is a
+// product of gates alpha <= 1, so no fp16 operand can overflow, whatever the gates:
+//   KG = K e^{g},  QG = Q e^{g},  K~ = K e^{g_l - g},  Gamma = e^{g_l}
+//   A  = strict_lower(Diag(beta) [K K^T . e^{g_r - g_i}]),  P = lower([Q K^T . e^{g_r - g_i}])
+//   T  = (I + A)^{-1} Diag(beta),  W = T KG,  U~ = T V
+//   M_s = Diag(Gamma) - K~^T W,   B_s = K~^T U~,   Q^_s = QG - P W,   O'_s = P U~
 // so that, entering with state S, the sub-chunk gives O = Q^_s S + O'_s and
-// leaves S <- M_s S + B_s.  Two sub-chunks compose into one 128-token block:
+// leaves S <- M_s S + B_s.  The pairwise decays e^{g_r - g_i} of A and P are
+// factored at a split point between i and r: a pair (r, i) belongs to the level l
+// of the highest bit in which r and i differ, and with s the first token of r's
+// half at that level, e^{g_r - g_i} = (prod_{u=s..r} alpha_u)(prod_{u=i+1..s-1} alpha_u).
+// Levels 5, 4 and 3 (pairs in different 8-token octets) are three tensor-core
+// products; pairs inside an octet are running products on the CUDA cores.
+// Two sub-chunks compose into one 128-token block:
 //   M = M_2 M_1,  B = M_2 B_1 + B_2,  R = [Q^_1 ; Q^_2 M_1],  O'' = [O'_1 ; Q^_2 B_1 + O'_2]
 // and the block maps S to O = R S + O'' and S <- M S + B.
 //
@@ -44,7 +48,6 @@ using namespace tc;
 constexpr int BLK = 128;          // tokens per block (one serial step)
 constexpr int SUB = 64;           // tokens per sub-chunk
 constexpr int D = 128;            // d_k = d_v
-constexpr float kRange = 9.f;     // max |g - g_m| allowed for the fp16 factors
 
 // Record per (batch item, head, block), all fp16:
 //   M   K-major operand image: 2 panels [128 rows][64 cols]            32 KB
@@ -60,12 +63,6 @@ constexpr size_t kBlockBytes = 131072;
 template <typename T> constexpr bool kIsHalf = false;
 template <> constexpr bool kIsHalf<__half> = true;
 
-__device__ __forceinline__ float2 ld_act2(const uint8_t* p, __half*) {
-  return __half22float2(*reinterpret_cast<const __half2*>(p));
-}
-__device__ __forceinline__ float2 ld_act2(const uint8_t* p, __nv_bfloat16*) {
-  return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
-}
 __device__ __forceinline__ void st_h2(uint8_t* p, float a, float b) {
   *reinterpret_cast<__half2*>(p) = __floats2half2_rn(a, b);
 }
@@ -110,19 +107,20 @@ __device__ __forceinline__ uint32_t tmem_at(uint32_t base, int lane0, int col) {
   return base + ((uint32_t)lane0 << 16) + (uint32_t)col;
 }
 
-// Waits for a TMA load counted on `bar`; on timeout records the status.  Returns false on timeout.
-__device__ __forceinline__ bool wait_tma(uint64_t* bar, uint32_t& phase, uint32_t* status, bool alive) {
+// Waits (at most tmo ns) for a TMA load counted on `bar`; on timeout records the status.
+// Returns false on timeout.
+__device__ __forceinline__ bool wait_tma(uint64_t* bar, uint32_t& phase, uint32_t* status, bool alive, uint64_t tmo) {
   if (!alive) return false;
-  const bool ok = mbar_wait(bar, phase);
+  const bool ok = mbar_wait(bar, phase, tmo);
   if (ok) phase ^= 1u;
   else set_status(status, KDA_ERR_TIMEOUT);
   return ok;
 }
 
-// Waits on the MMA barrier; on timeout records the status.  Returns false on timeout.
-__device__ __forceinline__ bool wait_mma(uint64_t* bar, uint32_t& phase, uint32_t* status, bool alive) {
+// Waits (at most tmo ns) on the MMA barrier; on timeout records the status.  Returns false on timeout.
+__device__ __forceinline__ bool wait_mma(uint64_t* bar, uint32_t& phase, uint32_t* status, bool alive, uint64_t tmo) {
   if (!alive) return false;   // nothing was issued
-  const bool ok = mbar_wait(bar, phase);
+  const bool ok = mbar_wait(bar, phase, tmo);
   phase ^= 1u;
   if (!ok) set_status(status, KDA_ERR_TIMEOUT);
   return ok;
@@ -132,28 +130,35 @@ __device__ __forceinline__ bool wait_mma(uint64_t* bar, uint32_t& phase, uint32_
 // kda_tc_prep
 // ---------------------------------------------------------------------------
 // shared memory map (bytes from a 1024-aligned base)
-constexpr uint32_t OFF_KQ = 0;          // [128 rows][128] fp16: rows 0-63 KG (later W'), 64-127 QG; later M_2
-constexpr uint32_t OFF_KN = 32768;      // [64][128] fp16: KN, then K~
+constexpr uint32_t OFF_KQ = 0;          // [128 rows][128] fp16: rows 0-63 K -> K Gamma (later W), 64-127 Q -> Q Gamma; later M_2
+constexpr uint32_t OFF_KN = 32768;      // [64][128] fp16: K~; staging of O'_1 and O''_2
 constexpr uint32_t OFF_VV = 49152;      // [64][128] fp16: V, then U~, then Q^_2
-constexpr uint32_t OFF_TT = 65536;      // [64][64] fp16: T
+constexpr uint32_t OFF_TT = 65536;      // [64][64] fp16: T   (TT and PP together: staging of R_1 and R_2)
 constexpr uint32_t OFF_PP = 73728;      // [64][64] fp16: P
 constexpr uint32_t OFF_M1 = 81920;      // [128][128] fp16: M_1 (MN-major operand image)
 constexpr uint32_t OFF_B1 = 114688;     // [128][128] fp16: B_1 (MN-major operand image)
-constexpr uint32_t OFF_AS = 147456;     // fp32 [64][LDA]: A (strictly lower, beta applied)
-constexpr uint32_t OFF_XS = 164864;     // fp32 [64][LDXS]: (I + A)^{-1}
-constexpr uint32_t OFF_YS = 182272;     // fp32 [32][36]: merge scratch / quarter totals
-constexpr uint32_t OFF_MISC = 186880;   // beta[64], egm, egl, ekt, gm, tot [128 each], barriers, tmem slot, flag
-constexpr uint32_t OFF_LA = 191232;     // fp32 [64 tokens][128]: log alpha of a sub-chunk (TMA), then x = g - g_m
-constexpr uint32_t PREP_SMEM = OFF_LA + 32768 + 1024;   // + alignment slack
+// 72 KB used three ways in turn: the log alpha of a sub-chunk (TMA target, [64 tokens][128] fp32), the
+// operand tiles of the three tensor-core Gram levels, and A, X, Y of the blocked inverse
+constexpr uint32_t OFF_G = 147456;
+constexpr uint32_t G_ROW = 0;           // level tiles, rows: [64][128] fp16 per level (5, 4, 3), 16 KB apart
+constexpr uint32_t G_COL = 49152;       // level tiles, columns: [32][128] fp16 per level, 8 KB apart
+constexpr uint32_t G_AS = 0;            // fp32 [64][LDA]: A (strictly lower, beta applied)
+constexpr uint32_t G_XS = 17408;        // fp32 [64][LDXS]: (I + A)^{-1}
+constexpr uint32_t G_YS = 34816;        // fp32 [32][36]: merge scratch
+constexpr uint32_t OFF_MISC = OFF_G + 73728;   // beta[64], Gamma_l[128], octet totals [8][128], octet Gram [8][64], barriers
+constexpr uint32_t PREP_SMEM = OFF_MISC + 8192 + 1024;   // + alignment slack
 
 constexpr int LDA = 68;    // row stride of A: rows 16-byte aligned (4-wide stores and loads)
 constexpr int LDXS = 68;   // row stride of X: rows 16-byte aligned for 4-wide loads
-static_assert(OFF_XS >= OFF_AS + 64 * LDA * 4 && OFF_YS >= OFF_XS + 64 * LDXS * 4, "prep shared-memory map");
-static_assert(OFF_LA % 128 == 0 && OFF_LA >= OFF_MISC + 4096, "prep shared-memory map");
+static_assert(G_XS >= G_AS + 64 * LDA * 4 && G_YS >= G_XS + 64 * LDXS * 4 && G_YS + 32 * 36 * 4 <= 73728,
+              "prep shared-memory map");
+static_assert(G_COL >= G_ROW + 3 * 16384 && G_COL + 3 * 8192 <= 73728, "prep shared-memory map");
+static_assert(PREP_SMEM <= 232448, "prep shared memory above the per-block limit");
 constexpr int LDY = 36;    // row stride of the merge scratch
 
 // TMEM columns
-constexpr int C_AP = 0, C_W = 64, C_U = 192;
+constexpr int C_G = 0;                   // the three Gram levels, 32 columns each (M = 64 layout)
+constexpr int C_W = 64, C_U = 192;
 constexpr int C_MK = 0, C_BK = 128, C_PW = 256, C_PU = 384;
 
 // TMA descriptors of the [B][N][H][128] inputs, box [1][64 tokens][1][64 or 128 channels]
@@ -168,6 +173,8 @@ struct PrepArgs {
   uint8_t* ws;            // block records
   int64_t N; int H; int BH; int n_blocks; int n_units;
   uint32_t* status;
+  uint64_t wait_ns;       // limit of every device wait
+  int fault;              // self-test: 1 = the first CTA never issues its first k/q/v load
 };
 
 // One 16x8 tile of C = A B with fp32 operands in shared memory (A row-major with
@@ -329,6 +336,53 @@ __device__ __forceinline__ void inverse_merge64(const float* As, const float* Xs
   }
 }
 
+// 4 consecutive activations (8 bytes, fp16 or bf16) -> fp32, and 4 fp32 -> fp16 (8 bytes)
+__device__ __forceinline__ void ld_act4(const uint8_t* p, float* v, __half*) {
+  const uint2 u = *reinterpret_cast<const uint2*>(p);
+  const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&u.x));
+  const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&u.y));
+  v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
+}
+__device__ __forceinline__ void ld_act4(const uint8_t* p, float* v, __nv_bfloat16*) {
+  const uint2 u = *reinterpret_cast<const uint2*>(p);
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+  v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
+}
+__device__ __forceinline__ void st_h4(uint8_t* p, float a, float b, float c, float d) {
+  *reinterpret_cast<uint2*>(p) = make_uint2(pack_h2(a, b), pack_h2(c, d));
+}
+
+// Position of token t (0..63) among the 32 tokens of its role at Gram level l: the
+// tokens whose bit l is set (rows) or clear (columns), in increasing order.
+__device__ __forceinline__ int level_pos(int t, int l) { return ((t >> (l + 1)) << l) | (t & ((1 << l) - 1)); }
+
+// v[0..N-1] summed over the 32 lanes of a warp, scattered: lane L ends with the
+// totals of v[2L] and v[2L + 1] (for N = 64) in v[0] and v[1].  Each round keeps the
+// half of the vector that the lane's bit S selects and adds the partner's copy of it.
+template <int S, int N>
+__device__ __forceinline__ void reduce_scatter_round(float (&v)[64], int lane) {
+  const bool up = (lane & S) != 0;
+#pragma unroll
+  for (int x = 0; x < N / 2; ++x) {
+    const float lo = v[x], hi = v[x + N / 2];
+    const float keep = up ? hi : lo, send = up ? lo : hi;
+    v[x] = keep + __shfl_xor_sync(0xffffffffu, send, S);
+  }
+}
+__device__ __forceinline__ void warp_reduce_scatter64(float (&v)[64], int lane) {
+  reduce_scatter_round<16, 64>(v, lane);
+  reduce_scatter_round<8, 32>(v, lane);
+  reduce_scatter_round<4, 16>(v, lane);
+  reduce_scatter_round<2, 8>(v, lane);
+  reduce_scatter_round<1, 4>(v, lane);
+}
+
+// Index of a pair (r, i) of one octet in the octet Gram: A pairs i < r at r(r-1)/2 + i
+// (28 of them), P pairs i <= r at 28 + r(r+1)/2 + i (36).
+__host__ __device__ constexpr int oct_a(int r, int i) { return r * (r - 1) / 2 + i; }
+__host__ __device__ constexpr int oct_p(int r, int i) { return 28 + r * (r + 1) / 2 + i; }
+
 template <typename TIn>
 __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_constant__ PrepMaps mp) {
   extern __shared__ uint8_t dyn[];
@@ -340,21 +394,19 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
   uint8_t* PP = sm + OFF_PP;
   uint8_t* M1 = sm + OFF_M1;
   uint8_t* B1 = sm + OFF_B1;
-  float* As = reinterpret_cast<float*>(sm + OFF_AS);
-  float* Xs = reinterpret_cast<float*>(sm + OFF_XS);
-  float* Ys = reinterpret_cast<float*>(sm + OFF_YS);
-  float* beta_s = reinterpret_cast<float*>(sm + OFF_MISC);     // 64
-  float* egm = beta_s + 64;                                     // 128: e^{g_m}
-  float* egl = egm + 128;                                       // 128: e^{g_l}
-  float* ekt = egl + 128;                                       // 128: e^{g_l - g_m}
-  float* gm_s = ekt + 128;                                      // 128
-  float* tot_s = gm_s + 128;                                    // 128
-  uint64_t* bar = reinterpret_cast<uint64_t*>(tot_s + 128);    // [0] MMA, [1] k/q/v tiles, [2] log alpha
+  uint8_t* G = sm + OFF_G;
+  const float* LA = reinterpret_cast<const float*>(G);      // log alpha of the sub-chunk (TMA)
+  float* As = reinterpret_cast<float*>(G + G_AS);
+  float* Xs = reinterpret_cast<float*>(G + G_XS);
+  float* Ys = reinterpret_cast<float*>(G + G_YS);
+  float* beta_s = reinterpret_cast<float*>(sm + OFF_MISC);  // 64
+  float* egl = beta_s + 64;                                 // 128: Gamma_l = e^{g_l}
+  float* tot = egl + 128;                                   // [8 octets][128]: decay over each octet
+  float* gscr = tot + 8 * 128;                              // [8 octets][64]: Gram pairs inside each octet
+  uint64_t* bar = reinterpret_cast<uint64_t*>(gscr + 8 * 64);   // [0] MMA, [1] k/q/v tiles, [2] log alpha
   uint64_t* kqv_bar = bar + 1;
   uint64_t* la_bar = bar + 2;
-  float* LAx = reinterpret_cast<float*>(sm + OFF_LA);   // log alpha, turned in place into x = g - g_m
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 4);
-  int* range_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int sub = warp & 3, chalf = warp >> 2;
@@ -366,7 +418,6 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
     mbar_init(kqv_bar, 1);
     mbar_init(la_bar, 1);
     fence_mbar_init();
-    *range_flag = 0;
   }
   fence_before_sync();
   __syncthreads();
@@ -405,73 +456,31 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
     }
   };
   bool kqv_early = false;   // thread 0: the next sub-chunk's tiles are already on their way
-  auto issue_la = [&](int u, int s_) {   // log alpha of sub-chunk s_ of unit u -> LAs (thread 0)
+  auto issue_la = [&](int u, int s_) {   // log alpha of sub-chunk s_ of unit u -> G (thread 0)
     const int blk_ = u / a.BH, bh_ = u - blk_ * a.BH;
     const int b_ = bh_ / a.H, h_ = bh_ - b_ * a.H;
     mbar_arrive_expect_tx(la_bar, 32768);
-    tma_load_4d(sm + OFF_LA, &mp.la, 0, h_, blk_ * BLK + s_ * SUB, b_, la_bar);
+    tma_load_4d(G, &mp.la, 0, h_, blk_ * BLK + s_ * SUB, b_, la_bar);
   };
   if (tid == 0 && (int)blockIdx.x < a.n_units) {
     issue_la(blockIdx.x, 0);
     la_inflight = true;
   }
-  // Decay exponents of a sub-chunk, in place in LAx (zero log alpha past the sequence end).
-  // Thread: channels 2 dp, 2 dp + 1 and tokens 16 dq .. 16 dq + 15.  Part 1 forms the running
-  // sums within the thread's 16 tokens and publishes their totals; part 2 (after a barrier)
-  // turns them into x = g - g_m, g_m = g_31, and records g_m and the decay over tokens 32..63.
-  const int dp = (tid & 31) + 32 * ((tid >> 5) & 1), dq = tid >> 6, dc = 2 * dp;
-  float2* qtot = reinterpret_cast<float2*>(Ys);   // [4][64] quarter totals
-  auto decay_part1 = [&](bool ok) -> bool {
-    ok = wait_tma(la_bar, la_phase, a.status, ok);
-    if (tid == 0) la_inflight = !ok && la_inflight;
-    if (!ok) return false;
-    float2 gl[16];
-#pragma unroll
-    for (int t = 0; t < 16; ++t) gl[t] = *reinterpret_cast<const float2*>(LAx + (16 * dq + t) * D + dc);
-#pragma unroll
-    for (int t = 1; t < 16; ++t) { gl[t].x += gl[t - 1].x; gl[t].y += gl[t - 1].y; }
-#pragma unroll
-    for (int t = 0; t < 16; ++t) *reinterpret_cast<float2*>(LAx + (16 * dq + t) * D + dc) = gl[t];
-    qtot[dq * 64 + dp] = gl[15];
-    return true;
-  };
-  auto decay_part2 = [&]() {
-    float2 pre = make_float2(0.f, 0.f), gmv = make_float2(0.f, 0.f), tot = make_float2(0.f, 0.f);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float2 v = qtot[j * 64 + dp];
-      if (j < dq) { pre.x += v.x; pre.y += v.y; }
-      if (j < 2) { gmv.x += v.x; gmv.y += v.y; } else { tot.x += v.x; tot.y += v.y; }
-    }
-    if (dq == 0) {
-      gm_s[dc] = gmv.x; gm_s[dc + 1] = gmv.y;       // g_m: decay through token 31
-      tot_s[dc] = tot.x; tot_s[dc + 1] = tot.y;     // decay over tokens 32..63
-    }
-    float2 x0 = make_float2(0.f, 0.f);
-#pragma unroll
-    for (int t = 0; t < 16; ++t) {
-      float2* p = reinterpret_cast<float2*>(LAx + (16 * dq + t) * D + dc);
-      const float2 g = *p;
-      const float2 x = make_float2(pre.x + g.x - gmv.x, pre.y + g.y - gmv.y);
-      if (t == 0) x0 = x;
-      *p = x;
-    }
-    // x is largest at token 0 and smallest (-tot) at token 63
-    if (dq == 0 && (x0.x > kRange || x0.y > kRange)) *range_flag = 1;
-    if (dq == 3 && (-tot.x > kRange || -tot.y > kRange)) *range_flag = 1;
-  };
-  bool x_ready = false;   // the current sub-chunk's exponents were formed during the previous one
 
   // operand descriptors of the fixed tiles (stepped along K by kstep / mstep)
   const uint64_t dKQk = kdesc0(smem_u32(KQ)), dKQm = mdesc0(smem_u32(KQ), 16384);
-  const uint64_t dKNk = kdesc0(smem_u32(KN)), dKNm = mdesc0(smem_u32(KN), 8192);
+  const uint64_t dKNm = mdesc0(smem_u32(KN), 8192);
   const uint64_t dVVk = kdesc0(smem_u32(VV)), dVVm = mdesc0(smem_u32(VV), 8192);
   const uint64_t dTTk = kdesc0(smem_u32(TT)), dPPk = kdesc0(smem_u32(PP));
   const uint64_t dM1m = mdesc0(smem_u32(M1), 16384), dB1m = mdesc0(smem_u32(B1), 16384);
-  const uint32_t id_ap = idesc_f16(128, 64, false, false);
+  const uint64_t dGrow = kdesc0(smem_u32(G + G_ROW)), dGcol = kdesc0(smem_u32(G + G_COL));
+  const uint32_t id_gram = idesc_f16(64, 32, false, false);
   const uint32_t id_64x128_kmn = idesc_f16(64, 128, false, true);
   const uint32_t id_128x128_mnmn = idesc_f16(128, 128, true, true);
   const uint32_t id_128x128_kmn = idesc_f16(128, 128, false, true);
+
+  // front-pass role of this thread: octet fo (tokens 8 fo .. 8 fo + 7), channels 4 lane .. 4 lane + 3
+  const int fo = warp, fpnl = lane >> 4, fpc = (4 * lane) & 63;
 
   for (int unit = blockIdx.x; unit < a.n_units && alive; unit += gridDim.x) {
     const int blk = unit / a.BH, bh = unit - blk * a.BH;
@@ -484,14 +493,15 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
 
     for (int s = 0; s < 2; ++s) {
       const int64_t t0 = (int64_t)blk * BLK + s * SUB;
-      const int nv = (int)max((int64_t)0, min((int64_t)SUB, a.N - t0));
       // ---------------- inputs ----------------
       // k -> KQ rows 0-63, q -> KQ rows 64-127, v -> VV: 128-byte-swizzled operand panels
-      // written by TMA; rows past the sequence end read as zero
+      // written by TMA; rows past the sequence end read as zero (log alpha too: alpha = 1)
       if (tid == 0 && alive) {
-        if (!kqv_early) issue_kqv(b, h, (int)t0);   // else issued while the previous unit finished
+        // self-test of the bounded waits: a load that is never issued, so the wait below gives up
+        const bool skip = a.fault == 1 && blockIdx.x == 0 && unit == 0 && s == 0;
+        if (!kqv_early && !skip) issue_kqv(b, h, (int)t0);   // else issued while the previous unit finished
         kqv_early = false;
-        kqv_inflight = true;
+        kqv_inflight = !skip;
       }
       if (tid == 128 && alive) {
         // the next sub-chunk's tiles and log alpha into L2 meanwhile
@@ -512,96 +522,209 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
         int nb_, nh_, nt0_;
         beta_next = next_sub(unit, s, nb_, nh_, nt0_) ? load_beta(nb_, nh_, nt0_ + tid) : 0.f;
       }
-      bool ok_in = alive;
-      if (!x_ready) {
-        // first sub-chunk of this CTA: its decay exponents are formed here (later ones are
-        // formed while the previous sub-chunk waits for its products)
-        ok_in = decay_part1(ok_in);
-        fence_before_sync();
-        __syncthreads();
-        decay_part2();
-      }
-      x_ready = false;
-      ok_in = wait_tma(kqv_bar, kqv_phase, a.status, ok_in);
-      alive = __syncthreads_and(ok_in);
-      if (tid == 0) kqv_inflight = false;
       {
-        // thread: channels 2cp, 2cp+1 and tokens 16*qt .. 16*qt+15; X holds x = g - g_m
-        const int cp = (tid & 31) + 32 * ((tid >> 5) & 1);
-        const int qt = tid >> 6;
-        const int c = 2 * cp;
-        const int pnl = c >> 6, cc = c & 63;
-        uint8_t* kq = KQ + pnl * 16384;
-        uint8_t* kn = KN + pnl * 8192;
-        uint8_t* vv = VV + pnl * 8192;
+        const bool ok_la = wait_tma(la_bar, la_phase, a.status, alive, a.wait_ns);
+        const bool ok_kqv = wait_tma(kqv_bar, kqv_phase, a.status, ok_la, a.wait_ns);
+        if (tid == 0) {
+          if (ok_la) la_inflight = false;
+          if (ok_kqv) kqv_inflight = false;
+        }
+        alive = __syncthreads_and(ok_kqv);
+      }
+      // ---------------- front pass ----------------
+      // Every factor is a product of gates alpha = e^{log alpha} <= 1, so none can overflow:
+      //   Gamma_t = prod_{u<=t} alpha_u,  e^{g_l - g_t} = prod_{u>t} alpha_u,
+      // and the Gram levels' factors, prefix products from a split point (rows) and suffix
+      // products up to it (columns).  Thread: octet fo, four channels; within the octet the
+      // prefix (pre) and suffix (suf) products are its own, across octets it uses the octet totals.
+      float al[8][4], kx[8][4], qx[8][4];
 #pragma unroll
-        for (int t = 0; t < 16; ++t) {
-          const int tok = 16 * qt + t;
-          const uint32_t off = swz_off(tok, cc), offq = swz_off(64 + tok, cc);
-          const float2 kv = ld_act2(kq + off, (TIn*)nullptr);
-          const float2 qv = ld_act2(kq + offq, (TIn*)nullptr);
-          const float2 x = *reinterpret_cast<const float2*>(LAx + tok * D + c);
-          const float ep0 = __expf(x.x), ep1 = __expf(x.y), en0 = __expf(-x.x), en1 = __expf(-x.y);
-          st_h2(kq + off, kv.x * ep0, kv.y * ep1);
-          st_h2(kq + offq, qv.x * ep0, qv.y * ep1);
-          st_h2(kn + off, kv.x * en0, kv.y * en1);
-          if constexpr (!kIsHalf<TIn>) {
-            const float2 vv2 = ld_act2(vv + off, (TIn*)nullptr);
-            st_h2(vv + off, vv2.x, vv2.y);
+      for (int j = 0; j < 8; ++j) {
+        const int tok = 8 * fo + j;
+        const float4 x = *reinterpret_cast<const float4*>(LA + tok * D + 4 * lane);
+        al[j][0] = __expf(x.x); al[j][1] = __expf(x.y); al[j][2] = __expf(x.z); al[j][3] = __expf(x.w);
+        ld_act4(KQ + fpnl * 16384 + swz_off(tok, fpc), kx[j], (TIn*)nullptr);
+        ld_act4(KQ + fpnl * 16384 + swz_off(64 + tok, fpc), qx[j], (TIn*)nullptr);
+        if constexpr (!kIsHalf<TIn>) {   // caller's bf16 v -> the fp16 operand image, in place
+          uint8_t* pv = VV + fpnl * 8192 + swz_off(tok, fpc);
+          float v4[4];
+          ld_act4(pv, v4, (TIn*)nullptr);
+          st_h4(pv, v4[0], v4[1], v4[2], v4[3]);
+        }
+      }
+      float pre[8][4], suf[8][4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        pre[0][c] = al[0][c];
+#pragma unroll
+        for (int j = 1; j < 8; ++j) pre[j][c] = pre[j - 1][c] * al[j][c];
+        suf[7][c] = 1.f;
+#pragma unroll
+        for (int j = 6; j >= 0; --j) suf[j][c] = suf[j + 1][c] * al[j + 1][c];
+      }
+      *reinterpret_cast<float4*>(tot + fo * D + 4 * lane) = make_float4(pre[7][0], pre[7][1], pre[7][2], pre[7][3]);
+      if (tid == 0) bulk_wait_read();   // staged record stores have read KN, TT and PP
+      __syncthreads();                  // octet totals published; log alpha read (G is free)
+      {
+        // outer factors from the octet totals (fo is uniform over the warp)
+        float gb[4], ka[4], f5[4], f4[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) gb[c] = ka[c] = f5[c] = f4[c] = 1.f;
+#pragma unroll
+        for (int o = 0; o < 8; ++o) {
+          const float4 t4 = *reinterpret_cast<const float4*>(tot + o * D + 4 * lane);
+          const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
+          const bool in5 = (fo & 4) ? (o >= 4 && o < fo) : (o > fo && o < 4);
+          const bool in4 = (fo & 2) ? ((fo & 1) && o == fo - 1) : (!(fo & 1) && o == fo + 1);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            if (o < fo) gb[c] *= tv[c];
+            if (o > fo) ka[c] *= tv[c];
+            if (in5) f5[c] *= tv[c];
+            if (in4) f4[c] *= tv[c];
+          }
+          if (fo == 0) {
+            // Gamma_l: the decay over the whole sub-chunk
+            if (o == 0) *reinterpret_cast<float4*>(egl + 4 * lane) = t4;
+            else {
+              float4 e = *reinterpret_cast<const float4*>(egl + 4 * lane);
+              e.x *= t4.x; e.y *= t4.y; e.z *= t4.z; e.w *= t4.w;
+              *reinterpret_cast<float4*>(egl + 4 * lane) = e;
+            }
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int tok = 8 * fo + j;
+          float g[4], kt[4], r3[4], r4[4], r5[4];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            g[c] = gb[c] * pre[j][c];
+            kt[c] = suf[j][c] * ka[c];
+            r3[c] = (fo & 1) ? pre[j][c] : suf[j][c];
+            r4[c] = (fo & 2) ? f4[c] * pre[j][c] : suf[j][c] * f4[c];
+            r5[c] = (fo & 4) ? f5[c] * pre[j][c] : suf[j][c] * f5[c];
+          }
+          const float* kk = kx[j];
+          const float* qq = qx[j];
+          const uint32_t o128 = swz_off(tok, fpc);
+          st_h4(KQ + fpnl * 16384 + o128, kk[0] * g[0], kk[1] * g[1], kk[2] * g[2], kk[3] * g[3]);
+          st_h4(KQ + fpnl * 16384 + swz_off(64 + tok, fpc), qq[0] * g[0], qq[1] * g[1], qq[2] * g[2], qq[3] * g[3]);
+          st_h4(KN + fpnl * 8192 + o128, kk[0] * kt[0], kk[1] * kt[1], kk[2] * kt[2], kk[3] * kt[3]);
+          // Gram levels 5, 4, 3 (tile li = 5 - level): role from bit `level` of the token
+#pragma unroll
+          for (int li = 0; li < 3; ++li) {
+            const int lvl = 5 - li;
+            const float* f = li == 0 ? r5 : (li == 1 ? r4 : r3);
+            const int pos = level_pos(tok, lvl);
+            if ((tok >> lvl) & 1) {
+              uint8_t* rt = G + G_ROW + li * 16384 + fpnl * 8192;
+              st_h4(rt + swz_off(pos, fpc), kk[0] * f[0], kk[1] * f[1], kk[2] * f[2], kk[3] * f[3]);
+              st_h4(rt + swz_off(32 + pos, fpc), qq[0] * f[0], qq[1] * f[1], qq[2] * f[2], qq[3] * f[3]);
+            } else {
+              uint8_t* ct = G + G_COL + li * 8192 + fpnl * 4096;
+              st_h4(ct + swz_off(pos, fpc), kk[0] * f[0], kk[1] * f[1], kk[2] * f[2], kk[3] * f[3]);
+            }
           }
         }
       }
       fence_proxy_async();
+      fence_before_sync();
       __syncthreads();
-      if (tid < 128) {
-        const float gmx = gm_s[tid], totx = tot_s[tid];
-        egm[tid] = __expf(gmx);
-        egl[tid] = __expf(gmx + totx);
-        ekt[tid] = __expf(totx);
-      }
-      if (tid == 0 && alive) {
-        // X consumed: fetch the log alpha of this CTA's next sub-chunk
-        const int nunit = s == 0 ? unit : unit + (int)gridDim.x;
-        if (nunit < a.n_units) {
-          issue_la(nunit, s ^ 1);
-          la_inflight = true;
-        }
-      }
-      // ---------------- A, P = [KG; QG] KN^T ----------------
+      // ---------------- Gram levels on the tensor cores ----------------
+      // Level l pairs the 32 tokens with bit l set (rows: k and q, scaled by the decay from
+      // the level's split point) with the 32 with bit l clear (columns: k, scaled by the
+      // decay up to it): entry (r, i) is valid when r and i share their bits above l, and
+      // then equals sum_c k_r (or q_r) k_i e^{g_r - g_i}.  Levels 5, 4, 3 cover every pair
+      // in different octets; pairs inside an octet follow on the CUDA cores.
       if (tid == 0 && alive) {
         fence_after_sync();
 #pragma unroll
-        for (int k16 = 0; k16 < 8; ++k16)
-          mma_ss(tmem_at(tm, 0, C_AP), dKQk + kstep(k16, 16384), dKNk + kstep(k16, 8192), id_ap, k16 > 0);
+        for (int li = 0; li < 3; ++li)
+#pragma unroll
+          for (int k16 = 0; k16 < 8; ++k16)
+            mma_ss(tmem_at(tm, 0, C_G + 32 * li), dGrow + ((uint32_t)li * 16384 >> 4) + kstep(k16, 8192),
+                   dGcol + ((uint32_t)li * 8192 >> 4) + kstep(k16, 4096), id_gram, k16 > 0);
         mma_commit(bar);
       }
-      if (tid == 0) bulk_wait_read();   // staged records read: their tiles may be rewritten
-      alive = __syncthreads_and(wait_mma(bar, phase, a.status, alive));
+      {
+        // pairs inside the octet: e^{g_r - g_i} = prod_{u=i+1..r} alpha_u as a running product
+        float acc[64];
+#pragma unroll
+        for (int x = 0; x < 64; ++x) acc[x] = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            float kf = kx[i][c];
+            acc[oct_p(i, i)] += qx[i][c] * kf;
+#pragma unroll
+            for (int r = i + 1; r < 8; ++r) {
+              kf *= al[r][c];
+              acc[oct_a(r, i)] += kx[r][c] * kf;
+              acc[oct_p(r, i)] += qx[r][c] * kf;
+            }
+          }
+        }
+        warp_reduce_scatter64(acc, lane);
+        *reinterpret_cast<float2*>(gscr + fo * 64 + 2 * lane) = make_float2(acc[0], acc[1]);
+      }
+      alive = __syncthreads_and(wait_mma(bar, phase, a.status, alive, a.wait_ns));
       fence_after_sync();
       {
-        // A rows (TMEM lanes 0-63) -> As (beta, strict lower); P rows (lanes 64-127) -> PP (lower)
-        const int row = 32 * sub + lane;
-        const int col0 = 32 * chalf;
-        float v[32];
-        tmem_ld32(tmem_at(tm, 32 * sub, C_AP + col0), v);
-        tmem_wait_ld();
-        if (sub < 2) {
-          const float bt = beta_s[row];
+        // Gram levels -> A (fp32, beta applied, As) and P (fp16, PP).  M = 64 accumulator layout:
+        // row m at lane 32 (m / 16) + m % 16; rows 0-31 are k rows (A), 32-63 q rows (P).
+        const int qd = warp & 3;
+        const bool isP = qd >= 2;
+        const int mr = 16 * (qd & 1) + lane;   // row among the 32 of its kind (lanes < 16)
+        auto put = [&](int r, int i0, const float* v, int n) {   // n = 8, 16 or 32 consecutive columns
+          if (!isP) {
+            const float bt = beta_s[r];
 #pragma unroll
-          for (int j = 0; j < 32; j += 4)
-            *reinterpret_cast<float4*>(As + row * LDA + col0 + j) =
-                make_float4(col0 + j < row ? bt * v[j] : 0.f, col0 + j + 1 < row ? bt * v[j + 1] : 0.f,
-                            col0 + j + 2 < row ? bt * v[j + 2] : 0.f, col0 + j + 3 < row ? bt * v[j + 3] : 0.f);
+            for (int j = 0; j < n; j += 4)
+              *reinterpret_cast<float4*>(As + r * LDA + i0 + j) =
+                  make_float4(bt * v[j], bt * v[j + 1], bt * v[j + 2], bt * v[j + 3]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < n; j += 8) *reinterpret_cast<uint4*>(PP + swz_off(r, i0 + j)) = pack8(v + j);
+          }
+        };
+        if (warp < 4) {
+          float v[32];   // level 5: rows 32..63 against columns 0..31, all valid
+          tmem_ld32(tmem_at(tm, 32 * qd, C_G), v);
+          tmem_wait_ld();
+          if (lane < 16) put(32 + mr, 0, v, 32);
         } else {
-          const int r = row - 64;
+          float v4[16], v3[16];
+          // level 4: this warp's 16 rows share one 16-column block; level 3: two 8-column blocks
+          tmem_ld16(tmem_at(tm, 32 * qd, C_G + 32 + 16 * (qd & 1)), v4);
+          tmem_ld16(tmem_at(tm, 32 * qd, C_G + 64 + 16 * (qd & 1)), v3);
+          tmem_wait_ld();
+          if (lane < 16) {
+            put(((mr >> 4) << 5) | 16 | (mr & 15), 32 * (mr >> 4), v4, 16);
+            float w8[8];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = (col0 + j <= r) ? v[j] : 0.f;
-          st_row32_h(PP, r, col0, v);
+            for (int c = 0; c < 8; ++c) w8[c] = (lane & 8) ? v3[8 + c] : v3[c];
+            put(((mr >> 3) << 4) | 8 | (mr & 7), 16 * (mr >> 3), w8, 8);
+          }
+        }
+        if (tid < SUB) {
+          // row r: the pairs inside its octet, and zeros above the diagonal of P
+          const int r = tid, o = r >> 3, jr = r & 7;
+          const float bt = beta_s[r];
+          const float* gs = gscr + o * 64;
+          for (int ji = 0; ji < jr; ++ji) As[r * LDA + 8 * o + ji] = bt * gs[oct_a(jr, ji)];
+          float pv[8];
+#pragma unroll
+          for (int ji = 0; ji < 8; ++ji) pv[ji] = ji <= jr ? gs[oct_p(jr, ji)] : 0.f;
+          *reinterpret_cast<uint4*>(PP + swz_off(r, 8 * o)) = pack8(pv);
+          for (int c8 = o + 1; c8 < 8; ++c8) *reinterpret_cast<uint4*>(PP + swz_off(r, 8 * c8)) = make_uint4(0, 0, 0, 0);
         }
       }
+      fence_proxy_async();
       fence_before_sync();
       __syncthreads();
-      // T = (I + A)^{-1} Diag(beta) -> TT; W' = T KG, U~ = T V over T's columns 32-63 first,
+      // T = (I + A)^{-1} Diag(beta) -> TT; W = T K Gamma, U~ = T V over T's columns 32-63 first,
       // issued as soon as they are written, then over columns 0-31
       inverse_diag32(As, Xs, Ys, TT, beta_s);
       inverse_merge64(As, Xs, Ys, TT, beta_s, [&]() {
@@ -625,26 +748,16 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
           mma_ss(tmem_at(tm, 0, C_U), ad, dVVm + mstep(k16), id_64x128_kmn, 1);
         }
         mma_commit(bar);
+        // A, X, Y consumed: G takes the log alpha of this CTA's next sub-chunk
+        const int nunit = s == 0 ? unit : unit + (int)gridDim.x;
+        if (nunit < a.n_units) {
+          issue_la(nunit, s ^ 1);
+          la_inflight = true;
+        }
       }
-      // KN -> K~ = KN e^{g_l - g_m} in place (KN is no longer read by the tensor core)
-      for (int e = tid; e < SUB * 16; e += 256) {
-        const int r = e >> 4, ch = (e & 15) * 8;
-        uint4* p = reinterpret_cast<uint4*>(KN + (ch >> 6) * 8192 + swz_off(r, ch & 63));
-        float f[8];
-        unpack8(*p, f);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) f[j] *= ekt[ch + j];
-        *p = pack8(f);
-      }
-      // meanwhile the next sub-chunk's decay exponents, part 1 (its log alpha has landed by now)
-      const bool have_next = (s == 0 ? unit : unit + (int)gridDim.x) < a.n_units;
-      bool ok_next = true;
-      if (have_next) ok_next = decay_part1(alive);
-      fence_proxy_async();
-      if (tid == 0) bulk_wait_read();   // staged records read: their tiles may be rewritten
-      alive = __syncthreads_and(wait_mma(bar, phase, a.status, alive) && ok_next);
+      alive = __syncthreads_and(wait_mma(bar, phase, a.status, alive, a.wait_ns));
       fence_after_sync();
-      // W' -> KQ rows 0-63, U~ -> VV (fp16); M=64 accumulator layout: rows 16*sub + lane (lane < 16)
+      // W -> KQ rows 0-63, U~ -> VV (fp16); M=64 accumulator layout: rows 16*sub + lane (lane < 16)
       {
         const int r = 16 * sub + lane;
         for (int cb = 0; cb < 2; ++cb) {
@@ -662,7 +775,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
       fence_proxy_async();
       fence_before_sync();
       __syncthreads();
-      // ---------------- K~^T W', K~^T U~, P W', P U~ ----------------
+      // ---------------- K~^T W, K~^T U~, P W, P U~ ----------------
       if (tid == 0 && alive) {
         fence_after_sync();
 #pragma unroll
@@ -678,17 +791,13 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
         }
         mma_commit(bar);
       }
-      if (have_next && alive) {
-        decay_part2();   // part 2 of the next sub-chunk's exponents
-        x_ready = true;
-      }
       if (tid == 0) bulk_wait_read();   // staged records read: their tiles may be rewritten
-      alive = __syncthreads_and(wait_mma(bar, phase, a.status, alive));
+      alive = __syncthreads_and(wait_mma(bar, phase, a.status, alive, a.wait_ns));
       fence_after_sync();
       const int row = 32 * sub + lane;        // M=128 layout row
       const int r64 = 16 * sub + lane;        // M=64 layout row (lane < 16)
       if (s == 0) {
-        // M_1 = Diag(e^{g_l}) - MK Diag(e^{g_m}) -> M1 tile;  B_1 -> B1 tile
+        // M_1 = Diag(Gamma_l) - K~^T W -> M1 tile;  B_1 -> B1 tile
         for (int cb = 0; cb < 2; ++cb) {
           const int col0 = 64 * chalf + 32 * cb;
           float m[32], bv[32];
@@ -696,13 +805,13 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
           tmem_ld32(tmem_at(tm, 32 * sub, C_BK + col0), bv);
           tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) m[j] = (row == col0 + j ? egl[row] : 0.f) - m[j] * egm[col0 + j];
+          for (int j = 0; j < 32; ++j) m[j] = (row == col0 + j ? egl[row] : 0.f) - m[j];
           st_row32_h(M1 + chalf * 16384, row, col0 & 63, m);
           st_row32_h(B1 + chalf * 16384, row, col0 & 63, bv);
         }
-        // R_1 = (QG - P W') Diag(e^{g_m}) and O'_1, staged for the record (R rows 0-63, O'' rows 0-63)
-        uint8_t* stR = reinterpret_cast<uint8_t*>(Xs);   // [panel][64 rows][128 B], swizzled
-        uint4* stO = reinterpret_cast<uint4*>(As);       // [c/8][64 rows][8]
+        // R_1 = Q Gamma - P W and O'_1, staged for the record (R rows 0-63, O'' rows 0-63)
+        uint8_t* stR = TT;                                  // [panel][64 rows][128 B], swizzled (TT and PP)
+        uint4* stO = reinterpret_cast<uint4*>(KN);          // [c/8][64 rows][8]
         for (int cb = 0; cb < 2; ++cb) {
           const int col0 = 64 * chalf + 32 * cb;
           float pw[32], pu[32];
@@ -714,7 +823,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
             ld_row16_h(KQ + chalf * 16384, 64 + r64, col0 & 63, qg);
             ld_row16_h(KQ + chalf * 16384, 64 + r64, (col0 & 63) + 16, qg + 16);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) qg[j] = (qg[j] - pw[j]) * egm[col0 + j];
+            for (int j = 0; j < 32; ++j) qg[j] -= pw[j];
             st_row32_h(stR + chalf * 8192, r64, col0 & 63, qg);
 #pragma unroll
             for (int i = 0; i < 4; ++i) stO[((col0 >> 3) + i) * 64 + r64] = pack8(pu + 8 * i);
@@ -724,7 +833,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
         fence_before_sync();
         __syncthreads();
         if (tid == 0) {
-          // KQ (QG read above) and VV are free: sub-chunk 1's tiles first, then the stores
+          // KQ (Q Gamma read above) and VV are free: sub-chunk 1's tiles first, then the stores
           if (alive) {
             issue_kqv(b, h, (int)t0 + SUB);
             kqv_early = true;
@@ -736,7 +845,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
           bulk_commit();
         }
       } else {
-        // Q^_2 = (QG - P W') Diag(e^{g_m}) -> VV region (U~ no longer needed)
+        // Q^_2 = Q Gamma - P W -> VV region (U~ no longer needed)
         for (int cb = 0; cb < 2; ++cb) {
           const int col0 = 64 * chalf + 32 * cb;
           float pw[32];
@@ -747,7 +856,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
             ld_row16_h(KQ + chalf * 16384, 64 + r64, col0 & 63, qg);
             ld_row16_h(KQ + chalf * 16384, 64 + r64, (col0 & 63) + 16, qg + 16);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) qg[j] = (qg[j] - pw[j]) * egm[col0 + j];
+            for (int j = 0; j < 32; ++j) qg[j] -= pw[j];
             st_row32_h(VV + chalf * 8192, r64, col0 & 63, qg);
           }
         }
@@ -759,7 +868,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
           tmem_ld32(tmem_at(tm, 32 * sub, C_MK + col0), m);
           tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) m[j] = (row == col0 + j ? egl[row] : 0.f) - m[j] * egm[col0 + j];
+          for (int j = 0; j < 32; ++j) m[j] = (row == col0 + j ? egl[row] : 0.f) - m[j];
           st_row32_h(KQ + chalf * 16384, row, col0 & 63, m);
         }
         fence_proxy_async();
@@ -783,7 +892,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
           mma_commit(bar);
         }
         if (tid == 0) bulk_wait_read();   // staged records read: their tiles may be rewritten
-        alive = __syncthreads_and(wait_mma(bar, phase, a.status, alive));
+        alive = __syncthreads_and(wait_mma(bar, phase, a.status, alive, a.wait_ns));
         fence_after_sync();
         if (tid == 0 && alive) {
           // KQ and VV are free now: start the next unit's tiles before this unit's stores
@@ -795,9 +904,9 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
           }
         }
         // records staged in tiles the combine products no longer read:
-        //   M -> M1 region, B -> B1 region, R_2 -> TT/PP region, O''_2 -> Xs region
+        //   M -> M1 region, B -> B1 region, R_2 -> TT/PP region, O''_2 -> KN region
         uint8_t* stR = TT;                               // [panel][64 rows][128 B], swizzled
-        uint4* stO = reinterpret_cast<uint4*>(Xs);       // [c/8][64 rows][8]
+        uint4* stO = reinterpret_cast<uint4*>(KN);       // [c/8][64 rows][8]
         for (int cb = 0; cb < 2; ++cb) {
           const int col0 = 64 * chalf + 32 * cb;
           float m[32], bv[32];
@@ -845,7 +954,6 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
     if (kqv_inflight) mbar_wait(kqv_bar, kqv_phase, 100000000ull);
     bulk_wait_all();
   }
-  if (tid == 0 && *range_flag) set_status(a.status, KDA_ERR_RANGE);
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
@@ -883,15 +991,17 @@ struct ChainArgs {
   __nv_bfloat16* o;
   int64_t N; int H; int n_blocks;
   uint32_t* status;
+  uint64_t wait_ns;       // limit of every device wait
+  int fault;              // self-test: 2 = CTA (0, 0, 0) never issues its first record load
 };
 
-// Bounded wait that also gives up as soon as another thread of the CTA gave up.
-__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+// Bounded wait (at most tmo ns) that also gives up as soon as another thread of the CTA gave up.
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag, uint64_t tmo) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try_wait(bar, parity)) {
     if (*abort_flag) return false;
-    if (globaltimer_ns() - t0 > 500000000ull) { *abort_flag = 1; return false; }
+    if (globaltimer_ns() - t0 > tmo) { *abort_flag = 1; return false; }
   }
   return true;
 }
@@ -948,9 +1058,12 @@ __global__ void __launch_bounds__(256, 1) kda_tc_chain(ChainArgs a) {
     };
     // thread 32 refills ring A, so thread 0 goes from the barrier straight to the next product
     const bool loaderA = tid == 32;
+    // self-test of the bounded waits: the first record load is never issued, so its wait gives up
+    const bool skipA0 = a.fault == 2 && qtr == 0 && h == 0 && b == 0;
     int issuedA = 0, mma_pending = 0;
     if (loaderA)
-      for (; issuedA < 2 && issuedA < nb; ++issuedA) load_A(issuedA);
+      for (; issuedA < 2 && issuedA < nb; ++issuedA)
+        if (!(skipA0 && issuedA == 0)) load_A(issuedA);
     float S[CW];
 #pragma unroll
     for (int c = 0; c < CW; ++c)
@@ -968,7 +1081,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_chain(ChainArgs a) {
     int j = 0;
     for (; j < nb && ok; ++j) {
       if (tid == 0) {
-        const bool landed = wait_or_abort(&fullA[j & 1], (uint32_t)(j >> 1) & 1u, abort_flag);
+        const bool landed = wait_or_abort(&fullA[j & 1], (uint32_t)(j >> 1) & 1u, abort_flag, a.wait_ns);
         if (landed) {
           fence_after_sync();
           const uint64_t da = dA + (uint32_t)(j & 1) * (CH_SLOT >> 4);
@@ -980,9 +1093,9 @@ __global__ void __launch_bounds__(256, 1) kda_tc_chain(ChainArgs a) {
           mma_pending = 1;
         }
       }
-      bool mine = wait_or_abort(msDone, (uint32_t)j & 1u, abort_flag);
+      bool mine = wait_or_abort(msDone, (uint32_t)j & 1u, abort_flag, a.wait_ns);
       if (tid == 0 && mine) mma_pending = 0;
-      mine = mine && wait_or_abort(&fullA[j & 1], (uint32_t)(j >> 1) & 1u, abort_flag);   // B_j visible here too
+      mine = mine && wait_or_abort(&fullA[j & 1], (uint32_t)(j >> 1) & 1u, abort_flag, a.wait_ns);   // B_j visible here too
       if (mine) {
         fence_after_sync();
         const uint4* Bs = reinterpret_cast<const uint4*>(sm + CH_OFF_A + (j & 1) * CH_SLOT + 32768);
@@ -1004,7 +1117,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_chain(ChainArgs a) {
         }
         if (j + 1 < nb) {
           // image (j+1)&1 last held S_{j-1}; R S_{j-1} must be done with it
-          if (j >= 1) mine = wait_or_abort(&sFree[(j - 1) & 1], (uint32_t)((j - 1) >> 1) & 1u, abort_flag);
+          if (j >= 1) mine = wait_or_abort(&sFree[(j - 1) & 1], (uint32_t)((j - 1) >> 1) & 1u, abort_flag, a.wait_ns);
           if (mine) store_S((j + 1) & 1);
         }
       }
@@ -1019,7 +1132,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_chain(ChainArgs a) {
     if (tid == 0 && mma_pending) mbar_wait(msDone, (uint32_t)(j - 1) & 1u, 100000000ull);
     if (loaderA)   // each slot's latest load lands before the CTA exits (consumed ones return at once)
       for (int jj = max(0, issuedA - 2); jj < issuedA; ++jj)
-        mbar_wait(&fullA[jj & 1], (uint32_t)(jj >> 1) & 1u, 100000000ull);
+        if (!(skipA0 && jj == 0)) mbar_wait(&fullA[jj & 1], (uint32_t)(jj >> 1) & 1u, 100000000ull);
   } else {
     // ---------------- output group ----------------
     const int r = tid - 128;   // token row of the block = TMEM lane
@@ -1042,10 +1155,10 @@ __global__ void __launch_bounds__(256, 1) kda_tc_chain(ChainArgs a) {
     __nv_bfloat16* obase = a.o + (int64_t)b * a.N * tok_stride + (int64_t)h * D + CW * qtr;
     for (int j = 0; j < nb && ok; ++j) {
       if (leader) {
-        bool go = wait_or_abort(&sReady[j & 1], (uint32_t)(j >> 1) & 1u, abort_flag);
+        bool go = wait_or_abort(&sReady[j & 1], (uint32_t)(j >> 1) & 1u, abort_flag, a.wait_ns);
         // issued once M S_j is done, so it does not share the tensor pipe with the serial product
-        go = go && wait_or_abort(&oGo[j & 1], (uint32_t)(j >> 1) & 1u, abort_flag);
-        go = go && wait_or_abort(&fullB[j & 1], (uint32_t)(j >> 1) & 1u, abort_flag);
+        go = go && wait_or_abort(&oGo[j & 1], (uint32_t)(j >> 1) & 1u, abort_flag, a.wait_ns);
+        go = go && wait_or_abort(&fullB[j & 1], (uint32_t)(j >> 1) & 1u, abort_flag, a.wait_ns);
         if (go) {
           fence_after_sync();
           const uint64_t da = dR + (uint32_t)(j & 1) * (CH_SLOT >> 4);
@@ -1058,9 +1171,9 @@ __global__ void __launch_bounds__(256, 1) kda_tc_chain(ChainArgs a) {
           o_pending = j;
         }
       }
-      bool mine = wait_or_abort(&oDone[j & 1], (uint32_t)(j >> 1) & 1u, abort_flag);
+      bool mine = wait_or_abort(&oDone[j & 1], (uint32_t)(j >> 1) & 1u, abort_flag, a.wait_ns);
       if (leader && mine) o_pending = -1;
-      mine = mine && wait_or_abort(&fullB[j & 1], (uint32_t)(j >> 1) & 1u, abort_flag);   // O''_j visible here too
+      mine = mine && wait_or_abort(&fullB[j & 1], (uint32_t)(j >> 1) & 1u, abort_flag, a.wait_ns);   // O''_j visible here too
       if (mine) {
         fence_after_sync();
         const uint4* Oo = reinterpret_cast<const uint4*>(sm + CH_OFF_B + (j & 1) * CH_SLOT + 32768);
@@ -1147,7 +1260,7 @@ cudaError_t launch_chain(const ChainArgs& ca, dim3 grid, cudaStream_t s) {
 template <typename TIn>
 cudaError_t launch_all(const Dims& d, const void* q, const void* k, const void* v, const float* la,
                        const void* beta, const float* S0, void* o, float* SN, uint8_t* ws, uint32_t* status,
-                       cudaStream_t s, int* launches) {
+                       cudaStream_t s, int* launches, int fault, uint64_t wait_ns) {
   const int n_blocks = (int)((d.N + BLK - 1) / BLK);
   cudaError_t e;
   int dev = 0, n_sm = 148;
@@ -1158,7 +1271,7 @@ cudaError_t launch_all(const Dims& d, const void* q, const void* k, const void* 
 
   const int BH = d.B * d.H;
   const int n_units = BH * n_blocks;
-  PrepArgs pa{q, k, v, la, beta, ws, d.N, d.H, BH, n_blocks, n_units, status};
+  PrepArgs pa{q, k, v, la, beta, ws, d.N, d.H, BH, n_blocks, n_units, status, wait_ns, fault};
   PrepMaps mp;
   const CUtensorMapDataType adt = kIsHalf<TIn> ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   if (!encode_act_map(&mp.q, q, adt, 2, d, 64, true) || !encode_act_map(&mp.k, k, adt, 2, d, 64, true) ||
@@ -1171,7 +1284,7 @@ cudaError_t launch_all(const Dims& d, const void* q, const void* k, const void* 
     kda_tc_prep<TIn><<<dim3((unsigned)min(n_units, n_sm)), 256, PREP_SMEM, s>>>(pa, mp);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  ChainArgs ca{ws, S0, SN, static_cast<__nv_bfloat16*>(o), d.N, d.H, n_blocks, status};
+  ChainArgs ca{ws, S0, SN, static_cast<__nv_bfloat16*>(o), d.N, d.H, n_blocks, status, wait_ns, fault};
   // the narrowest column split whose grid fits on the SMs (the serial pass is latency bound)
   const int bh = d.B * d.H;
   if (ChainLayout<16>::NQ * bh <= n_sm) e = launch_chain<16>(ca, dim3(ChainLayout<16>::NQ, d.H, d.B), s);
@@ -1194,13 +1307,14 @@ bool chunk_tc_supported(const Dims& d) { return d.dk == D && d.dv == D; }
 
 cudaError_t launch_chunk_tc(const Dims& d, bool in_f16, const void* q, const void* k, const void* v,
                             const float* log_alpha, const void* beta, const float* S0, void* o, float* SN,
-                            void* ws, uint32_t* status, cudaStream_t s, int* launches) {
+                            void* ws, uint32_t* status, cudaStream_t s, int* launches, int fault,
+                            uint64_t wait_ns) {
   // beta and o are bf16 (the problem dtype); q', k', v' are fp16 (internal conv output) or bf16 (caller)
   if (in_f16)
     return launch_all<__half>(d, q, k, v, log_alpha, beta, S0, o, SN, static_cast<uint8_t*>(ws), status, s,
-                              launches);
+                              launches, fault, wait_ns);
   return launch_all<__nv_bfloat16>(d, q, k, v, log_alpha, beta, S0, o, SN, static_cast<uint8_t*>(ws), status, s,
-                                   launches);
+                                   launches, fault, wait_ns);
 }
 
 }  // namespace kda

@@ -185,11 +185,13 @@ def forward(inp: dict, text_len: int, grid, S0=None, heads=None, text_k=4, vis_k
 
 
 def forward_columns(inp: dict, text_len: int, grid, items, S0=None, text_k=4, vis_k=(3, 3, 3),
-                    vis_causal_t=False, nthreads=None):
+                    vis_causal_t=False, nthreads=None, workers=1):
     """o[b, :, h, j] for each (h, j) in ``items`` and every batch item b.
 
     Column j of the state depends only on column j of v, so each sampled
-    column is exact at any sequence length.  Returns float64 [len(items), B, N].
+    column is exact at any sequence length.  ``workers`` > 1 evaluates the heads
+    concurrently on host threads (the C routines release the interpreter lock);
+    the arithmetic is the same.  Returns float64 [len(items), B, N].
     """
     B, N, H, d = inp["shape"]
     shape = conv_shape(B, N, text_len, grid, text_k, vis_k, vis_causal_t)
@@ -198,15 +200,26 @@ def forward_columns(inp: dict, text_len: int, grid, items, S0=None, text_k=4, vi
     by_head = {}
     for i, (h, j) in enumerate(items):
         by_head.setdefault(h, []).append((i, j))
-    for h, lst in by_head.items():
-        qh, kh, _, la, bt = _heads_inputs(inp, h, shape, d, nthreads, v_cols=(0, 1), xs=xs)
+
+    def one_head(h, lst, nt):
+        qh, kh, _, la, bt = _heads_inputs(inp, h, shape, d, nt, v_cols=(0, 1), xs=xs)
         for i, j in lst:
-            vj = shortconv(shape, xs[2], inp["w_text"][2], inp["w_vis"][2], h * d + j, h * d + j + 1, nthreads)
+            vj = shortconv(shape, xs[2], inp["w_text"][2], inp["w_vis"][2], h * d + j, h * d + j + 1, nt)
             vfull = np.zeros((B, N, d), dtype=np.float64)
             vfull[:, :, j] = vj[:, :, 0]
             s0 = None if S0 is None else np.asarray(S0)[:, h]
-            oh, _ = scan(qh, kh, vfull, la, bt, s0, j0=j, j1=j + 1, nthreads=nthreads)
+            oh, _ = scan(qh, kh, vfull, la, bt, s0, j0=j, j1=j + 1, nthreads=nt)
             res[i] = oh[:, :, j]
+
+    if workers <= 1:
+        for h, lst in by_head.items():
+            one_head(h, lst, nthreads)
+    else:
+        from concurrent.futures import ThreadPoolExecutor
+        nt = max(1, (nthreads or default_threads()) // workers)
+        with ThreadPoolExecutor(workers) as pool:
+            for f in [pool.submit(one_head, h, lst, nt) for h, lst in by_head.items()]:
+                f.result()
     return res
 
 
