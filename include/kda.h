@@ -51,10 +51,11 @@
  *    size (dk, dv, chunk, kernel extents), a data pointer that is not 16-byte
  *    aligned, or a workspace smaller than kda_workspace_bytes().
  *  - Outputs must not alias inputs.
- *  - Device-side conditions (bounded waits that gave up, the gate range check
- *    of the bf16 tensor-core path) are recorded in a status word at the start
- *    of the workspace; read it with kda_read_status() once the stream has
- *    reached the call.  Kernels never trap.
+ *  - Device-side conditions (bounded waits that gave up; the gate range check
+ *    of the backward pass) are recorded in a status word at the start of the
+ *    workspace; read it with kda_read_status() once the stream has reached the
+ *    call.  Kernels never trap.  The forward pass accepts any finite
+ *    log_alpha <= 0: its decay factors are products of gates alpha <= 1.
  */
 #ifndef KDA_H
 #define KDA_H
@@ -75,7 +76,7 @@ typedef enum {
   KDA_ERR_CUDA = 5,           /* a CUDA runtime call failed (launch, copy) */
   KDA_ERR_TIMEOUT = 6,        /* device: a bounded wait gave up */
   KDA_ERR_DEVICE_ASSERT = 7,  /* device: an internal consistency check failed */
-  KDA_ERR_RANGE = 8           /* device: a chunk's gate decay exceeds what the tensor path (or the backward) handles */
+  KDA_ERR_RANGE = 8           /* device: a chunk's gate decay exceeds what the backward pass handles */
 } kda_status;
 
 typedef enum { KDA_DT_BF16 = 0, KDA_DT_F32 = 1 } kda_dtype;
@@ -104,7 +105,10 @@ typedef struct {
   int32_t grid_t, grid_h, grid_w;   /* visual grid (each >= 0; all 0 or all > 0) */
   int32_t text_k;                   /* causal text kernel length, 1..8 */
   int32_t vis_kt, vis_kh, vis_kw;   /* 3D kernel extents; only 3,3,3 is implemented */
-  int32_t chunk;                    /* scan chunk length: 16, 32 or 64 (fp32); 64 (bf16) */
+  int32_t chunk;                    /* scan chunk length: 16, 32 or 64 for fp32 and for bf16 with
+                                       d = 64; exactly 64 for bf16 with d = 128 (the tensor-core
+                                       path's 64-token sub-chunks); anything else, 128 included,
+                                       returns KDA_ERR_UNSUPPORTED */
   uint32_t flags;                   /* KDA_FLAG_* */
 } kda_problem;
 
@@ -213,7 +217,9 @@ int kda_bwd(const kda_problem* p, kda_dtype dtype,
  *    on the bf16 d=128 tensor-core path) returns KDA_ERR_WORKSPACE without
  *    launching anything.
  *  - The first call on a device looks up that array's device address (once per
- *    device); make it before any stream capture.
+ *    device); make it before any stream capture.  The address belongs to the
+ *    device's primary context: do not use this entry point on a device again
+ *    after cudaDeviceReset in the same process.
  *  - Calls share the array: calls whose GPU work overlaps (other streams, other
  *    host threads on the same device) race.  Run them on one stream.
  *  - Device-side conditions (see kda_read_status) are written to *device_status
@@ -226,6 +232,25 @@ int kda_chunk_fwd_noalloc(const kda_problem* p, kda_dtype dtype,
                           const float* log_alpha, const void* beta,
                           const float* initial_state, void* o, float* final_state,
                           uint32_t* device_status, void* stream);
+
+/* Self-test of the bounded device waits; the pages have no counterpart.  Every wait of the kernels
+ * (for an asynchronous copy, a tensor-core product or another warp) gives up after a time limit and
+ * records KDA_ERR_TIMEOUT instead of hanging the GPU; this call makes one such wait run out on purpose
+ * so that a test can check the give-up path without faulting or hanging anything.  It runs
+ * kda_chunk_fwd's kernels on a bf16 problem with dk = dv = 128 (the tensor-core path; other problems
+ * return KDA_ERR_UNSUPPORTED) with every device wait limited to wait_us microseconds (>= 1), and one
+ * asynchronous load that is never issued:
+ *   stage 1: the first k/q/v tile load of the first CTA of the block-record kernel;
+ *   stage 2: the first record load of the first CTA of the serial state pass.
+ * The CTA whose wait gives up records KDA_ERR_TIMEOUT in the workspace status word, waits (bounded)
+ * for its other copies, frees its tensor memory and returns; CTAs and kernels that start later skip
+ * their work.  o is not valid afterwards.  Arguments as in kda_chunk_fwd (no states).  Returns
+ * KDA_OK once the work is enqueued; kda_read_status then reports KDA_ERR_TIMEOUT. */
+int kda_selftest_wait_timeout(const kda_problem* p, kda_dtype dtype,
+                              const void* q, const void* k, const void* v,
+                              const float* log_alpha, const void* beta, void* o,
+                              void* workspace, size_t workspace_bytes,
+                              int32_t stage, uint32_t wait_us, void* stream);
 
 /* Synchronises `stream`, then returns and clears the device status word kept
  * in `workspace` (KDA_OK if no device-side condition was recorded). */

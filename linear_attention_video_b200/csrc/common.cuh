@@ -65,13 +65,20 @@ size_t chunk_simt_smem_bytes(int dk, int chunk);
 // tcgen05 path (bf16 problems with d_k = d_v = 128)
 bool chunk_tc_supported(const Dims& d);
 size_t chunk_tc_workspace_bytes(const Dims& d);
+// fault (self-test of the bounded waits only): 1 = the record kernel's first CTA never issues its first
+// input load, 2 = the state pass's first CTA never issues its first record load; wait_ns bounds every
+// device wait of the two kernels.
+constexpr uint64_t kWaitNs = 500000000ull;
 cudaError_t launch_chunk_tc(const Dims& d, bool in_f16, const void* q, const void* k, const void* v,
                             const float* log_alpha, const void* beta, const float* S0, void* o, float* SN,
-                            void* ws, uint32_t* status, cudaStream_t s, int* launches);
+                            void* ws, uint32_t* status, cudaStream_t s, int* launches, int fault = 0,
+                            uint64_t wait_ns = kWaitNs);
 
 // Host-side validation (kda_api.cu), returning a kda_status.
 int validate_problem(const kda_problem* p, kda_dtype dt, Dims* d);
 int validate_scan_pointers(const void* q, const void* k, const void* v, const void* la, const void* beta, const void* o,
                            const void* s0, const void* sn);
+// Records the launch count that kda_last_launch_count() reports for this host thread.
+void set_last_launch_count(int launches);
 
 }  // namespace kda

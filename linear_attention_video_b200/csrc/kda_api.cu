@@ -52,6 +52,8 @@ int make_dims(const kda_problem* p, kda_dtype dt, kda::Dims* d) {
   d->qkv_f16 = (p->flags & KDA_FLAG_QKV_F16) != 0;
   // fp16 activations exist only where the tensor-core scan reads them (bf16, d = 128)
   if (d->qkv_f16 && !(dt == KDA_DT_BF16 && kda::chunk_tc_supported(*d))) return KDA_ERR_UNSUPPORTED;
+  // the tensor-core scan (bf16, d = 128) works on 64-token sub-chunks composed into 128-token blocks
+  if (dt == KDA_DT_BF16 && kda::chunk_tc_supported(*d) && d->chunk != 64) return KDA_ERR_UNSUPPORTED;
   return KDA_OK;
 }
 
@@ -158,6 +160,7 @@ int validate_scan_pointers(const void* q, const void* k, const void* v, const vo
                            const void* s0, const void* sn) {
   return check_ptrs({q, k, v, la, beta, o}, {s0, sn});
 }
+void set_last_launch_count(int launches) { g_last_launches = launches; }
 }  // namespace kda
 
 extern "C" {
@@ -415,6 +418,28 @@ int kda_fwd_host(const kda_problem* p, kda_dtype dtype, const void* q, const voi
   return KDA_OK;
 }
 
+int kda_selftest_wait_timeout(const kda_problem* p, kda_dtype dtype, const void* q, const void* k, const void* v,
+                              const float* log_alpha, const void* beta, void* o, void* workspace,
+                              size_t workspace_bytes_, int32_t stage, uint32_t wait_us, void* stream) {
+  g_last_launches = 0;
+  kda::Dims d;
+  int st = make_dims(p, dtype, &d);
+  if (st) return st;
+  if (!use_tc(d, dtype) || d.reuse_records || d.N == 0) return KDA_ERR_UNSUPPORTED;
+  if ((stage != 1 && stage != 2) || wait_us < 1) return KDA_ERR_INVALID_ARG;
+  if ((st = check_ptrs({q, k, v, log_alpha, beta, o}, {}))) return st;
+  if ((st = check_workspace(d, dtype, workspace, workspace_bytes_))) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t* status = static_cast<uint32_t*>(workspace);
+  if ((st = cuda_status(cudaMemsetAsync(status, 0, sizeof(uint32_t), s)))) return st;
+  int launches = 0;
+  void* rec = static_cast<char*>(workspace) + tc_records_offset(d, dtype);
+  st = cuda_status(kda::launch_chunk_tc(d, d.qkv_f16, q, k, v, log_alpha, beta, nullptr, o, nullptr, rec, status, s,
+                                        &launches, stage, (uint64_t)wait_us * 1000ull));
+  if (!st) g_last_launches = launches;
+  return st;
+}
+
 int kda_read_status(void* workspace, void* stream) {
   if (!workspace) return KDA_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -435,7 +460,7 @@ const char* kda_status_str(int s) {
     case KDA_ERR_CUDA: return "CUDA runtime error";
     case KDA_ERR_TIMEOUT: return "device wait timed out";
     case KDA_ERR_DEVICE_ASSERT: return "device consistency check failed";
-    case KDA_ERR_RANGE: return "gate decay within a chunk exceeds the bf16 tensor path's range";
+    case KDA_ERR_RANGE: return "gate decay within a chunk exceeds the backward pass's range";
     default: return "unknown status";
   }
 }

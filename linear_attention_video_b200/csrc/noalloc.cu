@@ -15,7 +15,10 @@
 // call before any stream capture.  Every call shares the array and it keeps the
 // last call's contents: the status word is cleared at the start of each call,
 // the records are fully rewritten.  Calls whose GPU work overlaps (different
-// streams, or different host threads on one device) race on the array.
+// streams, or different host threads on one device) race on the array.  The
+// cached address belongs to the device's primary context: after a
+// cudaDeviceReset in the process it is stale, and this entry point must not be
+// used again on that device.
 #include <mutex>
 
 #include "common.cuh"
@@ -51,6 +54,7 @@ extern "C" int kda_chunk_fwd_noalloc(const kda_problem* p, kda_dtype dtype, cons
                                      const void* v, const float* log_alpha, const void* beta,
                                      const float* initial_state, void* o, float* final_state,
                                      uint32_t* device_status, void* stream) {
+  kda::set_last_launch_count(0);
   kda::Dims d;
   int st = kda::validate_problem(p, dtype, &d);
   if (st) return st;
@@ -80,5 +84,7 @@ extern "C" int kda_chunk_fwd_noalloc(const kda_problem* p, kda_dtype dtype, cons
     e = kda::launch_chunk_simt(d, dtype, q, k, v, log_alpha, beta, initial_state, o, final_state, status, s,
                                &launches);
   }
-  return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+  if (e != cudaSuccess) return KDA_ERR_CUDA;
+  kda::set_last_launch_count(launches);
+  return KDA_OK;
 }

@@ -5,16 +5,17 @@
 // "How it works"; paper.rainbus.top, section 核心方法).  fp32 accumulation,
 // one rounding to the output type.
 //
-// Visual part (the bulk of the work, bound by the fp32 FMA pipe): a CTA owns
-// 32 channels of one tensor (one per lane) and a tile of 4 rows x (4 runs) of
-// the grid, and slides through time.  Input planes (the tile plus a one-pixel
-// halo, zero outside the grid) are copied as they are by cp.async into a ring
-// of four shared-memory slots, three planes ahead of the one being computed.
-// Each plane is read from shared memory once: a thread keeps the partial sums
-// of the three output frames that plane feeds (t = f + pt - a for temporal tap
-// a) in registers, so every value it reads feeds up to 27 taps.  The frame
-// whose last tap arrived is written out and its registers start the frame
-// three ahead.
+// Visual part (the bulk of the work, bound by the fp32 FMA pipe): a CTA of two
+// warps owns 32 channels of one tensor (one per lane) and a tile of TH = 2 grid
+// rows x one run of RUN columns (13 on 52-wide grids, 16 on 64- and 256-wide
+// ones), and slides through time; eight CTAs are resident per SM.  Input planes
+// (the tile plus a one-pixel halo, zero outside the grid) are copied as they are
+// by cp.async into a ring of NSLOT = 3 shared-memory slots, two planes ahead of
+// the one being computed.  Each plane is read from shared memory once: a thread
+// owns one output row of the run and keeps the partial sums of the three output
+// frames that plane feeds (t = f + pt - a for temporal tap a) in registers, so
+// every value it reads feeds up to 27 taps.  The frame whose last tap arrived is
+// written out and its registers start the frame three ahead.
 //
 // Text part: a small kernel, one thread per (token, 8 channels).
 #include <cuda_fp16.h>

@@ -134,3 +134,90 @@ def test_host_side_rejections_launch_nothing(kda):
     assert bwd(reuse) == kda.KDA_ERR_INVALID_ARG
     assert kda.kda_bwd_workspace_bytes(p, torch.bfloat16) > kda.kda_workspace_bytes(p, torch.bfloat16)
     assert kda.kda_last_launch_count() == 0
+
+
+def test_chunk_length_rules(kda):
+    """chunk: 16, 32 or 64 where the CUDA-core scan runs (fp32; bf16 with d = 64); exactly 64 on the
+    bf16 tensor-core path (d = 128), whose blocks are two 64-token sub-chunks; 128 nowhere."""
+    for dt, d, chunk, want in [(1, 64, 16, kda.KDA_OK), (1, 128, 32, kda.KDA_OK), (0, 64, 32, kda.KDA_OK),
+                               (0, 128, 64, kda.KDA_OK), (0, 128, 32, kda.KDA_ERR_UNSUPPORTED),
+                               (0, 128, 16, kda.KDA_ERR_UNSUPPORTED), (0, 128, 128, kda.KDA_ERR_UNSUPPORTED),
+                               (1, 64, 128, kda.KDA_ERR_UNSUPPORTED), (0, 64, 128, kda.KDA_ERR_UNSUPPORTED)]:
+        p = _p(kda, d=d, chunk=chunk)
+        assert (kda.kda_workspace_bytes(p, dt) > 0) == (want == kda.KDA_OK), (dt, d, chunk)
+        if want != kda.KDA_OK:
+            assert _call_fwd(kda, p, dt=dt) == want, (dt, d, chunk)
+
+
+def test_selftest_entry_rejects_other_paths(kda):
+    """The bounded-wait self-test runs only on the tensor-core path and for stages 1 and 2; host-side
+    rejections launch nothing."""
+    lib = kda._lib
+    call = lambda pp, dt=0, stage=1, wait_us=100: lib.kda_selftest_wait_timeout(   # noqa: E731
+        ctypes.byref(pp), dt, 256, 256, 256, 256, 256, 256, 512, 1 << 40, stage, wait_us, None)
+    assert call(_p(kda, d=64)) == kda.KDA_ERR_UNSUPPORTED
+    assert call(_p(kda, d=128), dt=1) == kda.KDA_ERR_UNSUPPORTED
+    assert call(_p(kda, d=128), stage=0) == kda.KDA_ERR_INVALID_ARG
+    assert call(_p(kda, d=128), stage=3) == kda.KDA_ERR_INVALID_ARG
+    assert call(_p(kda, d=128), wait_us=0) == kda.KDA_ERR_INVALID_ARG
+    assert kda.kda_last_launch_count() == 0
+
+
+def test_binding_checks_tensors_before_the_call(kda):
+    """The C ABI sees bare addresses, so the binding checks every tensor against the problem (element
+    count, dtype, device, contiguity) and raises KdaError(KDA_ERR_INVALID_ARG) before anything reaches
+    the library: a buffer too short for the problem never becomes an out-of-bounds device access.  Host
+    tensors stand in everywhere, so the checks run without a GPU."""
+    B, H, d, L, grid = 1, 2, 64, 8, (1, 2, 4)
+    N = L + 8
+    p = kda.problem(B, H, d, L, grid)
+    z = lambda *shape, dtype=torch.float32: torch.zeros(*shape, dtype=dtype)   # noqa: E731
+    base = dict(q=z(B, N, H, d), k=z(B, N, H, d), v=z(B, N, H, d), log_alpha=z(B, N, H, d), beta=z(B, N, H),
+                o=z(B, N, H, d), w_text=z(3, H * d, 4), w_vis=z(3, H * d, 27), s0=z(B, H, d, d), sn=z(B, H, d, d),
+                qo=z(B, N, H, d), ko=z(B, N, H, d), vo=z(B, N, H, d), ws=z(4096, dtype=torch.uint8),
+                d_o=z(B, N, H, d), dq=z(B, N, H, d), dk=z(B, N, H, d), dv=z(B, N, H, d), dla=z(B, N, H, d),
+                dbeta=z(B, N, H), dwt=z(3, H * d, 4), dwv=z(3, H * d, 27), ds0=z(B, H, d, d),
+                status=z(1, dtype=torch.int32))
+    calls = {
+        "kda_fwd": (lambda a: kda.kda_fwd(p, a["q"], a["k"], a["v"], a["log_alpha"], a["beta"], a["w_text"],
+                                          a["w_vis"], a["o"], a["ws"], initial_state=a["s0"], final_state=a["sn"]),
+                    ("q", "k", "v", "log_alpha", "beta", "w_text", "w_vis", "o", "s0", "sn")),
+        "kda_chunk_fwd": (lambda a: kda.kda_chunk_fwd(p, a["q"], a["k"], a["v"], a["log_alpha"], a["beta"], a["o"],
+                                                      a["ws"], initial_state=a["s0"], final_state=a["sn"]),
+                          ("q", "k", "v", "log_alpha", "beta", "o", "s0", "sn")),
+        "kda_shortconv_fwd": (lambda a: kda.kda_shortconv_fwd(p, a["q"], a["k"], a["v"], a["w_text"], a["w_vis"],
+                                                              a["qo"], a["ko"], a["vo"]),
+                              ("q", "k", "v", "w_text", "w_vis", "qo", "ko", "vo")),
+        "kda_chunk_fwd_noalloc": (lambda a: kda.kda_chunk_fwd_noalloc(p, a["q"], a["k"], a["v"], a["log_alpha"],
+                                                                      a["beta"], a["o"], a["s0"], a["sn"],
+                                                                      a["status"]),
+                                  ("q", "k", "v", "log_alpha", "beta", "o", "s0", "sn")),
+        "kda_bwd": (lambda a: kda.kda_bwd(p, a["q"], a["k"], a["v"], a["log_alpha"], a["beta"], a["w_text"],
+                                          a["w_vis"], a["d_o"], a["dq"], a["dk"], a["dv"], a["dla"], a["dbeta"],
+                                          a["dwt"], a["dwv"], a["ws"], initial_state=a["s0"], d_initial_state=a["ds0"]),
+                    ("q", "d_o", "dq", "dk", "dv", "dla", "dbeta", "dwt", "dwv", "s0", "ds0")),
+    }
+    for where, (call, names) in calls.items():
+        for n in names:
+            bad = dict(base)
+            bad[n] = base[n].reshape(-1)[:-1]          # one element short
+            with pytest.raises(kda.KdaError) as e:
+                call(bad)
+            assert e.value.status == kda.KDA_ERR_INVALID_ARG and "elements" in str(e.value), (where, n)
+        n = "beta" if "beta" in names else ("dbeta" if "dbeta" in names else "qo")
+        bad = dict(base, **{n: base[n].to(torch.bfloat16)})     # wrong dtype for an fp32 problem
+        with pytest.raises(kda.KdaError, match="dtype"):
+            call(bad)
+        bad = dict(base, v=base["v"].transpose(1, 2))            # right size, not contiguous
+        if "v" in names:
+            with pytest.raises(kda.KdaError, match="contiguous"):
+                call(bad)
+        with pytest.raises(kda.KdaError, match="CUDA tensor"):  # right sizes, host memory
+            call(base)
+    # kda_fwd_host takes q, k, v, log_alpha, beta, o on the host and the rest on the device
+    host = lambda a: kda.kda_fwd_host(p, a["q"], a["k"], a["v"], a["log_alpha"], a["beta"], a["w_text"],   # noqa: E731
+                                      a["w_vis"], a["o"], a["ws"], 2)
+    with pytest.raises(kda.KdaError, match="elements"):
+        host(dict(base, log_alpha=base["log_alpha"][:, :-1].contiguous()))
+    with pytest.raises(kda.KdaError, match="(w_text|workspace) must be a CUDA tensor"):
+        host(base)

@@ -51,8 +51,36 @@ def test_noalloc_matches_chunk_fwd_on_two_calls():
         assert rc == kda.KDA_OK, kda.kda_status_str(rc)
         torch.cuda.synchronize()
         assert int(status.item()) == kda.KDA_OK
+        assert kda.kda_last_launch_count() == 2     # record kernel + state pass
         assert_parity(o.float().cpu().numpy(), ref_o.float().cpu().numpy(), "bf16", f"call {call} o")
         assert_parity(sn.cpu().numpy(), ref_s.cpu().numpy(), "bf16", f"call {call} state")
+        # both entry points run the same kernels on the same inputs: the results agree bit for bit
+        assert torch.equal(o, ref_o) and torch.equal(sn, ref_s)
+
+
+def test_noalloc_matches_the_oracle_without_a_status_word():
+    """The same entry point with device_status = NULL (conditions then go to a word inside the static
+    array), against the oracle's recurrence on the same bf16 values."""
+    import linear_attention_video_b200 as kda
+    import oracle
+    lib = kda._lib
+    B, N, H, d = 1, 700, 4, 128
+    p = kda.problem(B, H, d, N, (0, 0, 0))
+    q, k, v, la, beta = _inputs(B, N, H, d, 13)
+    s0 = torch.randn(B, H, d, d, device="cuda") * 0.05
+    o = torch.full((B, N, H, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    sn = torch.full((B, H, d, d), float("nan"), device="cuda")
+    rc = lib.kda_chunk_fwd_noalloc(ctypes.byref(p), kda.KDA_DT_BF16, q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                   la.data_ptr(), beta.data_ptr(), s0.data_ptr(), o.data_ptr(), sn.data_ptr(), None,
+                                   torch.cuda.current_stream().cuda_stream)
+    assert rc == kda.KDA_OK, kda.kda_status_str(rc)
+    torch.cuda.synchronize()
+    wide = lambda x: x.float().cpu().numpy().astype(np.float64)   # noqa: E731
+    for h in (0, 3):
+        ref, ref_s = oracle.scan(wide(q[:, :, h]), wide(k[:, :, h]), wide(v[:, :, h]), wide(la[:, :, h]),
+                                 wide(beta[:, :, h]), wide(s0[:, h]))
+        assert_parity(o[:, :, h].float().cpu().numpy(), ref, "bf16", f"head {h} o")
+        assert_parity(sn[:, h].cpu().numpy(), ref_s, "bf16", f"head {h} state")
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch():
