@@ -90,12 +90,6 @@ __device__ __forceinline__ void st_row32_h(uint8_t* panel, int row, int col0, co
 #pragma unroll
   for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4*>(panel + swz_off(row, col0 + 8 * c)) = pack8(v + 8 * c);
 }
-// 16 consecutive fp16 values at (row, col0..) of a swizzled panel -> fp32
-__device__ __forceinline__ void ld_row16_h(const uint8_t* panel, int row, int col0, float* v) {
-  unpack8(*reinterpret_cast<const uint4*>(panel + swz_off(row, col0)), v);
-  unpack8(*reinterpret_cast<const uint4*>(panel + swz_off(row, col0 + 8)), v + 8);
-}
-
 // 16 or 32 consecutive TMEM columns of this warp's lanes
 template <int N>
 __device__ __forceinline__ void tmem_ld_n(uint32_t taddr, float (&v)[N]) {
@@ -130,18 +124,21 @@ __device__ __forceinline__ bool wait_mma(uint64_t* bar, uint32_t& phase, uint32_
 // kda_tc_prep
 // ---------------------------------------------------------------------------
 // shared memory map (bytes from a 1024-aligned base)
-constexpr uint32_t OFF_KQ = 0;          // [128 rows][128] fp16: rows 0-63 K -> K Gamma (later W), 64-127 Q -> Q Gamma; later M_2
-constexpr uint32_t OFF_KN = 32768;      // [64][128] fp16: K~; staging of O'_1 and O''_2
-constexpr uint32_t OFF_VV = 49152;      // [64][128] fp16: V, then U~, then Q^_2
-constexpr uint32_t OFF_TT = 65536;      // [64][64] fp16: T   (TT and PP together: staging of R_1 and R_2)
+constexpr uint32_t OFF_KK = 0;          // [64][128] fp16: K Gamma, then W^T ([128 channels][64 tokens]); with QQ: M_2
+constexpr uint32_t OFF_QQ = 16384;      // [64][128] fp16: Q Gamma
+constexpr uint32_t OFF_KN = 32768;      // [64][128] fp16: K~, then Q^_2; staging of O'_1 and O''_2
+constexpr uint32_t OFF_VV = 49152;      // [64][128] fp16: V (TMA), then U~^T ([128 channels][64 tokens])
+constexpr uint32_t OFF_TT = 65536;      // [64][64] fp16: T, then the identity (TT and PP together: staging of R_1, R_2)
 constexpr uint32_t OFF_PP = 73728;      // [64][64] fp16: P
 constexpr uint32_t OFF_M1 = 81920;      // [128][128] fp16: M_1 (MN-major operand image)
 constexpr uint32_t OFF_B1 = 114688;     // [128][128] fp16: B_1 (MN-major operand image)
-// 72 KB used three ways in turn: the log alpha of a sub-chunk (TMA target, [64 tokens][128] fp32), the
-// operand tiles of the three tensor-core Gram levels, and A, X, Y of the blocked inverse
+// 72 KB used three ways in turn: the inputs of a sub-chunk (TMA targets: log alpha [64 tokens][128] fp32,
+// raw k and q at G_IN), the operand tiles of the Gram, and A, X, Y of the blocked inverse
 constexpr uint32_t OFF_G = 147456;
+constexpr uint32_t G_IN = 32768;        // raw k (rows 0-63) and q (rows 64-127): 2 panels [128][64] of 16 KB
 constexpr uint32_t G_ROW = 0;           // level tiles, rows: [64][128] fp16 per level (5, 4, 3), 16 KB apart
 constexpr uint32_t G_COL = 49152;       // level tiles, columns: [32][128] fp16 per level, 8 KB apart
+constexpr uint32_t G_DCOL = 32768;      // direct Gram: rows [128][128] at G_ROW, columns [64][128] here
 constexpr uint32_t G_AS = 0;            // fp32 [64][LDA]: A (strictly lower, beta applied)
 constexpr uint32_t G_XS = 17408;        // fp32 [64][LDXS]: (I + A)^{-1}
 constexpr uint32_t G_YS = 34816;        // fp32 [32][36]: merge scratch
@@ -154,11 +151,15 @@ static_assert(G_XS >= G_AS + 64 * LDA * 4 && G_YS >= G_XS + 64 * LDXS * 4 && G_Y
               "prep shared-memory map");
 static_assert(G_COL >= G_ROW + 3 * 16384 && G_COL + 3 * 8192 <= 73728, "prep shared-memory map");
 static_assert(PREP_SMEM <= 232448, "prep shared memory above the per-block limit");
-constexpr int LDY = 36;    // row stride of the merge scratch
+// direct Gram factorisation (e^{g_r - g_31} e^{g_31 - g_i}) only while every fp16 factor stays small:
+// the decay over each half of the sub-chunk at most kHalfRange nats, |k|, |q| at most kMagRange
+// (operands then stay below kMagRange e^kHalfRange = 25,800, inside fp16)
+constexpr float kHalfRange = 6.f;
+constexpr float kMagRange = 64.f;
 
 // TMEM columns
 constexpr int C_G = 0;                   // the three Gram levels, 32 columns each (M = 64 layout)
-constexpr int C_W = 64, C_U = 192;
+constexpr int C_W = 128, C_U = 192;      // W^T, U~^T: M = 128 (channels) x 64 tokens
 constexpr int C_MK = 0, C_BK = 128, C_PW = 256, C_PU = 384;
 
 // TMA descriptors of the [B][N][H][128] inputs, box [1][64 tokens][1][64 or 128 channels]
@@ -220,120 +221,125 @@ __device__ __forceinline__ void mma_tile_3xtf32(const float* A, int lda, const f
   for (int i = 0; i < 4; ++i) d[i] = (dl[0][i] + dl[1][i]) + (dh[0][i] + dh[1][i]);
 }
 
-// Blocked inverse X = (I + A)^{-1} of the unit lower-triangular 64x64 matrix,
-// A strictly lower in As, delivered as T = X Diag(beta) in fp16 (TT, one
-// swizzled K-major panel).  16x16 diagonal blocks by forward substitution, then
-// two doubling merges (X_21 = -X_22 A_21 X_11) at 32 and 64.  Every loop has a
-// fixed trip count; the zero blocks above the diagonal of X_11 and X_22 are
-// written here, the rest of the upper triangle is never read.
-// Step 1 (inverse_diag32) leaves the two diagonal 32x32 blocks of X in Xs and
-// writes every part of T but its lower-left block, so products over T's
-// columns 32-63 can start while step 2 (inverse_merge64) forms that block.
-__device__ void inverse_diag32(const float* As, float* Xs, float* Ys, uint8_t* TT, const float* beta) {
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  if (warp < 4 && lane < 16) {
-    // diagonal block `warp`, column `lane`: right-looking substitution
-    const int o = 16 * warp, l = lane;
-    float x[16];
-#pragma unroll
-    for (int r = 0; r < 16; ++r) x[r] = r == l ? 1.f : 0.f;
-    // row r: x[r] -= A[r][m] x[m] for m = 0 .. r-1 in that order, A's row read 4 wide
-#pragma unroll
-    for (int r = 1; r < 16; ++r) {
-      const float4* arow = reinterpret_cast<const float4*>(As + (o + r) * LDA + o);
-#pragma unroll
-      for (int q = 0; q < (r + 3) / 4; ++q) {
-        const float4 a4 = arow[q];
-        const float av[4] = {a4.x, a4.y, a4.z, a4.w};
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-          if (4 * q + u < r) x[r] -= av[u] * x[4 * q + u];
-      }
-    }
-#pragma unroll
-    for (int r = 0; r < 16; ++r) Xs[(o + r) * LDXS + o + l] = x[r];
-  } else if (warp >= 4) {
-    // zero blocks (0,1) and (2,3)
-    const int e = tid - 128, r = e >> 3, c = 2 * (e & 7);   // 16 rows x 8 column pairs
-    Xs[r * LDXS + 16 + c] = 0.f;
-    Xs[r * LDXS + 17 + c] = 0.f;
-    Xs[(32 + r) * LDXS + 48 + c] = 0.f;
-    Xs[(32 + r) * LDXS + 49 + c] = 0.f;
-  }
-  __syncthreads();
-  {
-    // 32-merges p = 0, 1: X[32p+16.., 32p..] = -D_{2p+1} (A_{2p+1,2p} D_{2p}); 2x1 outputs per thread
-    const int p = tid >> 7, e = tid & 127;
-    const int o = 32 * p, i0 = 2 * (e >> 4), j = e & 15;
-    float* Y = Ys + p * 16 * 17;
-    float y0 = 0.f, y1 = 0.f;
-#pragma unroll
-    for (int m = 0; m < 16; ++m) {
-      const float d = Xs[(o + m) * LDXS + o + j];
-      y0 += As[(o + 16 + i0) * LDA + o + m] * d;
-      y1 += As[(o + 17 + i0) * LDA + o + m] * d;
-    }
-    Y[i0 * 17 + j] = y0;
-    Y[(i0 + 1) * 17 + j] = y1;
-    __syncthreads();
-    float z0 = 0.f, z1 = 0.f;
-#pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      const float y = Y[k * 17 + j];
-      z0 += Xs[(o + 16 + i0) * LDXS + o + 16 + k] * y;
-      z1 += Xs[(o + 17 + i0) * LDXS + o + 16 + k] * y;
-    }
-    Xs[(o + 16 + i0) * LDXS + o + j] = -z0;
-    Xs[(o + 17 + i0) * LDXS + o + j] = -z1;
-  }
-  __syncthreads();
-  // T = X Diag(beta) for rows 0-31 (X_11, then zeros) and the X_22 block of rows 32-63
-  for (int e = tid; e < 384; e += 256) {
-    const int r = e < 256 ? e >> 3 : 32 + ((e - 256) >> 2);
-    const int c0 = e < 256 ? (e & 7) * 8 : 32 + ((e - 256) & 3) * 8;
-    float v[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int cj = c0 + j;
-      v[j] = (cj <= r && (r < 32) == (cj < 32)) ? Xs[r * LDXS + cj] * beta[cj] : 0.f;
-    }
-    *reinterpret_cast<uint4*>(TT + swz_off(r, c0)) = pack8(v);
-  }
-  fence_proxy_async();
+// Named barrier over `count` threads (a multiple of 32) on hardware barrier `id` (1..15).
+__device__ __forceinline__ void named_sync(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" :: "r"(id), "r"(count) : "memory");
 }
 
-// Step 2: X_21 = -X_22 (A_21 X_11) -> T rows 32-63, columns 0-31.  `between`
-// runs on every thread after the barrier that follows the first product; the
-// caller's next barrier publishes the block.
-template <typename F>
-__device__ __forceinline__ void inverse_merge64(const float* As, const float* Xs, float* Ys, uint8_t* TT,
-                                                const float* beta, F&& between) {
+// Blocked inverse X = (I + A)^{-1} of the unit lower-triangular 64x64 matrix, A strictly
+// lower in As, delivered as T = X Diag(beta) in fp16 (TT, one swizzled K-major panel).
+// Warps 0-3 compute; warps 4-7 write the zero blocks of T above the diagonal blocks.
+//   1. warp w: diagonal 16x16 block D_w by forward substitution (lane = column, lanes 0-15);
+//      lanes 16-31 of warps 0 and 2 zero the blocks of X above D_0 and D_2 that step 3 reads.
+//   2. pairs (0, 1) and (2, 3): the diagonal 32x32 blocks, X_10 = -D_1 (A_10 D_0); each warp of
+//      the pair one 8-column tile of both products.
+//   3. warps 0-3: X_21 = -X_22 (A_21 X_11) of the 64x64 matrix; warp w the 8-column tile w of
+//      both products (32 rows).
+// The products run on the warp-level tensor cores in tf32 with split operands (about fp32
+// accuracy).  A tile's partial product Y goes through warp-private shared memory: a column
+// tile of the result needs only the same column tile of Y, so steps 2 and 3 synchronise only
+// the warps that produce their inputs (named barriers 1-3).  The caller's next barrier
+// publishes T.
+__device__ void inverse64(const float* As, float* Xs, float* Ys, uint8_t* TT, const float* beta) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  {
-    // 64-merge: X[32.., 0..31] = -X_22 (A_21 X_11), two 32x32x32 products on the
-    // warp-level tensor cores (m16n8k8, tf32).  Each operand is split into a tf32
-    // high part and a tf32 remainder and the product is formed as hi*hi + hi*lo +
-    // lo*hi, which keeps it at about fp32 accuracy.  Warp w owns the 16x8 output
-    // tile (rows 16*(w>>2), columns 8*(w&3)).
-    const int g = lane >> 2, t4 = lane & 3;
-    const int tm = warp >> 2, tn = warp & 3;
-    float d[4];
-    // Y = A_21 X_11 -> Ys
-    mma_tile_3xtf32(As + (32 + 16 * tm) * LDA, LDA, Xs + 8 * tn, LDXS, 4, g, t4, d);
-    Ys[(16 * tm + g) * LDY + 8 * tn + 2 * t4] = d[0];
-    Ys[(16 * tm + g) * LDY + 8 * tn + 2 * t4 + 1] = d[1];
-    Ys[(16 * tm + g + 8) * LDY + 8 * tn + 2 * t4] = d[2];
-    Ys[(16 * tm + g + 8) * LDY + 8 * tn + 2 * t4 + 1] = d[3];
-    __syncthreads();
-    between();
-    // X_21 = -X_22 Y, times beta of its column, into T
-    mma_tile_3xtf32(Xs + (32 + 16 * tm) * LDXS + 32, LDXS, Ys + 8 * tn, LDY, 4, g, t4, d);
-    const int r0 = 32 + 16 * tm + g, c = 8 * tn + 2 * t4;
-    const float b0 = beta[c], b1 = beta[c + 1];
-    st_h2(TT + swz_off(r0, c), -d[0] * b0, -d[1] * b1);
-    st_h2(TT + swz_off(r0 + 8, c), -d[2] * b0, -d[3] * b1);
+  const int g = lane >> 2, t4 = lane & 3;
+  auto st_t = [&](int r, int c, float v0, float v1) {   // T[r][c], T[r][c + 1] (c even)
+    st_h2(TT + swz_off(r, c), v0 * beta[c], v1 * beta[c + 1]);
+  };
+  if (warp >= 4) {
+    // 8-column chunks of T above the diagonal blocks: rows 0-15 chunks 2-7, rows 16-31 chunks 4-7,
+    // rows 32-47 chunks 6-7
+    for (int e = tid - 128; e < 192; e += 128) {
+      int r, c8;
+      if (e < 96) { r = e / 6; c8 = 2 + e % 6; }
+      else if (e < 160) { r = 16 + (e - 96) / 4; c8 = 4 + (e - 96) % 4; }
+      else { r = 32 + (e - 160) / 2; c8 = 6 + (e - 160) % 2; }
+      *reinterpret_cast<uint4*>(TT + swz_off(r, 8 * c8)) = make_uint4(0u, 0u, 0u, 0u);
+    }
     fence_proxy_async();
+    return;
   }
+  float* Yw = Ys + warp * 256;   // warp-private scratch, [16 or 32 rows][8]
+  {
+    // 1. diagonal block `warp`
+    const int o = 16 * warp;
+    if (lane < 16) {
+      const int l = lane;
+      float x[16];
+#pragma unroll
+      for (int r = 0; r < 16; ++r) x[r] = r == l ? 1.f : 0.f;
+      // row r: x[r] -= A[r][m] x[m] for m = 0 .. r-1, A's row read 4 wide
+#pragma unroll
+      for (int r = 1; r < 16; ++r) {
+        const float4* arow = reinterpret_cast<const float4*>(As + (o + r) * LDA + o);
+#pragma unroll
+        for (int q = 0; q < (r + 3) / 4; ++q) {
+          const float4 a4 = arow[q];
+          const float av[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            if (4 * q + u < r) x[r] -= av[u] * x[4 * q + u];
+        }
+      }
+      const float bl = beta[o + l];
+#pragma unroll
+      for (int r = 0; r < 16; ++r) {
+        Xs[(o + r) * LDXS + o + l] = x[r];
+        *reinterpret_cast<__half*>(TT + swz_off(o + r, o + l)) = __float2half_rn(x[r] * bl);
+      }
+    } else if ((warp & 1) == 0) {
+      // zero block of X above D_0 (rows 0-15, columns 16-31) or D_2 (rows 32-47, columns 48-63)
+      const int l = lane - 16;
+#pragma unroll
+      for (int r = 0; r < 16; ++r) Xs[(o + r) * LDXS + o + 16 + l] = 0.f;
+    }
+  }
+  named_sync(1 + (warp >> 1), 64);   // D_0, D_1 (or D_2, D_3) in place
+  {
+    // 2. 32x32 merge of pair p, column tile nt: X_10[:, nt] = -D_1 (A_10 D_0[:, nt])
+    const int p = warp >> 1, nt = warp & 1, o = 32 * p;
+    float d[4];
+    mma_tile_3xtf32(As + (o + 16) * LDA + o, LDA, Xs + o * LDXS + o + 8 * nt, LDXS, 2, g, t4, d);
+    Yw[g * 8 + 2 * t4] = d[0];
+    Yw[g * 8 + 2 * t4 + 1] = d[1];
+    Yw[(g + 8) * 8 + 2 * t4] = d[2];
+    Yw[(g + 8) * 8 + 2 * t4 + 1] = d[3];
+    __syncwarp();
+    mma_tile_3xtf32(Xs + (o + 16) * LDXS + o + 16, LDXS, Yw, 8, 2, g, t4, d);
+    const int r0 = o + 16 + g, c = o + 8 * nt + 2 * t4;
+    Xs[r0 * LDXS + c] = -d[0];
+    Xs[r0 * LDXS + c + 1] = -d[1];
+    Xs[(r0 + 8) * LDXS + c] = -d[2];
+    Xs[(r0 + 8) * LDXS + c + 1] = -d[3];
+    st_t(r0, c, -d[0], -d[1]);
+    st_t(r0 + 8, c, -d[2], -d[3]);
+  }
+  named_sync(3, 128);   // X_11 and X_22 in place
+  {
+    // 3. 64x64 merge, column tile `warp` of X_21 = -X_22 (A_21 X_11), rows 32-63
+    const int c0 = 8 * warp;
+    float d0[4], d1[4];
+    mma_tile_3xtf32(As + 32 * LDA, LDA, Xs + c0, LDXS, 4, g, t4, d0);   // rows 32-47 of A_21 X_11
+    mma_tile_3xtf32(As + 48 * LDA, LDA, Xs + c0, LDXS, 4, g, t4, d1);   // rows 48-63
+    __syncwarp();   // step 2's reads of the scratch are done
+    Yw[g * 8 + 2 * t4] = d0[0];
+    Yw[g * 8 + 2 * t4 + 1] = d0[1];
+    Yw[(g + 8) * 8 + 2 * t4] = d0[2];
+    Yw[(g + 8) * 8 + 2 * t4 + 1] = d0[3];
+    Yw[(g + 16) * 8 + 2 * t4] = d1[0];
+    Yw[(g + 16) * 8 + 2 * t4 + 1] = d1[1];
+    Yw[(g + 24) * 8 + 2 * t4] = d1[2];
+    Yw[(g + 24) * 8 + 2 * t4 + 1] = d1[3];
+    __syncwarp();
+    mma_tile_3xtf32(Xs + 32 * LDXS + 32, LDXS, Yw, 8, 4, g, t4, d0);   // X_22 rows 32-47 times Y
+    mma_tile_3xtf32(Xs + 48 * LDXS + 32, LDXS, Yw, 8, 4, g, t4, d1);   // rows 48-63
+    const int c = c0 + 2 * t4;
+    st_t(32 + g, c, -d0[0], -d0[1]);
+    st_t(40 + g, c, -d0[2], -d0[3]);
+    st_t(48 + g, c, -d1[0], -d1[1]);
+    st_t(56 + g, c, -d1[2], -d1[3]);
+  }
+  fence_proxy_async();
 }
 
 // 4 consecutive activations (8 bytes, fp16 or bf16) -> fp32, and 4 fp32 -> fp16 (8 bytes)
@@ -351,6 +357,28 @@ __device__ __forceinline__ void ld_act4(const uint8_t* p, float* v, __nv_bfloat1
 }
 __device__ __forceinline__ void st_h4(uint8_t* p, float a, float b, float c, float d) {
   *reinterpret_cast<uint2*>(p) = make_uint2(pack_h2(a, b), pack_h2(c, d));
+}
+
+// Two fp32 values in one 64-bit register pair, for the packed fp32x2 multiply of sm_100.
+__device__ __forceinline__ uint64_t f2pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ float2 f2unpack(uint64_t v) {
+  float a, b;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+  return make_float2(a, b);
+}
+__device__ __forceinline__ uint64_t f2mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+// 4 fp16 at p from two packed fp32 pairs
+__device__ __forceinline__ void st_h4x2(uint8_t* p, uint64_t lo, uint64_t hi) {
+  const float2 a = f2unpack(lo), b = f2unpack(hi);
+  st_h4(p, a.x, a.y, b.x, b.y);
 }
 
 // Position of token t (0..63) among the 32 tokens of its role at Gram level l: the
@@ -387,7 +415,8 @@ template <typename TIn>
 __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_constant__ PrepMaps mp) {
   extern __shared__ uint8_t dyn[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn) + 1023) & ~uintptr_t(1023));
-  uint8_t* KQ = sm + OFF_KQ;
+  uint8_t* KK = sm + OFF_KK;
+  uint8_t* QQ = sm + OFF_QQ;
   uint8_t* KN = sm + OFF_KN;
   uint8_t* VV = sm + OFF_VV;
   uint8_t* TT = sm + OFF_TT;
@@ -401,12 +430,13 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
   float* Ys = reinterpret_cast<float*>(G + G_YS);
   float* beta_s = reinterpret_cast<float*>(sm + OFF_MISC);  // 64
   float* egl = beta_s + 64;                                 // 128: Gamma_l = e^{g_l}
-  float* tot = egl + 128;                                   // [8 octets][128]: decay over each octet
+  float* tot = egl + 128;                                   // [8 octets][128]: log decay over each octet
   float* gscr = tot + 8 * 128;                              // [8 octets][64]: Gram pairs inside each octet
-  uint64_t* bar = reinterpret_cast<uint64_t*>(gscr + 8 * 64);   // [0] MMA, [1] k/q/v tiles, [2] log alpha
-  uint64_t* kqv_bar = bar + 1;
-  uint64_t* la_bar = bar + 2;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(gscr + 8 * 64);   // [0] MMA, [1] v tile, [2] log alpha, k, q
+  uint64_t* v_bar = bar + 1;
+  uint64_t* in_bar = bar + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 4);
+  uint64_t* bar2 = bar + 5;                                      // second MMA group of a round
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int sub = warp & 3, chalf = warp >> 2;
@@ -415,17 +445,18 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
   if (warp == 0) { tmem_alloc(tmem_slot, 512); tmem_relinquish(); }
   if (tid == 0) {
     mbar_init(bar, 1);
-    mbar_init(kqv_bar, 1);
-    mbar_init(la_bar, 1);
+    mbar_init(v_bar, 1);
+    mbar_init(in_bar, 1);
+    mbar_init(bar2, 1);
     fence_mbar_init();
   }
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
   const uint32_t tm = *tmem_slot;
-  uint32_t phase = 0, kqv_phase = 0, la_phase = 0;
+  uint32_t phase = 0, phase2 = 0, v_phase = 0, in_phase = 0;
   bool alive = true;
-  bool la_inflight = false, kqv_inflight = false;   // thread 0's view: TMA loads not yet waited for
+  bool in_inflight = false, v_inflight = false;   // thread 0: TMA loads not yet waited for
   // batch item, head and first token of the sub-chunk this CTA processes after (u, s_)
   auto next_sub = [&](int u, int s_, int& nb_, int& nh_, int& nt0_) -> bool {
     const int nu = s_ == 0 ? u : u + (int)gridDim.x;
@@ -436,47 +467,59 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
     nt0_ = blk_ * BLK + (s_ ^ 1) * SUB;
     return true;
   };
-  auto load_beta = [&](int b_, int h_, int t_) -> float {   // 0 past the sequence end
-    return t_ < a.N ? __bfloat162float(static_cast<const __nv_bfloat16*>(a.beta)[((int64_t)b_ * a.N + t_) * a.H + h_])
-                    : 0.f;
+  // beta as raw bf16 bits (0 past the sequence end), converted where it is used, so the load is
+  // waited for one sub-chunk later
+  auto load_beta = [&](int b_, int h_, int t_) -> uint32_t {
+    return t_ < a.N ? (uint32_t)static_cast<const uint16_t*>(a.beta)[((int64_t)b_ * a.N + t_) * a.H + h_] : 0u;
   };
-  float beta_next = 0.f;
+  uint32_t beta_next = 0u;
   if (tid < SUB && (int)blockIdx.x < a.n_units) {
     const int bh_ = (int)blockIdx.x % a.BH;   // unit blockIdx.x: block blockIdx.x / BH, sub-chunk 0
     beta_next = load_beta(bh_ / a.H, bh_ % a.H, ((int)blockIdx.x / a.BH) * BLK + tid);
   }
-  // k, q, v of the sub-chunk starting at token t0_ -> KQ rows 0-63 / 64-127 and VV (thread 0)
-  auto issue_kqv = [&](int b_, int h_, int t0_) {
-    mbar_arrive_expect_tx(kqv_bar, 6 * 8192);
+  // v of the sub-chunk starting at token t0_ -> VV (thread 0)
+  auto issue_v = [&](int b_, int h_, int t0_) {
+    mbar_arrive_expect_tx(v_bar, 2 * 8192);
+#pragma unroll
+    for (int pnl = 0; pnl < 2; ++pnl) tma_load_4d(VV + pnl * 8192, &mp.v, 64 * pnl, h_, t0_, b_, v_bar);
+  };
+  bool v_early = false;   // thread 0: the sub-chunk's v is already on its way
+  // log alpha, k and q of sub-chunk s_ of unit u -> G (thread 0)
+  auto issue_in = [&](int u, int s_) {
+    const int blk_ = u / a.BH, bh_ = u - blk_ * a.BH;
+    const int b_ = bh_ / a.H, h_ = bh_ - b_ * a.H, t0_ = blk_ * BLK + s_ * SUB;
+    mbar_arrive_expect_tx(in_bar, 32768 + 4 * 8192);
+    tma_load_4d(G, &mp.la, 0, h_, t0_, b_, in_bar);
 #pragma unroll
     for (int pnl = 0; pnl < 2; ++pnl) {
-      tma_load_4d(KQ + pnl * 16384, &mp.k, 64 * pnl, h_, t0_, b_, kqv_bar);
-      tma_load_4d(KQ + pnl * 16384 + 8192, &mp.q, 64 * pnl, h_, t0_, b_, kqv_bar);
-      tma_load_4d(VV + pnl * 8192, &mp.v, 64 * pnl, h_, t0_, b_, kqv_bar);
+      tma_load_4d(G + G_IN + pnl * 16384, &mp.k, 64 * pnl, h_, t0_, b_, in_bar);
+      tma_load_4d(G + G_IN + pnl * 16384 + 8192, &mp.q, 64 * pnl, h_, t0_, b_, in_bar);
     }
   };
-  bool kqv_early = false;   // thread 0: the next sub-chunk's tiles are already on their way
-  auto issue_la = [&](int u, int s_) {   // log alpha of sub-chunk s_ of unit u -> G (thread 0)
-    const int blk_ = u / a.BH, bh_ = u - blk_ * a.BH;
-    const int b_ = bh_ / a.H, h_ = bh_ - b_ * a.H;
-    mbar_arrive_expect_tx(la_bar, 32768);
-    tma_load_4d(G, &mp.la, 0, h_, blk_ * BLK + s_ * SUB, b_, la_bar);
-  };
-  if (tid == 0 && (int)blockIdx.x < a.n_units) {
-    issue_la(blockIdx.x, 0);
-    la_inflight = true;
+  // self-test of the bounded waits: the first CTA never issues its first inputs, so its wait gives up
+  if (tid == 0 && (int)blockIdx.x < a.n_units && !(a.fault == 1 && blockIdx.x == 0)) {
+    issue_in(blockIdx.x, 0);
+    in_inflight = true;
   }
 
   // operand descriptors of the fixed tiles (stepped along K by kstep / mstep)
-  const uint64_t dKQk = kdesc0(smem_u32(KQ)), dKQm = mdesc0(smem_u32(KQ), 16384);
+  const uint64_t dKQk = kdesc0(smem_u32(KK));                             // M_2: [128][128], panels 16 KB
+  const uint64_t dKKm = mdesc0(smem_u32(KK), 8192), dQQm = mdesc0(smem_u32(QQ), 8192);   // K Gamma, Q Gamma
+  const uint64_t dKKk = kdesc0(smem_u32(KK)), dVVk = kdesc0(smem_u32(VV));               // W^T, U~^T
   const uint64_t dKNm = mdesc0(smem_u32(KN), 8192);
-  const uint64_t dVVk = kdesc0(smem_u32(VV)), dVVm = mdesc0(smem_u32(VV), 8192);
+  const uint64_t dVVm = mdesc0(smem_u32(VV), 8192);
   const uint64_t dTTk = kdesc0(smem_u32(TT)), dPPk = kdesc0(smem_u32(PP));
   const uint64_t dM1m = mdesc0(smem_u32(M1), 16384), dB1m = mdesc0(smem_u32(B1), 16384);
   const uint64_t dGrow = kdesc0(smem_u32(G + G_ROW)), dGcol = kdesc0(smem_u32(G + G_COL));
+  const uint64_t dGdcol = kdesc0(smem_u32(G + G_DCOL));
+  const uint64_t dKNk = kdesc0(smem_u32(KN));
   const uint32_t id_gram = idesc_f16(64, 32, false, false);
+  const uint32_t id_direct = idesc_f16(128, 64, false, false);
   const uint32_t id_64x128_kmn = idesc_f16(64, 128, false, true);
-  const uint32_t id_128x128_mnmn = idesc_f16(128, 128, true, true);
+  const uint32_t id_64x128_kk = idesc_f16(64, 128, false, false);
+  const uint32_t id_64x128_kk_neg = idesc_f16(64, 128, false, false, true);   // D (+)= -A B
+  const uint32_t id_128x64_mnk = idesc_f16(128, 64, true, false);
+  const uint32_t id_128x128_mnk = idesc_f16(128, 128, true, false);
   const uint32_t id_128x128_kmn = idesc_f16(128, 128, false, true);
 
   // front-pass role of this thread: octet fo (tokens 8 fo .. 8 fo + 7), channels 4 lane .. 4 lane + 3
@@ -494,103 +537,145 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
     for (int s = 0; s < 2; ++s) {
       const int64_t t0 = (int64_t)blk * BLK + s * SUB;
       // ---------------- inputs ----------------
-      // k -> KQ rows 0-63, q -> KQ rows 64-127, v -> VV: 128-byte-swizzled operand panels
-      // written by TMA; rows past the sequence end read as zero (log alpha too: alpha = 1)
+      // log alpha, k, q in G (issued during the previous sub-chunk, after its inverse), v in VV
+      // (issued once the previous sub-chunk's products were done): TMA, rows past the sequence end
+      // read as zero (log alpha too: alpha = 1)
       if (tid == 0 && alive) {
-        // self-test of the bounded waits: a load that is never issued, so the wait below gives up
-        const bool skip = a.fault == 1 && blockIdx.x == 0 && unit == 0 && s == 0;
-        if (!kqv_early && !skip) issue_kqv(b, h, (int)t0);   // else issued while the previous unit finished
-        kqv_early = false;
-        kqv_inflight = !skip;
-      }
-      if (tid == 128 && alive) {
-        // the next sub-chunk's tiles and log alpha into L2 meanwhile
-        int nb_, nh_, nt0_;
-        if (next_sub(unit, s, nb_, nh_, nt0_)) {
-#pragma unroll
-          for (int pnl = 0; pnl < 2; ++pnl) {
-            tma_prefetch_4d(&mp.k, 64 * pnl, nh_, nt0_, nb_);
-            tma_prefetch_4d(&mp.q, 64 * pnl, nh_, nt0_, nb_);
-            tma_prefetch_4d(&mp.v, 64 * pnl, nh_, nt0_, nb_);
-          }
-          tma_prefetch_4d(&mp.la, 0, nh_, nt0_, nb_);
-        }
+        if (!v_early) issue_v(b, h, (int)t0);
+        v_early = false;
+        v_inflight = true;
       }
       if (tid < SUB) {
         // beta of this sub-chunk was read one sub-chunk ago; read the next one now
-        beta_s[tid] = beta_next;
+        beta_s[tid] = __uint_as_float(beta_next << 16);
         int nb_, nh_, nt0_;
-        beta_next = next_sub(unit, s, nb_, nh_, nt0_) ? load_beta(nb_, nh_, nt0_ + tid) : 0.f;
+        beta_next = next_sub(unit, s, nb_, nh_, nt0_) ? load_beta(nb_, nh_, nt0_ + tid) : 0u;
       }
       {
-        const bool ok_la = wait_tma(la_bar, la_phase, a.status, alive, a.wait_ns);
-        const bool ok_kqv = wait_tma(kqv_bar, kqv_phase, a.status, ok_la, a.wait_ns);
-        if (tid == 0) {
-          if (ok_la) la_inflight = false;
-          if (ok_kqv) kqv_inflight = false;
-        }
-        alive = __syncthreads_and(ok_kqv);
+        const bool ok_in = wait_tma(in_bar, in_phase, a.status, alive, a.wait_ns);
+        if (tid == 0 && ok_in) in_inflight = false;
+        alive = __syncthreads_and(ok_in);
       }
       // ---------------- front pass ----------------
-      // Every factor is a product of gates alpha = e^{log alpha} <= 1, so none can overflow:
-      //   Gamma_t = prod_{u<=t} alpha_u,  e^{g_l - g_t} = prod_{u>t} alpha_u,
-      // and the Gram levels' factors, prefix products from a split point (rows) and suffix
-      // products up to it (columns).  Thread: octet fo, four channels; within the octet the
-      // prefix (pre) and suffix (suf) products are its own, across octets it uses the octet totals.
-      float al[8][4], kx[8][4], qx[8][4];
+      // Thread: octet fo (tokens 8 fo .. 8 fo + 7), four channels.  Per-token factors referenced
+      // to the sub-chunk start, all <= 1: Gamma_t = e^{g_t} (rows of K Gamma, Q Gamma) and
+      // e^{g_l - g_t} (rows of K~).  The pairwise decays e^{g_r - g_i} of A and P take one of two
+      // factorisations, chosen for the whole sub-chunk:
+      //   direct: e^{g_r - g_31} e^{g_31 - g_i}, one tensor-core product, when every factor and
+      //     operand stays far inside fp16 (the decay over each half of the sub-chunk at most
+      //     kHalfRange nats in every channel, |k|, |q| <= kMagRange);
+      //   levels: split points between r and i (see the file header), for any gates.
+      float al[8][4], ls[8][4], kx[8][4], qx[8][4];
+      bool big = false;
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         const int tok = 8 * fo + j;
         const float4 x = *reinterpret_cast<const float4*>(LA + tok * D + 4 * lane);
-        al[j][0] = __expf(x.x); al[j][1] = __expf(x.y); al[j][2] = __expf(x.z); al[j][3] = __expf(x.w);
-        ld_act4(KQ + fpnl * 16384 + swz_off(tok, fpc), kx[j], (TIn*)nullptr);
-        ld_act4(KQ + fpnl * 16384 + swz_off(64 + tok, fpc), qx[j], (TIn*)nullptr);
-        if constexpr (!kIsHalf<TIn>) {   // caller's bf16 v -> the fp16 operand image, in place
-          uint8_t* pv = VV + fpnl * 8192 + swz_off(tok, fpc);
-          float v4[4];
-          ld_act4(pv, v4, (TIn*)nullptr);
-          st_h4(pv, v4[0], v4[1], v4[2], v4[3]);
+        const float xv[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          al[j][c] = __expf(xv[c]);
+          ls[j][c] = (j ? ls[j - 1][c] : 0.f) + xv[c];   // log decay from the octet start
+        }
+        ld_act4(G + G_IN + fpnl * 16384 + swz_off(tok, fpc), kx[j], (TIn*)nullptr);
+        ld_act4(G + G_IN + fpnl * 16384 + swz_off(64 + tok, fpc), qx[j], (TIn*)nullptr);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) big |= fabsf(kx[j][c]) > kMagRange || fabsf(qx[j][c]) > kMagRange;
+      }
+      *reinterpret_cast<float4*>(tot + fo * D + 4 * lane) = make_float4(ls[7][0], ls[7][1], ls[7][2], ls[7][3]);
+      if (tid == 0) bulk_wait_read();   // staged record stores have read KN, TT and PP
+      __syncthreads();                  // octet log totals published; log alpha, k, q read (G is free)
+      // log decay before this octet, over each half, and the choice of factorisation
+      float gb[4], h0[4], h1[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) gb[c] = h0[c] = h1[c] = 0.f;
+#pragma unroll
+      for (int o = 0; o < 8; ++o) {
+        const float4 t4 = *reinterpret_cast<const float4*>(tot + o * D + 4 * lane);
+        const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          if (o < fo) gb[c] += tv[c];
+          if (o < 4) h0[c] += tv[c]; else h1[c] += tv[c];
         }
       }
-      float pre[8][4], suf[8][4];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        pre[0][c] = al[0][c];
+      for (int c = 0; c < 4; ++c) big |= h0[c] < -kHalfRange || h1[c] < -kHalfRange;
+      const bool levels = __syncthreads_or(big);
+      if (fo == 0)   // Gamma_l = e^{g_l}
+        *reinterpret_cast<float4*>(egl + 4 * lane) =
+            make_float4(__expf(h0[0] + h1[0]), __expf(h0[1] + h1[1]), __expf(h0[2] + h1[2]), __expf(h0[3] + h1[3]));
+      if (!levels) {
+        // direct: x = g_t - g_31, within +-kHalfRange; Gamma_t = e^{g_31} e^x, e^{g_l - g_t} = e^{g_l - g_31} e^{-x}.
+        // e^x runs forward through the octet from its first token (times alpha), e^{-x} backward from
+        // its last; channel pairs go through the packed fp32x2 multiply.
+        uint64_t ep[8][2], en[8][2], e31[2], el31[2];
 #pragma unroll
-        for (int j = 1; j < 8; ++j) pre[j][c] = pre[j - 1][c] * al[j][c];
-        suf[7][c] = 1.f;
+        for (int pc = 0; pc < 2; ++pc) {
+          const int c0 = 2 * pc, c1 = 2 * pc + 1;
+          e31[pc] = f2pack(__expf(h0[c0]), __expf(h0[c1]));
+          el31[pc] = f2pack(__expf(h1[c0]), __expf(h1[c1]));
+          ep[0][pc] = f2pack(__expf(gb[c0] + ls[0][c0] - h0[c0]), __expf(gb[c1] + ls[0][c1] - h0[c1]));
+          en[7][pc] = f2pack(__expf(h0[c0] - gb[c0] - ls[7][c0]), __expf(h0[c1] - gb[c1] - ls[7][c1]));
 #pragma unroll
-        for (int j = 6; j >= 0; --j) suf[j][c] = suf[j + 1][c] * al[j + 1][c];
-      }
-      *reinterpret_cast<float4*>(tot + fo * D + 4 * lane) = make_float4(pre[7][0], pre[7][1], pre[7][2], pre[7][3]);
-      if (tid == 0) bulk_wait_read();   // staged record stores have read KN, TT and PP
-      __syncthreads();                  // octet totals published; log alpha read (G is free)
-      {
-        // outer factors from the octet totals (fo is uniform over the warp)
-        float gb[4], ka[4], f5[4], f4[4];
+          for (int j = 1; j < 8; ++j) ep[j][pc] = f2mul(ep[j - 1][pc], f2pack(al[j][c0], al[j][c1]));
 #pragma unroll
-        for (int c = 0; c < 4; ++c) gb[c] = ka[c] = f5[c] = f4[c] = 1.f;
+          for (int j = 6; j >= 0; --j) en[j][pc] = f2mul(en[j + 1][pc], f2pack(al[j + 1][c0], al[j + 1][c1]));
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int tok = 8 * fo + j;
+          const uint32_t o128 = swz_off(tok, fpc), oq = swz_off(64 + tok, fpc);
+          uint64_t kg[2], qg[2], kt[2], rk[2], rq[2], ck[2];
+#pragma unroll
+          for (int pc = 0; pc < 2; ++pc) {
+            const uint64_t k2 = f2pack(kx[j][2 * pc], kx[j][2 * pc + 1]);
+            const uint64_t q2 = f2pack(qx[j][2 * pc], qx[j][2 * pc + 1]);
+            const uint64_t gam = f2mul(e31[pc], ep[j][pc]), ktf = f2mul(el31[pc], en[j][pc]);
+            kg[pc] = f2mul(k2, gam);
+            qg[pc] = f2mul(q2, gam);
+            kt[pc] = f2mul(k2, ktf);
+            rk[pc] = f2mul(k2, ep[j][pc]);
+            rq[pc] = f2mul(q2, ep[j][pc]);
+            ck[pc] = f2mul(k2, en[j][pc]);
+          }
+          st_h4x2(KK + fpnl * 8192 + o128, kg[0], kg[1]);
+          st_h4x2(QQ + fpnl * 8192 + o128, qg[0], qg[1]);
+          st_h4x2(KN + fpnl * 8192 + o128, kt[0], kt[1]);
+          // Gram operands: rows [K e^x; Q e^x] (M = 128), columns K e^{-x} (N = 64)
+          uint8_t* rt = G + G_ROW + fpnl * 16384;
+          st_h4x2(rt + o128, rk[0], rk[1]);
+          st_h4x2(rt + oq, rq[0], rq[1]);
+          st_h4x2(G + G_DCOL + fpnl * 8192 + o128, ck[0], ck[1]);
+        }
+      } else {
+        // levels: prefix (pre) and suffix (suf) products of the gates within the octet, and across
+        // octets the octet totals
+        float pre[8][4], suf[8][4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          pre[0][c] = al[0][c];
+#pragma unroll
+          for (int j = 1; j < 8; ++j) pre[j][c] = pre[j - 1][c] * al[j][c];
+          suf[7][c] = 1.f;
+#pragma unroll
+          for (int j = 6; j >= 0; --j) suf[j][c] = suf[j + 1][c] * al[j + 1][c];
+        }
+        float gp[4], ka[4], f5[4], f4[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) gp[c] = ka[c] = f5[c] = f4[c] = 1.f;
 #pragma unroll
         for (int o = 0; o < 8; ++o) {
           const float4 t4 = *reinterpret_cast<const float4*>(tot + o * D + 4 * lane);
-          const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
+          const float tv[4] = {__expf(t4.x), __expf(t4.y), __expf(t4.z), __expf(t4.w)};
           const bool in5 = (fo & 4) ? (o >= 4 && o < fo) : (o > fo && o < 4);
           const bool in4 = (fo & 2) ? ((fo & 1) && o == fo - 1) : (!(fo & 1) && o == fo + 1);
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
-            if (o < fo) gb[c] *= tv[c];
+            if (o < fo) gp[c] *= tv[c];
             if (o > fo) ka[c] *= tv[c];
             if (in5) f5[c] *= tv[c];
             if (in4) f4[c] *= tv[c];
-          }
-          if (fo == 0) {
-            // Gamma_l: the decay over the whole sub-chunk
-            if (o == 0) *reinterpret_cast<float4*>(egl + 4 * lane) = t4;
-            else {
-              float4 e = *reinterpret_cast<const float4*>(egl + 4 * lane);
-              e.x *= t4.x; e.y *= t4.y; e.z *= t4.z; e.w *= t4.w;
-              *reinterpret_cast<float4*>(egl + 4 * lane) = e;
-            }
           }
         }
 #pragma unroll
@@ -599,7 +684,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
           float g[4], kt[4], r3[4], r4[4], r5[4];
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
-            g[c] = gb[c] * pre[j][c];
+            g[c] = gp[c] * pre[j][c];
             kt[c] = suf[j][c] * ka[c];
             r3[c] = (fo & 1) ? pre[j][c] : suf[j][c];
             r4[c] = (fo & 2) ? f4[c] * pre[j][c] : suf[j][c] * f4[c];
@@ -608,8 +693,8 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
           const float* kk = kx[j];
           const float* qq = qx[j];
           const uint32_t o128 = swz_off(tok, fpc);
-          st_h4(KQ + fpnl * 16384 + o128, kk[0] * g[0], kk[1] * g[1], kk[2] * g[2], kk[3] * g[3]);
-          st_h4(KQ + fpnl * 16384 + swz_off(64 + tok, fpc), qq[0] * g[0], qq[1] * g[1], qq[2] * g[2], qq[3] * g[3]);
+          st_h4(KK + fpnl * 8192 + o128, kk[0] * g[0], kk[1] * g[1], kk[2] * g[2], kk[3] * g[3]);
+          st_h4(QQ + fpnl * 8192 + o128, qq[0] * g[0], qq[1] * g[1], qq[2] * g[2], qq[3] * g[3]);
           st_h4(KN + fpnl * 8192 + o128, kk[0] * kt[0], kk[1] * kt[1], kk[2] * kt[2], kk[3] * kt[3]);
           // Gram levels 5, 4, 3 (tile li = 5 - level): role from bit `level` of the token
 #pragma unroll
@@ -631,23 +716,30 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
       fence_proxy_async();
       fence_before_sync();
       __syncthreads();
-      // ---------------- Gram levels on the tensor cores ----------------
-      // Level l pairs the 32 tokens with bit l set (rows: k and q, scaled by the decay from
-      // the level's split point) with the 32 with bit l clear (columns: k, scaled by the
-      // decay up to it): entry (r, i) is valid when r and i share their bits above l, and
-      // then equals sum_c k_r (or q_r) k_i e^{g_r - g_i}.  Levels 5, 4, 3 cover every pair
-      // in different octets; pairs inside an octet follow on the CUDA cores.
+      // ---------------- Gram on the tensor cores ----------------
+      // direct: [K e^x; Q e^x] (K e^{-x})^T, one M = 128 product: A in rows 0-63, P in rows 64-127.
+      // levels: level l pairs the 32 tokens with bit l set (rows: k and q, scaled by the decay
+      // from the level's split point) with the 32 with bit l clear (columns: k, scaled by the
+      // decay up to it): entry (r, i) is valid when r and i share their bits above l, and then
+      // equals sum_c k_r (or q_r) k_i e^{g_r - g_i}.  Levels 5, 4, 3 cover every pair in different
+      // octets; pairs inside an octet follow on the CUDA cores.
       if (tid == 0 && alive) {
         fence_after_sync();
-#pragma unroll
-        for (int li = 0; li < 3; ++li)
+        if (!levels) {
 #pragma unroll
           for (int k16 = 0; k16 < 8; ++k16)
-            mma_ss(tmem_at(tm, 0, C_G + 32 * li), dGrow + ((uint32_t)li * 16384 >> 4) + kstep(k16, 8192),
-                   dGcol + ((uint32_t)li * 8192 >> 4) + kstep(k16, 4096), id_gram, k16 > 0);
+            mma_ss(tmem_at(tm, 0, C_G), dGrow + kstep(k16, 16384), dGdcol + kstep(k16, 8192), id_direct, k16 > 0);
+        } else {
+#pragma unroll
+          for (int li = 0; li < 3; ++li)
+#pragma unroll
+            for (int k16 = 0; k16 < 8; ++k16)
+              mma_ss(tmem_at(tm, 0, C_G + 32 * li), dGrow + ((uint32_t)li * 16384 >> 4) + kstep(k16, 8192),
+                     dGcol + ((uint32_t)li * 8192 >> 4) + kstep(k16, 4096), id_gram, k16 > 0);
+        }
         mma_commit(bar);
       }
-      {
+      if (levels) {
         // pairs inside the octet: e^{g_r - g_i} = prod_{u=i+1..r} alpha_u as a running product
         float acc[64];
 #pragma unroll
@@ -671,7 +763,27 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
       }
       alive = __syncthreads_and(wait_mma(bar, phase, a.status, alive, a.wait_ns));
       fence_after_sync();
-      {
+      if (!levels) {
+        // A rows (TMEM lanes 0-63) -> As (beta, strict lower); P rows (lanes 64-127) -> PP (lower)
+        const int row = 32 * sub + lane;
+        const int col0 = 32 * chalf;
+        float v[32];
+        tmem_ld32(tmem_at(tm, 32 * sub, C_G + col0), v);
+        tmem_wait_ld();
+        if (sub < 2) {
+          const float bt = beta_s[row];
+#pragma unroll
+          for (int j = 0; j < 32; j += 4)
+            *reinterpret_cast<float4*>(As + row * LDA + col0 + j) =
+                make_float4(col0 + j < row ? bt * v[j] : 0.f, col0 + j + 1 < row ? bt * v[j + 1] : 0.f,
+                            col0 + j + 2 < row ? bt * v[j + 2] : 0.f, col0 + j + 3 < row ? bt * v[j + 3] : 0.f);
+        } else {
+          const int r = row - 64;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = (col0 + j <= r) ? v[j] : 0.f;
+          st_row32_h(PP, r, col0, v);
+        }
+      } else {
         // Gram levels -> A (fp32, beta applied, As) and P (fp16, PP).  M = 64 accumulator layout:
         // row m at lane 32 (m / 16) + m % 16; rows 0-31 are k rows (A), 32-63 q rows (P).
         const int qd = warp & 3;
@@ -721,147 +833,112 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
           for (int c8 = o + 1; c8 < 8; ++c8) *reinterpret_cast<uint4*>(PP + swz_off(r, 8 * c8)) = make_uint4(0, 0, 0, 0);
         }
       }
-      fence_proxy_async();
-      fence_before_sync();
-      __syncthreads();
-      // T = (I + A)^{-1} Diag(beta) -> TT; W = T K Gamma, U~ = T V over T's columns 32-63 first,
-      // issued as soon as they are written, then over columns 0-31
-      inverse_diag32(As, Xs, Ys, TT, beta_s);
-      inverse_merge64(As, Xs, Ys, TT, beta_s, [&]() {
-        if (tid == 0 && alive) {
-          fence_after_sync();
+      {
+        // v of this sub-chunk (issued a sub-chunk ago); a caller's bf16 v becomes the fp16 operand in place
+        const bool ok_v = wait_tma(v_bar, v_phase, a.status, alive, a.wait_ns);
+        if (tid == 0 && ok_v) v_inflight = false;
+        if constexpr (!kIsHalf<TIn>) {
+          for (int e = tid; e < 1024; e += 256) {
+            const int r = e >> 4, ch = (e & 15) * 8;
+            uint4* p = reinterpret_cast<uint4*>(VV + (ch >> 6) * 8192 + swz_off(r, ch & 63));
+            const uint4 u = *p;
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+            float f[8];
 #pragma unroll
-          for (int k16 = 2; k16 < 4; ++k16) {
-            const uint64_t ad = dTTk + kstep(k16, 8192);
-            mma_ss(tmem_at(tm, 0, C_W), ad, dKQm + mstep(k16), id_64x128_kmn, k16 > 2);
-            mma_ss(tmem_at(tm, 0, C_U), ad, dVVm + mstep(k16), id_64x128_kmn, k16 > 2);
+            for (int i = 0; i < 4; ++i) {
+              const float2 t2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+              f[2 * i] = t2.x;
+              f[2 * i + 1] = t2.y;
+            }
+            *p = pack8(f);
           }
         }
-      });
-      __syncthreads();
-      if (tid == 0 && alive) {
+        fence_proxy_async();
+        fence_before_sync();
+        alive = __syncthreads_and(ok_v);
+      }
+      // T = (I + A)^{-1} Diag(beta) -> TT; then W^T = (K Gamma)^T T^T and U~^T = V^T T^T (M = 128
+      // channels, N = 64 tokens)
+      inverse64(As, Xs, Ys, TT, beta_s);
+      fence_before_sync();
+      __syncthreads();   // T published
+      // two issuing threads in different warps: thread 0 the W^T products (commit on bar), thread 32
+      // the U~^T products (commit on bar2)
+      if ((tid == 0 || tid == 32) && alive) {
         fence_after_sync();
+        const uint32_t dmine = tid == 0 ? C_W : C_U;
+        const uint64_t amine = tid == 0 ? dKKm : dVVm;
 #pragma unroll
-        for (int k16 = 0; k16 < 2; ++k16) {
-          const uint64_t ad = dTTk + kstep(k16, 8192);
-          mma_ss(tmem_at(tm, 0, C_W), ad, dKQm + mstep(k16), id_64x128_kmn, 1);
-          mma_ss(tmem_at(tm, 0, C_U), ad, dVVm + mstep(k16), id_64x128_kmn, 1);
-        }
-        mma_commit(bar);
-        // A, X, Y consumed: G takes the log alpha of this CTA's next sub-chunk
+        for (int k16 = 0; k16 < 4; ++k16)
+          mma_ss(tmem_at(tm, 0, dmine), amine + mstep(k16), dTTk + kstep(k16, 8192), id_128x64_mnk, k16 > 0);
+        mma_commit(tid == 0 ? bar : bar2);
+      }
+      if (tid == 0 && alive) {
+        // A, X, Y consumed: G takes the log alpha, k and q of this CTA's next sub-chunk
         const int nunit = s == 0 ? unit : unit + (int)gridDim.x;
         if (nunit < a.n_units) {
-          issue_la(nunit, s ^ 1);
-          la_inflight = true;
+          issue_in(nunit, s ^ 1);
+          in_inflight = true;
         }
       }
-      alive = __syncthreads_and(wait_mma(bar, phase, a.status, alive, a.wait_ns));
-      fence_after_sync();
-      // W -> KQ rows 0-63, U~ -> VV (fp16); M=64 accumulator layout: rows 16*sub + lane (lane < 16)
       {
-        const int r = 16 * sub + lane;
-        for (int cb = 0; cb < 2; ++cb) {
-          const int col0 = 64 * chalf + 32 * cb;
-          float w[32], u[32];
-          tmem_ld32(tmem_at(tm, 32 * sub, C_W + col0), w);
-          tmem_ld32(tmem_at(tm, 32 * sub, C_U + col0), u);
-          tmem_wait_ld();
-          if (lane < 16) {
-            st_row32_h(KQ + chalf * 16384, r, col0 & 63, w);
-            st_row32_h(VV + chalf * 8192, r, col0 & 63, u);
-          }
+        const bool w1 = wait_mma(bar, phase, a.status, alive, a.wait_ns);
+        alive = __syncthreads_and(wait_mma(bar2, phase2, a.status, w1, a.wait_ns));
+      }
+      fence_after_sync();
+      // W^T -> KK, U~^T -> VV: [128 channels][64 tokens] fp16, K-major B operands of the next round
+      {
+        const int c = 32 * sub + lane, t0c = 32 * chalf;
+        float w[32], u[32];
+        tmem_ld32(tmem_at(tm, 32 * sub, C_W + t0c), w);
+        tmem_ld32(tmem_at(tm, 32 * sub, C_U + t0c), u);
+        tmem_wait_ld();
+        st_row32_h(KK, c, t0c, w);
+        st_row32_h(VV, c, t0c, u);
+        // T consumed: TT becomes the 64x64 identity, the A operand that adds Q Gamma to -P W
+        for (int e = tid; e < 512; e += 256) {
+          const int ir = e >> 3, c8 = e & 7;
+          float v8[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) v8[j] = (8 * c8 + j == ir) ? 1.f : 0.f;
+          *reinterpret_cast<uint4*>(TT + swz_off(ir, 8 * c8)) = pack8(v8);
         }
       }
       fence_proxy_async();
       fence_before_sync();
       __syncthreads();
-      // ---------------- K~^T W, K~^T U~, P W, P U~ ----------------
-      if (tid == 0 && alive) {
+      // ---------------- K~^T W, K~^T U~, then Q Gamma - P W, P U~ ----------------
+      // R = Q Gamma - P W comes out of the tensor core: D = (-P) W + I (Q Gamma), so Q Gamma is
+      // consumed there and KK, QQ, VV are free once the round completes
+      if (tid == 0 && alive) {   // first group: thread 0
         fence_after_sync();
 #pragma unroll
         for (int k16 = 0; k16 < 4; ++k16) {
           const uint64_t kt = dKNm + mstep(k16);
-          const uint64_t wd = dKQm + mstep(k16);
-          const uint64_t ud = dVVm + mstep(k16);
-          const uint64_t pd = dPPk + kstep(k16, 8192);
-          mma_ss(tmem_at(tm, 0, C_MK), kt, wd, id_128x128_mnmn, k16 > 0);
-          mma_ss(tmem_at(tm, 0, C_BK), kt, ud, id_128x128_mnmn, k16 > 0);
-          mma_ss(tmem_at(tm, 0, C_PW), pd, wd, id_64x128_kmn, k16 > 0);
-          mma_ss(tmem_at(tm, 0, C_PU), pd, ud, id_64x128_kmn, k16 > 0);
+          mma_ss(tmem_at(tm, 0, C_MK), kt, dKKk + kstep(k16, 16384), id_128x128_mnk, k16 > 0);
+          mma_ss(tmem_at(tm, 0, C_BK), kt, dVVk + kstep(k16, 16384), id_128x128_mnk, k16 > 0);
         }
         mma_commit(bar);
+      }
+      if (tid == 32 && alive) {  // second group: thread 32
+        fence_after_sync();
+#pragma unroll
+        for (int k16 = 0; k16 < 4; ++k16) {
+          const uint64_t pd = dPPk + kstep(k16, 8192);
+          mma_ss(tmem_at(tm, 0, C_PW), pd, dKKk + kstep(k16, 16384), id_64x128_kk_neg, k16 > 0);
+          mma_ss(tmem_at(tm, 0, C_PW), dTTk + kstep(k16, 8192), dQQm + mstep(k16), id_64x128_kmn, 1);
+          mma_ss(tmem_at(tm, 0, C_PU), pd, dVVk + kstep(k16, 16384), id_64x128_kk, k16 > 0);
+        }
+        mma_commit(bar2);
       }
       if (tid == 0) bulk_wait_read();   // staged records read: their tiles may be rewritten
       alive = __syncthreads_and(wait_mma(bar, phase, a.status, alive, a.wait_ns));
       fence_after_sync();
       const int row = 32 * sub + lane;        // M=128 layout row
       const int r64 = 16 * sub + lane;        // M=64 layout row (lane < 16)
-      if (s == 0) {
-        // M_1 = Diag(Gamma_l) - K~^T W -> M1 tile;  B_1 -> B1 tile
-        for (int cb = 0; cb < 2; ++cb) {
-          const int col0 = 64 * chalf + 32 * cb;
-          float m[32], bv[32];
-          tmem_ld32(tmem_at(tm, 32 * sub, C_MK + col0), m);
-          tmem_ld32(tmem_at(tm, 32 * sub, C_BK + col0), bv);
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) m[j] = (row == col0 + j ? egl[row] : 0.f) - m[j];
-          st_row32_h(M1 + chalf * 16384, row, col0 & 63, m);
-          st_row32_h(B1 + chalf * 16384, row, col0 & 63, bv);
-        }
-        // R_1 = Q Gamma - P W and O'_1, staged for the record (R rows 0-63, O'' rows 0-63)
-        uint8_t* stR = TT;                                  // [panel][64 rows][128 B], swizzled (TT and PP)
-        uint4* stO = reinterpret_cast<uint4*>(KN);          // [c/8][64 rows][8]
-        for (int cb = 0; cb < 2; ++cb) {
-          const int col0 = 64 * chalf + 32 * cb;
-          float pw[32], pu[32];
-          tmem_ld32(tmem_at(tm, 32 * sub, C_PW + col0), pw);
-          tmem_ld32(tmem_at(tm, 32 * sub, C_PU + col0), pu);
-          tmem_wait_ld();
-          if (lane < 16) {
-            float qg[32];
-            ld_row16_h(KQ + chalf * 16384, 64 + r64, col0 & 63, qg);
-            ld_row16_h(KQ + chalf * 16384, 64 + r64, (col0 & 63) + 16, qg + 16);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) qg[j] -= pw[j];
-            st_row32_h(stR + chalf * 8192, r64, col0 & 63, qg);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) stO[((col0 >> 3) + i) * 64 + r64] = pack8(pu + 8 * i);
-          }
-        }
-        fence_proxy_async();
-        fence_before_sync();
-        __syncthreads();
-        if (tid == 0) {
-          // KQ (Q Gamma read above) and VV are free: sub-chunk 1's tiles first, then the stores
-          if (alive) {
-            issue_kqv(b, h, (int)t0 + SUB);
-            kqv_early = true;
-            kqv_inflight = true;
-          }
-          bulk_s2g(gR, stR, 8192);
-          bulk_s2g(gR + 16384, stR + 8192, 8192);
-          bulk_s2g(gO, stO, 16384);
-          bulk_commit();
-        }
-      } else {
-        // Q^_2 = Q Gamma - P W -> VV region (U~ no longer needed)
-        for (int cb = 0; cb < 2; ++cb) {
-          const int col0 = 64 * chalf + 32 * cb;
-          float pw[32];
-          tmem_ld32(tmem_at(tm, 32 * sub, C_PW + col0), pw);
-          tmem_wait_ld();
-          if (lane < 16) {
-            float qg[32];
-            ld_row16_h(KQ + chalf * 16384, 64 + r64, col0 & 63, qg);
-            ld_row16_h(KQ + chalf * 16384, 64 + r64, (col0 & 63) + 16, qg + 16);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) qg[j] -= pw[j];
-            st_row32_h(VV + chalf * 8192, r64, col0 & 63, qg);
-          }
-        }
-        __syncthreads();
-        // M_2 -> KQ region (A operand, K-major, 2 panels of 16 KB)
+      // M_s = Diag(Gamma_l) - K~^T W: M_1 -> M1 tile and B_1 -> B1 tile while the second group runs;
+      // M_2 -> KK, QQ (combine A operand) once the second group no longer reads W^T and Q Gamma there
+      auto m_epilogue = [&](uint8_t* dst, bool with_b) {
         for (int cb = 0; cb < 2; ++cb) {
           const int col0 = 64 * chalf + 32 * cb;
           float m[32];
@@ -869,40 +946,93 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
           tmem_wait_ld();
 #pragma unroll
           for (int j = 0; j < 32; ++j) m[j] = (row == col0 + j ? egl[row] : 0.f) - m[j];
-          st_row32_h(KQ + chalf * 16384, row, col0 & 63, m);
+          st_row32_h(dst + chalf * 16384, row, col0 & 63, m);
+          if (with_b) {
+            float bv[32];
+            tmem_ld32(tmem_at(tm, 32 * sub, C_BK + col0), bv);
+            tmem_wait_ld();
+            st_row32_h(B1 + chalf * 16384, row, col0 & 63, bv);
+          }
+        }
+      };
+      if (s == 0) m_epilogue(M1, true);
+      alive = alive && wait_mma(bar2, phase2, a.status, alive, a.wait_ns);
+      fence_after_sync();
+      if (tid == 0 && alive) {
+        // U~^T (VV) consumed: the next sub-chunk's v may land now
+        int nb_, nh_, nt0_;
+        if (next_sub(unit, s, nb_, nh_, nt0_)) {
+          issue_v(nb_, nh_, nt0_);
+          v_early = true;
+          v_inflight = true;
+        }
+      }
+      if (s == 0) {
+        // R_1 = Q Gamma - P W and O'_1, staged for the record (R rows 0-63, O'' rows 0-63)
+        uint8_t* stR = TT;                                  // [panel][64 rows][128 B], swizzled (TT and PP)
+        uint4* stO = reinterpret_cast<uint4*>(KN);          // [c/8][64 rows][8]
+        for (int cb = 0; cb < 2; ++cb) {
+          const int col0 = 64 * chalf + 32 * cb;
+          float rr[32], pu[32];
+          tmem_ld32(tmem_at(tm, 32 * sub, C_PW + col0), rr);
+          tmem_ld32(tmem_at(tm, 32 * sub, C_PU + col0), pu);
+          tmem_wait_ld();
+          if (lane < 16) {
+            st_row32_h(stR + chalf * 8192, r64, col0 & 63, rr);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) stO[((col0 >> 3) + i) * 64 + r64] = pack8(pu + 8 * i);
+          }
         }
         fence_proxy_async();
         fence_before_sync();
-        __syncthreads();
+        alive = __syncthreads_and(alive);
+        if (tid == 0) {
+          bulk_s2g(gR, stR, 8192);
+          bulk_s2g(gR + 16384, stR + 8192, 8192);
+          bulk_s2g(gO, stO, 16384);
+          bulk_commit();
+        }
+      } else {
+        m_epilogue(KK, false);
+        // Q^_2 = Q Gamma - P W -> KN (K~ no longer needed; K-major A operand, 2 panels of 8 KB)
+        for (int cb = 0; cb < 2; ++cb) {
+          const int col0 = 64 * chalf + 32 * cb;
+          float rr[32];
+          tmem_ld32(tmem_at(tm, 32 * sub, C_PW + col0), rr);
+          tmem_wait_ld();
+          if (lane < 16) st_row32_h(KN + chalf * 8192, r64, col0 & 63, rr);
+        }
+        fence_proxy_async();
+        fence_before_sync();
+        alive = __syncthreads_and(alive);
         // ---------------- combine ----------------
-        if (tid == 0 && alive) {
+        if ((tid == 0 || tid == 32) && alive) {   // thread 0: M, B (bar); thread 32: R_2, O''_2 (bar2)
           fence_after_sync();
           const uint32_t id_q = idesc_f16(64, 128, false, true);
+          if (tid == 0) {
 #pragma unroll
-          for (int k16 = 0; k16 < 8; ++k16) {
-            const uint64_t m2 = dKQk + kstep(k16, 16384);
-            const uint64_t q2 = dVVk + kstep(k16, 8192);
-            const uint64_t m1 = dM1m + mstep(k16);
-            const uint64_t b1 = dB1m + mstep(k16);
-            mma_ss(tmem_at(tm, 0, C_MK), m2, m1, id_128x128_kmn, k16 > 0);   // M = M_2 M_1
-            mma_ss(tmem_at(tm, 0, C_BK), m2, b1, id_128x128_kmn, 1);         // B = B_2 + M_2 B_1
-            mma_ss(tmem_at(tm, 0, C_PW), q2, m1, id_q, k16 > 0);             // R_2 = Q^_2 M_1
-            mma_ss(tmem_at(tm, 0, C_PU), q2, b1, id_q, 1);                   // O''_2 = O'_2 + Q^_2 B_1
+            for (int k16 = 0; k16 < 8; ++k16) {
+              const uint64_t m2 = dKQk + kstep(k16, 16384);
+              mma_ss(tmem_at(tm, 0, C_MK), m2, dM1m + mstep(k16), id_128x128_kmn, k16 > 0);   // M = M_2 M_1
+              mma_ss(tmem_at(tm, 0, C_BK), m2, dB1m + mstep(k16), id_128x128_kmn, 1);         // B = B_2 + M_2 B_1
+            }
+            mma_commit(bar);
+          } else {
+#pragma unroll
+            for (int k16 = 0; k16 < 8; ++k16) {
+              const uint64_t q2 = dKNk + kstep(k16, 8192);
+              mma_ss(tmem_at(tm, 0, C_PW), q2, dM1m + mstep(k16), id_q, k16 > 0);             // R_2 = Q^_2 M_1
+              mma_ss(tmem_at(tm, 0, C_PU), q2, dB1m + mstep(k16), id_q, 1);                   // O''_2 = O'_2 + Q^_2 B_1
+            }
+            mma_commit(bar2);
           }
-          mma_commit(bar);
         }
         if (tid == 0) bulk_wait_read();   // staged records read: their tiles may be rewritten
-        alive = __syncthreads_and(wait_mma(bar, phase, a.status, alive, a.wait_ns));
-        fence_after_sync();
-        if (tid == 0 && alive) {
-          // KQ and VV are free now: start the next unit's tiles before this unit's stores
-          int nb_, nh_, nt0_;
-          if (next_sub(unit, 1, nb_, nh_, nt0_)) {
-            issue_kqv(nb_, nh_, nt0_);
-            kqv_early = true;
-            kqv_inflight = true;
-          }
+        {
+          const bool w1 = wait_mma(bar, phase, a.status, alive, a.wait_ns);
+          alive = __syncthreads_and(wait_mma(bar2, phase2, a.status, w1, a.wait_ns));
         }
+        fence_after_sync();
         // records staged in tiles the combine products no longer read:
         //   M -> M1 region, B -> B1 region, R_2 -> TT/PP region, O''_2 -> KN region
         uint8_t* stR = TT;                               // [panel][64 rows][128 B], swizzled
@@ -950,8 +1080,8 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
   }
   if (tid == 0) {
     // loads still in flight after a timeout land before the CTA exits
-    if (la_inflight) mbar_wait(la_bar, la_phase, 100000000ull);
-    if (kqv_inflight) mbar_wait(kqv_bar, kqv_phase, 100000000ull);
+    if (in_inflight) mbar_wait(in_bar, in_phase, 100000000ull);
+    if (v_inflight) mbar_wait(v_bar, v_phase, 100000000ull);
     bulk_wait_all();
   }
   fence_before_sync();
