@@ -52,8 +52,8 @@ constexpr int D = 128;            // d_k = d_v
 // Record per (batch item, head, block), all fp16:
 //   M   K-major operand image: 2 panels [128 rows][64 cols]            32 KB
 //   B   [c/8][row a][8]  (16-byte units)                               32 KB
-//   R   K-major operand image: 2 panels [128 rows][64 cols]            32 KB
-//   O'' [row half][c/8][row r % 64][8]  (16-byte units)                32 KB
+//   R   MN-major operand image: 2 token panels [128 channels][64 tokens]   32 KB
+//   O'' [token half][128 channels][64 tokens], 128-byte-swizzled rows   32 KB
 constexpr size_t kMOff = 0, kBOff = 32768, kROff = 65536, kOOff = 98304;
 constexpr size_t kBlockBytes = 131072;
 
@@ -124,10 +124,12 @@ __device__ __forceinline__ bool wait_mma(uint64_t* bar, uint32_t& phase, uint32_
 // kda_tc_prep
 // ---------------------------------------------------------------------------
 // shared memory map (bytes from a 1024-aligned base)
-constexpr uint32_t OFF_KK = 0;          // [64][128] fp16: K Gamma, then W^T ([128 channels][64 tokens]); with QQ: M_2
-constexpr uint32_t OFF_QQ = 16384;      // [64][128] fp16: Q Gamma
-constexpr uint32_t OFF_KN = 32768;      // [64][128] fp16: K~, then Q^_2; staging of O'_1 and O''_2
-constexpr uint32_t OFF_VV = 49152;      // [64][128] fp16: V (TMA), then U~^T ([128 channels][64 tokens])
+// KK and VV adjacent: W^T and U~^T form one [256][64] K-major operand (N = 256 products);
+// QQ and KN adjacent: M_2 ([128][128], two 16 KB panels) for the combine
+constexpr uint32_t OFF_KK = 0;          // [64][128] fp16: K Gamma, then W^T ([128 channels][64 tokens]), then -Q^_2
+constexpr uint32_t OFF_VV = 16384;      // [64][128] fp16: V (TMA), then U~^T ([128 channels][64 tokens])
+constexpr uint32_t OFF_QQ = 32768;      // [64][128] fp16: Q Gamma; with KN: M_2
+constexpr uint32_t OFF_KN = 49152;      // [64][128] fp16: K~; staging of O'_1 and O''_2
 constexpr uint32_t OFF_TT = 65536;      // [64][64] fp16: T, then the identity (TT and PP together: staging of R_1, R_2)
 constexpr uint32_t OFF_PP = 73728;      // [64][64] fp16: P
 constexpr uint32_t OFF_M1 = 81920;      // [128][128] fp16: M_1 (MN-major operand image)
@@ -160,7 +162,8 @@ constexpr float kMagRange = 64.f;
 // TMEM columns
 constexpr int C_G = 0;                   // the three Gram levels, 32 columns each (M = 64 layout)
 constexpr int C_W = 128, C_U = 192;      // W^T, U~^T: M = 128 (channels) x 64 tokens
-constexpr int C_MK = 0, C_BK = 128, C_PW = 256, C_PU = 384;
+constexpr int C_MK = 0, C_BK = 128;        // M = 128 x 128 each
+constexpr int C_RT = 256, C_OT = 320;      // R^T, O'^T (and the combine's R_2^T, O''_2^T): M = 128 x 64
 
 // TMA descriptors of the [B][N][H][128] inputs, box [1][64 tokens][1][64 or 128 channels]
 struct PrepMaps {
@@ -467,15 +470,19 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
     nt0_ = blk_ * BLK + (s_ ^ 1) * SUB;
     return true;
   };
-  // beta as raw bf16 bits (0 past the sequence end), converted where it is used, so the load is
-  // waited for one sub-chunk later
+  // beta as raw bf16 bits: loaded unconditionally from a clamped index and masked where it is
+  // used, one sub-chunk later, so nothing waits for the load meanwhile
   auto load_beta = [&](int b_, int h_, int t_) -> uint32_t {
-    return t_ < a.N ? (uint32_t)static_cast<const uint16_t*>(a.beta)[((int64_t)b_ * a.N + t_) * a.H + h_] : 0u;
+    const int64_t tc = t_ < a.N ? t_ : a.N - 1;
+    return (uint32_t)static_cast<const uint16_t*>(a.beta)[((int64_t)b_ * a.N + tc) * a.H + h_];
   };
   uint32_t beta_next = 0u;
+  bool beta_ok = false;
   if (tid < SUB && (int)blockIdx.x < a.n_units) {
     const int bh_ = (int)blockIdx.x % a.BH;   // unit blockIdx.x: block blockIdx.x / BH, sub-chunk 0
-    beta_next = load_beta(bh_ / a.H, bh_ % a.H, ((int)blockIdx.x / a.BH) * BLK + tid);
+    const int t_ = ((int)blockIdx.x / a.BH) * BLK + tid;
+    beta_next = load_beta(bh_ / a.H, bh_ % a.H, t_);
+    beta_ok = t_ < a.N;
   }
   // v of the sub-chunk starting at token t0_ -> VV (thread 0)
   auto issue_v = [&](int b_, int h_, int t0_) {
@@ -503,23 +510,24 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
   }
 
   // operand descriptors of the fixed tiles (stepped along K by kstep / mstep)
-  const uint64_t dKQk = kdesc0(smem_u32(KK));                             // M_2: [128][128], panels 16 KB
+  const uint64_t dM2k = kdesc0(smem_u32(QQ));                             // M_2: [128][128], panels 16 KB
   const uint64_t dKKm = mdesc0(smem_u32(KK), 8192), dQQm = mdesc0(smem_u32(QQ), 8192);   // K Gamma, Q Gamma
-  const uint64_t dKKk = kdesc0(smem_u32(KK)), dVVk = kdesc0(smem_u32(VV));               // W^T, U~^T
+  const uint64_t dWUk = kdesc0(smem_u32(KK));                             // [W^T; U~^T]: [256][64]
   const uint64_t dKNm = mdesc0(smem_u32(KN), 8192);
   const uint64_t dVVm = mdesc0(smem_u32(VV), 8192);
   const uint64_t dTTk = kdesc0(smem_u32(TT)), dPPk = kdesc0(smem_u32(PP));
   const uint64_t dM1m = mdesc0(smem_u32(M1), 16384), dB1m = mdesc0(smem_u32(B1), 16384);
   const uint64_t dGrow = kdesc0(smem_u32(G + G_ROW)), dGcol = kdesc0(smem_u32(G + G_COL));
   const uint64_t dGdcol = kdesc0(smem_u32(G + G_DCOL));
-  const uint64_t dKNk = kdesc0(smem_u32(KN));
+  const uint64_t dQ2m = mdesc0(smem_u32(KK), 16384);                      // Q^_2^T: [128 channels][64 tokens]
+  const uint64_t dUk = kdesc0(smem_u32(VV));                              // U~^T
   const uint32_t id_gram = idesc_f16(64, 32, false, false);
   const uint32_t id_direct = idesc_f16(128, 64, false, false);
-  const uint32_t id_64x128_kmn = idesc_f16(64, 128, false, true);
-  const uint32_t id_64x128_kk = idesc_f16(64, 128, false, false);
-  const uint32_t id_64x128_kk_neg = idesc_f16(64, 128, false, false, true);   // D (+)= -A B
+  const uint32_t id_128x64_kk = idesc_f16(128, 64, false, false);
+  const uint32_t id_128x64_kk_neg = idesc_f16(128, 64, false, false, true);   // D (+)= -A B
+  const uint32_t id_128x64_mnmn = idesc_f16(128, 64, true, true);
   const uint32_t id_128x64_mnk = idesc_f16(128, 64, true, false);
-  const uint32_t id_128x128_mnk = idesc_f16(128, 128, true, false);
+  const uint32_t id_128x256_mnk = idesc_f16(128, 256, true, false);
   const uint32_t id_128x128_kmn = idesc_f16(128, 128, false, true);
 
   // front-pass role of this thread: octet fo (tokens 8 fo .. 8 fo + 7), channels 4 lane .. 4 lane + 3
@@ -547,9 +555,11 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
       }
       if (tid < SUB) {
         // beta of this sub-chunk was read one sub-chunk ago; read the next one now
-        beta_s[tid] = __uint_as_float(beta_next << 16);
-        int nb_, nh_, nt0_;
-        beta_next = next_sub(unit, s, nb_, nh_, nt0_) ? load_beta(nb_, nh_, nt0_ + tid) : 0u;
+        beta_s[tid] = beta_ok ? __uint_as_float(beta_next << 16) : 0.f;
+        int nb_ = b, nh_ = h, nt0_ = (int)t0;
+        const bool more = next_sub(unit, s, nb_, nh_, nt0_);
+        beta_ok = more && nt0_ + tid < a.N;
+        beta_next = load_beta(more ? nb_ : b, more ? nh_ : h, more ? nt0_ + tid : (int)t0);
       }
       {
         const bool ok_in = wait_tma(in_bar, in_phase, a.status, alive, a.wait_ns);
@@ -583,7 +593,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
         for (int c = 0; c < 4; ++c) big |= fabsf(kx[j][c]) > kMagRange || fabsf(qx[j][c]) > kMagRange;
       }
       *reinterpret_cast<float4*>(tot + fo * D + 4 * lane) = make_float4(ls[7][0], ls[7][1], ls[7][2], ls[7][3]);
-      if (tid == 0) bulk_wait_read();   // staged record stores have read KN, TT and PP
+      if (tid == 0) bulk_wait_read_but1();   // the staged record store from KN has read it
       __syncthreads();                  // octet log totals published; log alpha, k, q read (G is free)
       // log decay before this octet, over each half, and the choice of factorisation
       float gb[4], h0[4], h1[4];
@@ -761,6 +771,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
         warp_reduce_scatter64(acc, lane);
         *reinterpret_cast<float2*>(gscr + fo * 64 + 2 * lane) = make_float2(acc[0], acc[1]);
       }
+      if (tid == 0) bulk_wait_read();   // every staged record store has read TT and PP
       alive = __syncthreads_and(wait_mma(bar, phase, a.status, alive, a.wait_ns));
       fence_after_sync();
       if (!levels) {
@@ -907,35 +918,34 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
       fence_proxy_async();
       fence_before_sync();
       __syncthreads();
-      // ---------------- K~^T W, K~^T U~, then Q Gamma - P W, P U~ ----------------
-      // R = Q Gamma - P W comes out of the tensor core: D = (-P) W + I (Q Gamma), so Q Gamma is
-      // consumed there and KK, QQ, VV are free once the round completes
+      // ---------------- K~^T [W | U~], then R^T = (Q Gamma)^T - W^T P^T and O'^T = U~^T P^T ----------------
+      // [MK | BK] = K~^T [W | U~] is one N = 256 product over [W^T; U~^T].  R and O' are formed
+      // transposed (M = 128 channels, N = 64 tokens; the identity tile adds (Q Gamma)^T), so Q Gamma
+      // is consumed on the tensor core and KK, VV, QQ are free once the round completes.
       if (tid == 0 && alive) {   // first group: thread 0
         fence_after_sync();
 #pragma unroll
-        for (int k16 = 0; k16 < 4; ++k16) {
-          const uint64_t kt = dKNm + mstep(k16);
-          mma_ss(tmem_at(tm, 0, C_MK), kt, dKKk + kstep(k16, 16384), id_128x128_mnk, k16 > 0);
-          mma_ss(tmem_at(tm, 0, C_BK), kt, dVVk + kstep(k16, 16384), id_128x128_mnk, k16 > 0);
-        }
+        for (int k16 = 0; k16 < 4; ++k16)
+          mma_ss(tmem_at(tm, 0, C_MK), dKNm + mstep(k16), dWUk + kstep(k16, 32768), id_128x256_mnk, k16 > 0);
         mma_commit(bar);
       }
       if (tid == 32 && alive) {  // second group: thread 32
         fence_after_sync();
 #pragma unroll
         for (int k16 = 0; k16 < 4; ++k16) {
-          const uint64_t pd = dPPk + kstep(k16, 8192);
-          mma_ss(tmem_at(tm, 0, C_PW), pd, dKKk + kstep(k16, 16384), id_64x128_kk_neg, k16 > 0);
-          mma_ss(tmem_at(tm, 0, C_PW), dTTk + kstep(k16, 8192), dQQm + mstep(k16), id_64x128_kmn, 1);
-          mma_ss(tmem_at(tm, 0, C_PU), pd, dVVk + kstep(k16, 16384), id_64x128_kk, k16 > 0);
+          const uint64_t pt = dPPk + kstep(k16, 8192);   // P^T: P's rows are the K-major B operand
+          mma_ss(tmem_at(tm, 0, C_RT), dWUk + kstep(k16, 16384), pt, id_128x64_kk_neg, k16 > 0);
+          mma_ss(tmem_at(tm, 0, C_OT), dUk + kstep(k16, 16384), pt, id_128x64_kk, k16 > 0);
         }
+#pragma unroll
+        for (int k16 = 0; k16 < 4; ++k16)
+          mma_ss(tmem_at(tm, 0, C_RT), dQQm + mstep(k16), dTTk + kstep(k16, 8192), id_128x64_mnk, 1);
         mma_commit(bar2);
       }
       if (tid == 0) bulk_wait_read();   // staged records read: their tiles may be rewritten
       alive = __syncthreads_and(wait_mma(bar, phase, a.status, alive, a.wait_ns));
       fence_after_sync();
       const int row = 32 * sub + lane;        // M=128 layout row
-      const int r64 = 16 * sub + lane;        // M=64 layout row (lane < 16)
       // M_s = Diag(Gamma_l) - K~^T W: M_1 -> M1 tile and B_1 -> B1 tile while the second group runs;
       // M_2 -> KK, QQ (combine A operand) once the second group no longer reads W^T and Q Gamma there
       auto m_epilogue = [&](uint8_t* dst, bool with_b) {
@@ -955,6 +965,13 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
           }
         }
       };
+      // transposed results (M = 128 layout: lane = channel) -> a swizzled [128 channels][64 tokens] panel
+      auto t_epilogue = [&](uint32_t col, uint8_t* panel) {
+        float v[32];
+        tmem_ld32(tmem_at(tm, 32 * sub, col + 32 * chalf), v);
+        tmem_wait_ld();
+        st_row32_h(panel, row, 32 * chalf, v);
+      };
       if (s == 0) m_epilogue(M1, true);
       alive = alive && wait_mma(bar2, phase2, a.status, alive, a.wait_ns);
       fence_after_sync();
@@ -968,51 +985,32 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
         }
       }
       if (s == 0) {
-        // R_1 = Q Gamma - P W and O'_1, staged for the record (R rows 0-63, O'' rows 0-63)
-        uint8_t* stR = TT;                                  // [panel][64 rows][128 B], swizzled (TT and PP)
-        uint4* stO = reinterpret_cast<uint4*>(KN);          // [c/8][64 rows][8]
-        for (int cb = 0; cb < 2; ++cb) {
-          const int col0 = 64 * chalf + 32 * cb;
-          float rr[32], pu[32];
-          tmem_ld32(tmem_at(tm, 32 * sub, C_PW + col0), rr);
-          tmem_ld32(tmem_at(tm, 32 * sub, C_PU + col0), pu);
-          tmem_wait_ld();
-          if (lane < 16) {
-            st_row32_h(stR + chalf * 8192, r64, col0 & 63, rr);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) stO[((col0 >> 3) + i) * 64 + r64] = pack8(pu + 8 * i);
-          }
-        }
+        // R_1^T and O'_1^T, staged for the record (token panel / half 0): TT and PP, KN
+        t_epilogue(C_RT, TT);
+        t_epilogue(C_OT, KN);
         fence_proxy_async();
         fence_before_sync();
         alive = __syncthreads_and(alive);
         if (tid == 0) {
-          bulk_s2g(gR, stR, 8192);
-          bulk_s2g(gR + 16384, stR + 8192, 8192);
-          bulk_s2g(gO, stO, 16384);
+          bulk_s2g(gO, KN, 16384);   // KN first, as its own group: the next sub-chunk rewrites it first
+          bulk_commit();
+          bulk_s2g(gR, TT, 16384);
           bulk_commit();
         }
       } else {
-        m_epilogue(KK, false);
-        // Q^_2 = Q Gamma - P W -> KN (K~ no longer needed; K-major A operand, 2 panels of 8 KB)
-        for (int cb = 0; cb < 2; ++cb) {
-          const int col0 = 64 * chalf + 32 * cb;
-          float rr[32];
-          tmem_ld32(tmem_at(tm, 32 * sub, C_PW + col0), rr);
-          tmem_wait_ld();
-          if (lane < 16) st_row32_h(KN + chalf * 8192, r64, col0 & 63, rr);
-        }
+        m_epilogue(QQ, false);
+        // Q^_2^T -> KK (MN-major B operand of the combine)
+        t_epilogue(C_RT, KK);
         fence_proxy_async();
         fence_before_sync();
         alive = __syncthreads_and(alive);
         // ---------------- combine ----------------
-        if ((tid == 0 || tid == 32) && alive) {   // thread 0: M, B (bar); thread 32: R_2, O''_2 (bar2)
+        if ((tid == 0 || tid == 32) && alive) {   // thread 0: M, B (bar); thread 32: R_2^T, O''_2^T (bar2)
           fence_after_sync();
-          const uint32_t id_q = idesc_f16(64, 128, false, true);
           if (tid == 0) {
 #pragma unroll
             for (int k16 = 0; k16 < 8; ++k16) {
-              const uint64_t m2 = dKQk + kstep(k16, 16384);
+              const uint64_t m2 = dM2k + kstep(k16, 16384);
               mma_ss(tmem_at(tm, 0, C_MK), m2, dM1m + mstep(k16), id_128x128_kmn, k16 > 0);   // M = M_2 M_1
               mma_ss(tmem_at(tm, 0, C_BK), m2, dB1m + mstep(k16), id_128x128_kmn, 1);         // B = B_2 + M_2 B_1
             }
@@ -1020,9 +1018,10 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
           } else {
 #pragma unroll
             for (int k16 = 0; k16 < 8; ++k16) {
-              const uint64_t q2 = dKNk + kstep(k16, 8192);
-              mma_ss(tmem_at(tm, 0, C_PW), q2, dM1m + mstep(k16), id_q, k16 > 0);             // R_2 = Q^_2 M_1
-              mma_ss(tmem_at(tm, 0, C_PU), q2, dB1m + mstep(k16), id_q, 1);                   // O''_2 = O'_2 + Q^_2 B_1
+              // M_1, B_1 serve transposed as MN-major A operands (their images as B operands)
+              const uint64_t q2 = dQ2m + mstep(k16);
+              mma_ss(tmem_at(tm, 0, C_RT), dM1m + mstep(k16), q2, id_128x64_mnmn, k16 > 0);   // R_2^T = M_1^T Q^_2^T
+              mma_ss(tmem_at(tm, 0, C_OT), dB1m + mstep(k16), q2, id_128x64_mnmn, 1);         // O''_2^T += B_1^T Q^_2^T
             }
             mma_commit(bar2);
           }
@@ -1034,9 +1033,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
         }
         fence_after_sync();
         // records staged in tiles the combine products no longer read:
-        //   M -> M1 region, B -> B1 region, R_2 -> TT/PP region, O''_2 -> KN region
-        uint8_t* stR = TT;                               // [panel][64 rows][128 B], swizzled
-        uint4* stO = reinterpret_cast<uint4*>(KN);       // [c/8][64 rows][8]
+        //   M -> M1 region, B -> B1 region, R_2^T -> TT/PP region, O''_2^T -> KN region
         for (int cb = 0; cb < 2; ++cb) {
           const int col0 = 64 * chalf + 32 * cb;
           float m[32], bv[32];
@@ -1049,27 +1046,17 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
 #pragma unroll
           for (int i = 0; i < 4; ++i) b16[((col0 >> 3) + i) * 128 + row] = pack8(bv + 8 * i);
         }
-        for (int cb = 0; cb < 2; ++cb) {
-          const int col0 = 64 * chalf + 32 * cb;
-          float rr[32], oo[32];
-          tmem_ld32(tmem_at(tm, 32 * sub, C_PW + col0), rr);
-          tmem_ld32(tmem_at(tm, 32 * sub, C_PU + col0), oo);
-          tmem_wait_ld();
-          if (lane < 16) {
-            st_row32_h(stR + chalf * 8192, r64, col0 & 63, rr);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) stO[((col0 >> 3) + i) * 64 + r64] = pack8(oo + 8 * i);
-          }
-        }
+        t_epilogue(C_RT, TT);
+        t_epilogue(C_OT, KN);
         fence_proxy_async();
         fence_before_sync();
         __syncthreads();
         if (tid == 0) {
+          bulk_s2g(gO + 16384, KN, 16384);   // KN first, as its own group
+          bulk_commit();
           bulk_s2g(gM, M1, 32768);
           bulk_s2g(gB, B1, 32768);
-          bulk_s2g(gR + 8192, stR, 8192);
-          bulk_s2g(gR + 16384 + 8192, stR + 8192, 8192);
-          bulk_s2g(gO + 16384, stO, 16384);
+          bulk_s2g(gR + 16384, TT, 16384);
           bulk_commit();
         }
         fence_before_sync();
@@ -1172,6 +1159,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_chain(ChainArgs a) {
   fence_after_sync();
   const uint32_t tm = *tmem_slot;
   const uint32_t idesc = idesc_f16(128, CW, false, true);
+  const uint32_t idesc_r = idesc_f16(128, CW, true, true);   // R: MN-major image [channels][tokens]
   const uint64_t dS = mdesc0(smem_u32(sm + CH_OFF_S), 16384);
   const int lane_base = 32 * (warp & 3);
   bool ok = true;
@@ -1280,7 +1268,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_chain(ChainArgs a) {
     int issuedB = 0, o_pending = -1;
     if (loaderB)
       for (; issuedB < 2 && issuedB < nb; ++issuedB) load_B(issuedB);
-    const uint64_t dR = kdesc0(smem_u32(sm + CH_OFF_B));
+    const uint64_t dR = mdesc0(smem_u32(sm + CH_OFF_B), 16384);
     const int64_t tok_stride = (int64_t)a.H * D;
     __nv_bfloat16* obase = a.o + (int64_t)b * a.N * tok_stride + (int64_t)h * D + CW * qtr;
     for (int j = 0; j < nb && ok; ++j) {
@@ -1295,7 +1283,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_chain(ChainArgs a) {
           const uint64_t db = dS + (uint32_t)(j & 1) * (16384u >> 4);
           const uint32_t d = tm + CT_O + CW * (uint32_t)(j & 1);
 #pragma unroll
-          for (int k16 = 0; k16 < 8; ++k16) mma_ss(d, da + kstep(k16, 16384), db + mstep(k16), idesc, k16 > 0);
+          for (int k16 = 0; k16 < 8; ++k16) mma_ss(d, da + mstep(k16), db + mstep(k16), idesc_r, k16 > 0);
           mma_commit(&oDone[j & 1]);
           mma_commit(&sFree[j & 1]);
           o_pending = j;
@@ -1306,22 +1294,24 @@ __global__ void __launch_bounds__(256, 1) kda_tc_chain(ChainArgs a) {
       mine = mine && wait_or_abort(&fullB[j & 1], (uint32_t)(j >> 1) & 1u, abort_flag, a.wait_ns);   // O''_j visible here too
       if (mine) {
         fence_after_sync();
-        const uint4* Oo = reinterpret_cast<const uint4*>(sm + CH_OFF_B + (j & 1) * CH_SLOT + 32768);
+        // O'': this token half's [CW channels][64 tokens], swizzled rows
+        const uint8_t* Oo = sm + CH_OFF_B + (j & 1) * CH_SLOT + 32768 + (r >> 6) * (CW_BYTES / 2);
         const int64_t tok = (int64_t)j * BLK + r;
         __nv_bfloat16* orow = obase + tok * tok_stride;
 #pragma unroll
         for (int c0 = 0; c0 < CW; c0 += CK) {
           float v[CK];
           tmem_ld_n(tmem_at(tm, lane_base, CT_O + CW * (j & 1) + c0), v);
-          uint4 ou[CK / 8];
+          __half ou[CK];
 #pragma unroll
-          for (int i = 0; i < CK / 8; ++i) ou[i] = Oo[((r >> 6) * (CW / 8) + (c0 >> 3) + i) * 64 + (r & 63)];
+          for (int e = 0; e < CK; ++e) ou[e] = *reinterpret_cast<const __half*>(Oo + swz_off(c0 + e, r & 63));
           tmem_wait_ld();
           if (tok < a.N) {
 #pragma unroll
             for (int i = 0; i < CK / 8; ++i) {
               float of[8];
-              unpack8(ou[i], of);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) of[e] = __half2float(ou[8 * i + e]);
               uint32_t w[4];
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
