@@ -169,6 +169,7 @@ constexpr int C_RT = 256, C_OT = 320;      // R^T, O'^T (and the combine's R_2^T
 struct PrepMaps {
   CUtensorMap q, k, v;   // 64-channel boxes, 128-byte swizzle: one operand panel each
   CUtensorMap la;        // 128-channel box, no swizzle
+  CUtensorMap o;         // output (bf16), 64-channel boxes, 128-byte swizzle: stores of the state role
 };
 
 struct PrepArgs {
@@ -178,7 +179,14 @@ struct PrepArgs {
   int64_t N; int H; int BH; int n_blocks; int n_units;
   uint32_t* status;
   uint64_t wait_ns;       // limit of every device wait
-  int fault;              // self-test: 1 = the first CTA never issues its first k/q/v load
+  int fault;              // self-test: 1 = the first record CTA never issues its first k/q/v load;
+                          //            2 = the state CTA of (0, 0) never issues its first record load
+  // with n_state > 0, CTAs 0 .. n_state-1 run the state pass (one per batch item and head) beside
+  // the record CTAs: a record CTA publishes each finished record by writing `token` to its flag
+  int n_state;
+  uint32_t* flags;        // [B][H][n_blocks]
+  uint32_t token;
+  const float* S0; float* SN; __nv_bfloat16* o;
 };
 
 // One 16x8 tile of C = A B with fp32 operands in shared memory (A row-major with
@@ -414,6 +422,316 @@ __device__ __forceinline__ void warp_reduce_scatter64(float (&v)[64], int lane) 
 __host__ __device__ constexpr int oct_a(int r, int i) { return r * (r - 1) / 2 + i; }
 __host__ __device__ constexpr int oct_p(int r, int i) { return 28 + r * (r + 1) / 2 + i; }
 
+// ---------------------------------------------------------------------------
+// State role (CTAs 0 .. n_state-1 of a launch that has them): for one (batch item, head),
+// block by block as the record CTAs publish them,
+//   S_{j+1} = M_j S_j + B_j   and   O_j = R_j S_j + O''_j,
+// both products at the full 128-column width of S, on the tensor core (thread 0 issues them).
+//   warps 0-3, the state group: row k = tid of S (TMEM lane k, columns 0-127): adds B_j and
+//     writes the fp16 image of S_{j+1}, the MN-major B operand of the next block's products;
+//   warps 4-7, the output group: token row r = tid - 128 (TMEM lane r): adds O''_j, stages the
+//     bf16 rows in shared memory and thread 128 stores them by TMA.
+// Only M_j S_j and the state group's epilogue are serial; R_j S_j goes to one of two TMEM
+// buffers, so the output group works on block j while block j+1's products run.  Each part of
+// a record is loaded as soon as its slot is consumed: M_{j+1} once M_j S_j is complete,
+// R_{j+1} once R_j S_j is, B_{j+1} and O''_{j+1} once their groups have read B_j and O''_j.
+// A record is read only after its flag is acquired; the loads then cross into the async proxy.
+// ---------------------------------------------------------------------------
+constexpr uint32_t ST_S = 0, ST_M = 32768, ST_R = 65536, ST_B = 98304, ST_O = 131072, ST_STG = 163840,
+                   ST_BAR = 196608;
+constexpr int ST_TS = 0, ST_TO = 128;   // TMEM: S at columns 0-127, O in two buffers at 128 and 256
+
+// Waits (at most tmo ns) until *flag == token; gives up early when another CTA recorded a timeout.
+__device__ __forceinline__ bool wait_flag(const uint32_t* flag, uint32_t token, uint32_t* status, uint64_t tmo) {
+  if (ld_acquire_gpu(flag) == token) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (ld_acquire_gpu(flag) != token) {
+    if (*(volatile uint32_t*)status == KDA_ERR_TIMEOUT) return false;
+    if (globaltimer_ns() - t0 > tmo) { set_status(status, KDA_ERR_TIMEOUT); return false; }
+    __nanosleep(64);
+  }
+  return true;
+}
+
+// Bounded mbarrier wait that also gives up once another thread of the CTA gave up.
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag, uint64_t tmo) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > tmo) { *abort_flag = 1; return false; }
+  }
+  return true;
+}
+
+__device__ __noinline__ void state_role(const PrepArgs& a, const CUtensorMap* o_map, uint8_t* sm) {
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + ST_BAR);
+  uint64_t* m_full = bars;        // record parts landed
+  uint64_t* r_full = bars + 1;
+  uint64_t* b_full = bars + 2;
+  uint64_t* o_full = bars + 3;
+  uint64_t* ms_done = bars + 4;   // M_j S_j complete
+  uint64_t* rs_done = bars + 5;   // [2] R_j S_j complete (TMEM buffer j & 1); S_j no longer read
+  uint64_t* o_free = bars + 7;    // [2] output group has read TMEM buffer j & 1 (128 arrivals)
+  uint64_t* fin = bars + 9;       // every product of the CTA complete (exit path)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 10);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int bh = (int)blockIdx.x, b = bh / a.H, h = bh - b * a.H;
+  const int nb = a.n_blocks;
+  const int64_t rec0 = (int64_t)bh * nb;
+  const uint64_t tmo = a.wait_ns;
+  auto rec = [&](int j) { return a.ws + (rec0 + j) * kBlockBytes; };
+  auto flag = [&](int j) { return a.flags + rec0 + j; };
+  if (warp == 0) { tmem_alloc(tmem_slot, 512); tmem_relinquish(); }
+  if (tid == 0) {
+    for (int i = 0; i < 10; ++i) mbar_init(&bars[i], (i == 7 || i == 8) ? 128 : 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  // S_0 -> fp16 image: row k of S at (panel n / 64, row k, column n % 64)
+  if (tid < 128) {
+    const float* s0 = a.S0 ? a.S0 + ((int64_t)bh * D + tid) * D : nullptr;
+#pragma unroll
+    for (int n0 = 0; n0 < D; n0 += 32) {
+      float v[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) v[e] = s0 ? s0[n0 + e] : 0.f;
+      st_row32_h(sm + ST_S + (n0 >> 6) * 16384, tid, n0 & 63, v);
+    }
+  }
+  fence_proxy_async();
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tm = *tmem_slot;
+  const int lane_base = 32 * (warp & 3);
+  bool ok = true;
+
+  if (warp < 4) {
+    // ---------------- state group; thread 0 also issues the products and loads M, R, B ----------------
+    const int k = tid;
+    const bool lead = tid == 0;
+    const uint64_t dM = kdesc0(smem_u32(sm + ST_M));            // M_j: K-major, two 16 KB K-panels
+    const uint64_t dR = mdesc0(smem_u32(sm + ST_R), 16384);     // R_j: MN-major, two token panels
+    const uint64_t dS = mdesc0(smem_u32(sm + ST_S), 16384);     // S_j: MN-major, two column panels
+    const uint32_t id_ms = idesc_f16(128, 128, false, true);
+    const uint32_t id_rs = idesc_f16(128, 128, true, true);
+    int m_in = -1, r_in = -1, b_in = -1;   // lead: block of a load issued and not yet waited for
+    bool issued = false;                   // lead: some product was issued
+    // self-test of the bounded waits: the first record load of (0, 0) is never issued
+    const bool skip0 = a.fault == 2 && bh == 0;
+    if (lead) {
+      ok = wait_flag(flag(0), a.token, a.status, tmo);
+      if (ok && !skip0) {
+        fence_proxy_async_global();
+        mbar_arrive_expect_tx(m_full, 32768);
+        bulk_g2s(sm + ST_M, rec(0) + kMOff, 32768, m_full);
+        mbar_arrive_expect_tx(r_full, 32768);
+        bulk_g2s(sm + ST_R, rec(0) + kROff, 32768, r_full);
+        mbar_arrive_expect_tx(b_full, 32768);
+        bulk_g2s(sm + ST_B, rec(0) + kBOff, 32768, b_full);
+        m_in = r_in = b_in = 0;
+      }
+      if (!ok) *abort_flag = 1;
+    }
+    ok = named_sync_and(1, 128, ok);
+    int j = 0;
+    for (; j < nb && ok; ++j) {
+      const uint32_t par = (uint32_t)j & 1u, par2 = (uint32_t)(j >> 1) & 1u;
+      if (lead) {
+        // M_j S_j as soon as M_j has landed (S_j's image was written before the last barrier)
+        bool go = wait_or_abort(m_full, par, abort_flag, tmo);
+        if (go) {
+          m_in = -1;
+          fence_after_sync();
+#pragma unroll
+          for (int k16 = 0; k16 < 8; ++k16)
+            mma_ss(tmem_at(tm, 0, ST_TS), dM + kstep(k16, 16384), dS + mstep(k16), id_ms, k16 > 0);
+          mma_commit(ms_done);
+          issued = true;
+        }
+        // R_j S_j into TMEM buffer j & 1 once R_j has landed and the output group has read that buffer
+        go = go && wait_or_abort(r_full, par, abort_flag, tmo);
+        if (go) r_in = -1;
+        if (go && j >= 2) go = wait_or_abort(&o_free[j & 1], par2 ^ 1u, abort_flag, tmo);
+        if (go) {
+          fence_after_sync();
+#pragma unroll
+          for (int k16 = 0; k16 < 8; ++k16)
+            mma_ss(tmem_at(tm, 0, ST_TO + 128 * (j & 1)), dR + mstep(k16), dS + mstep(k16), id_rs, k16 > 0);
+          mma_commit(&rs_done[j & 1]);
+        }
+      }
+      bool mine = wait_or_abort(ms_done, par, abort_flag, tmo);
+      if (lead && mine) {
+        if (j + 1 < nb) {   // M_j is consumed: M_{j+1} next
+          mine = wait_flag(flag(j + 1), a.token, a.status, tmo);
+          if (mine) {
+            fence_proxy_async_global();
+            mbar_arrive_expect_tx(m_full, 32768);
+            bulk_g2s(sm + ST_M, rec(j + 1) + kMOff, 32768, m_full);
+            m_in = j + 1;
+          } else {
+            *abort_flag = 1;
+          }
+        }
+      }
+      mine = mine && wait_or_abort(b_full, par, abort_flag, tmo);
+      if (lead && mine) b_in = -1;
+      uint4 pk[16];   // row k of S_{j+1} in fp16, 8 columns per entry
+      if (mine) {
+        fence_after_sync();
+        const uint4* Bs = reinterpret_cast<const uint4*>(sm + ST_B);   // [c/8][row][8]
+        float* sn = (j + 1 == nb && a.SN) ? a.SN + ((int64_t)bh * D + k) * D : nullptr;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          float sv[64];
+          tmem_ld32(tmem_at(tm, lane_base, ST_TS + 64 * half), *reinterpret_cast<float(*)[32]>(sv));
+          tmem_ld32(tmem_at(tm, lane_base, ST_TS + 64 * half + 32), *reinterpret_cast<float(*)[32]>(sv + 32));
+          uint4 bu[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) bu[i] = Bs[(8 * half + i) * 128 + k];
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            float bf[8];
+            unpack8(bu[i], bf);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) sv[8 * i + e] += bf[e];
+            pk[8 * half + i] = pack8(sv + 8 * i);
+          }
+          if (sn) {   // the final state, fp32
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              reinterpret_cast<float4*>(sn + 64 * half)[i] = make_float4(sv[4 * i], sv[4 * i + 1], sv[4 * i + 2], sv[4 * i + 3]);
+          }
+        }
+        // S_j is read by R_j S_j too: its image is rewritten only after that product
+        mine = wait_or_abort(&rs_done[j & 1], par2, abort_flag, tmo);
+        if (lead && mine && j + 1 < nb) {   // R_j is consumed: R_{j+1} next (its flag was acquired above)
+          mbar_arrive_expect_tx(r_full, 32768);
+          bulk_g2s(sm + ST_R, rec(j + 1) + kROff, 32768, r_full);
+          r_in = j + 1;
+        }
+      }
+      if (mine) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          *reinterpret_cast<uint4*>(sm + ST_S + (i >> 3) * 16384 + swz_off(k, 8 * (i & 7))) = pk[i];
+      }
+      fence_proxy_async();   // the image of S_{j+1}, read next by the tensor core
+      fence_before_sync();
+      ok = named_sync_and(1, 128, mine);   // S_{j+1} written; S TMEM and B_j read
+      fence_after_sync();
+      if (ok && lead && j + 1 < nb) {   // B_j is consumed: B_{j+1} next
+        mbar_arrive_expect_tx(b_full, 32768);
+        bulk_g2s(sm + ST_B, rec(j + 1) + kBOff, 32768, b_full);
+        b_in = j + 1;
+      }
+    }
+    if (lead) {
+      // work in flight after a timeout finishes before the CTA frees its memory
+      if (issued) {
+        mma_commit(fin);   // arrives once every product issued so far is complete
+        mbar_wait(fin, 0u, 100000000ull);
+      }
+      // a slot's pending load is its latest: the earlier phases of its barrier were all waited for
+      if (m_in >= 0) mbar_wait(m_full, (uint32_t)m_in & 1u, 100000000ull);
+      if (r_in >= 0) mbar_wait(r_full, (uint32_t)r_in & 1u, 100000000ull);
+      if (b_in >= 0) mbar_wait(b_full, (uint32_t)b_in & 1u, 100000000ull);
+    }
+  } else {
+    // ---------------- output group; thread 128 loads O'' and stores o ----------------
+    const int r = tid - 128;
+    const bool lead = r == 0;
+    int o_in = -1;   // lead: block of a load issued and not yet waited for
+    if (lead) {
+      bool got = wait_flag(flag(0), a.token, a.status, tmo);
+      if (got) {
+        fence_proxy_async_global();
+        mbar_arrive_expect_tx(o_full, 32768);
+        bulk_g2s(sm + ST_O, rec(0) + kOOff, 32768, o_full);
+        o_in = 0;
+      } else {
+        *abort_flag = 1;
+      }
+    }
+    const uint8_t* Oo = sm + ST_O + (r >> 6) * 16384;   // O'': [token half][128 channels][64 tokens]
+    for (int j = 0; j < nb && ok; ++j) {
+      const uint32_t par = (uint32_t)j & 1u, par2 = (uint32_t)(j >> 1) & 1u;
+      bool mine = wait_or_abort(&rs_done[j & 1], par2, abort_flag, tmo);
+      mine = mine && wait_or_abort(o_full, par, abort_flag, tmo);
+      if (lead && mine) o_in = -1;
+      uint4 po[16];   // token row r of O_j in bf16, 8 channels per entry
+      if (mine) {
+        fence_after_sync();
+#pragma unroll
+        for (int n0 = 0; n0 < D; n0 += 32) {
+          float ov[32];
+          tmem_ld32(tmem_at(tm, lane_base, ST_TO + 128 * (j & 1) + n0), ov);
+          __half ou[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) ou[e] = *reinterpret_cast<const __half*>(Oo + swz_off(n0 + e, r & 63));
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int c = 8 * i + 2 * e;
+              __nv_bfloat162 hh = __floats2bfloat162_rn(ov[c] + __half2float(ou[c]), ov[c + 1] + __half2float(ou[c + 1]));
+              w[e] = *reinterpret_cast<uint32_t*>(&hh);
+            }
+            po[(n0 >> 3) + i] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+        fence_before_sync();
+        mbar_arrive(&o_free[j & 1]);
+      }
+      // the previous block's TMA store has read the staging tile; O''_j is read by every thread
+      if (lead) bulk_wait_read();
+      mine = named_sync_and(2, 128, mine);
+      if (lead && mine && j + 1 < nb) {
+        mine = wait_flag(flag(j + 1), a.token, a.status, tmo);
+        if (mine) {
+          fence_proxy_async_global();
+          mbar_arrive_expect_tx(o_full, 32768);
+          bulk_g2s(sm + ST_O, rec(j + 1) + kOOff, 32768, o_full);
+          o_in = j + 1;
+        } else {
+          *abort_flag = 1;
+        }
+      }
+      if (mine) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          *reinterpret_cast<uint4*>(sm + ST_STG + (i >> 3) * 16384 + swz_off(r, 8 * (i & 7))) = po[i];
+      }
+      fence_proxy_async();   // staged rows, read next by the TMA store
+      ok = named_sync_and(2, 128, mine);
+      if (ok && lead) {
+        // rows past the sequence end are not stored (TMA clips them)
+#pragma unroll
+        for (int pnl = 0; pnl < 2; ++pnl)
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf)
+            tma_store_4d(o_map, sm + ST_STG + pnl * 16384 + hf * 8192, 64 * pnl, h, j * BLK + 64 * hf, b);
+        bulk_commit();
+      }
+    }
+    if (lead) {
+      bulk_wait_all();
+      if (o_in >= 0) mbar_wait(o_full, (uint32_t)o_in & 1u, 100000000ull);
+    }
+  }
+  if (tid == 0 && *abort_flag) set_status(a.status, KDA_ERR_TIMEOUT);
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  if (warp == 0) tmem_dealloc(tm, 512);
+}
+
 template <typename TIn>
 __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_constant__ PrepMaps mp) {
   extern __shared__ uint8_t dyn[];
@@ -445,6 +763,12 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
   const int sub = warp & 3, chalf = warp >> 2;
 
   if (*(volatile uint32_t*)a.status == KDA_ERR_TIMEOUT) return;   // an earlier CTA gave up: skip the work
+  if ((int)blockIdx.x < a.n_state) {
+    state_role(a, &mp.o, sm);
+    return;
+  }
+  // record CTA pcta of npcta: units pcta, pcta + npcta, ...
+  const int pcta = (int)blockIdx.x - a.n_state, npcta = (int)gridDim.x - a.n_state;
   if (warp == 0) { tmem_alloc(tmem_slot, 512); tmem_relinquish(); }
   if (tid == 0) {
     mbar_init(bar, 1);
@@ -462,7 +786,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
   bool in_inflight = false, v_inflight = false;   // thread 0: TMA loads not yet waited for
   // batch item, head and first token of the sub-chunk this CTA processes after (u, s_)
   auto next_sub = [&](int u, int s_, int& nb_, int& nh_, int& nt0_) -> bool {
-    const int nu = s_ == 0 ? u : u + (int)gridDim.x;
+    const int nu = s_ == 0 ? u : u + npcta;
     if (nu >= a.n_units) return false;
     const int blk_ = nu / a.BH, bh_ = nu - blk_ * a.BH;
     nb_ = bh_ / a.H;
@@ -478,9 +802,9 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
   };
   uint32_t beta_next = 0u;
   bool beta_ok = false;
-  if (tid < SUB && (int)blockIdx.x < a.n_units) {
-    const int bh_ = (int)blockIdx.x % a.BH;   // unit blockIdx.x: block blockIdx.x / BH, sub-chunk 0
-    const int t_ = ((int)blockIdx.x / a.BH) * BLK + tid;
+  if (tid < SUB && pcta < a.n_units) {
+    const int bh_ = pcta % a.BH;   // unit pcta: block pcta / BH, sub-chunk 0
+    const int t_ = (pcta / a.BH) * BLK + tid;
     beta_next = load_beta(bh_ / a.H, bh_ % a.H, t_);
     beta_ok = t_ < a.N;
   }
@@ -503,9 +827,9 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
       tma_load_4d(G + G_IN + pnl * 16384 + 8192, &mp.q, 64 * pnl, h_, t0_, b_, in_bar);
     }
   };
-  // self-test of the bounded waits: the first CTA never issues its first inputs, so its wait gives up
-  if (tid == 0 && (int)blockIdx.x < a.n_units && !(a.fault == 1 && blockIdx.x == 0)) {
-    issue_in(blockIdx.x, 0);
+  // self-test of the bounded waits: the first record CTA never issues its first inputs, so its wait gives up
+  if (tid == 0 && pcta < a.n_units && !(a.fault == 1 && pcta == 0)) {
+    issue_in(pcta, 0);
     in_inflight = true;
   }
 
@@ -533,7 +857,15 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
   // front-pass role of this thread: octet fo (tokens 8 fo .. 8 fo + 7), channels 4 lane .. 4 lane + 3
   const int fo = warp, fpnl = lane >> 4, fpc = (4 * lane) & 63;
 
-  for (int unit = blockIdx.x; unit < a.n_units && alive; unit += gridDim.x) {
+  // thread 0: the unit whose record stores are committed but not yet published (with state CTAs)
+  int pub_pending = -1;
+  auto publish = [&](int u) {
+    const int blk_ = u / a.BH, bh_ = u - blk_ * a.BH;
+    fence_proxy_async_global();   // the completed bulk stores, ordered before the release
+    st_release_gpu(a.flags + (int64_t)bh_ * a.n_blocks + blk_, a.token);
+  };
+
+  for (int unit = pcta; unit < a.n_units && alive; unit += npcta) {
     const int blk = unit / a.BH, bh = unit - blk * a.BH;
     const int b = bh / a.H, h = bh - b * a.H;
     uint8_t* rec = a.ws + (((int64_t)b * a.H + h) * a.n_blocks + blk) * kBlockBytes;
@@ -886,7 +1218,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
       }
       if (tid == 0 && alive) {
         // A, X, Y consumed: G takes the log alpha, k and q of this CTA's next sub-chunk
-        const int nunit = s == 0 ? unit : unit + (int)gridDim.x;
+        const int nunit = s == 0 ? unit : unit + npcta;
         if (nunit < a.n_units) {
           issue_in(nunit, s ^ 1);
           in_inflight = true;
@@ -996,6 +1328,12 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
           bulk_commit();
           bulk_s2g(gR, TT, 16384);
           bulk_commit();
+          if (pub_pending >= 0) {
+            // the previous unit's stores (older than these two groups) are long complete by now
+            bulk_wait_but2();
+            publish(pub_pending);
+            pub_pending = -1;
+          }
         }
       } else {
         m_epilogue(QQ, false);
@@ -1058,6 +1396,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
           bulk_s2g(gB, B1, 32768);
           bulk_s2g(gR + 16384, TT, 16384);
           bulk_commit();
+          if (a.n_state > 0) pub_pending = unit;
         }
         fence_before_sync();
         __syncthreads();   // TMEM and shared tiles free for the next unit
@@ -1070,6 +1409,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
     if (in_inflight) mbar_wait(in_bar, in_phase, 100000000ull);
     if (v_inflight) mbar_wait(v_bar, v_phase, 100000000ull);
     bulk_wait_all();
+    if (pub_pending >= 0) publish(pub_pending);
   }
   fence_before_sync();
   __syncthreads();
@@ -1111,17 +1451,6 @@ struct ChainArgs {
   uint64_t wait_ns;       // limit of every device wait
   int fault;              // self-test: 2 = CTA (0, 0, 0) never issues its first record load
 };
-
-// Bounded wait (at most tmo ns) that also gives up as soon as another thread of the CTA gave up.
-__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag, uint64_t tmo) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (*abort_flag) return false;
-    if (globaltimer_ns() - t0 > tmo) { *abort_flag = 1; return false; }
-  }
-  return true;
-}
 
 template <int CW>
 __global__ void __launch_bounds__(256, 1) kda_tc_chain(ChainArgs a) {
@@ -1391,13 +1720,44 @@ cudaError_t launch_all(const Dims& d, const void* q, const void* k, const void* 
 
   const int BH = d.B * d.H;
   const int n_units = BH * n_blocks;
-  PrepArgs pa{q, k, v, la, beta, ws, d.N, d.H, BH, n_blocks, n_units, status, wait_ns, fault};
+  PrepArgs pa{q, k, v, la, beta, ws, d.N, d.H, BH, n_blocks, n_units, status, wait_ns, fault,
+              0, nullptr, 0u, S0, SN, static_cast<__nv_bfloat16*>(o)};
   PrepMaps mp;
   const CUtensorMapDataType adt = kIsHalf<TIn> ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   if (!encode_act_map(&mp.q, q, adt, 2, d, 64, true) || !encode_act_map(&mp.k, k, adt, 2, d, 64, true) ||
       !encode_act_map(&mp.v, v, adt, 2, d, 64, true) ||
       !encode_act_map(&mp.la, la, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, d, 128, false))
     return cudaErrorInvalidValue;
+  // One launch: with few (batch item, head) pairs, one CTA per pair runs the serial state pass
+  // beside the record CTAs, consuming each record as soon as it is published.  Those CTAs wait on
+  // the others, so the launch is cooperative (every CTA resident at once) or not made this way.
+  if (!d.reuse_records && 4 * BH <= n_sm) {
+    int per_sm = 0;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kda_tc_prep<TIn>, 256, PREP_SMEM)) != cudaSuccess)
+      return e;
+    const int grid = BH + min(n_units, n_sm - BH);
+    if (per_sm >= 1 && grid <= per_sm * n_sm) {
+      if (!encode_act_map(&mp.o, o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, 64, true)) return cudaErrorInvalidValue;
+      pa.n_state = BH;
+      pa.flags = reinterpret_cast<uint32_t*>(ws + (size_t)n_units * kBlockBytes);
+      pa.token = 1u;
+      // cleared on the stream first, so no earlier content of the workspace reads as published
+      if ((e = cudaMemsetAsync(pa.flags, 0, (size_t)n_units * sizeof(uint32_t), s)) != cudaSuccess) return e;
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3((unsigned)grid);
+      cfg.blockDim = dim3(256);
+      cfg.dynamicSmemBytes = PREP_SMEM;
+      cfg.stream = s;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeCooperative;
+      attr[0].val.cooperative = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      if ((e = cudaLaunchKernelEx(&cfg, kda_tc_prep<TIn>, pa, mp)) != cudaSuccess) return e;
+      if (launches) *launches += 1;
+      return cudaSuccess;
+    }
+  }
   // the records depend on q, k, v, log alpha and beta only: a caller that kept them (same inputs,
   // same workspace) runs the state pass alone
   if (!d.reuse_records) {
@@ -1420,7 +1780,9 @@ cudaError_t launch_all(const Dims& d, const void* q, const void* k, const void* 
 
 size_t chunk_tc_workspace_bytes(const Dims& d) {
   const int64_t n_blocks = (d.N + BLK - 1) / BLK;
-  return (size_t)d.B * d.H * n_blocks * kBlockBytes;
+  const size_t units = (size_t)d.B * d.H * n_blocks;
+  // the records, then one publication flag per record
+  return units * kBlockBytes + ((units * sizeof(uint32_t) + 255) & ~size_t(255));
 }
 
 bool chunk_tc_supported(const Dims& d) { return d.dk == D && d.dv == D; }

@@ -43,6 +43,7 @@ def test_noalloc_matches_chunk_fwd_on_two_calls():
         ws = kda.alloc_workspace(p, torch.bfloat16)
         kda.kda_chunk_fwd(p, q, k, v, la, beta, ref_o, ws, initial_state=s0, final_state=ref_s)
         assert kda.kda_read_status(ws) == kda.KDA_OK
+        ref_launches = kda.kda_last_launch_count()
         o = torch.full_like(ref_o, float("nan"))
         sn = torch.full_like(ref_s, float("nan"))
         rc = lib.kda_chunk_fwd_noalloc(ctypes.byref(p), kda.KDA_DT_BF16, q.data_ptr(), k.data_ptr(), v.data_ptr(),
@@ -51,7 +52,7 @@ def test_noalloc_matches_chunk_fwd_on_two_calls():
         assert rc == kda.KDA_OK, kda.kda_status_str(rc)
         torch.cuda.synchronize()
         assert int(status.item()) == kda.KDA_OK
-        assert kda.kda_last_launch_count() == 2     # record kernel + state pass
+        assert kda.kda_last_launch_count() == ref_launches >= 1   # the same kernels as kda_chunk_fwd
         assert_parity(o.float().cpu().numpy(), ref_o.float().cpu().numpy(), "bf16", f"call {call} o")
         assert_parity(sn.cpu().numpy(), ref_s.cpu().numpy(), "bf16", f"call {call} state")
         # both entry points run the same kernels on the same inputs: the results agree bit for bit
