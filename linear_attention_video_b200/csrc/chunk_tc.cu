@@ -426,31 +426,47 @@ __host__ __device__ constexpr int oct_p(int r, int i) { return 28 + r * (r + 1) 
 // State role (CTAs 0 .. n_state-1 of a launch that has them): for one (batch item, head),
 // block by block as the record CTAs publish them,
 //   S_{j+1} = M_j S_j + B_j   and   O_j = R_j S_j + O''_j,
-// both products at the full 128-column width of S, on the tensor core (thread 0 issues them).
-//   warps 0-3, the state group: row k = tid of S (TMEM lane k, columns 0-127): adds B_j and
-//     writes the fp16 image of S_{j+1}, the MN-major B operand of the next block's products;
-//   warps 4-7, the output group: token row r = tid - 128 (TMEM lane r): adds O''_j, stages the
-//     bf16 rows in shared memory and thread 128 stores them by TMA.
-// Only M_j S_j and the state group's epilogue are serial; R_j S_j goes to one of two TMEM
-// buffers, so the output group works on block j while block j+1's products run.  Each part of
-// a record is loaded as soon as its slot is consumed: M_{j+1} once M_j S_j is complete,
-// R_{j+1} once R_j S_j is, B_{j+1} and O''_{j+1} once their groups have read B_j and O''_j.
-// A record is read only after its flag is acquired; the loads then cross into the async proxy.
+// on the tensor core at the full 128-column width of S.
+//   warps 0-3, the state group: thread 0 issues M_j S_j; row k = tid of S (TMEM lane k) adds B_j
+//     (read from L2 into registers while the product runs) and writes the fp16 image of S_{j+1},
+//     the MN-major B operand of the next block's products.  This is the serial part.
+//   warps 4-7, the output group: thread 128 issues R_j S_j and then O''_j I (the identity adds
+//     O'' in the accumulator) into one of two TMEM buffers; token row r = tid - 128 (TMEM lane r)
+//     converts O_j to bf16 and stages it; thread 128 stores the staged rows by TMA.
+// M_{j+1}, R_{j+1} and O''_{j+1} are loaded as soon as the product that read the slot is
+// complete.  Records are read only after their flags are acquired: a lead thread reads the
+// flags of up to eight blocks ahead with relaxed loads and acquires those published, in order,
+// with one fence; the loads then cross into the async proxy.
 // ---------------------------------------------------------------------------
-constexpr uint32_t ST_S = 0, ST_M = 32768, ST_R = 65536, ST_B = 98304, ST_O = 131072, ST_STG = 163840,
+constexpr uint32_t ST_S = 0, ST_M = 32768, ST_R = 65536, ST_O = 98304, ST_I = 131072, ST_STG = 163840,
                    ST_BAR = 196608;
 constexpr int ST_TS = 0, ST_TO = 128;   // TMEM: S at columns 0-127, O in two buffers at 128 and 256
 
-// Waits (at most tmo ns) until *flag == token; gives up early when another CTA recorded a timeout.
-__device__ __forceinline__ bool wait_flag(const uint32_t* flag, uint32_t token, uint32_t* status, uint64_t tmo) {
-  if (ld_acquire_gpu(flag) == token) return true;
-  const uint64_t t0 = globaltimer_ns();
-  while (ld_acquire_gpu(flag) != token) {
+// Acquires the flags of blocks ready, ready + 1, ... (up to eight per poll) until block `need`
+// is acquired; at most tmo ns, less if another CTA recorded a timeout.
+__device__ __forceinline__ bool acquire_through(const uint32_t* flags, int need, int nb, int& ready, uint32_t token,
+                                                uint32_t* status, uint64_t tmo) {
+  if (need < ready) return true;
+  uint64_t t0 = 0;
+  for (;;) {
+    const int n_poll = min(8, nb - ready);
+    uint32_t f[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) f[i] = i < n_poll ? ld_relaxed_gpu(flags + ready + i) : 0u;
+    int n = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) n += (n == i && f[i] == token) ? 1 : 0;   // published prefix
+    if (n > 0) {
+      fence_acq_rel_gpu();   // the relaxed reads that saw the releases become acquires
+      ready += n;
+      if (need < ready) return true;
+      continue;
+    }
+    if (t0 == 0) t0 = globaltimer_ns();
     if (*(volatile uint32_t*)status == KDA_ERR_TIMEOUT) return false;
     if (globaltimer_ns() - t0 > tmo) { set_status(status, KDA_ERR_TIMEOUT); return false; }
     __nanosleep(64);
   }
-  return true;
 }
 
 // Bounded mbarrier wait that also gives up once another thread of the CTA gave up.
@@ -466,38 +482,41 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
 
 __device__ __noinline__ void state_role(const PrepArgs& a, const CUtensorMap* o_map, uint8_t* sm) {
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + ST_BAR);
-  uint64_t* m_full = bars;        // record parts landed
+  uint64_t* m_full = bars;           // record parts landed
   uint64_t* r_full = bars + 1;
-  uint64_t* b_full = bars + 2;
-  uint64_t* o_full = bars + 3;
-  uint64_t* ms_done = bars + 4;   // M_j S_j complete
-  uint64_t* rs_done = bars + 5;   // [2] R_j S_j complete (TMEM buffer j & 1); S_j no longer read
-  uint64_t* o_free = bars + 7;    // [2] output group has read TMEM buffer j & 1 (128 arrivals)
-  uint64_t* fin = bars + 9;       // every product of the CTA complete (exit path)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 10);
+  uint64_t* o_full = bars + 2;
+  uint64_t* ms_issued = bars + 3;    // M_j S_j is in the tensor pipe (R_j S_j goes after it)
+  uint64_t* ms_done = bars + 4;      // M_j S_j complete
+  uint64_t* rs_done = bars + 5;      // R_j S_j complete: S_j and R_j no longer read
+  uint64_t* od_done = bars + 6;      // O''_j I complete: O_j in TMEM, O''_j no longer read
+  uint64_t* fin = bars + 7;          // [2] every product of thread 0 / 128 complete (exit path)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 9);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int tid = threadIdx.x, warp = tid >> 5;
   const int bh = (int)blockIdx.x, b = bh / a.H, h = bh - b * a.H;
   const int nb = a.n_blocks;
   const int64_t rec0 = (int64_t)bh * nb;
   const uint64_t tmo = a.wait_ns;
+  const uint32_t* flags = a.flags + rec0;
+  const uint64_t pol_once = l2_policy_evict_first();   // each record part is read once
   auto rec = [&](int j) { return a.ws + (rec0 + j) * kBlockBytes; };
-  auto flag = [&](int j) { return a.flags + rec0 + j; };
   if (warp == 0) { tmem_alloc(tmem_slot, 512); tmem_relinquish(); }
   if (tid == 0) {
-    for (int i = 0; i < 10; ++i) mbar_init(&bars[i], (i == 7 || i == 8) ? 128 : 1);
+    for (int i = 0; i < 9; ++i) mbar_init(&bars[i], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  // S_0 -> fp16 image: row k of S at (panel n / 64, row k, column n % 64)
-  if (tid < 128) {
-    const float* s0 = a.S0 ? a.S0 + ((int64_t)bh * D + tid) * D : nullptr;
+  // fp16 images, rows 0-127 at (panel n / 64, row, column n % 64): S_0 (threads 0-127) and the
+  // identity (threads 128-255)
+  {
+    const int row = tid & 127;
+    const float* s0 = (tid < 128 && a.S0) ? a.S0 + ((int64_t)bh * D + row) * D : nullptr;
 #pragma unroll
     for (int n0 = 0; n0 < D; n0 += 32) {
       float v[32];
 #pragma unroll
-      for (int e = 0; e < 32; ++e) v[e] = s0 ? s0[n0 + e] : 0.f;
-      st_row32_h(sm + ST_S + (n0 >> 6) * 16384, tid, n0 & 63, v);
+      for (int e = 0; e < 32; ++e) v[e] = tid < 128 ? (s0 ? s0[n0 + e] : 0.f) : (row == n0 + e ? 1.f : 0.f);
+      st_row32_h(sm + (tid < 128 ? ST_S : ST_I) + (n0 >> 6) * 16384, row, n0 & 63, v);
     }
   }
   fence_proxy_async();
@@ -506,43 +525,46 @@ __device__ __noinline__ void state_role(const PrepArgs& a, const CUtensorMap* o_
   fence_after_sync();
   const uint32_t tm = *tmem_slot;
   const int lane_base = 32 * (warp & 3);
+  const uint64_t dS = mdesc0(smem_u32(sm + ST_S), 16384);     // S_j: MN-major, two column panels
   bool ok = true;
 
   if (warp < 4) {
-    // ---------------- state group; thread 0 also issues the products and loads M, R, B ----------------
+    // ---------------- state group ----------------
     const int k = tid;
     const bool lead = tid == 0;
     const uint64_t dM = kdesc0(smem_u32(sm + ST_M));            // M_j: K-major, two 16 KB K-panels
-    const uint64_t dR = mdesc0(smem_u32(sm + ST_R), 16384);     // R_j: MN-major, two token panels
-    const uint64_t dS = mdesc0(smem_u32(sm + ST_S), 16384);     // S_j: MN-major, two column panels
     const uint32_t id_ms = idesc_f16(128, 128, false, true);
-    const uint32_t id_rs = idesc_f16(128, 128, true, true);
-    int m_in = -1, r_in = -1, b_in = -1;   // lead: block of a load issued and not yet waited for
-    bool issued = false;                   // lead: some product was issued
+    int m_in = -1;          // lead: block of a load issued and not yet waited for
+    bool issued = false;    // lead: some product was issued
+    int ready = 0;          // lead: flags of blocks < ready acquired
     // self-test of the bounded waits: the first record load of (0, 0) is never issued
     const bool skip0 = a.fault == 2 && bh == 0;
     if (lead) {
-      ok = wait_flag(flag(0), a.token, a.status, tmo);
+      ok = acquire_through(flags, 0, nb, ready, a.token, a.status, tmo);
       if (ok && !skip0) {
         fence_proxy_async_global();
         mbar_arrive_expect_tx(m_full, 32768);
-        bulk_g2s(sm + ST_M, rec(0) + kMOff, 32768, m_full);
-        mbar_arrive_expect_tx(r_full, 32768);
-        bulk_g2s(sm + ST_R, rec(0) + kROff, 32768, r_full);
-        mbar_arrive_expect_tx(b_full, 32768);
-        bulk_g2s(sm + ST_B, rec(0) + kBOff, 32768, b_full);
-        m_in = r_in = b_in = 0;
+        bulk_g2s_hint(sm + ST_M, rec(0) + kMOff, 32768, m_full, pol_once);
+        m_in = 0;
       }
       if (!ok) *abort_flag = 1;
     }
-    ok = named_sync_and(1, 128, ok);
+    ok = named_sync_and(1, 128, ok);   // also orders the B loads below after the lead's acquire
     int j = 0;
     for (; j < nb && ok; ++j) {
-      const uint32_t par = (uint32_t)j & 1u, par2 = (uint32_t)(j >> 1) & 1u;
+      const uint32_t par = (uint32_t)j & 1u;
+      // B_j row k from L2 into registers while M_j S_j runs ([c/8][row][8]; not cached in L1)
+      uint4 bu[16];
+      {
+        const uint4* Bg = reinterpret_cast<const uint4*>(rec(j) + kBOff);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) bu[i] = __ldcg(Bg + i * 128 + k);
+      }
+      bool mine = true;
       if (lead) {
-        // M_j S_j as soon as M_j has landed (S_j's image was written before the last barrier)
-        bool go = wait_or_abort(m_full, par, abort_flag, tmo);
-        if (go) {
+        // M_j S_j as soon as M_j has landed (the image of S_j was written before the last barrier)
+        mine = wait_or_abort(m_full, par, abort_flag, tmo);
+        if (mine) {
           m_in = -1;
           fence_after_sync();
 #pragma unroll
@@ -550,159 +572,158 @@ __device__ __noinline__ void state_role(const PrepArgs& a, const CUtensorMap* o_
             mma_ss(tmem_at(tm, 0, ST_TS), dM + kstep(k16, 16384), dS + mstep(k16), id_ms, k16 > 0);
           mma_commit(ms_done);
           issued = true;
+          mbar_arrive(ms_issued);
+          // the next record's flag, while the product runs
+          if (j + 1 < nb) mine = acquire_through(flags, j + 1, nb, ready, a.token, a.status, tmo);
         }
-        // R_j S_j into TMEM buffer j & 1 once R_j has landed and the output group has read that buffer
-        go = go && wait_or_abort(r_full, par, abort_flag, tmo);
-        if (go) r_in = -1;
-        if (go && j >= 2) go = wait_or_abort(&o_free[j & 1], par2 ^ 1u, abort_flag, tmo);
-        if (go) {
-          fence_after_sync();
-#pragma unroll
-          for (int k16 = 0; k16 < 8; ++k16)
-            mma_ss(tmem_at(tm, 0, ST_TO + 128 * (j & 1)), dR + mstep(k16), dS + mstep(k16), id_rs, k16 > 0);
-          mma_commit(&rs_done[j & 1]);
-        }
+        if (!mine) *abort_flag = 1;
       }
-      bool mine = wait_or_abort(ms_done, par, abort_flag, tmo);
-      if (lead && mine) {
-        if (j + 1 < nb) {   // M_j is consumed: M_{j+1} next
-          mine = wait_flag(flag(j + 1), a.token, a.status, tmo);
-          if (mine) {
-            fence_proxy_async_global();
-            mbar_arrive_expect_tx(m_full, 32768);
-            bulk_g2s(sm + ST_M, rec(j + 1) + kMOff, 32768, m_full);
-            m_in = j + 1;
-          } else {
-            *abort_flag = 1;
-          }
-        }
+      mine = mine && wait_or_abort(ms_done, par, abort_flag, tmo);
+      if (lead && mine && j + 1 < nb) {   // M_j is consumed: M_{j+1} next
+        fence_proxy_async_global();
+        mbar_arrive_expect_tx(m_full, 32768);
+        bulk_g2s_hint(sm + ST_M, rec(j + 1) + kMOff, 32768, m_full, pol_once);
+        m_in = j + 1;
       }
-      mine = mine && wait_or_abort(b_full, par, abort_flag, tmo);
-      if (lead && mine) b_in = -1;
-      uint4 pk[16];   // row k of S_{j+1} in fp16, 8 columns per entry
       if (mine) {
         fence_after_sync();
-        const uint4* Bs = reinterpret_cast<const uint4*>(sm + ST_B);   // [c/8][row][8]
         float* sn = (j + 1 == nb && a.SN) ? a.SN + ((int64_t)bh * D + k) * D : nullptr;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           float sv[64];
           tmem_ld32(tmem_at(tm, lane_base, ST_TS + 64 * half), *reinterpret_cast<float(*)[32]>(sv));
           tmem_ld32(tmem_at(tm, lane_base, ST_TS + 64 * half + 32), *reinterpret_cast<float(*)[32]>(sv + 32));
-          uint4 bu[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) bu[i] = Bs[(8 * half + i) * 128 + k];
           tmem_wait_ld();
+          uint4 pk[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             float bf[8];
-            unpack8(bu[i], bf);
+            unpack8(bu[8 * half + i], bf);
 #pragma unroll
             for (int e = 0; e < 8; ++e) sv[8 * i + e] += bf[e];
-            pk[8 * half + i] = pack8(sv + 8 * i);
+            pk[i] = pack8(sv + 8 * i);
           }
           if (sn) {   // the final state, fp32
 #pragma unroll
             for (int i = 0; i < 16; ++i)
               reinterpret_cast<float4*>(sn + 64 * half)[i] = make_float4(sv[4 * i], sv[4 * i + 1], sv[4 * i + 2], sv[4 * i + 3]);
           }
-        }
-        // S_j is read by R_j S_j too: its image is rewritten only after that product
-        mine = wait_or_abort(&rs_done[j & 1], par2, abort_flag, tmo);
-        if (lead && mine && j + 1 < nb) {   // R_j is consumed: R_{j+1} next (its flag was acquired above)
-          mbar_arrive_expect_tx(r_full, 32768);
-          bulk_g2s(sm + ST_R, rec(j + 1) + kROff, 32768, r_full);
-          r_in = j + 1;
-        }
-      }
-      if (mine) {
+          // S_j is read by R_j S_j too: its image is rewritten only after that product
+          if (half == 0) mine = wait_or_abort(rs_done, par, abort_flag, tmo);
+          if (mine) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          *reinterpret_cast<uint4*>(sm + ST_S + (i >> 3) * 16384 + swz_off(k, 8 * (i & 7))) = pk[i];
+            for (int i = 0; i < 8; ++i) *reinterpret_cast<uint4*>(sm + ST_S + half * 16384 + swz_off(k, 8 * i)) = pk[i];
+          }
+        }
       }
       fence_proxy_async();   // the image of S_{j+1}, read next by the tensor core
       fence_before_sync();
-      ok = named_sync_and(1, 128, mine);   // S_{j+1} written; S TMEM and B_j read
+      ok = named_sync_and(1, 128, mine);   // S_{j+1} written; S TMEM read; flag j+1 acquired
       fence_after_sync();
-      if (ok && lead && j + 1 < nb) {   // B_j is consumed: B_{j+1} next
-        mbar_arrive_expect_tx(b_full, 32768);
-        bulk_g2s(sm + ST_B, rec(j + 1) + kBOff, 32768, b_full);
-        b_in = j + 1;
-      }
     }
     if (lead) {
       // work in flight after a timeout finishes before the CTA frees its memory
       if (issued) {
-        mma_commit(fin);   // arrives once every product issued so far is complete
-        mbar_wait(fin, 0u, 100000000ull);
+        mma_commit(&fin[0]);   // arrives once every product this thread issued is complete
+        mbar_wait(&fin[0], 0u, 100000000ull);
       }
       // a slot's pending load is its latest: the earlier phases of its barrier were all waited for
       if (m_in >= 0) mbar_wait(m_full, (uint32_t)m_in & 1u, 100000000ull);
-      if (r_in >= 0) mbar_wait(r_full, (uint32_t)r_in & 1u, 100000000ull);
-      if (b_in >= 0) mbar_wait(b_full, (uint32_t)b_in & 1u, 100000000ull);
     }
   } else {
-    // ---------------- output group; thread 128 loads O'' and stores o ----------------
+    // ---------------- output group ----------------
     const int r = tid - 128;
     const bool lead = r == 0;
-    int o_in = -1;   // lead: block of a load issued and not yet waited for
+    const uint64_t dR = mdesc0(smem_u32(sm + ST_R), 16384);     // R_j: MN-major, two token panels
+    const uint64_t dO = mdesc0(smem_u32(sm + ST_O), 16384);     // O''_j: MN-major, two token panels
+    const uint64_t dI = mdesc0(smem_u32(sm + ST_I), 16384);
+    const uint32_t id_mn = idesc_f16(128, 128, true, true);
+    int r_in = -1, o_in = -1;   // lead: block of a load issued and not yet waited for
+    bool issued = false;
+    int ready = 0;              // lead: flags of blocks < ready acquired
     if (lead) {
-      bool got = wait_flag(flag(0), a.token, a.status, tmo);
-      if (got) {
+      ok = acquire_through(flags, 0, nb, ready, a.token, a.status, tmo);
+      if (ok) {
         fence_proxy_async_global();
+        mbar_arrive_expect_tx(r_full, 32768);
+        bulk_g2s_hint(sm + ST_R, rec(0) + kROff, 32768, r_full, pol_once);
         mbar_arrive_expect_tx(o_full, 32768);
-        bulk_g2s(sm + ST_O, rec(0) + kOOff, 32768, o_full);
-        o_in = 0;
+        bulk_g2s_hint(sm + ST_O, rec(0) + kOOff, 32768, o_full, pol_once);
+        r_in = o_in = 0;
       } else {
         *abort_flag = 1;
       }
     }
-    const uint8_t* Oo = sm + ST_O + (r >> 6) * 16384;   // O'': [token half][128 channels][64 tokens]
+    ok = named_sync_and(2, 128, ok);
     for (int j = 0; j < nb && ok; ++j) {
-      const uint32_t par = (uint32_t)j & 1u, par2 = (uint32_t)(j >> 1) & 1u;
-      bool mine = wait_or_abort(&rs_done[j & 1], par2, abort_flag, tmo);
-      mine = mine && wait_or_abort(o_full, par, abort_flag, tmo);
-      if (lead && mine) o_in = -1;
+      const uint32_t par = (uint32_t)j & 1u;
+      const uint32_t tbuf = ST_TO + 128u * (uint32_t)(j & 1);
+      bool mine = true;
+      if (lead) {
+        // R_j S_j behind M_j S_j, then O''_j I; TMEM buffer j & 1 was read two blocks ago
+        mine = wait_or_abort(ms_issued, par, abort_flag, tmo) && wait_or_abort(r_full, par, abort_flag, tmo);
+        if (mine) {
+          r_in = -1;
+          fence_after_sync();
+#pragma unroll
+          for (int k16 = 0; k16 < 8; ++k16)
+            mma_ss(tmem_at(tm, 0, tbuf), dR + mstep(k16), dS + mstep(k16), id_mn, k16 > 0);
+          mma_commit(rs_done);
+          issued = true;
+        }
+        mine = mine && wait_or_abort(o_full, par, abort_flag, tmo);
+        if (mine) {
+          o_in = -1;
+          fence_after_sync();
+#pragma unroll
+          for (int k16 = 0; k16 < 8; ++k16)
+            mma_ss(tmem_at(tm, 0, tbuf), dO + mstep(k16), dI + mstep(k16), id_mn, 1);
+          mma_commit(od_done);
+        }
+        if (mine && j + 1 < nb) {
+          mine = acquire_through(flags, j + 1, nb, ready, a.token, a.status, tmo);
+          // R_j, then O''_j, consumed as their products complete: the next block's parts
+          mine = mine && wait_or_abort(rs_done, par, abort_flag, tmo);
+          if (mine) {
+            fence_proxy_async_global();
+            mbar_arrive_expect_tx(r_full, 32768);
+            bulk_g2s_hint(sm + ST_R, rec(j + 1) + kROff, 32768, r_full, pol_once);
+            r_in = j + 1;
+          }
+          mine = mine && wait_or_abort(od_done, par, abort_flag, tmo);
+          if (mine) {
+            mbar_arrive_expect_tx(o_full, 32768);
+            bulk_g2s_hint(sm + ST_O, rec(j + 1) + kOOff, 32768, o_full, pol_once);
+            o_in = j + 1;
+          }
+        }
+        if (!mine) *abort_flag = 1;
+        bulk_wait_read();   // the previous block's TMA store has read the staging tile
+      }
+      mine = mine && wait_or_abort(od_done, par, abort_flag, tmo);
       uint4 po[16];   // token row r of O_j in bf16, 8 channels per entry
       if (mine) {
         fence_after_sync();
 #pragma unroll
-        for (int n0 = 0; n0 < D; n0 += 32) {
-          float ov[32];
-          tmem_ld32(tmem_at(tm, lane_base, ST_TO + 128 * (j & 1) + n0), ov);
-          __half ou[32];
-#pragma unroll
-          for (int e = 0; e < 32; ++e) ou[e] = *reinterpret_cast<const __half*>(Oo + swz_off(n0 + e, r & 63));
+        for (int n0 = 0; n0 < D; n0 += 64) {
+          float ov[64];
+          tmem_ld32(tmem_at(tm, lane_base, tbuf + n0), *reinterpret_cast<float(*)[32]>(ov));
+          tmem_ld32(tmem_at(tm, lane_base, tbuf + n0 + 32), *reinterpret_cast<float(*)[32]>(ov + 32));
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
+          for (int i = 0; i < 8; ++i) {
             uint32_t w[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const int c = 8 * i + 2 * e;
-              __nv_bfloat162 hh = __floats2bfloat162_rn(ov[c] + __half2float(ou[c]), ov[c + 1] + __half2float(ou[c + 1]));
+              __nv_bfloat162 hh = __floats2bfloat162_rn(ov[8 * i + 2 * e], ov[8 * i + 2 * e + 1]);
               w[e] = *reinterpret_cast<uint32_t*>(&hh);
             }
             po[(n0 >> 3) + i] = make_uint4(w[0], w[1], w[2], w[3]);
           }
         }
-        fence_before_sync();
-        mbar_arrive(&o_free[j & 1]);
       }
-      // the previous block's TMA store has read the staging tile; O''_j is read by every thread
-      if (lead) bulk_wait_read();
-      mine = named_sync_and(2, 128, mine);
-      if (lead && mine && j + 1 < nb) {
-        mine = wait_flag(flag(j + 1), a.token, a.status, tmo);
-        if (mine) {
-          fence_proxy_async_global();
-          mbar_arrive_expect_tx(o_full, 32768);
-          bulk_g2s(sm + ST_O, rec(j + 1) + kOOff, 32768, o_full);
-          o_in = j + 1;
-        } else {
-          *abort_flag = 1;
-        }
-      }
+      fence_before_sync();
+      mine = named_sync_and(2, 128, mine);   // staging tile free (lead waited above); TMEM buffer read
       if (mine) {
 #pragma unroll
         for (int i = 0; i < 16; ++i)
@@ -721,8 +742,13 @@ __device__ __noinline__ void state_role(const PrepArgs& a, const CUtensorMap* o_
       }
     }
     if (lead) {
-      bulk_wait_all();
+      if (issued) {
+        mma_commit(&fin[1]);
+        mbar_wait(&fin[1], 0u, 100000000ull);
+      }
+      if (r_in >= 0) mbar_wait(r_full, (uint32_t)r_in & 1u, 100000000ull);
       if (o_in >= 0) mbar_wait(o_full, (uint32_t)o_in & 1u, 100000000ull);
+      bulk_wait_all();
     }
   }
   if (tid == 0 && *abort_flag) set_status(a.status, KDA_ERR_TIMEOUT);
@@ -769,6 +795,9 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
   }
   // record CTA pcta of npcta: units pcta, pcta + npcta, ...
   const int pcta = (int)blockIdx.x - a.n_state, npcta = (int)gridDim.x - a.n_state;
+  // inputs are read once; records stay in L2 for the state CTAs of the same launch
+  const uint64_t pol_in = l2_policy_evict_first();
+  const uint64_t pol_rec = a.n_state > 0 ? l2_policy_evict_last() : l2_policy_evict_first();
   if (warp == 0) { tmem_alloc(tmem_slot, 512); tmem_relinquish(); }
   if (tid == 0) {
     mbar_init(bar, 1);
@@ -812,7 +841,7 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
   auto issue_v = [&](int b_, int h_, int t0_) {
     mbar_arrive_expect_tx(v_bar, 2 * 8192);
 #pragma unroll
-    for (int pnl = 0; pnl < 2; ++pnl) tma_load_4d(VV + pnl * 8192, &mp.v, 64 * pnl, h_, t0_, b_, v_bar);
+    for (int pnl = 0; pnl < 2; ++pnl) tma_load_4d_hint(VV + pnl * 8192, &mp.v, 64 * pnl, h_, t0_, b_, v_bar, pol_in);
   };
   bool v_early = false;   // thread 0: the sub-chunk's v is already on its way
   // log alpha, k and q of sub-chunk s_ of unit u -> G (thread 0)
@@ -820,11 +849,11 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
     const int blk_ = u / a.BH, bh_ = u - blk_ * a.BH;
     const int b_ = bh_ / a.H, h_ = bh_ - b_ * a.H, t0_ = blk_ * BLK + s_ * SUB;
     mbar_arrive_expect_tx(in_bar, 32768 + 4 * 8192);
-    tma_load_4d(G, &mp.la, 0, h_, t0_, b_, in_bar);
+    tma_load_4d_hint(G, &mp.la, 0, h_, t0_, b_, in_bar, pol_in);
 #pragma unroll
     for (int pnl = 0; pnl < 2; ++pnl) {
-      tma_load_4d(G + G_IN + pnl * 16384, &mp.k, 64 * pnl, h_, t0_, b_, in_bar);
-      tma_load_4d(G + G_IN + pnl * 16384 + 8192, &mp.q, 64 * pnl, h_, t0_, b_, in_bar);
+      tma_load_4d_hint(G + G_IN + pnl * 16384, &mp.k, 64 * pnl, h_, t0_, b_, in_bar, pol_in);
+      tma_load_4d_hint(G + G_IN + pnl * 16384 + 8192, &mp.q, 64 * pnl, h_, t0_, b_, in_bar, pol_in);
     }
   };
   // self-test of the bounded waits: the first record CTA never issues its first inputs, so its wait gives up
@@ -1324,9 +1353,9 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
         fence_before_sync();
         alive = __syncthreads_and(alive);
         if (tid == 0) {
-          bulk_s2g(gO, KN, 16384);   // KN first, as its own group: the next sub-chunk rewrites it first
+          bulk_s2g_hint(gO, KN, 16384, pol_rec);   // KN first, as its own group: the next sub-chunk rewrites it first
           bulk_commit();
-          bulk_s2g(gR, TT, 16384);
+          bulk_s2g_hint(gR, TT, 16384, pol_rec);
           bulk_commit();
           if (pub_pending >= 0) {
             // the previous unit's stores (older than these two groups) are long complete by now
@@ -1390,11 +1419,11 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
         fence_before_sync();
         __syncthreads();
         if (tid == 0) {
-          bulk_s2g(gO + 16384, KN, 16384);   // KN first, as its own group
+          bulk_s2g_hint(gO + 16384, KN, 16384, pol_rec);   // KN first, as its own group
           bulk_commit();
-          bulk_s2g(gM, M1, 32768);
-          bulk_s2g(gB, B1, 32768);
-          bulk_s2g(gR + 16384, TT, 16384);
+          bulk_s2g_hint(gM, M1, 32768, pol_rec);
+          bulk_s2g_hint(gB, B1, 32768, pol_rec);
+          bulk_s2g_hint(gR + 16384, TT, 16384, pol_rec);
           bulk_commit();
           if (a.n_state > 0) pub_pending = unit;
         }
@@ -1437,7 +1466,12 @@ struct ChainLayout {
   static constexpr uint32_t OFF_A = 0;                        // ring A: M_j, B_j   (2 slots)
   static constexpr uint32_t OFF_B = 2 * SLOT;                 // ring B: R_j, O''_j (2 slots)
   static constexpr uint32_t OFF_S = 4 * SLOT;                 // S_j fp16 MN-major images (2 x 16 KB)
-  static constexpr uint32_t OFF_BAR = OFF_S + 32768;
+  // with CW <= 32, O'' is added on the tensor core (O'' I, I the CW x CW identity, MN-major), as in
+  // the state role of kda_tc_prep, so both give the same bits; with CW = 64 (no room for I) the
+  // output threads add it
+  static constexpr bool O_MMA = CW <= 32;
+  static constexpr uint32_t OFF_I = OFF_S + 32768;
+  static constexpr uint32_t OFF_BAR = OFF_I + (O_MMA ? 4096 : 0);
   static constexpr uint32_t SMEM = OFF_BAR + 256 + 1024;
 };
 
@@ -1492,6 +1526,20 @@ __global__ void __launch_bounds__(256, 1) kda_tc_chain(ChainArgs a) {
   const uint64_t dS = mdesc0(smem_u32(sm + CH_OFF_S), 16384);
   const int lane_base = 32 * (warp & 3);
   bool ok = true;
+  if constexpr (L::O_MMA) {
+    // rows 0 .. CW-1 of the identity: the K = CW operand of O'' I
+    if (tid < CW) {
+#pragma unroll
+      for (int i = 0; i < CW / 8; ++i) {
+        float e8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) e8[e] = tid == 8 * i + e ? 1.f : 0.f;
+        *reinterpret_cast<uint4*>(sm + L::OFF_I + swz_off(tid, 8 * i)) = pack8(e8);
+      }
+    }
+    fence_proxy_async();
+    __syncthreads();
+  }
 
   if (warp < 4) {
     // ---------------- state group ----------------
@@ -1613,6 +1661,13 @@ __global__ void __launch_bounds__(256, 1) kda_tc_chain(ChainArgs a) {
           const uint32_t d = tm + CT_O + CW * (uint32_t)(j & 1);
 #pragma unroll
           for (int k16 = 0; k16 < 8; ++k16) mma_ss(d, da + mstep(k16), db + mstep(k16), idesc_r, k16 > 0);
+          if constexpr (L::O_MMA) {
+            // O'' of this slot: [token half][CW channels][64 tokens], an MN-major A operand (K = CW)
+            const uint64_t dO = mdesc0(smem_u32(sm + CH_OFF_B + (j & 1) * CH_SLOT + 32768), CW_BYTES / 2);
+            const uint64_t dI = mdesc0(smem_u32(sm + L::OFF_I), 16384);
+#pragma unroll
+            for (int k16 = 0; k16 < CW / 16; ++k16) mma_ss(d, dO + mstep(k16), dI + mstep(k16), idesc_r, 1);
+          }
           mma_commit(&oDone[j & 1]);
           mma_commit(&sFree[j & 1]);
           o_pending = j;
@@ -1631,20 +1686,23 @@ __global__ void __launch_bounds__(256, 1) kda_tc_chain(ChainArgs a) {
         for (int c0 = 0; c0 < CW; c0 += CK) {
           float v[CK];
           tmem_ld_n(tmem_at(tm, lane_base, CT_O + CW * (j & 1) + c0), v);
-          __half ou[CK];
+          if constexpr (!L::O_MMA) {   // O'' added here (with CW <= 32 it is in the accumulator)
+            __half ou[CK];
 #pragma unroll
-          for (int e = 0; e < CK; ++e) ou[e] = *reinterpret_cast<const __half*>(Oo + swz_off(c0 + e, r & 63));
-          tmem_wait_ld();
+            for (int e = 0; e < CK; ++e) ou[e] = *reinterpret_cast<const __half*>(Oo + swz_off(c0 + e, r & 63));
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < CK; ++e) v[e] += __half2float(ou[e]);
+          } else {
+            tmem_wait_ld();
+          }
           if (tok < a.N) {
 #pragma unroll
             for (int i = 0; i < CK / 8; ++i) {
-              float of[8];
-#pragma unroll
-              for (int e = 0; e < 8; ++e) of[e] = __half2float(ou[8 * i + e]);
               uint32_t w[4];
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
-                __nv_bfloat162 hh = __floats2bfloat162_rn(v[8 * i + 2 * e] + of[2 * e], v[8 * i + 2 * e + 1] + of[2 * e + 1]);
+                __nv_bfloat162 hh = __floats2bfloat162_rn(v[8 * i + 2 * e], v[8 * i + 2 * e + 1]);
                 w[e] = *reinterpret_cast<uint32_t*>(&hh);
               }
               reinterpret_cast<uint4*>(orow + c0)[i] = make_uint4(w[0], w[1], w[2], w[3]);
