@@ -20,6 +20,8 @@
 // Text part: a small kernel, one thread per (token, 8 channels).
 #include <cuda_fp16.h>
 
+#include <type_traits>
+
 
 #include "common.cuh"
 
@@ -277,6 +279,153 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) vis_conv_kernel(ConvArgs
   asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 
+// ---- visual kernel on packed fp16 (bf16 inputs, fp16 outputs) ------------------------
+// The conv feeding the tensor-core scan, whose operands are fp16: the same tiles, plane ring and
+// frame rotation as vis_conv_kernel, but a lane owns two adjacent channels (a CTA 64) and every
+// tap is one fma.rn.f16x2 over both, accumulating in fp16.  That halves the FMA instructions of
+// the issue-bound fp32 kernel; the outputs carry a relative error of about 8e-4 (27 fp16
+// roundings) instead of 2e-4 (one rounding of an fp32 sum), the size of the scan's own fp16
+// operand roundings.
+constexpr int CG2 = 64;   // channels per CTA: two per lane
+
+template <int RUN>
+struct VisPlaneH2 {
+  static constexpr int PWr = NRUN * RUN + 2;
+  static constexpr int WPP = CG2 / 2;                   // 32-bit words (channel pairs) per pixel
+  static constexpr int PIX_CHUNKS = CG2 * 2 / 16;       // 16-byte chunks per pixel
+  static constexpr int NCHUNK = PH * PWr * PIX_CHUNKS;
+  static constexpr int NPF = (NCHUNK + kThreads - 1) / kThreads;
+  static constexpr int BYTES = PH * PWr * CG2 * 2;
+};
+
+// two bf16 (one 32-bit word) -> fp16 pair
+__device__ __forceinline__ __half2 bf2_to_h2(uint32_t u) {
+  return __floats2half2_rn(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+}
+
+template <int RUN>
+__device__ __forceinline__ void vis_plane_step_h2(const uint32_t* pl, bool compute, const __half2 (&wv)[kVisTaps],
+                                                  __half2 (&an)[RUN], __half2 (&ac)[RUN], __half2 (&ap)[RUN],
+                                                  __half* yo, bool emit, int nrun, int64_t C) {
+  constexpr int PWr = VisPlaneH2<RUN>::PWr, WPP = VisPlaneH2<RUN>::WPP;
+  if (compute) {
+#pragma unroll
+    for (int tb = 0; tb < 3; ++tb) {   // plane row tb feeds the thread's output row through tap row tb
+      const uint32_t* src = pl + tb * PWr * WPP;
+      __half2 in[RUN + 2];
+#pragma unroll
+      for (int i = 0; i < RUN + 2; ++i) in[i] = bf2_to_h2(src[i * WPP]);
+#pragma unroll
+      for (int te = 0; te < 3; ++te) {
+        const __half2 c0 = wv[tb * 3 + te], c1 = wv[9 + tb * 3 + te], c2 = wv[18 + tb * 3 + te];
+#pragma unroll
+        for (int i = 0; i < RUN; ++i) {
+          an[i] = __hfma2(c0, in[i + te], an[i]);
+          ac[i] = __hfma2(c1, in[i + te], ac[i]);
+          ap[i] = __hfma2(c2, in[i + te], ap[i]);
+        }
+      }
+    }
+  }
+  if (emit) {
+#pragma unroll
+    for (int i = 0; i < RUN; ++i)
+      if (i < nrun) *reinterpret_cast<__half2*>(yo + (int64_t)i * C) = ap[i];
+  }
+#pragma unroll
+  for (int i = 0; i < RUN; ++i) ap[i] = __float2half2_rn(0.f);   // ap becomes the frame three ahead
+}
+
+template <int RUN, int PT>
+__global__ void __launch_bounds__(kThreads, kMinBlocks) vis_conv_h2_kernel(ConvArgs a) {
+  static_assert(RPT == 1, "one output row per thread");
+  using VP = VisPlaneH2<RUN>;
+  constexpr int PWr = VP::PWr;
+  extern __shared__ __align__(128) uint8_t slots[];   // [NSLOT][PH][PWr][CG2] of bf16
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tile = blockIdx.x;
+  const int wt = tile % a.n_wtiles, hb = tile / a.n_wtiles;
+  const int cg0 = blockIdx.y * CG2;
+  const int tensor = blockIdx.z % 3, b = blockIdx.z / 3;
+  const int C = a.C;
+  const int tw0 = wt * (NRUN * RUN), th0 = hb * TH;
+  const int TW = min(NRUN * RUN, a.Wg - tw0), THh = min(TH, a.Hg - th0);
+  const int64_t HW = (int64_t)a.Hg * a.Wg;
+  const void* xs = tensor == 0 ? a.x[0] : (tensor == 1 ? a.x[1] : a.x[2]);
+  void* ys = tensor == 0 ? a.y[0] : (tensor == 1 ? a.y[1] : a.y[2]);
+  const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(xs) + ((int64_t)b * a.N + a.L) * C + cg0;
+  __half* y = static_cast<__half*>(ys) + ((int64_t)b * a.N + a.L) * C + cg0;
+
+  const int row = warp % TH, run = warp / TH;
+  const int w0 = run * RUN;
+  const int nrun = max(0, min(RUN, TW - w0));
+  const bool active = nrun > 0 && row < THh;
+
+  __half2 wv[kVisTaps];
+  {
+    const float* w0p = a.w_vis + ((int64_t)tensor * C + cg0 + 2 * lane) * kVisTaps;
+#pragma unroll
+    for (int i = 0; i < kVisTaps; ++i) wv[i] = __floats2half2_rn(w0p[i], w0p[kVisTaps + i]);
+  }
+
+  int goff[VP::NPF];
+#pragma unroll
+  for (int i = 0; i < VP::NPF; ++i) {
+    const int e = tid + i * kThreads;
+    goff[i] = -2;
+    if (e < VP::NCHUNK) {
+      const int cb = e % VP::PIX_CHUNKS, pix = e / VP::PIX_CHUNKS;
+      const int pr = pix / PWr, pc = pix - pr * PWr;
+      const int hh = th0 + pr - 1, ww = tw0 + pc - 1;
+      goff[i] = (hh >= 0 && hh < a.Hg && ww >= 0 && ww < a.Wg) ? (hh * a.Wg + ww) * C + cb * 8 : -1;
+    }
+  }
+  const uint32_t slot0 = (uint32_t)__cvta_generic_to_shared(slots);
+  auto issue = [&](int f) {
+    if (f < a.T) {
+      const __nv_bfloat16* xf = x + (int64_t)f * HW * C;
+      const uint32_t dst = slot0 + (uint32_t)(f % NSLOT) * VP::BYTES;
+#pragma unroll
+      for (int i = 0; i < VP::NPF; ++i) {
+        if (goff[i] >= -1)
+          cp_async16_zfill(dst + (uint32_t)(tid + i * kThreads) * 16u, goff[i] >= 0 ? xf + goff[i] : x,
+                           goff[i] >= 0 ? 16u : 0u);
+      }
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+
+  __half2 s0[RUN], s1[RUN], s2[RUN];
+#pragma unroll
+  for (int i = 0; i < RUN; ++i) { s0[i] = __float2half2_rn(0.f); s1[i] = s0[i]; s2[i] = s0[i]; }
+  for (int f = 0; f < NSLOT - 1; ++f) issue(f);
+
+  const int f_end = a.T + 2 - PT;
+  const uint32_t* pl_base = reinterpret_cast<const uint32_t*>(slots) + (row * PWr + w0) * VP::WPP + lane;
+  __half* y_base = y + ((int64_t)(th0 + row) * a.Wg + tw0 + w0) * C + 2 * lane;
+  auto step = [&](int f, __half2 (&an)[RUN], __half2 (&ac)[RUN], __half2 (&ap)[RUN]) {
+    asm volatile("cp.async.wait_group %0;" :: "n"(NSLOT - 2) : "memory");
+    __syncthreads();
+    issue(f + NSLOT - 1);
+    const int t = f + PT - 2;
+    const bool tv = t >= 0 && t < a.T;
+    vis_plane_step_h2<RUN>(pl_base + (f % NSLOT) * (VP::BYTES / 4), active && f < a.T, wv, an, ac, ap,
+                           y_base + (int64_t)t * HW * C, active && tv, nrun, C);
+  };
+  for (int f = 0; f < f_end; f += 3) {
+    if (PT == 1) {
+      step(f, s1, s0, s2);
+      if (f + 1 < f_end) step(f + 1, s2, s1, s0);
+      if (f + 2 < f_end) step(f + 2, s0, s2, s1);
+    } else {
+      step(f, s2, s1, s0);
+      if (f + 1 < f_end) step(f + 1, s0, s2, s1);
+      if (f + 2 < f_end) step(f + 2, s1, s0, s2);
+    }
+  }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+}
+
 // ---- visual weight gradient ------------------------------------------------------
 // dw[c][a][b][e] = sum over t, h, w of dy[t, h, w, c] x[t + a - PT, h + b - 1, w + e - 1, c].
 // Same tiles and plane ring as the forward kernel: plane f of x meets the dy frames
@@ -489,13 +638,42 @@ cudaError_t launch_vis_any(const ConvArgs& a, cudaStream_t s) {
   return launch_vis<TIn, TOut, 8, MODE>(a, s);
 }
 
+template <int RUN>
+cudaError_t launch_vis_h2(const ConvArgs& a0, cudaStream_t s) {
+  ConvArgs a = a0;
+  a.n_wtiles = (a.Wg + NRUN * RUN - 1) / (NRUN * RUN);
+  const size_t smem = (size_t)NSLOT * VisPlaneH2<RUN>::BYTES;
+  dim3 grid((unsigned)(a.n_wtiles * a.n_hbands), (unsigned)(a.C / CG2), (unsigned)(3 * a.B));
+  cudaError_t e;
+  if (a.pt == 2) {
+    e = cudaFuncSetAttribute(vis_conv_h2_kernel<RUN, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    vis_conv_h2_kernel<RUN, 2><<<grid, kThreads, smem, s>>>(a);
+  } else {
+    e = cudaFuncSetAttribute(vis_conv_h2_kernel<RUN, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    vis_conv_h2_kernel<RUN, 1><<<grid, kThreads, smem, s>>>(a);
+  }
+  return cudaGetLastError();
+}
+
 template <typename TIn, typename TOut>
 cudaError_t launch_t(const ConvArgs& a, cudaStream_t s) {
   if (a.L > 0) {
     const int64_t total = (int64_t)a.B * a.L * (a.C / 8);
     text_conv_kernel<TIn, TOut><<<dim3((unsigned)((total + 255) / 256), 3), 256, 0, s>>>(a);
   }
-  if (a.T > 0) return launch_vis_any<TIn, TOut, 0>(a, s);
+  if (a.T > 0) {
+    // the fp16 outputs feed the tensor-core scan: the visual conv runs on packed fp16
+    if constexpr (std::is_same_v<TIn, __nv_bfloat16> && std::is_same_v<TOut, __half>) {
+      if (a.C % CG2 == 0) {
+        if (a.Wg % 52 == 0 || (a.Wg <= 52 && a.Wg > 48)) return launch_vis_h2<13>(a, s);
+        if (a.Wg % 64 == 0 || a.Wg > 52) return launch_vis_h2<16>(a, s);
+        return launch_vis_h2<8>(a, s);
+      }
+    }
+    return launch_vis_any<TIn, TOut, 0>(a, s);
+  }
   return cudaGetLastError();
 }
 
