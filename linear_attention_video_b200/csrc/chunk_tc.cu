@@ -1252,6 +1252,13 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
           issue_in(nunit, s ^ 1);
           in_inflight = true;
         }
+        // the previous unit's record, stored at its end, is published while the products run (the
+        // proxy fence may wait for this thread's copies in flight; the products take longer)
+        if (pub_pending >= 0) {
+          bulk_wait_all();
+          publish(pub_pending);
+          pub_pending = -1;
+        }
       }
       {
         const bool w1 = wait_mma(bar, phase, a.status, alive, a.wait_ns);
@@ -1357,12 +1364,6 @@ __global__ void __launch_bounds__(256, 1) kda_tc_prep(PrepArgs a, const __grid_c
           bulk_commit();
           bulk_s2g_hint(gR, TT, 16384, pol_rec);
           bulk_commit();
-          if (pub_pending >= 0) {
-            // the previous unit's stores (older than these two groups) are long complete by now
-            bulk_wait_but2();
-            publish(pub_pending);
-            pub_pending = -1;
-          }
         }
       } else {
         m_epilogue(QQ, false);

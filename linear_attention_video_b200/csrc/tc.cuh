@@ -299,8 +299,6 @@ __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.w
 __device__ __forceinline__ void bulk_wait_read_but1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 // Every committed bulk store is complete (visible in global memory).
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-// Every committed bulk store but the two most recent groups is complete.
-__device__ __forceinline__ void bulk_wait_but2() { asm volatile("cp.async.bulk.wait_group 2;" ::: "memory"); }
 // Orders this thread's async-proxy accesses of global memory with its generic-proxy ones.
 __device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
 // Release store / acquire load of a flag word at GPU scope.

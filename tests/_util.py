@@ -1,4 +1,5 @@
 """Helpers shared by the tests: inputs to torch tensors and error metrics."""
+import os
 import numpy as np
 import torch
 
@@ -37,6 +38,10 @@ def max_abs(x, ref):
 
 def assert_parity(x, ref, dtype, what=""):
     e, m = rel_l2(x, ref), max_abs(x, ref)
+    log = os.environ.get("KDA_PARITY_LOG")
+    if log:   # one line per comparison, for reporting the measured errors
+        with open(log, "a") as f:
+            f.write(f"{os.environ.get('PYTEST_CURRENT_TEST', '?').split(' ')[0]}\t{what}\t{dtype}\t{e:.3e}\t{m:.3e}\n")
     if dtype == "bf16":
         assert e <= TOL_BF16_REL_L2 and m <= TOL_BF16_MAX_ABS, f"{what}: rel_l2={e:.3e} max_abs={m:.3e}"
     else:
