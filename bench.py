@@ -500,6 +500,57 @@ def ours_arm(args, w, idx, rank, world, local_rank):
         print(json.dumps(line), flush=True)
 
 
+def mixer_arm(args, rank, world, local_rank):
+    """KDA/MLA 3:1 against MHA/MLA 3:1 token-mixer stacks as N grows (synthetic weights, one GPU
+    per rank, every rank the same sweep): forward latency and peak memory per stack."""
+    import torch
+    from linear_attention_video_b200 import mixer
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    H, d, text_len, Hg, Wg = 16, 128, 512, 30, 52   # the 480x832 video layout, 16 heads of 128
+    frames = [int(f) for f in args.mixer_frames.split(",")]
+    stream = torch.cuda.current_stream(dev)
+    rows = []
+    with ClockSampler(local_rank) as clk:
+        for T in frames:
+            N = text_len + T * Hg * Wg
+            row = {"frames": T, "tokens": N}
+            for kind in ("kda", "mha"):
+                torch.cuda.empty_cache()
+                torch.cuda.reset_peak_memory_stats(dev)
+                try:
+                    layers = mixer.stack(kind, 1, H, d, text_len, (T, Hg, Wg), dev)
+                    x = torch.randn(1, N, H * d, generator=torch.Generator().manual_seed(T)).to(dev, torch.bfloat16)
+
+                    def step():
+                        mixer.run_stack(layers, x)
+                    for _ in range(args.warmup):
+                        step()
+                    ms = time_calls(step, args.steps, stream)
+                    row[kind + "_ms"] = reduce_max(ms, dev, world)
+                    row[kind + "_peak_gb"] = torch.cuda.max_memory_allocated(dev) / 1e9
+                    del layers, x
+                except torch.cuda.OutOfMemoryError:
+                    row[kind + "_ms"] = None
+                    row[kind + "_peak_gb"] = "oom"
+            if row.get("kda_ms") and row.get("mha_ms"):
+                row["speedup"] = row["mha_ms"] / row["kda_ms"]
+            rows.append(row)
+    clocks = clk.summary()
+    if rank == 0:
+        last = rows[-1]
+        line = {"metric": "KDA/MLA 3:1 vs MHA/MLA 3:1 token-mixer stack forward latency, 1 B200",
+                "value": last.get("speedup"), "unit": "x (MHA/MLA time / KDA/MLA time at the largest N)",
+                "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": "mixer_sweep_480x832", "B": 1, "H": H, "d": d, "text_len": text_len,
+                           "grid_hw": [Hg, Wg], "layers": "4 per stack (3 KDA or MHA, 1 MLA), residual",
+                           "mla": {"d_latent": mixer.D_LATENT, "d_nope": mixer.D_NOPE, "d_direct": mixer.D_DIRECT},
+                           "parallelism": f"replicas{world}"},
+                "sweep": rows, "clocks": clocks}
+        print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -519,6 +570,10 @@ def main():
     ap.add_argument("--seq-ranks", type=int, default=2, help="--shard seq on one GPU: ranks run as threads")
     ap.add_argument("--causal-t", action="store_true",
                     help="temporal taps of the 3D conv cover frames t-2..t instead of t-1..t+1")
+    ap.add_argument("--mixer", action="store_true",
+                    help="time KDA/MLA 3:1 against MHA/MLA 3:1 token-mixer stacks as N grows")
+    ap.add_argument("--mixer-frames", default="20,40,80,121,163",
+                    help="visual frames of the --mixer sweep (N = 512 + frames x 30 x 52)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     idx, w = workload_by_name(args.workload)
@@ -535,6 +590,9 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     try:
+        if args.mixer:
+            mixer_arm(args, rank, world, local_rank)
+            return
         arm = bwd_arm if args.which == "bwd" else (seq_arm if args.shard == "seq" else ours_arm)
         arm(args, w, idx, rank, world, local_rank)
     finally:
