@@ -1790,7 +1790,9 @@ cudaError_t launch_all(const Dims& d, const void* q, const void* k, const void* 
   // One launch: with few (batch item, head) pairs, one CTA per pair runs the serial state pass
   // beside the record CTAs, consuming each record as soon as it is published.  Those CTAs wait on
   // the others, so the launch is cooperative (every CTA resident at once) or not made this way.
-  if (!d.reuse_records && 4 * BH <= n_sm) {
+  // Each state CTA takes an SM from the records; past about a fifth of the SMs the separate
+  // state-pass kernel after the record kernel costs less.
+  if (!d.reuse_records && 5 * BH <= n_sm) {
     int per_sm = 0;
     if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kda_tc_prep<TIn>, 256, PREP_SMEM)) != cudaSuccess)
       return e;

@@ -150,10 +150,11 @@ def test_bf16_tensor_core_state_io(kda):
         assert rel_l2(s[:, h], ref_s[:, h]) < 5e-3
 
 
-@pytest.mark.parametrize("B,H", [(1, 40), (3, 12)])
+@pytest.mark.parametrize("B,H", [(1, 40), (3, 12), (2, 12)])
 def test_bf16_tensor_core_many_heads(kda, B, H):
-    """More (batch item, head) pairs than fit 16- or 32-column chain CTAs on the SMs: the serial pass
-    runs with 64 value columns per CTA (40 pairs) or 32 (36 pairs); parity on a few heads."""
+    """Many (batch item, head) pairs: 40 and 36 pairs run the record kernel and then the state-pass
+    kernel, with 64 and 32 value columns per CTA; 24 pairs (two batch items) run records and state
+    pass in one launch with 24 state CTAs; parity on a few heads."""
     import dataclasses
     w = dataclasses.replace(kda_synth.WORKLOADS[1], B=B, H=H, text_len=70, grid=(2, 11, 13))
     inp = kda_synth.generate(w, 41 + H)
@@ -344,11 +345,16 @@ def test_strong_decay_takes_exact_branch(kda):
     assert_parity(o, ref, "f32", "strong decay")
 
 
-def test_bf16_record_reuse_reruns_only_the_state_pass(kda):
+@pytest.mark.parametrize("B,H", [(1, 16), (2, 12)])
+def test_bf16_record_reuse_reruns_only_the_state_pass(kda, B, H):
     """KDA_FLAG_REUSE_RECORDS: a second kda_chunk_fwd on the same inputs and workspace, from
-    another initial state, launches the state pass alone and equals a fresh call bit for bit."""
-    w = kda_synth.WORKLOADS[1]
-    inp = workload_inputs(1)
+    another initial state, launches the state pass alone and equals a fresh call bit for bit.  A
+    fresh call runs the records and the state pass in one launch; the reused-record call runs the
+    separate state-pass kernel, with 16 value columns per CTA for 16 (batch item, head) pairs and
+    32 for 24, so both column widths are checked against the single launch."""
+    import dataclasses
+    w = dataclasses.replace(kda_synth.WORKLOADS[1], B=B, H=H)
+    inp = kda_synth.generate(w, 60 + H) if (B, H) != (1, 16) else workload_inputs(1)
     B, N, H, d = inp["shape"]
     t = to_device(inp)
     args = [t[n] for n in ("q", "k", "v", "log_alpha", "beta")]
