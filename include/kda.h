@@ -130,7 +130,13 @@ int kda_shortconv_fwd(const kda_problem* p, kda_dtype dtype,
                       void* q_out, void* k_out, void* v_out, void* stream);
 
 /* KDA scan only, on already-convolved q', k', v'.  initial_state may be NULL
- * (zero state); final_state may be NULL (not written).  Returns a kda_status. */
+ * (zero state); final_state may be NULL (not written).  Returns a kda_status.
+ * On the bf16 d = 128 tensor-core path the scan writes per-block records (and, after them, one
+ * flag word per record) to the workspace.  With at most a fifth as many (batch item, head) pairs
+ * as SMs it is one cooperative launch, whose state-pass CTAs wait for the record CTAs' flags (all
+ * its CTAs are resident at once, so it may start only once the whole grid fits on the device);
+ * otherwise, and when the device refuses a cooperative launch of that size, the record kernel and
+ * then the state-pass kernel. */
 int kda_chunk_fwd(const kda_problem* p, kda_dtype dtype,
                   const void* q, const void* k, const void* v,
                   const float* log_alpha, const void* beta,

@@ -1814,9 +1814,17 @@ cudaError_t launch_all(const Dims& d, const void* q, const void* k, const void* 
       attr[0].val.cooperative = 1;
       cfg.attrs = attr;
       cfg.numAttrs = 1;
-      if ((e = cudaLaunchKernelEx(&cfg, kda_tc_prep<TIn>, pa, mp)) != cudaSuccess) return e;
-      if (launches) *launches += 1;
-      return cudaSuccess;
+      e = cudaLaunchKernelEx(&cfg, kda_tc_prep<TIn>, pa, mp);
+      if (e == cudaSuccess) {
+        if (launches) *launches += 1;
+        return cudaSuccess;
+      }
+      // a device that cannot hold the whole grid at once (a partitioned GPU, say) refuses the
+      // cooperative launch: the record and state-pass kernels below do the same work
+      if (e != cudaErrorCooperativeLaunchTooLarge) return e;
+      (void)cudaGetLastError();
+      pa.n_state = 0;
+      pa.flags = nullptr;
     }
   }
   // the records depend on q, k, v, log alpha and beta only: a caller that kept them (same inputs,
