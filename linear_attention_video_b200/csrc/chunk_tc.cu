@@ -26,10 +26,13 @@
 // Two kernels:
 //   kda_tc_prep   persistent, one CTA per SM, looping over (block, batch item,
 //                 head) units: everything above, written to the workspace as one
-//                 record per unit (M, B, R, O'' in fp16 operand images).
+//                 record per unit (M, B, R, O'' in fp16 operand images).  With few
+//                 (batch item, head) pairs it is a cooperative launch whose first
+//                 CTAs, one per pair, run the serial pass S <- M S + B and the block
+//                 outputs O = R S + O'' as the other CTAs publish the records.
 //   kda_tc_chain  one CTA per (batch item, head, 16, 32 or 64 value columns):
-//                 the serial pass S <- M S + B, state kept in registers (fp32),
-//                 and beside it the block outputs O = R S + O''.
+//                 the serial pass and the outputs over records already written
+//                 (records kept from an earlier call, or many pairs).
 // Padding tokens of the last block carry k = q = v = 0, beta = 0, log alpha = 0.
 #include "common.cuh"
 #include "tc.cuh"

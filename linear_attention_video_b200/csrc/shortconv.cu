@@ -3,7 +3,9 @@
 // Text tokens: causal 1D depthwise conv; visual tokens: depthwise 3D conv over
 // the (T, H, W) latent grid, zero outside the grid, per modality (genai-atlas,
 // "How it works"; paper.rainbus.top, section 核心方法).  fp32 accumulation,
-// one rounding to the output type.
+// one rounding to the output type, except where the visual conv writes the fp16
+// inputs of the tensor-core scan: there it runs on packed fp16 FMAs
+// (vis_conv_h2_kernel, below).
 //
 // Visual part (the bulk of the work, bound by the fp32 FMA pipe): a CTA of two
 // warps owns 32 channels of one tensor (one per lane) and a tile of TH = 2 grid
