@@ -338,6 +338,37 @@ __device__ __forceinline__ void vis_plane_step_h2(const uint32_t* pl, bool compu
   for (int i = 0; i < RUN; ++i) ap[i] = __float2half2_rn(0.f);   // ap becomes the frame three ahead
 }
 
+// The text tokens of one (64-channel group, tensor, batch item) in a CTA of the packed visual
+// launch: the causal 1D conv of text_conv_kernel (fp32 accumulation, one rounding to fp16), a lane
+// owning two channels and each warp half of the tokens.  These CTAs run beside the visual tiles.
+__device__ __noinline__ void text_part_h2(const ConvArgs& a, const void* xs, void* ys, int cg0, int tensor, int b) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int C = a.C, K = a.text_k, c = cg0 + 2 * lane;
+  const uint32_t* x = reinterpret_cast<const uint32_t*>(static_cast<const __nv_bfloat16*>(xs) + (int64_t)b * a.N * C + c);
+  __half* y = static_cast<__half*>(ys) + (int64_t)b * a.N * C + c;
+  const float* w = a.w_text + ((int64_t)tensor * C + c) * K;
+  float w0[8], w1[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    w0[j] = j < K ? w[j] : 0.f;
+    w1[j] = j < K ? w[K + j] : 0.f;
+  }
+  const int64_t per = (a.L + 1) / 2, n0 = warp * per, n1 = min(a.L, n0 + per);
+  for (int64_t n = n0; n < n1; ++n) {
+    float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int64_t src = n - (K - 1) + j;
+      if (j < K && src >= 0) {
+        const uint32_t u = __ldg(x + src * (C / 2));
+        acc0 = fmaf(w0[j], __uint_as_float(u << 16), acc0);
+        acc1 = fmaf(w1[j], __uint_as_float(u & 0xffff0000u), acc1);
+      }
+    }
+    *reinterpret_cast<__half2*>(y + n * C) = __floats2half2_rn(acc0, acc1);
+  }
+}
+
 template <int RUN, int PT>
 __global__ void __launch_bounds__(kThreads, kMinBlocks) vis_conv_h2_kernel(ConvArgs a) {
   static_assert(RPT == 1, "one output row per thread");
@@ -355,6 +386,10 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) vis_conv_h2_kernel(ConvA
   const int64_t HW = (int64_t)a.Hg * a.Wg;
   const void* xs = tensor == 0 ? a.x[0] : (tensor == 1 ? a.x[1] : a.x[2]);
   void* ys = tensor == 0 ? a.y[0] : (tensor == 1 ? a.y[1] : a.y[2]);
+  if (tile >= a.n_wtiles * a.n_hbands) {   // past the visual tiles: the text tokens
+    text_part_h2(a, xs, ys, cg0, tensor, b);
+    return;
+  }
   const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(xs) + ((int64_t)b * a.N + a.L) * C + cg0;
   __half* y = static_cast<__half*>(ys) + ((int64_t)b * a.N + a.L) * C + cg0;
 
@@ -645,7 +680,8 @@ cudaError_t launch_vis_h2(const ConvArgs& a0, cudaStream_t s) {
   ConvArgs a = a0;
   a.n_wtiles = (a.Wg + NRUN * RUN - 1) / (NRUN * RUN);
   const size_t smem = (size_t)NSLOT * VisPlaneH2<RUN>::BYTES;
-  dim3 grid((unsigned)(a.n_wtiles * a.n_hbands), (unsigned)(a.C / CG2), (unsigned)(3 * a.B));
+  // one more CTA column for the text tokens, when there are any
+  dim3 grid((unsigned)(a.n_wtiles * a.n_hbands + (a.L > 0 ? 1 : 0)), (unsigned)(a.C / CG2), (unsigned)(3 * a.B));
   cudaError_t e;
   if (a.pt == 2) {
     e = cudaFuncSetAttribute(vis_conv_h2_kernel<RUN, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -660,15 +696,20 @@ cudaError_t launch_vis_h2(const ConvArgs& a0, cudaStream_t s) {
 }
 
 template <typename TIn, typename TOut>
-cudaError_t launch_t(const ConvArgs& a, cudaStream_t s) {
-  if (a.L > 0) {
+cudaError_t launch_t(const ConvArgs& a, cudaStream_t s, int* launches) {
+  // the fp16 outputs feed the tensor-core scan: the visual conv runs on packed fp16, its launch
+  // doing the text tokens too
+  constexpr bool kPackedOut = std::is_same_v<TIn, __nv_bfloat16> && std::is_same_v<TOut, __half>;
+  const bool packed = kPackedOut && a.T > 0 && a.C % CG2 == 0;
+  if (a.L > 0 && !packed) {
     const int64_t total = (int64_t)a.B * a.L * (a.C / 8);
     text_conv_kernel<TIn, TOut><<<dim3((unsigned)((total + 255) / 256), 3), 256, 0, s>>>(a);
+    if (launches) ++*launches;
   }
   if (a.T > 0) {
-    // the fp16 outputs feed the tensor-core scan: the visual conv runs on packed fp16
-    if constexpr (std::is_same_v<TIn, __nv_bfloat16> && std::is_same_v<TOut, __half>) {
-      if (a.C % CG2 == 0) {
+    if (launches) ++*launches;
+    if constexpr (kPackedOut) {
+      if (packed) {
         if (a.Wg % 52 == 0 || (a.Wg <= 52 && a.Wg > 48)) return launch_vis_h2<13>(a, s);
         if (a.Wg % 64 == 0 || a.Wg > 52) return launch_vis_h2<16>(a, s);
         return launch_vis_h2<8>(a, s);
@@ -696,11 +737,12 @@ cudaError_t launch_shortconv(const Dims& d, kda_dtype dt, const void* q, const v
   a.n_hbands = d.T > 0 ? (d.Hg + TH - 1) / TH : 0;
   if ((int64_t)d.B * d.N == 0) return cudaSuccess;
   cudaError_t e;
-  if (dt == KDA_DT_BF16 && out_f32) e = launch_t<__nv_bfloat16, float>(a, s);
-  else if (dt == KDA_DT_BF16 && out_f16) e = launch_t<__nv_bfloat16, __half>(a, s);
-  else if (dt == KDA_DT_BF16) e = launch_t<__nv_bfloat16, __nv_bfloat16>(a, s);
-  else e = launch_t<float, float>(a, s);
-  if (e == cudaSuccess && launches) *launches += (a.L > 0) + (a.T > 0);
+  int n = 0;
+  if (dt == KDA_DT_BF16 && out_f32) e = launch_t<__nv_bfloat16, float>(a, s, &n);
+  else if (dt == KDA_DT_BF16 && out_f16) e = launch_t<__nv_bfloat16, __half>(a, s, &n);
+  else if (dt == KDA_DT_BF16) e = launch_t<__nv_bfloat16, __nv_bfloat16>(a, s, &n);
+  else e = launch_t<float, float>(a, s, &n);
+  if (e == cudaSuccess && launches) *launches += n;
   return e;
 }
 
