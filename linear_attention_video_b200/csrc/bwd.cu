@@ -24,6 +24,8 @@
 //                              the dO terms Z = P^T dO, Y = QG^T dO
 //   cbwd_chain_kernel<D, false>  per CW value columns: S_in of every chunk, U
 //   cbwd_chain_kernel<D, true>   per CW value columns, in reverse: dS of every chunk, dU, dS0
+//                              (fp32 problems; bf16 problems run both chains as one launch of
+//                              cbwd_chain_h_kernel, on fp16 operands)
 //   cbwd_state_grad_kernel     per chunk: the contractions with S_in and dS
 //                              (dQG, dW, dKt), dP, dU V^T
 //   cbwd_local_grad_kernel     per chunk: dT, the inverse's adjoint, dq, dk, dv,
@@ -62,6 +64,10 @@ __device__ __forceinline__ void cp_async16(float* dst, const float* src) {
 __device__ __forceinline__ void cp_async16z(float* dst, const float* src, bool valid) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" :: "r"((uint32_t)__cvta_generic_to_shared(dst)),
                "l"(src), "r"(valid ? 16u : 0u) : "memory");
+}
+__device__ __forceinline__ void cp_async16v(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" :: "r"((uint32_t)__cvta_generic_to_shared(dst)),
+               "l"(src) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
@@ -341,6 +347,7 @@ __global__ void __launch_bounds__(NT, 1) cbwd_prep_kernel(CbwdArgs a) {
   __syncthreads();
   bool bad = false;
   float* Kt = a.w.Kt + p.ch * CH * D;
+  __half* Kth = reinterpret_cast<__half*>(a.w.Kt) + p.ch * CH * D;
   for (int idx = tid; idx < CH * D / 4; idx += NT) {   // each thread transforms its own elements in place
     const int r = idx / (D / 4), c4 = (idx % (D / 4)) * 4;
     const float4 k4 = *reinterpret_cast<const float4*>(Kx + r * LDD + c4);
@@ -361,7 +368,13 @@ __global__ void __launch_bounds__(NT, 1) cbwd_prep_kernel(CbwdArgs a) {
     *reinterpret_cast<float4*>(Kx + r * LDD + c4) = make_float4(kx[0], kx[1], kx[2], kx[3]);
     *reinterpret_cast<float4*>(KN + r * LDD + c4) = make_float4(kn[0], kn[1], kn[2], kn[3]);
     *reinterpret_cast<float4*>(Qx + r * LDD + c4) = make_float4(qx[0], qx[1], qx[2], qx[3]);
-    *reinterpret_cast<float4*>(Kt + r * D + c4) = make_float4(kt[0], kt[1], kt[2], kt[3]);
+    if (SPLIT) {
+      *reinterpret_cast<float4*>(Kt + r * D + c4) = make_float4(kt[0], kt[1], kt[2], kt[3]);
+    } else {   // fp16 operand of the chains
+      const __half2 h0 = __floats2half2_rn(kt[0], kt[1]), h1 = __floats2half2_rn(kt[2], kt[3]);
+      *reinterpret_cast<uint2*>(Kth + r * D + c4) =
+          make_uint2(*reinterpret_cast<const uint32_t*>(&h0), *reinterpret_cast<const uint32_t*>(&h1));
+    }
   }
   if (tid < D) a.w.egl[p.ch * D + tid] = expf(gl[tid]);
   if (__syncthreads_or(bad) && tid == 0) set_status(a.status, KDA_ERR_RANGE);
@@ -440,10 +453,24 @@ __global__ void __launch_bounds__(NT, 1) cbwd_prep_kernel(CbwdArgs a) {
     float acc[2][NTD][4];
     zero4(acc);
     wmma3<2, NTD, false, SPLIT>(acc, As, LDC, 1, Kx, LDD, 1, CH, m0, n0, lane);
-    float* W = a.w.W + p.ch * CH * D;
-    FRAG_LOOP(2, NTD) {
-      const int r = FRAG_R(m0), c = FRAG_C(n0);
-      W[r * D + c] = acc[mt][nt][i] * egm[c];
+    if (SPLIT) {
+      float* W = a.w.W + p.ch * CH * D;
+      FRAG_LOOP(2, NTD) {
+        const int r = FRAG_R(m0), c = FRAG_C(n0);
+        W[r * D + c] = acc[mt][nt][i] * egm[c];
+      }
+    } else {   // fp16 operand of the chains
+      __half* W = reinterpret_cast<__half*>(a.w.W) + p.ch * CH * D;
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < NTD; ++nt)
+#pragma unroll
+          for (int hi = 0; hi < 2; ++hi) {
+            const int r = m0 + 16 * mt + g + 8 * hi, c = n0 + 8 * nt + 2 * t;
+            *reinterpret_cast<__half2*>(W + r * D + c) =
+                __floats2half2_rn(acc[mt][nt][2 * hi] * egm[c], acc[mt][nt][2 * hi + 1] * egm[c + 1]);
+          }
     }
     zero4(acc);
     wmma3<2, NTD, false, SPLIT>(acc, As, LDC, 1, KN, LDD, 1, CH, m0, n0, lane);
@@ -589,6 +616,192 @@ __global__ void __launch_bounds__(NT, 1) cbwd_chain_kernel(CbwdArgs a) {
       a.dS0[(bh * D + r) * D + c0 + j] = S[r * LS + j];
     }
   }
+}
+
+// ---- the two chains of bf16 problems: fp16 operands, one launch ---------------------------
+// W and Kt arrive in fp16 (written so by the prep kernel) and the state (or its gradient) and U
+// (or dU) are rounded to fp16 as they enter a product, which accumulates in fp32 on mma.sync
+// m16n8k16: the operand precision of the forward's tensor-core state pass.  The state itself stays
+// fp32 in shared memory.  The forward chain (S of every chunk) and the reverse chain (dS) do not
+// depend on each other, so both run in one launch, blockIdx.z = 2 b + direction, two CTAs per SM.
+// Row strides: the fp16 tiles D + 8 halves (ldmatrix rows 16-byte aligned, 4 mod 32 words: free
+// of bank conflicts); the fp32 state and U columns CW + 4 (rows 2t and 2t + 1 of a B fragment
+// fall in distinct banks).
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+__device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+  asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+               : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+               : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+// two fp32 values as an fp16 pair, lo in the low half (the smaller k of a B fragment)
+__device__ __forceinline__ uint32_t h2_bits(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+template <int D>
+struct ChainH {
+  static constexpr int LH = D + 8, LS = CW + 4;
+};
+
+template <int D>
+constexpr size_t chain_h_smem() {
+  using L = ChainH<D>;
+  return sizeof(__half) * 2 * 2 * CH * L::LH +
+         sizeof(float) * (2 * CH * CW + 2 * D * CW + 2 * D + D * L::LS + CH * L::LS);
+}
+
+template <int D, bool BWD>
+__device__ __forceinline__ void chain_h_pass(const CbwdArgs& a, int b, uint8_t* smraw) {
+  using L = ChainH<D>;
+  constexpr int LH = L::LH, LS = L::LS;
+  __half* T1 = reinterpret_cast<__half*>(smraw);           // [2][CH][LH] W (forward) or Kt (backward)
+  __half* T2 = T1 + 2 * CH * LH;                            // [2][CH][LH] Kt (forward) or W (backward)
+  float* Vb = reinterpret_cast<float*>(T2 + 2 * CH * LH);   // [2][CH][CW] U~ (forward) or Z (backward)
+  float* Yb = Vb + 2 * CH * CW;                             // [2][D][CW]  Y columns (backward)
+  float* eb = Yb + 2 * D * CW;                              // [2][D]      e^{gl}
+  float* S = eb + 2 * D;                                    // [D][LS]     state or its gradient
+  float* Us = S + D * LS;                                   // [CH][LS]    U or dU
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int c0 = blockIdx.x * CW, h = blockIdx.y;
+  const int64_t bh = (int64_t)b * a.H + h, ch0 = bh * a.nc;
+  const float* init = BWD ? a.dSN : a.S0;
+  for (int idx = tid; idx < D * CW; idx += NT) {
+    const int r = idx / CW, j = idx % CW;
+    S[r * LS + j] = init ? init[(bh * D + r) * D + c0 + j] : 0.f;
+  }
+  const __half* H1 = reinterpret_cast<const __half*>(BWD ? a.w.Kt : a.w.W);
+  const __half* H2 = reinterpret_cast<const __half*>(BWD ? a.w.W : a.w.Kt);
+  auto issue = [&](int c) {
+    if (c >= 0 && c < a.nc) {
+      const int s = c & 1;
+      const int64_t ch = ch0 + c;
+      const __half* M1 = H1 + ch * CH * D;
+      const __half* M2 = H2 + ch * CH * D;
+      const float* V = (BWD ? a.w.Z : a.w.Ut) + ch * CH * D;
+      for (int i = tid; i < CH * D / 8; i += NT) {
+        const int r = i / (D / 8), c8 = (i % (D / 8)) * 8;
+        cp_async16v(T1 + (s * CH + r) * LH + c8, M1 + r * D + c8);
+        cp_async16v(T2 + (s * CH + r) * LH + c8, M2 + r * D + c8);
+      }
+      for (int i = tid; i < CH * CW / 4; i += NT) {
+        const int r = i / (CW / 4), c4 = (i % (CW / 4)) * 4;
+        cp_async16(Vb + (s * CH + r) * CW + c4, V + r * D + c0 + c4);
+      }
+      if (BWD) {
+        const float* Y = a.w.Y + ch * D * D;
+        for (int i = tid; i < D * CW / 4; i += NT) {
+          const int r = i / (CW / 4), c4 = (i % (CW / 4)) * 4;
+          cp_async16(Yb + (s * D + r) * CW + c4, Y + r * D + c0 + c4);
+        }
+      }
+      for (int i = tid; i < D / 4; i += NT) cp_async16(eb + s * D + 4 * i, a.w.egl + ch * D + 4 * i);
+    }
+    cp_async_commit();
+  };
+  // warp tiles: the CH x CW product as 4 x 2 tiles of 16 x 8, one per warp; the D x CW product
+  // as (D / 16) x 2 tiles, D / 64 per warp
+  const int g = lane >> 2, t = lane & 3;
+  const int m1 = 16 * (warp & 3), n1 = 8 * (warp >> 2);
+  constexpr int MT2 = D / 64;
+  const int m2 = 16 * MT2 * (warp & 3), n2 = 8 * (warp >> 2);
+  // ldmatrix row addresses: the A fragment of a row-major tile (rows m, 16-half steps along k) and
+  // of a tile stored transposed (rows k, the fragment's m along the row)
+  const int ar = (lane & 7) + 8 * ((lane >> 3) & 1), ac = 8 * (lane >> 4);
+  const int tr = (lane & 7) + 8 * (lane >> 4), tc = 8 * ((lane >> 3) & 1);
+  const uint32_t t1_0 = (uint32_t)__cvta_generic_to_shared(T1 + (m1 + ar) * LH + ac);
+  const uint32_t t2_0 = (uint32_t)__cvta_generic_to_shared(T2 + tr * LH + m2 + tc);
+  issue(BWD ? a.nc - 1 : 0);
+  for (int step = 0; step < a.nc; ++step) {
+    const int c = BWD ? a.nc - 1 - step : step;
+    const int s = c & 1;
+    const int64_t ch = ch0 + c;
+    cp_async_wait_all();
+    __syncthreads();   // chunk c's tiles in place; every thread is done with the other buffer
+    issue(BWD ? c - 1 : c + 1);
+    {  // the state entering the chunk (forward) or the gradient reaching its exit (backward)
+      float* out = (BWD ? a.w.dS : a.w.S) + ch * D * D;
+      for (int idx = tid; idx < D * CW; idx += NT) {
+        const int r = idx / CW, j = idx % CW;
+        out[r * D + c0 + j] = S[r * LS + j];
+      }
+    }
+    {  // forward: U = U~ - W S;  backward: dU = Z + Kt dS
+      float u[4] = {0.f, 0.f, 0.f, 0.f}, u2[4] = {0.f, 0.f, 0.f, 0.f};
+      const uint32_t abase = t1_0 + (uint32_t)(s * CH * LH * 2);
+      const float* sb = S + 2 * t * LS + n1 + g;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        uint32_t af[4], bf[2];
+        ldsm_x4(af, abase + 32u * kk);
+        const float* pb = sb + 16 * kk * LS;
+        bf[0] = h2_bits(pb[0], pb[LS]);
+        bf[1] = h2_bits(pb[8 * LS], pb[9 * LS]);
+        mma_f16((kk & 1) ? u2 : u, af, bf);
+      }
+      float* out = (BWD ? a.w.dU : a.w.U) + ch * CH * D;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = m1 + g + 8 * (i >> 1), j = n1 + 2 * t + (i & 1);
+        const float prod = u[i] + u2[i];
+        const float val = BWD ? Vb[(s * CH + r) * CW + j] + prod : Vb[(s * CH + r) * CW + j] - prod;
+        Us[r * LS + j] = val;
+        out[r * D + c0 + j] = val;
+      }
+    }
+    __syncthreads();
+    {  // forward: S = Diag(e^{gl}) S + Kt^T U;  backward: dS = Diag(e^{gl}) dS - W^T dU + Y
+      float sv[MT2][4];
+#pragma unroll
+      for (int mt = 0; mt < MT2; ++mt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) sv[mt][i] = 0.f;
+      const uint32_t abase = t2_0 + (uint32_t)(s * CH * LH * 2);
+      const float* ub = Us + 2 * t * LS + n2 + g;
+#pragma unroll
+      for (int kk = 0; kk < CH / 16; ++kk) {
+        uint32_t bf[2];
+        const float* pb = ub + 16 * kk * LS;
+        bf[0] = h2_bits(pb[0], pb[LS]);
+        bf[1] = h2_bits(pb[8 * LS], pb[9 * LS]);
+#pragma unroll
+        for (int mt = 0; mt < MT2; ++mt) {
+          uint32_t af[4];
+          ldsm_x4_t(af, abase + (uint32_t)((16 * kk * LH + 16 * mt) * 2));
+          mma_f16(sv[mt], af, bf);
+        }
+      }
+#pragma unroll
+      for (int mt = 0; mt < MT2; ++mt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = m2 + 16 * mt + g + 8 * (i >> 1), j = n2 + 2 * t + (i & 1);
+          const float prev = eb[s * D + r] * S[r * LS + j];
+          S[r * LS + j] = BWD ? prev - sv[mt][i] + Yb[(s * D + r) * CW + j] : prev + sv[mt][i];
+        }
+    }
+  }
+  if (BWD && a.dS0) {
+    __syncthreads();
+    for (int idx = tid; idx < D * CW; idx += NT) {
+      const int r = idx / CW, j = idx % CW;
+      a.dS0[(bh * D + r) * D + c0 + j] = S[r * LS + j];
+    }
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(NT, 2) cbwd_chain_h_kernel(CbwdArgs a) {
+  extern __shared__ __align__(16) uint8_t smh[];
+  if (blockIdx.z & 1) chain_h_pass<D, true>(a, (int)(blockIdx.z >> 1), smh);
+  else chain_h_pass<D, false>(a, (int)(blockIdx.z >> 1), smh);
 }
 
 // ---- contractions with the chunk's entry state and exit gradient -------------------------
@@ -1024,8 +1237,9 @@ cudaError_t set_smem(K kernel, size_t bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
-// SPLIT: the per-chunk kernels' products at fp32 accuracy (fp32 problems); bf16 problems take one
-// tf32 product there.  The chains always split: their error compounds from chunk to chunk.
+// SPLIT: every product at fp32 accuracy (fp32 problems: split tf32 products, fp32 chain
+// operands).  bf16 problems take one tf32 product of rounded operands in the per-chunk kernels and
+// fp16 operands in the chains, which run together in one launch.
 template <int D, bool SPLIT>
 cudaError_t launch_scan_bwd(const CbwdArgs& a, const Dims& d, cudaStream_t s) {
   cudaError_t e;
@@ -1033,10 +1247,16 @@ cudaError_t launch_scan_bwd(const CbwdArgs& a, const Dims& d, cudaStream_t s) {
   const dim3 cols((unsigned)(D / CW), (unsigned)d.H, (unsigned)d.B);
   if ((e = set_smem(cbwd_prep_kernel<D, SPLIT>, prep_smem<D>())) != cudaSuccess) return e;
   cbwd_prep_kernel<D, SPLIT><<<chunks, NT, prep_smem<D>(), s>>>(a);
-  if ((e = set_smem(cbwd_chain_kernel<D, false>, chain_smem<D, false>())) != cudaSuccess) return e;
-  cbwd_chain_kernel<D, false><<<cols, NT, chain_smem<D, false>(), s>>>(a);
-  if ((e = set_smem(cbwd_chain_kernel<D, true>, chain_smem<D, true>())) != cudaSuccess) return e;
-  cbwd_chain_kernel<D, true><<<cols, NT, chain_smem<D, true>(), s>>>(a);
+  if (SPLIT) {
+    if ((e = set_smem(cbwd_chain_kernel<D, false>, chain_smem<D, false>())) != cudaSuccess) return e;
+    cbwd_chain_kernel<D, false><<<cols, NT, chain_smem<D, false>(), s>>>(a);
+    if ((e = set_smem(cbwd_chain_kernel<D, true>, chain_smem<D, true>())) != cudaSuccess) return e;
+    cbwd_chain_kernel<D, true><<<cols, NT, chain_smem<D, true>(), s>>>(a);
+  } else {
+    const dim3 both((unsigned)(D / CW), (unsigned)d.H, (unsigned)(2 * d.B));
+    if ((e = set_smem(cbwd_chain_h_kernel<D>, chain_h_smem<D>())) != cudaSuccess) return e;
+    cbwd_chain_h_kernel<D><<<both, NT, chain_h_smem<D>(), s>>>(a);
+  }
   if ((e = set_smem(cbwd_state_grad_kernel<D, SPLIT>, state_grad_smem<D>())) != cudaSuccess) return e;
   cbwd_state_grad_kernel<D, SPLIT><<<chunks, NT, state_grad_smem<D>(), s>>>(a);
   if ((e = set_smem(cbwd_local_grad_kernel<D, SPLIT>, local_grad_smem<D>())) != cudaSuccess) return e;

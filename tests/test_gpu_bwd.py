@@ -7,6 +7,7 @@ fp32 bound (1e-5) for fp32 problems; for bf16 problems within the bf16 bounds
 magnitude, since gradients carry the scale of d_o rather than of o).
 """
 import dataclasses
+import os
 
 import numpy as np
 import pytest
@@ -50,9 +51,14 @@ def run_bwd(kda, w, inp, dO, S0=None, dSN=None, causal=False, status=None):
 
 
 def check(got, ref, dtype):
+    log = os.environ.get("KDA_PARITY_LOG")
     for n in ("dq", "dk", "dv", "dla", "dbeta", "dw_text", "dw_vis", "dS0"):
         x, r = got[n].reshape(ref[n].shape), ref[n]
         e = rel_l2(x, r)
+        if log:   # one line per gradient, for reporting the measured errors
+            m = float(np.abs(x - r).max() / max(np.abs(r).max(), 1e-30)) if r.size else 0.0
+            with open(log, "a") as f:
+                f.write(f"{os.environ.get('PYTEST_CURRENT_TEST', '?').split(' ')[0]}\t{n}\t{dtype}\t{e:.3e}\t{m:.3e}\n")
         if dtype == "f32":
             assert e <= 1e-5, f"{n}: rel_l2={e:.3e}"
         else:
@@ -120,6 +126,9 @@ def test_bwd_bf16_full_size_sampled_v_columns(kda):
     x = np.stack([got["dv"][:, :, h, j] for h, j in items])
     e = rel_l2(x, ref)
     m = float(np.abs(x - ref).max() / np.abs(ref).max())
+    if os.environ.get("KDA_PARITY_LOG"):
+        with open(os.environ["KDA_PARITY_LOG"], "a") as f:
+            f.write(f"test_bwd_bf16_full_size_sampled_v_columns\tdv columns\tbf16\t{e:.3e}\t{m:.3e}\n")
     assert e <= 5e-3 and m <= 2e-2, f"dv columns: rel_l2={e:.3e} rel max-abs={m:.3e}"
 
 
@@ -143,3 +152,21 @@ def test_bwd_bf16_d64(kda):
     """bf16 with d = 64 (the per-chunk kernels' single-product mode at D = 64), 13 text tokens + 3 x 5 x 7."""
     w = kda_synth.Workload("bwd_bf16_d64", 1, 2, 64, 13, (3, 5, 7), "bf16", 0.1)
     _case(kda, w, 38)
+
+
+def test_bwd_bf16_long_chain(kda):
+    """bf16, d = 128, 33 chunks (the last one ragged) under slow decay (log alpha near -0.02), so the
+    chains' fp16 operand roundings compound over many chunks: every gradient against the oracle."""
+    w = kda_synth.Workload("bwd_bf16_long", 1, 2, 128, 64, (4, 16, 32), "bf16", 0.02)
+    _case(kda, w, 39)
+
+
+def test_bwd_bf16_strong_decay_inside_a_chunk(kda):
+    """bf16, d = 128: 37 nats of decay inside one chunk in one channel (W and Kt of that chunk span
+    e^-37 in fp16, below its normal range) still matches the oracle."""
+    w = kda_synth.Workload("bwd_bf16", 1, 4, 128, 64, (3, 8, 8), "bf16", 0.1)
+    inp = kda_synth.generate(w, 40)
+    B, N, H, d = inp["shape"]
+    la = inp["log_alpha"].reshape(B, N, H, d).copy()
+    la[0, 70:107, 2, 9] = -1.0
+    _case(kda, w, 40, inp=dict(inp, log_alpha=la.reshape(inp["log_alpha"].shape)))
