@@ -358,7 +358,7 @@ def bwd_arm(args, w, idx, rank, world, local_rank):
             "metric": "KDA+shortconv bwd tokens/sec on 1 B200", "value": w.tokens * world / (ms * 1e-3),
             "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "tf32 per-chunk products, split-tf32 chains, f32 accumulation, bf16 storage"
+            "dtype": "tf32 per-chunk products, fp16 chain operands, f32 accumulation, bf16 storage"
             if w.dtype == "bf16" else "f32 (split-tf32 tensor products)", "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "N": w.N, "H": w.H, "d": w.d, "text_len": w.text_len,
                        "grid": list(w.grid), "pass": "backward", "parallelism": f"replicas{world}",

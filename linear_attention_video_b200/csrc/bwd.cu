@@ -619,14 +619,15 @@ __global__ void __launch_bounds__(NT, 1) cbwd_chain_kernel(CbwdArgs a) {
 }
 
 // ---- the two chains of bf16 problems: fp16 operands, one launch ---------------------------
-// W and Kt arrive in fp16 (written so by the prep kernel) and the state (or its gradient) and U
-// (or dU) are rounded to fp16 as they enter a product, which accumulates in fp32 on mma.sync
-// m16n8k16: the operand precision of the forward's tensor-core state pass.  The state itself stays
-// fp32 in shared memory.  The forward chain (S of every chunk) and the reverse chain (dS) do not
-// depend on each other, so both run in one launch, blockIdx.z = 2 b + direction, two CTAs per SM.
-// Row strides: the fp16 tiles D + 8 halves (ldmatrix rows 16-byte aligned, 4 mod 32 words: free
-// of bank conflicts); the fp32 state and U columns CW + 4 (rows 2t and 2t + 1 of a B fragment
-// fall in distinct banks).
+// W and Kt arrive in fp16 (written so by the prep kernel), and the state (or its gradient) and U
+// (or dU) enter the products as fp16 images, which accumulate in fp32 on mma.sync m16n8k16: the
+// operand precision of the forward's tensor-core state pass.  The state itself stays fp32 in
+// shared memory; each update also writes its fp16 image, transposed (value column major) so that
+// the B fragments of both products load by ldmatrix, like the A fragments.  The forward chain (S
+// of every chunk) and the reverse chain (dS) do not depend on each other, so both run in one
+// launch, blockIdx.z = 2 b + direction, two CTAs per SM.  Row strides: the fp16 tiles and images
+// a multiple of 16 bytes and 4 mod 32 words (ldmatrix free of bank conflicts); the fp32 state CW + 8
+// (the update's 8-byte accesses free of bank conflicts).
 __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
@@ -640,42 +641,42 @@ __device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], c
                : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
                : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
-// two fp32 values as an fp16 pair, lo in the low half (the smaller k of a B fragment)
-__device__ __forceinline__ uint32_t h2_bits(float lo, float hi) {
-  const __half2 h = __floats2half2_rn(lo, hi);
-  return *reinterpret_cast<const uint32_t*>(&h);
-}
-
 template <int D>
 struct ChainH {
-  static constexpr int LH = D + 8, LS = CW + 4;
+  static constexpr int LH = D + 8;    // W / Kt tiles, halves per row
+  static constexpr int LT = D + 8;    // fp16 image of the state, [CW][LT]: value column major
+  static constexpr int LU = CH + 8;   // fp16 image of U, [CW][LU]
+  static constexpr int LS = CW + 8;   // fp32 state, [D][LS]
 };
 
 template <int D>
 constexpr size_t chain_h_smem() {
   using L = ChainH<D>;
-  return sizeof(__half) * 2 * 2 * CH * L::LH +
-         sizeof(float) * (2 * CH * CW + 2 * D * CW + 2 * D + D * L::LS + CH * L::LS);
+  return sizeof(__half) * (2 * 2 * CH * L::LH + CW * L::LT + CW * L::LU) +
+         sizeof(float) * (2 * CH * CW + 2 * D * CW + 2 * D + D * L::LS);
 }
 
 template <int D, bool BWD>
 __device__ __forceinline__ void chain_h_pass(const CbwdArgs& a, int b, uint8_t* smraw) {
   using L = ChainH<D>;
-  constexpr int LH = L::LH, LS = L::LS;
+  constexpr int LH = L::LH, LT = L::LT, LU = L::LU, LS = L::LS;
   __half* T1 = reinterpret_cast<__half*>(smraw);           // [2][CH][LH] W (forward) or Kt (backward)
   __half* T2 = T1 + 2 * CH * LH;                            // [2][CH][LH] Kt (forward) or W (backward)
-  float* Vb = reinterpret_cast<float*>(T2 + 2 * CH * LH);   // [2][CH][CW] U~ (forward) or Z (backward)
+  __half* ST = T2 + 2 * CH * LH;                            // [CW][LT]    fp16 state, transposed
+  __half* UT = ST + CW * LT;                                // [CW][LU]    fp16 U or dU, transposed
+  float* Vb = reinterpret_cast<float*>(UT + CW * LU);       // [2][CH][CW] U~ (forward) or Z (backward)
   float* Yb = Vb + 2 * CH * CW;                             // [2][D][CW]  Y columns (backward)
   float* eb = Yb + 2 * D * CW;                              // [2][D]      e^{gl}
   float* S = eb + 2 * D;                                    // [D][LS]     state or its gradient
-  float* Us = S + D * LS;                                   // [CH][LS]    U or dU
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int c0 = blockIdx.x * CW, h = blockIdx.y;
   const int64_t bh = (int64_t)b * a.H + h, ch0 = bh * a.nc;
   const float* init = BWD ? a.dSN : a.S0;
   for (int idx = tid; idx < D * CW; idx += NT) {
     const int r = idx / CW, j = idx % CW;
-    S[r * LS + j] = init ? init[(bh * D + r) * D + c0 + j] : 0.f;
+    const float v = init ? init[(bh * D + r) * D + c0 + j] : 0.f;
+    S[r * LS + j] = v;
+    ST[j * LT + r] = __float2half_rn(v);
   }
   const __half* H1 = reinterpret_cast<const __half*>(BWD ? a.w.Kt : a.w.W);
   const __half* H2 = reinterpret_cast<const __half*>(BWD ? a.w.W : a.w.Kt);
@@ -712,48 +713,56 @@ __device__ __forceinline__ void chain_h_pass(const CbwdArgs& a, int b, uint8_t* 
   const int m1 = 16 * (warp & 3), n1 = 8 * (warp >> 2);
   constexpr int MT2 = D / 64;
   const int m2 = 16 * MT2 * (warp & 3), n2 = 8 * (warp >> 2);
-  // ldmatrix row addresses: the A fragment of a row-major tile (rows m, 16-half steps along k) and
-  // of a tile stored transposed (rows k, the fragment's m along the row)
+  // ldmatrix row addresses.  A of a row-major tile (rows m, 16-half steps along k): matrices
+  // (m 0-7, k 0-7), (m 8-15, k 0-7), (m 0-7, k 8-15), (m 8-15, k 8-15).  A of a tile stored
+  // transposed (rows k): the same four, read with .trans.  B from a value-column-major image
+  // (rows n): matrices k 0-7, 8-15, 16-23, 24-31, i.e. the B fragments of two k-steps.
   const int ar = (lane & 7) + 8 * ((lane >> 3) & 1), ac = 8 * (lane >> 4);
   const int tr = (lane & 7) + 8 * (lane >> 4), tc = 8 * ((lane >> 3) & 1);
+  const int br = lane & 7, bc = 8 * (lane >> 3);
   const uint32_t t1_0 = (uint32_t)__cvta_generic_to_shared(T1 + (m1 + ar) * LH + ac);
   const uint32_t t2_0 = (uint32_t)__cvta_generic_to_shared(T2 + tr * LH + m2 + tc);
+  const uint32_t st_0 = (uint32_t)__cvta_generic_to_shared(ST + (n1 + br) * LT + bc);
+  const uint32_t ut_0 = (uint32_t)__cvta_generic_to_shared(UT + (n2 + br) * LU + bc);
   issue(BWD ? a.nc - 1 : 0);
   for (int step = 0; step < a.nc; ++step) {
     const int c = BWD ? a.nc - 1 - step : step;
     const int s = c & 1;
     const int64_t ch = ch0 + c;
     cp_async_wait_all();
-    __syncthreads();   // chunk c's tiles in place; every thread is done with the other buffer
+    __syncthreads();   // chunk c's tiles in place, the state and its image updated; every thread is
+                       // done with the other buffer
     issue(BWD ? c - 1 : c + 1);
     {  // the state entering the chunk (forward) or the gradient reaching its exit (backward)
       float* out = (BWD ? a.w.dS : a.w.S) + ch * D * D;
-      for (int idx = tid; idx < D * CW; idx += NT) {
-        const int r = idx / CW, j = idx % CW;
-        out[r * D + c0 + j] = S[r * LS + j];
+#pragma unroll
+      for (int i = 0; i < D * CW / 4 / NT; ++i) {
+        const int idx = tid + i * NT, r = idx / (CW / 4), j4 = (idx % (CW / 4)) * 4;
+        *reinterpret_cast<float4*>(out + r * D + c0 + j4) = *reinterpret_cast<const float4*>(S + r * LS + j4);
       }
     }
     {  // forward: U = U~ - W S;  backward: dU = Z + Kt dS
       float u[4] = {0.f, 0.f, 0.f, 0.f}, u2[4] = {0.f, 0.f, 0.f, 0.f};
       const uint32_t abase = t1_0 + (uint32_t)(s * CH * LH * 2);
-      const float* sb = S + 2 * t * LS + n1 + g;
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        uint32_t af[4], bf[2];
-        ldsm_x4(af, abase + 32u * kk);
-        const float* pb = sb + 16 * kk * LS;
-        bf[0] = h2_bits(pb[0], pb[LS]);
-        bf[1] = h2_bits(pb[8 * LS], pb[9 * LS]);
-        mma_f16((kk & 1) ? u2 : u, af, bf);
+      for (int k2 = 0; k2 < D / 32; ++k2) {
+        uint32_t bq[4], af[4];
+        ldsm_x4(bq, st_0 + 64u * k2);
+        ldsm_x4(af, abase + 64u * k2);
+        mma_f16(u, af, {bq[0], bq[1]});
+        ldsm_x4(af, abase + 64u * k2 + 32u);
+        mma_f16(u2, af, {bq[2], bq[3]});
       }
       float* out = (BWD ? a.w.dU : a.w.U) + ch * CH * D;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int r = m1 + g + 8 * (i >> 1), j = n1 + 2 * t + (i & 1);
-        const float prod = u[i] + u2[i];
-        const float val = BWD ? Vb[(s * CH + r) * CW + j] + prod : Vb[(s * CH + r) * CW + j] - prod;
-        Us[r * LS + j] = val;
-        out[r * D + c0 + j] = val;
+      for (int hi = 0; hi < 2; ++hi) {
+        const int r = m1 + g + 8 * hi, j = n1 + 2 * t;
+        const float2 vb = *reinterpret_cast<const float2*>(Vb + (s * CH + r) * CW + j);
+        const float p0 = u[2 * hi] + u2[2 * hi], p1 = u[2 * hi + 1] + u2[2 * hi + 1];
+        const float v0 = BWD ? vb.x + p0 : vb.x - p0, v1 = BWD ? vb.y + p1 : vb.y - p1;
+        UT[j * LU + r] = __float2half_rn(v0);
+        UT[(j + 1) * LU + r] = __float2half_rn(v1);
+        *reinterpret_cast<float2*>(out + r * D + c0 + j) = make_float2(v0, v1);
       }
     }
     __syncthreads();
@@ -764,27 +773,38 @@ __device__ __forceinline__ void chain_h_pass(const CbwdArgs& a, int b, uint8_t* 
 #pragma unroll
         for (int i = 0; i < 4; ++i) sv[mt][i] = 0.f;
       const uint32_t abase = t2_0 + (uint32_t)(s * CH * LH * 2);
-      const float* ub = Us + 2 * t * LS + n2 + g;
 #pragma unroll
-      for (int kk = 0; kk < CH / 16; ++kk) {
-        uint32_t bf[2];
-        const float* pb = ub + 16 * kk * LS;
-        bf[0] = h2_bits(pb[0], pb[LS]);
-        bf[1] = h2_bits(pb[8 * LS], pb[9 * LS]);
+      for (int k2 = 0; k2 < CH / 32; ++k2) {
+        uint32_t bq[4];
+        ldsm_x4(bq, ut_0 + 64u * k2);
 #pragma unroll
-        for (int mt = 0; mt < MT2; ++mt) {
-          uint32_t af[4];
-          ldsm_x4_t(af, abase + (uint32_t)((16 * kk * LH + 16 * mt) * 2));
-          mma_f16(sv[mt], af, bf);
+        for (int half = 0; half < 2; ++half) {
+          const int kk = 2 * k2 + half;
+#pragma unroll
+          for (int mt = 0; mt < MT2; ++mt) {
+            uint32_t af[4];
+            ldsm_x4_t(af, abase + (uint32_t)((16 * kk * LH + 16 * mt) * 2));
+            mma_f16(sv[mt], af, {bq[2 * half], bq[2 * half + 1]});
+          }
         }
       }
 #pragma unroll
       for (int mt = 0; mt < MT2; ++mt)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int r = m2 + 16 * mt + g + 8 * (i >> 1), j = n2 + 2 * t + (i & 1);
-          const float prev = eb[s * D + r] * S[r * LS + j];
-          S[r * LS + j] = BWD ? prev - sv[mt][i] + Yb[(s * D + r) * CW + j] : prev + sv[mt][i];
+        for (int hi = 0; hi < 2; ++hi) {
+          const int r = m2 + 16 * mt + g + 8 * hi, j = n2 + 2 * t;
+          const float e = eb[s * D + r];
+          float2 sp = *reinterpret_cast<const float2*>(S + r * LS + j);
+          const float a0 = sv[mt][2 * hi], a1 = sv[mt][2 * hi + 1];
+          if (BWD) {
+            const float2 y = *reinterpret_cast<const float2*>(Yb + (s * D + r) * CW + j);
+            sp = make_float2(e * sp.x - a0 + y.x, e * sp.y - a1 + y.y);
+          } else {
+            sp = make_float2(e * sp.x + a0, e * sp.y + a1);
+          }
+          *reinterpret_cast<float2*>(S + r * LS + j) = sp;
+          ST[j * LT + r] = __float2half_rn(sp.x);
+          ST[(j + 1) * LT + r] = __float2half_rn(sp.y);
         }
     }
   }
