@@ -170,3 +170,16 @@ def test_bwd_bf16_strong_decay_inside_a_chunk(kda):
     la = inp["log_alpha"].reshape(B, N, H, d).copy()
     la[0, 70:107, 2, 9] = -1.0
     _case(kda, w, 40, inp=dict(inp, log_alpha=la.reshape(inp["log_alpha"].shape)))
+
+
+@pytest.mark.parametrize("case", ["batch2_ragged", "causal_t", "text_only"])
+def test_bwd_bf16_edge_shapes(kda, case):
+    """bf16, d = 128 (the fp16 chains, whose launch interleaves batch items and directions in
+    blockIdx.z): two batch items with a ragged last chunk, the temporally causal conv, text only."""
+    w = kda_synth.Workload("bwd_bf16_edge", 1, 2, 128, 13, (2, 7, 9), "bf16", 0.1)
+    if case == "batch2_ragged":
+        _case(kda, dataclasses.replace(w, B=2), 41)
+    elif case == "causal_t":
+        _case(kda, w, 42, causal=True)
+    else:
+        _case(kda, dataclasses.replace(w, text_len=150, grid=(0, 0, 0)), 43)
