@@ -314,6 +314,27 @@ __device__ __forceinline__ ChunkPos chunk_pos(const CbwdArgs& a) {
 #define FRAG_R(m0) ((m0) + 16 * mt + g + 8 * (i >> 1))
 #define FRAG_C(n0) ((n0) + 8 * nt + 2 * t + (i & 1))
 
+// A warp's accumulator tiles into a row-major [.][ld] array at element offset off: fp32, or, for
+// bf16 problems (!SPLIT), fp16 at the same element offset (the chains' additive terms)
+template <int MT, int NT_, bool SPLIT>
+__device__ __forceinline__ void store_tile(float* base, int64_t off, int ld, const float (&acc)[MT][NT_][4], int m0,
+                                           int n0, int g, int t) {
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+    for (int nt = 0; nt < NT_; ++nt)
+#pragma unroll
+      for (int hi = 0; hi < 2; ++hi) {
+        const int r = m0 + 16 * mt + g + 8 * hi, c = n0 + 8 * nt + 2 * t;
+        if (SPLIT) {
+          *reinterpret_cast<float2*>(base + off + r * ld + c) = make_float2(acc[mt][nt][2 * hi], acc[mt][nt][2 * hi + 1]);
+        } else {
+          *reinterpret_cast<__half2*>(reinterpret_cast<__half*>(base) + off + r * ld + c) =
+              __floats2half2_rn(acc[mt][nt][2 * hi], acc[mt][nt][2 * hi + 1]);
+        }
+      }
+}
+
 template <int D>
 constexpr size_t prep_smem() { return sizeof(float) * (4 * CH * (D + 4) + 2 * CH * LDC + 4 * D + CH); }
 
@@ -474,23 +495,18 @@ __global__ void __launch_bounds__(NT, 1) cbwd_prep_kernel(CbwdArgs a) {
     }
     zero4(acc);
     wmma3<2, NTD, false, SPLIT>(acc, As, LDC, 1, KN, LDD, 1, CH, m0, n0, lane);
-    float* Ut = a.w.Ut + p.ch * CH * D;
-    FRAG_LOOP(2, NTD) Ut[FRAG_R(m0) * D + FRAG_C(n0)] = acc[mt][nt][i];
+    store_tile<2, NTD, SPLIT>(a.w.Ut, p.ch * CH * D, D, acc, m0, n0, g, t);
     zero4(acc);
     wmma3<2, NTD, false, SPLIT>(acc, Ps, 1, LDC, Gs, LDD, 1, CH, m0, n0, lane);
-    float* Z = a.w.Z + p.ch * CH * D;
-    FRAG_LOOP(2, NTD) Z[FRAG_R(m0) * D + FRAG_C(n0)] = acc[mt][nt][i];
+    store_tile<2, NTD, SPLIT>(a.w.Z, p.ch * CH * D, D, acc, m0, n0, g, t);
   }
   {  // Y = QG^T dO = Diag(e^{g_m}) Qx^T dO
     const int m0 = (D / 4) * (warp & 3), n0 = (D / 2) * (warp >> 2);
     float acc[D / 64][D / 16][4];
     zero4(acc);
     wmma3<D / 64, D / 16, false, SPLIT>(acc, Qx, 1, LDD, Gs, LDD, 1, CH, m0, n0, lane);
-    float* Y = a.w.Y + p.ch * D * D;
-    FRAG_LOOP(D / 64, D / 16) {
-      const int r = FRAG_R(m0);
-      Y[r * D + FRAG_C(n0)] = acc[mt][nt][i] * egm[r];
-    }
+    FRAG_LOOP(D / 64, D / 16) acc[mt][nt][i] *= egm[FRAG_R(m0)];
+    store_tile<D / 64, D / 16, SPLIT>(a.w.Y, p.ch * D * D, D, acc, m0, n0, g, t);
   }
 }
 
@@ -652,8 +668,8 @@ struct ChainH {
 template <int D>
 constexpr size_t chain_h_smem() {
   using L = ChainH<D>;
-  return sizeof(__half) * (2 * 2 * CH * L::LH + CW * L::LT + CW * L::LU) +
-         sizeof(float) * (2 * CH * CW + 2 * D * CW + 2 * D + D * L::LS);
+  return sizeof(__half) * (2 * 2 * CH * L::LH + CW * L::LT + CW * L::LU + 2 * CH * CW + 2 * D * CW) +
+         sizeof(float) * (2 * D + D * L::LS);
 }
 
 template <int D, bool BWD>
@@ -664,9 +680,9 @@ __device__ __forceinline__ void chain_h_pass(const CbwdArgs& a, int b, uint8_t* 
   __half* T2 = T1 + 2 * CH * LH;                            // [2][CH][LH] Kt (forward) or W (backward)
   __half* ST = T2 + 2 * CH * LH;                            // [CW][LT]    fp16 state, transposed
   __half* UT = ST + CW * LT;                                // [CW][LU]    fp16 U or dU, transposed
-  float* Vb = reinterpret_cast<float*>(UT + CW * LU);       // [2][CH][CW] U~ (forward) or Z (backward)
-  float* Yb = Vb + 2 * CH * CW;                             // [2][D][CW]  Y columns (backward)
-  float* eb = Yb + 2 * D * CW;                              // [2][D]      e^{gl}
+  __half* Vb = UT + CW * LU;                                // [2][CH][CW] U~ (forward) or Z (backward), fp16
+  __half* Yb = Vb + 2 * CH * CW;                            // [2][D][CW]  Y columns (backward), fp16
+  float* eb = reinterpret_cast<float*>(Yb + 2 * D * CW);    // [2][D]      e^{gl}
   float* S = eb + 2 * D;                                    // [D][LS]     state or its gradient
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int c0 = blockIdx.x * CW, h = blockIdx.y;
@@ -686,21 +702,21 @@ __device__ __forceinline__ void chain_h_pass(const CbwdArgs& a, int b, uint8_t* 
       const int64_t ch = ch0 + c;
       const __half* M1 = H1 + ch * CH * D;
       const __half* M2 = H2 + ch * CH * D;
-      const float* V = (BWD ? a.w.Z : a.w.Ut) + ch * CH * D;
+      const __half* V = reinterpret_cast<const __half*>(BWD ? a.w.Z : a.w.Ut) + ch * CH * D;
       for (int i = tid; i < CH * D / 8; i += NT) {
         const int r = i / (D / 8), c8 = (i % (D / 8)) * 8;
         cp_async16v(T1 + (s * CH + r) * LH + c8, M1 + r * D + c8);
         cp_async16v(T2 + (s * CH + r) * LH + c8, M2 + r * D + c8);
       }
-      for (int i = tid; i < CH * CW / 4; i += NT) {
-        const int r = i / (CW / 4), c4 = (i % (CW / 4)) * 4;
-        cp_async16(Vb + (s * CH + r) * CW + c4, V + r * D + c0 + c4);
+      for (int i = tid; i < CH * CW / 8; i += NT) {
+        const int r = i / (CW / 8), c8 = (i % (CW / 8)) * 8;
+        cp_async16v(Vb + (s * CH + r) * CW + c8, V + r * D + c0 + c8);
       }
       if (BWD) {
-        const float* Y = a.w.Y + ch * D * D;
-        for (int i = tid; i < D * CW / 4; i += NT) {
-          const int r = i / (CW / 4), c4 = (i % (CW / 4)) * 4;
-          cp_async16(Yb + (s * D + r) * CW + c4, Y + r * D + c0 + c4);
+        const __half* Y = reinterpret_cast<const __half*>(a.w.Y) + ch * D * D;
+        for (int i = tid; i < D * CW / 8; i += NT) {
+          const int r = i / (CW / 8), c8 = (i % (CW / 8)) * 8;
+          cp_async16v(Yb + (s * D + r) * CW + c8, Y + r * D + c0 + c8);
         }
       }
       for (int i = tid; i < D / 4; i += NT) cp_async16(eb + s * D + 4 * i, a.w.egl + ch * D + 4 * i);
@@ -757,7 +773,7 @@ __device__ __forceinline__ void chain_h_pass(const CbwdArgs& a, int b, uint8_t* 
 #pragma unroll
       for (int hi = 0; hi < 2; ++hi) {
         const int r = m1 + g + 8 * hi, j = n1 + 2 * t;
-        const float2 vb = *reinterpret_cast<const float2*>(Vb + (s * CH + r) * CW + j);
+        const float2 vb = __half22float2(*reinterpret_cast<const __half2*>(Vb + (s * CH + r) * CW + j));
         const float p0 = u[2 * hi] + u2[2 * hi], p1 = u[2 * hi + 1] + u2[2 * hi + 1];
         const float v0 = BWD ? vb.x + p0 : vb.x - p0, v1 = BWD ? vb.y + p1 : vb.y - p1;
         UT[j * LU + r] = __float2half_rn(v0);
@@ -797,7 +813,7 @@ __device__ __forceinline__ void chain_h_pass(const CbwdArgs& a, int b, uint8_t* 
           float2 sp = *reinterpret_cast<const float2*>(S + r * LS + j);
           const float a0 = sv[mt][2 * hi], a1 = sv[mt][2 * hi + 1];
           if (BWD) {
-            const float2 y = *reinterpret_cast<const float2*>(Yb + (s * D + r) * CW + j);
+            const float2 y = __half22float2(*reinterpret_cast<const __half2*>(Yb + (s * D + r) * CW + j));
             sp = make_float2(e * sp.x - a0 + y.x, e * sp.y - a1 + y.y);
           } else {
             sp = make_float2(e * sp.x + a0, e * sp.y + a1);
