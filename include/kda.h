@@ -188,8 +188,8 @@ int kda_fwd_host(const kda_problem* p, kda_dtype dtype,
  * pass, the gradient reaching every chunk's exit by a reverse pass, and each chunk's token
  * gradients follow from the two).  The products run on the tensor cores: for fp32 problems in
  * tf32 split into two terms per operand (three products, fp32 accuracy); for bf16 problems one
- * tf32 product of rounded operands in the per-chunk passes and fp16 operands with fp32
- * accumulation in the passes over chunks (the state itself kept in fp32).
+ * tf32 product of rounded operands in the per-chunk passes and fp16 operands and additive terms
+ * with fp32 accumulation in the passes over chunks (the state itself kept in fp32).
  *   d_o                    [B, N, H, d] of dtype; d_final_state [B, H, d, d] fp32 or NULL (zero)
  *   dq, dk, dv             [B, N, H, d] of dtype: gradients of the raw (unconvolved) q, k, v
  *   d_log_alpha            [B, N, H, d] fp32;  d_beta [B, N, H] of dtype
