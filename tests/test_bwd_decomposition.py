@@ -29,21 +29,25 @@ def _chunk_prep(q, k, v, la, beta, dO, C, plant=False):
     return dict(W=W, Ut=T @ v, Kt=KN * np.exp(gl - gm)[None, :], Z=P.T @ dO, Y=Y, X=X, Ab=Ab, egl=np.exp(gl))
 
 
-def _decomposed_bwd(q, k, v, la, beta, dO, S0, dSN, C, plant=False):
+def _decomposed_bwd(q, k, v, la, beta, dO, S0, dSN, C, plant=False, h16=False):
+    """h16: the passes over chunks as bf16 problems run them: W, Kt, U~, Z, Y stored in fp16, and
+    the state (or its gradient) and U (or dU) rounded to fp16 where they enter a product."""
     N, D = q.shape
     pad = lambda a, s: np.concatenate([a[s], np.zeros((C - len(a[s]),) + a.shape[1:])])   # noqa: E731
+    h = (lambda a: a.astype(np.float16).astype(np.float64)) if h16 else (lambda a: a)   # noqa: E731
     chunks = [[pad(a, slice(s, s + C)) for a in (q, k, v, la, beta, dO)] for s in range(0, N, C)]
     pre = [_chunk_prep(*c, C, plant) for c in chunks]
+    hp = [{n: (h(x) if n in ("W", "Kt", "Ut", "Z", "Y") else x) for n, x in p.items()} for p in pre]
     S, U = [S0], []
-    for p in pre:                                   # forward pass over chunks
-        U.append(p["Ut"] - p["W"] @ S[-1])
-        S.append(p["egl"][:, None] * S[-1] + p["Kt"].T @ U[-1])
+    for p in hp:                                    # forward pass over chunks
+        U.append(p["Ut"] - p["W"] @ h(S[-1]))
+        S.append(p["egl"][:, None] * S[-1] + p["Kt"].T @ h(U[-1]))
     dS, dSx, dU = dSN, [None] * len(pre), [None] * len(pre)
     for i in range(len(pre) - 1, -1, -1):           # reverse pass
-        p = pre[i]
+        p = hp[i]
         dSx[i] = dS
-        dU[i] = p["Z"] + p["Kt"] @ dS
-        dS = p["egl"][:, None] * dS - p["W"].T @ dU[i] + p["Y"]
+        dU[i] = p["Z"] + p["Kt"] @ h(dS)
+        dS = p["egl"][:, None] * dS - p["W"].T @ h(dU[i]) + p["Y"]
     out = {n: [] for n in ("dq", "dk", "dv", "dla", "dbeta")}
     for i, (qc, kc, vc, lac, bc, dOc) in enumerate(chunks):
         p = pre[i]
@@ -107,3 +111,26 @@ def test_a_double_counted_chain_term_is_caught():
     ref = oracle.scan_bwd(q[None], k[None], v[None], la[None], beta[None], dO[None], S0[None], dSN[None])
     got = _decomposed_bwd(q, k, v, la, beta, dO, S0, dSN, C, plant=True)
     assert np.abs(got["dS0"] - ref["dS0"][0]).max() > 1e-3
+
+
+@pytest.mark.parametrize("la_scale", [0.02, 0.0])
+def test_fp16_chain_rounding_stays_bounded_over_many_chunks(la_scale):
+    """The passes over chunks of bf16 problems round their operands and additive terms to fp16 (relative
+    2^-11 each) but keep the state in fp32.  Over 60 chunks of slow decay (log alpha near -0.02) and of
+    none at all (alpha = 1), with keys of norm 1 (beta |k|^2 < 2: the delta-rule update contracts), every
+    gradient of that arrangement stays within 2.5e-3 relative L2 of the exact one (measured: 5e-4 and
+    8e-4, no growth with the chunk count): half the bf16 parity bound, the other half left to the bf16
+    storage of inputs and gradients."""
+    rng = np.random.default_rng(11)
+    N, D, C = 60 * 64 - 17, 16, 64
+    q, k, v = (rng.standard_normal((N, D)) for _ in range(3))
+    k /= np.linalg.norm(k, axis=1, keepdims=True)
+    q /= np.linalg.norm(q, axis=1, keepdims=True)
+    la = -np.abs(rng.standard_normal((N, D))) * la_scale
+    beta = 1 / (1 + np.exp(-rng.standard_normal(N)))
+    dO, S0, dSN = rng.standard_normal((N, D)), rng.standard_normal((D, D)), rng.standard_normal((D, D)) * 0.1
+    exact = _decomposed_bwd(q, k, v, la, beta, dO, S0, dSN, C)
+    h16 = _decomposed_bwd(q, k, v, la, beta, dO, S0, dSN, C, h16=True)
+    for name in ("dq", "dk", "dv", "dla", "dbeta", "dS0"):
+        e = np.linalg.norm(h16[name] - exact[name]) / np.linalg.norm(exact[name])
+        assert 0 < e <= 2.5e-3, f"{name}: {e:.2e}"
