@@ -315,7 +315,8 @@ __device__ __forceinline__ ChunkPos chunk_pos(const CbwdArgs& a) {
 #define FRAG_C(n0) ((n0) + 8 * nt + 2 * t + (i & 1))
 
 // A warp's accumulator tiles into a row-major [.][ld] array at element offset off: fp32, or, for
-// bf16 problems (!SPLIT), fp16 at the same element offset (the chains' additive terms)
+// bf16 problems (!SPLIT), fp16 at the same element offset (what the chains read: W and their
+// additive terms)
 template <int MT, int NT_, bool SPLIT>
 __device__ __forceinline__ void store_tile(float* base, int64_t off, int ld, const float (&acc)[MT][NT_][4], int m0,
                                            int n0, int g, int t) {
@@ -474,25 +475,8 @@ __global__ void __launch_bounds__(NT, 1) cbwd_prep_kernel(CbwdArgs a) {
     float acc[2][NTD][4];
     zero4(acc);
     wmma3<2, NTD, false, SPLIT>(acc, As, LDC, 1, Kx, LDD, 1, CH, m0, n0, lane);
-    if (SPLIT) {
-      float* W = a.w.W + p.ch * CH * D;
-      FRAG_LOOP(2, NTD) {
-        const int r = FRAG_R(m0), c = FRAG_C(n0);
-        W[r * D + c] = acc[mt][nt][i] * egm[c];
-      }
-    } else {   // fp16 operand of the chains
-      __half* W = reinterpret_cast<__half*>(a.w.W) + p.ch * CH * D;
-#pragma unroll
-      for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-        for (int nt = 0; nt < NTD; ++nt)
-#pragma unroll
-          for (int hi = 0; hi < 2; ++hi) {
-            const int r = m0 + 16 * mt + g + 8 * hi, c = n0 + 8 * nt + 2 * t;
-            *reinterpret_cast<__half2*>(W + r * D + c) =
-                __floats2half2_rn(acc[mt][nt][2 * hi] * egm[c], acc[mt][nt][2 * hi + 1] * egm[c + 1]);
-          }
-    }
+    FRAG_LOOP(2, NTD) acc[mt][nt][i] *= egm[FRAG_C(n0)];
+    store_tile<2, NTD, SPLIT>(a.w.W, p.ch * CH * D, D, acc, m0, n0, g, t);
     zero4(acc);
     wmma3<2, NTD, false, SPLIT>(acc, As, LDC, 1, KN, LDD, 1, CH, m0, n0, lane);
     store_tile<2, NTD, SPLIT>(a.w.Ut, p.ch * CH * D, D, acc, m0, n0, g, t);
